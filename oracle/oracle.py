@@ -1,0 +1,256 @@
+"""fp64 CPU oracle for the KDA forward scan and mShortConv -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may
+import this module.  The product path (the CUDA library and its Python binding) never
+does, and shares no code with it.
+
+The arithmetic lives in ``kda_oracle.c`` (plain loops in double precision); this file
+only builds it with gcc and marshals arrays.  What each routine computes, and the
+passages of the Chimera paper it follows, is stated in that file's header:
+
+* ``kda_forward``: Eq. 14 of the paper, section 3.3 (decay, rank-one erase, write, in
+  that order), read out as o_t = S_t^T q_t with S_t the state after token t.
+* ``mshortconv``: section 3.4 -- per-segment depthwise conv, 1-D causal for text,
+  3x3 spatial for an image, 3x3x3 causal-in-time / symmetric-in-space for video,
+  zero padding inside each segment, time-first raster order of Eq. 12.
+* ``l2norm_heads``: unit-norm rows per head (no epsilon; zero stays zero).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+DT_F32, DT_BF16, DT_F64 = 0, 1, 2
+MOD_TEXT, MOD_IMAGE, MOD_VIDEO = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c into liboracle.so next to it (gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("modality", ctypes.c_int32), ("pad0", ctypes.c_int32),
+                ("start", ctypes.c_int64), ("F", ctypes.c_int32), ("Hgt", ctypes.c_int32),
+                ("Wid", ctypes.c_int32), ("weight_set", ctypes.c_int32)]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P, I, L = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+            lib.oracle_kda_forward.restype = I
+            lib.oracle_kda_forward.argtypes = [P, P, P, P, P, I, P, P, L, L, L, P,
+                                               I, I, I, I, I, P, I, I]
+            lib.oracle_mshortconv.restype = I
+            lib.oracle_mshortconv.argtypes = [P, I, P, I, I, I, I, I, P, I, I, P, P, P, I]
+            lib.oracle_l2norm_heads.restype = None
+            lib.oracle_l2norm_heads.argtypes = [P, L, I, I]
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def _as_input(a):
+    """Return (contiguous numpy array, dtype code) holding the values at stored precision.
+
+    Accepts numpy arrays (float32 / float64) or torch CPU tensors (float32, bfloat16,
+    float64).  bf16 is passed as its raw 16-bit patterns; the C side widens them
+    exactly."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            a = a.detach().contiguous().cpu()
+            if a.dtype == torch.bfloat16:
+                return a.view(torch.int16).numpy().view(np.uint16), DT_BF16
+            if a.dtype == torch.float32:
+                return a.numpy(), DT_F32
+            if a.dtype == torch.float64:
+                return a.numpy(), DT_F64
+            raise TypeError(f"unsupported tensor dtype {a.dtype}")
+    except ImportError:  # pragma: no cover
+        pass
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, DT_F32
+    if a.dtype == np.float64:
+        return a, DT_F64
+    if a.dtype == np.uint16:
+        return a, DT_BF16
+    raise TypeError(f"unsupported array dtype {a.dtype}")
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def kda_forward(q, k, v, g, beta, S0=None, *, pairs=None, want_o=True, nthreads=None):
+    """Token-by-token KDA scan in fp64.
+
+    q, k, g: [B,T,H,Dk]; v: [B,T,H,Dv]; beta: [B,T,H]; S0: [B,H,Dk,Dv] or None (zeros).
+    All five inputs must share one storage dtype.  ``pairs`` optionally restricts the
+    work to a list of (b, h) pairs; outputs of other pairs are left at zero.
+
+    Returns (o [B,T,H,Dv] float64 or None, S_T [B,H,Dk,Dv] float64).
+    """
+    lib = _load()
+    arrs = [_as_input(x) for x in (q, k, v, g, beta)]
+    dts = {d for _, d in arrs}
+    if len(dts) != 1:
+        raise TypeError("q, k, v, g, beta must share one dtype")
+    dt = dts.pop()
+    (qa, _), (ka, _), (va, _), (ga, _), (ba, _) = arrs
+    B, T, H, Dk = qa.shape
+    Dv = va.shape[-1]
+    if ka.shape != (B, T, H, Dk) or ga.shape != (B, T, H, Dk) or va.shape != (B, T, H, Dv) \
+            or ba.shape != (B, T, H):
+        raise ValueError("shape mismatch")
+    s0 = None
+    if S0 is not None:
+        s0 = np.ascontiguousarray(np.asarray(S0, dtype=np.float64))
+        if s0.shape != (B, H, Dk, Dv):
+            raise ValueError("S0 shape")
+    o = np.zeros((B, T, H, Dv), dtype=np.float64) if want_o else None
+    ST = np.zeros((B, H, Dk, Dv), dtype=np.float64)
+    pr = None
+    npairs = 0
+    if pairs is not None:
+        pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        npairs = pr.shape[0]
+    nt = nthreads or default_threads()
+    rc = lib.oracle_kda_forward(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _ptr(ba), dt, _ptr(s0),
+                                _ptr(o), T * H * Dv, H * Dv, Dv, _ptr(ST),
+                                B, T, H, Dk, Dv, _ptr(pr), npairs, nt)
+    if rc != 0:
+        raise ValueError("oracle_kda_forward rejected its arguments")
+    return o, ST
+
+
+def kda_forward_head(q, k, v, g, beta, b, h, S0_head=None, nthreads=1):
+    """One (b, h) scan over the full length; returns (o [T,Dv], S_T [Dk,Dv]) in fp64.
+
+    Memory is O(T*Dv) for the output of that head only, so full-length streams can be
+    checked one head at a time."""
+    lib = _load()
+    arrs = [_as_input(x) for x in (q, k, v, g, beta)]
+    dt = arrs[0][1]
+    (qa, _), (ka, _), (va, _), (ga, _), (ba, _) = arrs
+    B, T, H, Dk = qa.shape
+    Dv = va.shape[-1]
+    s0 = None
+    if S0_head is not None:
+        s0 = np.zeros((B, H, Dk, Dv), dtype=np.float64)
+        s0[b, h] = np.asarray(S0_head, dtype=np.float64)
+    o = np.zeros((T, Dv), dtype=np.float64)
+    ST = np.zeros((B, H, Dk, Dv), dtype=np.float64) if B * H * Dk * Dv <= (1 << 24) else None
+    pr = np.array([[b, h]], dtype=np.int32)
+    if ST is None:
+        raise ValueError("state buffer too large")
+    # o[b*o_sb + t*o_st + h*o_sh]: address the single-head buffer with o_sb = o_sh = 0.
+    rc = lib.oracle_kda_forward(_ptr(qa), _ptr(ka), _ptr(va), _ptr(ga), _ptr(ba), dt, _ptr(s0),
+                                _ptr(o), 0, Dv, 0, _ptr(ST), B, T, H, Dk, Dv, _ptr(pr), 1, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_kda_forward rejected its arguments")
+    return o, ST[b, h].copy()
+
+
+def make_segments(table):
+    """table: iterable of (modality, start, F, Hgt, Wid, weight_set) -> ctypes array."""
+    rows = list(table)
+    arr = (Segment * max(1, len(rows)))()
+    for i, (m, s, F, Hh, W, ws) in enumerate(rows):
+        arr[i] = Segment(int(m), 0, int(s), int(F), int(Hh), int(W), int(ws))
+    return arr, len(rows)
+
+
+def mshortconv(x, segments, Kt, w_text=None, w_image=None, w_video=None, *, c_range=None,
+               nthreads=None):
+    """Direct-loop mShortConv in fp64.  x: [B,T,C] (fp32 / bf16 / fp64); weights fp32:
+    text [n,C,Kt], image [n,C,3,3], video [n,C,3,3,3].  Returns y [B,T,C'] float64 for
+    the channel range c_range=(lo,hi) (all channels by default); positions outside
+    every segment are zero."""
+    lib = _load()
+    xa, dt = _as_input(x)
+    B, T, C = xa.shape
+    lo, hi = c_range if c_range is not None else (0, C)
+    y = np.zeros((B, T, C), dtype=np.float64)
+    segs, n = make_segments(segments)
+
+    def wp(w):
+        if w is None:
+            return None, None
+        try:
+            import torch
+            if isinstance(w, torch.Tensor):
+                w = w.detach().cpu().float().numpy()
+        except ImportError:  # pragma: no cover
+            pass
+        w = np.ascontiguousarray(np.asarray(w, dtype=np.float32))
+        return w, _ptr(w)
+
+    wt, pt = wp(w_text)
+    wi, pi = wp(w_image)
+    wv, pv = wp(w_video)
+    nt = nthreads or default_threads()
+    rc = lib.oracle_mshortconv(_ptr(xa), dt, _ptr(y), B, T, C, lo, hi,
+                               ctypes.cast(segs, ctypes.c_void_p), n, int(Kt), pt, pi, pv, nt)
+    if rc != 0:
+        raise ValueError("oracle_mshortconv rejected its arguments")
+    return y[:, :, lo:hi]
+
+
+def l2norm_heads(x, H):
+    """Unit-normalise every head slice of the last axis (length H*D); returns a copy."""
+    a = np.array(x, dtype=np.float64, copy=True, order="C")
+    D = a.shape[-1] // H
+    lib = _load()
+    rows = a.size // (H * D)
+    lib.oracle_l2norm_heads(_ptr(a), rows, H, D)
+    return a
+
+
+def fused_forward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, H, S0=None, *, pairs=None,
+                  nthreads=None):
+    """mShortConv of x_q, x_k, x_v (each [B,T,H*D]) -> L2-normalised q, k per head ->
+    KDA scan (Eq. 13 feeding Eq. 14).  w* = (w_text, w_image, w_video) per tensor."""
+    yq = mshortconv(xq, segments, Kt, *wq, nthreads=nthreads)
+    yk = mshortconv(xk, segments, Kt, *wk, nthreads=nthreads)
+    yv = mshortconv(xv, segments, Kt, *wv, nthreads=nthreads)
+    B, T, C = yq.shape
+    D = C // H
+    q = l2norm_heads(yq, H).reshape(B, T, H, D)
+    k = l2norm_heads(yk, H).reshape(B, T, H, D)
+    v = yv.reshape(B, T, H, D)
+    return kda_forward(q, k, v, _to_f64(g), _to_f64(beta), S0, pairs=pairs, nthreads=nthreads)
+
+
+def _to_f64(a):
+    """Widen an input (torch tensor or numpy array, bf16 bit patterns included) to fp64
+    at its stored precision."""
+    arr, dt = _as_input(a)
+    if dt == DT_BF16:
+        return (arr.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return arr.astype(np.float64)
