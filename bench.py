@@ -1,0 +1,426 @@
+#!/usr/bin/env python3
+"""Benchmark of the KDA forward scan (and the fused mShortConv -> KDA path) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libkda|reference]
+                    [--workload NAME] [--extra] [--no-cpu-baseline]
+
+One JSON line on stdout (rank 0).  A step is one kda_forward call over one batch of
+the workload (inputs resident in HBM).  Timing: W untimed warm-up steps, then K steps
+bracketed by a barrier and torch.cuda.synchronize() on both sides, CUDA events on the
+launching stream, max over ranks.  The inputs (672 MB per step for the video clip)
+are larger than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling over
+independent (batch, head) scans; no collective on the data path).  `--impl reference`
+times the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from linear_attention_sequence_mshortconv_b200 import inputs as W  # noqa: E402
+
+METRIC = "KDA fwd Mtokens/s (H=16,d=128,T≈32k) and % of B200 roofline"
+UNIT = "Mtokens/s"
+DEFAULT_WORKLOAD = W.VIDEO_CLIP.name
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------------
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def algorithmic_bytes(w: W.Workload) -> int:
+    """Bytes a single pass must move: q, k, v, g read and o written at the run dtype,
+    beta read, plus the fp32 final state written."""
+    es = torch.tensor([], dtype=w.dtype).element_size()
+    per_tok_head = 5 * w.D * es + es
+    state = w.B * w.H * w.D * w.D * 4
+    return w.B * w.T * w.H * per_tok_head + state
+
+
+def traffic_record(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            recs = json.load(f)
+    except (OSError, ValueError):
+        return None
+    rec = recs.get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec.get("source", ""))
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if sha != rec.get("source_sha256"):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls NVML (SM clock and throttle reasons) in a thread during the timed region."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ----------------------------------------------------------------------------------
+
+def oracle_sample_tokens(w: W.Workload, target_s: float, threads: int) -> int:
+    """Prefix length (all heads, batch row 0) that takes about target_s on the oracle."""
+    from oracle import oracle as O
+    probe = w.resized(B=1, T=min(w.T, 128), name="probe")
+    inp = W.make_kda_inputs(probe)
+    t0 = time.perf_counter()
+    O.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], want_o=True, nthreads=threads)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    per_tok = dt / probe.T
+    return int(max(64, min(w.T, target_s / per_tok)))
+
+
+def time_oracle(w: W.Workload, T_s: int, threads: int):
+    """Runs the oracle on the first T_s tokens (batch row 0, all heads); returns
+    (seconds, tokens processed)."""
+    from oracle import oracle as O
+    sample = w.resized(B=1, T=T_s, name="sample")
+    inp = W.make_kda_inputs(sample)
+    t0 = time.perf_counter()
+    O.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], want_o=True, nthreads=threads)
+    return time.perf_counter() - t0, T_s
+
+
+def cpu_baseline(w: W.Workload, target_s: float = 12.0):
+    from oracle import oracle as O
+    threads = O.default_threads()
+    T_s = oracle_sample_tokens(w, target_s, threads)
+    secs, toks = time_oracle(w, T_s, threads)
+    return {"value": toks / secs / 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"fp64 token loop, first {T_s} of {w.T} tokens of batch row 0, all {w.H} "
+                      f"heads ({secs:.1f} s)"}
+
+
+def run_reference(args, ws, rank, w: W.Workload):
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    threads = O.default_threads()
+    per_step = max(0.5, 90.0 / max(1, args.steps + args.warmup))
+    T_s = oracle_sample_tokens(w, per_step, threads)
+    for _ in range(args.warmup):
+        time_oracle(w, T_s, threads)
+    total, toks = 0.0, 0
+    for _ in range(args.steps):
+        s, n = time_oracle(w, T_s, threads)
+        total += s
+        toks += n
+    value = toks / total / 1e6
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, ws),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"each step: fp64 token loop over the first {T_s} of "
+                                       f"{w.T} tokens of batch row 0, all {w.H} heads"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: W.Workload, ws: int):
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.D, "chunk": w.chunk,
+            "fused_conv": w.fused, "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush)" if algorithmic_bytes(w) > 126e6
+                  else "L2 flushed between steps"}
+
+
+# ----------------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------------
+
+def make_step(w: W.Workload, rank: int):
+    from linear_attention_sequence_mshortconv_b200 import kda
+    dev = torch.device("cuda")
+    wr = w if rank == 0 else W.dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    if w.fused:
+        inp = W.make_fused_inputs(wr, device=dev)
+        o = torch.empty((w.B, w.T, w.H, w.D), dtype=w.dtype, device=dev)
+        S_T = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+        wsz = kda.mshortconv_workspace_size(w.B, w.T, w.H, w.D, w.dtype, w.chunk, o_dtype=w.dtype)
+        ws = torch.empty(max(wsz, 1), dtype=torch.uint8, device=dev)
+
+        def step():
+            kda.mshortconv_kda_forward(inp["xq"], inp["xk"], inp["xv"], inp["segments"], w.Kt,
+                                       inp["wq"], inp["wk"], inp["wv"], inp["g"], inp["beta"],
+                                       chunk=w.chunk, o=o, S_T=S_T, workspace=ws)
+        return step, inp, o, S_T
+    inp = W.make_kda_inputs(wr, device=dev)
+    o = torch.empty((w.B, w.T, w.H, w.D), dtype=w.dtype, device=dev)
+    S_T = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    wsz = kda.workspace_size(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+    ws = torch.empty(max(wsz, 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=w.chunk,
+                    o=o, S_T=S_T, workspace=ws)
+    return step, inp, o, S_T
+
+
+def timed(step, K, ws):
+    barrier(ws)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(K):
+        step()
+    b.record(s)
+    torch.cuda.synchronize()
+    barrier(ws)
+    return a.elapsed_time(b)
+
+
+def e2e_measure(w: W.Workload, K: int, ws: int, rank: int):
+    """Same metric through the public API with HOST buffers: each step copies the
+    inputs from pinned host memory, runs the call and reads o and S_T back."""
+    from linear_attention_sequence_mshortconv_b200 import kda
+    dev = torch.device("cuda")
+    host = W.make_kda_inputs(w, device="cpu") if not w.fused else None
+    if host is None:
+        return None
+    host = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor)}
+    dv = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    o = torch.empty((w.B, w.T, w.H, w.D), dtype=w.dtype, device=dev)
+    S_T = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device=dev)
+    o_h = torch.empty_like(o, device="cpu").pin_memory()
+    S_h = torch.empty_like(S_T, device="cpu").pin_memory()
+    wsz = kda.workspace_size(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+    wbuf = torch.empty(max(wsz, 1), dtype=torch.uint8, device=dev)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o.numel() * o.element_size() + S_T.numel() * 4
+
+    def step():
+        for k_, v in host.items():
+            dv[k_].copy_(v, non_blocking=True)
+        kda.forward(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], chunk=w.chunk, o=o, S_T=S_T,
+                    workspace=wbuf)
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(S_T, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(timed(step, K, ws), ws)
+    return {"value": ws * w.tokens / (ms / K * 1e-3) / 1e6, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / K}
+
+
+def run_gpu(args, ws, rank, local, w: W.Workload):
+    from linear_attention_sequence_mshortconv_b200 import build as libbuild
+    from linear_attention_sequence_mshortconv_b200 import kda
+    if rank == 0:
+        libbuild.build()
+    barrier(ws)
+    kda.load_library()
+    step, inp, o, S_T = make_step(w, rank)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if not torch.isfinite(o.float()).all():
+        raise RuntimeError("non-finite output")
+
+    launches0 = kda.kernel_launches()
+    kda.profile_enable(True)
+    sampler = ClockSampler(local)
+    with sampler:
+        ms = timed(step, args.steps, ws)
+    kda.profile_enable(False)
+    launches = kda.kernel_launches() - launches0
+    ms = max_over_ranks(ms, ws)
+    ms_step = ms / args.steps
+    value = ws * w.tokens / (ms_step * 1e-3) / 1e6
+
+    peaks, peak_kind = read_peaks()
+    prof = {}
+    for name in ("kda_generic", "kda_tc_chunk", "kda_tc_state", "kda_tc_output", "conv"):
+        r = kda.profile_collect(name)
+        if r and r[1] > 0:
+            prof[name] = {"ms_total": r[0], "launches": r[1], "ms_per_launch": r[0] / r[1]}
+    dominant = max(prof, key=lambda n: prof[n]["ms_total"]) if prof else None
+    roof = None
+    if dominant:
+        per_launch_s = prof[dominant]["ms_per_launch"] * 1e-3
+        # the dominant kernel moves the whole scan's algorithmic bytes once per launch
+        launches_per_step = prof[dominant]["launches"] / args.steps
+        alg = algorithmic_bytes(w) / launches_per_step
+        achieved = alg / per_launch_s / 1e9
+        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+        roof = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_record(dominant),
+                "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind,
+                "kernel_ms_per_launch": prof[dominant]["ms_per_launch"]}
+
+    e2e = e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": workload_config(w, ws), "roofline": roof, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary(),
+            "kernels": prof}
+    if args.extra and rank == 0:
+        extra = []
+        for other in W.WORKLOADS:
+            if other.name == w.name:
+                continue
+            st, _, _, _ = make_step(other, rank)
+            for _ in range(3):
+                st()
+            m = timed(st, max(3, args.steps // 4), 1) / max(3, args.steps // 4)
+            extra.append({"workload": other.name, "ms_per_step": m,
+                          "value": other.tokens / (m * 1e-3) / 1e6, "unit": UNIT,
+                          "alg_GBps": algorithmic_bytes(other) / (m * 1e-3) / 1e9})
+        line["extra_workloads"] = extra
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libkda", choices=["libkda", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--extra", action="store_true", help="also time the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = dist_setup()
+    w = W.BY_NAME[args.workload]
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank, w)
+        else:
+            run_gpu(args, ws, rank, local, w)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

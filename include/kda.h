@@ -1,0 +1,195 @@
+/*
+ * kda.h -- C ABI of libkda: the Kimi Delta Attention (KDA) forward scan and the
+ * modality-aware short convolution (mShortConv) that feeds it, for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operations are those of the Chimera paper ("Chimera: hybrid attention +
+ * Chinchilla scaling", pchao.org translation):
+ *   - section 3.3, Eq. 14 -- per head, with S_t in R^{Dk x Dv} the state AFTER token t,
+ *         S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     alpha_t in (0,1)^{Dk} a per-key-channel forget gate, beta_t in (0,1) one scalar
+ *     per head and token; the parenthesisation (decay, then erase, then write) is the
+ *     one printed in LaTeX by the agifrontier summary of the paper;
+ *   - section 3.3, Eq. 15 (inner term) -- the readout o_t = S_t^T q_t;
+ *   - section 3.3 -- the state restarts from S_0 = 0 at a packed-sample boundary
+ *     (here: at the start of every batch row, or from the caller's S0);
+ *   - section 3.3, Eq. 13 and section 3.4 -- (Q,K,V) = mShortConv(...): a depthwise
+ *     convolution applied inside each modality segment of the packed stream, causal
+ *     1-D for text, 3x3 spatial for an image, 3x3x3 for video (causal in time,
+ *     symmetric in space, per the agifrontier summary), with visual tokens in the
+ *     time-first raster order of Eq. 12, m = f*H*W + r*W + c.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     token-major; the library never frees or retains them.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *     Argument errors are detected on the host and returned before any launch.
+ *     Launch failures return KDA_ERR_CUDA.  Faults detected by the kernels on the
+ *     device (a bounded wait that ran out) are recorded in a per-device status word
+ *     read by kda_last_device_error() after the caller synchronises.
+ *   - Floating point: inputs are bf16 or fp32 (kda_dtype); all accumulation and the
+ *     recurrent state are fp32.  The fp32 path computes in fp32 on CUDA cores; the
+ *     bf16 path feeds bf16 operands to the tensor cores with fp32 accumulation.
+ *   - The gate is passed as g = ln(alpha) (g <= 0, finite), not as alpha: alpha close
+ *     to 1 is not representable in bf16 (the spacing just below 1 is 2^-8), while its
+ *     logarithm is.
+ *   - No 1/sqrt(Dk) scaling and no normalisation happen inside kda_forward; q and k
+ *     are used as given.
+ */
+#ifndef LIBKDA_KDA_H
+#define LIBKDA_KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad segment table, ... */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. Dk not in {32,64,128}) */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+    KDA_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out (see kda_last_device_error) */
+    KDA_ERR_WORKSPACE = 5      /* caller-provided workspace smaller than required */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* kda_status_string(kda_status s);
+
+/* Reads and clears the calling thread's current device's status word, in which
+ * kernels record device-side failures (KDA_OK if none).  Synchronous: it waits for
+ * all work on the device to finish. */
+kda_status kda_last_device_error(void);
+
+/* Bytes of device workspace kda_forward needs for this problem (0 if none).  The
+ * value depends only on the arguments and the current device's SM count. */
+size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                                  kda_dtype o_dtype, int chunk);
+
+/*
+ * kda_forward -- KDA forward scan (Eq. 14) with readout o_t = S_t^T q_t (Eq. 15).
+ *
+ *   q, k, g : [B, T, H, Dk]  dtype          g = ln(alpha), finite, <= 0
+ *   v       : [B, T, H, Dv]  dtype
+ *   beta    : [B, T, H]      dtype          erase/write strength, one per (token, head)
+ *   S0      : [B, H, Dk, Dv] fp32, or NULL  initial state (NULL = zeros)
+ *   o       : [B, T, H, Dv]  o_dtype        written for every token
+ *   S_T     : [B, H, Dk, Dv] fp32, or NULL  final state (NULL = not written)
+ *   Dk, Dv  : each in {32, 64, 128}
+ *   o_dtype : KDA_BF16 or KDA_F32.  The output is accumulated in fp32 and rounded
+ *             once to o_dtype (round to nearest even); a bf16 o is exactly the fp32 o
+ *             of the same call rounded.  (bf16 output rounding alone is up to 2^-9 of
+ *             |o|, which for heavy-tailed outputs exceeds a few percent of RMS(o).)
+ *   chunk   : tokens per chunk of the chunkwise evaluation: 0 = the default for
+ *             the dtype, else one of {16, 32, 64}.  The result does not depend on it
+ *             beyond rounding.
+ *   workspace, workspace_bytes : device scratch of at least
+ *             kda_forward_workspace_size(...) bytes, 256-byte aligned; or NULL, in
+ *             which case the library takes and returns it with cudaMallocAsync /
+ *             cudaFreeAsync on `stream`.  The workspace must not be used by
+ *             another call that may run concurrently.
+ *
+ * Batch rows are independent scans (each starts from its S0 slice or zero).  T may
+ * be any non-negative length (0: o untouched, S_T = S0).  o must not alias an input.
+ */
+kda_status kda_forward(const void* q, const void* k, const void* v, const void* g,
+                       const void* beta, const float* S0, void* o, float* S_T,
+                       int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                       kda_dtype o_dtype, int chunk, void* workspace, size_t workspace_bytes,
+                       kda_stream_t stream);
+
+/* Modalities of a packed-stream segment (section 3.4). */
+typedef enum { MSC_TEXT = 0, MSC_IMAGE = 1, MSC_VIDEO = 2 } msc_modality;
+
+/* One modality segment of a packed row.  The same table applies to every batch
+ * row.  Tokens of the segment are [start, start + len) with len = Wid (text),
+ * Hgt*Wid (image) or F*Hgt*Wid (video, time-first raster order, Eq. 12).
+ * weight_set selects the kernel among the sets of that modality. */
+typedef struct {
+    int32_t modality;     /* msc_modality */
+    int32_t reserved;     /* must be 0 */
+    int64_t start;
+    int32_t F, Hgt, Wid;  /* text: F = Hgt = 1, Wid = length; image: F = 1 */
+    int32_t weight_set;
+} msc_segment;
+
+/*
+ * mshortconv_forward -- depthwise modality-aware short convolution (section 3.4).
+ *
+ *   x, y     : [B, T, C] dtype (device).  y must not alias x.
+ *   segs     : HOST array of n_segs segments, in increasing start order, without
+ *              overlap, inside [0, T).  Tokens covered by no segment get y = 0.
+ *   Kt       : text kernel length, 1..8.
+ *   w_text   : [n_text_sets, C, Kt] fp32 (device); y[t] = sum_j w[c,j] x[t-(Kt-1)+j]
+ *   w_image  : [n_image_sets, C, 3, 3] fp32;  y[r,s] = sum_{a,e} w[c,a,e] x[r-1+a, s-1+e]
+ *   w_video  : [n_video_sets, C, 3, 3, 3] fp32;
+ *              y[f,r,s] = sum_{tau,a,e} w[c,tau,a,e] x[f-2+tau, r-1+a, s-1+e]
+ *              Positions outside the segment (before its first token/frame, outside
+ *              its grid) read as zero: no kernel crosses a segment boundary.
+ *   n_*_sets : number of weight sets of each modality (bounds weight_set).
+ * A weight pointer may be NULL only if no segment uses that modality.  C must be a
+ * multiple of 8.  No bias, no activation.
+ */
+kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_dtype dtype,
+                              const msc_segment* segs, int n_segs, int Kt,
+                              const float* w_text, int n_text_sets,
+                              const float* w_image, int n_image_sets,
+                              const float* w_video, int n_video_sets,
+                              kda_stream_t stream);
+
+/* Bytes of workspace kda_mshortconv_forward needs. */
+size_t kda_mshortconv_workspace_size(int B, int T, int H, int D, kda_dtype dtype,
+                                     kda_dtype o_dtype, int chunk);
+
+/*
+ * kda_mshortconv_forward -- Eq. 13 feeding Eq. 14: q = L2norm_h(mShortConv(x_q)),
+ * k = L2norm_h(mShortConv(x_k)), v = mShortConv(x_v), then kda_forward(q,k,v,g,beta).
+ *
+ *   xq, xk, xv : [B, T, H*D] dtype (device), the projected inputs before the conv.
+ *   segs, n_segs, Kt : as for mshortconv_forward (one table for all three tensors).
+ *   wq, wk, wv : each an array of 3 device pointers {w_text, w_image, w_video} with
+ *                the layouts of mshortconv_forward and ONE weight set per modality.
+ *   L2norm_h   : per (token, head) division by the Euclidean norm of the D channels
+ *                of that head (no epsilon; an all-zero vector stays zero).
+ *   g, beta, S0, o, S_T, o_dtype, chunk : as for kda_forward with Dk = Dv = D.
+ *   q, k, v are kept between the conv and the scan in the workspace as fp16 for
+ *   bf16 inputs (fp32 for fp32 inputs).
+ *   workspace  : as for kda_forward, sized by kda_mshortconv_workspace_size.
+ */
+kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv,
+                                  const msc_segment* segs, int n_segs, int Kt,
+                                  const float* const wq[3], const float* const wk[3],
+                                  const float* const wv[3],
+                                  const void* g, const void* beta, const float* S0,
+                                  void* o, float* S_T, int B, int T, int H, int D,
+                                  kda_dtype dtype, kda_dtype o_dtype, int chunk,
+                                  void* workspace, size_t workspace_bytes,
+                                  kda_stream_t stream);
+
+/* ---- diagnostics ---------------------------------------------------------------- */
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t kda_kernel_launches(void);
+
+/* When `on` is non-zero, every later call records a pair of CUDA events on its
+ * stream around each of its kernels, keyed by kernel name.  Off by default. */
+void kda_profile_enable(int on);
+
+/* Waits for the recorded events and returns, for kernel `name`, the summed
+ * device time in milliseconds and the number of launches timed since the last
+ * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
+ * record.  Names: "kda_generic", "kda_tc_chunk", "kda_tc_state", "kda_tc_output",
+ * "conv". */
+int kda_profile_collect(const char* name, double* total_ms, int* launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LIBKDA_KDA_H */

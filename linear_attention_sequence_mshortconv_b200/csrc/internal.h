@@ -1,0 +1,82 @@
+// Internal declarations shared by the translation units of libkda (not installed).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// ---- element types ----------------------------------------------------------------
+// Public tensors are fp32 or bf16 (kda_dtype).  fp16 is used internally for the
+// fused path's conv outputs (q, k, v between the conv and the scan): its 11-bit
+// significand keeps the extra rounding well inside the parity bound, where a bf16
+// intermediate alone costs about 2% of RMS(o) in max error.
+enum ElemType : int { ET_F32 = 0, ET_BF16 = 1, ET_F16 = 2 };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+
+// ---- launch accounting and optional per-kernel event timing ------------------------
+void count_launch();
+// Records CUDA events around the kernels launched in its lifetime when profiling is
+// enabled (kda_profile_enable); a no-op otherwise.
+class ProfileScope {
+  public:
+    ProfileScope(const char* name, cudaStream_t s);
+    ~ProfileScope();
+  private:
+    const char* name_;
+    cudaStream_t s_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
+// ---- device status word -------------------------------------------------------------
+// Codes a kernel may record (first writer wins).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+// Address of this device's status word (set up once per device; thread-safe).
+int* device_status_ptr();
+
+// ---- launchers (each returns cudaGetLastError() of its launches) ------------------
+struct KdaArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float* S0;
+    void* o;
+    float* ST;
+    int B, T, H, Dk, Dv, chunk;
+    ElemType in_t;   // q, k, v
+    ElemType out_t;  // o
+    ElemType gb_t;   // g, beta
+};
+
+// Generic chunkwise scan on CUDA cores in fp32 (any supported dtype/shape).
+cudaError_t launch_kda_generic(const KdaArgs& a, cudaStream_t s);
+
+// Tensor-core path (bf16, Dk = Dv = 128).  Workspace bytes it needs:
+size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms);
+bool kda_tc_supported(const KdaArgs& a);
+cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status,
+                          cudaStream_t s);
+
+struct ConvSeg {
+    int32_t modality;
+    int64_t start;
+    int32_t F, Hgt, Wid, weight_set;
+};
+// Depthwise modality-aware conv of one segment; optional per-head L2 normalisation
+// (head width D, 0 = none).  x, y: [B,T,C].
+cudaError_t launch_conv_segment(const void* x, void* y, int B, int T, int C, ElemType in_t,
+                                ElemType out_t, const ConvSeg& seg, int Kt, const float* w,
+                                int norm_D, cudaStream_t s);
+
+}  // namespace kda

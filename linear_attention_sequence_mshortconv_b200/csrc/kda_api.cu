@@ -1,0 +1,351 @@
+// C ABI of libkda: argument validation, workspace handling and dispatch.
+// The operations and their conventions are documented in include/kda.h.
+
+#include <mutex>
+#include <vector>
+
+#include "internal.h"
+
+namespace kda {
+
+namespace {
+__device__ int g_status;  // device-side failure word (DEV_*), first writer wins
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+int default_chunk(kda_dtype dt, int Dk) {
+    (void)Dk;
+    return dt == KDA_F32 ? 16 : 64;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+}  // namespace
+
+int* device_status_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = (int*)p;
+    }
+    return g_status_ptr[dev];
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+namespace {
+
+kda_status check_kda_args(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, const void* o, int B, int T, int H, int Dk,
+                          int Dv, kda_dtype dtype, kda_dtype o_dtype, int chunk)
+{
+    if (B < 0 || T < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (o_dtype != KDA_F32 && o_dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(Dk) || !dim_ok(Dv)) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Runs the scan given a resolved chunk and a workspace of the required size.
+kda_status run_kda(const KdaArgs& a, void* ws, size_t ws_bytes, cudaStream_t s)
+{
+    if (kda_tc_supported(a)) {
+        int* st = device_status_ptr();
+        if (!st) return KDA_ERR_CUDA;
+        return from_cuda(launch_kda_tc(a, ws, ws_bytes, st, s));
+    }
+    return from_cuda(launch_kda_generic(a, s));
+}
+
+size_t kda_ws_bytes(const KdaArgs& a)
+{
+    if (!kda_tc_supported(a)) return 0;
+    return kda_tc_workspace_bytes(a.B, a.T, a.H, a.chunk, num_sms());
+}
+
+// Takes the caller's workspace or a stream-ordered allocation of `need` bytes.
+struct Workspace {
+    void* ptr = nullptr;
+    bool owned = false;
+    cudaStream_t stream = nullptr;
+    kda_status acquire(void* user, size_t user_bytes, size_t need, cudaStream_t s) {
+        stream = s;
+        if (need == 0) { ptr = user; return KDA_OK; }
+        if (user) {
+            if (user_bytes < need) return KDA_ERR_WORKSPACE;
+            if (((uintptr_t)user & 255) != 0) return KDA_ERR_INVALID_ARG;
+            ptr = user;
+            return KDA_OK;
+        }
+        if (cudaMallocAsync(&ptr, need, s) != cudaSuccess) return KDA_ERR_CUDA;
+        owned = true;
+        return KDA_OK;
+    }
+    ~Workspace() { if (owned) cudaFreeAsync(ptr, stream); }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status s)
+{
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+kda_status kda_last_device_error(void)
+{
+    int* p = device_status_ptr();
+    if (!p) return KDA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KDA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+    return v == DEV_OK ? KDA_OK : (v == DEV_TIMEOUT ? KDA_ERR_TIMEOUT : KDA_ERR_CUDA);
+}
+
+static ElemType et_of(kda_dtype d) { return d == KDA_F32 ? ET_F32 : ET_BF16; }
+
+size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                                  kda_dtype o_dtype, int chunk)
+{
+    if (B < 0 || T < 0 || H <= 0 || !dim_ok(Dk) || !dim_ok(Dv)) return 0;
+    KdaArgs a{};
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv;
+    a.in_t = a.gb_t = et_of(dtype);
+    a.out_t = et_of(o_dtype);
+    a.chunk = chunk ? chunk : default_chunk(dtype, Dk);
+    return kda_ws_bytes(a);
+}
+
+kda_status kda_forward(const void* q, const void* k, const void* v, const void* g,
+                       const void* beta, const float* S0, void* o, float* S_T,
+                       int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                       kda_dtype o_dtype, int chunk, void* workspace, size_t workspace_bytes,
+                       kda_stream_t stream)
+{
+    kda_status st = check_kda_args(q, k, v, g, beta, o, B, T, H, Dk, Dv, dtype, o_dtype, chunk);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (B == 0) return KDA_OK;
+    if (T == 0) {
+        if (!S_T) return KDA_OK;
+        const size_t bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+        return from_cuda(S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(S_T, 0, bytes, s));
+    }
+    KdaArgs a{q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv,
+              chunk ? chunk : default_chunk(dtype, Dk), et_of(dtype), et_of(o_dtype), et_of(dtype)};
+    Workspace ws;
+    st = ws.acquire(workspace, workspace_bytes, kda_ws_bytes(a), s);
+    if (st != KDA_OK) return st;
+    return run_kda(a, ws.ptr, kda_ws_bytes(a), s);
+}
+
+static kda_status check_segments(const msc_segment* segs, int n_segs, int T, int Kt,
+                                 const float* w_text, int n_text, const float* w_image,
+                                 int n_image, const float* w_video, int n_video)
+{
+    if (n_segs < 0 || (n_segs > 0 && !segs)) return KDA_ERR_INVALID_ARG;
+    if (Kt < 1 || Kt > 8) return KDA_ERR_UNSUPPORTED;
+    int64_t prev_end = 0;
+    for (int i = 0; i < n_segs; ++i) {
+        const msc_segment& sg = segs[i];
+        if (sg.reserved != 0) return KDA_ERR_INVALID_ARG;
+        int64_t len;
+        if (sg.modality == MSC_TEXT) {
+            if (sg.F != 1 || sg.Hgt != 1 || sg.Wid < 1) return KDA_ERR_INVALID_ARG;
+            if (!w_text || sg.weight_set < 0 || sg.weight_set >= n_text) return KDA_ERR_INVALID_ARG;
+            len = sg.Wid;
+        } else if (sg.modality == MSC_IMAGE) {
+            if (sg.F != 1 || sg.Hgt < 1 || sg.Wid < 1) return KDA_ERR_INVALID_ARG;
+            if (!w_image || sg.weight_set < 0 || sg.weight_set >= n_image) return KDA_ERR_INVALID_ARG;
+            len = (int64_t)sg.Hgt * sg.Wid;
+        } else if (sg.modality == MSC_VIDEO) {
+            if (sg.F < 1 || sg.Hgt < 1 || sg.Wid < 1) return KDA_ERR_INVALID_ARG;
+            if (!w_video || sg.weight_set < 0 || sg.weight_set >= n_video) return KDA_ERR_INVALID_ARG;
+            len = (int64_t)sg.F * sg.Hgt * sg.Wid;
+        } else {
+            return KDA_ERR_INVALID_ARG;
+        }
+        if (sg.start < prev_end || sg.start + len > T) return KDA_ERR_INVALID_ARG;
+        prev_end = sg.start + len;
+    }
+    return KDA_OK;
+}
+
+static int64_t seg_len(const msc_segment& sg)
+{
+    return sg.modality == MSC_TEXT ? sg.Wid
+         : sg.modality == MSC_IMAGE ? (int64_t)sg.Hgt * sg.Wid : (int64_t)sg.F * sg.Hgt * sg.Wid;
+}
+
+// Zeroes the token ranges of y that no segment covers.
+static cudaError_t zero_gaps(void* y, int B, int T, int C, size_t esz, const msc_segment* segs,
+                             int n_segs, cudaStream_t s)
+{
+    std::vector<std::pair<int64_t, int64_t>> gaps;
+    int64_t pos = 0;
+    for (int i = 0; i < n_segs; ++i) {
+        if (segs[i].start > pos) gaps.push_back({pos, segs[i].start});
+        pos = segs[i].start + seg_len(segs[i]);
+    }
+    if (pos < T) gaps.push_back({pos, T});
+    for (auto& gp : gaps)
+        for (int b = 0; b < B; ++b) {
+            char* base = (char*)y + (((int64_t)b * T + gp.first) * C) * esz;
+            cudaError_t e = cudaMemsetAsync(base, 0, (size_t)(gp.second - gp.first) * C * esz, s);
+            if (e != cudaSuccess) return e;
+        }
+    return cudaSuccess;
+}
+
+static const float* seg_weights(const msc_segment& sg, int C, int Kt, const float* wt,
+                                const float* wi, const float* wv)
+{
+    if (sg.modality == MSC_TEXT) return wt + (int64_t)sg.weight_set * C * Kt;
+    if (sg.modality == MSC_IMAGE) return wi + (int64_t)sg.weight_set * C * 9;
+    return wv + (int64_t)sg.weight_set * C * 27;
+}
+
+static ConvSeg to_conv_seg(const msc_segment& sg)
+{
+    return ConvSeg{sg.modality, sg.start, sg.F, sg.Hgt, sg.Wid, sg.weight_set};
+}
+
+kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_dtype dtype,
+                              const msc_segment* segs, int n_segs, int Kt,
+                              const float* w_text, int n_text_sets,
+                              const float* w_image, int n_image_sets,
+                              const float* w_video, int n_video_sets,
+                              kda_stream_t stream)
+{
+    if (B < 0 || T < 0 || C <= 0 || (C % 8) != 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * T > 0 && (!x || !y)) return KDA_ERR_INVALID_ARG;
+    if (x && x == y) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_segments(segs, n_segs, T, Kt, w_text, n_text_sets, w_image,
+                                   n_image_sets, w_video, n_video_sets);
+    if (st != KDA_OK) return st;
+    if ((int64_t)B * T == 0) return KDA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t esz = dtype == KDA_F32 ? 4 : 2;
+    cudaError_t e = zero_gaps(y, B, T, C, esz, segs, n_segs, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    for (int i = 0; i < n_segs; ++i) {
+        const ElemType et = dtype == KDA_F32 ? ET_F32 : ET_BF16;
+        e = launch_conv_segment(x, y, B, T, C, et, et, to_conv_seg(segs[i]), Kt,
+                                seg_weights(segs[i], C, Kt, w_text, w_image, w_video), 0, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+// The fused path keeps q, k, v between the conv and the scan as fp16 (fp32 inputs:
+// fp32) in the workspace.
+static KdaArgs fused_kda_args(int B, int T, int H, int D, kda_dtype dtype, kda_dtype o_dtype,
+                              int chunk)
+{
+    KdaArgs a{};
+    a.B = B; a.T = T; a.H = H; a.Dk = D; a.Dv = D;
+    a.chunk = chunk ? chunk : default_chunk(dtype, D);
+    a.in_t = dtype == KDA_F32 ? ET_F32 : ET_F16;
+    a.gb_t = et_of(dtype);
+    a.out_t = et_of(o_dtype);
+    return a;
+}
+
+size_t kda_mshortconv_workspace_size(int B, int T, int H, int D, kda_dtype dtype,
+                                     kda_dtype o_dtype, int chunk)
+{
+    if (B < 0 || T < 0 || H <= 0 || !dim_ok(D)) return 0;
+    const size_t qkv = align256((size_t)B * T * H * D * (dtype == KDA_F32 ? 4 : 2));
+    return 3 * qkv + align256(kda_ws_bytes(fused_kda_args(B, T, H, D, dtype, o_dtype, chunk)));
+}
+
+kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv,
+                                  const msc_segment* segs, int n_segs, int Kt,
+                                  const float* const wq[3], const float* const wk[3],
+                                  const float* const wv[3],
+                                  const void* g, const void* beta, const float* S0,
+                                  void* o, float* S_T, int B, int T, int H, int D,
+                                  kda_dtype dtype, kda_dtype o_dtype, int chunk,
+                                  void* workspace, size_t workspace_bytes,
+                                  kda_stream_t stream)
+{
+    if (!wq || !wk || !wv) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_kda_args(xq, xk, xv, g, beta, o, B, T, H, D, D, dtype, o_dtype, chunk);
+    if (st != KDA_OK) return st;
+    const int C = H * D;
+    for (const float* const* w : {wq, wk, wv}) {
+        st = check_segments(segs, n_segs, T, Kt, w[0], 1, w[1], 1, w[2], 1);
+        if (st != KDA_OK) return st;
+    }
+    if (B == 0) return KDA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0)
+        return kda_forward(xq, xk, xv, g, beta, S0, o, S_T, B, T, H, D, D, dtype, o_dtype,
+                           chunk, nullptr, 0, stream);
+    const size_t need = kda_mshortconv_workspace_size(B, T, H, D, dtype, o_dtype, chunk);
+    Workspace ws;
+    st = ws.acquire(workspace, workspace_bytes, need, s);
+    if (st != KDA_OK) return st;
+    const size_t esz = dtype == KDA_F32 ? 4 : 2;
+    const size_t qkv = align256((size_t)B * T * H * D * esz);
+    const ElemType in_t = dtype == KDA_F32 ? ET_F32 : ET_BF16;
+    const ElemType mid_t = dtype == KDA_F32 ? ET_F32 : ET_F16;
+    char* base = (char*)ws.ptr;
+    void* qb = base;
+    void* kb = base + qkv;
+    void* vb = base + 2 * qkv;
+    void* kws = base + 3 * qkv;
+    const void* xs[3] = {xq, xk, xv};
+    void* ys[3] = {qb, kb, vb};
+    const float* const* ws3[3] = {wq, wk, wv};
+    for (int tsr = 0; tsr < 3; ++tsr) {
+        cudaError_t e = zero_gaps(ys[tsr], B, T, C, esz, segs, n_segs, s);  // esz: fp16 = bf16 size
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        for (int i = 0; i < n_segs; ++i) {
+            msc_segment sg = segs[i];
+            sg.weight_set = 0;
+            e = launch_conv_segment(xs[tsr], ys[tsr], B, T, C, in_t, mid_t, to_conv_seg(sg), Kt,
+                                    seg_weights(sg, C, Kt, ws3[tsr][0], ws3[tsr][1], ws3[tsr][2]),
+                                    tsr < 2 ? D : 0, s);
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+        }
+    }
+    KdaArgs a = fused_kda_args(B, T, H, D, dtype, o_dtype, chunk);
+    a.q = qb; a.k = kb; a.v = vb; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
+    return run_kda(a, kws, need - 3 * qkv, s);
+}
+
+}  // extern "C"

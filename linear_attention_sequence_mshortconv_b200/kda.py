@@ -1,0 +1,254 @@
+"""Thin Python binding of libkda (ctypes).  Argument marshalling only: every step of
+the scan and of the convolution runs in the CUDA library; PyTorch supplies device
+memory and the current stream.
+
+There is no fallback.  If ``libkda.so`` has not been built, or a call is made with
+tensors that are not on a CUDA device, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_F32, KDA_BF16 = 0, 1
+MSC_TEXT, MSC_IMAGE, MSC_VIDEO = 0, 1, 2
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_CUDA",
+          4: "KDA_ERR_TIMEOUT", 5: "KDA_ERR_WORKSPACE"}
+
+# Every symbol include/kda.h declares.
+EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace_size",
+            "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
+            "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
+            "kda_profile_collect")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class MscSegment(ctypes.Structure):
+    _fields_ = [("modality", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("start", ctypes.c_int64), ("F", ctypes.c_int32), ("Hgt", ctypes.c_int32),
+                ("Wid", ctypes.c_int32), ("weight_set", ctypes.c_int32)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libkda.so and declares its signatures (raises if it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with "
+                              "`python -m linear_attention_sequence_mshortconv_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.kda_status_string.restype = ctypes.c_char_p
+        lib.kda_status_string.argtypes = [I]
+        lib.kda_last_device_error.restype = I
+        lib.kda_last_device_error.argtypes = []
+        lib.kda_forward_workspace_size.restype = Z
+        lib.kda_forward_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+        lib.kda_forward.restype = I
+        lib.kda_forward.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+        lib.mshortconv_forward.restype = I
+        lib.mshortconv_forward.argtypes = [P, P, I, I, I, I, P, I, I, P, I, P, I, P, I, P]
+        lib.kda_mshortconv_workspace_size.restype = Z
+        lib.kda_mshortconv_workspace_size.argtypes = [I, I, I, I, I, I, I]
+        lib.kda_mshortconv_forward.restype = I
+        lib.kda_mshortconv_forward.argtypes = [P, P, P, P, I, I, P, P, P, P, P, P, P, P,
+                                               I, I, I, I, I, I, I, P, Z, P]
+        lib.kda_kernel_launches.restype = ctypes.c_uint64
+        lib.kda_kernel_launches.argtypes = []
+        lib.kda_profile_enable.restype = None
+        lib.kda_profile_enable.argtypes = [I]
+        lib.kda_profile_collect.restype = I
+        lib.kda_profile_collect.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                            ctypes.POINTER(ctypes.c_int)]
+        _lib = lib
+        return lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise KdaError(fn, rc)
+
+
+def _code(dtype) -> int:
+    return KDA_F32 if dtype == torch.float32 else KDA_BF16
+
+
+def workspace_size(B, T, H, Dk, Dv, dtype=torch.bfloat16, chunk=0, o_dtype=None) -> int:
+    lib = load_library()
+    return int(lib.kda_forward_workspace_size(B, T, H, Dk, Dv, _code(dtype),
+                                              _code(o_dtype or dtype), chunk))
+
+
+def forward(q, k, v, g, beta, S0=None, *, chunk: int = 0, o=None, S_T=None,
+            want_state: bool = True, workspace=None, stream=None, o_dtype=None):
+    """KDA forward scan (Eq. 14) with readout o_t = S_t^T q_t.
+
+    q, k, g: [B,T,H,Dk]; v: [B,T,H,Dv]; beta: [B,T,H] -- all bf16 or all fp32 CUDA
+    tensors; S0: [B,H,Dk,Dv] fp32 or None.  o_dtype: torch.float32 or torch.bfloat16
+    (default: the input dtype).  Returns (o, S_T or None)."""
+    lib = load_library()
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q)
+    for name, t, shape in (("k", k, (B, T, H, Dk)), ("g", g, (B, T, H, Dk)),
+                           ("v", v, (B, T, H, Dv)), ("beta", beta, (B, T, H))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q's {q.dtype}")
+    o_dtype = o_dtype or (o.dtype if o is not None else q.dtype)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    if S0 is not None and tuple(S0.shape) != (B, H, Dk, Dv):
+        raise ValueError("S0 shape")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.kda_forward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"),
+                         _dev(beta, "beta"), _dev(S0, "S0", torch.float32), _dev(o, "o", o_dtype),
+                         _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv, dt, _code(o_dtype),
+                         chunk, ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_forward", rc)
+    return o, S_T
+
+
+def make_segments(segments: Sequence[Sequence[int]]):
+    """(modality, start, F, Hgt, Wid, weight_set) tuples -> ctypes array (host)."""
+    rows = list(segments)
+    arr = (MscSegment * max(1, len(rows)))()
+    for i, (m, s, F, Hh, W, ws) in enumerate(rows):
+        arr[i] = MscSegment(int(m), 0, int(s), int(F), int(Hh), int(W), int(ws))
+    return arr, len(rows)
+
+
+def mshortconv(x, segments, Kt, w_text=None, w_image=None, w_video=None, *, y=None,
+               stream=None):
+    """Depthwise modality-aware short convolution of x [B,T,C] (section 3.4)."""
+    lib = load_library()
+    B, T, C = x.shape
+    dt = _dtype_code(x)
+    if y is None:
+        y = torch.empty_like(x)
+    segs, n = make_segments(segments)
+
+    def wsets(w):
+        return (0 if w is None else int(w.shape[0]))
+
+    rc = lib.mshortconv_forward(_dev(x, "x"), _dev(y, "y", x.dtype), B, T, C, dt,
+                                ctypes.cast(segs, ctypes.c_void_p), n, int(Kt),
+                                _dev(w_text, "w_text", torch.float32), wsets(w_text),
+                                _dev(w_image, "w_image", torch.float32), wsets(w_image),
+                                _dev(w_video, "w_video", torch.float32), wsets(w_video),
+                                _stream(stream))
+    _check("mshortconv_forward", rc)
+    return y
+
+
+def mshortconv_workspace_size(B, T, H, D, dtype=torch.bfloat16, chunk=0, o_dtype=None) -> int:
+    lib = load_library()
+    return int(lib.kda_mshortconv_workspace_size(B, T, H, D, _code(dtype),
+                                                 _code(o_dtype or dtype), chunk))
+
+
+def mshortconv_kda_forward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, S0=None, *,
+                           chunk: int = 0, o=None, S_T=None, want_state: bool = True,
+                           workspace=None, stream=None, o_dtype=None):
+    """Fused Eq. 13 -> Eq. 14: conv of x_q, x_k, x_v, per-head L2 norm of q and k,
+    KDA scan.  x*: [B,T,H*D]; w* = (w_text [1,C,Kt], w_image [1,C,3,3], w_video [1,C,3,3,3]);
+    g: [B,T,H,D]; beta: [B,T,H]."""
+    lib = load_library()
+    B, T, H, D = g.shape
+    dt = _dtype_code(xq)
+    o_dtype = o_dtype or (o.dtype if o is not None else xq.dtype)
+    if o is None:
+        o = torch.empty((B, T, H, D), dtype=o_dtype, device=xq.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=xq.device)
+    segs, n = make_segments(segments)
+    arrs = []
+    for name, w in (("wq", wq), ("wk", wk), ("wv", wv)):
+        a = (ctypes.c_void_p * 3)()
+        for i in range(3):
+            a[i] = _dev(w[i], f"{name}[{i}]", torch.float32) if w[i] is not None else None
+        arrs.append(a)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.kda_mshortconv_forward(_dev(xq, "xq"), _dev(xk, "xk"), _dev(xv, "xv"),
+                                    ctypes.cast(segs, ctypes.c_void_p), n, int(Kt),
+                                    ctypes.cast(arrs[0], ctypes.c_void_p),
+                                    ctypes.cast(arrs[1], ctypes.c_void_p),
+                                    ctypes.cast(arrs[2], ctypes.c_void_p),
+                                    _dev(g, "g", xq.dtype), _dev(beta, "beta", xq.dtype),
+                                    _dev(S0, "S0", torch.float32), _dev(o, "o", o_dtype),
+                                    _dev(S_T, "S_T", torch.float32), B, T, H, D, dt,
+                                    _code(o_dtype), chunk,
+                                    ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_mshortconv_forward", rc)
+    return o, S_T
+
+
+def kernel_launches() -> int:
+    """Kernels launched by libkda in this process so far."""
+    return int(load_library().kda_kernel_launches())
+
+
+def profile_enable(on: bool = True) -> None:
+    load_library().kda_profile_enable(1 if on else 0)
+
+
+def profile_collect(name: str):
+    """(total device ms, launches) of kernel `name` since the last collection, or None."""
+    ms, n = ctypes.c_double(0.0), ctypes.c_int(0)
+    rc = load_library().kda_profile_collect(name.encode(), ctypes.byref(ms), ctypes.byref(n))
+    return None if rc != 0 else (ms.value, n.value)
+
+
+def last_device_error() -> int:
+    """Reads and clears the device status word (0 = no device-side failure)."""
+    return int(load_library().kda_last_device_error())

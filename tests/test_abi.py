@@ -1,0 +1,97 @@
+"""The C ABI library loads, exports every symbol include/kda.h declares, and rejects bad
+arguments on the host before any launch (no GPU needed for these)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_sequence_mshortconv_b200 import build as B
+from linear_attention_sequence_mshortconv_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(",
+                                 src, flags=re.M)) - {"defined"})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return kda.load_library()
+
+
+def test_header_declares_the_boundary():
+    fns = _header_functions()
+    assert set(kda.EXPORTED) == set(fns), fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for fn in _header_functions():
+        assert hasattr(lib, fn), fn
+
+
+def test_status_strings(lib):
+    for code, name in kda.STATUS.items():
+        assert lib.kda_status_string(code).decode() == name
+
+
+def test_host_rejects_bad_arguments(lib):
+    P = None
+    # unsupported head width, before touching the device
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 48, 48, 1, 1, 0, P, 0, P) == 2
+    # negative batch
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, -1, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 1
+    # null tensors with work to do
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 1
+    # chunk not in {16, 32, 64}
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 1, 24, P, 0, P) == 2
+    # bad dtype / output dtype
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 7, 1, 0, P, 0, P) == 1
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 9, 0, P, 0, P) == 1
+    # empty problem is a no-op
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 0, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 0
+
+
+def test_conv_rejects_bad_segment_tables(lib):
+    segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
+    dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
+    sp = ctypes.cast(segs, ctypes.c_void_p)
+    # segment runs past T
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 8, 16, 1, sp, n, 4,
+                                  dummy, 1, None, 0, None, 0, None) == 1
+    # C not a multiple of 8
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 10, 12, 1, sp, n, 4,
+                                  dummy, 1, None, 0, None, 0, None) == 1
+    # text segment without text weights
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 10, 16, 1, sp, n, 4,
+                                  None, 0, None, 0, None, 0, None) == 1
+    # weight_set out of range
+    segs2, n2 = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 3)])
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 10, 16, 1,
+                                  ctypes.cast(segs2, ctypes.c_void_p), n2, 4,
+                                  dummy, 1, None, 0, None, 0, None) == 1
+    # overlapping segments
+    segs3, n3 = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 6, 0), (kda.MSC_TEXT, 4, 1, 1, 4, 0)])
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 10, 16, 1,
+                                  ctypes.cast(segs3, ctypes.c_void_p), n3, 4,
+                                  dummy, 1, None, 0, None, 0, None) == 1
+    # Kt out of range
+    assert lib.mshortconv_forward(dummy, ctypes.c_void_p(32), 1, 10, 16, 1, sp, n, 9,
+                                  dummy, 1, None, 0, None, 0, None) == 2
+
+
+def test_segment_record_layout_matches_header():
+    assert ctypes.sizeof(kda.MscSegment) == 32
+    assert kda.MscSegment.start.offset == 8 and kda.MscSegment.weight_set.offset == 28
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    z = torch.zeros(1, 4, 1, 32)
+    with pytest.raises(TypeError):
+        kda.forward(z, z, z, z, torch.zeros(1, 4, 1))
