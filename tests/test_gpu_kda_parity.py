@@ -65,6 +65,16 @@ def test_small_shapes_ragged_tail(dtype, B, T, H, Dk, Dv):
     compare_heads(to_np(o), o_ref, to_np(ST), S_ref, tol_for(dtype), what=f"{dtype} {B}x{T}x{H}")
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 150, 80), (1, 1000, 1), (3, 700, 5)])
+def test_many_heads_and_segment_splits(B, T, H):
+    """Covers one segment per head (B*H >= SM count) and long per-head segment chains."""
+    inp = _custom(B, T, H, 128, 128, torch.bfloat16, seed=B * T + H)
+    o, ST = _run_gpu(inp)
+    pairs = [(b, h) for b in range(B) for h in range(H)][:12]
+    o_ref, S_ref = _oracle(inp, pairs=pairs)
+    compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", pairs=pairs, what=f"{B}x{T}x{H}")
+
+
 @pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 63, 64, 65])
 def test_short_and_boundary_lengths(T):
     inp = _custom(1, T, 2, 128, 128, torch.bfloat16, seed=T)
