@@ -351,7 +351,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
 
     peaks, peak_kind = read_peaks()
     prof = {}
-    for name in ("kda_generic", "kda_tc_chunk", "kda_tc_state", "kda_tc_output", "conv"):
+    for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "conv"):
         r = kda.profile_collect(name)
         if r and r[1] > 0:
             prof[name] = {"ms_total": r[0], "launches": r[1], "ms_per_launch": r[0] / r[1]}
@@ -369,10 +369,10 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                 "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind,
                 "kernel_ms_per_launch": prof[dominant]["ms_per_launch"]}
 
-    e2e = e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
+    e2e = None if args.quick else e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.quick:
         cpu = cpu_baseline(w)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -408,9 +408,15 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
     ap.add_argument("--extra", action="store_true", help="also time the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="device timing only: no end-to-end leg, no CPU baseline (for profiling)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload on its first N tokens (smaller profiling cases)")
     args = ap.parse_args()
     ws, rank, local = dist_setup()
     w = W.BY_NAME[args.workload]
+    if args.tokens:
+        w = w.resized(T=args.tokens, name=f"{w.name}_first{args.tokens}")
     try:
         if args.impl == "reference":
             run_reference(args, ws, rank, w)

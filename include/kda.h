@@ -185,8 +185,8 @@ void kda_profile_enable(int on);
 /* Waits for the recorded events and returns, for kernel `name`, the summed
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
- * record.  Names: "kda_generic", "kda_tc_chunk", "kda_tc_state", "kda_tc_output",
- * "conv". */
+ * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
+ * "kda_tc_output", "conv". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

@@ -25,7 +25,7 @@
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
 //   pass 2 (MODE_OUTPUT, all segments): run the recurrence from S_start(p) and write
 //          o (and S_T from the last segment).
-// Each pass is one CTA per (b, h, segment), 256 threads, ~200 KB of shared memory.
+// Each pass is one CTA per (b, h, segment), 512 threads, ~200 KB of shared memory.
 //
 // Shared-memory operand tiles use the no-swizzle core-matrix layout: 8 rows x 16 B
 // blocks of 128 contiguous bytes.  A thread that owns one key channel writes 8
@@ -48,7 +48,7 @@ using namespace sm100;
 
 constexpr int C = 64;         // chunk length
 constexpr int D = 128;        // Dk = Dv
-constexpr int NT = 256;       // threads per CTA
+constexpr int NT = 512;       // threads per CTA
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
@@ -56,8 +56,7 @@ enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int NS = 128;                 // state columns (values only)
-    static constexpr int STG = 0;                  // q,k,v,g staging: 4 x [64][128] bf16
-    static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;
+    static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, bf16 [64][128]
     static constexpr int X = 65536;                // K+ | V interleaved (i-group stride 4096); later W
     static constexpr int QP = 98304;               // Q+ (channel-major, i-group stride 2048)
     static constexpr int KM = 114688;              // K-, then fp32 T (16 KB), then T' (8 KB) | P (8 KB)
@@ -69,7 +68,6 @@ template <> struct Plan<MODE_OUTPUT> {
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int NS = 256;                 // [S | Phi]
-    static constexpr int STG = 0;
     static constexpr int stQ = -1, stK = 0, stV = 16384, stG = 32768;
     static constexpr int X = 49152;
     static constexpr int QP = -1;
@@ -82,13 +80,12 @@ template <> struct Plan<MODE_STATE> {
 };
 // MISC sub-layout
 constexpr int M_BETA = 0;        // float[64]
-constexpr int M_REF = 256;       // float[128]  b at row 31 (reference)
-constexpr int M_BC = 768;        // float[128]  b at row 63
-constexpr int M_XS = 1280;       // float[3][256] block products of the inverse
-constexpr int M_BAR = 4352;      // 2 x uint64 mbarriers
-constexpr int M_TMEM = 4368;     // uint32 TMEM base
-constexpr int M_ABORT = 4372;    // int
-constexpr int MISC_BYTES = 4384;
+constexpr int M_TOT = 256;       // float[4][128] per-row-block sums of g
+constexpr int M_XS = 2304;       // float[6][128] per-warp block products of the inverse
+constexpr int M_BAR = 5376;      // 2 x uint64 mbarriers
+constexpr int M_TMEM = 5392;     // uint32 TMEM base
+constexpr int M_ABORT = 5396;    // int
+constexpr int MISC_BYTES = 5408;
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
@@ -123,27 +120,61 @@ struct Ctl {
     uint32_t tma_phase, mma_phase;
 };
 
-// Bounded wait on the MMA barrier; every thread calls it, and the CTA agrees on the
-// outcome at the following __syncthreads.
-__device__ __forceinline__ void wait_mma(Ctl& c)
+// Bounded waits.  One thread polls the mbarrier; the others wait at the barrier
+// (no issue slots spent polling); the CTA then agrees on the outcome through the
+// shared abort flag.  After an MMA wait every thread orders its TMEM reads behind it.
+__device__ __forceinline__ void wait_mma(Ctl& c, int t)
 {
-    if (!mbar_wait_bounded(c.mma_bar, c.mma_phase, kWaitNs)) {
+    if (t == 0 && !mbar_wait_bounded(c.mma_bar, c.mma_phase, kWaitNs)) {
         *c.abort_flag = 1;
         atomicCAS(c.status, DEV_OK, DEV_TIMEOUT);
     }
+    __syncthreads();
     c.mma_phase ^= 1;
     tc_fence_after();
 }
-__device__ __forceinline__ void wait_tma(Ctl& c)
+__device__ __forceinline__ void wait_tma(Ctl& c, int t)
 {
-    if (!mbar_wait_bounded(c.tma_bar, c.tma_phase, kWaitNs)) {
+    if (t == 0 && !mbar_wait_bounded(c.tma_bar, c.tma_phase, kWaitNs)) {
         *c.abort_flag = 1;
         atomicCAS(c.status, DEV_OK, DEV_TIMEOUT);
     }
+    __syncthreads();
     c.tma_phase ^= 1;
 }
 
+// Output rows of one chunk from TMEM (M = 64 layout) to global memory.  Warp (q4, cq)
+// holds rows 16*q4 .. +15 in lanes 0..15 and columns 32*cq .. +31.
+__device__ __forceinline__ void store_o(uint32_t tl, int q4, int cq, int lane, void* o, int o_f32,
+                                        int b, int T, int H, int h, int t0)
+{
+    float v[32];
+    tmem_ld32(tl + TO_O + 32 * cq, v);
+    const int i = 16 * q4 + lane;
+    if (lane < 16 && t0 + i < T) {
+        const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + 32 * cq;
+        if (o_f32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o) + off);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 u;
+                __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+                dst[j] = u;
+            }
+        }
+    }
+}
+
 // The kernel ---------------------------------------------------------------------------
+// Thread roles (512 threads): in the prologue thread t owns key channel c = t & 127 and
+// chunk rows 16*(t >> 7) .. +15; for TMEM, warp w reads lane quarter w & 3 and the
+// column quarter w >> 2 of the accumulator it works on.
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -154,11 +185,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 {
     using PL = Plan<MODE>;
     constexpr int NS = PL::NS;
+    constexpr int NQ = NS / 4;                // state columns per column quarter
     extern __shared__ __align__(1024) uint8_t sm[];
 
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    const int q4 = w & 3, hf = w >> 2;        // TMEM lane quarter, column half
-    const int c = t & 127, rb = t >> 7;       // channel / TMEM row, row block of the prologue
+    const int q4 = w & 3, cq = w >> 2;        // TMEM lane quarter, column quarter
+    const int c = t & 127, rb = t >> 7;       // channel / TMEM row; 16-row block of the prologue
     const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
     const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
     const int b = bh / H, h = bh % H;
@@ -166,8 +198,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int n0 = p * L, n1 = min(NC, n0 + L);
 
     float* sBeta = reinterpret_cast<float*>(sm + PL::MISC + M_BETA);
-    float* sRef = reinterpret_cast<float*>(sm + PL::MISC + M_REF);
-    float* sBC = reinterpret_cast<float*>(sm + PL::MISC + M_BC);
+    float* sTot = reinterpret_cast<float*>(sm + PL::MISC + M_TOT);
     float* sXs = reinterpret_cast<float*>(sm + PL::MISC + M_XS);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
@@ -208,8 +239,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     // ---- initial state in TMEM ------------------------------------------------------
     {
-        const int col0 = hf * (NS / 2);
-        for (int cc = 0; cc < NS / 2; cc += 32) {
+        const int col0 = cq * NQ;
+        for (int cc = 0; cc < NQ; cc += 32) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -229,35 +260,37 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
 
+    int prev_t0 = -1;   // chunk whose output still sits in TMEM (MODE_OUTPUT)
     for (int n = n0; n < n1 && !*sAbort; ++n) {
         const int t0 = n * C;
         // ---- 1. prologue: staging -> fp16 operand tiles --------------------------------
-        wait_tma(ctl);
-        __syncthreads();
+        wait_tma(ctl, t);
         if (*sAbort) break;
         tma_in_flight = false;
         if (t < C) sBeta[t] = (t0 + t < T) ? __bfloat162float(beta[((size_t)b * T + t0 + t) * H + h]) : 0.f;
-        float bl[32];
+        const bool full = t0 + C <= T;   // no ragged rows in this chunk
+        float bl[16];
         {
             const __nv_bfloat16* stg = reinterpret_cast<const __nv_bfloat16*>(sm + PL::stG);
             float run = 0.f;
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int i = 32 * rb + r;
-                run += (t0 + i < T) ? __bfloat162float(stg[i * D + c]) : 0.f;
+            for (int r = 0; r < 16; ++r) {
+                const int i = 16 * rb + r;
+                run += (full || t0 + i < T) ? __bfloat162float(stg[i * D + c]) : 0.f;
                 bl[r] = run;
             }
-            if (rb == 0) sRef[c] = run;
+            sTot[rb * 128 + c] = run;
         }
         __syncthreads();
-        const float rc = sRef[c];
-        if (rb == 1) {
+        float rc, bC;
+        {
+            const float s0 = sTot[c], s1 = sTot[128 + c], s2 = sTot[256 + c], s3 = sTot[384 + c];
+            const float off = (rb > 0 ? s0 : 0.f) + (rb > 1 ? s1 : 0.f) + (rb > 2 ? s2 : 0.f);
 #pragma unroll
-            for (int r = 0; r < 32; ++r) bl[r] += rc;
-            sBC[c] = bl[31];
+            for (int r = 0; r < 16; ++r) bl[r] += off;
+            rc = s0 + s1;               // b at row 31: the reference point
+            bC = s0 + s1 + s2 + s3;     // b at row 63
         }
-        __syncthreads();
-        const float bC = sBC[c];
         {
             const float eCr = __expf(bC - rc);
             const TQ* sk = reinterpret_cast<const TQ*>(sm + PL::stK);
@@ -265,12 +298,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const TQ* sq = reinterpret_cast<const TQ*>(sm + (MODE == MODE_OUTPUT ? PL::stQ : PL::stK));
             const int cofs = (c >> 3) * 128 + (c & 7) * 16;
 #pragma unroll
-            for (int grp = 0; grp < 4; ++grp) {
+            for (int grp = 0; grp < 2; ++grp) {
                 float kp[8], km[8], kt[8], vh[8], qp[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int r = grp * 8 + j, i = 32 * rb + r;
-                    const bool valid = t0 + i < T;
+                    const int r = grp * 8 + j, i = 16 * rb + r;
+                    const bool valid = full || t0 + i < T;
                     const float kk = valid ? ld_in(sk + i * D + c) : 0.f;
                     const float vv = valid ? ld_in(sv + i * D + c) : 0.f;
                     const float x = bl[r] - rc;
@@ -281,7 +314,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     vh[j] = vv;
                     if (MODE == MODE_OUTPUT) qp[j] = (valid ? ld_in(sq + i * D + c) : 0.f) * ep;
                 }
-                const int ig = 4 * rb + grp;   // 8-row group of chunk positions
+                const int ig = 2 * rb + grp;   // 8-row group of chunk positions
                 *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + cofs) = pack8_f16(kp);
                 *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + 2048 + cofs) = pack8_f16(vh);
                 *reinterpret_cast<uint4*>(sm + PL::KM + ig * 2048 + cofs) = pack8_f16(km);
@@ -290,11 +323,29 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(sm + PL::QP + ig * 2048 + cofs) = pack8_f16(qp);
             }
         }
-        // ---- 2. state: S^ = diag(e^r) S (fp16 tile), master *= e^{b_C} ----------------
+        fence_async_smem();
+        __syncthreads();
+        // ---- 2. next chunk's TMA; A = K+ K-^T and P = Q+ K-^T on the tensor core ----------
+        if (t == 0) {
+            if (n + 1 < n1) issue_tma(n + 1);
+            tc_fence_after();
+            const uint32_t id = idesc_f16(64, 64, true, true);
+            const uint32_t tA = (MODE == MODE_OUTPUT) ? TO_A : TS_A;
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t bd = sdesc(sbase + PL::KM + 256 * kk, 128, 2048);
+                umma_f16(tmem + tA, sdesc(sbase + PL::X + 256 * kk, 128, 4096), bd, id, kk > 0);
+                if (MODE == MODE_OUTPUT)
+                    umma_f16(tmem + TO_P, sdesc(sbase + PL::QP + 256 * kk, 128, 2048), bd, id, kk > 0);
+            }
+            umma_commit(ctl.mma_bar);
+        }
+        tma_in_flight = n + 1 < n1;
+        mma_in_flight = true;
+        // ---- 3. while it runs: S^ = diag(e^r) S (fp16 tile), master *= e^{b_C} ----------
         {
             const float er = __expf(rc), eC = __expf(bC);
-            const int col0 = hf * (NS / 2);
-            for (int cc = 0; cc < NS / 2; cc += 32) {
+            const int col0 = cq * NQ;
+            for (int cc = 0; cc < NQ; cc += 32) {
                 float v[32];
                 tmem_ld32(tl + TM_S + col0 + cc, v);
 #pragma unroll
@@ -311,41 +362,31 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_st32(tl + TM_S + col0 + cc, v);
             }
         }
+        // ... and the previous chunk's output leaves TMEM before O is overwritten
+        if (MODE == MODE_OUTPUT && prev_t0 >= 0) store_o(tl, q4, cq, lane, o, o_f32, b, T, H, h, prev_t0);
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // next chunk's inputs can stream in while this one computes
-        if (t == 0 && n + 1 < n1) issue_tma(n + 1);
-        tma_in_flight = n + 1 < n1;
-
-        // ---- 3. A = K+ K-^T (and P = Q+ K-^T) ------------------------------------------
-        if (t == 0) {
+        if (MODE == MODE_OUTPUT && t == 0) {
             tc_fence_after();
-            const uint32_t id = idesc_f16(64, 64, true, true);
-            const uint32_t tA = (MODE == MODE_OUTPUT) ? TO_A : TS_A;
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bd = sdesc(sbase + PL::KM + 256 * kk, 128, 2048);
-                umma_f16(tmem + tA, sdesc(sbase + PL::X + 256 * kk, 128, 4096), bd, id, kk > 0);
-                if (MODE == MODE_OUTPUT)
-                    umma_f16(tmem + TO_P, sdesc(sbase + PL::QP + 256 * kk, 128, 2048), bd, id, kk > 0);
-            }
-            umma_commit(ctl.mma_bar);
+            const uint32_t idq = idesc_f16(64, 128, true, true);
+            for (int kk = 0; kk < 8; ++kk)
+                umma_f16(tmem + TO_O, sdesc(sbase + PL::QP + 256 * kk, 128, 2048),
+                         sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
         }
-        mma_in_flight = true;
-        wait_mma(ctl);
-        mma_in_flight = false;
+        wait_mma(ctl, t);   // A and P are ready (O may still run)
         // A rows -> fp32 (beta-scaled, strictly lower)
         {
-            float v[32];
+            float v[16];
             const uint32_t tA = (MODE == MODE_OUTPUT) ? TO_A : TS_A;
-            tmem_ld32(tl + tA + 32 * hf, v);
+            tmem_ld16(tl + tA + 16 * cq, v);
             if (lane < 16) {
                 const int i = 16 * q4 + lane;
                 const float bi = sBeta[i];
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
+                for (int j4 = 0; j4 < 4; ++j4) {
                     float4 f;
-                    const int j = 32 * hf + 4 * j4;
+                    const int j = 16 * cq + 4 * j4;
                     f.x = (j + 0 < i) ? bi * v[4 * j4 + 0] : 0.f;
                     f.y = (j + 1 < i) ? bi * v[4 * j4 + 1] : 0.f;
                     f.z = (j + 2 < i) ? bi * v[4 * j4 + 2] : 0.f;
@@ -372,67 +413,81 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int r = 0; r < 16; ++r) Tfp[sw(base + r, base + m)] = tc_[r];
         }
         __syncthreads();
+        // block diagonal d: warp (block J, 8-column half) computes
+        //   X = sum_{K=J}^{I-1} A_IK T_KJ  and  T_IJ = -T_II X   (I = J + d)
+        // with m16n8k16 warp MMAs (fp16 operands, fp32 accumulation).
         for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            for (int idx = t; idx < nb * 256; idx += NT) {
-                const int J = idx >> 8, I = J + d, r = (idx >> 4) & 15, cc = idx & 15;
-                float s = 0.f;
-                for (int K = J; K < I; ++K)
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        s = fmaf(Afp[sw(16 * I + r, 16 * K + k)], Tfp[sw(16 * K + k, 16 * J + cc)], s);
-                sXs[idx] = s;
-            }
-            __syncthreads();
-            for (int idx = t; idx < nb * 256; idx += NT) {
-                const int J = idx >> 8, I = J + d, r = (idx >> 4) & 15, cc = idx & 15;
-                float s = 0.f;
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    s = fmaf(Tfp[sw(16 * I + r, 16 * I + k)], sXs[(J << 8) + k * 16 + cc], s);
-                Tfp[sw(16 * I + r, 16 * J + cc)] = -s;
+            if (w < 2 * (4 - d)) {
+                const int J = w >> 1, I = J + d, N0 = 16 * J + 8 * (w & 1);
+                const int g = lane >> 2, q = lane & 3;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int K = J; K < I; ++K) {
+                    uint32_t a[4], bb[2];
+                    const int r0 = 16 * I + g, c0 = 16 * K + 2 * q;
+                    a[0] = pack_f16x2(Afp[sw(r0, c0)], Afp[sw(r0, c0 + 1)]);
+                    a[1] = pack_f16x2(Afp[sw(r0 + 8, c0)], Afp[sw(r0 + 8, c0 + 1)]);
+                    a[2] = pack_f16x2(Afp[sw(r0, c0 + 8)], Afp[sw(r0, c0 + 9)]);
+                    a[3] = pack_f16x2(Afp[sw(r0 + 8, c0 + 8)], Afp[sw(r0 + 8, c0 + 9)]);
+                    const int k0 = 16 * K + 2 * q, n = N0 + g;
+                    bb[0] = pack_f16x2(Tfp[sw(k0, n)], Tfp[sw(k0 + 1, n)]);
+                    bb[1] = pack_f16x2(Tfp[sw(k0 + 8, n)], Tfp[sw(k0 + 9, n)]);
+                    mma16816(acc, a, bb);
+                }
+                // X (C fragment) -> this warp's scratch, then back as a B fragment
+                float* xs = sXs + 128 * w;      // [16][8]
+                xs[g * 8 + 2 * q] = acc[0];
+                xs[g * 8 + 2 * q + 1] = acc[1];
+                xs[(g + 8) * 8 + 2 * q] = acc[2];
+                xs[(g + 8) * 8 + 2 * q + 1] = acc[3];
+                __syncwarp();
+                uint32_t a[4], bb[2];
+                {
+                    const int r0 = 16 * I + g, c0 = 16 * I + 2 * q;
+                    a[0] = pack_f16x2(Tfp[sw(r0, c0)], Tfp[sw(r0, c0 + 1)]);
+                    a[1] = pack_f16x2(Tfp[sw(r0 + 8, c0)], Tfp[sw(r0 + 8, c0 + 1)]);
+                    a[2] = pack_f16x2(Tfp[sw(r0, c0 + 8)], Tfp[sw(r0, c0 + 9)]);
+                    a[3] = pack_f16x2(Tfp[sw(r0 + 8, c0 + 8)], Tfp[sw(r0 + 8, c0 + 9)]);
+                    bb[0] = pack_f16x2(xs[(2 * q) * 8 + g], xs[(2 * q + 1) * 8 + g]);
+                    bb[1] = pack_f16x2(xs[(2 * q + 8) * 8 + g], xs[(2 * q + 9) * 8 + g]);
+                }
+                float tt[4] = {0.f, 0.f, 0.f, 0.f};
+                mma16816(tt, a, bb);
+                const int r0 = 16 * I + g, c0 = N0 + 2 * q;
+                *reinterpret_cast<float2*>(Tfp + sw(r0, c0)) = make_float2(-tt[0], -tt[1]);
+                *reinterpret_cast<float2*>(Tfp + sw(r0 + 8, c0)) = make_float2(-tt[2], -tt[3]);
             }
             __syncthreads();
         }
         // T' = T diag(beta), lower part only, fp16 K-major tile [i][j] at KM
         {
-            float vals[2][8];
-            int ii[2], jg[2];
+            const int ii = t >> 3, jg = t & 7;     // 512 (row, 8-column group) pairs
+            float vals[8];
+            const float4 a0 = *reinterpret_cast<const float4*>(Tfp + sw(ii, 8 * jg));
+            const float4 a1 = *reinterpret_cast<const float4*>(Tfp + sw(ii, 8 * jg + 4));
+            const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int idx = t + u * NT;       // 512 (row, 8-column group) pairs
-                ii[u] = idx >> 3;
-                jg[u] = idx & 7;
-                const float4 a0 = *reinterpret_cast<const float4*>(Tfp + sw(ii[u], 8 * jg[u]));
-                const float4 a1 = *reinterpret_cast<const float4*>(Tfp + sw(ii[u], 8 * jg[u] + 4));
-                const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int col = 8 * jg[u] + j;
-                    vals[u][j] = (col <= ii[u]) ? f[j] * sBeta[col] : 0.f;
-                }
+            for (int j = 0; j < 8; ++j) {
+                const int col = 8 * jg + j;
+                vals[j] = (col <= ii) ? f[j] * sBeta[col] : 0.f;
             }
             __syncthreads();
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-                *reinterpret_cast<uint4*>(sm + PL::KM + jg[u] * 1024 + (ii[u] >> 3) * 128 + (ii[u] & 7) * 16) =
-                    pack8_f16(vals[u]);
+            *reinterpret_cast<uint4*>(sm + PL::KM + jg * 1024 + (ii >> 3) * 128 + (ii & 7) * 16) = pack8_f16(vals);
         }
         // P (masked, fp16 K-major) next to T'
         if (MODE == MODE_OUTPUT) {
-            float v[32];
-            tmem_ld32(tl + TO_P + 32 * hf, v);
+            float v[16];
+            tmem_ld16(tl + TO_P + 16 * cq, v);
             if (lane < 16) {
                 const int i = 16 * q4 + lane;
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
+                for (int g8 = 0; g8 < 2; ++g8) {
                     float f[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const int col = 32 * hf + 8 * g8 + j;
+                        const int col = 16 * cq + 8 * g8 + j;
                         f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
                     }
-                    const int jgp = 4 * hf + g8;
+                    const int jgp = 2 * cq + g8;
                     *reinterpret_cast<uint4*>(sm + PL::KM + 8192 + jgp * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
                         pack8_f16(f);
                 }
@@ -441,7 +496,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- 5. U~ = T' V,  W = T' K+  (and O = Q+ S^) ---------------------------------
+        // ---- 5. U~ = T' V,  W = T' K+ -----------------------------------------------------
         if (t == 0) {
             tc_fence_after();
             const uint32_t id128 = idesc_f16(64, 128, false, false);
@@ -452,31 +507,21 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 umma_f16(tmem + tU, ad, sdesc(sbase + PL::X + 2048 + 8192 * kk, 4096, 128), id128, kk > 0);
                 umma_f16(tmem + tW, ad, sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id128, kk > 0);
             }
-            if (MODE == MODE_OUTPUT) {
-                const uint32_t idq = idesc_f16(64, 128, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + TO_O, sdesc(sbase + PL::QP + 256 * kk, 128, 2048),
-                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
-            }
             umma_commit(ctl.mma_bar);
         }
-        mma_in_flight = true;
-        wait_mma(ctl);
-        mma_in_flight = false;
+        wait_mma(ctl, t);
         // W -> fp16 K-major tile [i][c] at X (K+ | V are no longer needed)
         {
             const uint32_t tW = (MODE == MODE_OUTPUT) ? TO_W : TS_W;
-            for (int cc = 0; cc < 64; cc += 32) {
-                float v[32];
-                tmem_ld32(tl + tW + 64 * hf + cc, v);
-                if (lane < 16) {
-                    const int i = 16 * q4 + lane;
+            float v[32];
+            tmem_ld32(tl + tW + 32 * cq, v);
+            if (lane < 16) {
+                const int i = 16 * q4 + lane;
 #pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        const int cg = (64 * hf + cc) / 8 + g8;
-                        *reinterpret_cast<uint4*>(sm + PL::X + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                            pack8_f16(&v[8 * g8]);
-                    }
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int cg = 4 * cq + g8;
+                    *reinterpret_cast<uint4*>(sm + PL::X + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
+                        pack8_f16(&v[8 * g8]);
                 }
             }
         }
@@ -500,21 +545,18 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             umma_commit(ctl.mma_bar);
         }
-        mma_in_flight = true;
-        wait_mma(ctl);
-        mma_in_flight = false;
+        wait_mma(ctl, t);
         // U -> fp16 MN-major tile [i][col] at U
         {
             const uint32_t tU = (MODE == MODE_OUTPUT) ? TO_U : TS_R;
-            constexpr int NU = NS;                 // 128 or 256 columns (contiguous in TMEM)
-            for (int cc = 0; cc < NU / 2; cc += 32) {
+            for (int cc = 0; cc < NQ; cc += 32) {
                 float v[32];
-                tmem_ld32(tl + tU + hf * (NU / 2) + cc, v);
+                tmem_ld32(tl + tU + cq * NQ + cc, v);
                 if (lane < 16) {
                     const int i = 16 * q4 + lane;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
-                        const int cg = (hf * (NU / 2) + cc) / 8 + g8;
+                        const int cg = (cq * NQ + cc) / 8 + g8;
                         *reinterpret_cast<uint4*>(sm + PL::U + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
                             pack8_f16(&v[8 * g8]);
                     }
@@ -539,38 +581,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             umma_commit(ctl.mma_bar);
         }
-        mma_in_flight = true;
-        wait_mma(ctl);
+        wait_mma(ctl, t);
         mma_in_flight = false;
-        // ---- 8. outputs ----------------------------------------------------------------
-        if (MODE == MODE_OUTPUT) {
-            for (int cc = 0; cc < 64; cc += 32) {
-                float v[32];
-                tmem_ld32(tl + TO_O + 64 * hf + cc, v);
-                const int i = 16 * q4 + lane;
-                if (lane < 16 && t0 + i < T) {
-                    const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + 64 * hf + cc;
-                    if (o_f32) {
-                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    } else {
-                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o) + off);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 u;
-                            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-                            dst[j] = u;
-                        }
-                    }
-                }
-            }
-        }
+        prev_t0 = t0;
         tc_fence_before();
         __syncthreads();
     }
+    if (MODE == MODE_OUTPUT && !*sAbort && prev_t0 >= 0)
+        store_o(tl, q4, cq, lane, o, o_f32, b, T, H, h, prev_t0);
 
     // ---- end of segment: write the state ------------------------------------------------
     if (!*sAbort) {
@@ -578,8 +596,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (MODE == MODE_STATE) dst = maps + (size_t)(bh * (P - 1) + p) * 2 * D * D;  // [N | M]
         else if (S_T && p == P - 1) dst = S_T + (size_t)bh * D * D;
         if (dst) {
-            const int col0 = hf * (NS / 2);
-            for (int cc = 0; cc < NS / 2; cc += 32) {
+            const int col0 = cq * NQ;
+            for (int cc = 0; cc < NQ; cc += 32) {
                 float v[32];
                 tmem_ld32(tl + TM_S + col0 + cc, v);
 #pragma unroll
@@ -605,40 +623,68 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
-// S_start(p+1) = M_p S_start(p) + N_p, fp32 on CUDA cores.  Grid (D/8, H, B), 128
-// threads: thread c owns row c of an 8-column slice of the state.
-__global__ void __launch_bounds__(128)
+// S_start(p+1) = M_p S_start(p) + N_p in fp32 on CUDA cores.  Grid (D/16, H, B), 256
+// threads: thread t owns row t/2 and 8 of the CTA's 16 state columns.  M_{p+1} streams
+// into the second shared buffer (cp.async) while step p computes from the first.
+constexpr int CB_THREADS = 256;
+constexpr int CB_LD = 132;      // row stride in floats (16-byte rows for cp.async)
+constexpr int cb_smem_bytes() { return (2 * D * CB_LD + D * 16) * (int)sizeof(float); }
+
+__device__ __forceinline__ void cb_stage(float* dst, const float* M, int t)
+{
+#pragma unroll
+    for (int u = 0; u < D * D / 4 / CB_THREADS; ++u) {
+        const int i = t + u * CB_THREADS, row = i >> 5, col = (i & 31) * 4;
+        cp_async16(dst + row * CB_LD + col, M + (size_t)row * D + col);
+    }
+    cp_async_commit();
+}
+
+__global__ void __launch_bounds__(CB_THREADS)
 kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
                    float* __restrict__ starts, int H, int P)
 {
-    __shared__ float sS[D][8];
-    const int c = threadIdx.x, col0 = blockIdx.x * 8;
+    extern __shared__ __align__(16) float csm[];
+    float* sS = csm + 2 * D * CB_LD;     // [128][16]
+    const int t = threadIdx.x, col0 = blockIdx.x * 16;
     const int bh = blockIdx.z * H + blockIdx.y;
+    const int r = t >> 1, c8 = (t & 1) * 8;
+    const float* mp = maps + (size_t)bh * (P - 1) * 2 * D * D;   // [P-1][N | M]
+    if (P > 1) cb_stage(csm, mp + D * D, t);
     float s[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s[j] = S0 ? S0[((size_t)bh * D + c) * D + col0 + j] : 0.f;
+    for (int j = 0; j < 8; ++j) s[j] = S0 ? S0[((size_t)bh * D + r) * D + col0 + c8 + j] : 0.f;
     for (int p = 0; p < P; ++p) {
-        float* out = starts + ((size_t)bh * P + p) * D * D + (size_t)c * D + col0;
+        float* out = starts + ((size_t)bh * P + p) * D * D + (size_t)r * D + col0 + c8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) out[j] = s[j];
         if (p == P - 1) break;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) sS[c][j] = s[j];
-        __syncthreads();
-        const float* Nm = maps + ((size_t)bh * (P - 1) + p) * 2 * D * D;
-        const float* Mm = Nm + D * D;
+        const float* Nm = mp + (size_t)p * 2 * D * D;
         float acc[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = Nm[(size_t)c * D + col0 + j];
-        const float4* mrow = reinterpret_cast<const float4*>(Mm + (size_t)c * D);
+        for (int j = 0; j < 8; ++j) acc[j] = Nm[(size_t)r * D + col0 + c8 + j];
+        __syncthreads();                         // sS and the other buffer are free
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sS[r * 16 + c8 + j] = s[j];
+        if (p + 1 < P - 1) cb_stage(csm + ((p + 1) & 1) * D * CB_LD, mp + (size_t)(p + 1) * 2 * D * D + D * D, t);
+        if (p + 1 < P - 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else cp_async_wait_all();
+        __syncthreads();                         // M_p staged, sS written
+        const float* sM = csm + (p & 1) * D * CB_LD;
+#pragma unroll 4
         for (int k4 = 0; k4 < D / 4; ++k4) {
-            const float4 m = mrow[k4];
+            const float4 m = *reinterpret_cast<const float4*>(sM + r * CB_LD + 4 * k4);
             const float mk[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk[u], sS[4 * k4 + u][j], acc[j]);
+            for (int u = 0; u < 4; ++u) {
+                const int k = 4 * k4 + u;
+                const float4 s0 = *reinterpret_cast<const float4*>(sS + k * 16 + c8);
+                const float4 s1 = *reinterpret_cast<const float4*>(sS + k * 16 + c8 + 4);
+                acc[0] = fmaf(mk[u], s0.x, acc[0]); acc[1] = fmaf(mk[u], s0.y, acc[1]);
+                acc[2] = fmaf(mk[u], s0.z, acc[2]); acc[3] = fmaf(mk[u], s0.w, acc[3]);
+                acc[4] = fmaf(mk[u], s1.x, acc[4]); acc[5] = fmaf(mk[u], s1.y, acc[5]);
+                acc[6] = fmaf(mk[u], s1.z, acc[6]); acc[7] = fmaf(mk[u], s1.w, acc[7]);
+            }
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) s[j] = acc[j];
@@ -731,9 +777,11 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
     cudaError_t e = launch_pass<MODE_STATE, TQ>(mq, mk, mv, mg, a, nullptr, 0, maps, sp.P, sp.L, status, s);
     if (e != cudaSuccess) return e;
     {
+        e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb_smem_bytes());
+        if (e != cudaSuccess) return e;
         ProfileScope prof("kda_tc_combine", s);
         count_launch();
-        kda_combine_kernel<<<dim3(D / 8, a.H, a.B), 128, 0, s>>>(maps, a.S0, starts, a.H, sp.P);
+        kda_combine_kernel<<<dim3(D / 16, a.H, a.B), CB_THREADS, cb_smem_bytes(), s>>>(maps, a.S0, starts, a.H, sp.P);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
