@@ -105,6 +105,36 @@ kda_status kda_forward(const void* q, const void* k, const void* v, const void* 
                        kda_dtype o_dtype, int chunk, void* workspace, size_t workspace_bytes,
                        kda_stream_t stream);
 
+/* Size of the scratch array compiled into the library for kda_forward_noalloc. */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * kda_forward_noalloc -- kda_forward that allocates no device memory.  The paper has
+ * no counterpart to this call; it exists for callers that cannot allocate during a
+ * call: code inside a host framework that owns all device memory through its own
+ * allocator and forbids raw allocation in its call path (inference-engine plugins,
+ * serving loops on a fixed memory plan), or code that must not risk an allocation
+ * failing or stalling mid-call.
+ *
+ * Same arguments and results as kda_forward, minus the workspace.  Its scratch comes
+ * from one array of KDA_NOALLOC_SCRATCH_BYTES compiled into the library, held in the
+ * device memory of every GPU on which the library is loaded until the process exits.
+ *   - The first call on a device looks up that array's device address (once per
+ *     device, with the device current); make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the array and it keeps the last call's contents.
+ *     Every byte a call reads from it is written earlier in the same call, so nothing
+ *     needs clearing; calls whose GPU work may overlap (different streams without
+ *     ordering between them) race on it.
+ *   - A problem whose scratch need exceeds KDA_NOALLOC_SCRATCH_BYTES returns
+ *     KDA_ERR_WORKSPACE before any launch (on a 148-SM B200 every shape fits: the
+ *     need is at most about 28 MiB).
+ */
+kda_status kda_forward_noalloc(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* S0, void* o, float* S_T,
+                               int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                               kda_dtype o_dtype, int chunk, kda_stream_t stream);
+
 /* Modalities of a packed-stream segment (section 3.4). */
 typedef enum { MSC_TEXT = 0, MSC_IMAGE = 1, MSC_VIDEO = 2 } msc_modality;
 

@@ -26,7 +26,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace_size",
             "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
-            "kda_profile_collect")
+            "kda_profile_collect", "kda_forward_noalloc")
 
 
 class KdaError(RuntimeError):
@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH):
         lib.kda_mshortconv_forward.restype = I
         lib.kda_mshortconv_forward.argtypes = [P, P, P, P, I, I, P, P, P, P, P, P, P, P,
                                                I, I, I, I, I, I, I, P, Z, P]
+        lib.kda_forward_noalloc.restype = I
+        lib.kda_forward_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
         lib.kda_kernel_launches.restype = ctypes.c_uint64
         lib.kda_kernel_launches.argtypes = []
         lib.kda_profile_enable.restype = None
@@ -154,6 +156,32 @@ def forward(q, k, v, g, beta, S0=None, *, chunk: int = 0, o=None, S_T=None,
                          _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv, dt, _code(o_dtype),
                          chunk, ws_ptr, ws_bytes, _stream(stream))
     _check("kda_forward", rc)
+    return o, S_T
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def forward_noalloc(q, k, v, g, beta, S0=None, *, chunk: int = 0, o=None, S_T=None,
+                    stream=None, o_dtype=None):
+    """kda_forward_noalloc: the same scan as forward() with its scratch taken from the
+    array compiled into the library (no device allocation inside the call).  The
+    caller supplies every tensor, outputs included (created here only for convenience
+    when not given)."""
+    lib = load_library()
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o_dtype = o_dtype or (o.dtype if o is not None else q.dtype)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    rc = lib.kda_forward_noalloc(_dev(q, "q"), _dev(k, "k", q.dtype), _dev(v, "v", q.dtype),
+                                 _dev(g, "g", q.dtype), _dev(beta, "beta", q.dtype),
+                                 _dev(S0, "S0", torch.float32), _dev(o, "o", o_dtype),
+                                 _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv,
+                                 _dtype_code(q), _code(o_dtype), chunk, _stream(stream))
+    _check("kda_forward_noalloc", rc)
     return o, S_T
 
 
