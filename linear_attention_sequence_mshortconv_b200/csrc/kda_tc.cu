@@ -6,10 +6,10 @@
 // entry state S0, b_i = sum_{r<=i} g_r (fp32, per key channel), a reference point
 // r = b_31 (the middle of the chunk) keeps every exponential within e^{+-|b|/2}:
 //   K+ = k e^{b - r},  Q+ = q e^{b - r},  K- = k e^{r - b},  Kt = k e^{b_C - b}
-//   A  = diag(beta) strict_lower(K+ K-^T),   P = lower(Q+ K-^T)      (incl. diagonal)
-//   T' = (I + A)^{-1} diag(beta)                                  (blocked, fp32)
+//   A  = strict_lower((diag(beta) K+) K-^T),   P = lower(Q+ K-^T)  (incl. diagonal)
+//   T  = (I + A)^{-1}                     (16x16 blocks on warp MMAs, fp16 operands)
 //   S^ = diag(e^{r}) S0                                           (state seen by K+, Q+)
-//   U  = T' V - (T' K+) S^              O = Q+ S^ + P U
+//   U  = T (beta V) - (T (beta K+)) S^     O = Q+ S^ + P U
 //   S_C = diag(e^{b_C}) S0 + Kt^T U
 // Every MMA operand is fp16 in shared memory (11-bit significand: bf16 operands
 // would cost ~3% of RMS(o) in max error), accumulation is fp32 in TMEM, and the
@@ -25,7 +25,7 @@
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
 //   pass 2 (MODE_OUTPUT, all segments): run the recurrence from S_start(p) and write
 //          o (and S_T from the last segment).
-// Each pass is one CTA per (b, h, segment), 512 threads, ~200 KB of shared memory.
+// Each pass is one CTA per (b, h, segment), 512 threads, up to ~222 KB of shared memory.
 //
 // Shared-memory operand tiles use the no-swizzle core-matrix layout: 8 rows x 16 B
 // blocks of 128 contiguous bytes.  A thread that owns one key channel writes 8
@@ -53,48 +53,52 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
 // ---- shared-memory plan (bytes) --------------------------------------------------
+// MODE_OUTPUT stacks Q+ under K+ so that one M = 128 MMA gives A and P: the block
+// XY holds, per 8-row group of chunk positions ig, [K+ | V] at XY + ig*4096 and
+// [Q+ | K-] at XY + 32768 + ig*4096 (channel-major 2 KB halves).
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int NS = 128;                 // state columns (values only)
-    static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, bf16 [64][128]
-    static constexpr int X = 65536;                // K+ | V interleaved (i-group stride 4096); later W
-    static constexpr int QP = 98304;               // Q+ (channel-major, i-group stride 2048)
-    static constexpr int KM = 114688;              // K-, then fp32 T (16 KB), then T' (8 KB) | P (8 KB)
-    static constexpr int KT = 131072;              // Kt
-    static constexpr int U = 147456;               // fp32 A during the inverse, then U (64 x 128 fp16)
-    static constexpr int S = 163840;               // S^ (128 x 128 fp16)
-    static constexpr int MISC = 196608;
+    static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, [64][128]
+    static constexpr int X = 65536;                // [K+ | V]; later W (64 x 128 fp16, K-major)
+    static constexpr int Y = 98304;                // [Q+ | K-]
+    static constexpr int TF = 131072;              // T = (I + A)^{-1} (64 x 64 fp16, K-major), 8 KB used
+    static constexpr int PT = 147456;              // P (8 KB)
+    static constexpr int KT = 155648;              // Kt
+    static constexpr int U = 172032;               // fp16 A during the inverse, then U (64 x 128)
+    static constexpr int S = 188416;               // S^ (128 x 128 fp16)
+    static constexpr int MISC = 221184;
     static constexpr int TMA_BYTES = 4 * 16384;
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int NS = 256;                 // [S | Phi]
     static constexpr int stQ = -1, stK = 0, stV = 16384, stG = 32768;
-    static constexpr int X = 49152;
-    static constexpr int QP = -1;
-    static constexpr int KM = 81920;
+    static constexpr int X = 49152;                // [K+ | V]; later W
+    static constexpr int Y = -1;
+    static constexpr int TF = 81920;               // K- (the T tile lives at U + 8192 here)
+    static constexpr int PT = -1;
     static constexpr int KT = 98304;
-    static constexpr int U = 114688;               // 64 x 256 fp16
-    static constexpr int S = 147456;               // 128 x 256 fp16
+    static constexpr int U = 114688;               // fp16 A and T during the inverse, then U (64 x 256)
+    static constexpr int S = 147456;               // S^ (128 x 256 fp16)
     static constexpr int MISC = 212992;
     static constexpr int TMA_BYTES = 3 * 16384;
 };
 // MISC sub-layout
 constexpr int M_BETA = 0;        // float[64]
 constexpr int M_TOT = 256;       // float[4][128] per-row-block sums of g
-constexpr int M_XS = 2304;       // float[6][128] per-warp block products of the inverse
-constexpr int M_BAR = 5376;      // 2 x uint64 mbarriers
-constexpr int M_TMEM = 5392;     // uint32 TMEM base
-constexpr int M_ABORT = 5396;    // int
-constexpr int MISC_BYTES = 5408;
+constexpr int M_XS = 2304;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 6400;      // 2 x uint64 mbarriers
+constexpr int M_TMEM = 6416;     // uint32 TMEM base
+constexpr int M_ABORT = 6420;    // int
+constexpr int MISC_BYTES = 6432;
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
-// TMEM columns
-constexpr uint32_t TM_S = 0;       // state master (fp32), 128 or 256 columns
-// MODE_OUTPUT
-constexpr uint32_t TO_U = 128, TO_A = 256, TO_P = 320, TO_W = 256, TO_O = 384;
-// MODE_STATE
-constexpr uint32_t TS_A = 256, TS_R = 256, TS_W = 384;
+// TMEM columns.  W and U~ come out of one N = 256 MMA as [W | U~].
+constexpr uint32_t TM_S = 0;                      // state master (fp32), 128 or 256 columns
+constexpr uint32_t TO_O = 128;                    // MODE_OUTPUT: O (M = 64), 128 columns
+constexpr uint32_t T_AP = 256;                    // A (and P below it in MODE_OUTPUT), 64 columns
+constexpr uint32_t T_W = 256, T_U = 384;          // W, then U~ -> U (M = 64), 128 columns each
 
 // ---- helpers ------------------------------------------------------------------------
 __device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat162float(*p); }
@@ -109,8 +113,46 @@ __device__ __forceinline__ uint4 pack8_f16(const float* f)
     return u;
 }
 
-// fp32 64x64 with an XOR swizzle on 4-column groups (conflict-free row and column use)
-__device__ __forceinline__ int sw(int i, int j) { return i * 64 + (j ^ ((i & 7) << 2)); }
+// Byte offset of (row i, column j), j % 8 == 0, in a 64 x 64 fp16 tile in the
+// K-major core-matrix layout the tensor-core MMA reads (8-column groups 1 KB apart).
+__device__ __forceinline__ uint32_t cm64(int i, int j) { return (j >> 3) * 1024 + (i >> 3) * 128 + (i & 7) * 16; }
+// Same for a 16 x 16 scratch block (8-column groups 256 B apart).
+__device__ __forceinline__ uint32_t cm16(int i, int j) { return (j >> 3) * 256 + (i >> 3) * 128 + (i & 7) * 16; }
+
+// Warp-MMA helpers on 16x16 blocks.  A C fragment pair (two n-halves) is exactly the
+// A fragment of the next product; B fragments go through a per-warp scratch block.
+__device__ __forceinline__ void c_to_a(uint32_t (&a)[4], const float (&c0)[4], const float (&c1)[4])
+{
+    a[0] = pack_f16x2(c0[0], c0[1]);
+    a[1] = pack_f16x2(c0[2], c0[3]);
+    a[2] = pack_f16x2(c1[0], c1[1]);
+    a[3] = pack_f16x2(c1[2], c1[3]);
+}
+// C fragments (rows g, g+8; columns 2q, 2q+1 of each n-half) -> 16x16 fp16 scratch
+__device__ __forceinline__ void c_to_scr(uint32_t scr, int lane, const float (&c0)[4], const float (&c1)[4])
+{
+    const int g = lane >> 2, q = lane & 3;
+    st_shared_b32(scr + cm16(g, 0) + 4 * q, pack_f16x2(c0[0], c0[1]));
+    st_shared_b32(scr + cm16(g + 8, 0) + 4 * q, pack_f16x2(c0[2], c0[3]));
+    st_shared_b32(scr + cm16(g, 8) + 4 * q, pack_f16x2(c1[0], c1[1]));
+    st_shared_b32(scr + cm16(g + 8, 8) + 4 * q, pack_f16x2(c1[2], c1[3]));
+}
+// B fragments (both n-halves) of a 16x16 block stored [k][n] in the scratch
+__device__ __forceinline__ void scr_to_b(uint32_t (&b)[4], uint32_t scr, int lane)
+{
+    ldsm_x4_t(b, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 8 * (lane >> 4)));
+}
+__device__ __forceinline__ void mma_16x16(float (&c0)[4], float (&c1)[4], const uint32_t (&a)[4], const uint32_t (&b)[4])
+{
+    const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
+    mma16816(c0, a, b0);
+    mma16816(c1, a, b1);
+}
+
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 struct Ctl {
     uint64_t* tma_bar;
@@ -120,61 +162,60 @@ struct Ctl {
     uint32_t tma_phase, mma_phase;
 };
 
-// Bounded waits.  One thread polls the mbarrier; the others wait at the barrier
-// (no issue slots spent polling); the CTA then agrees on the outcome through the
-// shared abort flag.  After an MMA wait every thread orders its TMEM reads behind it.
-__device__ __forceinline__ void wait_mma(Ctl& c, int t)
+// Bounded waits.  One thread polls the mbarrier; the others wait at a barrier (no
+// issue slots spent polling): the whole CTA (bar_id 0) or one 256-thread group.  The
+// CTA agrees on a timeout through the shared abort flag.  After an MMA wait every
+// thread orders its TMEM reads behind it.
+__device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t& phase, Ctl& c, bool poller, int bar_id)
 {
-    if (t == 0 && !mbar_wait_bounded(c.mma_bar, c.mma_phase, kWaitNs)) {
+    if (poller && !mbar_wait_bounded(bar, phase, kWaitNs)) {
         *c.abort_flag = 1;
         atomicCAS(c.status, DEV_OK, DEV_TIMEOUT);
     }
-    __syncthreads();
-    c.mma_phase ^= 1;
+    if (bar_id == 0) __syncthreads();
+    else named_sync(bar_id, NT / 2);
+    phase ^= 1;
     tc_fence_after();
 }
-__device__ __forceinline__ void wait_tma(Ctl& c, int t)
-{
-    if (t == 0 && !mbar_wait_bounded(c.tma_bar, c.tma_phase, kWaitNs)) {
-        *c.abort_flag = 1;
-        atomicCAS(c.status, DEV_OK, DEV_TIMEOUT);
-    }
-    __syncthreads();
-    c.tma_phase ^= 1;
-}
+__device__ __forceinline__ void wait_mma(Ctl& c, int t) { wait_bar(c.mma_bar, c.mma_phase, c, t == 0, 0); }
+__device__ __forceinline__ void wait_tma(Ctl& c, int t) { wait_bar(c.tma_bar, c.tma_phase, c, t == 0, 0); }
 
-// Output rows of one chunk from TMEM (M = 64 layout) to global memory.  Warp (q4, cq)
-// holds rows 16*q4 .. +15 in lanes 0..15 and columns 32*cq .. +31.
-__device__ __forceinline__ void store_o(uint32_t tl, int q4, int cq, int lane, void* o, int o_f32,
+// Output rows of one chunk from TMEM (M = 64 layout: row 16*q4 + l in lane 32*q4 + l,
+// l < 16) to global memory; this warp stores columns col0 .. col0 + 32*nld - 1.
+__device__ __forceinline__ void store_o(uint32_t tl, int q4, int col0, int nld, int lane, void* o, int o_f32,
                                         int b, int T, int H, int h, int t0)
 {
-    float v[32];
-    tmem_ld32(tl + TO_O + 32 * cq, v);
-    const int i = 16 * q4 + lane;
-    if (lane < 16 && t0 + i < T) {
-        const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + 32 * cq;
-        if (o_f32) {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
+    for (int u = 0; u < nld; ++u) {
+        float v[32];
+        const int cc = col0 + 32 * u;
+        tmem_ld32(tl + TO_O + cc, v);
+        const int i = 16 * q4 + lane;
+        if (lane < 16 && t0 + i < T) {
+            const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + cc;
+            if (o_f32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o) + off);
+                for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o) + off);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 u;
-                __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&u);
+                for (int j = 0; j < 4; ++j) {
+                    uint4 uu;
+                    __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-                dst[j] = u;
+                    for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+                    dst[j] = uu;
+                }
             }
         }
     }
 }
 
 // The kernel ---------------------------------------------------------------------------
-// Thread roles (512 threads): in the prologue thread t owns key channel c = t & 127 and
-// chunk rows 16*(t >> 7) .. +15; for TMEM, warp w reads lane quarter w & 3 and the
-// column quarter w >> 2 of the accumulator it works on.
+// 512 threads.  Prologue: thread t owns key channel c = t & 127 and chunk rows
+// 16*(t >> 7) .. +15.  TMEM: warp w reads lane quarter w & 3.  While warps 0-7 read A
+// and invert (I + A), warps 8-15 rescale the state, store the previous chunk's output
+// and read P.
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -185,11 +226,16 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 {
     using PL = Plan<MODE>;
     constexpr int NS = PL::NS;
-    constexpr int NQ = NS / 4;                // state columns per column quarter
+    constexpr int NQ = NS / 4;                // state columns per column quarter (all 16 warps)
+    constexpr int KM = (MODE == MODE_OUTPUT) ? PL::Y + 2048 : PL::TF;   // K- tile base
+    constexpr int KM_IG = (MODE == MODE_OUTPUT) ? 4096 : 2048;          // its 8-row group stride
+    constexpr int TT = (MODE == MODE_OUTPUT) ? PL::TF : PL::U + 8192;   // T tile base
     extern __shared__ __align__(1024) uint8_t sm[];
 
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     const int q4 = w & 3, cq = w >> 2;        // TMEM lane quarter, column quarter
+    const bool grpY = w >= 8;                 // second 256-thread group
+    const int hg = (w >> 2) & 1;              // column half inside a group
     const int c = t & 127, rb = t >> 7;       // channel / TMEM row; 16-row block of the prologue
     const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
     const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
@@ -203,8 +249,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
     int* sAbort = reinterpret_cast<int*>(sm + PL::MISC + M_ABORT);
-    float* Afp = reinterpret_cast<float*>(sm + PL::U);    // during the inverse
-    float* Tfp = reinterpret_cast<float*>(sm + PL::KM);   // during the inverse
     const uint32_t sbase = smem_addr(sm);
 
     Ctl ctl{&bars[0], &bars[1], sAbort, status, 0u, 0u};
@@ -234,8 +278,16 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tma_load_3d(sm + PL::stV, &tm_v, ctl.tma_bar, 0, h, row);
         tma_load_3d(sm + PL::stG, &tm_g, ctl.tma_bar, 0, h, row);
     };
+    // beta is prefetched one chunk ahead as raw bf16 bits (no use until the next chunk,
+    // so the load never stalls the thread); the index is clamped to stay in bounds.
+    auto load_beta_bits = [&](int n) -> uint32_t {
+        const int tt = n * C + t;
+        const int ts = (n < n1 && tt < T) ? tt : 0;
+        return *reinterpret_cast<const unsigned short*>(beta + ((size_t)b * T + ts) * H + h);
+    };
     if (t == 0 && n0 < n1) issue_tma(n0);
     tma_in_flight = n0 < n1;
+    uint32_t beta_bits = (t < C) ? load_beta_bits(n0) : 0u;
 
     // ---- initial state in TMEM ------------------------------------------------------
     {
@@ -267,7 +319,10 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         wait_tma(ctl, t);
         if (*sAbort) break;
         tma_in_flight = false;
-        if (t < C) sBeta[t] = (t0 + t < T) ? __bfloat162float(beta[((size_t)b * T + t0 + t) * H + h]) : 0.f;
+        if (t < C) {
+            sBeta[t] = (t0 + t < T) ? __uint_as_float(beta_bits << 16) : 0.f;
+            beta_bits = load_beta_bits(n + 1);    // in flight during this chunk
+        }
         const bool full = t0 + C <= T;   // no ragged rows in this chunk
         float bl[16];
         {
@@ -306,215 +361,248 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const bool valid = full || t0 + i < T;
                     const float kk = valid ? ld_in(sk + i * D + c) : 0.f;
                     const float vv = valid ? ld_in(sv + i * D + c) : 0.f;
+                    const float bi = sBeta[i];
                     const float x = bl[r] - rc;
                     const float ep = __expf(x), em = __expf(-x);
-                    kp[j] = kk * ep;
                     km[j] = kk * em;
                     kt[j] = km[j] * eCr;
-                    vh[j] = vv;
+                    kp[j] = kk * ep * bi;     // beta K+: A comes out row-scaled, W = T (beta K+)
+                    vh[j] = vv * bi;          // beta V:  U~ = T (beta V)
                     if (MODE == MODE_OUTPUT) qp[j] = (valid ? ld_in(sq + i * D + c) : 0.f) * ep;
                 }
                 const int ig = 2 * rb + grp;   // 8-row group of chunk positions
-                *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + cofs) = pack8_f16(kp);
+                *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + cofs) = pack8_f16(kp);   // [beta K+ | beta V]
                 *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + 2048 + cofs) = pack8_f16(vh);
-                *reinterpret_cast<uint4*>(sm + PL::KM + ig * 2048 + cofs) = pack8_f16(km);
+                *reinterpret_cast<uint4*>(sm + KM + ig * KM_IG + cofs) = pack8_f16(km);
                 *reinterpret_cast<uint4*>(sm + PL::KT + ig * 2048 + cofs) = pack8_f16(kt);
                 if (MODE == MODE_OUTPUT)
-                    *reinterpret_cast<uint4*>(sm + PL::QP + ig * 2048 + cofs) = pack8_f16(qp);
+                    *reinterpret_cast<uint4*>(sm + PL::Y + ig * 4096 + cofs) = pack8_f16(qp);
             }
         }
         fence_async_smem();
         __syncthreads();
-        // ---- 2. next chunk's TMA; A = K+ K-^T and P = Q+ K-^T on the tensor core ----------
+        // ---- 2. next chunk's TMA; A (and P) on the tensor core ----------------------------
+        if (t == NT / 2 && n + 1 < n1) issue_tma(n + 1);
         if (t == 0) {
-            if (n + 1 < n1) issue_tma(n + 1);
             tc_fence_after();
-            const uint32_t id = idesc_f16(64, 64, true, true);
-            const uint32_t tA = (MODE == MODE_OUTPUT) ? TO_A : TS_A;
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bd = sdesc(sbase + PL::KM + 256 * kk, 128, 2048);
-                umma_f16(tmem + tA, sdesc(sbase + PL::X + 256 * kk, 128, 4096), bd, id, kk > 0);
-                if (MODE == MODE_OUTPUT)
-                    umma_f16(tmem + TO_P, sdesc(sbase + PL::QP + 256 * kk, 128, 2048), bd, id, kk > 0);
+            if (MODE == MODE_OUTPUT) {
+                // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
+                const uint32_t id = idesc_f16(128, 64, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + T_AP, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
+                             sdesc(sbase + KM + 256 * kk, 128, 4096), id, kk > 0);
+            } else {
+                const uint32_t id = idesc_f16(64, 64, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + T_AP, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
+                             sdesc(sbase + KM + 256 * kk, 128, 2048), id, kk > 0);
             }
             umma_commit(ctl.mma_bar);
         }
         tma_in_flight = n + 1 < n1;
         mma_in_flight = true;
-        // ---- 3. while it runs: S^ = diag(e^r) S (fp16 tile), master *= e^{b_C} ----------
-        {
-            const float er = __expf(rc), eC = __expf(bC);
-            const int col0 = cq * NQ;
-            for (int cc = 0; cc < NQ; cc += 32) {
+        if (!grpY) {
+            // ---- 3X. warps 0-7: A -> fp16 tile, then T = (I + A)^{-1} ---------------------------
+            // A = diag(beta) strict_lower(K+ K-^T) (beta is already in K+).
+            wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == 0, 1);
+            const uint32_t Ah = sbase + PL::U;       // A, fp16 K-major core-matrix tile
+            const uint32_t Tt = sbase + TT;          // T, same layout: the next MMA's operand
+            {
                 float v[32];
-                tmem_ld32(tl + TM_S + col0 + cc, v);
+                int i = -1;
+                if (MODE == MODE_OUTPUT) {
+                    // M = 128 layout: row i in lane i; rows 0-63 (quarters 0, 1) are A
+                    if (q4 < 2) {
+                        tmem_ld32(tl + T_AP + 32 * hg, v);
+                        i = 32 * q4 + lane;
+                    }
+                } else {
+                    // M = 64 layout: row 16*q4 + l in lane 32*q4 + l (l < 16)
+                    tmem_ld32(tl + T_AP + 32 * hg, v);
+                    if (lane < 16) i = 16 * q4 + lane;
+                }
+                if (i >= 0) {
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        float f[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int col = 32 * hg + 8 * g8 + j;
+                            f[j] = (col < i) ? v[8 * g8 + j] : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(sm + PL::U + cm64(i, 32 * hg + 8 * g8)) = pack8_f16(f);
+                    }
+                }
+                // the six upper 16x16 blocks of T are zero
+                if (t < 192) {
+                    const int e = t >> 5, u = t & 31;
+                    const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
+                    const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
+                    const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
+                    *reinterpret_cast<uint4*>(sm + TT + cm64(row, col)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            named_sync(1, NT / 2);
+            // diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
+            // N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs
+            if (w < 4) {
+                const int b0 = 16 * w, g = lane >> 2, q = lane & 3;
+                const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
+                uint32_t aN[4], bN[4], bP[4], aX[4];
+                ldsm_x4(aN, Ah + cm64(b0 + (lane & 15), b0 + 8 * (lane >> 4)));
+                ldsm_x4_t(bN, Ah + cm64(b0 + (lane & 7) + 8 * ((lane >> 3) & 1), b0 + 8 * (lane >> 4)));
+                float n2a[4] = {0.f, 0.f, 0.f, 0.f}, n2b[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_16x16(n2a, n2b, aN, bN);                                   // N^2
+                c_to_scr(scr, lane, n2a, n2b);
+                __syncwarp();
+                scr_to_b(bP, scr, lane);                                       // bP = N^2
+                __syncwarp();
+                c_to_a(aX, n2a, n2b);
+                float n4a[4] = {0.f, 0.f, 0.f, 0.f}, n4b[4] = {0.f, 0.f, 0.f, 0.f};
+                float n3a[4] = {0.f, 0.f, 0.f, 0.f}, n3b[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_16x16(n4a, n4b, aX, bP);                                   // N^4
+                mma_16x16(n3a, n3b, aN, bP);                                   // N^3
+                c_to_scr(scr, lane, n4a, n4b);
+                __syncwarp();
+                scr_to_b(bP, scr, lane);                                       // bP = N^4
+                __syncwarp();
+                c_to_a(aX, n4a, n4b);
+                float n8a[4] = {0.f, 0.f, 0.f, 0.f}, n8b[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_16x16(n8a, n8b, aX, bP);                                   // N^8
+                // Z = I - N + N^2 - N^3, in the C layout (rows g, g+8; columns 2q, 2q+1 of
+                // each 8-column half); N's values come from its A fragment
+                float za[4], zb[4];
+                {
+                    const float2 n00 = unpack_f16x2(aN[0]), n10 = unpack_f16x2(aN[1]);
+                    const float2 n01 = unpack_f16x2(aN[2]), n11 = unpack_f16x2(aN[3]);
+                    const float d0 = (g == 2 * q) ? 1.f : 0.f, d1 = (g == 2 * q + 1) ? 1.f : 0.f;
+                    za[0] = d0 - n00.x + n2a[0] - n3a[0];
+                    za[1] = d1 - n00.y + n2a[1] - n3a[1];
+                    za[2] = -n10.x + n2a[2] - n3a[2];
+                    za[3] = -n10.y + n2a[3] - n3a[3];
+                    zb[0] = -n01.x + n2b[0] - n3b[0];
+                    zb[1] = -n01.y + n2b[1] - n3b[1];
+                    zb[2] = d0 - n11.x + n2b[2] - n3b[2];
+                    zb[3] = d1 - n11.y + n2b[3] - n3b[3];
+                }
+                {   // Z += Z N^4
+                    float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
+                    c_to_a(aX, za, zb);
+                    mma_16x16(ta, tb, aX, bP);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
+                }
+                c_to_scr(scr, lane, n8a, n8b);
+                __syncwarp();
+                scr_to_b(bP, scr, lane);                                       // bP = N^8
+                {   // Z += Z N^8
+                    float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
+                    c_to_a(aX, za, zb);
+                    mma_16x16(ta, tb, aX, bP);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
+                }
+                st_shared_b32(Tt + cm64(b0 + g, b0) + 4 * q, pack_f16x2(za[0], za[1]));
+                st_shared_b32(Tt + cm64(b0 + g + 8, b0) + 4 * q, pack_f16x2(za[2], za[3]));
+                st_shared_b32(Tt + cm64(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
+                st_shared_b32(Tt + cm64(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
+            }
+            named_sync(1, NT / 2);
+            // block diagonal d: warp (block J, 8-column half) computes
+            //   X = sum_{K=J}^{I-1} A_IK T_KJ  and  T_IJ = -T_II X   (I = J + d)
+            for (int d = 1; d < 4; ++d) {
+                if (w < 2 * (4 - d)) {
+                    const int J = w >> 1, I = J + d, N0 = 16 * J + 8 * (w & 1);
+                    const int g = lane >> 2, q = lane & 3;
+                    const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int K = J; K < I; ++K) {
+                        uint32_t aA[4], bT[2];
+                        ldsm_x4(aA, Ah + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
+                        ldsm_x2_t(bT, Tt + cm64(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
+                        mma16816(x, aA, bT);
+                    }
+                    st_shared_b32(scr + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
+                    st_shared_b32(scr + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
+                    __syncwarp();
+                    uint32_t bX[2], aT[4];
+                    ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+                    ldsm_x4(aT, Tt + cm64(16 * I + (lane & 15), 16 * I + 8 * (lane >> 4)));
+                    float tt[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma16816(tt, aT, bX);
+                    st_shared_b32(Tt + cm64(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
+                    st_shared_b32(Tt + cm64(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
+                }
+                named_sync(1, NT / 2);
+            }
+            fence_async_smem();
+        } else {
+            // ---- 3Y. warps 8-15: S^ = diag(e^r) S, master *= e^{b_C}; previous output; P --
+            {
+                const float er = __expf(rc), eC = __expf(bC);
+                const int col0 = hg * (NS / 2);
+                for (int cc = 0; cc < NS / 2; cc += 32) {
+                    float v[32];
+                    tmem_ld32(tl + TM_S + col0 + cc, v);
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        float f[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) f[j] = v[g8 * 8 + j] * er;
+                        const int col = col0 + cc + g8 * 8;
+                        *reinterpret_cast<uint4*>(sm + PL::S + (col >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
+                            pack8_f16(f);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= eC;
+                    tmem_st32(tl + TM_S + col0 + cc, v);
+                }
+            }
+            if (MODE == MODE_OUTPUT && prev_t0 >= 0)
+                store_o(tl, q4, 64 * hg, 2, lane, o, o_f32, b, T, H, h, prev_t0);
+            wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == NT / 2, 2);
+            if (MODE == MODE_OUTPUT && q4 >= 2) {
+                // P rows: lanes 64-127 of the M = 128 accumulator
+                float v[32];
+                tmem_ld32(tl + T_AP + 32 * hg, v);
+                const int i = 32 * (q4 - 2) + lane;
 #pragma unroll
                 for (int g8 = 0; g8 < 4; ++g8) {
                     float f[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = v[g8 * 8 + j] * er;
-                    const int col = col0 + cc + g8 * 8;
-                    *reinterpret_cast<uint4*>(sm + PL::S + (col >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
-                        pack8_f16(f);
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= eC;
-                tmem_st32(tl + TM_S + col0 + cc, v);
-            }
-        }
-        // ... and the previous chunk's output leaves TMEM before O is overwritten
-        if (MODE == MODE_OUTPUT && prev_t0 >= 0) store_o(tl, q4, cq, lane, o, o_f32, b, T, H, h, prev_t0);
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (MODE == MODE_OUTPUT && t == 0) {
-            tc_fence_after();
-            const uint32_t idq = idesc_f16(64, 128, true, true);
-            for (int kk = 0; kk < 8; ++kk)
-                umma_f16(tmem + TO_O, sdesc(sbase + PL::QP + 256 * kk, 128, 2048),
-                         sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
-        }
-        wait_mma(ctl, t);   // A and P are ready (O may still run)
-        // A rows -> fp32 (beta-scaled, strictly lower)
-        {
-            float v[16];
-            const uint32_t tA = (MODE == MODE_OUTPUT) ? TO_A : TS_A;
-            tmem_ld16(tl + tA + 16 * cq, v);
-            if (lane < 16) {
-                const int i = 16 * q4 + lane;
-                const float bi = sBeta[i];
-#pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
-                    float4 f;
-                    const int j = 16 * cq + 4 * j4;
-                    f.x = (j + 0 < i) ? bi * v[4 * j4 + 0] : 0.f;
-                    f.y = (j + 1 < i) ? bi * v[4 * j4 + 1] : 0.f;
-                    f.z = (j + 2 < i) ? bi * v[4 * j4 + 2] : 0.f;
-                    f.w = (j + 3 < i) ? bi * v[4 * j4 + 3] : 0.f;
-                    *reinterpret_cast<float4*>(Afp + sw(i, j)) = f;
-                }
-            }
-        }
-        __syncthreads();
-        if (*sAbort) break;
-        // ---- 4. T = (I + A)^{-1}: 16x16 diagonal blocks by substitution, then the
-        //         off-diagonal blocks T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ -------------
-        if (t < 64) {
-            const int blk = t >> 4, m = t & 15, base = 16 * blk;
-            float tc_[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float s = (r == m) ? 1.f : 0.f;
-#pragma unroll
-                for (int j = 0; j < r; ++j) s = fmaf(-Afp[sw(base + r, base + j)], tc_[j], s);
-                tc_[r] = s;
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tfp[sw(base + r, base + m)] = tc_[r];
-        }
-        __syncthreads();
-        // block diagonal d: warp (block J, 8-column half) computes
-        //   X = sum_{K=J}^{I-1} A_IK T_KJ  and  T_IJ = -T_II X   (I = J + d)
-        // with m16n8k16 warp MMAs (fp16 operands, fp32 accumulation).
-        for (int d = 1; d < 4; ++d) {
-            if (w < 2 * (4 - d)) {
-                const int J = w >> 1, I = J + d, N0 = 16 * J + 8 * (w & 1);
-                const int g = lane >> 2, q = lane & 3;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int K = J; K < I; ++K) {
-                    uint32_t a[4], bb[2];
-                    const int r0 = 16 * I + g, c0 = 16 * K + 2 * q;
-                    a[0] = pack_f16x2(Afp[sw(r0, c0)], Afp[sw(r0, c0 + 1)]);
-                    a[1] = pack_f16x2(Afp[sw(r0 + 8, c0)], Afp[sw(r0 + 8, c0 + 1)]);
-                    a[2] = pack_f16x2(Afp[sw(r0, c0 + 8)], Afp[sw(r0, c0 + 9)]);
-                    a[3] = pack_f16x2(Afp[sw(r0 + 8, c0 + 8)], Afp[sw(r0 + 8, c0 + 9)]);
-                    const int k0 = 16 * K + 2 * q, n = N0 + g;
-                    bb[0] = pack_f16x2(Tfp[sw(k0, n)], Tfp[sw(k0 + 1, n)]);
-                    bb[1] = pack_f16x2(Tfp[sw(k0 + 8, n)], Tfp[sw(k0 + 9, n)]);
-                    mma16816(acc, a, bb);
-                }
-                // X (C fragment) -> this warp's scratch, then back as a B fragment
-                float* xs = sXs + 128 * w;      // [16][8]
-                xs[g * 8 + 2 * q] = acc[0];
-                xs[g * 8 + 2 * q + 1] = acc[1];
-                xs[(g + 8) * 8 + 2 * q] = acc[2];
-                xs[(g + 8) * 8 + 2 * q + 1] = acc[3];
-                __syncwarp();
-                uint32_t a[4], bb[2];
-                {
-                    const int r0 = 16 * I + g, c0 = 16 * I + 2 * q;
-                    a[0] = pack_f16x2(Tfp[sw(r0, c0)], Tfp[sw(r0, c0 + 1)]);
-                    a[1] = pack_f16x2(Tfp[sw(r0 + 8, c0)], Tfp[sw(r0 + 8, c0 + 1)]);
-                    a[2] = pack_f16x2(Tfp[sw(r0, c0 + 8)], Tfp[sw(r0, c0 + 9)]);
-                    a[3] = pack_f16x2(Tfp[sw(r0 + 8, c0 + 8)], Tfp[sw(r0 + 8, c0 + 9)]);
-                    bb[0] = pack_f16x2(xs[(2 * q) * 8 + g], xs[(2 * q + 1) * 8 + g]);
-                    bb[1] = pack_f16x2(xs[(2 * q + 8) * 8 + g], xs[(2 * q + 9) * 8 + g]);
-                }
-                float tt[4] = {0.f, 0.f, 0.f, 0.f};
-                mma16816(tt, a, bb);
-                const int r0 = 16 * I + g, c0 = N0 + 2 * q;
-                *reinterpret_cast<float2*>(Tfp + sw(r0, c0)) = make_float2(-tt[0], -tt[1]);
-                *reinterpret_cast<float2*>(Tfp + sw(r0 + 8, c0)) = make_float2(-tt[2], -tt[3]);
-            }
-            __syncthreads();
-        }
-        // T' = T diag(beta), lower part only, fp16 K-major tile [i][j] at KM
-        {
-            const int ii = t >> 3, jg = t & 7;     // 512 (row, 8-column group) pairs
-            float vals[8];
-            const float4 a0 = *reinterpret_cast<const float4*>(Tfp + sw(ii, 8 * jg));
-            const float4 a1 = *reinterpret_cast<const float4*>(Tfp + sw(ii, 8 * jg + 4));
-            const float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int col = 8 * jg + j;
-                vals[j] = (col <= ii) ? f[j] * sBeta[col] : 0.f;
-            }
-            __syncthreads();
-            *reinterpret_cast<uint4*>(sm + PL::KM + jg * 1024 + (ii >> 3) * 128 + (ii & 7) * 16) = pack8_f16(vals);
-        }
-        // P (masked, fp16 K-major) next to T'
-        if (MODE == MODE_OUTPUT) {
-            float v[16];
-            tmem_ld16(tl + TO_P + 16 * cq, v);
-            if (lane < 16) {
-                const int i = 16 * q4 + lane;
-#pragma unroll
-                for (int g8 = 0; g8 < 2; ++g8) {
-                    float f[8];
-#pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const int col = 16 * cq + 8 * g8 + j;
+                        const int col = 32 * hg + 8 * g8 + j;
                         f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
                     }
-                    const int jgp = 2 * cq + g8;
-                    *reinterpret_cast<uint4*>(sm + PL::KM + 8192 + jgp * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                        pack8_f16(f);
+                    const int jgp = 4 * hg + g8;
+                    *reinterpret_cast<uint4*>(sm + PL::PT + jgp * 1024 + (i >> 3) * 128 + (i & 7) * 16) = pack8_f16(f);
                 }
             }
+            fence_async_smem();
         }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- 5. U~ = T' V,  W = T' K+ -----------------------------------------------------
+        if (*sAbort) break;
+        // ---- 4. [W | U~] = T [beta K+ | beta V]  (and O = Q+ S^) ----------------------------
         if (t == 0) {
             tc_fence_after();
-            const uint32_t id128 = idesc_f16(64, 128, false, false);
-            const uint32_t tU = (MODE == MODE_OUTPUT) ? TO_U : TS_R;
-            const uint32_t tW = (MODE == MODE_OUTPUT) ? TO_W : TS_W;
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = sdesc(sbase + PL::KM + 2048 * kk, 1024, 128);
-                umma_f16(tmem + tU, ad, sdesc(sbase + PL::X + 2048 + 8192 * kk, 4096, 128), id128, kk > 0);
-                umma_f16(tmem + tW, ad, sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id128, kk > 0);
+            const uint32_t id256 = idesc_f16(64, 256, false, false);
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(tmem + T_W, sdesc(sbase + TT + 2048 * kk, 1024, 128),
+                         sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id256, kk > 0);
+            if (MODE == MODE_OUTPUT) {
+                const uint32_t idq = idesc_f16(64, 128, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + TO_O, sdesc(sbase + PL::Y + 256 * kk, 128, 4096),
+                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
             }
             umma_commit(ctl.mma_bar);
         }
         wait_mma(ctl, t);
-        // W -> fp16 K-major tile [i][c] at X (K+ | V are no longer needed)
+        // W -> fp16 K-major tile [i][c] at X ([K+ | V] are no longer needed)
         {
-            const uint32_t tW = (MODE == MODE_OUTPUT) ? TO_W : TS_W;
             float v[32];
-            tmem_ld32(tl + tW + 32 * cq, v);
+            tmem_ld32(tl + T_W + 32 * cq, v);
             if (lane < 16) {
                 const int i = 16 * q4 + lane;
 #pragma unroll
@@ -529,34 +617,35 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
         if (*sAbort) break;
-        // ---- 6. U = U~ - W S^  (critical path) -----------------------------------------
+        // ---- 5. U = U~ - W S^  (critical path) -----------------------------------------
         if (t == 0) {
             tc_fence_after();
             const uint32_t idn = idesc_f16(64, 128, false, true, true);
-            const uint32_t tU = (MODE == MODE_OUTPUT) ? TO_U : TS_R;
             for (int kk = 0; kk < 8; ++kk)
-                umma_f16(tmem + tU, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
+                umma_f16(tmem + T_U, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
                          sdesc(sbase + PL::S + 256 * kk, 128, 2048), idn, 1);
             if (MODE == MODE_STATE) {
-                // identity columns carry no values: their U starts at -W Phi^
+                // identity columns carry no values: their U starts at -W Phi^ (in W's columns)
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + TS_W, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
+                    umma_f16(tmem + T_W, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
                              sdesc(sbase + PL::S + 32768 + 256 * kk, 128, 2048), idn, kk > 0);
             }
             umma_commit(ctl.mma_bar);
         }
         wait_mma(ctl, t);
-        // U -> fp16 MN-major tile [i][col] at U
+        // U -> fp16 MN-major tile [i][col] at U.  Value columns come from T_U, identity
+        // columns (MODE_STATE) from T_W.
         {
-            const uint32_t tU = (MODE == MODE_OUTPUT) ? TO_U : TS_R;
             for (int cc = 0; cc < NQ; cc += 32) {
+                const int col = cq * NQ + cc;            // U tile column
+                const uint32_t src = (col < D) ? (T_U + col) : (T_W + col - D);
                 float v[32];
-                tmem_ld32(tl + tU + cq * NQ + cc, v);
+                tmem_ld32(tl + src, v);
                 if (lane < 16) {
                     const int i = 16 * q4 + lane;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
-                        const int cg = (cq * NQ + cc) / 8 + g8;
+                        const int cg = col / 8 + g8;
                         *reinterpret_cast<uint4*>(sm + PL::U + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
                             pack8_f16(&v[8 * g8]);
                     }
@@ -566,7 +655,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- 7. S += Kt^T U  (and O += P U) ---------------------------------------------
+        // ---- 6. S += Kt^T U  (and O += P U) ---------------------------------------------
         if (t == 0) {
             tc_fence_after();
             const uint32_t ids = idesc_f16(128, NS, false, true);
@@ -576,7 +665,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (MODE == MODE_OUTPUT) {
                 const uint32_t ido = idesc_f16(64, 128, false, true);
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TO_O, sdesc(sbase + PL::KM + 8192 + 2048 * kk, 1024, 128),
+                    umma_f16(tmem + TO_O, sdesc(sbase + PL::PT + 2048 * kk, 1024, 128),
                              sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
             }
             umma_commit(ctl.mma_bar);
@@ -584,11 +673,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         wait_mma(ctl, t);
         mma_in_flight = false;
         prev_t0 = t0;
-        tc_fence_before();
-        __syncthreads();
     }
     if (MODE == MODE_OUTPUT && !*sAbort && prev_t0 >= 0)
-        store_o(tl, q4, cq, lane, o, o_f32, b, T, H, h, prev_t0);
+        store_o(tl, q4, 32 * cq, 1, lane, o, o_f32, b, T, H, h, prev_t0);
 
     // ---- end of segment: write the state ------------------------------------------------
     if (!*sAbort) {

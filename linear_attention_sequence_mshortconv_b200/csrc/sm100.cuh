@@ -208,6 +208,38 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ldmatrix: four (x4) or two (x2) 8x8 fp16 matrices; lane l gives the address of one
+// 16-byte matrix row (lanes 0-7 matrix 0, 8-15 matrix 1, ...).  .trans transposes.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], uint32_t addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r[0]), "=r"(r[1])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t u)
+{
+    return __half22float2(*reinterpret_cast<const __half2*>(&u));
+}
+
 // ---- cp.async (global -> shared, 16 bytes) ---------------------------------------------
 __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
