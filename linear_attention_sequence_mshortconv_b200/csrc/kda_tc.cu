@@ -62,12 +62,12 @@ template <> struct Plan<MODE_OUTPUT> {
     static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, [64][128]
     static constexpr int X = 65536;                // [K+ | V]; later W (64 x 128 fp16, K-major)
     static constexpr int Y = 98304;                // [Q+ | K-]
-    static constexpr int TF = 131072;              // T = (I + A)^{-1} (64 x 64 fp16, K-major), 8 KB used
-    static constexpr int PT = 147456;              // P (8 KB)
-    static constexpr int KT = 155648;              // Kt
-    static constexpr int U = 172032;               // fp16 A during the inverse, then U (64 x 128)
-    static constexpr int S = 188416;               // S^ (128 x 128 fp16)
-    static constexpr int MISC = 221184;
+    static constexpr int TF = 131072;              // T (64 x 64 fp16, K-major, 8-column groups 2 KB
+                                                   // apart) interleaved with P in the other 1 KB halves
+    static constexpr int KT = 147456;              // Kt
+    static constexpr int U = 163840;               // fp16 A during the inverse, then U (64 x 128)
+    static constexpr int S = 180224;               // S^ (128 x 128 fp16)
+    static constexpr int MISC = 212992;
     static constexpr int TMA_BYTES = 4 * 16384;
 };
 template <> struct Plan<MODE_STATE> {
@@ -76,7 +76,6 @@ template <> struct Plan<MODE_STATE> {
     static constexpr int X = 49152;                // [K+ | V]; later W
     static constexpr int Y = -1;
     static constexpr int TF = 81920;               // K- (the T tile lives at U + 8192 here)
-    static constexpr int PT = -1;
     static constexpr int KT = 98304;
     static constexpr int U = 114688;               // fp16 A and T during the inverse, then U (64 x 256)
     static constexpr int S = 147456;               // S^ (128 x 256 fp16)
@@ -87,18 +86,18 @@ template <> struct Plan<MODE_STATE> {
 constexpr int M_BETA = 0;        // float[64]
 constexpr int M_TOT = 256;       // float[4][128] per-row-block sums of g
 constexpr int M_XS = 2304;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 6400;      // 2 x uint64 mbarriers
-constexpr int M_TMEM = 6416;     // uint32 TMEM base
-constexpr int M_ABORT = 6420;    // int
+constexpr int M_BAR = 6400;      // 3 x uint64 mbarriers (TMA, MMA, second MMA issuer)
+constexpr int M_TMEM = 6424;     // uint32 TMEM base
+constexpr int M_ABORT = 6428;    // int
 constexpr int MISC_BYTES = 6432;
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
-// TMEM columns.  W and U~ come out of one N = 256 MMA as [W | U~].
+// TMEM columns.
 constexpr uint32_t TM_S = 0;                      // state master (fp32), 128 or 256 columns
-constexpr uint32_t TO_O = 128;                    // MODE_OUTPUT: O (M = 64), 128 columns
+constexpr uint32_t T_YO = 128;                    // MODE_OUTPUT: [Y; O] (M = 128), 128 columns
 constexpr uint32_t T_AP = 256;                    // A (and P below it in MODE_OUTPUT), 64 columns
-constexpr uint32_t T_W = 256, T_U = 384;          // W, then U~ -> U (M = 64), 128 columns each
+constexpr uint32_t T_W = 256, T_U = 384;          // MODE_STATE: [W | U~] (N = 256); both: U (M = 64)
 
 // ---- helpers ------------------------------------------------------------------------
 __device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat162float(*p); }
@@ -180,17 +179,18 @@ __device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t& phase, Ctl& c,
 __device__ __forceinline__ void wait_mma(Ctl& c, int t) { wait_bar(c.mma_bar, c.mma_phase, c, t == 0, 0); }
 __device__ __forceinline__ void wait_tma(Ctl& c, int t) { wait_bar(c.tma_bar, c.tma_phase, c, t == 0, 0); }
 
-// Output rows of one chunk from TMEM (M = 64 layout: row 16*q4 + l in lane 32*q4 + l,
-// l < 16) to global memory; this warp stores columns col0 .. col0 + 32*nld - 1.
+// Output rows of one chunk from TMEM to global memory.  O is rows 64-127 of the
+// M = 128 accumulator [Y; O]: output row i sits in lane 64 + i, so warps of lane
+// quarters 2 and 3 store it; this warp stores columns col0 .. col0 + 32*nld - 1.
 __device__ __forceinline__ void store_o(uint32_t tl, int q4, int col0, int nld, int lane, void* o, int o_f32,
                                         int b, int T, int H, int h, int t0)
 {
     for (int u = 0; u < nld; ++u) {
         float v[32];
         const int cc = col0 + 32 * u;
-        tmem_ld32(tl + TO_O + cc, v);
-        const int i = 16 * q4 + lane;
-        if (lane < 16 && t0 + i < T) {
+        tmem_ld32(tl + T_YO + cc, v);
+        const int i = 32 * (q4 - 2) + lane;
+        if (t0 + i < T) {
             const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + cc;
             if (o_f32) {
                 float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
@@ -230,6 +230,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     constexpr int KM = (MODE == MODE_OUTPUT) ? PL::Y + 2048 : PL::TF;   // K- tile base
     constexpr int KM_IG = (MODE == MODE_OUTPUT) ? 4096 : 2048;          // its 8-row group stride
     constexpr int TT = (MODE == MODE_OUTPUT) ? PL::TF : PL::U + 8192;   // T tile base
+    constexpr int T_LBO = (MODE == MODE_OUTPUT) ? 2048 : 1024;          // T's 8-column group stride
+    auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     extern __shared__ __align__(1024) uint8_t sm[];
 
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
@@ -252,9 +254,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t sbase = smem_addr(sm);
 
     Ctl ctl{&bars[0], &bars[1], sAbort, status, 0u, 0u};
+    uint64_t* yo_bar = &bars[2];      // MMAs issued by thread NT/2 ([Y; O] = [beta K+; Q+] S^)
+    uint32_t yo_phase = 0;
+    bool yo_in_flight = false;
     if (t == 0) {
         mbar_init(ctl.tma_bar, 1);
         mbar_init(ctl.mma_bar, 1);
+        mbar_init(yo_bar, 1);
         *sAbort = 0;
         fence_mbar_init();
     }
@@ -439,7 +445,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
                     const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
                     const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
-                    *reinterpret_cast<uint4*>(sm + TT + cm64(row, col)) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(sm + TT + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             named_sync(1, NT / 2);
@@ -502,10 +508,10 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
                 }
-                st_shared_b32(Tt + cm64(b0 + g, b0) + 4 * q, pack_f16x2(za[0], za[1]));
-                st_shared_b32(Tt + cm64(b0 + g + 8, b0) + 4 * q, pack_f16x2(za[2], za[3]));
-                st_shared_b32(Tt + cm64(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
-                st_shared_b32(Tt + cm64(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
+                st_shared_b32(Tt + cmT(b0 + g, b0) + 4 * q, pack_f16x2(za[0], za[1]));
+                st_shared_b32(Tt + cmT(b0 + g + 8, b0) + 4 * q, pack_f16x2(za[2], za[3]));
+                st_shared_b32(Tt + cmT(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
+                st_shared_b32(Tt + cmT(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
             }
             named_sync(1, NT / 2);
             // block diagonal d: warp (block J, 8-column half) computes
@@ -519,7 +525,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int K = J; K < I; ++K) {
                         uint32_t aA[4], bT[2];
                         ldsm_x4(aA, Ah + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
-                        ldsm_x2_t(bT, Tt + cm64(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
+                        ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
                         mma16816(x, aA, bT);
                     }
                     st_shared_b32(scr + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
@@ -527,17 +533,19 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     __syncwarp();
                     uint32_t bX[2], aT[4];
                     ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
-                    ldsm_x4(aT, Tt + cm64(16 * I + (lane & 15), 16 * I + 8 * (lane >> 4)));
+                    ldsm_x4(aT, Tt + cmT(16 * I + (lane & 15), 16 * I + 8 * (lane >> 4)));
                     float tt[4] = {0.f, 0.f, 0.f, 0.f};
                     mma16816(tt, aT, bX);
-                    st_shared_b32(Tt + cm64(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
-                    st_shared_b32(Tt + cm64(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
+                    st_shared_b32(Tt + cmT(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
+                    st_shared_b32(Tt + cmT(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
                 }
                 named_sync(1, NT / 2);
             }
             fence_async_smem();
         } else {
-            // ---- 3Y. warps 8-15: S^ = diag(e^r) S, master *= e^{b_C}; previous output; P --
+            // ---- 3Y. warps 8-15: previous output; S^ = diag(e^r) S, master *= e^{b_C}; P; Y --
+            if (MODE == MODE_OUTPUT && prev_t0 >= 0 && q4 >= 2)
+                store_o(tl, q4, 64 * hg, 2, lane, o, o_f32, b, T, H, h, prev_t0);
             {
                 const float er = __expf(rc), eC = __expf(bC);
                 const int col0 = hg * (NS / 2);
@@ -558,11 +566,26 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_st32(tl + TM_S + col0 + cc, v);
                 }
             }
-            if (MODE == MODE_OUTPUT && prev_t0 >= 0)
-                store_o(tl, q4, 64 * hg, 2, lane, o, o_f32, b, T, H, h, prev_t0);
+            if (MODE == MODE_OUTPUT) {
+                // [Y; O] = [beta K+; Q+] S^ (M = 128), issued by thread NT/2 while warps 0-7
+                // invert: Y feeds U = T (beta V) - T Y, O is the inter-chunk output part
+                fence_async_smem();
+                tc_fence_before();
+                named_sync(2, NT / 2);
+                if (t == NT / 2) {
+                    tc_fence_after();
+                    const uint32_t idq = idesc_f16(128, 128, true, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + T_YO, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
+                                 sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
+                    umma_commit(yo_bar);
+                }
+                yo_in_flight = true;
+            }
             wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == NT / 2, 2);
             if (MODE == MODE_OUTPUT && q4 >= 2) {
-                // P rows: lanes 64-127 of the M = 128 accumulator
+                // P rows: lanes 64-127 of the M = 128 accumulator; P goes to the free 1 KB
+                // halves of the T region, so that [T; P] reads as one M = 128 operand
                 float v[32];
                 tmem_ld32(tl + T_AP + 32 * hg, v);
                 const int i = 32 * (q4 - 2) + lane;
@@ -574,8 +597,25 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         const int col = 32 * hg + 8 * g8 + j;
                         f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
                     }
-                    const int jgp = 4 * hg + g8;
-                    *reinterpret_cast<uint4*>(sm + PL::PT + jgp * 1024 + (i >> 3) * 128 + (i & 7) * 16) = pack8_f16(f);
+                    *reinterpret_cast<uint4*>(sm + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)) = pack8_f16(f);
+                }
+            }
+            if (MODE == MODE_OUTPUT) {
+                wait_bar(yo_bar, yo_phase, ctl, t == NT / 2, 2);
+                yo_in_flight = false;
+                if (q4 < 2) {
+                    // Y rows j (lanes 0-63) -> fp16 MN-major B tile in the beta K+ halves of X
+                    const int j = 32 * q4 + lane;
+                    for (int cc = 0; cc < 64; cc += 32) {
+                        float v[32];
+                        tmem_ld32(tl + T_YO + 64 * hg + cc, v);
+#pragma unroll
+                        for (int g8 = 0; g8 < 4; ++g8) {
+                            const int cg = (64 * hg + cc) / 8 + g8;
+                            *reinterpret_cast<uint4*>(sm + PL::X + (j >> 3) * 4096 + cg * 128 + (j & 7) * 16) =
+                                pack8_f16(&v[8 * g8]);
+                        }
+                    }
                 }
             }
             fence_async_smem();
@@ -583,56 +623,64 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
         if (*sAbort) break;
-        // ---- 4. [W | U~] = T [beta K+ | beta V]  (and O = Q+ S^) ----------------------------
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t id256 = idesc_f16(64, 256, false, false);
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + T_W, sdesc(sbase + TT + 2048 * kk, 1024, 128),
-                         sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id256, kk > 0);
-            if (MODE == MODE_OUTPUT) {
-                const uint32_t idq = idesc_f16(64, 128, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + TO_O, sdesc(sbase + PL::Y + 256 * kk, 128, 4096),
-                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
+        if (MODE == MODE_OUTPUT) {
+            // ---- 4. U = T (beta V) - T Y  (critical path) -----------------------------------
+            if (t == 0) {
+                tc_fence_after();
+                const uint32_t idv = idesc_f16(64, 128, false, false);
+                const uint32_t idy = idesc_f16(64, 128, false, true, true);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + T_U, sdesc(sbase + TT + 4096 * kk, 2048, 128),
+                             sdesc(sbase + PL::X + 2048 + 8192 * kk, 4096, 128), idv, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + T_U, sdesc(sbase + TT + 4096 * kk, 2048, 128),
+                             sdesc(sbase + PL::X + 8192 * kk, 4096, 128), idy, 1);
+                umma_commit(ctl.mma_bar);
             }
-            umma_commit(ctl.mma_bar);
-        }
-        wait_mma(ctl, t);
-        // W -> fp16 K-major tile [i][c] at X ([K+ | V] are no longer needed)
-        {
-            float v[32];
-            tmem_ld32(tl + T_W + 32 * cq, v);
-            if (lane < 16) {
-                const int i = 16 * q4 + lane;
+            wait_mma(ctl, t);
+        } else {
+            // ---- 4. [W | U~] = T [beta K+ | beta V] ---------------------------------------------
+            if (t == 0) {
+                tc_fence_after();
+                const uint32_t id256 = idesc_f16(64, 256, false, false);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + T_W, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
+                             sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id256, kk > 0);
+                umma_commit(ctl.mma_bar);
+            }
+            wait_mma(ctl, t);
+            // W -> fp16 K-major tile [i][c] at X ([K+ | V] are no longer needed)
+            {
+                float v[32];
+                tmem_ld32(tl + T_W + 32 * cq, v);
+                if (lane < 16) {
+                    const int i = 16 * q4 + lane;
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    const int cg = 4 * cq + g8;
-                    *reinterpret_cast<uint4*>(sm + PL::X + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                        pack8_f16(&v[8 * g8]);
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        const int cg = 4 * cq + g8;
+                        *reinterpret_cast<uint4*>(sm + PL::X + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
+                            pack8_f16(&v[8 * g8]);
+                    }
                 }
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (*sAbort) break;
-        // ---- 5. U = U~ - W S^  (critical path) -----------------------------------------
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t idn = idesc_f16(64, 128, false, true, true);
-            for (int kk = 0; kk < 8; ++kk)
-                umma_f16(tmem + T_U, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
-                         sdesc(sbase + PL::S + 256 * kk, 128, 2048), idn, 1);
-            if (MODE == MODE_STATE) {
-                // identity columns carry no values: their U starts at -W Phi^ (in W's columns)
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (*sAbort) break;
+            // ---- 5. U = U~ - W S^, identity columns -W Phi^ (in W's columns) -----------------
+            if (t == 0) {
+                tc_fence_after();
+                const uint32_t idn = idesc_f16(64, 128, false, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + T_U, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
+                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idn, 1);
                 for (int kk = 0; kk < 8; ++kk)
                     umma_f16(tmem + T_W, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
                              sdesc(sbase + PL::S + 32768 + 256 * kk, 128, 2048), idn, kk > 0);
+                umma_commit(ctl.mma_bar);
             }
-            umma_commit(ctl.mma_bar);
+            wait_mma(ctl, t);
         }
-        wait_mma(ctl, t);
         // U -> fp16 MN-major tile [i][col] at U.  Value columns come from T_U, identity
         // columns (MODE_STATE) from T_W.
         {
@@ -663,9 +711,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 umma_f16(tmem + TM_S, sdesc(sbase + PL::KT + 4096 * kk, 2048, 128),
                          sdesc(sbase + PL::U + 256 * kk, 128, 1024), ids, 1);
             if (MODE == MODE_OUTPUT) {
-                const uint32_t ido = idesc_f16(64, 128, false, true);
+                // O += P U as rows 64-127 of an M = 128 MMA whose rows 0-63 read T (their
+                // result lands on Y's rows, already consumed)
+                const uint32_t ido = idesc_f16(128, 128, false, true);
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TO_O, sdesc(sbase + PL::PT + 2048 * kk, 1024, 128),
+                    umma_f16(tmem + T_YO, sdesc(sbase + PL::TF + 4096 * kk, 2048, 128),
                              sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
             }
             umma_commit(ctl.mma_bar);
@@ -674,7 +724,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_in_flight = false;
         prev_t0 = t0;
     }
-    if (MODE == MODE_OUTPUT && !*sAbort && prev_t0 >= 0)
+    if (MODE == MODE_OUTPUT && !*sAbort && prev_t0 >= 0 && q4 >= 2)
         store_o(tl, q4, 32 * cq, 1, lane, o, o_f32, b, T, H, h, prev_t0);
 
     // ---- end of segment: write the state ------------------------------------------------
@@ -701,6 +751,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (*sAbort) {
         if (mma_in_flight) mbar_wait_bounded(ctl.mma_bar, ctl.mma_phase, kWaitNs);
         if (tma_in_flight) mbar_wait_bounded(ctl.tma_bar, ctl.tma_phase, kWaitNs);
+        if (yo_in_flight && t == NT / 2) mbar_wait_bounded(yo_bar, yo_phase, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
