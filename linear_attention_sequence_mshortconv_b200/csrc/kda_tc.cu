@@ -5,15 +5,17 @@
 // the chunk algebra is derived from Eq. 14.  Inside a chunk of C = 64 tokens with
 // entry state S0, b_i = sum_{r<=i} g_r (fp32, per key channel), a reference point
 // r = b_31 (the middle of the chunk) keeps every exponential within e^{+-|b|/2}:
-//   K+ = k e^{b - r},  Q+ = q e^{b - r},  K- = k e^{r - b},  Kt = k e^{b_C - b}
+//   K+ = k e^{b - r},  Q+ = q e^{b - r},  K- = k e^{r - b}
 //   A  = strict_lower((diag(beta) K+) K-^T),   P = lower(Q+ K-^T)  (incl. diagonal)
 //   T  = (I + A)^{-1}                     (16x16 blocks on warp MMAs, fp16 operands)
-//   S^ = diag(e^{r}) S0                                           (state seen by K+, Q+)
-//   U  = T (beta V) - (T (beta K+)) S^     O = Q+ S^ + P U
-//   S_C = diag(e^{b_C}) S0 + Kt^T U
-// Every MMA operand is fp16 in shared memory (11-bit significand: bf16 operands
-// would cost ~3% of RMS(o) in max error), accumulation is fp32 in TMEM, and the
-// state's master copy stays fp32 in TMEM across chunks.
+//   S^ = diag(e^{r}) S0,   Y = (diag(beta) K+) S^
+//   U  = T (beta V) - T Y                 O = Q+ S^ + P U
+//   S_C = diag(e^{b_C - r}) (S^ + K-^T U)     (k e^{b_C - b} = K- diag(e^{b_C - r}))
+// The state's fp32 master copy lives in TMEM in the scaled form S^ + K-^T U: the row
+// scale e^{b_C - r} of one chunk and e^{r'} of the next are applied together, once,
+// when the next chunk reads it.  Every MMA operand is fp16 in shared memory (11-bit
+// significand: bf16 operands would cost ~3% of RMS(o) in max error); accumulation is
+// fp32 in TMEM.  Exponents are kept in base 2 (g log2(e) summed in fp32).
 //
 // Parallelism.  A head's scan is sequential over chunks, and one B200 workload has
 // only B*H = 16 heads for 148 SMs, so each head's chunk sequence is cut into P
@@ -25,7 +27,7 @@
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
 //   pass 2 (MODE_OUTPUT, all segments): run the recurrence from S_start(p) and write
 //          o (and S_T from the last segment).
-// Each pass is one CTA per (b, h, segment), 512 threads, up to ~222 KB of shared memory.
+// Each pass is one CTA per (b, h, segment), 512 threads, ~200 KB of shared memory.
 //
 // Shared-memory operand tiles use the no-swizzle core-matrix layout: 8 rows x 16 B
 // blocks of 128 contiguous bytes.  A thread that owns one key channel writes 8
@@ -50,54 +52,61 @@ constexpr int C = 64;         // chunk length
 constexpr int D = 128;        // Dk = Dv
 constexpr int NT = 512;       // threads per CTA
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
+constexpr float kLog2e = 1.4426950408889634f;
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
 // ---- shared-memory plan (bytes) --------------------------------------------------
-// MODE_OUTPUT stacks Q+ under K+ so that one M = 128 MMA gives A and P: the block
-// XY holds, per 8-row group of chunk positions ig, [K+ | V] at XY + ig*4096 and
-// [Q+ | K-] at XY + 32768 + ig*4096 (channel-major 2 KB halves).
+// Channel-major fp16 tiles (K+ beta, Q+, K-, beta V): 8-position group ig at
+// tile + ig*2048, channel c at (c >> 3)*128 + (c & 7)*16 inside it.  Q+ follows K+ beta
+// directly, so [beta K+; Q+] is one M = 128 operand.  After the Y MMA the S^ region
+// holds Y (position-major: 8-position group j at j*NS*16, 8 columns per 16 bytes).
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int NS = 128;                 // state columns (values only)
     static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, [64][128]
-    static constexpr int X = 65536;                // [K+ | V]; later W (64 x 128 fp16, K-major)
-    static constexpr int Y = 98304;                // [Q+ | K-]
+    static constexpr int KP = 65536;               // beta K+
+    static constexpr int QP = 81920;               // Q+
+    static constexpr int KM = 98304;               // K-
+    static constexpr int VB = 114688;              // beta V
     static constexpr int TF = 131072;              // T (64 x 64 fp16, K-major, 8-column groups 2 KB
                                                    // apart) interleaved with P in the other 1 KB halves
-    static constexpr int KT = 147456;              // Kt
-    static constexpr int U = 163840;               // fp16 A during the inverse, then U (64 x 128)
-    static constexpr int S = 180224;               // S^ (128 x 128 fp16)
-    static constexpr int MISC = 212992;
+    static constexpr int U = 147456;               // fp16 A during the inverse, then U (64 x 128)
+    static constexpr int S = 163840;               // S^ (128 x 128 fp16), then Y
+    static constexpr int MISC = 196608;
     static constexpr int TMA_BYTES = 4 * 16384;
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int NS = 256;                 // [S | Phi]
     static constexpr int stQ = -1, stK = 0, stV = 16384, stG = 32768;
-    static constexpr int X = 49152;                // [K+ | V]; later W
-    static constexpr int Y = -1;
-    static constexpr int TF = 81920;               // K- (the T tile lives at U + 8192 here)
-    static constexpr int KT = 98304;
-    static constexpr int U = 114688;               // fp16 A and T during the inverse, then U (64 x 256)
-    static constexpr int S = 147456;               // S^ (128 x 256 fp16)
-    static constexpr int MISC = 212992;
+    static constexpr int KP = 49152;
+    static constexpr int QP = -1;
+    static constexpr int KM = 65536;
+    static constexpr int VB = 81920;
+    static constexpr int TF = -1;                  // T lives at U + 8192
+    static constexpr int U = 98304;                // fp16 A and T during the inverse, then U (64 x 256)
+    static constexpr int S = 131072;               // [S^ | Phi^] (128 x 256 fp16), then Y
+    static constexpr int MISC = 196608;
     static constexpr int TMA_BYTES = 3 * 16384;
 };
 // MISC sub-layout
 constexpr int M_BETA = 0;        // float[64]
-constexpr int M_TOT = 256;       // float[4][128] per-row-block sums of g
-constexpr int M_XS = 2304;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 6400;      // 3 x uint64 mbarriers (TMA, MMA, second MMA issuer)
-constexpr int M_TMEM = 6424;     // uint32 TMEM base
-constexpr int M_ABORT = 6428;    // int
-constexpr int MISC_BYTES = 6432;
+constexpr int M_TOT = 256;       // float[8][128] per-8-row-block sums of g log2(e)
+constexpr int M_XS = 4352;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 8448;      // 4 x uint64 mbarriers (TMA, MMA, second issuer, A read)
+constexpr int M_TMEM = 8480;     // uint32 TMEM base
+constexpr int M_ABORT = 8484;    // int
+constexpr int MISC_BYTES = 8496;
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
 // TMEM columns.
-constexpr uint32_t TM_S = 0;                      // state master (fp32), 128 or 256 columns
-constexpr uint32_t T_YO = 128;                    // MODE_OUTPUT: [Y; O] (M = 128), 128 columns
-constexpr uint32_t T_AP = 256;                    // A (and P below it in MODE_OUTPUT), 64 columns
-constexpr uint32_t T_W = 256, T_U = 384;          // MODE_STATE: [W | U~] (N = 256); both: U (M = 64)
+constexpr uint32_t TM_S = 0;     // state master (fp32), 128 or 256 columns
+constexpr uint32_t T_AP = 256;   // A (and P below it in MODE_OUTPUT), 64 columns
+// MODE_OUTPUT: [Y; O] (M = 128) at 128, U (M = 64) at 384.
+// MODE_STATE:  Y, then U (M = 64, 256 columns) at 256, once A has been read.
+template <int MODE> struct Tm;
+template <> struct Tm<MODE_OUTPUT> { static constexpr uint32_t Y = 128, UU = 384; };
+template <> struct Tm<MODE_STATE> { static constexpr uint32_t Y = 256, UU = 256; };
 
 // ---- helpers ------------------------------------------------------------------------
 __device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat162float(*p); }
@@ -179,6 +188,13 @@ __device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t& phase, Ctl& c,
 __device__ __forceinline__ void wait_mma(Ctl& c, int t) { wait_bar(c.mma_bar, c.mma_phase, c, t == 0, 0); }
 __device__ __forceinline__ void wait_tma(Ctl& c, int t) { wait_bar(c.tma_bar, c.tma_phase, c, t == 0, 0); }
 
+// Two adjacent 2-byte input elements -> fp32
+__device__ __forceinline__ float2 in2(uint32_t u, const __nv_bfloat16*)
+{
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ float2 in2(uint32_t u, const __half*) { return unpack_f16x2(u); }
+
 // Output rows of one chunk from TMEM to global memory.  O is rows 64-127 of the
 // M = 128 accumulator [Y; O]: output row i sits in lane 64 + i, so warps of lane
 // quarters 2 and 3 store it; this warp stores columns col0 .. col0 + 32*nld - 1.
@@ -188,7 +204,7 @@ __device__ __forceinline__ void store_o(uint32_t tl, int q4, int col0, int nld, 
     for (int u = 0; u < nld; ++u) {
         float v[32];
         const int cc = col0 + 32 * u;
-        tmem_ld32(tl + T_YO + cc, v);
+        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + cc, v);
         const int i = 32 * (q4 - 2) + lane;
         if (t0 + i < T) {
             const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + cc;
@@ -212,10 +228,10 @@ __device__ __forceinline__ void store_o(uint32_t tl, int q4, int col0, int nld, 
 }
 
 // The kernel ---------------------------------------------------------------------------
-// 512 threads.  Prologue: thread t owns key channel c = t & 127 and chunk rows
-// 16*(t >> 7) .. +15.  TMEM: warp w reads lane quarter w & 3.  While warps 0-7 read A
-// and invert (I + A), warps 8-15 rescale the state, store the previous chunk's output
-// and read P.
+// 512 threads.  Prologue: thread t owns key channels 2*(t & 63) + {0, 1} and chunk rows
+// 8*(t >> 6) .. +7.  TMEM: warp w reads lane quarter w & 3.  While warps 0-7 read A and
+// invert (I + A), warps 8-15 store the previous chunk's output, rescale the state,
+// issue Y (and O) from S^, and read P and Y.
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -225,12 +241,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status)
 {
     using PL = Plan<MODE>;
+    constexpr bool OUT = MODE == MODE_OUTPUT;
     constexpr int NS = PL::NS;
     constexpr int NQ = NS / 4;                // state columns per column quarter (all 16 warps)
-    constexpr int KM = (MODE == MODE_OUTPUT) ? PL::Y + 2048 : PL::TF;   // K- tile base
-    constexpr int KM_IG = (MODE == MODE_OUTPUT) ? 4096 : 2048;          // its 8-row group stride
-    constexpr int TT = (MODE == MODE_OUTPUT) ? PL::TF : PL::U + 8192;   // T tile base
-    constexpr int T_LBO = (MODE == MODE_OUTPUT) ? 2048 : 1024;          // T's 8-column group stride
+    constexpr int YJ = NS * 16;               // Y tile: bytes per 8-position group
+    constexpr uint32_t T_Y = Tm<MODE>::Y, T_UU = Tm<MODE>::UU;
+    constexpr int TT = OUT ? PL::TF : PL::U + 8192;   // T tile base
+    constexpr int T_LBO = OUT ? 2048 : 1024;          // T's 8-column group stride
     auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     extern __shared__ __align__(1024) uint8_t sm[];
 
@@ -238,7 +255,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int q4 = w & 3, cq = w >> 2;        // TMEM lane quarter, column quarter
     const bool grpY = w >= 8;                 // second 256-thread group
     const int hg = (w >> 2) & 1;              // column half inside a group
-    const int c = t & 127, rb = t >> 7;       // channel / TMEM row; 16-row block of the prologue
+    const int c = t & 127;                    // channel / TMEM row of the state steps
+    const int cp = t & 63, rb = t >> 6;       // prologue: channel pair, 8-row block
     const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
     const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
     const int b = bh / H, h = bh % H;
@@ -247,20 +265,21 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     float* sBeta = reinterpret_cast<float*>(sm + PL::MISC + M_BETA);
     float* sTot = reinterpret_cast<float*>(sm + PL::MISC + M_TOT);
-    float* sXs = reinterpret_cast<float*>(sm + PL::MISC + M_XS);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
     int* sAbort = reinterpret_cast<int*>(sm + PL::MISC + M_ABORT);
     const uint32_t sbase = smem_addr(sm);
 
     Ctl ctl{&bars[0], &bars[1], sAbort, status, 0u, 0u};
-    uint64_t* yo_bar = &bars[2];      // MMAs issued by thread NT/2 ([Y; O] = [beta K+; Q+] S^)
-    uint32_t yo_phase = 0;
-    bool yo_in_flight = false;
+    uint64_t* y_bar = &bars[2];       // MMAs issued by thread NT/2 (Y, and O in MODE_OUTPUT)
+    uint64_t* a_bar = &bars[3];       // MODE_STATE: A has been read out of TMEM
+    uint32_t y_phase = 0, a_phase = 0;
+    bool y_in_flight = false;
     if (t == 0) {
         mbar_init(ctl.tma_bar, 1);
         mbar_init(ctl.mma_bar, 1);
-        mbar_init(yo_bar, 1);
+        mbar_init(y_bar, 1);
+        mbar_init(a_bar, 1);
         *sAbort = 0;
         fence_mbar_init();
     }
@@ -279,7 +298,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     auto issue_tma = [&](int n) {
         const int row = b * T + n * C;
         mbar_arrive_expect_tx(ctl.tma_bar, PL::TMA_BYTES);
-        if (MODE == MODE_OUTPUT) tma_load_3d(sm + PL::stQ, &tm_q, ctl.tma_bar, 0, h, row);
+        if (OUT) tma_load_3d(sm + PL::stQ, &tm_q, ctl.tma_bar, 0, h, row);
         tma_load_3d(sm + PL::stK, &tm_k, ctl.tma_bar, 0, h, row);
         tma_load_3d(sm + PL::stV, &tm_v, ctl.tma_bar, 0, h, row);
         tma_load_3d(sm + PL::stG, &tm_g, ctl.tma_bar, 0, h, row);
@@ -318,6 +337,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
 
+    // The master holds diag(2^{-carry}) S for channel c (log2 units; 0 before any chunk).
+    float carry = 0.f;
     int prev_t0 = -1;   // chunk whose output still sits in TMEM (MODE_OUTPUT)
     for (int n = n0; n < n1 && !*sAbort; ++n) {
         const int t0 = n * C;
@@ -330,60 +351,90 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             beta_bits = load_beta_bits(n + 1);    // in flight during this chunk
         }
         const bool full = t0 + C <= T;   // no ragged rows in this chunk
-        float bl[16];
+        const int nvalid = T - t0;       // rows i < nvalid are tokens
+        float2 bl[8];                    // b log2(e) for this thread's two channels, rows 8*rb + r
         {
-            const __nv_bfloat16* stg = reinterpret_cast<const __nv_bfloat16*>(sm + PL::stG);
-            float run = 0.f;
+            const uint32_t* stg = reinterpret_cast<const uint32_t*>(sm + PL::stG) + cp;
+            float2 run = make_float2(0.f, 0.f);
+            const float2 l2e = make_float2(kLog2e, kLog2e);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int i = 16 * rb + r;
-                run += (full || t0 + i < T) ? __bfloat162float(stg[i * D + c]) : 0.f;
+            for (int r = 0; r < 8; ++r) {
+                const int i = 8 * rb + r;
+                float2 gv = in2(stg[i * (D / 2)], (const __nv_bfloat16*)nullptr);
+                if (!full && i >= nvalid) gv = make_float2(0.f, 0.f);
+                run = __ffma2_rn(gv, l2e, run);
                 bl[r] = run;
             }
-            sTot[rb * 128 + c] = run;
+            *reinterpret_cast<float2*>(sTot + rb * D + 2 * cp) = run;
         }
         __syncthreads();
-        float rc, bC;
+        float2 xo;              // (sum of the earlier row blocks) - r, this thread's channel pair
+        float s_scale;          // state row scale for channel c: 2^{r + carry}
         {
-            const float s0 = sTot[c], s1 = sTot[128 + c], s2 = sTot[256 + c], s3 = sTot[384 + c];
-            const float off = (rb > 0 ? s0 : 0.f) + (rb > 1 ? s1 : 0.f) + (rb > 2 ? s2 : 0.f);
+            float2 off = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
+            float rc = 0.f, bc = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) bl[r] += off;
-            rc = s0 + s1;               // b at row 31: the reference point
-            bC = s0 + s1 + s2 + s3;     // b at row 63
+            for (int qb = 0; qb < 8; ++qb) {
+                const float2 v = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
+                if (qb < rb) off = __fadd2_rn(off, v);
+                if (qb < 4) r2 = __fadd2_rn(r2, v);
+                bc += sTot[qb * D + c];
+                if (qb == 3) rc = bc;
+            }
+            xo = make_float2(off.x - r2.x, off.y - r2.y);
+            s_scale = ex2_approx(rc + carry);
+            carry = bc - rc;
         }
         {
-            const float eCr = __expf(bC - rc);
-            const TQ* sk = reinterpret_cast<const TQ*>(sm + PL::stK);
-            const TQ* sv = reinterpret_cast<const TQ*>(sm + PL::stV);
-            const TQ* sq = reinterpret_cast<const TQ*>(sm + (MODE == MODE_OUTPUT ? PL::stQ : PL::stK));
-            const int cofs = (c >> 3) * 128 + (c & 7) * 16;
+            const TQ* tq = nullptr;
+            const uint32_t* sk = reinterpret_cast<const uint32_t*>(sm + PL::stK) + cp;
+            const uint32_t* sv = reinterpret_cast<const uint32_t*>(sm + PL::stV) + cp;
+            const uint32_t* sq = reinterpret_cast<const uint32_t*>(sm + (OUT ? PL::stQ : PL::stK)) + cp;
+            // packed fp16 pairs (rows 2m, 2m+1) per channel: [channel][m]
+            uint32_t pk[2][4], pm[2][4], pv[2][4], pq[2][4];
+            float2 lk, lm, lv, lq;   // even row, waiting for its odd partner
 #pragma unroll
-            for (int grp = 0; grp < 2; ++grp) {
-                float kp[8], km[8], kt[8], vh[8], qp[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int r = grp * 8 + j, i = 16 * rb + r;
-                    const bool valid = full || t0 + i < T;
-                    const float kk = valid ? ld_in(sk + i * D + c) : 0.f;
-                    const float vv = valid ? ld_in(sv + i * D + c) : 0.f;
-                    const float bi = sBeta[i];
-                    const float x = bl[r] - rc;
-                    const float ep = __expf(x), em = __expf(-x);
-                    km[j] = kk * em;
-                    kt[j] = km[j] * eCr;
-                    kp[j] = kk * ep * bi;     // beta K+: A comes out row-scaled, W = T (beta K+)
-                    vh[j] = vv * bi;          // beta V:  U~ = T (beta V)
-                    if (MODE == MODE_OUTPUT) qp[j] = (valid ? ld_in(sq + i * D + c) : 0.f) * ep;
+            for (int r = 0; r < 8; ++r) {
+                const int i = 8 * rb + r;
+                const bool valid = full || i < nvalid;
+                float2 kk = in2(sk[i * (D / 2)], tq), vv = in2(sv[i * (D / 2)], tq);
+                float2 qq = OUT ? in2(sq[i * (D / 2)], tq) : make_float2(0.f, 0.f);
+                if (!valid) kk = vv = qq = make_float2(0.f, 0.f);
+                const float bi = sBeta[i];
+                const float2 b2 = make_float2(bi, bi);
+                const float2 x = __fadd2_rn(bl[r], xo);
+                const float2 ep = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                const float2 em = make_float2(ex2_approx(-x.x), ex2_approx(-x.y));
+                const float2 kp = __fmul2_rn(__fmul2_rn(kk, b2), ep);   // beta K+
+                const float2 km = __fmul2_rn(kk, em);                   // K-
+                const float2 vb = __fmul2_rn(vv, b2);                   // beta V
+                const float2 qp = __fmul2_rn(qq, ep);                   // Q+
+                if (r & 1) {
+                    const int m = r >> 1;
+                    pk[0][m] = pack_f16x2(lk.x, kp.x); pk[1][m] = pack_f16x2(lk.y, kp.y);
+                    pm[0][m] = pack_f16x2(lm.x, km.x); pm[1][m] = pack_f16x2(lm.y, km.y);
+                    pv[0][m] = pack_f16x2(lv.x, vb.x); pv[1][m] = pack_f16x2(lv.y, vb.y);
+                    pq[0][m] = pack_f16x2(lq.x, qp.x); pq[1][m] = pack_f16x2(lq.y, qp.y);
+                } else {
+                    lk = kp; lm = km; lv = vb; lq = qp;
                 }
-                const int ig = 2 * rb + grp;   // 8-row group of chunk positions
-                *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + cofs) = pack8_f16(kp);   // [beta K+ | beta V]
-                *reinterpret_cast<uint4*>(sm + PL::X + ig * 4096 + 2048 + cofs) = pack8_f16(vh);
-                *reinterpret_cast<uint4*>(sm + KM + ig * KM_IG + cofs) = pack8_f16(km);
-                *reinterpret_cast<uint4*>(sm + PL::KT + ig * 2048 + cofs) = pack8_f16(kt);
-                if (MODE == MODE_OUTPUT)
-                    *reinterpret_cast<uint4*>(sm + PL::Y + ig * 4096 + cofs) = pack8_f16(qp);
             }
+            // Threads with (cp & 4) store their odd channel first: each 8-thread phase of a
+            // 16-byte store then covers all 32 banks once.
+            const bool sw = (cp & 4) != 0;
+            const int c_first = 2 * cp + (sw ? 1 : 0), c_second = 2 * cp + (sw ? 0 : 1);
+            const uint32_t o1 = rb * 2048 + (c_first >> 3) * 128 + (c_first & 7) * 16;
+            const uint32_t o2 = rb * 2048 + (c_second >> 3) * 128 + (c_second & 7) * 16;
+            auto st2 = [&](int tile, const uint32_t (&pp)[2][4]) {
+                const uint4 a0 = make_uint4(pp[0][0], pp[0][1], pp[0][2], pp[0][3]);
+                const uint4 a1 = make_uint4(pp[1][0], pp[1][1], pp[1][2], pp[1][3]);
+                *reinterpret_cast<uint4*>(sm + tile + o1) = sw ? a1 : a0;
+                *reinterpret_cast<uint4*>(sm + tile + o2) = sw ? a0 : a1;
+            };
+            st2(PL::KP, pk);
+            st2(PL::KM, pm);
+            st2(PL::VB, pv);
+            if (OUT) st2(PL::QP, pq);
         }
         fence_async_smem();
         __syncthreads();
@@ -391,18 +442,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (t == NT / 2 && n + 1 < n1) issue_tma(n + 1);
         if (t == 0) {
             tc_fence_after();
-            if (MODE == MODE_OUTPUT) {
-                // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
-                const uint32_t id = idesc_f16(128, 64, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_AP, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
-                             sdesc(sbase + KM + 256 * kk, 128, 4096), id, kk > 0);
-            } else {
-                const uint32_t id = idesc_f16(64, 64, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_AP, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
-                             sdesc(sbase + KM + 256 * kk, 128, 2048), id, kk > 0);
-            }
+            // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
+            const uint32_t id = idesc_f16(OUT ? 128 : 64, 64, true, true);
+            for (int kk = 0; kk < 8; ++kk)
+                umma_f16(tmem + T_AP, sdesc(sbase + PL::KP + 256 * kk, 128, 2048),
+                         sdesc(sbase + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
             umma_commit(ctl.mma_bar);
         }
         tma_in_flight = n + 1 < n1;
@@ -412,11 +456,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // A = diag(beta) strict_lower(K+ K-^T) (beta is already in K+).
             wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == 0, 1);
             const uint32_t Ah = sbase + PL::U;       // A, fp16 K-major core-matrix tile
-            const uint32_t Tt = sbase + TT;          // T, same layout: the next MMA's operand
+            const uint32_t Tt = sbase + TT;          // T: the next MMA's operand
             {
                 float v[32];
                 int i = -1;
-                if (MODE == MODE_OUTPUT) {
+                if (OUT) {
                     // M = 128 layout: row i in lane i; rows 0-63 (quarters 0, 1) are A
                     if (q4 < 2) {
                         tmem_ld32(tl + T_AP + 32 * hg, v);
@@ -448,7 +492,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(sm + TT + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
+            tc_fence_before();
             named_sync(1, NT / 2);
+            if (MODE == MODE_STATE && t == 0) mbar_arrive(a_bar);   // Y may now overwrite A's columns
             // diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
             // N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs
             if (w < 4) {
@@ -543,76 +589,95 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             fence_async_smem();
         } else {
-            // ---- 3Y. warps 8-15: previous output; S^ = diag(e^r) S, master *= e^{b_C}; P; Y --
-            if (MODE == MODE_OUTPUT && prev_t0 >= 0 && q4 >= 2)
+            // ---- 3Y. warps 8-15: previous output; S^; Y (and O) = [beta K+ (; Q+)] S^; P; Y --
+            if (OUT && prev_t0 >= 0 && q4 >= 2)
                 store_o(tl, q4, 64 * hg, 2, lane, o, o_f32, b, T, H, h, prev_t0);
             {
-                const float er = __expf(rc), eC = __expf(bC);
+                // master (scaled form) -> S^ = 2^{r + carry} master: fp16 operand tile and the
+                // fp32 master both take the new scale
                 const int col0 = hg * (NS / 2);
                 for (int cc = 0; cc < NS / 2; cc += 32) {
                     float v[32];
                     tmem_ld32(tl + TM_S + col0 + cc, v);
 #pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        float f[8];
+                    for (int j = 0; j < 32; ++j) v[j] *= s_scale;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) f[j] = v[g8 * 8 + j] * er;
+                    for (int g8 = 0; g8 < 4; ++g8) {
                         const int col = col0 + cc + g8 * 8;
                         *reinterpret_cast<uint4*>(sm + PL::S + (col >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
-                            pack8_f16(f);
+                            pack8_f16(&v[8 * g8]);
                     }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] *= eC;
                     tmem_st32(tl + TM_S + col0 + cc, v);
                 }
             }
-            if (MODE == MODE_OUTPUT) {
-                // [Y; O] = [beta K+; Q+] S^ (M = 128), issued by thread NT/2 while warps 0-7
-                // invert: Y feeds U = T (beta V) - T Y, O is the inter-chunk output part
-                fence_async_smem();
-                tc_fence_before();
+            fence_async_smem();
+            tc_fence_before();
+            if (OUT) {
                 named_sync(2, NT / 2);
-                if (t == NT / 2) {
-                    tc_fence_after();
-                    const uint32_t idq = idesc_f16(128, 128, true, true);
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + T_YO, sdesc(sbase + PL::X + 256 * kk, 128, 4096),
-                                 sdesc(sbase + PL::S + 256 * kk, 128, 2048), idq, kk > 0);
-                    umma_commit(yo_bar);
-                }
-                yo_in_flight = true;
+            } else {
+                // Y's TMEM columns hold A until warps 0-7 have read it
+                wait_bar(a_bar, a_phase, ctl, t == NT / 2, 2);
             }
-            wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == NT / 2, 2);
-            if (MODE == MODE_OUTPUT && q4 >= 2) {
-                // P rows: lanes 64-127 of the M = 128 accumulator; P goes to the free 1 KB
-                // halves of the T region, so that [T; P] reads as one M = 128 operand
-                float v[32];
-                tmem_ld32(tl + T_AP + 32 * hg, v);
-                const int i = 32 * (q4 - 2) + lane;
+            if (t == NT / 2) {
+                tc_fence_after();
+                // OUT:   [Y; O] = [beta K+; Q+] S^   (M = 128, N = 128)
+                // STATE: Y = beta K+ [S^ | Phi^]     (M = 64,  N = 256)
+                const uint32_t idy = idesc_f16(OUT ? 128 : 64, NS, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + T_Y, sdesc(sbase + PL::KP + 256 * kk, 128, 2048),
+                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idy, kk > 0);
+                umma_commit(y_bar);
+            }
+            y_in_flight = true;
+            if (OUT) {
+                wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == NT / 2, 2);
+                if (q4 >= 2) {
+                    // P rows: lanes 64-127 of the M = 128 accumulator; P goes to the free 1 KB
+                    // halves of the T region, so that [T; P] reads as one M = 128 operand
+                    float v[32];
+                    tmem_ld32(tl + T_AP + 32 * hg, v);
+                    const int i = 32 * (q4 - 2) + lane;
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    float f[8];
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        float f[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int col = 32 * hg + 8 * g8 + j;
-                        f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
+                        for (int j = 0; j < 8; ++j) {
+                            const int col = 32 * hg + 8 * g8 + j;
+                            f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
+                        }
+                        *reinterpret_cast<uint4*>(sm + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)) = pack8_f16(f);
                     }
-                    *reinterpret_cast<uint4*>(sm + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)) = pack8_f16(f);
                 }
+            } else {
+                ctl.mma_phase ^= 1;   // A's phase: complete, since warps 0-7 have read A
             }
-            if (MODE == MODE_OUTPUT) {
-                wait_bar(yo_bar, yo_phase, ctl, t == NT / 2, 2);
-                yo_in_flight = false;
+            wait_bar(y_bar, y_phase, ctl, t == NT / 2, 2);
+            y_in_flight = false;
+            // Y -> fp16 position-major tile in the S^ region (S^ is no longer needed)
+            if (OUT) {
                 if (q4 < 2) {
-                    // Y rows j (lanes 0-63) -> fp16 MN-major B tile in the beta K+ halves of X
-                    const int j = 32 * q4 + lane;
+                    const int j = 32 * q4 + lane;    // M = 128 layout: row j in lane j
                     for (int cc = 0; cc < 64; cc += 32) {
                         float v[32];
-                        tmem_ld32(tl + T_YO + 64 * hg + cc, v);
+                        tmem_ld32(tl + T_Y + 64 * hg + cc, v);
 #pragma unroll
                         for (int g8 = 0; g8 < 4; ++g8) {
                             const int cg = (64 * hg + cc) / 8 + g8;
-                            *reinterpret_cast<uint4*>(sm + PL::X + (j >> 3) * 4096 + cg * 128 + (j & 7) * 16) =
+                            *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
+                                pack8_f16(&v[8 * g8]);
+                        }
+                    }
+                }
+            } else {
+                const int j = 16 * q4 + lane;        // M = 64 layout: lanes 0-15 of each quarter
+                for (int cc = 0; cc < 128; cc += 32) {
+                    float v[32];
+                    tmem_ld32(tl + T_Y + 128 * hg + cc, v);
+                    if (lane < 16) {
+#pragma unroll
+                        for (int g8 = 0; g8 < 4; ++g8) {
+                            const int cg = (128 * hg + cc) / 8 + g8;
+                            *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
                                 pack8_f16(&v[8 * g8]);
                         }
                     }
@@ -623,72 +688,35 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
         if (*sAbort) break;
-        if (MODE == MODE_OUTPUT) {
-            // ---- 4. U = T (beta V) - T Y  (critical path) -----------------------------------
-            if (t == 0) {
-                tc_fence_after();
-                const uint32_t idv = idesc_f16(64, 128, false, false);
-                const uint32_t idy = idesc_f16(64, 128, false, true, true);
+        // ---- 4. U = T (beta V) - T Y  (value columns; identity columns: -T Y) -------------
+        if (t == 0) {
+            tc_fence_after();
+            const uint32_t idv = idesc_f16(64, 128, false, false);
+            const uint32_t idy = idesc_f16(64, NS, false, true, true);
+            if (OUT) {
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_U, sdesc(sbase + TT + 4096 * kk, 2048, 128),
-                             sdesc(sbase + PL::X + 2048 + 8192 * kk, 4096, 128), idv, kk > 0);
+                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
+                             sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_U, sdesc(sbase + TT + 4096 * kk, 2048, 128),
-                             sdesc(sbase + PL::X + 8192 * kk, 4096, 128), idy, 1);
-                umma_commit(ctl.mma_bar);
-            }
-            wait_mma(ctl, t);
-        } else {
-            // ---- 4. [W | U~] = T [beta K+ | beta V] ---------------------------------------------
-            if (t == 0) {
-                tc_fence_after();
-                const uint32_t id256 = idesc_f16(64, 256, false, false);
+                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
+                             sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, 1);
+            } else {
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_W, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
-                             sdesc(sbase + PL::X + 8192 * kk, 4096, 128), id256, kk > 0);
-                umma_commit(ctl.mma_bar);
+                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
+                             sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
+                             sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, 1);
             }
-            wait_mma(ctl, t);
-            // W -> fp16 K-major tile [i][c] at X ([K+ | V] are no longer needed)
-            {
-                float v[32];
-                tmem_ld32(tl + T_W + 32 * cq, v);
-                if (lane < 16) {
-                    const int i = 16 * q4 + lane;
-#pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        const int cg = 4 * cq + g8;
-                        *reinterpret_cast<uint4*>(sm + PL::X + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                            pack8_f16(&v[8 * g8]);
-                    }
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (*sAbort) break;
-            // ---- 5. U = U~ - W S^, identity columns -W Phi^ (in W's columns) -----------------
-            if (t == 0) {
-                tc_fence_after();
-                const uint32_t idn = idesc_f16(64, 128, false, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_U, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
-                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idn, 1);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_W, sdesc(sbase + PL::X + 2048 * kk, 1024, 128),
-                             sdesc(sbase + PL::S + 32768 + 256 * kk, 128, 2048), idn, kk > 0);
-                umma_commit(ctl.mma_bar);
-            }
-            wait_mma(ctl, t);
+            umma_commit(ctl.mma_bar);
         }
-        // U -> fp16 MN-major tile [i][col] at U.  Value columns come from T_U, identity
-        // columns (MODE_STATE) from T_W.
+        wait_mma(ctl, t);
+        // U -> fp16 MN-major tile [i][col] at U (M = 64 layout: row 16*q4 + l in lane 32*q4 + l)
         {
             for (int cc = 0; cc < NQ; cc += 32) {
                 const int col = cq * NQ + cc;            // U tile column
-                const uint32_t src = (col < D) ? (T_U + col) : (T_W + col - D);
                 float v[32];
-                tmem_ld32(tl + src, v);
+                tmem_ld32(tl + T_UU + col, v);
                 if (lane < 16) {
                     const int i = 16 * q4 + lane;
 #pragma unroll
@@ -703,19 +731,19 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- 6. S += Kt^T U  (and O += P U) ---------------------------------------------
+        // ---- 5. master += K-^T U  (and O += P U) ------------------------------------------
         if (t == 0) {
             tc_fence_after();
             const uint32_t ids = idesc_f16(128, NS, false, true);
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + TM_S, sdesc(sbase + PL::KT + 4096 * kk, 2048, 128),
+                umma_f16(tmem + TM_S, sdesc(sbase + PL::KM + 4096 * kk, 2048, 128),
                          sdesc(sbase + PL::U + 256 * kk, 128, 1024), ids, 1);
-            if (MODE == MODE_OUTPUT) {
+            if (OUT) {
                 // O += P U as rows 64-127 of an M = 128 MMA whose rows 0-63 read T (their
                 // result lands on Y's rows, already consumed)
                 const uint32_t ido = idesc_f16(128, 128, false, true);
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_YO, sdesc(sbase + PL::TF + 4096 * kk, 2048, 128),
+                    umma_f16(tmem + T_Y, sdesc(sbase + PL::TF + 4096 * kk, 2048, 128),
                              sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
             }
             umma_commit(ctl.mma_bar);
@@ -724,15 +752,16 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mma_in_flight = false;
         prev_t0 = t0;
     }
-    if (MODE == MODE_OUTPUT && !*sAbort && prev_t0 >= 0 && q4 >= 2)
+    if (OUT && !*sAbort && prev_t0 >= 0 && q4 >= 2)
         store_o(tl, q4, 32 * cq, 1, lane, o, o_f32, b, T, H, h, prev_t0);
 
-    // ---- end of segment: write the state ------------------------------------------------
+    // ---- end of segment: write the state S = diag(2^{carry}) master ---------------------
     if (!*sAbort) {
         float* dst = nullptr;
         if (MODE == MODE_STATE) dst = maps + (size_t)(bh * (P - 1) + p) * 2 * D * D;  // [N | M]
         else if (S_T && p == P - 1) dst = S_T + (size_t)bh * D * D;
         if (dst) {
+            const float sc = ex2_approx(carry);
             const int col0 = cq * NQ;
             for (int cc = 0; cc < NQ; cc += 32) {
                 float v[32];
@@ -742,7 +771,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const int col = col0 + cc + j;
                     // maps: N block (value columns) then M block (identity columns)
                     const size_t idx = (col < D) ? ((size_t)c * D + col) : ((size_t)D * D + (size_t)c * D + (col - D));
-                    dst[idx] = v[j];
+                    dst[idx] = v[j] * sc;
                 }
             }
         }
@@ -751,7 +780,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (*sAbort) {
         if (mma_in_flight) mbar_wait_bounded(ctl.mma_bar, ctl.mma_phase, kWaitNs);
         if (tma_in_flight) mbar_wait_bounded(ctl.tma_bar, ctl.tma_phase, kWaitNs);
-        if (yo_in_flight && t == NT / 2) mbar_wait_bounded(yo_bar, yo_phase, kWaitNs);
+        if (y_in_flight && t == NT / 2) mbar_wait_bounded(y_bar, y_phase, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
