@@ -319,17 +319,23 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int col0 = cq * NQ;
         for (int cc = 0; cc < NQ; cc += 32) {
             float v[32];
+            if (MODE == MODE_STATE) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int col = col0 + cc + j;
-                float x = 0.f;
-                if (MODE == MODE_STATE) {
-                    x = (col >= D && col - D == c) ? 1.f : 0.f;
-                } else if (S_in) {
-                    const size_t idx = s_in_per_segment ? (size_t)bh * P + p : (size_t)bh;
-                    x = S_in[(idx * D + c) * D + col];
+                for (int j = 0; j < 32; ++j) {
+                    const int col = col0 + cc + j;
+                    v[j] = (col >= D && col - D == c) ? 1.f : 0.f;
                 }
-                v[j] = x;
+            } else if (S_in) {
+                const size_t idx = s_in_per_segment ? (size_t)bh * P + p : (size_t)bh;
+                const float4* s4 = reinterpret_cast<const float4*>(S_in + (idx * D + c) * D + col0 + cc);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 x = s4[j];
+                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = 0.f;
             }
             tmem_st32(tl + TM_S + col0 + cc, v);
         }
@@ -438,8 +444,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         fence_async_smem();
         __syncthreads();
-        // ---- 2. next chunk's TMA; A (and P) on the tensor core ----------------------------
-        if (t == NT / 2 && n + 1 < n1) issue_tma(n + 1);
+        // ---- 2. A (and P) on the tensor core ----------------------------------------------
         if (t == 0) {
             tc_fence_after();
             // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
@@ -627,6 +632,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     umma_f16(tmem + T_Y, sdesc(sbase + PL::KP + 256 * kk, 128, 2048),
                              sdesc(sbase + PL::S + 256 * kk, 128, 2048), idy, kk > 0);
                 umma_commit(y_bar);
+                // the next chunk's q, k, v, g land while the inverse runs (the staging
+                // buffer was last read by this chunk's prologue)
+                if (n + 1 < n1) issue_tma(n + 1);
             }
             y_in_flight = true;
             if (OUT) {
@@ -766,13 +774,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int cc = 0; cc < NQ; cc += 32) {
                 float v[32];
                 tmem_ld32(tl + TM_S + col0 + cc, v);
+                // maps: N block (value columns) then M block (identity columns); a 32-column
+                // run never straddles the two
+                const int col = col0 + cc;
+                const size_t idx = (col < D) ? ((size_t)c * D + col) : ((size_t)D * D + (size_t)c * D + (col - D));
+                float4* d4 = reinterpret_cast<float4*>(dst + idx);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int col = col0 + cc + j;
-                    // maps: N block (value columns) then M block (identity columns)
-                    const size_t idx = (col < D) ? ((size_t)c * D + col) : ((size_t)D * D + (size_t)c * D + (col - D));
-                    dst[idx] = v[j] * sc;
-                }
+                for (int j = 0; j < 8; ++j)
+                    d4[j] = make_float4(v[4 * j] * sc, v[4 * j + 1] * sc, v[4 * j + 2] * sc, v[4 * j + 3] * sc);
             }
         }
     }
