@@ -1,4 +1,4 @@
-// Tensor-core (tcgen05 / TMEM / TMA) chunkwise KDA forward for Dk = Dv = 128, chunk 64.
+// Tensor-core (tcgen05 / TMEM) chunkwise KDA forward for Dk = Dv = 128, chunk 64.
 //
 // What it computes is Eq. 14 of the Chimera paper (section 3.3) with the readout
 // o_t = S_t^T q_t (Eq. 15, inner term).  The pages only say the kernel is "chunked";
@@ -27,15 +27,31 @@
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
 //   pass 2 (MODE_OUTPUT, all segments): run the recurrence from S_start(p) and write
 //          o (and S_T from the last segment).
-// Each pass is one CTA per (b, h, segment), 512 threads, ~200 KB of shared memory.
+//
+// Inside a CTA (one per (b, h, segment), 512 threads) two warp groups form a
+// two-stage pipeline over the segment's chunks:
+//   producer (warps 0-7): forms beta K+, Q+, K- (fp16 tiles) of chunk n+1, issues
+//     A|P, reads A and P out of TMEM and inverts I + A.  Everything it does is
+//     independent of the state.
+//   consumer (warps 8-15): chunk n's state chain: S^ from the master, [Y; O] MMA,
+//     beta V, U MMA, master += K-^T U and O += P U, output store.
+// The per-chunk tiles are double-buffered; mbarriers hand a buffer over (full) and
+// back (empty, committed by the consumer's last MMA that reads it).  Inputs arrive by
+// TMA straight into the tiles that consume them and are converted in place: q and k
+// of chunk n+2 land in the Q+ / beta K+ slots of their buffer set as soon as the
+// consumer's [Y; O] MMA of chunk n has read them, v of chunk n+1 lands in the beta V
+// tile once chunk n's U MMA has read it, and g of chunk n+1 in a staging tile once the
+// producer has summed chunk n's.
 //
 // Shared-memory operand tiles use the no-swizzle core-matrix layout: 8 rows x 16 B
 // blocks of 128 contiguous bytes.  A thread that owns one key channel writes 8
 // consecutive chunk positions as one 16-byte store, so the channel-major tiles serve
 // both as MN-major operands (chunk position = M/N) and K-major ones (position = K).
 //
-// All waits are bounded (kWaitNs); on expiry the kernel records DEV_TIMEOUT in the
-// device status word, drains its own copies and MMAs, frees TMEM and returns.
+// All waits are bounded (kWaitNs).  On expiry the kernel records DEV_TIMEOUT in the
+// device status word and stops waiting: both warp groups still run every barrier of
+// their loop (so neither can hang on the other), results are undefined, and before
+// TMEM is freed each MMA-issuing thread drains its own MMAs.
 
 #include <mutex>
 #include <type_traits>
@@ -51,51 +67,60 @@ using namespace sm100;
 constexpr int C = 64;         // chunk length
 constexpr int D = 128;        // Dk = Dv
 constexpr int NT = 512;       // threads per CTA
+constexpr int NG = 256;       // threads per warp group
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
 constexpr float kLog2e = 1.4426950408889634f;
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
 // ---- shared-memory plan (bytes) --------------------------------------------------
-// Channel-major fp16 tiles (K+ beta, Q+, K-, beta V): 8-position group ig at
-// tile + ig*2048, channel c at (c >> 3)*128 + (c & 7)*16 inside it.  Q+ follows K+ beta
-// directly, so [beta K+; Q+] is one M = 128 operand.  After the Y MMA the S^ region
-// holds Y (position-major: 8-position group j at j*NS*16, 8 columns per 16 bytes).
+// Two buffer sets (one per chunk parity) of channel-major fp16 tiles: 8-position group
+// ig at tile + ig*2048, channel c at (c >> 3)*128 + (c & 7)*16 inside it.  Q+ follows
+// beta K+ directly, so [beta K+; Q+] is one M = 128 operand.  T (and P) sit in the
+// set: 8-column groups of T are T_LBO apart; in MODE_OUTPUT P fills the other 1 KB
+// halves, so [T; P] is one M = 128 operand.  The consumer's S^ region holds Y
+// (position-major: 8-position group j at j*NS*16, 8 columns per 16 bytes) once the
+// [Y; O] MMA has read S^.
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int NS = 128;                 // state columns (values only)
-    static constexpr int stQ = 0, stK = 16384, stV = 32768, stG = 49152;  // TMA staging, [64][128]
-    static constexpr int KP = 65536;               // beta K+
-    static constexpr int QP = 81920;               // Q+
-    static constexpr int KM = 98304;               // K-
-    static constexpr int VB = 114688;              // beta V
-    static constexpr int TF = 131072;              // T (64 x 64 fp16, K-major, 8-column groups 2 KB
-                                                   // apart) interleaved with P in the other 1 KB halves
-    static constexpr int U = 147456;               // fp16 A during the inverse, then U (64 x 128)
-    static constexpr int S = 163840;               // S^ (128 x 128 fp16), then Y
-    static constexpr int MISC = 196608;
-    static constexpr int TMA_BYTES = 4 * 16384;
+    static constexpr int SET = 65536;              // buffer set stride
+    static constexpr int KP = 0, QP = 16384, KM = 32768, TF = 49152;   // inside a set
+    static constexpr int T_LBO = 2048;
+    static constexpr int VB = 131072;              // beta V (consumer)
+    static constexpr int AT = 147456;              // A, fp16 (producer)
+    static constexpr int U = 155648;               // U (64 x 128)
+    static constexpr int S = 172032;               // S^ (128 x 128 fp16), then Y
+    static constexpr int GST = 204800;             // g staging ([64][128] bf16, TMA)
+    static constexpr int MISC = 221184;
+    static constexpr int QK_BYTES = 2 * 16384;     // q and k of one chunk
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int NS = 256;                 // [S | Phi]
-    static constexpr int stQ = -1, stK = 0, stV = 16384, stG = 32768;
-    static constexpr int KP = 49152;
-    static constexpr int QP = -1;
-    static constexpr int KM = 65536;
+    static constexpr int SET = 40960;
+    static constexpr int KP = 0, QP = -1, KM = 16384, TF = 32768;
+    static constexpr int T_LBO = 1024;
     static constexpr int VB = 81920;
-    static constexpr int TF = -1;                  // T lives at U + 8192
-    static constexpr int U = 98304;                // fp16 A and T during the inverse, then U (64 x 256)
-    static constexpr int S = 131072;               // [S^ | Phi^] (128 x 256 fp16), then Y
-    static constexpr int MISC = 196608;
-    static constexpr int TMA_BYTES = 3 * 16384;
+    static constexpr int AT = 98304;
+    static constexpr int U = 106496;               // U (64 x 256)
+    static constexpr int S = 139264;               // [S^ | Phi^] (128 x 256 fp16), then Y
+    static constexpr int GST = 204800;
+    static constexpr int MISC = 221184;
+    static constexpr int QK_BYTES = 16384;         // k of one chunk
 };
 // MISC sub-layout
-constexpr int M_BETA = 0;        // float[64]
-constexpr int M_TOT = 256;       // float[8][128] per-8-row-block sums of g log2(e)
-constexpr int M_XS = 4352;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 8448;      // 4 x uint64 mbarriers (TMA, MMA, second issuer, A read)
-constexpr int M_TMEM = 8480;     // uint32 TMEM base
-constexpr int M_ABORT = 8484;    // int
-constexpr int MISC_BYTES = 8496;
+constexpr int M_BETAP = 0;       // float[64]  beta of the producer's chunk
+constexpr int M_BETAC = 256;     // float[64]  beta of the consumer's chunk
+constexpr int M_TOT = 512;       // float[4][128] per-16-row sums of g log2(e)
+constexpr int M_RB = 2560;       // float2[2][128] (r, b_C) per channel, per buffer set
+constexpr int M_XS = 4608;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 8704;      // mbarriers, see Bar
+constexpr int M_TMEM = 8848;     // uint32 TMEM base
+constexpr int M_ABORT = 8852;    // int
+constexpr int MISC_BYTES = 8864;
+// PRO: a set's beta K+, Q+, K- tiles and r, b_C are ready; INV: its T (and P) too;
+// EMPTY: the consumer's last MMA on the set is done.
+enum Bar { B_PRO = 0, B_EMPTY = 2, B_AP = 4, B_Y = 5, B_U = 6, B_S = 7, B_AFREE = 8, B_UREAD = 9,
+           B_DRAIN = 10, B_DRAIN2 = 11, B_TQK = 12, B_TG = 14, B_TV = 15, B_INV = 16, NBAR = 18 };
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
@@ -109,9 +134,6 @@ template <> struct Tm<MODE_OUTPUT> { static constexpr uint32_t Y = 128, UU = 384
 template <> struct Tm<MODE_STATE> { static constexpr uint32_t Y = 256, UU = 256; };
 
 // ---- helpers ------------------------------------------------------------------------
-__device__ __forceinline__ float ld_in(const __nv_bfloat16* p) { return __bfloat162float(*p); }
-__device__ __forceinline__ float ld_in(const __half* p) { return __half2float(*p); }
-
 __device__ __forceinline__ uint4 pack8_f16(const float* f)
 {
     uint4 u;
@@ -120,6 +142,13 @@ __device__ __forceinline__ uint4 pack8_f16(const float* f)
     for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
     return u;
 }
+
+// Two adjacent 2-byte input elements -> fp32
+__device__ __forceinline__ float2 in2(uint32_t u, const __nv_bfloat16*)
+{
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ float2 in2(uint32_t u, const __half*) { return unpack_f16x2(u); }
 
 // Byte offset of (row i, column j), j % 8 == 0, in a 64 x 64 fp16 tile in the
 // K-major core-matrix layout the tensor-core MMA reads (8-column groups 1 KB apart).
@@ -162,76 +191,105 @@ __device__ __forceinline__ void named_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-struct Ctl {
-    uint64_t* tma_bar;
-    uint64_t* mma_bar;
-    int* abort_flag;
+// Shared abort state.  A wait that runs out records DEV_TIMEOUT and raises the flag;
+// once it is up, pollers stop waiting (barriers still run, so no group can hang).
+struct Abort {
+    int* flag;
     int* status;
-    uint32_t tma_phase, mma_phase;
 };
-
-// Bounded waits.  One thread polls the mbarrier; the others wait at a barrier (no
-// issue slots spent polling): the whole CTA (bar_id 0) or one 256-thread group.  The
-// CTA agrees on a timeout through the shared abort flag.  After an MMA wait every
-// thread orders its TMEM reads behind it.
-__device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t& phase, Ctl& c, bool poller, int bar_id)
+// One thread polls; the group (bar_id, NG threads) waits at its named barrier.
+__device__ __forceinline__ void group_wait(uint64_t* bar, uint32_t parity, const Abort& a, bool poller, int bar_id)
 {
-    if (poller && !mbar_wait_bounded(bar, phase, kWaitNs)) {
-        *c.abort_flag = 1;
-        atomicCAS(c.status, DEV_OK, DEV_TIMEOUT);
+    if (poller && !*a.flag && !mbar_wait_bounded(bar, parity, kWaitNs)) {
+        *a.flag = 1;
+        atomicCAS(a.status, DEV_OK, DEV_TIMEOUT);
     }
-    if (bar_id == 0) __syncthreads();
-    else named_sync(bar_id, NT / 2);
-    phase ^= 1;
+    named_sync(bar_id, NG);
     tc_fence_after();
 }
-__device__ __forceinline__ void wait_mma(Ctl& c, int t) { wait_bar(c.mma_bar, c.mma_phase, c, t == 0, 0); }
-__device__ __forceinline__ void wait_tma(Ctl& c, int t) { wait_bar(c.tma_bar, c.tma_phase, c, t == 0, 0); }
-
-// Two adjacent 2-byte input elements -> fp32
-__device__ __forceinline__ float2 in2(uint32_t u, const __nv_bfloat16*)
+// One thread waits alone (before issuing MMAs that depend on the other group).
+__device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, const Abort& a)
 {
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    if (!*a.flag && !mbar_wait_bounded(bar, parity, kWaitNs)) {
+        *a.flag = 1;
+        atomicCAS(a.status, DEV_OK, DEV_TIMEOUT);
+    }
 }
-__device__ __forceinline__ float2 in2(uint32_t u, const __half*) { return unpack_f16x2(u); }
 
-// Output rows of one chunk from TMEM to global memory.  O is rows 64-127 of the
-// M = 128 accumulator [Y; O]: output row i sits in lane 64 + i, so warps of lane
-// quarters 2 and 3 store it; this warp stores columns col0 .. col0 + 32*nld - 1.
-__device__ __forceinline__ void store_o(uint32_t tl, int q4, int col0, int nld, int lane, void* o, int o_f32,
-                                        int b, int T, int H, int h, int t0)
+// Output rows of one chunk, TMEM -> global memory.  O is rows 64-127 of the M = 128
+// accumulator [Y; O] (output row i in lane 64 + i), so warps of lane quarters 2 and 3
+// copy it into a row-major staging tile (rows padded by 16 bytes: the 8 rows of a
+// 16-byte store phase hit 8 different bank groups); after the group barrier every warp
+// of the group writes whole rows with coalesced 16-byte stores.
+__device__ __forceinline__ void stage_o(uint32_t tl, int q4, int hg, int lane, uint8_t* stg, int o_f32)
 {
-    for (int u = 0; u < nld; ++u) {
+    if (q4 < 2) return;
+    const int i = 32 * (q4 - 2) + lane;
+    const int es = o_f32 ? 4 : 2, ld = D * es + 16;
+    for (int u = 0; u < 2; ++u) {
         float v[32];
-        const int cc = col0 + 32 * u;
+        const int cc = 64 * hg + 32 * u;
         tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + cc, v);
-        const int i = 32 * (q4 - 2) + lane;
-        if (t0 + i < T) {
-            const size_t off = (((size_t)b * T + t0 + i) * H + h) * D + cc;
-            if (o_f32) {
-                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(o) + off);
+        uint8_t* row = stg + i * ld + cc * es;
+        if (o_f32) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            } else {
-                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(o) + off);
+            for (int j = 0; j < 8; ++j)
+                reinterpret_cast<float4*>(row)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4 uu;
-                    __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
+            for (int j = 0; j < 4; ++j) {
+                uint4 uu;
+                __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-                    dst[j] = uu;
-                }
+                for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+                reinterpret_cast<uint4*>(row)[j] = uu;
             }
         }
     }
 }
+__device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int b, int T, int H, int h,
+                                        int t0)
+{
+    const int es = o_f32 ? 4 : 2, ld = D * es + 16;
+    const int per_row = D * es / 16;                 // 16-byte pieces per row
+    for (int e = tg; e < C * per_row; e += NG) {
+        const int i = e / per_row, pc = e % per_row;
+        if (t0 + i < T) {
+            const uint4 x = *reinterpret_cast<const uint4*>(stg + i * ld + pc * 16);
+            uint8_t* dst = reinterpret_cast<uint8_t*>(o) + ((((size_t)b * T + t0 + i) * H + h) * D) * es + pc * 16;
+            *reinterpret_cast<uint4*>(dst) = x;
+        }
+    }
+}
+
+// 16 rows x 2 channels (one 4-byte word per row) of a [64][128] 2-byte tile in shared
+// memory, as TMA lands it: a warp reads 128 contiguous bytes per row.
+__device__ __forceinline__ void ld_rows16(uint32_t (&dst)[16], const uint8_t* tile, int r0, int cp)
+{
+#pragma unroll
+    for (int r = 0; r < 16; ++r) dst[r] = *reinterpret_cast<const uint32_t*>(tile + (r0 + r) * 256 + 4 * cp);
+}
+__device__ __forceinline__ uint32_t load_beta(const __nv_bfloat16* beta, int b, int T, int H, int h, int t0, int i,
+                                              bool live)
+{
+    const int tt = t0 + i;
+    return (live && tt < T) ? (uint32_t) * reinterpret_cast<const unsigned short*>(beta + ((size_t)b * T + tt) * H + h)
+                            : 0u;
+}
+// Store two channels' packed fp16 rows (one 16-byte vector per channel) into a
+// channel-major tile.  Threads with (cp & 4) store their odd channel first: each
+// 8-thread phase of a 16-byte store then covers all 32 banks once.
+__device__ __forceinline__ void st_pair(uint8_t* tile, int ig, int cp, const uint32_t (&pp)[2][4])
+{
+    const bool sw = (cp & 4) != 0;
+    const int c_first = 2 * cp + (sw ? 1 : 0), c_second = 2 * cp + (sw ? 0 : 1);
+    const uint4 a0 = make_uint4(pp[0][0], pp[0][1], pp[0][2], pp[0][3]);
+    const uint4 a1 = make_uint4(pp[1][0], pp[1][1], pp[1][2], pp[1][3]);
+    *reinterpret_cast<uint4*>(tile + ig * 2048 + (c_first >> 3) * 128 + (c_first & 7) * 16) = sw ? a1 : a0;
+    *reinterpret_cast<uint4*>(tile + ig * 2048 + (c_second >> 3) * 128 + (c_second & 7) * 16) = sw ? a0 : a1;
+}
 
 // The kernel ---------------------------------------------------------------------------
-// 512 threads.  Prologue: thread t owns key channels 2*(t & 63) + {0, 1} and chunk rows
-// 8*(t >> 6) .. +7.  TMEM: warp w reads lane quarter w & 3.  While warps 0-7 read A and
-// invert (I + A), warps 8-15 store the previous chunk's output, rescale the state,
-// issue Y (and O) from S^, and read P and Y.
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -243,43 +301,37 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     using PL = Plan<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
     constexpr int NS = PL::NS;
-    constexpr int NQ = NS / 4;                // state columns per column quarter (all 16 warps)
     constexpr int YJ = NS * 16;               // Y tile: bytes per 8-position group
+    constexpr int T_LBO = PL::T_LBO;          // T's 8-column group stride
     constexpr uint32_t T_Y = Tm<MODE>::Y, T_UU = Tm<MODE>::UU;
-    constexpr int TT = OUT ? PL::TF : PL::U + 8192;   // T tile base
-    constexpr int T_LBO = OUT ? 2048 : 1024;          // T's 8-column group stride
     auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     extern __shared__ __align__(1024) uint8_t sm[];
 
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-    const int q4 = w & 3, cq = w >> 2;        // TMEM lane quarter, column quarter
-    const bool grpY = w >= 8;                 // second 256-thread group
-    const int hg = (w >> 2) & 1;              // column half inside a group
+    const int q4 = w & 3;                     // TMEM lane quarter of this warp
+    const int hg = (w >> 2) & 1;              // column half inside a warp group
+    const int tg = t & (NG - 1);              // thread index inside its group
+    const int cp = tg & 63, rq = tg >> 6;     // channel pair, 16-row quarter (loads, prologue)
     const int c = t & 127;                    // channel / TMEM row of the state steps
-    const int cp = t & 63, rb = t >> 6;       // prologue: channel pair, 8-row block
     const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
     const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
     const int b = bh / H, h = bh % H;
     const int NC = (T + C - 1) / C;
     const int n0 = p * L, n1 = min(NC, n0 + L);
+    const int nk = max(0, n1 - n0);
 
-    float* sBeta = reinterpret_cast<float*>(sm + PL::MISC + M_BETA);
+    float* sBetaP = reinterpret_cast<float*>(sm + PL::MISC + M_BETAP);
+    float* sBetaC = reinterpret_cast<float*>(sm + PL::MISC + M_BETAC);
     float* sTot = reinterpret_cast<float*>(sm + PL::MISC + M_TOT);
+    float2* sRB = reinterpret_cast<float2*>(sm + PL::MISC + M_RB);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
     int* sAbort = reinterpret_cast<int*>(sm + PL::MISC + M_ABORT);
     const uint32_t sbase = smem_addr(sm);
+    const Abort ab{sAbort, status};
 
-    Ctl ctl{&bars[0], &bars[1], sAbort, status, 0u, 0u};
-    uint64_t* y_bar = &bars[2];       // MMAs issued by thread NT/2 (Y, and O in MODE_OUTPUT)
-    uint64_t* a_bar = &bars[3];       // MODE_STATE: A has been read out of TMEM
-    uint32_t y_phase = 0, a_phase = 0;
-    bool y_in_flight = false;
     if (t == 0) {
-        mbar_init(ctl.tma_bar, 1);
-        mbar_init(ctl.mma_bar, 1);
-        mbar_init(y_bar, 1);
-        mbar_init(a_bar, 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
         *sAbort = 0;
         fence_mbar_init();
     }
@@ -292,189 +344,142 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *sTmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);   // this warp's lane quarter
-    bool tma_in_flight = false;
-    bool mma_in_flight = false;
-
-    auto issue_tma = [&](int n) {
-        const int row = b * T + n * C;
-        mbar_arrive_expect_tx(ctl.tma_bar, PL::TMA_BYTES);
-        if (OUT) tma_load_3d(sm + PL::stQ, &tm_q, ctl.tma_bar, 0, h, row);
-        tma_load_3d(sm + PL::stK, &tm_k, ctl.tma_bar, 0, h, row);
-        tma_load_3d(sm + PL::stV, &tm_v, ctl.tma_bar, 0, h, row);
-        tma_load_3d(sm + PL::stG, &tm_g, ctl.tma_bar, 0, h, row);
+    // TMA of chunk n's [64][128] tiles (rows b*T + n*C ..; rows past the segment's data
+    // come from the next batch row or the zero fill and are masked where they are used)
+    auto tma_qk = [&](int n) {   // q (MODE_OUTPUT) and k into the Q+ / beta K+ slots of set n&1
+        const int bs = (n - n0) & 1, row = b * T + n * C;
+        mbar_arrive_expect_tx(&bars[B_TQK + bs], PL::QK_BYTES);
+        if (OUT) tma_load_3d(sm + bs * PL::SET + PL::QP, &tm_q, &bars[B_TQK + bs], 0, h, row);
+        tma_load_3d(sm + bs * PL::SET + PL::KP, &tm_k, &bars[B_TQK + bs], 0, h, row);
     };
-    // beta is prefetched one chunk ahead as raw bf16 bits (no use until the next chunk,
-    // so the load never stalls the thread); the index is clamped to stay in bounds.
-    auto load_beta_bits = [&](int n) -> uint32_t {
-        const int tt = n * C + t;
-        const int ts = (n < n1 && tt < T) ? tt : 0;
-        return *reinterpret_cast<const unsigned short*>(beta + ((size_t)b * T + ts) * H + h);
+    auto tma_g = [&](int n) {
+        mbar_arrive_expect_tx(&bars[B_TG], 16384);
+        tma_load_3d(sm + PL::GST, &tm_g, &bars[B_TG], 0, h, b * T + n * C);
     };
-    if (t == 0 && n0 < n1) issue_tma(n0);
-    tma_in_flight = n0 < n1;
-    uint32_t beta_bits = (t < C) ? load_beta_bits(n0) : 0u;
+    auto tma_v = [&](int n) {
+        mbar_arrive_expect_tx(&bars[B_TV], 16384);
+        tma_load_3d(sm + PL::VB, &tm_v, &bars[B_TV], 0, h, b * T + n * C);
+    };
 
-    // ---- initial state in TMEM ------------------------------------------------------
-    {
-        const int col0 = cq * NQ;
-        for (int cc = 0; cc < NQ; cc += 32) {
-            float v[32];
-            if (MODE == MODE_STATE) {
+    if (t < NG) {
+        // ================= producer: state-independent work of chunk n0 + kc ==============
+        const TQ* tq = nullptr;
+        uint32_t betaR = 0;
+        int g_issued = 0;   // thread 0: g tiles requested so far
+        if (tg == 0 && nk > 0) {
+            tma_g(n0);
+            g_issued = 1;
+        }
+        if (tg < C) betaR = load_beta(beta, b, T, H, h, n0 * C, tg, nk > 0);
+        for (int kc = 0; kc < nk; ++kc) {
+            const int n = n0 + kc, t0 = n * C, bs = kc & 1;
+            uint8_t* set = sm + bs * PL::SET;
+            const uint32_t sset = sbase + bs * PL::SET;
+            // buffer set bs is free once the consumer is done with chunk kc - 2 (its K- and
+            // T tiles); this chunk's q, k (in the set) and g (staging) have landed
+            if (tg == 0) {
+                if (kc >= 2) thread_wait(&bars[B_EMPTY + bs], ((kc >> 1) - 1) & 1, ab);
+                thread_wait(&bars[B_TQK + bs], (kc >> 1) & 1, ab);
+            }
+            group_wait(&bars[B_TG], kc & 1, ab, tg == 0, 1);
+            // ---- prologue: cumulative log-decay, beta K+, Q+, K- tiles (in place) -------
+            {
+                uint32_t gR[16], kR[16], qR[16];
+                ld_rows16(gR, sm + PL::GST, 16 * rq, cp);
+                ld_rows16(kR, set + PL::KP, 16 * rq, cp);
+                if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
+                const bool full = t0 + C <= T;
+                if (!full) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int col = col0 + cc + j;
-                    v[j] = (col >= D && col - D == c) ? 1.f : 0.f;
+                    for (int r = 0; r < 16; ++r)
+                        if (t0 + 16 * rq + r >= T) gR[r] = kR[r] = qR[r] = 0u;
                 }
-            } else if (S_in) {
-                const size_t idx = s_in_per_segment ? (size_t)bh * P + p : (size_t)bh;
-                const float4* s4 = reinterpret_cast<const float4*>(S_in + (idx * D + c) * D + col0 + cc);
+                const float2 l2e = make_float2(kLog2e, kLog2e);
+                float2 tot = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 x = s4[j];
-                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                for (int r = 0; r < 16; ++r) tot = __ffma2_rn(in2(gR[r], (const __nv_bfloat16*)nullptr), l2e, tot);
+                *reinterpret_cast<float2*>(sTot + rq * D + 2 * cp) = tot;
+                if (tg < C) sBetaP[tg] = __uint_as_float(betaR << 16);
+                named_sync(1, NG);   // every staged value of this chunk is in registers now
+                if (tg == 0 && n + 1 < n1 && !*sAbort) {
+                    tma_g(n + 1);
+                    g_issued = kc + 2;
                 }
-            } else {
+                if (tg < C) betaR = load_beta(beta, b, T, H, h, (n + 1) * C, tg, n + 1 < n1);
+                float2 tq4[4];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            }
-            tmem_st32(tl + TM_S + col0 + cc, v);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // The master holds diag(2^{-carry}) S for channel c (log2 units; 0 before any chunk).
-    float carry = 0.f;
-    int prev_t0 = -1;   // chunk whose output still sits in TMEM (MODE_OUTPUT)
-    for (int n = n0; n < n1 && !*sAbort; ++n) {
-        const int t0 = n * C;
-        // ---- 1. prologue: staging -> fp16 operand tiles --------------------------------
-        wait_tma(ctl, t);
-        if (*sAbort) break;
-        tma_in_flight = false;
-        if (t < C) {
-            sBeta[t] = (t0 + t < T) ? __uint_as_float(beta_bits << 16) : 0.f;
-            beta_bits = load_beta_bits(n + 1);    // in flight during this chunk
-        }
-        const bool full = t0 + C <= T;   // no ragged rows in this chunk
-        const int nvalid = T - t0;       // rows i < nvalid are tokens
-        float2 bl[8];                    // b log2(e) for this thread's two channels, rows 8*rb + r
-        {
-            const uint32_t* stg = reinterpret_cast<const uint32_t*>(sm + PL::stG) + cp;
-            float2 run = make_float2(0.f, 0.f);
-            const float2 l2e = make_float2(kLog2e, kLog2e);
+                for (int qb = 0; qb < 4; ++qb) tq4[qb] = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
+                const float2 r2 = __fadd2_rn(tq4[0], tq4[1]);                  // b at row 31
+                const float2 bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));  // b at row 63
+                float2 run = make_float2(-r2.x, -r2.y);                        // running b - r
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int i = 8 * rb + r;
-                float2 gv = in2(stg[i * (D / 2)], (const __nv_bfloat16*)nullptr);
-                if (!full && i >= nvalid) gv = make_float2(0.f, 0.f);
-                run = __ffma2_rn(gv, l2e, run);
-                bl[r] = run;
-            }
-            *reinterpret_cast<float2*>(sTot + rb * D + 2 * cp) = run;
-        }
-        __syncthreads();
-        float2 xo;              // (sum of the earlier row blocks) - r, this thread's channel pair
-        float s_scale;          // state row scale for channel c: 2^{r + carry}
-        {
-            float2 off = make_float2(0.f, 0.f), r2 = make_float2(0.f, 0.f);
-            float rc = 0.f, bc = 0.f;
+                for (int qb = 0; qb < 3; ++qb)
+                    if (qb < rq) run = __fadd2_rn(run, tq4[qb]);
+                if (rq == 0) {
+                    sRB[bs * D + 2 * cp] = make_float2(r2.x, bC.x);
+                    sRB[bs * D + 2 * cp + 1] = make_float2(r2.y, bC.y);
+                }
 #pragma unroll
-            for (int qb = 0; qb < 8; ++qb) {
-                const float2 v = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
-                if (qb < rb) off = __fadd2_rn(off, v);
-                if (qb < 4) r2 = __fadd2_rn(r2, v);
-                bc += sTot[qb * D + c];
-                if (qb == 3) rc = bc;
-            }
-            xo = make_float2(off.x - r2.x, off.y - r2.y);
-            s_scale = ex2_approx(rc + carry);
-            carry = bc - rc;
-        }
-        {
-            const TQ* tq = nullptr;
-            const uint32_t* sk = reinterpret_cast<const uint32_t*>(sm + PL::stK) + cp;
-            const uint32_t* sv = reinterpret_cast<const uint32_t*>(sm + PL::stV) + cp;
-            const uint32_t* sq = reinterpret_cast<const uint32_t*>(sm + (OUT ? PL::stQ : PL::stK)) + cp;
-            // packed fp16 pairs (rows 2m, 2m+1) per channel: [channel][m]
-            uint32_t pk[2][4], pm[2][4], pv[2][4], pq[2][4];
-            float2 lk, lm, lv, lq;   // even row, waiting for its odd partner
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[2][4], pm[2][4], pq[2][4];
+                    float2 lk = make_float2(0.f, 0.f), lm = lk, lq = lk;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int i = 8 * rb + r;
-                const bool valid = full || i < nvalid;
-                float2 kk = in2(sk[i * (D / 2)], tq), vv = in2(sv[i * (D / 2)], tq);
-                float2 qq = OUT ? in2(sq[i * (D / 2)], tq) : make_float2(0.f, 0.f);
-                if (!valid) kk = vv = qq = make_float2(0.f, 0.f);
-                const float bi = sBeta[i];
-                const float2 b2 = make_float2(bi, bi);
-                const float2 x = __fadd2_rn(bl[r], xo);
-                const float2 ep = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                const float2 em = make_float2(ex2_approx(-x.x), ex2_approx(-x.y));
-                const float2 kp = __fmul2_rn(__fmul2_rn(kk, b2), ep);   // beta K+
-                const float2 km = __fmul2_rn(kk, em);                   // K-
-                const float2 vb = __fmul2_rn(vv, b2);                   // beta V
-                const float2 qp = __fmul2_rn(qq, ep);                   // Q+
-                if (r & 1) {
-                    const int m = r >> 1;
-                    pk[0][m] = pack_f16x2(lk.x, kp.x); pk[1][m] = pack_f16x2(lk.y, kp.y);
-                    pm[0][m] = pack_f16x2(lm.x, km.x); pm[1][m] = pack_f16x2(lm.y, km.y);
-                    pv[0][m] = pack_f16x2(lv.x, vb.x); pv[1][m] = pack_f16x2(lv.y, vb.y);
-                    pq[0][m] = pack_f16x2(lq.x, qp.x); pq[1][m] = pack_f16x2(lq.y, qp.y);
-                } else {
-                    lk = kp; lm = km; lv = vb; lq = qp;
+                    for (int r8 = 0; r8 < 8; ++r8) {
+                        const int r = 8 * half + r8, i = 16 * rq + r;
+                        run = __ffma2_rn(in2(gR[r], (const __nv_bfloat16*)nullptr), l2e, run);
+                        const float2 kk = in2(kR[r], tq);
+                        const float bi = sBetaP[i];
+                        const float2 ep = make_float2(ex2_approx(run.x), ex2_approx(run.y));
+                        const float2 em = make_float2(ex2_approx(-run.x), ex2_approx(-run.y));
+                        const float2 kp = __fmul2_rn(__fmul2_rn(kk, make_float2(bi, bi)), ep);   // beta K+
+                        const float2 km = __fmul2_rn(kk, em);                                   // K-
+                        const float2 qp = OUT ? __fmul2_rn(in2(qR[r], tq), ep) : make_float2(0.f, 0.f);   // Q+
+                        if (r8 & 1) {
+                            const int m = r8 >> 1;
+                            pk[0][m] = pack_f16x2(lk.x, kp.x); pk[1][m] = pack_f16x2(lk.y, kp.y);
+                            pm[0][m] = pack_f16x2(lm.x, km.x); pm[1][m] = pack_f16x2(lm.y, km.y);
+                            pq[0][m] = pack_f16x2(lq.x, qp.x); pq[1][m] = pack_f16x2(lq.y, qp.y);
+                        } else {
+                            lk = kp; lm = km; lq = qp;
+                        }
+                    }
+                    const int ig = 2 * rq + half;
+                    st_pair(set + PL::KP, ig, cp, pk);
+                    st_pair(set + PL::KM, ig, cp, pm);
+                    if (OUT) st_pair(set + PL::QP, ig, cp, pq);
                 }
             }
-            // Threads with (cp & 4) store their odd channel first: each 8-thread phase of a
-            // 16-byte store then covers all 32 banks once.
-            const bool sw = (cp & 4) != 0;
-            const int c_first = 2 * cp + (sw ? 1 : 0), c_second = 2 * cp + (sw ? 0 : 1);
-            const uint32_t o1 = rb * 2048 + (c_first >> 3) * 128 + (c_first & 7) * 16;
-            const uint32_t o2 = rb * 2048 + (c_second >> 3) * 128 + (c_second & 7) * 16;
-            auto st2 = [&](int tile, const uint32_t (&pp)[2][4]) {
-                const uint4 a0 = make_uint4(pp[0][0], pp[0][1], pp[0][2], pp[0][3]);
-                const uint4 a1 = make_uint4(pp[1][0], pp[1][1], pp[1][2], pp[1][3]);
-                *reinterpret_cast<uint4*>(sm + tile + o1) = sw ? a1 : a0;
-                *reinterpret_cast<uint4*>(sm + tile + o2) = sw ? a0 : a1;
-            };
-            st2(PL::KP, pk);
-            st2(PL::KM, pm);
-            st2(PL::VB, pv);
-            if (OUT) st2(PL::QP, pq);
-        }
-        fence_async_smem();
-        __syncthreads();
-        // ---- 2. A (and P) on the tensor core ----------------------------------------------
-        if (t == 0) {
-            tc_fence_after();
-            // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
-            const uint32_t id = idesc_f16(OUT ? 128 : 64, 64, true, true);
-            for (int kk = 0; kk < 8; ++kk)
-                umma_f16(tmem + T_AP, sdesc(sbase + PL::KP + 256 * kk, 128, 2048),
-                         sdesc(sbase + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
-            umma_commit(ctl.mma_bar);
-        }
-        tma_in_flight = n + 1 < n1;
-        mma_in_flight = true;
-        if (!grpY) {
-            // ---- 3X. warps 0-7: A -> fp16 tile, then T = (I + A)^{-1} ---------------------------
-            // A = diag(beta) strict_lower(K+ K-^T) (beta is already in K+).
-            wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == 0, 1);
-            const uint32_t Ah = sbase + PL::U;       // A, fp16 K-major core-matrix tile
-            const uint32_t Tt = sbase + TT;          // T: the next MMA's operand
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(1, NG);
+            if (tg == 0) mbar_arrive(&bars[B_PRO + bs]);     // tiles, r and b_C ready
+            // ---- A (and P) on the tensor core -------------------------------------------
+            if (tg == 0) {
+                // MODE_STATE: A's TMEM columns are the consumer's U until it has read U
+                if (MODE == MODE_STATE && kc >= 1) thread_wait(&bars[B_UREAD], (kc - 1) & 1, ab);
+                tc_fence_after();
+                // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
+                const uint32_t id = idesc_f16(OUT ? 128 : 64, 64, true, true);
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_f16(tmem + T_AP, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
+                             sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
+                umma_commit(&bars[B_AP]);
+            }
+            group_wait(&bars[B_AP], kc & 1, ab, tg == 0, 1);
+            // ---- A -> fp16 tile (and P -> the T region's other halves) ------------------
+            const uint32_t Ah = sbase + PL::AT;          // A, fp16 K-major core-matrix tile
+            const uint32_t Tt = sset + PL::TF;           // T: the consumer's operand
             {
                 float v[32];
+                tmem_ld32(tl + T_AP + 32 * hg, v);
                 int i = -1;
+                bool isP = false;
                 if (OUT) {
-                    // M = 128 layout: row i in lane i; rows 0-63 (quarters 0, 1) are A
-                    if (q4 < 2) {
-                        tmem_ld32(tl + T_AP + 32 * hg, v);
-                        i = 32 * q4 + lane;
-                    }
-                } else {
-                    // M = 64 layout: row 16*q4 + l in lane 32*q4 + l (l < 16)
-                    tmem_ld32(tl + T_AP + 32 * hg, v);
-                    if (lane < 16) i = 16 * q4 + lane;
+                    // M = 128 layout: row i in lane i; rows 0-63 are A, rows 64-127 are P
+                    i = 32 * (q4 & 1) + lane;
+                    isP = q4 >= 2;
+                } else if (lane < 16) {
+                    i = 16 * q4 + lane;                  // M = 64 layout
                 }
                 if (i >= 0) {
 #pragma unroll
@@ -483,23 +488,25 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
                             const int col = 32 * hg + 8 * g8 + j;
-                            f[j] = (col < i) ? v[8 * g8 + j] : 0.f;
+                            f[j] = (isP ? (col <= i) : (col < i)) ? v[8 * g8 + j] : 0.f;
                         }
-                        *reinterpret_cast<uint4*>(sm + PL::U + cm64(i, 32 * hg + 8 * g8)) = pack8_f16(f);
+                        uint8_t* dst = isP ? set + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)
+                                           : sm + PL::AT + cm64(i, 32 * hg + 8 * g8);
+                        *reinterpret_cast<uint4*>(dst) = pack8_f16(f);
                     }
                 }
                 // the six upper 16x16 blocks of T are zero
-                if (t < 192) {
-                    const int e = t >> 5, u = t & 31;
+                if (tg < 192) {
+                    const int e = tg >> 5, u = tg & 31;
                     const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
                     const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
                     const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
-                    *reinterpret_cast<uint4*>(sm + TT + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(set + PL::TF + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             tc_fence_before();
-            named_sync(1, NT / 2);
-            if (MODE == MODE_STATE && t == 0) mbar_arrive(a_bar);   // Y may now overwrite A's columns
+            named_sync(1, NG);
+            if (MODE == MODE_STATE && tg == 0) mbar_arrive(&bars[B_AFREE]);   // Y may overwrite A
             // diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
             // N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs
             if (w < 4) {
@@ -593,187 +600,260 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 named_sync(1, NT / 2);
             }
             fence_async_smem();
-        } else {
-            // ---- 3Y. warps 8-15: previous output; S^; Y (and O) = [beta K+ (; Q+)] S^; P; Y --
-            if (OUT && prev_t0 >= 0 && q4 >= 2)
-                store_o(tl, q4, 64 * hg, 2, lane, o, o_f32, b, T, H, h, prev_t0);
+            named_sync(1, NG);
+            if (tg == 0) mbar_arrive(&bars[B_INV + bs]);    // T (and P) ready
+        }
+        // after a timeout some requested g tile may not have been waited for: let it land
+        if (tg == 0 && *sAbort && g_issued > 0) mbar_wait_bounded(&bars[B_TG], (g_issued - 1) & 1, kWaitNs);
+    } else {
+        // ================= consumer: the state chain of chunk n0 + kc =====================
+        const TQ* tq = nullptr;
+        // initial state in TMEM: warp (q4, hg) holds lanes 32*q4.. and columns hg*NS/2 ..
+        {
+            const int col0 = hg * (NS / 2);
+            for (int cc = 0; cc < NS / 2; cc += 32) {
+                float vv[32];
+                if (MODE == MODE_STATE) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) vv[j] = (col0 + cc + j == D + c) ? 1.f : 0.f;
+                } else if (S_in) {
+                    const size_t idx = s_in_per_segment ? (size_t)bh * P + p : (size_t)bh;
+                    const float4* s4 = reinterpret_cast<const float4*>(S_in + (idx * D + c) * D + col0 + cc);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 x = s4[j];
+                        vv[4 * j] = x.x; vv[4 * j + 1] = x.y; vv[4 * j + 2] = x.z; vv[4 * j + 3] = x.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) vv[j] = 0.f;
+                }
+                tmem_st32(tl + TM_S + col0 + cc, vv);
+            }
+        }
+        uint32_t betaR = 0;
+        int v_issued = 0, qk_last[2] = {-1, -1};   // thread NG: TMA requests so far
+        if (tg == 0 && nk > 0) {
+            tma_v(n0);
+            v_issued = 1;
+            tma_qk(n0);
+            qk_last[0] = 0;
+            if (nk > 1) {
+                tma_qk(n0 + 1);
+                qk_last[1] = 1;
+            }
+        }
+        if (tg < C) betaR = load_beta(beta, b, T, H, h, n0 * C, tg, nk > 0);
+        // the master holds diag(2^{-carry}) S for channel c (log2 units; 0 before any chunk)
+        float carry = 0.f;
+        const bool poller = tg == 0;
+        for (int kc = 0; kc < nk; ++kc) {
+            const int n = n0 + kc, t0 = n * C, bs = kc & 1;
+            const uint32_t sset = sbase + bs * PL::SET;
+            group_wait(&bars[B_PRO + bs], (kc >> 1) & 1, ab, poller, 2);
+            // ---- previous chunk's output (staged in the free U and Y regions) -----------
+            if (OUT && kc > 0) {
+                stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
+                named_sync(2, NG);
+                flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, t0 - C);
+                named_sync(2, NG);
+            }
+            // ---- S^ = 2^{r + carry} master ------------------------------------------------
             {
-                // master (scaled form) -> S^ = 2^{r + carry} master: fp16 operand tile and the
-                // fp32 master both take the new scale
+                const float2 rb = sRB[bs * D + c];
+                const float s_scale = ex2_approx(rb.x + carry);
+                carry = rb.y - rb.x;
                 const int col0 = hg * (NS / 2);
                 for (int cc = 0; cc < NS / 2; cc += 32) {
-                    float v[32];
-                    tmem_ld32(tl + TM_S + col0 + cc, v);
+                    float vv[32];
+                    tmem_ld32(tl + TM_S + col0 + cc, vv);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] *= s_scale;
+                    for (int j = 0; j < 32; ++j) vv[j] *= s_scale;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
                         const int col = col0 + cc + g8 * 8;
                         *reinterpret_cast<uint4*>(sm + PL::S + (col >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
-                            pack8_f16(&v[8 * g8]);
+                            pack8_f16(&vv[8 * g8]);
                     }
-                    tmem_st32(tl + TM_S + col0 + cc, v);
+                    tmem_st32(tl + TM_S + col0 + cc, vv);
                 }
             }
+            if (tg < C) sBetaC[tg] = __uint_as_float(betaR << 16);
             fence_async_smem();
             tc_fence_before();
-            if (OUT) {
-                named_sync(2, NT / 2);
-            } else {
-                // Y's TMEM columns hold A until warps 0-7 have read it
-                wait_bar(a_bar, a_phase, ctl, t == NT / 2, 2);
-            }
-            if (t == NT / 2) {
+            named_sync(2, NG);
+            if (poller) {
+                // MODE_STATE: Y's TMEM columns hold A until the producer has read it
+                if (MODE == MODE_STATE) thread_wait(&bars[B_AFREE], kc & 1, ab);
                 tc_fence_after();
                 // OUT:   [Y; O] = [beta K+; Q+] S^   (M = 128, N = 128)
                 // STATE: Y = beta K+ [S^ | Phi^]     (M = 64,  N = 256)
                 const uint32_t idy = idesc_f16(OUT ? 128 : 64, NS, true, true);
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_Y, sdesc(sbase + PL::KP + 256 * kk, 128, 2048),
+                    umma_f16(tmem + T_Y, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
                              sdesc(sbase + PL::S + 256 * kk, 128, 2048), idy, kk > 0);
-                umma_commit(y_bar);
-                // the next chunk's q, k, v, g land while the inverse runs (the staging
-                // buffer was last read by this chunk's prologue)
-                if (n + 1 < n1) issue_tma(n + 1);
+                umma_commit(&bars[B_Y]);
             }
-            y_in_flight = true;
-            if (OUT) {
-                wait_bar(ctl.mma_bar, ctl.mma_phase, ctl, t == NT / 2, 2);
-                if (q4 >= 2) {
-                    // P rows: lanes 64-127 of the M = 128 accumulator; P goes to the free 1 KB
-                    // halves of the T region, so that [T; P] reads as one M = 128 operand
-                    float v[32];
-                    tmem_ld32(tl + T_AP + 32 * hg, v);
-                    const int i = 32 * (q4 - 2) + lane;
+            // ---- beta V while Y runs: v (landed in the beta V tile) converted in place ---------
+            group_wait(&bars[B_TV], kc & 1, ab, poller, 2);
+            {
+                uint32_t vR[16];
+                ld_rows16(vR, sm + PL::VB, 16 * rq, cp);
+                if (t0 + C > T) {
 #pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        float f[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int col = 32 * hg + 8 * g8 + j;
-                            f[j] = (col <= i) ? v[8 * g8 + j] : 0.f;
-                        }
-                        *reinterpret_cast<uint4*>(sm + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)) = pack8_f16(f);
-                    }
+                    for (int r = 0; r < 16; ++r)
+                        if (t0 + 16 * rq + r >= T) vR[r] = 0u;
                 }
-            } else {
-                ctl.mma_phase ^= 1;   // A's phase: complete, since warps 0-7 have read A
+                named_sync(2, NG);
+                uint32_t pv[2][4];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float2 lv = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r8 = 0; r8 < 8; ++r8) {
+                        const int r = 8 * half + r8;
+                        const float bi = sBetaC[16 * rq + r];
+                        const float2 vb = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
+                        if (r8 & 1) {
+                            pv[0][r8 >> 1] = pack_f16x2(lv.x, vb.x);
+                            pv[1][r8 >> 1] = pack_f16x2(lv.y, vb.y);
+                        } else {
+                            lv = vb;
+                        }
+                    }
+                    st_pair(sm + PL::VB, 2 * rq + half, cp, pv);
+                }
             }
-            wait_bar(y_bar, y_phase, ctl, t == NT / 2, 2);
-            y_in_flight = false;
-            // Y -> fp16 position-major tile in the S^ region (S^ is no longer needed)
+            if (tg < C) betaR = load_beta(beta, b, T, H, h, (n + 1) * C, tg, n + 1 < n1);
+            group_wait(&bars[B_Y], kc & 1, ab, poller, 2);
+            // [Y; O] has read this set's Q+ / beta K+ slots: chunk n+2's q, k may land there
+            if (poller && n + 2 < n1 && !*sAbort) {
+                tma_qk(n + 2);
+                qk_last[bs] = kc + 2;
+            }
+            // ---- Y -> fp16 position-major tile in the S^ region --------------------------
             if (OUT) {
                 if (q4 < 2) {
                     const int j = 32 * q4 + lane;    // M = 128 layout: row j in lane j
                     for (int cc = 0; cc < 64; cc += 32) {
-                        float v[32];
-                        tmem_ld32(tl + T_Y + 64 * hg + cc, v);
+                        float vv[32];
+                        tmem_ld32(tl + T_Y + 64 * hg + cc, vv);
 #pragma unroll
                         for (int g8 = 0; g8 < 4; ++g8) {
                             const int cg = (64 * hg + cc) / 8 + g8;
                             *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
-                                pack8_f16(&v[8 * g8]);
+                                pack8_f16(&vv[8 * g8]);
                         }
                     }
                 }
             } else {
                 const int j = 16 * q4 + lane;        // M = 64 layout: lanes 0-15 of each quarter
                 for (int cc = 0; cc < 128; cc += 32) {
-                    float v[32];
-                    tmem_ld32(tl + T_Y + 128 * hg + cc, v);
+                    float vv[32];
+                    tmem_ld32(tl + T_Y + 128 * hg + cc, vv);
                     if (lane < 16) {
 #pragma unroll
                         for (int g8 = 0; g8 < 4; ++g8) {
                             const int cg = (128 * hg + cc) / 8 + g8;
                             *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
-                                pack8_f16(&v[8 * g8]);
+                                pack8_f16(&vv[8 * g8]);
                         }
                     }
                 }
             }
             fence_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (*sAbort) break;
-        // ---- 4. U = T (beta V) - T Y  (value columns; identity columns: -T Y) -------------
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t idv = idesc_f16(64, 128, false, false);
-            const uint32_t idy = idesc_f16(64, NS, false, true, true);
-            if (OUT) {
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
-                             sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
-                             sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, 1);
-            } else {
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
-                             sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, kk > 0);
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_UU, sdesc(sbase + TT + 2 * T_LBO * kk, T_LBO, 128),
-                             sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, 1);
+            tc_fence_before();
+            named_sync(2, NG);
+            // ---- U = T (beta V) - T Y  (value columns; identity columns: -T Y) -------------
+            if (poller) {
+                thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
+                tc_fence_after();
+                const uint32_t idv = idesc_f16(64, 128, false, false);
+                const uint32_t idy = idesc_f16(64, NS, false, true, true);
+                const uint32_t Tb = sset + PL::TF;
+                if (OUT) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
+                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
+                                 sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, 1);
+                } else {
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
+                                 sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
+                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, 1);
+                }
+                umma_commit(&bars[B_U]);
             }
-            umma_commit(ctl.mma_bar);
-        }
-        wait_mma(ctl, t);
-        // U -> fp16 MN-major tile [i][col] at U (M = 64 layout: row 16*q4 + l in lane 32*q4 + l)
-        {
-            for (int cc = 0; cc < NQ; cc += 32) {
-                const int col = cq * NQ + cc;            // U tile column
-                float v[32];
-                tmem_ld32(tl + T_UU + col, v);
+            group_wait(&bars[B_U], kc & 1, ab, poller, 2);
+            // the U MMA has read beta V: chunk n+1's v may land in its tile
+            if (poller && n + 1 < n1 && !*sAbort) {
+                tma_v(n + 1);
+                v_issued = kc + 2;
+            }
+            // U -> fp16 MN-major tile [i][col] at U (M = 64 layout: row 16*q4 + l in lane 32*q4 + l)
+            for (int cc = 0; cc < NS / 2; cc += 32) {
+                const int col = hg * (NS / 2) + cc;
+                float vv[32];
+                tmem_ld32(tl + T_UU + col, vv);
                 if (lane < 16) {
                     const int i = 16 * q4 + lane;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
                         const int cg = col / 8 + g8;
                         *reinterpret_cast<uint4*>(sm + PL::U + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                            pack8_f16(&v[8 * g8]);
+                            pack8_f16(&vv[8 * g8]);
                     }
                 }
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // ---- 5. master += K-^T U  (and O += P U) ------------------------------------------
-        if (t == 0) {
-            tc_fence_after();
-            const uint32_t ids = idesc_f16(128, NS, false, true);
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16(tmem + TM_S, sdesc(sbase + PL::KM + 4096 * kk, 2048, 128),
-                         sdesc(sbase + PL::U + 256 * kk, 128, 1024), ids, 1);
-            if (OUT) {
-                // O += P U as rows 64-127 of an M = 128 MMA whose rows 0-63 read T (their
-                // result lands on Y's rows, already consumed)
-                const uint32_t ido = idesc_f16(128, 128, false, true);
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(2, NG);
+            // ---- master += K-^T U  (and O += P U) ------------------------------------------
+            if (poller) {
+                if (MODE == MODE_STATE) mbar_arrive(&bars[B_UREAD]);   // A may take U's columns
+                tc_fence_after();
+                const uint32_t ids = idesc_f16(128, NS, false, true);
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + T_Y, sdesc(sbase + PL::TF + 4096 * kk, 2048, 128),
-                             sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
+                    umma_f16(tmem + TM_S, sdesc(sset + PL::KM + 4096 * kk, 2048, 128),
+                             sdesc(sbase + PL::U + 256 * kk, 128, 1024), ids, 1);
+                if (OUT) {
+                    // O += P U as rows 64-127 of an M = 128 MMA whose rows 0-63 read T (their
+                    // result lands on Y's rows, already consumed)
+                    const uint32_t ido = idesc_f16(128, 128, false, true);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_Y, sdesc(sset + PL::TF + 4096 * kk, 2048, 128),
+                                 sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
+                }
+                umma_commit(&bars[B_S]);
+                umma_commit(&bars[B_EMPTY + bs]);   // buffer set bs may be refilled
             }
-            umma_commit(ctl.mma_bar);
+            group_wait(&bars[B_S], kc & 1, ab, poller, 2);
         }
-        wait_mma(ctl, t);
-        mma_in_flight = false;
-        prev_t0 = t0;
-    }
-    if (OUT && !*sAbort && prev_t0 >= 0 && q4 >= 2)
-        store_o(tl, q4, 32 * cq, 1, lane, o, o_f32, b, T, H, h, prev_t0);
-
-    // ---- end of segment: write the state S = diag(2^{carry}) master ---------------------
-    if (!*sAbort) {
+        if (OUT && nk > 0) {
+            stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
+            named_sync(2, NG);
+            flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, (n1 - 1) * C);
+        }
+        // after a timeout some requested tiles may not have been waited for: let them land
+        if (tg == 0 && *sAbort) {
+            if (v_issued > 0) mbar_wait_bounded(&bars[B_TV], (v_issued - 1) & 1, kWaitNs);
+            for (int s2 = 0; s2 < 2; ++s2)
+                if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
+        }
+        // ---- end of segment: write the state S = diag(2^{carry}) master -----------------
         float* dst = nullptr;
         if (MODE == MODE_STATE) dst = maps + (size_t)(bh * (P - 1) + p) * 2 * D * D;  // [N | M]
         else if (S_T && p == P - 1) dst = S_T + (size_t)bh * D * D;
-        if (dst) {
+        if (dst && !*sAbort) {
             const float sc = ex2_approx(carry);
-            const int col0 = cq * NQ;
-            for (int cc = 0; cc < NQ; cc += 32) {
-                float v[32];
-                tmem_ld32(tl + TM_S + col0 + cc, v);
+            const int col0 = hg * (NS / 2);
+            for (int cc = 0; cc < NS / 2; cc += 32) {
+                float vv[32];
+                tmem_ld32(tl + TM_S + col0 + cc, vv);
                 // maps: N block (value columns) then M block (identity columns); a 32-column
                 // run never straddles the two
                 const int col = col0 + cc;
@@ -781,15 +861,15 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 float4* d4 = reinterpret_cast<float4*>(dst + idx);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    d4[j] = make_float4(v[4 * j] * sc, v[4 * j + 1] * sc, v[4 * j + 2] * sc, v[4 * j + 3] * sc);
+                    d4[j] = make_float4(vv[4 * j] * sc, vv[4 * j + 1] * sc, vv[4 * j + 2] * sc, vv[4 * j + 3] * sc);
             }
         }
     }
-    // ---- teardown: drain what is in flight, free TMEM ---------------------------------
-    if (*sAbort) {
-        if (mma_in_flight) mbar_wait_bounded(ctl.mma_bar, ctl.mma_phase, kWaitNs);
-        if (tma_in_flight) mbar_wait_bounded(ctl.tma_bar, ctl.tma_phase, kWaitNs);
-        if (y_in_flight && t == NT / 2) mbar_wait_bounded(y_bar, y_phase, kWaitNs);
+    // ---- teardown: after a timeout, each MMA issuer drains its own MMAs; free TMEM --------
+    if (*sAbort && (t == 0 || t == NG)) {
+        uint64_t* dr = &bars[t == 0 ? B_DRAIN : B_DRAIN2];
+        umma_commit(dr);
+        mbar_wait_bounded(dr, 0, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
@@ -901,6 +981,10 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+struct Maps {
+    CUtensorMap q, k, v, g;
+};
+
 struct Split {
     int P, L;
 };
@@ -915,9 +999,8 @@ Split split_for(int B, int T, int H, int num_sms)
 }
 
 template <int MODE, typename TQ>
-cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        const CUtensorMap& mg, const KdaArgs& a, const float* S_in, int per_seg,
-                        float* maps, int P, int L, int* status, cudaStream_t s)
+cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int per_seg, float* maps, int P, int L,
+                        int* status, cudaStream_t s)
 {
     auto kern = kda_tc_kernel<MODE, TQ>;
     const int smem = smem_bytes<MODE>();
@@ -927,7 +1010,7 @@ cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     const unsigned grid = (unsigned)(a.B * a.H * nseg);
     ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mq, mk, mv, mg, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status);
     return cudaGetLastError();
 }
@@ -941,16 +1024,15 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
     const Split sp = split_for(a.B, a.T, a.H, sms);
     const CUtensorMapDataType dq =
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    CUtensorMap mq, mk, mv, mg;
-    if (!make_map(&mq, a.q, dq, a.B, a.T, a.H) || !make_map(&mk, a.k, dq, a.B, a.T, a.H) ||
-        !make_map(&mv, a.v, dq, a.B, a.T, a.H) ||
-        !make_map(&mg, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
+    Maps mp;
+    if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    if (sp.P == 1)
-        return launch_pass<MODE_OUTPUT, TQ>(mq, mk, mv, mg, a, a.S0, 0, nullptr, 1, sp.L, status, s);
+    if (sp.P == 1) return launch_pass<MODE_OUTPUT, TQ>(mp, a, a.S0, 0, nullptr, 1, sp.L, status, s);
     float* maps = reinterpret_cast<float*>(ws);
     float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
-    cudaError_t e = launch_pass<MODE_STATE, TQ>(mq, mk, mv, mg, a, nullptr, 0, maps, sp.P, sp.L, status, s);
+    cudaError_t e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, sp.P, sp.L, status, s);
     if (e != cudaSuccess) return e;
     {
         e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb_smem_bytes());
@@ -961,7 +1043,7 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    return launch_pass<MODE_OUTPUT, TQ>(mq, mk, mv, mg, a, starts, 1, maps, sp.P, sp.L, status, s);
+    return launch_pass<MODE_OUTPUT, TQ>(mp, a, starts, 1, maps, sp.P, sp.L, status, s);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
