@@ -208,6 +208,18 @@ kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv
 /* Number of kernels this library has launched in this process (all devices). */
 uint64_t kda_kernel_launches(void);
 
+/* Test hook for the device-side failure path (the pages have no counterpart; this is
+ * how the timeout handling is exercised without a fault or a hang).  While `on` is
+ * non-zero, every later launch of the tensor-core scan withholds, in each CTA, the
+ * first "tiles ready" signal from its producer warps to its consumer warps.  The
+ * consumer's bounded wait (2 s) then runs out: the CTA records the timeout in the device
+ * status word, stops waiting, drains its own tensor-core and TMA work, frees its tensor
+ * memory and exits.  The call still returns KDA_OK (errors on the device are reported
+ * asynchronously); o and S_T are undefined; kda_last_device_error() then returns
+ * KDA_ERR_TIMEOUT, and later calls with the hook off run normally.  Off by default;
+ * process-wide; not for production use. */
+void kda_debug_drop_handoff(int on);
+
 /* When `on` is non-zero, every later call records a pair of CUDA events on its
  * stream around each of its kernels, keyed by kernel name.  Off by default. */
 void kda_profile_enable(int on);

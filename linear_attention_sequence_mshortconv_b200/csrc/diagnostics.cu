@@ -11,11 +11,13 @@ namespace kda {
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_profile{0};
+std::atomic<int> g_drop_handoff{0};
 std::mutex g_mu;
 std::map<std::string, std::vector<std::pair<cudaEvent_t, cudaEvent_t>>> g_events;
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+int debug_drop_handoff() { return g_drop_handoff.load(std::memory_order_relaxed); }
 
 ProfileScope::ProfileScope(const char* name, cudaStream_t s) : name_(name), s_(s)
 {
@@ -38,6 +40,8 @@ ProfileScope::~ProfileScope()
 }  // namespace kda
 
 extern "C" {
+
+void kda_debug_drop_handoff(int on) { kda::g_drop_handoff.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 uint64_t kda_kernel_launches(void) { return kda::g_launches.load(); }
 

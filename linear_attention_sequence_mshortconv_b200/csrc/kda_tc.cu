@@ -296,7 +296,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
               const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
-              float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status)
+              float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop)
 {
     using PL = Plan<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
@@ -452,7 +452,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             fence_async_smem();
             tc_fence_before();
             named_sync(1, NG);
-            if (tg == 0) mbar_arrive(&bars[B_PRO + bs]);     // tiles, r and b_C ready
+            // tiles, r and b_C ready (the test hook withholds chunk 0's signal)
+            if (tg == 0 && !(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + bs]);
             // ---- A (and P) on the tensor core -------------------------------------------
             if (tg == 0) {
                 // MODE_STATE: A's TMEM columns are the consumer's U until it has read U
@@ -1011,7 +1012,7 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
     count_launch();
     kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
-                                S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status);
+                                S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff());
     return cudaGetLastError();
 }
 
