@@ -247,6 +247,29 @@ __device__ __forceinline__ void stage_o(uint32_t tl, int q4, int hg, int lane, u
         }
     }
 }
+// bf16 output through TMA: O rows go into two 64-channel x 64-row tiles (128-byte
+// rows, 128-byte swizzle: 16-byte chunk j of row i at i*128 + ((j ^ (i & 7)) * 16), so
+// the 8 rows of a store phase hit 8 different bank groups); one thread then stores
+// both tiles with the TMA (rows past the end of the sequence are clipped).
+__device__ __forceinline__ void stage_o_swz(uint32_t tl, int q4, int hg, int lane, uint8_t* tiles)
+{
+    if (q4 < 2) return;
+    const int i = 32 * (q4 - 2) + lane;
+    uint8_t* tile = tiles + hg * 8192;
+    for (int u = 0; u < 2; ++u) {
+        float v[32];
+        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint4 uu;
+            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
+            const int chunk = 4 * u + j;
+            *reinterpret_cast<uint4*>(tile + i * 128 + ((chunk ^ (i & 7)) * 16)) = uu;
+        }
+    }
+}
 __device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int b, int T, int H, int h,
                                         int t0)
 {
@@ -294,7 +317,7 @@ template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-              const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
+              const __grid_constant__ CUtensorMap tm_o, const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop)
 {
@@ -633,8 +656,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         uint32_t betaR = 0;
-        int v_issued = 0, qk_last[2] = {-1, -1};   // thread NG: TMA requests so far
-        if (tg == 0 && nk > 0) {
+        // thread NG + 32 (not the MMA issuer) requests the consumer-side TMA loads, just
+        // before a barrier at which the group waits for an MMA anyway
+        const bool loader = tg == 32;
+        int v_issued = 0, qk_last[2] = {-1, -1};   // its TMA requests so far
+        bool o_pending = false;                    // poller: a bf16 output store is in flight
+        if (loader && nk > 0) {
             tma_v(n0);
             v_issued = 1;
             tma_qk(n0);
@@ -652,12 +679,24 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int n = n0 + kc, t0 = n * C, bs = kc & 1;
             const uint32_t sset = sbase + bs * PL::SET;
             group_wait(&bars[B_PRO + bs], (kc >> 1) & 1, ab, poller, 2);
-            // ---- previous chunk's output (staged in the free U and Y regions) -----------
+            // ---- previous chunk's output (staged in the free U (and Y) regions) ---------
             if (OUT && kc > 0) {
-                stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
-                named_sync(2, NG);
-                flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, t0 - C);
-                named_sync(2, NG);
+                if (o_f32) {
+                    stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
+                    named_sync(2, NG);
+                    flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, t0 - C);
+                    named_sync(2, NG);
+                } else {
+                    stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                    fence_async_smem();
+                    named_sync(2, NG);
+                    if (poller) {
+                        tma_store_4d(&tm_o, sm + PL::U, 0, h, t0 - C, b);
+                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, t0 - C, b);
+                        bulk_commit();
+                        o_pending = true;
+                    }
+                }
             }
             // ---- S^ = 2^{r + carry} master ------------------------------------------------
             {
@@ -726,12 +765,21 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             if (tg < C) betaR = load_beta(beta, b, T, H, h, (n + 1) * C, tg, n + 1 < n1);
-            group_wait(&bars[B_Y], kc & 1, ab, poller, 2);
-            // [Y; O] has read this set's Q+ / beta K+ slots: chunk n+2's q, k may land there
-            if (poller && n + 2 < n1 && !*sAbort) {
-                tma_qk(n + 2);
-                qk_last[bs] = kc + 2;
+            if (OUT) {
+                // U = T (beta V) - T Y: the first half needs no Y, so it queues behind [Y; O]
+                fence_async_smem();
+                named_sync(2, NG);
+                if (poller) {
+                    thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
+                    tc_fence_after();
+                    const uint32_t idv = idesc_f16(64, 128, false, false);
+                    const uint32_t Tb = sset + PL::TF;
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
+                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
+                }
             }
+            group_wait(&bars[B_Y], kc & 1, ab, poller, 2);
             // ---- Y -> fp16 position-major tile in the S^ region --------------------------
             if (OUT) {
                 if (q4 < 2) {
@@ -767,15 +815,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             named_sync(2, NG);
             // ---- U = T (beta V) - T Y  (value columns; identity columns: -T Y) -------------
             if (poller) {
-                thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
+                if (!OUT) thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
                 tc_fence_after();
                 const uint32_t idv = idesc_f16(64, 128, false, false);
                 const uint32_t idy = idesc_f16(64, NS, false, true, true);
                 const uint32_t Tb = sset + PL::TF;
                 if (OUT) {
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
-                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
                                  sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, 1);
@@ -789,12 +834,18 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 umma_commit(&bars[B_U]);
             }
-            group_wait(&bars[B_U], kc & 1, ab, poller, 2);
-            // the U MMA has read beta V: chunk n+1's v may land in its tile
-            if (poller && n + 1 < n1 && !*sAbort) {
-                tma_v(n + 1);
-                v_issued = kc + 2;
+            // [Y; O] of this chunk is done: chunk n+2's q, k may land in this set's
+            // Q+ / beta K+ slots
+            if (loader && n + 2 < n1 && !*sAbort) {
+                tma_qk(n + 2);
+                qk_last[bs] = kc + 2;
             }
+            // the output store must have read the U region before U is written there
+            if (poller && o_pending) {
+                bulk_wait_read0();
+                o_pending = false;
+            }
+            group_wait(&bars[B_U], kc & 1, ab, poller, 2);
             // U -> fp16 MN-major tile [i][col] at U (M = 64 layout: row 16*q4 + l in lane 32*q4 + l)
             for (int cc = 0; cc < NS / 2; cc += 32) {
                 const int col = hg * (NS / 2) + cc;
@@ -832,15 +883,32 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 umma_commit(&bars[B_S]);
                 umma_commit(&bars[B_EMPTY + bs]);   // buffer set bs may be refilled
             }
+            // the U MMA has read beta V: chunk n+1's v may land in its tile
+            if (loader && n + 1 < n1 && !*sAbort) {
+                tma_v(n + 1);
+                v_issued = kc + 2;
+            }
             group_wait(&bars[B_S], kc & 1, ab, poller, 2);
         }
         if (OUT && nk > 0) {
-            stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
-            named_sync(2, NG);
-            flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, (n1 - 1) * C);
+            if (o_f32) {
+                stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
+                named_sync(2, NG);
+                flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, (n1 - 1) * C);
+            } else {
+                stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                fence_async_smem();
+                named_sync(2, NG);
+                if (poller) {
+                    tma_store_4d(&tm_o, sm + PL::U, 0, h, (n1 - 1) * C, b);
+                    tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (n1 - 1) * C, b);
+                    bulk_commit();
+                }
+            }
         }
+        if (poller) bulk_wait0();   // every output store has landed before the CTA exits
         // after a timeout some requested tiles may not have been waited for: let them land
-        if (tg == 0 && *sAbort) {
+        if (loader && *sAbort) {
             if (v_issued > 0) mbar_wait_bounded(&bars[B_TV], (v_issued - 1) & 1, kWaitNs);
             for (int s2 = 0; s2 < 2; ++s2)
                 if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
@@ -982,8 +1050,24 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output o [B, T, H, 128] as a 4-D tensor (channels, heads, tokens, batch), box =
+// 64 channels x 1 head x 64 tokens, 128-byte swizzle.  Tokens past T are clipped by the
+// T dimension, so a ragged last chunk never writes into the next batch row.
+bool make_map_o(CUtensorMap* m, void* base, int B, int T, int H)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)C, 1u};
+    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Maps {
-    CUtensorMap q, k, v, g;
+    CUtensorMap q, k, v, g, o;   // o: only for a bf16 output (else a copy of q, unused)
 };
 
 struct Split {
@@ -1011,7 +1095,7 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     const unsigned grid = (unsigned)(a.B * a.H * nseg);
     ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff());
     return cudaGetLastError();
 }
@@ -1030,6 +1114,8 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
         !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    if (a.out_t == ET_F32) mp.o = mp.q;
+    else if (!make_map_o(&mp.o, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     if (sp.P == 1) return launch_pass<MODE_OUTPUT, TQ>(mp, a, a.S0, 0, nullptr, 1, sp.L, status, s);
     float* maps = reinterpret_cast<float*>(ws);
     float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
