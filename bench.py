@@ -62,6 +62,33 @@ def algorithmic_bytes(w: W.Workload) -> int:
     return w.B * w.T * w.H * per_tok_head + state
 
 
+def conv_fmas(w: W.Workload) -> int:
+    """Multiply-adds of mShortConv per step: taps x channels x tokens, for q, k and v."""
+    taps = {0: w.Kt, 1: 9, 2: 27}
+    C = w.H * w.D
+    n = 0
+    for (mod, _start, Fr, Hh, Wd, _ws) in w.segments:
+        toks = Wd if mod == 0 else (Hh * Wd if mod == 1 else Fr * Hh * Wd)
+        n += toks * taps[mod] * C
+    return 3 * w.B * n
+
+
+_FMA_RATE = None
+
+
+def conv_alu_roofline(w: W.Workload, conv_ms: float):
+    """The conv's plain-ALU term: its multiply-adds per second against this GPU's fp32
+    FMA rate measured by the library's probe kernel."""
+    global _FMA_RATE
+    from linear_attention_sequence_mshortconv_b200 import kda
+    if _FMA_RATE is None:
+        _FMA_RATE = kda.fma_probe()
+    achieved = conv_fmas(w) / (conv_ms * 1e-3)
+    return {"bound": "alu", "achieved": achieved / 1e12, "peak": _FMA_RATE / 1e12, "unit": "TFMA/s",
+            "frac": achieved / _FMA_RATE, "peak_source": "measured (kda_fma_probe)",
+            "fmas_per_step": conv_fmas(w)}
+
+
 def traffic_record(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current source of that kernel (else None)."""
@@ -390,10 +417,21 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             st, _, _, _ = make_step(other, rank)
             for _ in range(3):
                 st()
-            m = timed(st, max(3, args.steps // 4), 1) / max(3, args.steps // 4)
-            extra.append({"workload": other.name, "ms_per_step": m,
-                          "value": other.tokens / (m * 1e-3) / 1e6, "unit": UNIT,
-                          "alg_GBps": algorithmic_bytes(other) / (m * 1e-3) / 1e9})
+            k_other = max(3, args.steps // 4)
+            kda.profile_enable(True)
+            m = timed(st, k_other, 1) / k_other
+            kda.profile_enable(False)
+            kern = {}
+            for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "conv"):
+                r = kda.profile_collect(name)
+                if r and r[1] > 0:
+                    kern[name] = {"ms_per_step": r[0] / k_other, "launches_per_step": r[1] / k_other}
+            rec = {"workload": other.name, "ms_per_step": m,
+                   "value": other.tokens / (m * 1e-3) / 1e6, "unit": UNIT,
+                   "alg_GBps": algorithmic_bytes(other) / (m * 1e-3) / 1e9, "kernels": kern}
+            if other.fused and "conv" in kern:
+                rec["conv_alu"] = conv_alu_roofline(other, kern["conv"]["ms_per_step"])
+            extra.append(rec)
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

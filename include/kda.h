@@ -220,6 +220,13 @@ uint64_t kda_kernel_launches(void);
  * process-wide; not for production use. */
 void kda_debug_drop_handoff(int on);
 
+/* Measures this GPU's fp32 fused-multiply-add rate (FMAs per second) with a synthetic
+ * kernel of independent FMA chains on every SM, timed with CUDA events on the default
+ * stream (synchronous; allocates 4 bytes).  It is the denominator of the conv's
+ * plain-ALU roofline in the benchmark; the pages have no counterpart.  Returns 0, or -1
+ * on a CUDA error. */
+int kda_fma_probe(double* fma_per_s);
+
 /* When `on` is non-zero, every later call records a pair of CUDA events on its
  * stream around each of its kernels, keyed by kernel name.  Off by default. */
 void kda_profile_enable(int on);

@@ -37,9 +37,55 @@ ProfileScope::~ProfileScope()
     g_events[name_].push_back({a_, b_});
 }
 
+// fp32 FMA throughput probe: 8 independent FMA chains per thread, enough blocks to fill
+// every SM several times; the result is stored only if it is a sentinel no input hits,
+// so the compiler cannot drop the chains.
+__global__ void __launch_bounds__(512) fma_probe_kernel(float a, float b, int iters, float* sink)
+{
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = a + i * 1e-3f + threadIdx.x * 1e-6f;
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = fmaf(x[i], b, a);
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += x[i];
+    if (s == -12345.678f) *sink = s;
+}
+
 }  // namespace kda
 
 extern "C" {
+
+int kda_fma_probe(double* fma_per_s)
+{
+    if (!fma_per_s) return -1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    float* sink = nullptr;
+    if (cudaMalloc(&sink, sizeof(float)) != cudaSuccess) return -1;
+    const int blocks = sms * 8, threads = 512, iters = 4096;
+    cudaEvent_t e0, e1;
+    cudaEventCreate(&e0);
+    cudaEventCreate(&e1);
+    kda::fma_probe_kernel<<<blocks, threads>>>(0.5f, 0.999f, iters, sink);   // warm-up
+    cudaEventRecord(e0);
+    kda::fma_probe_kernel<<<blocks, threads>>>(0.5f, 0.999f, iters, sink);
+    cudaEventRecord(e1);
+    const cudaError_t err = cudaEventSynchronize(e1);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    cudaFree(sink);
+    if (err != cudaSuccess || ms <= 0.f) return -1;
+    *fma_per_s = (double)blocks * threads * iters * 8 / (ms * 1e-3);
+    return 0;
+}
+
 
 void kda_debug_drop_handoff(int on) { kda::g_drop_handoff.store(on ? 1 : 0, std::memory_order_relaxed); }
 

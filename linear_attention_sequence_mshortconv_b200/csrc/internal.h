@@ -81,5 +81,10 @@ struct ConvSeg {
 cudaError_t launch_conv_segment(const void* x, void* y, int B, int T, int C, ElemType in_t,
                                 ElemType out_t, const ConvSeg& seg, int Kt, const float* w,
                                 int norm_D, cudaStream_t s);
+// The same for nt <= 3 tensors sharing the segment (weights ws[i], norm width norm_Ds[i]);
+// image and video segments of bf16 input go to one launch of the tiled kernel.
+cudaError_t launch_conv_segment_multi(int nt, const void* const* xs, void* const* ys, int B, int T, int C,
+                                      ElemType in_t, ElemType out_t, const ConvSeg& seg, int Kt,
+                                      const float* const* ws, const int* norm_Ds, cudaStream_t s);
 
 }  // namespace kda

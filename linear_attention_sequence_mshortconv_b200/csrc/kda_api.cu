@@ -263,8 +263,11 @@ kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_d
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     for (int i = 0; i < n_segs; ++i) {
         const ElemType et = dtype == KDA_F32 ? ET_F32 : ET_BF16;
-        e = launch_conv_segment(x, y, B, T, C, et, et, to_conv_seg(segs[i]), Kt,
-                                seg_weights(segs[i], C, Kt, w_text, w_image, w_video), 0, s);
+        const void* xs[1] = {x};
+        void* ys[1] = {y};
+        const float* wsel[1] = {seg_weights(segs[i], C, Kt, w_text, w_image, w_video)};
+        const int nd[1] = {0};
+        e = launch_conv_segment_multi(1, xs, ys, B, T, C, et, et, to_conv_seg(segs[i]), Kt, wsel, nd, s);
         if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     return KDA_OK;
@@ -334,14 +337,15 @@ kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv
     for (int tsr = 0; tsr < 3; ++tsr) {
         cudaError_t e = zero_gaps(ys[tsr], B, T, C, esz, segs, n_segs, s);  // esz: fp16 = bf16 size
         if (e != cudaSuccess) return KDA_ERR_CUDA;
-        for (int i = 0; i < n_segs; ++i) {
-            msc_segment sg = segs[i];
-            sg.weight_set = 0;
-            e = launch_conv_segment(xs[tsr], ys[tsr], B, T, C, in_t, mid_t, to_conv_seg(sg), Kt,
-                                    seg_weights(sg, C, Kt, ws3[tsr][0], ws3[tsr][1], ws3[tsr][2]),
-                                    tsr < 2 ? D : 0, s);
-            if (e != cudaSuccess) return KDA_ERR_CUDA;
-        }
+    }
+    const int norms[3] = {D, D, 0};
+    for (int i = 0; i < n_segs; ++i) {
+        msc_segment sg = segs[i];
+        sg.weight_set = 0;
+        const float* wsel[3];
+        for (int tsr = 0; tsr < 3; ++tsr) wsel[tsr] = seg_weights(sg, C, Kt, ws3[tsr][0], ws3[tsr][1], ws3[tsr][2]);
+        cudaError_t e = launch_conv_segment_multi(3, xs, ys, B, T, C, in_t, mid_t, to_conv_seg(sg), Kt, wsel, norms, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
     }
     KdaArgs a = fused_kda_args(B, T, H, D, dtype, o_dtype, chunk);
     a.q = qb; a.k = kb; a.v = vb; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;

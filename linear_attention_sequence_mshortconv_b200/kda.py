@@ -26,7 +26,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace_size",
             "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
-            "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff")
+            "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe")
 
 
 class KdaError(RuntimeError):
@@ -79,6 +79,8 @@ def load_library(path: str = LIB_PATH):
         lib.kda_profile_enable.argtypes = [I]
         lib.kda_debug_drop_handoff.restype = None
         lib.kda_debug_drop_handoff.argtypes = [I]
+        lib.kda_fma_probe.restype = I
+        lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
         lib.kda_profile_collect.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
                                             ctypes.POINTER(ctypes.c_int)]
@@ -283,6 +285,13 @@ def debug_drop_handoff(on: bool) -> None:
     """Test hook: while on, the tensor-core scan withholds one producer -> consumer
     hand-off per CTA, so its bounded wait runs out and the call reports a timeout."""
     load_library().kda_debug_drop_handoff(1 if on else 0)
+
+
+def fma_probe() -> float:
+    """Measured fp32 FMA rate of the current GPU (FMAs per second)."""
+    r = ctypes.c_double(0.0)
+    _check("kda_fma_probe", load_library().kda_fma_probe(ctypes.byref(r)))
+    return r.value
 
 
 def last_device_error() -> int:

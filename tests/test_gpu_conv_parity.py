@@ -61,6 +61,30 @@ def test_conv_bf16_output_is_the_rounded_fp32_sum():
     assert torch.all((y.double() - ref).abs() <= 0.5 * ulp + 1e-5 * ref.abs().max())
 
 
+@pytest.mark.parametrize("B", [1, 2])
+def test_conv_tiled_path_wide_channels(B):
+    """C = 256 (whole 128-channel blocks): image and video segments take the tiled kernel.
+    Ragged tiles in both directions, a video long enough for the frame ring to wrap, an
+    image that is an exact multiple of the tile, both weight sets, and a text segment
+    between visual ones.  bf16 output = the fp32 sum rounded once."""
+    segs, pos = [], 0
+    for (m, Fr, Hh, Wd, ws) in [(TEXT, 1, 1, 7, 0), (IMAGE, 1, 17, 33, 0), (VIDEO, 7, 11, 19, 1),
+                                (TEXT, 1, 1, 5, 1), (IMAGE, 1, 8, 16, 1), (VIDEO, 3, 8, 16, 0)]:
+        segs.append((m, pos, Fr, Hh, Wd, ws))
+        pos += Wd if m == TEXT else (Hh * Wd if m == IMAGE else Fr * Hh * Wd)
+    T, C, Kt = pos, 256, 4
+    x = torch.randn(B, T, C, generator=torch.Generator().manual_seed(21)).to(torch.bfloat16)
+    wt, wi, wv = _weights(C, Kt, 22)
+    y = kda.mshortconv(x.to(DEV), segs, Kt, wt.to(DEV), wi.to(DEV), wv.to(DEV))
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == 0
+    ref = torch.from_numpy(O.mshortconv(x, segs, Kt, wt, wi, wv))
+    y = y.float().cpu().double()
+    ulp = torch.clamp(ref.abs(), min=1e-30) * 2.0 ** -7
+    bad = (y - ref).abs() > 0.5 * ulp + 1e-5 * ref.abs().max()
+    assert not bool(bad.any()), f"{int(bad.sum())} elements off, first at {bad.nonzero()[0].tolist()}"
+
+
 def test_fused_small_mixed_stream():
     segs, T = _mixed_segments()
     B, H, D, Kt = 1, 2, 128, 4
