@@ -14,6 +14,9 @@ passages of the Chimera paper it follows, is stated in that file's header:
   3x3 spatial for an image, 3x3x3 causal-in-time / symmetric-in-space for video,
   zero padding inside each segment, time-first raster order of Eq. 12.
 * ``l2norm_heads``: unit-norm rows per head (no epsilon; zero stays zero).
+* ``gated_rmsnorm`` / ``kda_forward_gated``: the output side of Eq. 15 (section 3.3),
+  Sigmoid(gate) * RMSNorm(S_t^T q_t) per (token, head), before the output projection
+  W_o (numpy, fp64).
 """
 from __future__ import annotations
 
@@ -245,6 +248,28 @@ def fused_forward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, H, S0=None, *, 
     k = l2norm_heads(yk, H).reshape(B, T, H, D)
     v = yv.reshape(B, T, H, D)
     return kda_forward(q, k, v, _to_f64(g), _to_f64(beta), S0, pairs=pairs, nthreads=nthreads)
+
+
+def gated_rmsnorm(o, gate, gamma=None, eps=1e-6):
+    """Output side of Eq. 15 before W_o: for every (token, head) row r of o [..., H, Dv],
+    y = sigmoid(gate_r) * gamma_h * r / sqrt(mean(r^2) + eps).  The RMS runs over the
+    head's Dv channels; gamma [H, Dv] is the RMSNorm gain (None = ones); gate has o's
+    shape and holds the pre-sigmoid values W_gate x.  fp64 throughout."""
+    r = _to_f64(o)
+    gt = _to_f64(gate)
+    H, Dv = r.shape[-2], r.shape[-1]
+    gm = np.ones((H, Dv)) if gamma is None else _to_f64(gamma).reshape(H, Dv)
+    rms = np.sqrt(np.mean(r * r, axis=-1, keepdims=True) + float(eps))
+    sig = 1.0 / (1.0 + np.exp(-gt))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        y = np.where(rms > 0, r / rms, 0.0)
+    return sig * gm * y
+
+
+def kda_forward_gated(q, k, v, g, beta, gate, gamma=None, eps=1e-6, S0=None, *, pairs=None, nthreads=None):
+    """kda_forward followed by gated_rmsnorm of its readout; returns (y, S_T)."""
+    o, S_T = kda_forward(q, k, v, g, beta, S0, pairs=pairs, nthreads=nthreads)
+    return gated_rmsnorm(o, gate, gamma, eps), S_T
 
 
 def _to_f64(a):

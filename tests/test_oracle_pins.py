@@ -270,3 +270,53 @@ def test_rejects_bad_arguments():
         O.kda_forward(z, z, z, z, np.zeros((1, 4, 2)))
     with pytest.raises(TypeError):
         O.kda_forward(z.astype(np.float32), z, z, z, np.zeros((1, 4, 1)))
+
+
+# ---- output side of Eq. 15: Sigmoid(gate) * RMSNorm(o) -----------------------------------
+def _small_gated(seed=0, B=1, T=9, H=2, D=8):
+    gen = torch.Generator().manual_seed(seed)
+    f = dict(generator=gen, dtype=torch.float64)
+    unit = lambda z: z / torch.linalg.vector_norm(z, dim=-1, keepdim=True)
+    q, k = unit(torch.randn(B, T, H, D, **f)), unit(torch.randn(B, T, H, D, **f))
+    v = torch.randn(B, T, H, D, **f)
+    g = -0.1 * torch.rand(B, T, H, D, **f)
+    beta = torch.rand(B, T, H, **f)
+    gate = torch.randn(B, T, H, D, **f)
+    gamma = 0.5 + torch.rand(H, D, **f)
+    return q, k, v, g, beta, gate, gamma
+
+
+def test_gated_rmsnorm_is_invariant_to_scaling_the_values():
+    """RMSNorm removes the scale: o is linear in v (S0 = 0), so scaling v by c > 0
+    leaves the gated output unchanged (eps = 0)."""
+    q, k, v, g, beta, gate, gamma = _small_gated(1)
+    y1, _ = O.kda_forward_gated(q, k, v, g, beta, gate, gamma, eps=0.0)
+    y2, _ = O.kda_forward_gated(q, k, 37.5 * v, g, beta, gate, gamma, eps=0.0)
+    np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-14)
+
+
+def test_gated_rmsnorm_unit_rms_and_gate_limits():
+    """With gamma = 1 and a gate far above zero the sigmoid is 1 and every (token, head)
+    row has unit RMS; a zero gate halves it; a gate far below zero closes it."""
+    q, k, v, g, beta, gate, _ = _small_gated(2)
+    o, _ = O.kda_forward(q, k, v, g, beta)
+    y_open = O.gated_rmsnorm(o, np.full(o.shape, 60.0), None, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y_open ** 2, axis=-1)), 1.0, rtol=1e-12)
+    y_half = O.gated_rmsnorm(o, np.zeros(o.shape), None, eps=0.0)
+    np.testing.assert_allclose(y_half, 0.5 * y_open, rtol=1e-12, atol=1e-15)
+    y_shut = O.gated_rmsnorm(o, np.full(o.shape, -60.0), None, eps=0.0)
+    assert np.abs(y_shut).max() < 1e-25
+
+
+def test_gated_rmsnorm_gain_and_eps():
+    """gamma multiplies channel-wise per head; eps enters as mean(o^2) + eps (an all-zero
+    row stays zero, a row of constant c gets c / sqrt(c^2 + eps))."""
+    q, k, v, g, beta, gate, gamma = _small_gated(3)
+    o, _ = O.kda_forward(q, k, v, g, beta)
+    y1 = O.gated_rmsnorm(o, gate, None, eps=1e-3)
+    y2 = O.gated_rmsnorm(o, gate, gamma, eps=1e-3)
+    np.testing.assert_allclose(y2, y1 * gamma.numpy()[None, None], rtol=1e-12, atol=1e-15)
+    row = np.full((1, 1, 1, 4), 0.2)
+    y = O.gated_rmsnorm(row, np.full(row.shape, 60.0), None, eps=0.01)
+    np.testing.assert_allclose(y, 0.2 / np.sqrt(0.04 + 0.01), rtol=1e-12)
+    assert np.all(O.gated_rmsnorm(np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)), None, eps=0.0) == 0.0)
