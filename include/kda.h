@@ -109,6 +109,26 @@ kda_status kda_forward(const void* q, const void* k, const void* v, const void* 
 #define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /*
+ * kda_forward_gated -- kda_forward followed by the output side of Eq. 15 (Chimera
+ * paper, section 3.3) before the output projection W_o:
+ *     y[b,t,h,:] = Sigmoid(gate[b,t,h,:]) * gamma[h,:] * r / sqrt(mean(r^2) + eps),
+ *     r = S_t^T q_t (the readout kda_forward would write), mean over the head's Dv values.
+ *   gate  : [B,T,H,Dv] device, dtype `dtype`; the pre-sigmoid values W_gate x (the
+ *           projection itself is outside this library).  Required when B*T > 0.
+ *   gamma : [H,Dv] fp32 device, the RMSNorm gain per head; NULL = all ones.
+ *   eps   : >= 0 and finite; a row with mean(r^2) + eps == 0 yields zeros.
+ *   o     : receives y (o_dtype).  Every other argument, the workspace and the errors
+ *           are those of kda_forward; S_T is unaffected by the epilogue.
+ * On the tensor-core path with a bf16 output the epilogue runs inside the scan's output
+ * stage (r never reaches global memory); otherwise a separate kernel rewrites o in place.
+ */
+kda_status kda_forward_gated(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* S0, const void* gate, const float* gamma,
+                             float eps, void* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                             kda_dtype dtype, kda_dtype o_dtype, int chunk, void* workspace,
+                             size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_forward_noalloc -- kda_forward that allocates no device memory.  The paper has
  * no counterpart to this call; it exists for callers that cannot allocate during a
  * call: code inside a host framework that owns all device memory through its own
@@ -235,7 +255,7 @@ void kda_profile_enable(int on);
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
  * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
- * "kda_tc_output", "conv". */
+ * "kda_tc_output", "conv", "gate_norm". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

@@ -60,7 +60,14 @@ struct KdaArgs {
     ElemType in_t;   // q, k, v
     ElemType out_t;  // o
     ElemType gb_t;   // g, beta
+    // output side of Eq. 15 (gated path only): o <- Sigmoid(gate) * gamma * RMSNorm(o)
+    const void* gate = nullptr;   // [B,T,H,Dv], dtype of q (nullptr: plain readout)
+    const float* gamma = nullptr; // [H,Dv] fp32 or nullptr (ones)
+    float eps = 0.f;
 };
+
+// In-place gated RMSNorm of o (a.gate != nullptr), one warp per (token, head).
+cudaError_t launch_gate_rmsnorm(const KdaArgs& a, cudaStream_t s);
 
 // Generic chunkwise scan on CUDA cores in fp32 (any supported dtype/shape).
 cudaError_t launch_kda_generic(const KdaArgs& a, cudaStream_t s);

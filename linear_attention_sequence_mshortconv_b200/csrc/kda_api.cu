@@ -74,7 +74,9 @@ kda_status run_kda(const KdaArgs& a, void* ws, size_t ws_bytes, cudaStream_t s)
         if (!st) return KDA_ERR_CUDA;
         return from_cuda(launch_kda_tc(a, ws, ws_bytes, st, s));
     }
-    return from_cuda(launch_kda_generic(a, s));
+    cudaError_t e = launch_kda_generic(a, s);
+    if (e == cudaSuccess && a.gate) e = launch_gate_rmsnorm(a, s);
+    return from_cuda(e);
 }
 
 size_t kda_ws_bytes(const KdaArgs& a)
@@ -165,6 +167,32 @@ kda_status kda_forward(const void* q, const void* k, const void* v, const void* 
     }
     KdaArgs a{q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv,
               chunk ? chunk : default_chunk(dtype, Dk), et_of(dtype), et_of(o_dtype), et_of(dtype)};
+    Workspace ws;
+    st = ws.acquire(workspace, workspace_bytes, kda_ws_bytes(a), s);
+    if (st != KDA_OK) return st;
+    return run_kda(a, ws.ptr, kda_ws_bytes(a), s);
+}
+
+kda_status kda_forward_gated(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* S0, const void* gate, const float* gamma,
+                             float eps, void* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                             kda_dtype dtype, kda_dtype o_dtype, int chunk, void* workspace,
+                             size_t workspace_bytes, kda_stream_t stream)
+{
+    kda_status st = check_kda_args(q, k, v, g, beta, o, B, T, H, Dk, Dv, dtype, o_dtype, chunk);
+    if (st != KDA_OK) return st;
+    if ((int64_t)B * T > 0 && !gate) return KDA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 1e30f) return KDA_ERR_INVALID_ARG;   // also rejects NaN
+    cudaStream_t s = (cudaStream_t)stream;
+    if (B == 0) return KDA_OK;
+    if (T == 0)
+        return kda_forward(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, dtype, o_dtype, chunk, workspace,
+                           workspace_bytes, stream);
+    KdaArgs a{q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv,
+              chunk ? chunk : default_chunk(dtype, Dk), et_of(dtype), et_of(o_dtype), et_of(dtype)};
+    a.gate = gate;
+    a.gamma = gamma;
+    a.eps = eps;
     Workspace ws;
     st = ws.acquire(workspace, workspace_bytes, kda_ws_bytes(a), s);
     if (st != KDA_OK) return st;

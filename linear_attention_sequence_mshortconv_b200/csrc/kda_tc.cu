@@ -114,13 +114,14 @@ constexpr int M_TOT = 512;       // float[4][128] per-16-row sums of g log2(e)
 constexpr int M_RB = 2560;       // float2[2][128] (r, b_C) per channel, per buffer set
 constexpr int M_XS = 4608;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
 constexpr int M_BAR = 8704;      // mbarriers, see Bar
-constexpr int M_TMEM = 8848;     // uint32 TMEM base
-constexpr int M_ABORT = 8852;    // int
+constexpr int M_TMEM = 8856;     // uint32 TMEM base
+constexpr int M_ABORT = 8860;    // int
 constexpr int MISC_BYTES = 8864;
 // PRO: a set's beta K+, Q+, K- tiles and r, b_C are ready; INV: its T (and P) too;
 // EMPTY: the consumer's last MMA on the set is done.
 enum Bar { B_PRO = 0, B_EMPTY = 2, B_AP = 4, B_Y = 5, B_U = 6, B_S = 7, B_AFREE = 8, B_UREAD = 9,
-           B_DRAIN = 10, B_DRAIN2 = 11, B_TQK = 12, B_TG = 14, B_TV = 15, B_INV = 16, NBAR = 18 };
+           B_DRAIN = 10, B_DRAIN2 = 11, B_TQK = 12, B_TG = 14, B_TV = 15, B_INV = 16, B_TGATE = 18,
+           NBAR = 19 };
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 
@@ -270,6 +271,65 @@ __device__ __forceinline__ void stage_o_swz(uint32_t tl, int q4, int hg, int lan
         }
     }
 }
+// Output side of Eq. 15 for a bf16 output: y = Sigmoid(gate) * gamma_h * RMSNorm(o) per
+// output row, written into the same swizzled tiles as stage_o_swz.  The gate arrives by
+// TMA as two swizzled 64-channel tiles (the layout of the output tiles).  A row's 128
+// channels sit in two warps (column halves), so its sum of squares is exchanged through
+// `red` between two group barriers; TMEM is read twice instead of holding 64 values.
+__device__ __forceinline__ void stage_o_gated(uint32_t tl, int q4, int hg, int lane, uint8_t* tiles,
+                                              const uint8_t* gtiles, float* red, const float* gamma_h, float eps)
+{
+    const int i = 32 * (q4 - 2) + lane;
+    if (q4 >= 2) {
+        float ss = 0.f;
+        for (int u = 0; u < 2; ++u) {
+            float v[32];
+            tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+        }
+        red[2 * i + hg] = ss;
+    }
+    named_sync(2, NG);
+    if (q4 < 2) return;
+    const float m = (red[2 * i] + red[2 * i + 1]) * (1.f / D) + eps;
+    const float inv = m > 0.f ? rsqrtf(m) : 0.f;
+    uint8_t* tile = tiles + hg * 8192;
+    const uint8_t* gtile = gtiles + hg * 8192;
+    for (int u = 0; u < 2; ++u) {
+        float v[32];
+        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int chunk = 4 * u + j;
+            const int off = i * 128 + ((chunk ^ (i & 7)) * 16);
+            const uint4 gu = *reinterpret_cast<const uint4*>(gtile + off);
+            const __nv_bfloat162* gb = reinterpret_cast<const __nv_bfloat162*>(&gu);
+            const int c0 = 64 * hg + 8 * chunk;
+            float gm[8];
+            if (gamma_h) {
+                const float4 g0 = *reinterpret_cast<const float4*>(gamma_h + c0);
+                const float4 g1 = *reinterpret_cast<const float4*>(gamma_h + c0 + 4);
+                gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
+                gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gm[e] = 1.f;
+            }
+            uint4 uu;
+            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 gv = __bfloat1622float2(gb[e]);
+                const float y0 = v[8 * j + 2 * e] * inv * gm[2 * e] / (1.f + __expf(-gv.x));
+                const float y1 = v[8 * j + 2 * e + 1] * inv * gm[2 * e + 1] / (1.f + __expf(-gv.y));
+                hh[e] = __floats2bfloat162_rn(y0, y1);
+            }
+            *reinterpret_cast<uint4*>(tile + off) = uu;
+        }
+    }
+}
+
 __device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int b, int T, int H, int h,
                                         int t0)
 {
@@ -317,9 +377,11 @@ template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-              const __grid_constant__ CUtensorMap tm_o, const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
+              const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_gate,
+              const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
-              float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop)
+              float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop,
+              const float* __restrict__ gamma, float eps, int gated)
 {
     using PL = Plan<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
@@ -383,6 +445,15 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_arrive_expect_tx(&bars[B_TV], 16384);
         tma_load_3d(sm + PL::VB, &tm_v, &bars[B_TV], 0, h, b * T + n * C);
     };
+    // gated bf16 output: chunk n's gate as two swizzled 64-channel tiles in the upper half
+    // of the S^ region (free from the end of chunk n's [Y; O] MMA to chunk n+1's S^)
+    auto tma_gate = [&](int n) {
+        mbar_arrive_expect_tx(&bars[B_TGATE], 16384);
+        tma_load_3d(sm + PL::S + 16384, &tm_gate, &bars[B_TGATE], 0, h, b * T + n * C);
+        tma_load_3d(sm + PL::S + 24576, &tm_gate, &bars[B_TGATE], 64, h, b * T + n * C);
+    };
+    const bool gate_fused = OUT && gated && !o_f32;
+    const float* gamma_h = gamma ? gamma + (size_t)h * D : nullptr;
 
     if (t < NG) {
         // ================= producer: state-independent work of chunk n0 + kc ==============
@@ -659,7 +730,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // thread NG + 32 (not the MMA issuer) requests the consumer-side TMA loads, just
         // before a barrier at which the group waits for an MMA anyway
         const bool loader = tg == 32;
-        int v_issued = 0, qk_last[2] = {-1, -1};   // its TMA requests so far
+        int v_issued = 0, qk_last[2] = {-1, -1}, gate_issued = 0;   // its TMA requests so far
         bool o_pending = false;                    // poller: a bf16 output store is in flight
         if (loader && nk > 0) {
             tma_v(n0);
@@ -687,7 +758,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, t0 - C);
                     named_sync(2, NG);
                 } else {
-                    stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                    if (gate_fused) {
+                        group_wait(&bars[B_TGATE], (kc - 1) & 1, ab, poller, 2);
+                        stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
+                                      reinterpret_cast<float*>(sm + PL::S), gamma_h, eps);
+                    } else {
+                        stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                    }
                     fence_async_smem();
                     named_sync(2, NG);
                     if (poller) {
@@ -835,10 +912,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 umma_commit(&bars[B_U]);
             }
             // [Y; O] of this chunk is done: chunk n+2's q, k may land in this set's
-            // Q+ / beta K+ slots
+            // Q+ / beta K+ slots (and this chunk's gate in the upper half of S^)
             if (loader && n + 2 < n1 && !*sAbort) {
                 tma_qk(n + 2);
                 qk_last[bs] = kc + 2;
+            }
+            if (gate_fused && loader && !*sAbort) {
+                tma_gate(n);
+                gate_issued = kc + 1;
             }
             // the output store must have read the U region before U is written there
             if (poller && o_pending) {
@@ -896,7 +977,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 named_sync(2, NG);
                 flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, (n1 - 1) * C);
             } else {
-                stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                if (gate_fused) {
+                    group_wait(&bars[B_TGATE], (nk - 1) & 1, ab, poller, 2);
+                    stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
+                                  reinterpret_cast<float*>(sm + PL::S), gamma_h, eps);
+                } else {
+                    stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                }
                 fence_async_smem();
                 named_sync(2, NG);
                 if (poller) {
@@ -909,6 +996,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (poller) bulk_wait0();   // every output store has landed before the CTA exits
         // after a timeout some requested tiles may not have been waited for: let them land
         if (loader && *sAbort) {
+            if (gate_issued > 0) mbar_wait_bounded(&bars[B_TGATE], (gate_issued - 1) & 1, kWaitNs);
             if (v_issued > 0) mbar_wait_bounded(&bars[B_TV], (v_issued - 1) & 1, kWaitNs);
             for (int s2 = 0; s2 < 2; ++s2)
                 if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
@@ -1066,8 +1154,24 @@ bool make_map_o(CUtensorMap* m, void* base, int B, int T, int H)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Gate [B*T, H, 128] bf16 as two 64-channel halves per chunk (box 64 x 1 x 64), 128-byte
+// swizzle: lands in the layout of the swizzled output tiles.
+bool make_map_gate(CUtensorMap* m, const void* base, int B, int T, int H)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    const cuuint32_t box[3] = {64u, 1u, (cuuint32_t)C};
+    const cuuint32_t es[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Maps {
     CUtensorMap q, k, v, g, o;   // o: only for a bf16 output (else a copy of q, unused)
+    CUtensorMap gate;            // only for the fused gated epilogue (else a copy of q)
 };
 
 struct Split {
@@ -1095,8 +1199,9 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     const unsigned grid = (unsigned)(a.B * a.H * nseg);
     ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
-                                S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff());
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, mp.gate, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+                                S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
+                                a.gamma, a.eps, a.gate != nullptr ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -1116,6 +1221,11 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         return cudaErrorInvalidValue;
     if (a.out_t == ET_F32) mp.o = mp.q;
     else if (!make_map_o(&mp.o, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    if (a.gate && a.out_t == ET_BF16) {
+        if (!make_map_gate(&mp.gate, a.gate, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    } else {
+        mp.gate = mp.q;
+    }
     if (sp.P == 1) return launch_pass<MODE_OUTPUT, TQ>(mp, a, a.S0, 0, nullptr, 1, sp.L, status, s);
     float* maps = reinterpret_cast<float*>(ws);
     float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
@@ -1144,6 +1254,7 @@ bool kda_tc_supported(const KdaArgs& a)
     if (a.gb_t != ET_BF16) return false;
     if (a.out_t != ET_BF16 && a.out_t != ET_F32) return false;
     if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.g) || !aligned16(a.o)) return false;
+    if (a.gate && (a.in_t != ET_BF16 || !aligned16(a.gate) || (a.gamma && !aligned16(a.gamma)))) return false;
     return encode_fn() != nullptr;
 }
 
@@ -1158,8 +1269,14 @@ size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms)
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status, cudaStream_t s)
 {
     (void)ws_bytes;
-    if (a.in_t == ET_F16) return launch_all<__half>(a, ws, status, s);
-    return launch_all<__nv_bfloat16>(a, ws, status, s);
+    // the gated epilogue is fused into the output stage for a bf16 output; an fp32 output
+    // gets the plain scan followed by the separate epilogue kernel
+    KdaArgs scan = a;
+    if (a.gate && a.out_t == ET_F32) scan.gate = nullptr;
+    const cudaError_t e = a.in_t == ET_F16 ? launch_all<__half>(scan, ws, status, s)
+                                           : launch_all<__nv_bfloat16>(scan, ws, status, s);
+    if (e != cudaSuccess || !a.gate || a.out_t != ET_F32) return e;
+    return launch_gate_rmsnorm(a, s);
 }
 
 }  // namespace kda

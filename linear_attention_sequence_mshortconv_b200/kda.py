@@ -26,7 +26,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace_size",
             "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
-            "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe")
+            "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
+            "kda_forward_gated")
 
 
 class KdaError(RuntimeError):
@@ -79,6 +80,9 @@ def load_library(path: str = LIB_PATH):
         lib.kda_profile_enable.argtypes = [I]
         lib.kda_debug_drop_handoff.restype = None
         lib.kda_debug_drop_handoff.argtypes = [I]
+        lib.kda_forward_gated.restype = I
+        lib.kda_forward_gated.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_float, P, P, I, I, I, I, I, I, I,
+                                          I, P, Z, P]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -160,6 +164,42 @@ def forward(q, k, v, g, beta, S0=None, *, chunk: int = 0, o=None, S_T=None,
                          _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv, dt, _code(o_dtype),
                          chunk, ws_ptr, ws_bytes, _stream(stream))
     _check("kda_forward", rc)
+    return o, S_T
+
+
+def forward_gated(q, k, v, g, beta, gate, gamma=None, eps: float = 1e-6, S0=None, *, chunk: int = 0,
+                  o=None, S_T=None, want_state: bool = True, workspace=None, stream=None, o_dtype=None):
+    """kda_forward_gated: the scan of forward() with the output side of Eq. 15 applied,
+    y = Sigmoid(gate) * gamma_h * RMSNorm(S_t^T q_t) per (token, head).  gate: [B,T,H,Dv]
+    in q's dtype; gamma: [H,Dv] fp32 or None.  Returns (y, S_T or None)."""
+    lib = load_library()
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q)
+    for name, t, shape in (("k", k, (B, T, H, Dk)), ("g", g, (B, T, H, Dk)),
+                           ("v", v, (B, T, H, Dv)), ("beta", beta, (B, T, H)), ("gate", gate, (B, T, H, Dv))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q's {q.dtype}")
+    if gamma is not None and tuple(gamma.shape) != (H, Dv):
+        raise ValueError("gamma shape")
+    o_dtype = o_dtype or (o.dtype if o is not None else q.dtype)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    if S0 is not None and tuple(S0.shape) != (B, H, Dk, Dv):
+        raise ValueError("S0 shape")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.kda_forward_gated(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+                               _dev(S0, "S0", torch.float32), _dev(gate, "gate"),
+                               _dev(gamma, "gamma", torch.float32), float(eps), _dev(o, "o", o_dtype),
+                               _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv, dt, _code(o_dtype),
+                               chunk, ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_forward_gated", rc)
     return o, S_T
 
 

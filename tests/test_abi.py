@@ -57,6 +57,19 @@ def test_host_rejects_bad_arguments(lib):
     assert lib.kda_forward(P, P, P, P, P, P, P, P, 0, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 0
 
 
+def test_gated_forward_rejects_bad_arguments(lib):
+    P = None
+    d = ctypes.c_void_p(256)   # never dereferenced: validation fails first
+    args = lambda gate, eps, Dk=32: (d, d, d, d, d, P, gate, P, eps, d, P, 1, 8, 1, Dk, Dk, 1, 1, 0, P, 0, P)
+    assert lib.kda_forward_gated(*args(P, 1e-6)) == 1                    # no gate with work to do
+    assert lib.kda_forward_gated(*args(d, -1.0)) == 1                    # eps < 0
+    assert lib.kda_forward_gated(*args(d, float("nan"))) == 1            # eps NaN
+    assert lib.kda_forward_gated(*args(d, float("inf"))) == 1            # eps not finite
+    assert lib.kda_forward_gated(*args(d, 1e-6, Dk=48)) == 2             # unsupported head width
+    # empty batch is a no-op
+    assert lib.kda_forward_gated(d, d, d, d, d, P, P, P, 1e-6, d, P, 0, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 0
+
+
 def test_conv_rejects_bad_segment_tables(lib):
     segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
     dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
