@@ -14,6 +14,8 @@ passages of the Chimera paper it follows, is stated in that file's header:
   3x3 spatial for an image, 3x3x3 causal-in-time / symmetric-in-space for video,
   zero padding inside each segment, time-first raster order of Eq. 12.
 * ``l2norm_heads``: unit-norm rows per head (no epsilon; zero stays zero).
+* ``kda_forward_varlen``: packed samples on one token axis, each scanned from its own
+  S0 (zero by default): the reset at a sample start of section 3.3.
 * ``gated_rmsnorm`` / ``kda_forward_gated``: the output side of Eq. 15 (section 3.3),
   Sigmoid(gate) * RMSNorm(S_t^T q_t) per (token, head), before the output projection
   W_o (numpy, fp64).
@@ -248,6 +250,29 @@ def fused_forward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, H, S0=None, *, 
     k = l2norm_heads(yk, H).reshape(B, T, H, D)
     v = yv.reshape(B, T, H, D)
     return kda_forward(q, k, v, _to_f64(g), _to_f64(beta), S0, pairs=pairs, nthreads=nthreads)
+
+
+def kda_forward_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, nthreads=None):
+    """Packed samples: q, k, g [T,H,Dk], v [T,H,Dv], beta [T,H]; sample i is tokens
+    [cu[i], cu[i+1]) and runs kda_forward from S0[i] (zeros if S0 is None).  Returns
+    (o [T,H,Dv], S_T [n,H,Dk,Dv]) in fp64."""
+    cu = [int(x) for x in cu_seqlens]
+    n = len(cu) - 1
+    T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    o = np.zeros((T, H, Dv))
+    S_T = np.zeros((n, H, Dk, Dv))
+    for i in range(n):
+        a, b = cu[i], cu[i + 1]
+        s0 = None if S0 is None else _to_f64(S0)[i:i + 1]
+        if b == a:
+            S_T[i] = 0.0 if s0 is None else s0[0]
+            continue
+        sl = lambda t: t[a:b][None]
+        oi, si = kda_forward(sl(q), sl(k), sl(v), sl(g), sl(beta), s0, nthreads=nthreads)
+        o[a:b] = oi[0]
+        S_T[i] = si[0]
+    return o, S_T
 
 
 def gated_rmsnorm(o, gate, gamma=None, eps=1e-6):

@@ -320,3 +320,30 @@ def test_gated_rmsnorm_gain_and_eps():
     y = O.gated_rmsnorm(row, np.full(row.shape, 60.0), None, eps=0.01)
     np.testing.assert_allclose(y, 0.2 / np.sqrt(0.04 + 0.01), rtol=1e-12)
     assert np.all(O.gated_rmsnorm(np.zeros((1, 2, 1, 4)), np.zeros((1, 2, 1, 4)), None, eps=0.0) == 0.0)
+
+
+# ---- packed samples --------------------------------------------------------------------
+def test_varlen_samples_are_independent_scans():
+    """Each packed sample is the scan of that sample alone from its own S0 (the reset at a
+    sample start): a single sample equals kda_forward, and changing one sample's values
+    leaves every other sample's output and final state bit-for-bit unchanged."""
+    gen = torch.Generator().manual_seed(11)
+    T, H, D = 23, 2, 4
+    f = dict(generator=gen, dtype=torch.float64)
+    q, k, g = torch.randn(T, H, D, **f), torch.randn(T, H, D, **f), -0.2 * torch.rand(T, H, D, **f)
+    v, beta = torch.randn(T, H, D, **f), torch.rand(T, H, **f)
+    S0 = torch.randn(4, H, D, D, **f)
+    cu = [0, 6, 6, 15, 23]
+    o, S = O.kda_forward_varlen(q, k, v, g, beta, cu, S0)
+    o1, S1 = O.kda_forward(q[6:15][None], k[6:15][None], v[6:15][None], g[6:15][None], beta[6:15][None],
+                           S0[2:3].numpy())
+    np.testing.assert_array_equal(o[6:15], o1[0])
+    np.testing.assert_array_equal(S[2], S1[0])
+    np.testing.assert_array_equal(S[1], S0[1].numpy())          # empty sample: S_T = S0
+    v2 = v.clone()
+    v2[6:15] *= -3.0
+    o2, Sb = O.kda_forward_varlen(q, k, v2, g, beta, cu, S0)
+    for (a, b, i) in [(0, 6, 0), (15, 23, 3)]:
+        np.testing.assert_array_equal(o2[a:b], o[a:b])
+        np.testing.assert_array_equal(Sb[i], S[i])
+    assert not np.array_equal(o2[6:15], o[6:15])
