@@ -432,6 +432,30 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             if other.fused and "conv" in kern:
                 rec["conv_alu"] = conv_alu_roofline(other, kern["conv"]["ms_per_step"])
             extra.append(rec)
+        # the headline workload with the output side of Eq. 15 fused (Sigmoid(gate) *
+        # RMSNorm(readout)); its extra bytes are the gate read
+        if not w.fused:
+            inp_g = W.make_kda_inputs(w, device="cuda")
+            gen = torch.Generator().manual_seed(7)
+            gate = torch.randn(w.B, w.T, w.H, w.D, generator=gen).to(w.dtype).cuda()
+            gamma = (0.5 + torch.rand(w.H, w.D, generator=gen)).cuda()
+            og = torch.empty((w.B, w.T, w.H, w.D), dtype=w.dtype, device="cuda")
+            Sg = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32, device="cuda")
+            wsz = kda.workspace_size(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+            wsb = torch.empty(max(wsz, 1), dtype=torch.uint8, device="cuda")
+
+            def gstep():
+                kda.forward_gated(inp_g["q"], inp_g["k"], inp_g["v"], inp_g["g"], inp_g["beta"], gate, gamma,
+                                  1e-6, chunk=w.chunk, o=og, S_T=Sg, workspace=wsb)
+            for _ in range(3):
+                gstep()
+            k_g = max(3, args.steps // 4)
+            mg = timed(gstep, k_g, 1) / k_g
+            gbytes = algorithmic_bytes(w) + w.B * w.T * w.H * w.D * torch.tensor([], dtype=w.dtype).element_size()
+            extra.append({"workload": w.name + "_gated_output", "ms_per_step": mg,
+                          "value": w.tokens / (mg * 1e-3) / 1e6, "unit": UNIT,
+                          "alg_GBps": gbytes / (mg * 1e-3) / 1e9,
+                          "epilogue": "Sigmoid(gate) * RMSNorm(S_t^T q_t), fused in the output stage"})
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -129,6 +129,27 @@ kda_status kda_forward_gated(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_forward_varlen -- kda_forward over packed samples: n_seqs sequences laid end to end
+ * on one token axis, the state reset at the start of every sample (Eq. 14 runs from S0
+ * of that sample, section 3.3: a sample starts from the zero state).
+ *   cu_seqlens : HOST array of n_seqs + 1 int32 offsets, cu_seqlens[0] = 0, non-decreasing;
+ *                sample i is tokens [cu_seqlens[i], cu_seqlens[i+1]) (empty samples allowed).
+ *   q, k, g    : [T_total, H, Dk] with T_total = cu_seqlens[n_seqs]; v, o: [T_total, H, Dv];
+ *   beta       : [T_total, H];  all device memory, dtypes as for kda_forward.
+ *   S0, S_T    : [n_seqs, H, Dk, Dv] fp32 or NULL (zeros / not written); an empty
+ *                sample's S_T is its S0.
+ *   workspace  : as for kda_forward, sized by kda_forward_varlen_workspace_size (which
+ *                depends on the offsets).
+ * Errors as for kda_forward; bad offsets give KDA_ERR_INVALID_ARG.
+ */
+size_t kda_forward_varlen_workspace_size(const int32_t* cu_seqlens, int n_seqs, int H, int Dk, int Dv,
+                                         kda_dtype dtype, kda_dtype o_dtype, int chunk);
+kda_status kda_forward_varlen(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                              const float* S0, void* o, float* S_T, const int32_t* cu_seqlens, int n_seqs,
+                              int H, int Dk, int Dv, kda_dtype dtype, kda_dtype o_dtype, int chunk,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_forward_noalloc -- kda_forward that allocates no device memory.  The paper has
  * no counterpart to this call; it exists for callers that cannot allocate during a
  * call: code inside a host framework that owns all device memory through its own

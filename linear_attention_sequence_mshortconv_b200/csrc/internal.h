@@ -77,6 +77,9 @@ size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms);
 bool kda_tc_supported(const KdaArgs& a);
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status,
                           cudaStream_t s);
+// Packed samples: a.B = 1, a.T = cu[n] tokens; host array cu[0..n] of sample offsets.
+size_t kda_tc_varlen_workspace_bytes(const int* cu, int n, int H, int num_sms);
+cudaError_t launch_kda_tc_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int* status, cudaStream_t s);
 
 struct ConvSeg {
     int32_t modality;

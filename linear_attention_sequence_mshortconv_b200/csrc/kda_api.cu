@@ -199,6 +199,89 @@ kda_status kda_forward_gated(const void* q, const void* k, const void* v, const 
     return run_kda(a, ws.ptr, kda_ws_bytes(a), s);
 }
 
+// ---- packed samples -------------------------------------------------------------------
+static kda_status check_cu(const int32_t* cu, int n_seqs)
+{
+    if (n_seqs < 0 || !cu) return KDA_ERR_INVALID_ARG;
+    if (cu[0] != 0) return KDA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_seqs; ++i)
+        if (cu[i + 1] < cu[i]) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
+static KdaArgs varlen_args(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                           const float* S0, void* o, float* S_T, int T_total, int H, int Dk, int Dv,
+                           kda_dtype dtype, kda_dtype o_dtype, int chunk)
+{
+    return KdaArgs{q, k, v, g, beta, S0, o, S_T, 1, T_total, H, Dk, Dv,
+                   chunk ? chunk : default_chunk(dtype, Dk), et_of(dtype), et_of(o_dtype), et_of(dtype)};
+}
+
+size_t kda_forward_varlen_workspace_size(const int32_t* cu_seqlens, int n_seqs, int H, int Dk, int Dv,
+                                         kda_dtype dtype, kda_dtype o_dtype, int chunk)
+{
+    if (check_cu(cu_seqlens, n_seqs) != KDA_OK || H <= 0 || !dim_ok(Dk) || !dim_ok(Dv)) return 0;
+    if (n_seqs == 0 || cu_seqlens[n_seqs] == 0) return 0;
+    const KdaArgs a = varlen_args(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                                  cu_seqlens[n_seqs], H, Dk, Dv, dtype, o_dtype, chunk);
+    if (!kda_tc_supported(a)) return 0;
+    return kda_tc_varlen_workspace_bytes(cu_seqlens, n_seqs, H, num_sms());
+}
+
+kda_status kda_forward_varlen(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                              const float* S0, void* o, float* S_T, const int32_t* cu_seqlens, int n_seqs,
+                              int H, int Dk, int Dv, kda_dtype dtype, kda_dtype o_dtype, int chunk,
+                              void* workspace, size_t workspace_bytes, kda_stream_t stream)
+{
+    kda_status st = check_cu(cu_seqlens, n_seqs);
+    if (st != KDA_OK) return st;
+    const int T = n_seqs ? cu_seqlens[n_seqs] : 0;
+    st = check_kda_args(q, k, v, g, beta, o, 1, T, H, Dk, Dv, dtype, o_dtype, chunk);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (n_seqs == 0) return KDA_OK;
+    // empty samples: S_T = S0 (or zero)
+    const size_t sbytes = (size_t)H * Dk * Dv * sizeof(float);
+    for (int i = 0; i < n_seqs; ++i) {
+        if (cu_seqlens[i + 1] != cu_seqlens[i] || !S_T) continue;
+        float* dst = S_T + (size_t)i * H * Dk * Dv;
+        const cudaError_t e = S0 ? cudaMemcpyAsync(dst, S0 + (size_t)i * H * Dk * Dv, sbytes, cudaMemcpyDeviceToDevice, s)
+                                 : cudaMemsetAsync(dst, 0, sbytes, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (T == 0) return KDA_OK;
+    const KdaArgs a = varlen_args(q, k, v, g, beta, S0, o, S_T, T, H, Dk, Dv, dtype, o_dtype, chunk);
+    if (kda_tc_supported(a)) {
+        const size_t need = kda_tc_varlen_workspace_bytes(cu_seqlens, n_seqs, H, num_sms());
+        Workspace ws;
+        st = ws.acquire(workspace, workspace_bytes, need, s);
+        if (st != KDA_OK) return st;
+        int* dst = device_status_ptr();
+        if (!dst) return KDA_ERR_CUDA;
+        return from_cuda(launch_kda_tc_varlen(a, cu_seqlens, n_seqs, ws.ptr, dst, s));
+    }
+    // CUDA-core path: one launch per non-empty sample on its slice of the packed axis
+    const size_t es = dtype == KDA_F32 ? 4 : 2, eo = o_dtype == KDA_F32 ? 4 : 2;
+    for (int i = 0; i < n_seqs; ++i) {
+        const int t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
+        if (len == 0) continue;
+        const size_t kq = (size_t)t0 * H * Dk, kv = (size_t)t0 * H * Dv, kb = (size_t)t0 * H;
+        KdaArgs ai = a;
+        ai.T = len;
+        ai.q = (const char*)q + kq * es;
+        ai.k = (const char*)k + kq * es;
+        ai.g = (const char*)g + kq * es;
+        ai.v = (const char*)v + kv * es;
+        ai.beta = (const char*)beta + kb * es;
+        ai.o = (char*)o + kv * eo;
+        ai.S0 = S0 ? S0 + (size_t)i * H * Dk * Dv : nullptr;
+        ai.ST = S_T ? S_T + (size_t)i * H * Dk * Dv : nullptr;
+        const cudaError_t e = launch_kda_generic(ai, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
 static kda_status check_segments(const msc_segment* segs, int n_segs, int T, int Kt,
                                  const float* w_text, int n_text, const float* w_image,
                                  int n_image, const float* w_video, int n_video)

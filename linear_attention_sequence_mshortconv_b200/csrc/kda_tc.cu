@@ -55,6 +55,7 @@
 
 #include <mutex>
 #include <type_traits>
+#include <vector>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -116,7 +117,8 @@ constexpr int M_XS = 4608;       // 8 x 512 B per-warp 16x16 fp16 scratch of the
 constexpr int M_BAR = 8704;      // mbarriers, see Bar
 constexpr int M_TMEM = 8856;     // uint32 TMEM base
 constexpr int M_ABORT = 8860;    // int
-constexpr int MISC_BYTES = 8864;
+constexpr int M_GAMMA = 8864;    // float[128] RMSNorm gain of this CTA's head (gated output)
+constexpr int MISC_BYTES = 9376;
 // PRO: a set's beta K+, Q+, K- tiles and r, b_C are ready; INV: its T (and P) too;
 // EMPTY: the consumer's last MMA on the set is done.
 enum Bar { B_PRO = 0, B_EMPTY = 2, B_AP = 4, B_Y = 5, B_U = 6, B_S = 7, B_AFREE = 8, B_UREAD = 9,
@@ -277,7 +279,7 @@ __device__ __forceinline__ void stage_o_swz(uint32_t tl, int q4, int hg, int lan
 // channels sit in two warps (column halves), so its sum of squares is exchanged through
 // `red` between two group barriers; TMEM is read twice instead of holding 64 values.
 __device__ __forceinline__ void stage_o_gated(uint32_t tl, int q4, int hg, int lane, uint8_t* tiles,
-                                              const uint8_t* gtiles, float* red, const float* gamma_h, float eps)
+                                              const uint8_t* gtiles, float* red, const float* sGamma, float eps)
 {
     const int i = 32 * (q4 - 2) + lane;
     if (q4 >= 2) {
@@ -306,23 +308,16 @@ __device__ __forceinline__ void stage_o_gated(uint32_t tl, int q4, int hg, int l
             const uint4 gu = *reinterpret_cast<const uint4*>(gtile + off);
             const __nv_bfloat162* gb = reinterpret_cast<const __nv_bfloat162*>(&gu);
             const int c0 = 64 * hg + 8 * chunk;
-            float gm[8];
-            if (gamma_h) {
-                const float4 g0 = *reinterpret_cast<const float4*>(gamma_h + c0);
-                const float4 g1 = *reinterpret_cast<const float4*>(gamma_h + c0 + 4);
-                gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
-                gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) gm[e] = 1.f;
-            }
+            const float4 g0 = *reinterpret_cast<const float4*>(sGamma + c0);
+            const float4 g1 = *reinterpret_cast<const float4*>(sGamma + c0 + 4);
+            const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
             uint4 uu;
             __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 gv = __bfloat1622float2(gb[e]);
-                const float y0 = v[8 * j + 2 * e] * inv * gm[2 * e] / (1.f + __expf(-gv.x));
-                const float y1 = v[8 * j + 2 * e + 1] * inv * gm[2 * e + 1] / (1.f + __expf(-gv.y));
+                const float y0 = __fdividef(v[8 * j + 2 * e] * inv * gm[2 * e], 1.f + __expf(-gv.x));
+                const float y1 = __fdividef(v[8 * j + 2 * e + 1] * inv * gm[2 * e + 1], 1.f + __expf(-gv.y));
                 hh[e] = __floats2bfloat162_rn(y0, y1);
             }
             *reinterpret_cast<uint4*>(tile + off) = uu;
@@ -330,8 +325,8 @@ __device__ __forceinline__ void stage_o_gated(uint32_t tl, int q4, int hg, int l
     }
 }
 
-__device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int b, int T, int H, int h,
-                                        int t0)
+__device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int64_t rowbase, int T, int H,
+                                        int h, int t0)
 {
     const int es = o_f32 ? 4 : 2, ld = D * es + 16;
     const int per_row = D * es / 16;                 // 16-byte pieces per row
@@ -339,7 +334,7 @@ __device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int
         const int i = e / per_row, pc = e % per_row;
         if (t0 + i < T) {
             const uint4 x = *reinterpret_cast<const uint4*>(stg + i * ld + pc * 16);
-            uint8_t* dst = reinterpret_cast<uint8_t*>(o) + ((((size_t)b * T + t0 + i) * H + h) * D) * es + pc * 16;
+            uint8_t* dst = reinterpret_cast<uint8_t*>(o) + ((((size_t)rowbase + t0 + i) * H + h) * D) * es + pc * 16;
             *reinterpret_cast<uint4*>(dst) = x;
         }
     }
@@ -352,11 +347,12 @@ __device__ __forceinline__ void ld_rows16(uint32_t (&dst)[16], const uint8_t* ti
 #pragma unroll
     for (int r = 0; r < 16; ++r) dst[r] = *reinterpret_cast<const uint32_t*>(tile + (r0 + r) * 256 + 4 * cp);
 }
-__device__ __forceinline__ uint32_t load_beta(const __nv_bfloat16* beta, int b, int T, int H, int h, int t0, int i,
-                                              bool live)
+// beta of token t0 + i of a sequence that starts at packed token `rowbase` and has T tokens
+__device__ __forceinline__ uint32_t load_beta(const __nv_bfloat16* beta, int64_t rowbase, int T, int H, int h, int t0,
+                                              int i, bool live)
 {
     const int tt = t0 + i;
-    return (live && tt < T) ? (uint32_t) * reinterpret_cast<const unsigned short*>(beta + ((size_t)b * T + tt) * H + h)
+    return (live && tt < T) ? (uint32_t) * reinterpret_cast<const unsigned short*>(beta + ((size_t)rowbase + tt) * H + h)
                             : 0u;
 }
 // Store two channels' packed fp16 rows (one 16-byte vector per channel) into a
@@ -381,7 +377,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop,
-              const float* __restrict__ gamma, float eps, int gated)
+              const float* __restrict__ gamma, float eps, int gated, const int* __restrict__ items)
 {
     using PL = Plan<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
@@ -398,12 +394,35 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int tg = t & (NG - 1);              // thread index inside its group
     const int cp = tg & 63, rq = tg >> 6;     // channel pair, 16-row quarter (loads, prologue)
     const int c = t & 127;                    // channel / TMEM row of the state steps
-    const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
-    const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
-    const int b = bh / H, h = bh % H;
-    const int NC = (T + C - 1) / C;
-    const int n0 = p * L, n1 = min(NC, n0 + L);
+    // This CTA's work: chunks [n0, n1) of head h of one sequence that starts at packed
+    // token `rowbase` and has `Tq` tokens.  Uniform batch: sequence b of B rows of T
+    // tokens, segment p of P; packed samples: one entry of the host-built item table
+    // {rowbase, Tq, n0, n1, h, sequence, slot, last}.  `slot` indexes the maps (state
+    // pass) or the start states (output pass); `last` marks the sequence's final segment.
+    int64_t rowbase;
+    int Tq, n0, n1, h, seq, slot, last;
+    if (items) {
+        const int* it = items + 8 * blockIdx.x;
+        rowbase = it[0]; Tq = it[1]; n0 = it[2]; n1 = it[3]; h = it[4]; seq = it[5]; slot = it[6]; last = it[7];
+    } else {
+        const int nseg = (MODE == MODE_STATE) ? P - 1 : P;
+        const int bh = blockIdx.x / nseg, p = blockIdx.x % nseg;
+        seq = bh / H;
+        h = bh % H;
+        rowbase = (int64_t)seq * T;
+        Tq = T;
+        const int NC = (T + C - 1) / C;
+        n0 = p * L;
+        n1 = min(NC, n0 + L);
+        slot = (MODE == MODE_STATE) ? bh * (P - 1) + p : (s_in_per_segment ? bh * P + p : bh);
+        last = p == P - 1;
+    }
     const int nk = max(0, n1 - n0);
+    // the bf16 output leaves by TMA store through a [B, T, H, 128] map that clips at the
+    // end of a row; packed samples share one row, so a chunk that runs past its sample's
+    // end is written with masked stores instead
+    const int o_b = items ? 0 : seq;
+    const int64_t o_t = items ? rowbase : 0;
 
     float* sBetaP = reinterpret_cast<float*>(sm + PL::MISC + M_BETAP);
     float* sBetaC = reinterpret_cast<float*>(sm + PL::MISC + M_BETAC);
@@ -429,31 +448,31 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *sTmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);   // this warp's lane quarter
-    // TMA of chunk n's [64][128] tiles (rows b*T + n*C ..; rows past the segment's data
+    // TMA of chunk n's [64][128] tiles (packed rows rowbase + n*C ..; rows past the sequence
     // come from the next batch row or the zero fill and are masked where they are used)
     auto tma_qk = [&](int n) {   // q (MODE_OUTPUT) and k into the Q+ / beta K+ slots of set n&1
-        const int bs = (n - n0) & 1, row = b * T + n * C;
+        const int bs = (n - n0) & 1, row = (int)(rowbase + n * C);
         mbar_arrive_expect_tx(&bars[B_TQK + bs], PL::QK_BYTES);
         if (OUT) tma_load_3d(sm + bs * PL::SET + PL::QP, &tm_q, &bars[B_TQK + bs], 0, h, row);
         tma_load_3d(sm + bs * PL::SET + PL::KP, &tm_k, &bars[B_TQK + bs], 0, h, row);
     };
     auto tma_g = [&](int n) {
         mbar_arrive_expect_tx(&bars[B_TG], 16384);
-        tma_load_3d(sm + PL::GST, &tm_g, &bars[B_TG], 0, h, b * T + n * C);
+        tma_load_3d(sm + PL::GST, &tm_g, &bars[B_TG], 0, h, (int)(rowbase + n * C));
     };
     auto tma_v = [&](int n) {
         mbar_arrive_expect_tx(&bars[B_TV], 16384);
-        tma_load_3d(sm + PL::VB, &tm_v, &bars[B_TV], 0, h, b * T + n * C);
+        tma_load_3d(sm + PL::VB, &tm_v, &bars[B_TV], 0, h, (int)(rowbase + n * C));
     };
     // gated bf16 output: chunk n's gate as two swizzled 64-channel tiles in the upper half
     // of the S^ region (free from the end of chunk n's [Y; O] MMA to chunk n+1's S^)
     auto tma_gate = [&](int n) {
         mbar_arrive_expect_tx(&bars[B_TGATE], 16384);
-        tma_load_3d(sm + PL::S + 16384, &tm_gate, &bars[B_TGATE], 0, h, b * T + n * C);
-        tma_load_3d(sm + PL::S + 24576, &tm_gate, &bars[B_TGATE], 64, h, b * T + n * C);
+        tma_load_3d(sm + PL::S + 16384, &tm_gate, &bars[B_TGATE], 0, h, (int)(rowbase + n * C));
+        tma_load_3d(sm + PL::S + 24576, &tm_gate, &bars[B_TGATE], 64, h, (int)(rowbase + n * C));
     };
     const bool gate_fused = OUT && gated && !o_f32;
-    const float* gamma_h = gamma ? gamma + (size_t)h * D : nullptr;
+    float* sGamma = reinterpret_cast<float*>(sm + PL::MISC + M_GAMMA);
 
     if (t < NG) {
         // ================= producer: state-independent work of chunk n0 + kc ==============
@@ -464,7 +483,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tma_g(n0);
             g_issued = 1;
         }
-        if (tg < C) betaR = load_beta(beta, b, T, H, h, n0 * C, tg, nk > 0);
+        if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0);
         for (int kc = 0; kc < nk; ++kc) {
             const int n = n0 + kc, t0 = n * C, bs = kc & 1;
             uint8_t* set = sm + bs * PL::SET;
@@ -482,11 +501,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 ld_rows16(gR, sm + PL::GST, 16 * rq, cp);
                 ld_rows16(kR, set + PL::KP, 16 * rq, cp);
                 if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
-                const bool full = t0 + C <= T;
+                const bool full = t0 + C <= Tq;
                 if (!full) {
 #pragma unroll
                     for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= T) gR[r] = kR[r] = qR[r] = 0u;
+                        if (t0 + 16 * rq + r >= Tq) gR[r] = kR[r] = qR[r] = 0u;
                 }
                 const float2 l2e = make_float2(kLog2e, kLog2e);
                 float2 tot = make_float2(0.f, 0.f);
@@ -499,7 +518,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tma_g(n + 1);
                     g_issued = kc + 2;
                 }
-                if (tg < C) betaR = load_beta(beta, b, T, H, h, (n + 1) * C, tg, n + 1 < n1);
+                if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
                 float2 tq4[4];
 #pragma unroll
                 for (int qb = 0; qb < 4; ++qb) tq4[qb] = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
@@ -712,7 +731,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int j = 0; j < 32; ++j) vv[j] = (col0 + cc + j == D + c) ? 1.f : 0.f;
                 } else if (S_in) {
-                    const size_t idx = s_in_per_segment ? (size_t)bh * P + p : (size_t)bh;
+                    const size_t idx = s_in_per_segment ? (size_t)slot : (size_t)seq * H + h;
                     const float4* s4 = reinterpret_cast<const float4*>(S_in + (idx * D + c) * D + col0 + cc);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -726,6 +745,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_st32(tl + TM_S + col0 + cc, vv);
             }
         }
+        if (gate_fused && tg < D) sGamma[tg] = gamma ? gamma[(size_t)h * D + tg] : 1.f;   // read after later barriers
         uint32_t betaR = 0;
         // thread NG + 32 (not the MMA issuer) requests the consumer-side TMA loads, just
         // before a barrier at which the group waits for an MMA anyway
@@ -742,7 +762,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 qk_last[1] = 1;
             }
         }
-        if (tg < C) betaR = load_beta(beta, b, T, H, h, n0 * C, tg, nk > 0);
+        if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0);
         // the master holds diag(2^{-carry}) S for channel c (log2 units; 0 before any chunk)
         float carry = 0.f;
         const bool poller = tg == 0;
@@ -752,24 +772,24 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             group_wait(&bars[B_PRO + bs], (kc >> 1) & 1, ab, poller, 2);
             // ---- previous chunk's output (staged in the free U (and Y) regions) ---------
             if (OUT && kc > 0) {
-                if (o_f32) {
+                if (o_f32 || (items && t0 > Tq)) {
                     stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
                     named_sync(2, NG);
-                    flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, t0 - C);
+                    flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, t0 - C);
                     named_sync(2, NG);
                 } else {
                     if (gate_fused) {
                         group_wait(&bars[B_TGATE], (kc - 1) & 1, ab, poller, 2);
                         stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
-                                      reinterpret_cast<float*>(sm + PL::S), gamma_h, eps);
+                                      reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
                     } else {
                         stage_o_swz(tl, q4, hg, lane, sm + PL::U);
                     }
                     fence_async_smem();
                     named_sync(2, NG);
                     if (poller) {
-                        tma_store_4d(&tm_o, sm + PL::U, 0, h, t0 - C, b);
-                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, t0 - C, b);
+                        tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + t0 - C), o_b);
+                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + t0 - C), o_b);
                         bulk_commit();
                         o_pending = true;
                     }
@@ -816,10 +836,10 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             {
                 uint32_t vR[16];
                 ld_rows16(vR, sm + PL::VB, 16 * rq, cp);
-                if (t0 + C > T) {
+                if (t0 + C > Tq) {
 #pragma unroll
                     for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= T) vR[r] = 0u;
+                        if (t0 + 16 * rq + r >= Tq) vR[r] = 0u;
                 }
                 named_sync(2, NG);
                 uint32_t pv[2][4];
@@ -841,7 +861,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     st_pair(sm + PL::VB, 2 * rq + half, cp, pv);
                 }
             }
-            if (tg < C) betaR = load_beta(beta, b, T, H, h, (n + 1) * C, tg, n + 1 < n1);
+            if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
             if (OUT) {
                 // U = T (beta V) - T Y: the first half needs no Y, so it queues behind [Y; O]
                 fence_async_smem();
@@ -972,23 +992,23 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             group_wait(&bars[B_S], kc & 1, ab, poller, 2);
         }
         if (OUT && nk > 0) {
-            if (o_f32) {
+            if (o_f32 || (items && n1 * C > Tq)) {
                 stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
                 named_sync(2, NG);
-                flush_o(sm + PL::U, tg, o, o_f32, b, T, H, h, (n1 - 1) * C);
+                flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, (n1 - 1) * C);
             } else {
                 if (gate_fused) {
                     group_wait(&bars[B_TGATE], (nk - 1) & 1, ab, poller, 2);
                     stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
-                                  reinterpret_cast<float*>(sm + PL::S), gamma_h, eps);
+                                  reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
                 } else {
                     stage_o_swz(tl, q4, hg, lane, sm + PL::U);
                 }
                 fence_async_smem();
                 named_sync(2, NG);
                 if (poller) {
-                    tma_store_4d(&tm_o, sm + PL::U, 0, h, (n1 - 1) * C, b);
-                    tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (n1 - 1) * C, b);
+                    tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + (n1 - 1) * C), o_b);
+                    tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + (n1 - 1) * C), o_b);
                     bulk_commit();
                 }
             }
@@ -1003,8 +1023,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         // ---- end of segment: write the state S = diag(2^{carry}) master -----------------
         float* dst = nullptr;
-        if (MODE == MODE_STATE) dst = maps + (size_t)(bh * (P - 1) + p) * 2 * D * D;  // [N | M]
-        else if (S_T && p == P - 1) dst = S_T + (size_t)bh * D * D;
+        if (MODE == MODE_STATE) dst = maps + (size_t)slot * 2 * D * D;  // [N | M]
+        else if (S_T && last) dst = S_T + ((size_t)seq * H + h) * D * D;
         if (dst && !*sAbort) {
             const float sc = ex2_approx(carry);
             const int col0 = hg * (NS / 2);
@@ -1053,22 +1073,33 @@ __device__ __forceinline__ void cb_stage(float* dst, const float* M, int t)
     cp_async_commit();
 }
 
+// Uniform batch (seqinfo == nullptr): sequence z = blockIdx.z has P segments, its maps at
+// (z*H + h)*(P-1) and start states at (z*H + h)*P.  Packed samples: seqinfo[3z..3z+2] =
+// {P_z, map base, start base}, head h's maps at map base + h*(P_z-1) and starts at start
+// base + h*P_z (P_z = 0: empty sample, nothing to do).
 __global__ void __launch_bounds__(CB_THREADS)
 kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
-                   float* __restrict__ starts, int H, int P)
+                   float* __restrict__ starts, int H, int P, const int* __restrict__ seqinfo)
 {
     extern __shared__ __align__(16) float csm[];
     float* sS = csm + 2 * D * CB_LD;     // [128][16]
     const int t = threadIdx.x, col0 = blockIdx.x * 16;
     const int bh = blockIdx.z * H + blockIdx.y;
     const int r = t >> 1, c8 = (t & 1) * 8;
-    const float* mp = maps + (size_t)bh * (P - 1) * 2 * D * D;   // [P-1][N | M]
+    size_t map0 = (size_t)bh * (P - 1), start0 = (size_t)bh * P;
+    if (seqinfo) {
+        P = seqinfo[3 * blockIdx.z];
+        map0 = (size_t)seqinfo[3 * blockIdx.z + 1] + (size_t)blockIdx.y * (P > 0 ? P - 1 : 0);
+        start0 = (size_t)seqinfo[3 * blockIdx.z + 2] + (size_t)blockIdx.y * P;
+        if (P == 0) return;
+    }
+    const float* mp = maps + map0 * 2 * D * D;   // [P-1][N | M]
     if (P > 1) cb_stage(csm, mp + D * D, t);
     float s[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) s[j] = S0 ? S0[((size_t)bh * D + r) * D + col0 + c8 + j] : 0.f;
     for (int p = 0; p < P; ++p) {
-        float* out = starts + ((size_t)bh * P + p) * D * D + (size_t)r * D + col0 + c8;
+        float* out = starts + (start0 + p) * D * D + (size_t)r * D + col0 + c8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) out[j] = s[j];
         if (p == P - 1) break;
@@ -1189,19 +1220,20 @@ Split split_for(int B, int T, int H, int num_sms)
 
 template <int MODE, typename TQ>
 cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int per_seg, float* maps, int P, int L,
-                        int* status, cudaStream_t s)
+                        int* status, cudaStream_t s, const int* items = nullptr, int nitems = 0)
 {
     auto kern = kda_tc_kernel<MODE, TQ>;
     const int smem = smem_bytes<MODE>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int nseg = MODE == MODE_STATE ? P - 1 : P;
-    const unsigned grid = (unsigned)(a.B * a.H * nseg);
+    const unsigned grid = items ? (unsigned)nitems : (unsigned)(a.B * a.H * nseg);
+    if (grid == 0) return cudaSuccess;
     ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
     count_launch();
     kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, mp.gate, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
-                                a.gamma, a.eps, a.gate != nullptr ? 1 : 0);
+                                a.gamma, a.eps, a.gate != nullptr ? 1 : 0, items);
     return cudaGetLastError();
 }
 
@@ -1236,11 +1268,132 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         if (e != cudaSuccess) return e;
         ProfileScope prof("kda_tc_combine", s);
         count_launch();
-        kda_combine_kernel<<<dim3(D / 16, a.H, a.B), CB_THREADS, cb_smem_bytes(), s>>>(maps, a.S0, starts, a.H, sp.P);
+        kda_combine_kernel<<<dim3(D / 16, a.H, a.B), CB_THREADS, cb_smem_bytes(), s>>>(maps, a.S0, starts, a.H, sp.P,
+                                                                                        nullptr);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return launch_pass<MODE_OUTPUT, TQ>(mp, a, starts, 1, maps, sp.P, sp.L, status, s);
+}
+
+// ---- packed samples (cu_seqlens) ------------------------------------------------------
+// Every sample gets P_i = ceil(NC_i / L) segments of L chunks, with one L for the call,
+// the smallest that keeps sum_i H * P_i within one wave of CTAs (or L = the longest
+// sample).  Items are 8 ints {rowbase, length, n0, n1, head, sample, slot, last}.
+struct VarlenPlan {
+    int L = 1;
+    std::vector<int> st_items, out_items, seqinfo;   // state pass, output pass, per sample
+    size_t n_maps = 0, n_starts = 0;
+};
+
+VarlenPlan plan_varlen(const int* cu, int n, int H, int sms)
+{
+    VarlenPlan pl;
+    int64_t work = 0;
+    int max_nc = 0;
+    for (int i = 0; i < n; ++i) {
+        const int nc = (cu[i + 1] - cu[i] + C - 1) / C;
+        work += (int64_t)nc * H;
+        max_nc = max(max_nc, nc);
+    }
+    if (max_nc > 0) {
+        int64_t L0 = (work + sms - 1) / sms;
+        int L = (int)(L0 < 1 ? 1 : L0);
+        auto ctas = [&](int Lc) {
+            int64_t m = 0;
+            for (int i = 0; i < n; ++i) m += (int64_t)H * (((cu[i + 1] - cu[i] + C - 1) / C + Lc - 1) / Lc);
+            return m;
+        };
+        while (L < max_nc && ctas(L) > sms) ++L;
+        pl.L = min(L, max_nc);
+    }
+    pl.seqinfo.resize(3 * (size_t)n);
+    for (int i = 0; i < n; ++i) {
+        const int len = cu[i + 1] - cu[i], nc = (len + C - 1) / C;
+        const int Pi = nc ? (nc + pl.L - 1) / pl.L : 0;
+        const size_t map_base = pl.n_maps, start_base = pl.n_starts;
+        pl.seqinfo[3 * i] = Pi;
+        pl.seqinfo[3 * i + 1] = (int)map_base;
+        pl.seqinfo[3 * i + 2] = (int)start_base;
+        for (int h = 0; h < H; ++h)
+            for (int p = 0; p < Pi; ++p) {
+                const int n0 = p * pl.L, n1 = min(nc, n0 + pl.L);
+                if (p < Pi - 1) {
+                    const int st[8] = {cu[i], len, n0, n1, h, i, (int)(map_base + (size_t)h * (Pi - 1) + p), 0};
+                    pl.st_items.insert(pl.st_items.end(), st, st + 8);
+                }
+                const int ot[8] = {cu[i], len, n0, n1, h, i, (int)(start_base + (size_t)h * Pi + p), p == Pi - 1};
+                pl.out_items.insert(pl.out_items.end(), ot, ot + 8);
+            }
+        pl.n_maps += (size_t)H * (Pi > 0 ? Pi - 1 : 0);
+        pl.n_starts += (size_t)H * Pi;
+    }
+    return pl;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t varlen_ws_bytes(const VarlenPlan& pl, int n)
+{
+    return a256(pl.n_maps * 2 * D * D * sizeof(float)) + a256(pl.n_starts * D * D * sizeof(float)) +
+           a256(pl.st_items.size() * sizeof(int)) + a256(pl.out_items.size() * sizeof(int)) +
+           a256(3 * (size_t)n * sizeof(int));
+}
+
+template <typename TQ>
+cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int* status, cudaStream_t s)
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const VarlenPlan pl = plan_varlen(cu, n, a.H, sms);
+    const CUtensorMapDataType dq =
+        std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    Maps mp;
+    if (!make_map(&mp.q, a.q, dq, 1, a.T, a.H) || !make_map(&mp.k, a.k, dq, 1, a.T, a.H) ||
+        !make_map(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
+        return cudaErrorInvalidValue;
+    if (a.out_t == ET_F32) mp.o = mp.q;
+    else if (!make_map_o(&mp.o, a.o, 1, a.T, a.H)) return cudaErrorInvalidValue;
+    mp.gate = mp.q;
+    char* base = reinterpret_cast<char*>(ws);
+    float* maps = reinterpret_cast<float*>(base);
+    base += a256(pl.n_maps * 2 * D * D * sizeof(float));
+    float* starts = reinterpret_cast<float*>(base);
+    base += a256(pl.n_starts * D * D * sizeof(float));
+    int* st_items = reinterpret_cast<int*>(base);
+    base += a256(pl.st_items.size() * sizeof(int));
+    int* out_items = reinterpret_cast<int*>(base);
+    base += a256(pl.out_items.size() * sizeof(int));
+    int* seqinfo = reinterpret_cast<int*>(base);
+    // pageable sources: the copies are staged before the calls return
+    cudaError_t e = cudaSuccess;
+    if (!pl.st_items.empty())
+        e = cudaMemcpyAsync(st_items, pl.st_items.data(), pl.st_items.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !pl.out_items.empty())
+        e = cudaMemcpyAsync(out_items, pl.out_items.data(), pl.out_items.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(seqinfo, pl.seqinfo.data(), pl.seqinfo.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    KdaArgs b1 = a;
+    b1.B = 1;
+    const int n_st = (int)(pl.st_items.size() / 8), n_out = (int)(pl.out_items.size() / 8);
+    if (n_st > 0) {
+        e = launch_pass<MODE_STATE, TQ>(mp, b1, nullptr, 0, maps, 0, pl.L, status, s, st_items, n_st);
+        if (e != cudaSuccess) return e;
+    }
+    if (n_out == 0) return cudaSuccess;
+    {
+        e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb_smem_bytes());
+        if (e != cudaSuccess) return e;
+        ProfileScope prof("kda_tc_combine", s);
+        count_launch();
+        kda_combine_kernel<<<dim3(D / 16, a.H, n), CB_THREADS, cb_smem_bytes(), s>>>(maps, a.S0, starts, a.H, 0,
+                                                                                    seqinfo);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pass<MODE_OUTPUT, TQ>(mp, b1, starts, 1, maps, 0, pl.L, status, s, out_items, n_out);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -1264,6 +1417,18 @@ size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms)
     const Split sp = split_for(B, T, H, num_sms);
     if (sp.P == 1) return 0;
     return (size_t)B * H * ((size_t)(sp.P - 1) * 2 + sp.P) * D * D * sizeof(float);
+}
+
+size_t kda_tc_varlen_workspace_bytes(const int* cu, int n, int H, int num_sms)
+{
+    const VarlenPlan pl = plan_varlen(cu, n, H, num_sms);
+    return varlen_ws_bytes(pl, n);
+}
+
+cudaError_t launch_kda_tc_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int* status, cudaStream_t s)
+{
+    if (a.in_t == ET_F16) return launch_varlen<__half>(a, cu, n, ws, status, s);
+    return launch_varlen<__nv_bfloat16>(a, cu, n, ws, status, s);
 }
 
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status, cudaStream_t s)

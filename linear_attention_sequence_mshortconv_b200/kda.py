@@ -27,7 +27,7 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
             "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
-            "kda_forward_gated")
+            "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size")
 
 
 class KdaError(RuntimeError):
@@ -83,6 +83,10 @@ def load_library(path: str = LIB_PATH):
         lib.kda_forward_gated.restype = I
         lib.kda_forward_gated.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_float, P, P, I, I, I, I, I, I, I,
                                           I, P, Z, P]
+        lib.kda_forward_varlen.restype = I
+        lib.kda_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
+        lib.kda_forward_varlen_workspace_size.restype = Z
+        lib.kda_forward_varlen_workspace_size.argtypes = [P, I, I, I, I, I, I, I]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -200,6 +204,53 @@ def forward_gated(q, k, v, g, beta, gate, gamma=None, eps: float = 1e-6, S0=None
                                _dev(S_T, "S_T", torch.float32), B, T, H, Dk, Dv, dt, _code(o_dtype),
                                chunk, ws_ptr, ws_bytes, _stream(stream))
     _check("kda_forward_gated", rc)
+    return o, S_T
+
+
+def _cu_array(cu_seqlens):
+    arr = (ctypes.c_int32 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
+    return arr, len(cu_seqlens) - 1
+
+
+def varlen_workspace_size(cu_seqlens, H, Dk, Dv, dtype=torch.bfloat16, chunk: int = 0, o_dtype=None) -> int:
+    arr, n = _cu_array(cu_seqlens)
+    return int(load_library().kda_forward_varlen_workspace_size(
+        ctypes.cast(arr, ctypes.c_void_p), n, H, Dk, Dv, _code(dtype), _code(o_dtype or dtype), chunk))
+
+
+def forward_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, chunk: int = 0, o=None, S_T=None,
+                   want_state: bool = True, workspace=None, stream=None, o_dtype=None):
+    """kda_forward_varlen: packed samples on one token axis, the state reset at every
+    sample start.  q, k, g: [T_total,H,Dk]; v: [T_total,H,Dv]; beta: [T_total,H];
+    cu_seqlens: host sequence of n+1 offsets (0, ..., T_total); S0: [n,H,Dk,Dv] fp32 or
+    None.  Returns (o [T_total,H,Dv], S_T [n,H,Dk,Dv] or None)."""
+    lib = load_library()
+    T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    arr, n = _cu_array(cu_seqlens)
+    if n < 0 or int(arr[n]) != T:
+        raise ValueError("cu_seqlens must end at the packed length")
+    dt = _dtype_code(q)
+    for name, t, shape in (("k", k, (T, H, Dk)), ("g", g, (T, H, Dk)), ("v", v, (T, H, Dv)), ("beta", beta, (T, H))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q's {q.dtype}")
+    o_dtype = o_dtype or (o.dtype if o is not None else q.dtype)
+    if o is None:
+        o = torch.empty((T, H, Dv), dtype=o_dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((n, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    if S0 is not None and tuple(S0.shape) != (n, H, Dk, Dv):
+        raise ValueError("S0 shape")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.kda_forward_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+                                _dev(S0, "S0", torch.float32), _dev(o, "o", o_dtype), _dev(S_T, "S_T", torch.float32),
+                                ctypes.cast(arr, ctypes.c_void_p), n, H, Dk, Dv, dt, _code(o_dtype), chunk,
+                                ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_forward_varlen", rc)
     return o, S_T
 
 
