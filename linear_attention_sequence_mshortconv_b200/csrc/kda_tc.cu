@@ -1095,18 +1095,24 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
     }
     const float* mp = maps + map0 * 2 * D * D;   // [P-1][N | M]
     if (P > 1) cb_stage(csm, mp + D * D, t);
-    float s[8];
+    float s[8], nxt[8];   // nxt: this thread's 8 values of N_p, loaded one step ahead
 #pragma unroll
     for (int j = 0; j < 8; ++j) s[j] = S0 ? S0[((size_t)bh * D + r) * D + col0 + c8 + j] : 0.f;
+    auto load_n = [&](int p) {
+        const float4* n4 = reinterpret_cast<const float4*>(mp + (size_t)p * 2 * D * D + (size_t)r * D + col0 + c8);
+        const float4 a = n4[0], b = n4[1];
+        nxt[0] = a.x; nxt[1] = a.y; nxt[2] = a.z; nxt[3] = a.w; nxt[4] = b.x; nxt[5] = b.y; nxt[6] = b.z; nxt[7] = b.w;
+    };
+    if (P > 1) load_n(0);
     for (int p = 0; p < P; ++p) {
-        float* out = starts + (start0 + p) * D * D + (size_t)r * D + col0 + c8;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = s[j];
+        float4* out = reinterpret_cast<float4*>(starts + (start0 + p) * D * D + (size_t)r * D + col0 + c8);
+        out[0] = make_float4(s[0], s[1], s[2], s[3]);
+        out[1] = make_float4(s[4], s[5], s[6], s[7]);
         if (p == P - 1) break;
-        const float* Nm = mp + (size_t)p * 2 * D * D;
         float acc[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = Nm[(size_t)r * D + col0 + c8 + j];
+        for (int j = 0; j < 8; ++j) acc[j] = nxt[j];
+        if (p + 1 < P - 1) load_n(p + 1);        // in flight during this step
         __syncthreads();                         // sS and the other buffer are free
 #pragma unroll
         for (int j = 0; j < 8; ++j) sS[r * 16 + c8 + j] = s[j];
