@@ -484,28 +484,22 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             g_issued = 1;
         }
         if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0);
+        uint32_t gP[16];     // this chunk's g rows, kept from part 1 to part 2 of the prologue
         for (int kc = 0; kc < nk; ++kc) {
             const int n = n0 + kc, t0 = n * C, bs = kc & 1;
             uint8_t* set = sm + bs * PL::SET;
             const uint32_t sset = sbase + bs * PL::SET;
-            // buffer set bs is free once the consumer is done with chunk kc - 2 (its K- and
-            // T tiles); this chunk's q, k (in the set) and g (staging) have landed
-            if (tg == 0) {
-                if (kc >= 2) thread_wait(&bars[B_EMPTY + bs], ((kc >> 1) - 1) & 1, ab);
-                thread_wait(&bars[B_TQK + bs], (kc >> 1) & 1, ab);
-            }
+            // ---- prologue, part 1: g of this chunk (staging) -> cumulative log-decay ------
+            // (needs only the g tile, so it runs before the wait for the buffer set)
             group_wait(&bars[B_TG], kc & 1, ab, tg == 0, 1);
-            // ---- prologue: cumulative log-decay, beta K+, Q+, K- tiles (in place) -------
             {
-                uint32_t gR[16], kR[16], qR[16];
+                uint32_t gR[16];
                 ld_rows16(gR, sm + PL::GST, 16 * rq, cp);
-                ld_rows16(kR, set + PL::KP, 16 * rq, cp);
-                if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
                 const bool full = t0 + C <= Tq;
                 if (!full) {
 #pragma unroll
                     for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= Tq) gR[r] = kR[r] = qR[r] = 0u;
+                        if (t0 + 16 * rq + r >= Tq) gR[r] = 0u;
                 }
                 const float2 l2e = make_float2(kLog2e, kLog2e);
                 float2 tot = make_float2(0.f, 0.f);
@@ -513,21 +507,42 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int r = 0; r < 16; ++r) tot = __ffma2_rn(in2(gR[r], (const __nv_bfloat16*)nullptr), l2e, tot);
                 *reinterpret_cast<float2*>(sTot + rq * D + 2 * cp) = tot;
                 if (tg < C) sBetaP[tg] = __uint_as_float(betaR << 16);
-                named_sync(1, NG);   // every staged value of this chunk is in registers now
-                if (tg == 0 && n + 1 < n1 && !*sAbort) {
-                    tma_g(n + 1);
-                    g_issued = kc + 2;
-                }
-                if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) gP[r] = gR[r];
+            }
+            named_sync(1, NG);   // the g tile is in registers: the next chunk's may land
+            if (tg == 0 && n + 1 < n1 && !*sAbort) {
+                tma_g(n + 1);
+                g_issued = kc + 2;
+            }
+            if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
+            float2 r2, bC, run;
+            {
                 float2 tq4[4];
 #pragma unroll
                 for (int qb = 0; qb < 4; ++qb) tq4[qb] = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
-                const float2 r2 = __fadd2_rn(tq4[0], tq4[1]);                  // b at row 31
-                const float2 bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));  // b at row 63
-                float2 run = make_float2(-r2.x, -r2.y);                        // running b - r
+                r2 = __fadd2_rn(tq4[0], tq4[1]);                     // b at row 31
+                bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));     // b at row 63
+                run = make_float2(-r2.x, -r2.y);                     // running b - r
 #pragma unroll
                 for (int qb = 0; qb < 3; ++qb)
                     if (qb < rq) run = __fadd2_rn(run, tq4[qb]);
+            }
+            // ---- part 2: buffer set bs is free once the consumer is done with chunk kc - 2
+            // (its K- and T tiles, and r, b_C); this chunk's q, k have landed in the set -----
+            if (tg == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + bs], ((kc >> 1) - 1) & 1, ab);
+            group_wait(&bars[B_TQK + bs], (kc >> 1) & 1, ab, tg == 0, 1);
+            {
+                uint32_t kR[16], qR[16];
+                const uint32_t (&gR)[16] = gP;
+                ld_rows16(kR, set + PL::KP, 16 * rq, cp);
+                if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
+                if (t0 + C > Tq) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r)
+                        if (t0 + 16 * rq + r >= Tq) kR[r] = qR[r] = 0u;
+                }
+                const float2 l2e = make_float2(kLog2e, kLog2e);
                 if (rq == 0) {
                     sRB[bs * D + 2 * cp] = make_float2(r2.x, bC.x);
                     sRB[bs * D + 2 * cp + 1] = make_float2(r2.y, bC.y);
