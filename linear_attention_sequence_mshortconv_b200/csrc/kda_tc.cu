@@ -701,32 +701,66 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 st_shared_b32(Tt + cmT(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
             }
             named_sync(1, NT / 2);
-            // block diagonal d: warp (block J, 8-column half) computes
-            //   X = sum_{K=J}^{I-1} A_IK T_KJ  and  T_IJ = -T_II X   (I = J + d)
-            for (int d = 1; d < 4; ++d) {
-                if (w < 2 * (4 - d)) {
-                    const int J = w >> 1, I = J + d, N0 = 16 * J + 8 * (w & 1);
-                    const int g = lane >> 2, q = lane & 3;
-                    const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
-                    float x[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int K = J; K < I; ++K) {
-                        uint32_t aA[4], bT[2];
-                        ldsm_x4(aA, Ah + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
-                        ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
-                        mma16816(x, aA, bT);
-                    }
-                    st_shared_b32(scr + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
-                    st_shared_b32(scr + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
-                    __syncwarp();
-                    uint32_t bX[2], aT[4];
-                    ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
-                    ldsm_x4(aT, Tt + cmT(16 * I + (lane & 15), 16 * I + 8 * (lane >> 4)));
-                    float tt[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma16816(tt, aT, bX);
+            // off-diagonal blocks by halves of the matrix (each warp: one 8-column half of one
+            // 16x16 block; X products through per-warp fp16 scratch):
+            //   level 1: T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)
+            //   level 2: X_IJ = sum_{K=J}^{1} A_IK T_KJ  (I = 2, 3; J = 0, 1), then
+            //            T_IJ = -sum_{K=2}^{I} T_IK X_KJ
+            {
+                const int g = lane >> 2, q = lane & 3, half = w & 1;
+                const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
+                auto scr_of = [&](int wx) { return sbase + PL::MISC + M_XS + 512 * wx; };
+                auto put_x = [&](uint32_t dst, const float (&x)[4]) {
+                    st_shared_b32(dst + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
+                    st_shared_b32(dst + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
+                };
+                auto put_t = [&](int I, int N0, const float (&tt)[4]) {
                     st_shared_b32(Tt + cmT(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
                     st_shared_b32(Tt + cmT(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
+                };
+                auto a_frag = [&](uint32_t (&fr)[4], uint32_t base, int I, int K, bool isT) {
+                    if (isT) ldsm_x4(fr, base + cmT(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
+                    else ldsm_x4(fr, base + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
+                };
+                if (w < 4) {   // level 1
+                    const int I = (w >> 1) ? 3 : 1, J = I - 1, N0 = 16 * J + 8 * half;
+                    uint32_t aA[4], bT[2], bX[2], aT[4];
+                    float x[4] = {0.f, 0.f, 0.f, 0.f}, tt[4] = {0.f, 0.f, 0.f, 0.f};
+                    a_frag(aA, Ah, I, J, false);
+                    ldsm_x2_t(bT, Tt + cmT(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
+                    mma16816(x, aA, bT);
+                    put_x(scr, x);
+                    __syncwarp();
+                    ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+                    a_frag(aT, Tt, I, I, true);
+                    mma16816(tt, aT, bX);
+                    put_t(I, N0, tt);
                 }
-                named_sync(1, NT / 2);
+                named_sync(1, NG);
+                // level 2, X: warp w -> block (I, J) = (2 + (w >> 2), (w >> 1) & 1), half w & 1
+                const int I2 = 2 + (w >> 2), J2 = (w >> 1) & 1, N2 = 16 * J2 + 8 * half;
+                {
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int K = J2; K < 2; ++K) {
+                        uint32_t aA[4], bT[2];
+                        a_frag(aA, Ah, I2, K, false);
+                        ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N2));
+                        mma16816(x, aA, bT);
+                    }
+                    put_x(scr, x);
+                }
+                named_sync(1, NG);
+                // level 2, T: the same (I, J, half); X_KJ half was written by warp 4(K-2) + 2J + half
+                {
+                    float tt[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int K = 2; K <= I2; ++K) {
+                        uint32_t aT[4], bX[2];
+                        a_frag(aT, Tt, I2, K, true);
+                        ldsm_x2_t(bX, scr_of(4 * (K - 2) + 2 * J2 + half) + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+                        mma16816(tt, aT, bX);
+                    }
+                    put_t(I2, N2, tt);
+                }
             }
             fence_async_smem();
             named_sync(1, NG);
