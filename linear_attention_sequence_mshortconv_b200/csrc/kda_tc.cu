@@ -819,31 +819,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int n = n0 + kc, t0 = n * C, bs = kc & 1;
             const uint32_t sset = sbase + bs * PL::SET;
             group_wait(&bars[B_PRO + bs], (kc >> 1) & 1, ab, poller, 2);
-            // ---- previous chunk's output (staged in the free U (and Y) regions) ---------
-            if (OUT && kc > 0) {
-                if (o_f32 || (items && t0 > Tq)) {
-                    stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
-                    named_sync(2, NG);
-                    flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, t0 - C);
-                    named_sync(2, NG);
-                } else {
-                    if (gate_fused) {
-                        group_wait(&bars[B_TGATE], (kc - 1) & 1, ab, poller, 2);
-                        stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
-                                      reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
-                    } else {
-                        stage_o_swz(tl, q4, hg, lane, sm + PL::U);
-                    }
-                    fence_async_smem();
-                    named_sync(2, NG);
-                    if (poller) {
-                        tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + t0 - C), o_b);
-                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + t0 - C), o_b);
-                        bulk_commit();
-                        o_pending = true;
-                    }
-                }
-            }
             // ---- S^ = 2^{r + carry} master ------------------------------------------------
             {
                 const float2 rb = sRB[bs * D + c];
@@ -1039,26 +1014,30 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 v_issued = kc + 2;
             }
             group_wait(&bars[B_S], kc & 1, ab, poller, 2);
-        }
-        if (OUT && nk > 0) {
-            if (o_f32 || (items && n1 * C > Tq)) {
-                stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
-                named_sync(2, NG);
-                flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, (n1 - 1) * C);
-            } else {
-                if (gate_fused) {
-                    group_wait(&bars[B_TGATE], (nk - 1) & 1, ab, poller, 2);
-                    stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
-                                  reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
+            // ---- this chunk's output, staged in the free U (and Y) regions; done here, at
+            // the end of the chunk, it overlaps the wait for the producer's next tiles -----
+            if (OUT) {
+                if (o_f32 || (items && t0 + C > Tq)) {
+                    stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
+                    named_sync(2, NG);
+                    flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, t0);
+                    named_sync(2, NG);
                 } else {
-                    stage_o_swz(tl, q4, hg, lane, sm + PL::U);
-                }
-                fence_async_smem();
-                named_sync(2, NG);
-                if (poller) {
-                    tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + (n1 - 1) * C), o_b);
-                    tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + (n1 - 1) * C), o_b);
-                    bulk_commit();
+                    if (gate_fused) {
+                        group_wait(&bars[B_TGATE], kc & 1, ab, poller, 2);
+                        stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
+                                      reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
+                    } else {
+                        stage_o_swz(tl, q4, hg, lane, sm + PL::U);
+                    }
+                    fence_async_smem();
+                    named_sync(2, NG);
+                    if (poller) {
+                        tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + t0), o_b);
+                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + t0), o_b);
+                        bulk_commit();
+                        o_pending = true;
+                    }
                 }
             }
         }
