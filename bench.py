@@ -456,6 +456,42 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                           "value": w.tokens / (mg * 1e-3) / 1e6, "unit": UNIT,
                           "alg_GBps": gbytes / (mg * 1e-3) / 1e9,
                           "epilogue": "Sigmoid(gate) * RMSNorm(S_t^T q_t), fused in the output stage"})
+        # one rank's local work in a sequence-parallel run: the last of 8 time shards of
+        # the long video row (its transition, the prefix over the 7 earlier shards' maps,
+        # its output pass); the all-gather of the maps (2 MiB per rank) is not included
+        if not w.fused:
+            R = 8
+            sw = W.LONG_VIDEO.resized(T=W.LONG_VIDEO.T // R, name="long_video_shard_8_of_8")
+            si = W.make_kda_inputs(sw, device="cuda")
+            wss = kda.sp_workspace(si["q"], sw.chunk)
+            MN_all = torch.zeros((R, sw.B, sw.H, 2, sw.D, sw.D), dtype=torch.float32, device="cuda")
+            S_in = torch.empty((sw.B, sw.H, sw.D, sw.D), dtype=torch.float32, device="cuda")
+            o_s = torch.empty((sw.B, sw.T, sw.H, sw.D), dtype=sw.dtype, device="cuda")
+            S_s = torch.empty_like(S_in)
+            kda.sp_transition(si["q"], si["k"], si["v"], si["g"], si["beta"], wss, chunk=sw.chunk, MN=MN_all[R - 1])
+            MN_all[: R - 1].copy_(MN_all[R - 1].expand(R - 1, *MN_all.shape[1:]))
+
+            def sstep():
+                kda.sp_transition(si["q"], si["k"], si["v"], si["g"], si["beta"], wss, chunk=sw.chunk,
+                                  MN=MN_all[R - 1])
+                kda.sp_prefix(MN_all, R - 1, None, S_in=S_in)
+                kda.sp_output(si["q"], si["k"], si["v"], si["g"], si["beta"], S_in, wss, chunk=sw.chunk,
+                              o=o_s, S_T=S_s)
+            for _ in range(3):
+                sstep()
+            k_s = max(3, args.steps // 4)
+            kda.profile_enable(True)
+            ms_s = timed(sstep, k_s, 1) / k_s
+            kda.profile_enable(False)
+            kern = {}
+            for name in ("kda_tc_state", "kda_sp_fold", "kda_tc_combine", "kda_tc_output"):
+                r = kda.profile_collect(name)
+                if r and r[1] > 0:
+                    kern[name] = {"ms_per_step": r[0] / k_s, "launches_per_step": r[1] / k_s}
+            extra.append({"workload": sw.name, "shard_tokens": sw.T, "ranks": R, "ms_per_step": ms_s,
+                          "value": sw.T / (ms_s * 1e-3) / 1e6, "unit": UNIT + " (one rank's shard)",
+                          "alg_GBps": algorithmic_bytes(sw) / (ms_s * 1e-3) / 1e9, "kernels": kern,
+                          "excludes": "the all-gather of the ranks' maps"})
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

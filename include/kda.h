@@ -176,6 +176,67 @@ kda_status kda_forward_noalloc(const void* q, const void* k, const void* v, cons
                                int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
                                kda_dtype o_dtype, int chunk, kda_stream_t stream);
 
+/*
+ * Sequence-parallel forward: each of the B rows is cut along time into R consecutive
+ * shards, one per device (the pages run one long stream per device and name no
+ * multi-device scheme; this follows from Eq. 14 of section 3.3 being affine in the
+ * state).  Over a shard, S_out = M S_in + N with
+ *   M = prod_t (I - beta_t k_t k_t^T) Diag(alpha_t)   (latest token leftmost), [D, D]
+ *   N = the state the shard reaches from S_in = 0,    [D, D]  (state layout [Dk, Dv])
+ * A rank r runs kda_sp_transition on its shard, the ranks exchange the [N | M] blocks
+ * (an all-gather: the library does no communication), kda_sp_prefix folds shards
+ * 0..r-1 over the row's S0 into the shard's entry state, and kda_sp_output scans the
+ * shard from it.  Concatenating the ranks' o gives kda_forward's o of the whole rows;
+ * the last rank's S_T is the rows' final state.  Dk = Dv = D in {32, 64, 128}; the
+ * other arguments are as for kda_forward on the shard ([B, T_r, H, D] tensors).
+ *
+ * kda_sp_workspace_size -- bytes of device workspace kda_sp_transition and
+ *   kda_sp_output need (0 if none).  The workspace is required (the calls allocate
+ *   nothing), 256-byte aligned, and is the same buffer for both calls of a shard.
+ */
+size_t kda_sp_workspace_size(int B, int T, int H, int D, kda_dtype dtype, int chunk);
+
+/*
+ * kda_sp_transition -- this shard's affine map.
+ *   MN : [B, H, 2, D, D] fp32 (device, written): block 0 = N, block 1 = M, row-major,
+ *        so S_out[i][j] = sum_c M[i][c] S_in[c][j] + N[i][j].
+ * On the tensor-core route the per-segment maps of the shard stay in the workspace for
+ * kda_sp_output: pass that call the same workspace, unmodified, and the same q, k, v, g,
+ * beta.  T = 0 gives N = 0, M = I.  Errors: KDA_ERR_INVALID_ARG (null tensor, bad
+ * sizes), KDA_ERR_UNSUPPORTED (D, chunk, B*H > 65535), KDA_ERR_WORKSPACE (workspace null
+ * or smaller than kda_sp_workspace_size), KDA_ERR_CUDA.
+ */
+kda_status kda_sp_transition(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, float* MN, int B, int T, int H, int D,
+                             kda_dtype dtype, int chunk, void* workspace,
+                             size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_sp_prefix -- the entry state of shard r:
+ *   S_in = (M_{r-1} (... (M_0 S0 + N_0) ...) + N_{r-1})
+ *   MN_all : [R, B, H, 2, D, D] fp32 (device): every rank's kda_sp_transition result,
+ *            in rank order (may be NULL when r = 0).
+ *   S0     : [B, H, D, D] fp32 or NULL (zeros) -- the rows' initial state.
+ *   S_in   : [B, H, D, D] fp32 (device, written).
+ * Errors: KDA_ERR_INVALID_ARG (r outside [0, R), null S_in), KDA_ERR_UNSUPPORTED (D),
+ * KDA_ERR_CUDA.
+ */
+kda_status kda_sp_prefix(const float* MN_all, int R, int r, const float* S0, float* S_in,
+                         int B, int H, int D, kda_stream_t stream);
+
+/*
+ * kda_sp_output -- the scan of this shard from S_in (as kda_forward with S0 = S_in):
+ * o [B, T, H, D] in o_dtype and, if S_T is not NULL, the shard's final state.  On the
+ * tensor-core route it reads the segment maps kda_sp_transition left in the workspace
+ * (one output pass instead of a full scan); otherwise it runs the whole scan.
+ * Errors: as kda_sp_transition.
+ */
+kda_status kda_sp_output(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* S_in, void* o, float* S_T,
+                         int B, int T, int H, int D, kda_dtype dtype, kda_dtype o_dtype,
+                         int chunk, void* workspace, size_t workspace_bytes,
+                         kda_stream_t stream);
+
 /* Modalities of a packed-stream segment (section 3.4). */
 typedef enum { MSC_TEXT = 0, MSC_IMAGE = 1, MSC_VIDEO = 2 } msc_modality;
 
@@ -276,7 +337,7 @@ void kda_profile_enable(int on);
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
  * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
- * "kda_tc_output", "conv", "gate_norm". */
+ * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

@@ -80,6 +80,19 @@ cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* stat
 // Packed samples: a.B = 1, a.T = cu[n] tokens; host array cu[0..n] of sample offsets.
 size_t kda_tc_varlen_workspace_bytes(const int* cu, int n, int H, int num_sms);
 cudaError_t launch_kda_tc_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int* status, cudaStream_t s);
+// One shard of a sequence cut across devices (a.B rows of a.T tokens each).  The state
+// pass over all of the shard's P segments leaves the per-segment maps in the workspace:
+// head bh's segments 0..P-2 at maps + (bh*(P-1) + p)*2*D*D, its last segment at
+// tail + bh*2*D*D ([N | M] blocks of D x D fp32 each).  The output pass then takes the
+// shard's entry state as a.S0 and reuses those maps.
+struct TcShardMaps {
+    int P;
+    const float* maps;
+    const float* tail;
+};
+size_t kda_tc_sp_workspace_bytes(int B, int T, int H, int num_sms);
+cudaError_t launch_kda_tc_sp_state(const KdaArgs& a, void* ws, int* status, cudaStream_t s, TcShardMaps* out);
+cudaError_t launch_kda_tc_sp_output(const KdaArgs& a, void* ws, int* status, cudaStream_t s);
 
 struct ConvSeg {
     int32_t modality;

@@ -1272,33 +1272,39 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
 }
 
 template <typename TQ>
-cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
+bool build_maps(const KdaArgs& a, Maps& mp)
+{
+    const CUtensorMapDataType dq =
+        std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
+        return false;
+    if (a.out_t == ET_F32 || !a.o) mp.o = mp.q;
+    else if (!make_map_o(&mp.o, a.o, a.B, a.T, a.H)) return false;
+    if (a.gate && a.out_t == ET_BF16) return make_map_gate(&mp.gate, a.gate, a.B, a.T, a.H);
+    mp.gate = mp.q;
+    return true;
+}
+
+int sm_count()
 {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const Split sp = split_for(a.B, a.T, a.H, sms);
-    const CUtensorMapDataType dq =
-        std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    Maps mp;
-    if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
-        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
-        !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
-        return cudaErrorInvalidValue;
-    if (a.out_t == ET_F32) mp.o = mp.q;
-    else if (!make_map_o(&mp.o, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
-    if (a.gate && a.out_t == ET_BF16) {
-        if (!make_map_gate(&mp.gate, a.gate, a.B, a.T, a.H)) return cudaErrorInvalidValue;
-    } else {
-        mp.gate = mp.q;
-    }
+    return sms;
+}
+
+// Start states of every segment from a.S0 and the maps of segments 0..P-2 (uniform
+// layout, head bh's at bh*(P-1)), then the output pass.
+template <typename TQ>
+cudaError_t combine_output(const Maps& mp, const KdaArgs& a, const Split& sp, float* maps, float* starts,
+                           int* status, cudaStream_t s)
+{
     if (sp.P == 1) return launch_pass<MODE_OUTPUT, TQ>(mp, a, a.S0, 0, nullptr, 1, sp.L, status, s);
-    float* maps = reinterpret_cast<float*>(ws);
-    float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
-    cudaError_t e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, sp.P, sp.L, status, s);
-    if (e != cudaSuccess) return e;
     {
-        e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb_smem_bytes());
+        cudaError_t e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             cb_smem_bytes());
         if (e != cudaSuccess) return e;
         ProfileScope prof("kda_tc_combine", s);
         count_launch();
@@ -1308,6 +1314,85 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         if (e != cudaSuccess) return e;
     }
     return launch_pass<MODE_OUTPUT, TQ>(mp, a, starts, 1, maps, sp.P, sp.L, status, s);
+}
+
+template <typename TQ>
+cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
+{
+    const Split sp = split_for(a.B, a.T, a.H, sm_count());
+    Maps mp;
+    if (!build_maps<TQ>(a, mp)) return cudaErrorInvalidValue;
+    float* maps = reinterpret_cast<float*>(ws);
+    float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
+    if (sp.P > 1) {
+        const cudaError_t e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, sp.P, sp.L, status, s);
+        if (e != cudaSuccess) return e;
+    }
+    return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
+}
+
+// ---- one shard of a sequence cut across devices -----------------------------------------
+// The state pass runs every segment of the shard, the last one included: segments
+// 0..P-2 write their maps in the uniform layout (the output pass reads them), the last
+// one into a tail slot per head after them.  Workspace: maps [B*H*P][N | M], start
+// states [B*H*P][D][D], the item table.
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct SpLayout {
+    Split sp;
+    size_t maps_bytes, starts_bytes, items_bytes;
+    size_t total() const { return maps_bytes + starts_bytes + items_bytes; }
+};
+
+SpLayout sp_layout(int B, int T, int H, int sms)
+{
+    SpLayout l;
+    l.sp = split_for(B, T, H, sms);
+    const size_t bhp = (size_t)B * H * l.sp.P;
+    l.maps_bytes = a256(bhp * 2 * D * D * sizeof(float));
+    l.starts_bytes = a256(bhp * D * D * sizeof(float));
+    l.items_bytes = a256(bhp * 8 * sizeof(int));
+    return l;
+}
+
+template <typename TQ>
+cudaError_t launch_sp_state(const KdaArgs& a, void* ws, int* status, cudaStream_t s, TcShardMaps* out)
+{
+    const SpLayout l = sp_layout(a.B, a.T, a.H, sm_count());
+    const int P = l.sp.P, L = l.sp.L, NC = (a.T + C - 1) / C, BH = a.B * a.H;
+    Maps mp;
+    if (!build_maps<TQ>(a, mp)) return cudaErrorInvalidValue;
+    float* maps = reinterpret_cast<float*>(ws);
+    int* items = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + l.maps_bytes + l.starts_bytes);
+    std::vector<int> it;
+    it.reserve((size_t)BH * P * 8);
+    for (int b = 0; b < a.B; ++b)
+        for (int h = 0; h < a.H; ++h)
+            for (int p = 0; p < P; ++p) {
+                const int bh = b * a.H + h;
+                const int slot = p < P - 1 ? bh * (P - 1) + p : BH * (P - 1) + bh;
+                const int e[8] = {b * a.T, a.T, p * L, min(NC, (p + 1) * L), h, b, slot, p == P - 1};
+                it.insert(it.end(), e, e + 8);
+            }
+    // pageable source: the copy is staged before the call returns
+    cudaError_t e = cudaMemcpyAsync(items, it.data(), it.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, P, L, status, s, items, BH * P);
+    out->P = P;
+    out->maps = maps;
+    out->tail = maps + (size_t)BH * (P - 1) * 2 * D * D;
+    return e;
+}
+
+template <typename TQ>
+cudaError_t launch_sp_output(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
+{
+    const SpLayout l = sp_layout(a.B, a.T, a.H, sm_count());
+    Maps mp;
+    if (!build_maps<TQ>(a, mp)) return cudaErrorInvalidValue;
+    float* maps = reinterpret_cast<float*>(ws);
+    float* starts = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + l.maps_bytes);
+    return combine_output<TQ>(mp, a, l.sp, maps, starts, status, s);
 }
 
 // ---- packed samples (cu_seqlens) ------------------------------------------------------
@@ -1365,8 +1450,6 @@ VarlenPlan plan_varlen(const int* cu, int n, int H, int sms)
     return pl;
 }
 
-size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
-
 size_t varlen_ws_bytes(const VarlenPlan& pl, int n)
 {
     return a256(pl.n_maps * 2 * D * D * sizeof(float)) + a256(pl.n_starts * D * D * sizeof(float)) +
@@ -1377,10 +1460,7 @@ size_t varlen_ws_bytes(const VarlenPlan& pl, int n)
 template <typename TQ>
 cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int* status, cudaStream_t s)
 {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const VarlenPlan pl = plan_varlen(cu, n, a.H, sms);
+    const VarlenPlan pl = plan_varlen(cu, n, a.H, sm_count());
     const CUtensorMapDataType dq =
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     Maps mp;
@@ -1463,6 +1543,24 @@ cudaError_t launch_kda_tc_varlen(const KdaArgs& a, const int* cu, int n, void* w
 {
     if (a.in_t == ET_F16) return launch_varlen<__half>(a, cu, n, ws, status, s);
     return launch_varlen<__nv_bfloat16>(a, cu, n, ws, status, s);
+}
+
+size_t kda_tc_sp_workspace_bytes(int B, int T, int H, int num_sms)
+{
+    if (B < 1 || T < 1) return 0;
+    return sp_layout(B, T, H, num_sms).total();
+}
+
+cudaError_t launch_kda_tc_sp_state(const KdaArgs& a, void* ws, int* status, cudaStream_t s, TcShardMaps* out)
+{
+    if (a.in_t == ET_F16) return launch_sp_state<__half>(a, ws, status, s, out);
+    return launch_sp_state<__nv_bfloat16>(a, ws, status, s, out);
+}
+
+cudaError_t launch_kda_tc_sp_output(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
+{
+    if (a.in_t == ET_F16) return launch_sp_output<__half>(a, ws, status, s);
+    return launch_sp_output<__nv_bfloat16>(a, ws, status, s);
 }
 
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status, cudaStream_t s)

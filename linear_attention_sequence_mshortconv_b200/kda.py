@@ -27,7 +27,8 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_forward", "mshortconv_forward", "kda_mshortconv_workspace_size",
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
             "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
-            "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size")
+            "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size",
+            "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output")
 
 
 class KdaError(RuntimeError):
@@ -87,6 +88,14 @@ def load_library(path: str = LIB_PATH):
         lib.kda_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
         lib.kda_forward_varlen_workspace_size.restype = Z
         lib.kda_forward_varlen_workspace_size.argtypes = [P, I, I, I, I, I, I, I]
+        lib.kda_sp_workspace_size.restype = Z
+        lib.kda_sp_workspace_size.argtypes = [I, I, I, I, I, I]
+        lib.kda_sp_transition.restype = I
+        lib.kda_sp_transition.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P]
+        lib.kda_sp_prefix.restype = I
+        lib.kda_sp_prefix.argtypes = [P, I, I, P, P, I, I, I, P]
+        lib.kda_sp_output.restype = I
+        lib.kda_sp_output.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -251,6 +260,89 @@ def forward_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, chunk: int = 0, o=N
                                 ctypes.cast(arr, ctypes.c_void_p), n, H, Dk, Dv, dt, _code(o_dtype), chunk,
                                 ws_ptr, ws_bytes, _stream(stream))
     _check("kda_forward_varlen", rc)
+    return o, S_T
+
+
+def _shard_inputs(q, k, v, g, beta):
+    B, T, H, D = q.shape
+    for name, t, shape in (("k", k, (B, T, H, D)), ("g", g, (B, T, H, D)), ("v", v, (B, T, H, D)),
+                           ("beta", beta, (B, T, H))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q's {q.dtype}")
+    return B, T, H, D, _dtype_code(q)
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+
+
+def sp_workspace_size(B, T, H, D, dtype=torch.bfloat16, chunk: int = 0) -> int:
+    """Bytes of the workspace one shard's kda_sp_transition / kda_sp_output share."""
+    return int(load_library().kda_sp_workspace_size(B, T, H, D, _code(dtype), chunk))
+
+
+def sp_workspace(q, chunk: int = 0):
+    """A workspace tensor for the shard q belongs to (None if the shard needs none)."""
+    B, T, H, D = q.shape
+    n = sp_workspace_size(B, T, H, D, q.dtype, chunk)
+    return torch.empty(n, dtype=torch.uint8, device=q.device) if n else None
+
+
+def sp_transition(q, k, v, g, beta, workspace, *, chunk: int = 0, MN=None, stream=None):
+    """kda_sp_transition: the shard's affine map S_out = M S_in + N as MN [B,H,2,D,D]
+    fp32 (block 0 = N, block 1 = M).  `workspace` (see sp_workspace) must be passed
+    unchanged to sp_output for the same shard."""
+    lib = load_library()
+    B, T, H, D, dt = _shard_inputs(q, k, v, g, beta)
+    if MN is None:
+        MN = torch.empty((B, H, 2, D, D), dtype=torch.float32, device=q.device)
+    ws_ptr, ws_bytes = _ws(workspace)
+    rc = lib.kda_sp_transition(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+                               _dev(MN, "MN", torch.float32), B, T, H, D, dt, chunk, ws_ptr, ws_bytes,
+                               _stream(stream))
+    _check("kda_sp_transition", rc)
+    return MN
+
+
+def sp_prefix(MN_all, r: int, S0=None, *, S_in=None, stream=None):
+    """kda_sp_prefix: entry state [B,H,D,D] of shard r from the ranks' maps
+    MN_all [R,B,H,2,D,D] (rank order) and the rows' S0 (None = zeros)."""
+    lib = load_library()
+    R, B, H, two, D, D2 = MN_all.shape
+    if two != 2 or D2 != D:
+        raise ValueError("MN_all must be [R,B,H,2,D,D]")
+    if S0 is not None and tuple(S0.shape) != (B, H, D, D):
+        raise ValueError("S0 shape")
+    if S_in is None:
+        S_in = torch.empty((B, H, D, D), dtype=torch.float32, device=MN_all.device)
+    rc = lib.kda_sp_prefix(_dev(MN_all, "MN_all", torch.float32), R, int(r), _dev(S0, "S0", torch.float32),
+                           _dev(S_in, "S_in", torch.float32), B, H, D, _stream(stream))
+    _check("kda_sp_prefix", rc)
+    return S_in
+
+
+def sp_output(q, k, v, g, beta, S_in, workspace, *, chunk: int = 0, o=None, S_T=None,
+              want_state: bool = True, o_dtype=None, stream=None):
+    """kda_sp_output: the shard's scan from S_in, reusing what sp_transition left in
+    `workspace`.  Returns (o [B,T,H,D], S_T or None)."""
+    lib = load_library()
+    B, T, H, D, dt = _shard_inputs(q, k, v, g, beta)
+    o_dtype = o_dtype or (o.dtype if o is not None else q.dtype)
+    if o is None:
+        o = torch.empty((B, T, H, D), dtype=o_dtype, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+    if S_in is not None and tuple(S_in.shape) != (B, H, D, D):
+        raise ValueError("S_in shape")
+    ws_ptr, ws_bytes = _ws(workspace)
+    rc = lib.kda_sp_output(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+                           _dev(S_in, "S_in", torch.float32), _dev(o, "o", o_dtype), _dev(S_T, "S_T", torch.float32),
+                           B, T, H, D, dt, _code(o_dtype), chunk, ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_sp_output", rc)
     return o, S_T
 
 

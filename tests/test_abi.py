@@ -70,6 +70,25 @@ def test_gated_forward_rejects_bad_arguments(lib):
     assert lib.kda_forward_gated(d, d, d, d, d, P, P, P, 1e-6, d, P, 0, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 0
 
 
+def test_sequence_parallel_calls_reject_bad_arguments(lib):
+    P = None
+    d = ctypes.c_void_p(256)   # never dereferenced: validation fails first
+    # transition: unsupported head width, null MN with work to do, no workspace, empty batch
+    assert lib.kda_sp_transition(d, d, d, d, d, d, 1, 8, 1, 48, 1, 0, P, 0, P) == 2
+    assert lib.kda_sp_transition(d, d, d, d, d, P, 1, 8, 1, 32, 1, 0, P, 0, P) == 1
+    assert lib.kda_sp_transition(d, d, d, d, d, d, 1, 8, 1, 32, 1, 0, P, 0, P) == 5
+    assert lib.kda_sp_transition(d, d, d, d, d, d, 0, 8, 1, 32, 1, 0, P, 0, P) == 0
+    # prefix: rank outside [0, R), null output, unsupported head width
+    assert lib.kda_sp_prefix(d, 2, 2, P, d, 1, 1, 32, P) == 1
+    assert lib.kda_sp_prefix(d, 2, -1, P, d, 1, 1, 32, P) == 1
+    assert lib.kda_sp_prefix(d, 2, 1, P, P, 1, 1, 32, P) == 1
+    assert lib.kda_sp_prefix(d, 2, 1, P, d, 1, 1, 48, P) == 2
+    # output: bad output dtype, chunk not in {16, 32, 64}
+    assert lib.kda_sp_output(d, d, d, d, d, P, d, P, 1, 8, 1, 32, 1, 9, 0, P, 0, P) == 1
+    assert lib.kda_sp_output(d, d, d, d, d, P, d, P, 1, 8, 1, 32, 1, 1, 24, P, 0, P) == 2
+    assert lib.kda_sp_workspace_size(1, 8, 1, 48, 1, 0) == 0
+
+
 def test_conv_rejects_bad_segment_tables(lib):
     segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
     dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
