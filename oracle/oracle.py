@@ -19,6 +19,10 @@ passages of the Chimera paper it follows, is stated in that file's header:
 * ``gated_rmsnorm`` / ``kda_forward_gated``: the output side of Eq. 15 (section 3.3),
   Sigmoid(gate) * RMSNorm(S_t^T q_t) per (token, head), before the output projection
   W_o (numpy, fp64).
+* ``kda_backward``: the reverse-mode derivative of the token recurrence of Eq. 14 with
+  the readout of Eq. 15 (the pages give only the forward; the paper trains with it).
+  Plain reverse sweep over the tokens in fp64 (numpy), from the states of a forward
+  sweep.
 """
 from __future__ import annotations
 
@@ -295,6 +299,72 @@ def kda_forward_gated(q, k, v, g, beta, gate, gamma=None, eps=1e-6, S0=None, *, 
     """kda_forward followed by gated_rmsnorm of its readout; returns (y, S_T)."""
     o, S_T = kda_forward(q, k, v, g, beta, S0, pairs=pairs, nthreads=nthreads)
     return gated_rmsnorm(o, gate, gamma, eps), S_T
+
+
+def kda_backward(q, k, v, g, beta, do, S0=None, dS_T=None, *, block=64):
+    """Gradients of L = sum(do * o) + sum(dS_T * S_T) through the scan of kda_forward.
+
+    q, k, g: [B,T,H,Dk]; v, do: [B,T,H,Dv]; beta: [B,T,H]; S0, dS_T: [B,H,Dk,Dv] or
+    None (zeros).  Inputs are read at their stored precision.  Returns fp64
+    (dq, dk, dv, dg, dbeta, dS0) with the shapes of q, k, v, g, beta, S0.
+
+    Per token t, with a = exp(g_t), X = Diag(a) S_{t-1}, w = v_t - X^T k_t:
+      S_t = X + beta_t k_t w^T,   o_t = S_t^T q_t.
+    The reverse sweep carries G = dL/dS_t (starting from dS_T):
+      G      += q_t do_t^T                     (readout)
+      dq_t    = S_t do_t
+      dv_t    = beta_t G^T k_t
+      dbeta_t = k_t^T G w
+      dk_t    = beta_t (G w - X G^T k_t)
+      dX      = G - beta_t k_t (k_t^T G)
+      dg_t    = a * rowsum(dX * S_{t-1})       (dX/dg through X = Diag(e^g) S_{t-1})
+      G       = Diag(a) dX                     (dL/dS_{t-1})
+    and dS0 = G after token 1.  States are kept every `block` tokens and the ones in
+    between recomputed by the same forward steps."""
+    Q, K, V, Gl, Bt, dO = (_to_f64(x) for x in (q, k, v, g, beta, do))
+    B, T, H, Dk = Q.shape
+    Dv = V.shape[-1]
+    s0 = None if S0 is None else _to_f64(S0)
+    dst = None if dS_T is None else _to_f64(dS_T)
+    dq, dk, dg = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(Gl)
+    dv, dbeta = np.zeros_like(V), np.zeros_like(Bt)
+    dS0 = np.zeros((B, H, Dk, Dv))
+
+    def step(S, b, t, h):
+        X = np.exp(Gl[b, t, h])[:, None] * S
+        kk = K[b, t, h]
+        return X + Bt[b, t, h] * np.outer(kk, V[b, t, h] - kk @ X)
+
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((Dk, Dv)) if s0 is None else s0[b, h].copy()
+            ckpt = {}
+            for t in range(T):
+                if t % block == 0:
+                    ckpt[t] = S.copy()
+                S = step(S, b, t, h)
+            G = np.zeros((Dk, Dv)) if dst is None else dst[b, h].copy()
+            for t0 in reversed(range(0, T, block)):
+                states = [ckpt[t0]]            # states[i] = S_{t0 + i - 1}, the state before token t0+i
+                for t in range(t0, min(T, t0 + block)):
+                    states.append(step(states[-1], b, t, h))
+                for t in reversed(range(t0, min(T, t0 + block))):
+                    S_prev, S_t = states[t - t0], states[t - t0 + 1]
+                    a = np.exp(Gl[b, t, h])
+                    kk, bt = K[b, t, h], Bt[b, t, h]
+                    X = a[:, None] * S_prev
+                    w = V[b, t, h] - kk @ X
+                    G = G + np.outer(Q[b, t, h], dO[b, t, h])
+                    dq[b, t, h] = S_t @ dO[b, t, h]
+                    Gk = G.T @ kk
+                    dv[b, t, h] = bt * Gk
+                    dbeta[b, t, h] = Gk @ w
+                    dk[b, t, h] = bt * (G @ w - X @ Gk)
+                    dX = G - bt * np.outer(kk, Gk)
+                    dg[b, t, h] = a * np.sum(dX * S_prev, axis=1)
+                    G = a[:, None] * dX
+            dS0[b, h] = G
+    return dq, dk, dv, dg, dbeta, dS0
 
 
 def _to_f64(a):
