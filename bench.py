@@ -492,6 +492,32 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                           "value": sw.T / (ms_s * 1e-3) / 1e6, "unit": UNIT + " (one rank's shard)",
                           "alg_GBps": algorithmic_bytes(sw) / (ms_s * 1e-3) / 1e9, "kernels": kern,
                           "excludes": "the all-gather of the ranks' maps"})
+        # the backward of the headline workload (kda_backward: fp32 gradients of q, k, v,
+        # g, beta, S0 for a random dL/do); algorithmic bytes: the forward's inputs and do
+        # read once, the fp32 gradients written once
+        if not w.fused:
+            inp_b = W.make_kda_inputs(w, device="cuda")
+            do_b = torch.randn(w.B, w.T, w.H, w.D, generator=torch.Generator().manual_seed(8)).to(w.dtype).cuda()
+            f32 = dict(dtype=torch.float32, device="cuda")
+            outs = (torch.empty((w.B, w.T, w.H, w.D), **f32), torch.empty((w.B, w.T, w.H, w.D), **f32),
+                    torch.empty((w.B, w.T, w.H, w.D), **f32), torch.empty((w.B, w.T, w.H, w.D), **f32),
+                    torch.empty((w.B, w.T, w.H), **f32), torch.empty((w.B, w.H, w.D, w.D), **f32))
+            wsb_b = torch.empty(max(kda.backward_workspace_size(w.B, w.T, w.H, w.D, w.D), 1), dtype=torch.uint8,
+                                device="cuda")
+
+            def bstep():
+                kda.backward(inp_b["q"], inp_b["k"], inp_b["v"], inp_b["g"], inp_b["beta"], do_b,
+                             workspace=wsb_b, out=outs)
+            for _ in range(3):
+                bstep()
+            k_b = 5
+            mb = timed(bstep, k_b, 1) / k_b
+            esz = torch.tensor([], dtype=w.dtype).element_size()
+            bbytes = algorithmic_bytes(w) + w.B * w.T * w.H * (4 * w.D * 4 + 4)
+            extra.append({"workload": w.name + "_backward", "ms_per_step": mb,
+                          "value": w.tokens / (mb * 1e-3) / 1e6, "unit": UNIT,
+                          "alg_GBps": bbytes / (mb * 1e-3) / 1e9, "alg_bytes": bbytes,
+                          "path": "fp32 CUDA cores, one CTA per (b, h, 32 value columns)"})
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -237,6 +237,32 @@ kda_status kda_sp_output(const void* q, const void* k, const void* v, const void
                          int chunk, void* workspace, size_t workspace_bytes,
                          kda_stream_t stream);
 
+/*
+ * kda_backward -- gradients of the scan of kda_forward (the pages give only the forward;
+ * this is its reverse-mode derivative).  For a loss L with dL/do = d_o and dL/dS_T = dS_T:
+ *   q, k, v, g, beta, S0, B, T, H, Dk, Dv, dtype : exactly as passed to kda_forward.
+ *   d_o   : [B, T, H, Dv] in do_dtype (device).
+ *   dS_T  : [B, H, Dk, Dv] fp32 or NULL (zeros).
+ *   dq, dk, dg : [B, T, H, Dk] fp32 (device, written);  dv : [B, T, H, Dv] fp32;
+ *   dbeta : [B, T, H] fp32;  dS0 : [B, H, Dk, Dv] fp32 or NULL (not written).
+ * The gradient of g is that of the natural-log decay (alpha = e^g).  The call reruns
+ * the forward to store each 32-token chunk's entry state in the workspace
+ * (kda_backward_workspace_size bytes: B*H*ceil(T/32)*Dk*Dv*4), then sweeps the chunks in
+ * reverse; arithmetic is fp32.  Per key channel the decay over any 32 consecutive tokens
+ * must satisfy |sum g| < 80; beyond that the gradients are not finite.
+ * workspace: as for kda_forward (NULL: a stream-ordered allocation inside the call).
+ * Errors: KDA_ERR_INVALID_ARG (null tensor with work to do, bad sizes or dtypes),
+ * KDA_ERR_UNSUPPORTED (Dk or Dv outside {32, 64, 128}; B or H > 65535),
+ * KDA_ERR_WORKSPACE, KDA_ERR_CUDA.
+ */
+size_t kda_backward_workspace_size(int B, int T, int H, int Dk, int Dv);
+kda_status kda_backward(const void* q, const void* k, const void* v, const void* g,
+                        const void* beta, const float* S0, const void* d_o,
+                        const float* dS_T, float* dq, float* dk, float* dv, float* dg,
+                        float* dbeta, float* dS0, int B, int T, int H, int Dk, int Dv,
+                        kda_dtype dtype, kda_dtype do_dtype, void* workspace,
+                        size_t workspace_bytes, kda_stream_t stream);
+
 /* Modalities of a packed-stream segment (section 3.4). */
 typedef enum { MSC_TEXT = 0, MSC_IMAGE = 1, MSC_VIDEO = 2 } msc_modality;
 
@@ -337,7 +363,7 @@ void kda_profile_enable(int on);
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
  * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
- * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold". */
+ * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold", "kda_bwd". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

@@ -94,6 +94,20 @@ size_t kda_tc_sp_workspace_bytes(int B, int T, int H, int num_sms);
 cudaError_t launch_kda_tc_sp_state(const KdaArgs& a, void* ws, int* status, cudaStream_t s, TcShardMaps* out);
 cudaError_t launch_kda_tc_sp_output(const KdaArgs& a, void* ws, int* status, cudaStream_t s);
 
+// Backward of the scan (fp32 on CUDA cores, any supported dtype / Dk / Dv): gradients
+// in fp32; dq, dk, dg, dbeta are zeroed and then accumulated by the launch.
+struct KdaBwdArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float* S0;
+    const void* dout;
+    const float* dST;
+    float *dq, *dk, *dv, *dg, *dbeta, *dS0;
+    int B, T, H, Dk, Dv;
+    ElemType in_t, do_t;
+};
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv);
+cudaError_t launch_kda_bwd(const KdaBwdArgs& a, void* ws, cudaStream_t s);
+
 struct ConvSeg {
     int32_t modality;
     int64_t start;

@@ -282,6 +282,41 @@ kda_status kda_forward_varlen(const void* q, const void* k, const void* v, const
     return KDA_OK;
 }
 
+// ---- backward ---------------------------------------------------------------------------
+size_t kda_backward_workspace_size(int B, int T, int H, int Dk, int Dv)
+{
+    if (B < 0 || T < 0 || H <= 0 || !dim_ok(Dk) || !dim_ok(Dv)) return 0;
+    return kda_bwd_workspace_bytes(B, T, H, Dk, Dv);
+}
+
+kda_status kda_backward(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        const float* S0, const void* d_o, const float* dS_T, float* dq, float* dk, float* dv,
+                        float* dg, float* dbeta, float* dS0, int B, int T, int H, int Dk, int Dv,
+                        kda_dtype dtype, kda_dtype do_dtype, void* workspace, size_t workspace_bytes,
+                        kda_stream_t stream)
+{
+    if (B < 0 || T < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if ((dtype != KDA_F32 && dtype != KDA_BF16) || (do_dtype != KDA_F32 && do_dtype != KDA_BF16))
+        return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(Dk) || !dim_ok(Dv) || B > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > 0 && (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (B == 0) return KDA_OK;
+    if (T == 0) {   // no tokens: dS0 = dS_T
+        if (!dS0) return KDA_OK;
+        const size_t bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+        return from_cuda(dS_T ? cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(dS0, 0, bytes, s));
+    }
+    const KdaBwdArgs a{q, k, v, g, beta, S0, d_o, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H, Dk, Dv,
+                       et_of(dtype), et_of(do_dtype)};
+    Workspace ws;
+    kda_status st = ws.acquire(workspace, workspace_bytes, kda_bwd_workspace_bytes(B, T, H, Dk, Dv), s);
+    if (st != KDA_OK) return st;
+    return from_cuda(launch_kda_bwd(a, ws.ptr, s));
+}
+
 static kda_status check_segments(const msc_segment* segs, int n_segs, int T, int Kt,
                                  const float* w_text, int n_text, const float* w_image,
                                  int n_image, const float* w_video, int n_video)

@@ -1,0 +1,432 @@
+// Backward of the KDA forward scan (Eq. 14 of the Chimera paper, section 3.3, with the
+// readout o_t = S_t^T q_t of Eq. 15): given dL/do and dL/dS_T, the gradients of q, k, v,
+// g = log(alpha), beta and S0.  The pages give only the forward; this is its
+// reverse-mode derivative, taken through the chunk form of the scan.
+//
+// Chunk form (C = 32 tokens, entry state S, b_i = sum_{r<=i} g_r per key channel, b_C
+// the chunk's last b, r = b at row 15 a per-channel reference):
+//   K+ = k e^{b-r},  K- = k e^{r-b},  Q+ = q e^{b-r},  Se = Diag(e^r) S
+//   Kd = K+ K-^T (used strictly below the diagonal),  A = Diag(beta) Kd,  T = (I + A)^{-1}
+//   P  = lower(Q+ K-^T)                      (diagonal included)
+//   VX = V - K+ Se,  Rb = Diag(beta) VX,  U = T Rb
+//   O  = Q+ Se + P U,   S' = Diag(e^{b_C - r}) (Se + K-^T U)
+// Reverse, with G' = dL/dS' and Gc = Diag(e^{b_C - r}) G':
+//   dU  = P^T dO + K- Gc           dR = T^T dU            dv = Diag(beta) dR
+//   dbeta_i = VX_i . dR_i + sum_{j<i} dA_ij Kd_ij        (dRb = Diag(beta) dR)
+//   dT  = dU Rb^T,  dA = -T^T dT T^T (strictly lower),   dAb = Diag(beta) dA
+//   dP  = lower(dO U^T)
+//   dQ+ = dO Se^T + dP K-          dK+ = -dRb Se^T + dAb K-
+//   dK- = U Gc^T + dAb^T K+ + dP^T Q+
+//   G   = Diag(e^r) (Gc + Q+^T dO - K+^T dRb)             (dL/dS, to the previous chunk)
+//   dq  = dQ+ e^{b-r},  dk = dK+ e^{b-r} + dK- e^{r-b}
+//   db  = dQ+ Q+ + dK+ K+ - dK- K-,  plus at b_C: sum_j (U Gc^T)_j K-_j + rowsum(Gc Se)
+//   dg  = reverse cumulative sum of db over the chunk's rows
+// r cancels out of the loss, so it is held fixed.  Every exponent that reaches a used
+// value is <= 0 or within e^{|b_C|}: per key channel the decay over 32 consecutive
+// tokens must stay within |sum g| < ~80 (mean g > -2.5 per token); beyond that the
+// results are not finite.
+//
+// Parallel split: the state's value columns evolve independently, so one CTA owns 32
+// value columns of one (b, h).  It first runs the forward over all chunks and stores
+// each chunk's entry state (its 32 columns) in the workspace, then walks the chunks in
+// reverse.  dv and dS0 columns belong to one CTA; dq, dk, dg and dbeta are sums over
+// the value columns and are accumulated with atomic adds (the outputs are zeroed first).
+// All arithmetic is fp32 on CUDA cores.
+
+#include "internal.h"
+
+namespace kda {
+namespace {
+
+constexpr int BC = 32;        // chunk length
+constexpr int BVC = 32;       // value columns per CTA
+constexpr int BT = 256;       // threads per CTA
+constexpr int LDV = BVC + 1;  // row stride of [BC][BVC] tiles (floats)
+constexpr int LDC = BC + 1;   // row stride of [BC][BC] tiles
+
+template <int DK> struct BwdPlan {
+    static constexpr int LDK = DK + 1;    // [BC][DK] tiles
+    static constexpr int LDS = BVC + 1;   // [DK][BVC] tiles
+    static constexpr int KP = 0, KM = KP + BC * LDK, QP = KM + BC * LDK;
+    static constexpr int DQP = QP + BC * LDK, DKP = DQP + BC * LDK, DKM = DKP + BC * LDK;
+    static constexpr int SE = DKM + BC * LDK, GP = SE + DK * LDS;
+    static constexpr int VX = GP + DK * LDS, RB = VX + BC * LDV, UU = RB + BC * LDV, DU = UU + BC * LDV,
+                         DR = DU + BC * LDV, DO = DR + BC * LDV;
+    static constexpr int KD = DO + BC * LDV, PP = KD + BC * LDC, TT = PP + BC * LDC, X1 = TT + BC * LDC,
+                         X2 = X1 + BC * LDC, DP = X2 + BC * LDC;
+    static constexpr int BETA = DP + BC * LDC, RR = BETA + BC, BCC = RR + DK, DBC = BCC + DK, DBETA = DBC + DK;
+    static constexpr int TOTAL = DBETA + BC;
+    static constexpr int BYTES = TOTAL * (int)sizeof(float);
+};
+
+enum { MM_SET = 0, MM_ADD = 1, MM_SUB = 2, MM_NEG = 3 };
+
+// out(i, j) op= sum_{k<K} A(i, k) B(k, j) for i < M, j < N, over threads
+// [tid0, tid0 + nthr).  A(i, k) = A[i*ai + k*ak], B(k, j) = B[k*bk + j*bj],
+// out(i, j) = O[i*oi + j].  A thread owns a TM x TN micro-tile with strided rows and
+// columns (ti + m*M/TM, tj + n*N/TN), so a warp's B reads hit consecutive columns.
+template <int M, int N, int K, int TM, int TN, int OP>
+__device__ __forceinline__ void mm(float* O, int oi, const float* A, int ai, int ak, const float* B, int bk, int bj,
+                                   int tid0 = 0, int nthr = BT)
+{
+    static_assert(M % TM == 0 && N % TN == 0, "micro-tile");
+    constexpr int GM = M / TM, GN = N / TN, NTILE = GM * GN;
+    for (int tile = (int)threadIdx.x - tid0; tile < NTILE; tile += nthr) {
+        if (tile < 0) break;
+        const int ti = tile / GN, tj = tile % GN;
+        float acc[TM][TN];
+#pragma unroll
+        for (int m = 0; m < TM; ++m)
+#pragma unroll
+            for (int n = 0; n < TN; ++n) acc[m][n] = 0.f;
+#pragma unroll 4
+        for (int k = 0; k < K; ++k) {
+            float a[TM], b[TN];
+#pragma unroll
+            for (int m = 0; m < TM; ++m) a[m] = A[(ti + m * GM) * ai + k * ak];
+#pragma unroll
+            for (int n = 0; n < TN; ++n) b[n] = B[k * bk + (tj + n * GN) * bj];
+#pragma unroll
+            for (int m = 0; m < TM; ++m)
+#pragma unroll
+                for (int n = 0; n < TN; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
+        }
+#pragma unroll
+        for (int m = 0; m < TM; ++m)
+#pragma unroll
+            for (int n = 0; n < TN; ++n) {
+                float* o = O + (ti + m * GM) * oi + (tj + n * GN);
+                if (OP == MM_SET) *o = acc[m][n];
+                else if (OP == MM_ADD) *o += acc[m][n];
+                else if (OP == MM_SUB) *o -= acc[m][n];
+                else *o = -acc[m][n];
+            }
+    }
+}
+
+// Micro-tile sizes for an M x N output over 256 threads.
+template <int M, int N> struct Tile {
+    static constexpr int per = M * N / BT;
+    static constexpr int TM = per >= 16 ? 4 : 2;
+    static constexpr int TN = per / TM;
+};
+
+template <int M, int N, int K, int OP>
+__device__ __forceinline__ void mmt(float* O, int oi, const float* A, int ai, int ak, const float* B, int bk, int bj,
+                                    int tid0 = 0, int nthr = BT)
+{
+    mm<M, N, K, Tile<M, N>::TM, Tile<M, N>::TN, OP>(O, oi, A, ai, ak, B, bk, bj, tid0, nthr);
+}
+
+template <typename T> __device__ __forceinline__ float ld(const T* p) { return to_f32(*p); }
+
+// T = (I + Diag(beta) Kd_strictlower)^{-1} by forward substitution on one warp: lane j
+// holds column j of T in registers; row i needs only rows < i.
+__device__ __forceinline__ void invert_warp(float* Tm, const float* Kd, const float* beta, int lane)
+{
+    float col[BC];
+#pragma unroll
+    for (int i = 0; i < BC; ++i) {
+        const float bi = beta[i];
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < i; ++m) {
+            const float a = bi * Kd[i * LDC + m];
+            if (m & 1) a1 = fmaf(a, col[m], a1);
+            else a0 = fmaf(a, col[m], a0);
+        }
+        col[i] = (i == lane ? 1.f : 0.f) - (a0 + a1);
+    }
+#pragma unroll
+    for (int i = 0; i < BC; ++i) Tm[i * LDC + lane] = col[i];
+}
+
+template <int DK, typename TIn, typename TDo>
+__global__ void __launch_bounds__(BT, 1)
+kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+               const TIn* __restrict__ g, const TIn* __restrict__ beta, const float* __restrict__ S0,
+               const TDo* __restrict__ dout, const float* __restrict__ dST, float* __restrict__ dq,
+               float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
+               float* __restrict__ dS0, float* __restrict__ ckpt, int T, int H, int Dv)
+{
+    using PL = BwdPlan<DK>;
+    constexpr int LDK = PL::LDK, LDS = PL::LDS;
+    extern __shared__ __align__(16) float sm[];
+    float *sKP = sm + PL::KP, *sKM = sm + PL::KM, *sQP = sm + PL::QP;
+    float *sDQP = sm + PL::DQP, *sDKP = sm + PL::DKP, *sDKM = sm + PL::DKM;
+    float *sSe = sm + PL::SE, *sGp = sm + PL::GP;
+    float *sVX = sm + PL::VX, *sRb = sm + PL::RB, *sU = sm + PL::UU, *sDU = sm + PL::DU, *sDR = sm + PL::DR,
+          *sDO = sm + PL::DO;
+    float *sKd = sm + PL::KD, *sP = sm + PL::PP, *sT = sm + PL::TT, *sX1 = sm + PL::X1, *sX2 = sm + PL::X2,
+          *sDP = sm + PL::DP;
+    float *sBeta = sm + PL::BETA, *sR = sm + PL::RR, *sBC = sm + PL::BCC, *sDbC = sm + PL::DBC,
+          *sDbeta = sm + PL::DBETA;
+
+    const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+    const int cb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int col0 = cb * BVC;
+    const int NC = (T + BC - 1) / BC;
+    const size_t rowH = (size_t)H;                 // tokens -> rows of [B, T, H, *]
+    const size_t tok0 = (size_t)b * T;             // first token row of this sequence
+    float* ck = ckpt + ((size_t)(b * H + h) * (Dv / BVC) + cb) * (size_t)NC * DK * BVC;
+
+    // per-channel prologue of chunk n: K+, K- (and Q+), r, b_C; masked rows past T
+    auto prologue = [&](int n, bool with_q) {
+        const int t0 = n * BC;
+        if (t < BC) sBeta[t] = (t0 + t < T) ? ld(beta + (tok0 + t0 + t) * rowH + h) : 0.f;
+        if (t < DK) {
+            const int c = t;
+            float bb[BC];
+            float run = 0.f;
+#pragma unroll
+            for (int i = 0; i < BC; ++i) {
+                const bool live = t0 + i < T;
+                run += live ? ld(g + ((tok0 + t0 + i) * rowH + h) * DK + c) : 0.f;
+                bb[i] = run;
+            }
+            const float r = bb[15], bC = bb[BC - 1];
+            sR[c] = r;
+            sBC[c] = bC;
+#pragma unroll
+            for (int i = 0; i < BC; ++i) {
+                const bool live = t0 + i < T;
+                const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
+                const float kk = live ? ld(k + idx) : 0.f;
+                const float ep = expf(bb[i] - r), em = expf(r - bb[i]);
+                sKP[i * LDK + c] = kk * ep;
+                sKM[i * LDK + c] = kk * em;
+                if (with_q) sQP[i * LDK + c] = (live ? ld(q + idx) : 0.f) * ep;
+            }
+        }
+    };
+    // [BC][BVC] tile of a [B, T, H, Dv] tensor (this CTA's columns), zero past T
+    auto load_rows = [&](float* dst, auto src, int n) {
+        const int t0 = n * BC;
+        for (int e = t; e < BC * BVC; e += BT) {
+            const int i = e / BVC, j = e % BVC;
+            dst[i * LDV + j] = (t0 + i < T) ? ld(src + ((tok0 + t0 + i) * rowH + h) * Dv + col0 + j) : 0.f;
+        }
+    };
+
+    // ---------------- forward sweep: entry state of every chunk -> workspace ----------------
+    for (int e = t; e < DK * BVC; e += BT) {
+        const int c = e / BVC, j = e % BVC;
+        sSe[c * LDS + j] = S0 ? S0[((size_t)(b * H + h) * DK + c) * Dv + col0 + j] : 0.f;
+    }
+    __syncthreads();
+    for (int n = 0; n < NC; ++n) {
+        float* ckn = ck + (size_t)n * DK * BVC;
+        for (int e = t; e < DK * BVC; e += BT) ckn[e] = sSe[(e / BVC) * LDS + e % BVC];
+        prologue(n, false);
+        load_rows(sVX, v, n);
+        __syncthreads();
+        mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK);
+        for (int e = t; e < DK * BVC; e += BT) {
+            const int c = e / BVC, j = e % BVC;
+            sSe[c * LDS + j] *= expf(sR[c]);
+        }
+        __syncthreads();
+        if (w == 0) invert_warp(sT, sKd, sBeta, lane);
+        else mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 32, BT - 32);
+        __syncthreads();
+        for (int e = t; e < BC * BVC; e += BT) {
+            const int i = e / BVC, j = e % BVC;
+            sRb[i * LDV + j] = sBeta[i] * sVX[i * LDV + j];
+        }
+        __syncthreads();
+        mmt<BC, BVC, BC, MM_SET>(sU, LDV, sT, LDC, 1, sRb, LDV, 1);
+        __syncthreads();
+        mmt<DK, BVC, BC, MM_ADD>(sSe, LDS, sKM, 1, LDK, sU, LDV, 1);
+        __syncthreads();
+        for (int e = t; e < DK * BVC; e += BT) {
+            const int c = e / BVC, j = e % BVC;
+            sSe[c * LDS + j] *= expf(sBC[c] - sR[c]);
+        }
+        __syncthreads();
+    }
+
+    // ---------------- reverse sweep ----------------
+    for (int e = t; e < DK * BVC; e += BT) {
+        const int c = e / BVC, j = e % BVC;
+        sGp[c * LDS + j] = dST ? dST[((size_t)(b * H + h) * DK + c) * Dv + col0 + j] : 0.f;
+    }
+    for (int n = NC - 1; n >= 0; --n) {
+        const int t0 = n * BC;
+        const float* ckn = ck + (size_t)n * DK * BVC;
+        __syncthreads();   // the previous chunk is done with every tile
+        prologue(n, true);
+        load_rows(sVX, v, n);
+        load_rows(sDO, dout, n);
+        for (int e = t; e < DK * BVC; e += BT) sSe[(e / BVC) * LDS + e % BVC] = ckn[e];
+        __syncthreads();
+        // Kd, P; Se = Diag(e^r) S; Gc = Diag(e^{b_C - r}) G'
+        mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK);
+        mmt<BC, BC, DK, MM_SET>(sP, LDC, sQP, LDK, 1, sKM, 1, LDK);
+        for (int e = t; e < DK * BVC; e += BT) {
+            const int c = e / BVC, j = e % BVC;
+            sSe[c * LDS + j] *= expf(sR[c]);
+            sGp[c * LDS + j] *= expf(sBC[c] - sR[c]);
+        }
+        __syncthreads();
+        // T (warp 0) | VX = V - K+ Se, dU = K- Gc, P masked (the other warps)
+        if (w == 0) {
+            invert_warp(sT, sKd, sBeta, lane);
+        } else {
+            mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 32, BT - 32);
+            mmt<BC, BVC, DK, MM_SET>(sDU, LDV, sKM, LDK, 1, sGp, LDS, 1, 32, BT - 32);
+            for (int e = t - 32; e < BC * BC; e += BT - 32) {
+                const int i = e / BC, j = e % BC;
+                if (j > i) sP[i * LDC + j] = 0.f;
+            }
+        }
+        __syncthreads();
+        for (int e = t; e < BC * BVC; e += BT) {
+            const int i = e / BVC, j = e % BVC;
+            sRb[i * LDV + j] = sBeta[i] * sVX[i * LDV + j];
+        }
+        mmt<BC, BVC, BC, MM_ADD>(sDU, LDV, sP, 1, LDC, sDO, LDV, 1);   // dU += P^T dO
+        __syncthreads();
+        mmt<BC, BVC, BC, MM_SET>(sU, LDV, sT, LDC, 1, sRb, LDV, 1);    // U = T Rb
+        mmt<BC, BVC, BC, MM_SET>(sDR, LDV, sT, 1, LDC, sDU, LDV, 1);   // dR = T^T dU
+        __syncthreads();
+        if (t < BC) {
+            float s = 0.f;
+            for (int j = 0; j < BVC; ++j) s = fmaf(sVX[t * LDV + j], sDR[t * LDV + j], s);
+            sDbeta[t] = s;
+        }
+        for (int e = t; e < BC * BVC; e += BT) {
+            const int i = e / BVC, j = e % BVC;
+            if (t0 + i < T) dv[((tok0 + t0 + i) * rowH + h) * Dv + col0 + j] = sBeta[i] * sDR[i * LDV + j];
+        }
+        mmt<BC, BC, BVC, MM_SET>(sX1, LDC, sDU, LDV, 1, sRb, 1, LDV);  // dT = dU Rb^T
+        mmt<BC, BC, BVC, MM_SET>(sDP, LDC, sDO, LDV, 1, sU, 1, LDV);   // dO U^T
+        __syncthreads();
+        for (int e = t; e < BC * BVC; e += BT) {                        // dRb = Diag(beta) dR
+            const int i = e / BVC, j = e % BVC;
+            sDR[i * LDV + j] *= sBeta[i];
+        }
+        for (int e = t; e < BC * BC; e += BT) {                         // dP = lower(dO U^T)
+            const int i = e / BC, j = e % BC;
+            if (j > i) sDP[i * LDC + j] = 0.f;
+        }
+        mmt<BC, BC, BC, MM_SET>(sX2, LDC, sX1, LDC, 1, sT, 1, LDC);    // dT T^T
+        __syncthreads();
+        mmt<BC, BC, BC, MM_NEG>(sX1, LDC, sT, 1, LDC, sX2, LDC, 1);    // dA = -T^T dT T^T
+        __syncthreads();
+        if (t < BC) {   // strictly lower part; dbeta from A; dAb = Diag(beta) dA
+            const int i = t;
+            float s = sDbeta[i];
+            for (int j = 0; j < BC; ++j) {
+                const float da = (j < i) ? sX1[i * LDC + j] : 0.f;
+                s = fmaf(da, sKd[i * LDC + j], s);
+                sX1[i * LDC + j] = sBeta[i] * da;
+            }
+            sDbeta[i] = s;
+        }
+        mmt<BC, DK, BVC, MM_SET>(sDQP, LDK, sDO, LDV, 1, sSe, 1, LDS);  // dQ+ = dO Se^T
+        mmt<BC, DK, BVC, MM_NEG>(sDKP, LDK, sDR, LDV, 1, sSe, 1, LDS);  // dK+ = -dRb Se^T
+        mmt<BC, DK, BVC, MM_SET>(sDKM, LDK, sU, LDV, 1, sGp, 1, LDS);   // dK- = U Gc^T
+        __syncthreads();
+        if (t < DK) {   // the b_C terms: sum_j (U Gc^T)_j K-_j + rowsum(Gc Se)
+            const int c = t;
+            float s = 0.f;
+            for (int i = 0; i < BC; ++i) s = fmaf(sDKM[i * LDK + c], sKM[i * LDK + c], s);
+            for (int j = 0; j < BVC; ++j) s = fmaf(sGp[c * LDS + j], sSe[c * LDS + j], s);
+            sDbC[c] = s;
+        }
+        mmt<BC, DK, BC, MM_ADD>(sDQP, LDK, sDP, LDC, 1, sKM, LDK, 1);   // dQ+ += dP K-
+        mmt<BC, DK, BC, MM_ADD>(sDKP, LDK, sX1, LDC, 1, sKM, LDK, 1);   // dK+ += dAb K-
+        __syncthreads();
+        mmt<BC, DK, BC, MM_ADD>(sDKM, LDK, sX1, 1, LDC, sKP, LDK, 1);   // dK- += dAb^T K+
+        mmt<BC, DK, BC, MM_ADD>(sDKM, LDK, sDP, 1, LDC, sQP, LDK, 1);   // dK- += dP^T Q+
+        mmt<DK, BVC, BC, MM_ADD>(sGp, LDS, sQP, 1, LDK, sDO, LDV, 1);   // Gc + Q+^T dO
+        mmt<DK, BVC, BC, MM_SUB>(sGp, LDS, sKP, 1, LDK, sDR, LDV, 1);   //    - K+^T dRb
+        __syncthreads();
+        if (t < DK) {   // per channel: dq, dk, db -> dg (reverse cumulative sum); G row scale
+            const int c = t;
+            float bb[BC];
+            float run = 0.f;
+#pragma unroll
+            for (int i = 0; i < BC; ++i) {
+                run += (t0 + i < T) ? ld(g + ((tok0 + t0 + i) * rowH + h) * DK + c) : 0.f;
+                bb[i] = run;
+            }
+            const float r = sR[c];
+            float acc = sDbC[c];
+#pragma unroll
+            for (int i = BC - 1; i >= 0; --i) {
+                const float ep = expf(bb[i] - r), em = expf(r - bb[i]);
+                const float dqp = sDQP[i * LDK + c], dkp = sDKP[i * LDK + c], dkm = sDKM[i * LDK + c];
+                acc += dqp * sQP[i * LDK + c] + dkp * sKP[i * LDK + c] - dkm * sKM[i * LDK + c];
+                if (t0 + i < T) {
+                    const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
+                    atomicAdd(dq + idx, dqp * ep);
+                    atomicAdd(dk + idx, dkp * ep + dkm * em);
+                    atomicAdd(dg + idx, acc);
+                }
+            }
+            const float er = expf(r);
+            for (int j = 0; j < BVC; ++j) sGp[c * LDS + j] *= er;
+        }
+        if (t < BC && t0 + t < T) atomicAdd(dbeta + (tok0 + t0 + t) * rowH + h, sDbeta[t]);
+    }
+    __syncthreads();
+    if (dS0)
+        for (int e = t; e < DK * BVC; e += BT) {
+            const int c = e / BVC, j = e % BVC;
+            dS0[((size_t)(b * H + h) * DK + c) * Dv + col0 + j] = sGp[c * LDS + j];
+        }
+}
+
+template <int DK, typename TIn, typename TDo>
+cudaError_t launch_t(const KdaBwdArgs& a, void* ws, cudaStream_t s)
+{
+    auto kern = kda_bwd_kernel<DK, TIn, TDo>;
+    const int smem = BwdPlan<DK>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    ProfileScope prof("kda_bwd", s);
+    count_launch();
+    kern<<<dim3(a.Dv / BVC, a.H, a.B), BT, smem, s>>>(
+        (const TIn*)a.q, (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.g, (const TIn*)a.beta, a.S0,
+        (const TDo*)a.dout, a.dST, a.dq, a.dk, a.dv, a.dg, a.dbeta, a.dS0, reinterpret_cast<float*>(ws), a.T, a.H,
+        a.Dv);
+    return cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_d(const KdaBwdArgs& a, void* ws, cudaStream_t s)
+{
+    const bool in_f32 = a.in_t == ET_F32, do_f32 = a.do_t == ET_F32;
+    if (in_f32 && do_f32) return launch_t<DK, float, float>(a, ws, s);
+    if (in_f32) return launch_t<DK, float, __nv_bfloat16>(a, ws, s);
+    if (do_f32) return launch_t<DK, __nv_bfloat16, float>(a, ws, s);
+    return launch_t<DK, __nv_bfloat16, __nv_bfloat16>(a, ws, s);
+}
+
+}  // namespace
+
+size_t kda_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv)
+{
+    if (B <= 0 || T <= 0) return 0;
+    const size_t NC = (size_t)(T + BC - 1) / BC;
+    return (size_t)B * H * NC * Dk * Dv * sizeof(float);
+}
+
+cudaError_t launch_kda_bwd(const KdaBwdArgs& a, void* ws, cudaStream_t s)
+{
+    const size_t tok = (size_t)a.B * a.T * a.H;
+    cudaError_t e = cudaMemsetAsync(a.dq, 0, tok * a.Dk * sizeof(float), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dk, 0, tok * a.Dk * sizeof(float), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dg, 0, tok * a.Dk * sizeof(float), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(a.dbeta, 0, tok * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    switch (a.Dk) {
+        case 32: return launch_d<32>(a, ws, s);
+        case 64: return launch_d<64>(a, ws, s);
+        case 128: return launch_d<128>(a, ws, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

@@ -28,7 +28,8 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_mshortconv_forward", "kda_kernel_launches", "kda_profile_enable",
             "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
             "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size",
-            "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output")
+            "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output",
+            "kda_backward", "kda_backward_workspace_size")
 
 
 class KdaError(RuntimeError):
@@ -96,6 +97,10 @@ def load_library(path: str = LIB_PATH):
         lib.kda_sp_prefix.argtypes = [P, I, I, P, P, I, I, I, P]
         lib.kda_sp_output.restype = I
         lib.kda_sp_output.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
+        lib.kda_backward_workspace_size.restype = Z
+        lib.kda_backward_workspace_size.argtypes = [I, I, I, I, I]
+        lib.kda_backward.restype = I
+        lib.kda_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -344,6 +349,48 @@ def sp_output(q, k, v, g, beta, S_in, workspace, *, chunk: int = 0, o=None, S_T=
                            B, T, H, D, dt, _code(o_dtype), chunk, ws_ptr, ws_bytes, _stream(stream))
     _check("kda_sp_output", rc)
     return o, S_T
+
+
+def backward_workspace_size(B, T, H, Dk, Dv) -> int:
+    return int(load_library().kda_backward_workspace_size(B, T, H, Dk, Dv))
+
+
+def backward(q, k, v, g, beta, do, S0=None, dS_T=None, *, want_dS0: bool = True, workspace=None,
+             stream=None, out=None):
+    """kda_backward: gradients (fp32) of L with dL/do = do and dL/dS_T = dS_T through the
+    scan of forward().  q, k, v, g, beta, S0 as passed to forward(); do: [B,T,H,Dv] bf16
+    or fp32.  Returns (dq, dk, dv, dg, dbeta, dS0 or None); `out` may hold preallocated
+    fp32 tensors in that order."""
+    lib = load_library()
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = _dtype_code(q)
+    for name, t, shape in (("k", k, (B, T, H, Dk)), ("g", g, (B, T, H, Dk)),
+                           ("v", v, (B, T, H, Dv)), ("beta", beta, (B, T, H))):
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q's {q.dtype}")
+    if tuple(do.shape) != (B, T, H, Dv):
+        raise ValueError("do shape")
+    for name, t in (("S0", S0), ("dS_T", dS_T)):
+        if t is not None and tuple(t.shape) != (B, H, Dk, Dv):
+            raise ValueError(f"{name} shape")
+    f = dict(dtype=torch.float32, device=q.device)
+    if out is None:
+        out = (torch.empty((B, T, H, Dk), **f), torch.empty((B, T, H, Dk), **f),
+               torch.empty((B, T, H, Dv), **f), torch.empty((B, T, H, Dk), **f),
+               torch.empty((B, T, H), **f), torch.empty((B, H, Dk, Dv), **f) if want_dS0 else None)
+    dq, dk, dv, dg, dbeta, dS0 = out
+    ws_ptr, ws_bytes = _ws(workspace)
+    rc = lib.kda_backward(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(g, "g"), _dev(beta, "beta"),
+                          _dev(S0, "S0", torch.float32), _dev(do, "do"), _dev(dS_T, "dS_T", torch.float32),
+                          _dev(dq, "dq", torch.float32), _dev(dk, "dk", torch.float32),
+                          _dev(dv, "dv", torch.float32), _dev(dg, "dg", torch.float32),
+                          _dev(dbeta, "dbeta", torch.float32), _dev(dS0, "dS0", torch.float32),
+                          B, T, H, Dk, Dv, dt, _dtype_code(do), ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_backward", rc)
+    return dq, dk, dv, dg, dbeta, dS0
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20

@@ -89,6 +89,24 @@ def test_sequence_parallel_calls_reject_bad_arguments(lib):
     assert lib.kda_sp_workspace_size(1, 8, 1, 48, 1, 0) == 0
 
 
+def test_backward_rejects_bad_arguments(lib):
+    P = None
+    d = ctypes.c_void_p(256)   # never dereferenced: validation fails first
+    full = lambda **kw: tuple(kw.get(n, d) for n in ("q", "k", "v", "g", "beta")) + (P, d, P) + \
+        tuple(kw.get(n, d) for n in ("dq", "dk", "dv", "dg", "dbeta")) + (P,)
+    sizes = lambda Dk=32, Dv=32, B=1, T=8, dt=1, dodt=1: (B, T, 1, Dk, Dv, dt, dodt, P, 0, P)
+    assert lib.kda_backward(*full(), *sizes(Dk=48)) == 2            # unsupported head width
+    assert lib.kda_backward(*full(), *sizes(Dv=96)) == 2
+    assert lib.kda_backward(*full(dg=P), *sizes()) == 1             # missing gradient buffer
+    assert lib.kda_backward(*full(q=P), *sizes()) == 1              # missing input
+    assert lib.kda_backward(*full(), *sizes(dt=4)) == 1             # bad dtype
+    assert lib.kda_backward(*full(), *sizes(dodt=4)) == 1           # bad d_o dtype
+    assert lib.kda_backward(*full(), *sizes(B=-1)) == 1
+    assert lib.kda_backward(*full(), *sizes(B=0)) == 0              # empty batch: no-op
+    assert lib.kda_backward_workspace_size(1, 64, 2, 32, 64) == 2 * 2 * 32 * 64 * 4
+    assert lib.kda_backward_workspace_size(1, 64, 2, 48, 64) == 0
+
+
 def test_conv_rejects_bad_segment_tables(lib):
     segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
     dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
