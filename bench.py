@@ -514,9 +514,19 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             mb = timed(bstep, k_b, 1) / k_b
             esz = torch.tensor([], dtype=w.dtype).element_size()
             bbytes = algorithmic_bytes(w) + w.B * w.T * w.H * (4 * w.D * 4 + 4)
+            # the kernel's own fp32 multiply-adds per (32-token chunk, 32 value columns):
+            # forward sweep 3 C*C*D-class + C^2*Vc, reverse sweep 12 C*D*Vc-class + 7 C^2*Vc
+            C_, Vc_, D_ = 32, 32, w.D
+            fma_chunk = (3 * C_ * D_ * Vc_ + C_ * C_ * Vc_) + (12 * C_ * D_ * Vc_ + 7 * C_ * C_ * Vc_)
+            fmas = fma_chunk * w.B * w.H * (w.D // Vc_) * ((w.T + C_ - 1) // C_)
+            fma_rate = kda.fma_probe()
             extra.append({"workload": w.name + "_backward", "ms_per_step": mb,
                           "value": w.tokens / (mb * 1e-3) / 1e6, "unit": UNIT,
                           "alg_GBps": bbytes / (mb * 1e-3) / 1e9, "alg_bytes": bbytes,
+                          "roofline": {"bound": "alu", "achieved": fmas / (mb * 1e-3) / 1e12,
+                                       "peak": fma_rate / 1e12, "unit": "TFMA/s",
+                                       "frac": fmas / (mb * 1e-3) / fma_rate, "fmas_per_step": fmas,
+                                       "peak_source": "kda_fma_probe on this GPU"},
                           "path": "fp32 CUDA cores, one CTA per (b, h, 32 value columns)"})
         line["extra_workloads"] = extra
     if rank == 0:

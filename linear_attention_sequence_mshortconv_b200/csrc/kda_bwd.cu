@@ -33,6 +33,8 @@
 // the value columns and are accumulated with atomic adds (the outputs are zeroed first).
 // All arithmetic is fp32 on CUDA cores.
 
+#include <type_traits>
+
 #include "internal.h"
 
 namespace kda {
@@ -54,7 +56,8 @@ template <int DK> struct BwdPlan {
                          DR = DU + BC * LDV, DO = DR + BC * LDV;
     static constexpr int KD = DO + BC * LDV, PP = KD + BC * LDC, TT = PP + BC * LDC, X1 = TT + BC * LDC,
                          X2 = X1 + BC * LDC, DP = X2 + BC * LDC;
-    static constexpr int BETA = DP + BC * LDC, RR = BETA + BC, BCC = RR + DK, DBC = BCC + DK, DBETA = DBC + DK;
+    static constexpr int BB = DP + BC * LDC;   // b = cumsum(g) of the chunk, [BC][DK]
+    static constexpr int BETA = BB + BC * LDK, RR = BETA + BC, BCC = RR + DK, DBC = BCC + DK, DBETA = DBC + DK;
     static constexpr int TOTAL = DBETA + BC;
     static constexpr int BYTES = TOTAL * (int)sizeof(float);
 };
@@ -120,6 +123,21 @@ __device__ __forceinline__ void mmt(float* O, int oi, const float* A, int ai, in
 
 template <typename T> __device__ __forceinline__ float ld(const T* p) { return to_f32(*p); }
 
+// 16 bytes of fp32 or bf16 values -> floats
+__device__ __forceinline__ void unpack16(const uint4& u, float (&f)[4], const float*)
+{
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y); f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack16(const uint4& u, float (&f)[8], const __nv_bfloat16*)
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
 // T = (I + Diag(beta) Kd_strictlower)^{-1} by forward substitution on one warp: lane j
 // holds column j of T in registers; row i needs only rows < i.
 __device__ __forceinline__ void invert_warp(float* Tm, const float* Kd, const float* beta, int lane)
@@ -159,6 +177,7 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
           *sDO = sm + PL::DO;
     float *sKd = sm + PL::KD, *sP = sm + PL::PP, *sT = sm + PL::TT, *sX1 = sm + PL::X1, *sX2 = sm + PL::X2,
           *sDP = sm + PL::DP;
+    float* sB = sm + PL::BB;
     float *sBeta = sm + PL::BETA, *sR = sm + PL::RR, *sBC = sm + PL::BCC, *sDbC = sm + PL::DBC,
           *sDbeta = sm + PL::DBETA;
 
@@ -170,41 +189,62 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
     const size_t tok0 = (size_t)b * T;             // first token row of this sequence
     float* ck = ckpt + ((size_t)(b * H + h) * (Dv / BVC) + cb) * (size_t)NC * DK * BVC;
 
-    // per-channel prologue of chunk n: K+, K- (and Q+), r, b_C; masked rows past T
-    auto prologue = [&](int n, bool with_q) {
+    // rows [t0, t0 + BC) of a [B, T, H, W] tensor, columns [c0, c0 + NCOL), into an fp32
+    // tile with row stride ld (16-byte vector loads, zero past T)
+    auto stage = [&](float* dst, int ld, auto src, int W, int c0, auto ncol_tag, int n) {
+        using TS = typename std::remove_cv<typename std::remove_pointer<decltype(src)>::type>::type;
+        constexpr int NCOL = decltype(ncol_tag)::value;
+        constexpr int VE = 16 / (int)sizeof(TS), VPR = NCOL / VE;
         const int t0 = n * BC;
-        if (t < BC) sBeta[t] = (t0 + t < T) ? ld(beta + (tok0 + t0 + t) * rowH + h) : 0.f;
-        if (t < DK) {
-            const int c = t;
-            float bb[BC];
-            float run = 0.f;
+        for (int e = t; e < BC * VPR; e += BT) {
+            const int i = e / VPR, cv = (e % VPR) * VE;
+            float f[VE];
+            if (t0 + i < T) {
+                const uint4 u = *reinterpret_cast<const uint4*>(src + ((tok0 + t0 + i) * rowH + h) * W + c0 + cv);
+                unpack16(u, f, src);
+            } else {
 #pragma unroll
-            for (int i = 0; i < BC; ++i) {
-                const bool live = t0 + i < T;
-                run += live ? ld(g + ((tok0 + t0 + i) * rowH + h) * DK + c) : 0.f;
-                bb[i] = run;
+                for (int j = 0; j < VE; ++j) f[j] = 0.f;
             }
-            const float r = bb[15], bC = bb[BC - 1];
-            sR[c] = r;
-            sBC[c] = bC;
 #pragma unroll
-            for (int i = 0; i < BC; ++i) {
-                const bool live = t0 + i < T;
-                const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
-                const float kk = live ? ld(k + idx) : 0.f;
-                const float ep = expf(bb[i] - r), em = expf(r - bb[i]);
-                sKP[i * LDK + c] = kk * ep;
-                sKM[i * LDK + c] = kk * em;
-                if (with_q) sQP[i * LDK + c] = (live ? ld(q + idx) : 0.f) * ep;
-            }
+            for (int j = 0; j < VE; ++j) dst[i * ld + cv + j] = f[j];
         }
     };
-    // [BC][BVC] tile of a [B, T, H, Dv] tensor (this CTA's columns), zero past T
-    auto load_rows = [&](float* dst, auto src, int n) {
+    using KCols = std::integral_constant<int, DK>;
+    using VCols = std::integral_constant<int, BVC>;
+    // chunk n's k (-> K+ / K-), q (-> Q+), g (-> b), beta, v (and do) staged; then per
+    // channel: b = cumsum(g), r, b_C and the decay-scaled operands, in place
+    auto prologue = [&](int n, bool bwd) {
         const int t0 = n * BC;
-        for (int e = t; e < BC * BVC; e += BT) {
-            const int i = e / BVC, j = e % BVC;
-            dst[i * LDV + j] = (t0 + i < T) ? ld(src + ((tok0 + t0 + i) * rowH + h) * Dv + col0 + j) : 0.f;
+        if (t < BC) sBeta[t] = (t0 + t < T) ? ld(beta + (tok0 + t0 + t) * rowH + h) : 0.f;
+        stage(sKP, LDK, k, DK, 0, KCols{}, n);
+        stage(sB, LDK, g, DK, 0, KCols{}, n);
+        stage(sVX, LDV, v, Dv, col0, VCols{}, n);
+        if (bwd) {
+            stage(sQP, LDK, q, DK, 0, KCols{}, n);
+            stage(sDO, LDV, dout, Dv, col0, VCols{}, n);
+        }
+        __syncthreads();
+        if (t < DK) {
+            const int c = t;
+            float run = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < BC; ++i) {
+                run += sB[i * LDK + c];
+                sB[i * LDK + c] = run;
+            }
+            const float r = sB[15 * LDK + c];
+            sR[c] = r;
+            sBC[c] = run;
+#pragma unroll 4
+            for (int i = 0; i < BC; ++i) {
+                const float bi = sB[i * LDK + c];
+                const float ep = expf(bi - r), em = expf(r - bi);
+                const float kk = sKP[i * LDK + c];
+                sKP[i * LDK + c] = kk * ep;
+                sKM[i * LDK + c] = kk * em;
+                if (bwd) sQP[i * LDK + c] *= ep;
+            }
         }
     };
 
@@ -216,9 +256,11 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
     __syncthreads();
     for (int n = 0; n < NC; ++n) {
         float* ckn = ck + (size_t)n * DK * BVC;
-        for (int e = t; e < DK * BVC; e += BT) ckn[e] = sSe[(e / BVC) * LDS + e % BVC];
+        for (int e = t; e < DK * BVC / 4; e += BT) {
+            const float* d = sSe + (4 * e / BVC) * LDS + (4 * e) % BVC;
+            reinterpret_cast<float4*>(ckn)[e] = make_float4(d[0], d[1], d[2], d[3]);
+        }
         prologue(n, false);
-        load_rows(sVX, v, n);
         __syncthreads();
         mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK);
         for (int e = t; e < DK * BVC; e += BT) {
@@ -254,10 +296,12 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         const int t0 = n * BC;
         const float* ckn = ck + (size_t)n * DK * BVC;
         __syncthreads();   // the previous chunk is done with every tile
+        for (int e = t; e < DK * BVC / 4; e += BT) {
+            const float4 c4 = reinterpret_cast<const float4*>(ckn)[e];
+            float* d = sSe + (4 * e / BVC) * LDS + (4 * e) % BVC;
+            d[0] = c4.x; d[1] = c4.y; d[2] = c4.z; d[3] = c4.w;
+        }
         prologue(n, true);
-        load_rows(sVX, v, n);
-        load_rows(sDO, dout, n);
-        for (int e = t; e < DK * BVC; e += BT) sSe[(e / BVC) * LDS + e % BVC] = ckn[e];
         __syncthreads();
         // Kd, P; Se = Diag(e^r) S; Gc = Diag(e^{b_C - r}) G'
         mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK);
@@ -342,31 +386,34 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         mmt<DK, BVC, BC, MM_ADD>(sGp, LDS, sQP, 1, LDK, sDO, LDV, 1);   // Gc + Q+^T dO
         mmt<DK, BVC, BC, MM_SUB>(sGp, LDS, sKP, 1, LDK, sDR, LDV, 1);   //    - K+^T dRb
         __syncthreads();
-        if (t < DK) {   // per channel: dq, dk, db -> dg (reverse cumulative sum); G row scale
+        if (t < DK) {   // per channel: dq, dk, db -> dg (reverse cumulative sum), in place; G row scale
             const int c = t;
-            float bb[BC];
-            float run = 0.f;
-#pragma unroll
-            for (int i = 0; i < BC; ++i) {
-                run += (t0 + i < T) ? ld(g + ((tok0 + t0 + i) * rowH + h) * DK + c) : 0.f;
-                bb[i] = run;
-            }
             const float r = sR[c];
             float acc = sDbC[c];
-#pragma unroll
+#pragma unroll 4
             for (int i = BC - 1; i >= 0; --i) {
-                const float ep = expf(bb[i] - r), em = expf(r - bb[i]);
+                const float bi = sB[i * LDK + c];
+                const float ep = expf(bi - r), em = expf(r - bi);
                 const float dqp = sDQP[i * LDK + c], dkp = sDKP[i * LDK + c], dkm = sDKM[i * LDK + c];
                 acc += dqp * sQP[i * LDK + c] + dkp * sKP[i * LDK + c] - dkm * sKM[i * LDK + c];
-                if (t0 + i < T) {
-                    const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
-                    atomicAdd(dq + idx, dqp * ep);
-                    atomicAdd(dk + idx, dkp * ep + dkm * em);
-                    atomicAdd(dg + idx, acc);
-                }
+                sDQP[i * LDK + c] = dqp * ep;
+                sDKP[i * LDK + c] = dkp * ep + dkm * em;
+                sDKM[i * LDK + c] = acc;
             }
             const float er = expf(r);
             for (int j = 0; j < BVC; ++j) sGp[c * LDS + j] *= er;
+        }
+        __syncthreads();
+        for (int e = t; e < BC * DK / 4; e += BT) {   // dq, dk, dg += this CTA's part, 16 bytes at a time
+            const int i = e / (DK / 4), c = (e % (DK / 4)) * 4;
+            if (t0 + i >= T) continue;
+            const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
+            const float* a1 = sDQP + i * LDK + c;
+            const float* a2 = sDKP + i * LDK + c;
+            const float* a3 = sDKM + i * LDK + c;
+            atomicAdd(reinterpret_cast<float4*>(dq + idx), make_float4(a1[0], a1[1], a1[2], a1[3]));
+            atomicAdd(reinterpret_cast<float4*>(dk + idx), make_float4(a2[0], a2[1], a2[2], a2[3]));
+            atomicAdd(reinterpret_cast<float4*>(dg + idx), make_float4(a3[0], a3[1], a3[2], a3[3]));
         }
         if (t < BC && t0 + t < T) atomicAdd(dbeta + (tok0 + t0 + t) * rowH + h, sDbeta[t]);
     }
