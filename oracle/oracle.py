@@ -19,6 +19,9 @@ passages of the Chimera paper it follows, is stated in that file's header:
 * ``gated_rmsnorm`` / ``kda_forward_gated``: the output side of Eq. 15 (section 3.3),
   Sigmoid(gate) * RMSNorm(S_t^T q_t) per (token, head), before the output projection
   W_o (numpy, fp64).
+* ``mshortconv_backward``: the adjoint of ``mshortconv`` (linear in x and in w): dx and
+  the weight gradients per modality, by the same per-segment taps read backwards (numpy,
+  fp64).
 * ``kda_backward``: the reverse-mode derivative of the token recurrence of Eq. 14 with
   the readout of Eq. 15 (the pages give only the forward; the paper trains with it).
   Plain reverse sweep over the tokens in fp64 (numpy), from the states of a forward
@@ -299,6 +302,58 @@ def kda_forward_gated(q, k, v, g, beta, gate, gamma=None, eps=1e-6, S0=None, *, 
     """kda_forward followed by gated_rmsnorm of its readout; returns (y, S_T)."""
     o, S_T = kda_forward(q, k, v, g, beta, S0, pairs=pairs, nthreads=nthreads)
     return gated_rmsnorm(o, gate, gamma, eps), S_T
+
+
+def _taps(modality, Kt):
+    """(tap index, (df, dr, ds)) with y[f, r, s] += w[tap] * x[f + df, r + dr, s + ds]:
+    text j -> (0, 0, j - (Kt-1)); image (a, e) -> (0, a-1, e-1); video (tau, a, e) ->
+    (tau-2, a-1, e-1), taps numbered in the weight layout's row-major order."""
+    if modality == MOD_TEXT:
+        return [(j, (0, 0, j - (Kt - 1))) for j in range(Kt)]
+    if modality == MOD_IMAGE:
+        return [(3 * a + e, (0, a - 1, e - 1)) for a in range(3) for e in range(3)]
+    return [(9 * tau + 3 * a + e, (tau - 2, a - 1, e - 1)) for tau in range(3) for a in range(3) for e in range(3)]
+
+
+def mshortconv_backward(x, dy, segments, Kt, w_text=None, w_image=None, w_video=None):
+    """Gradients of L = sum(dy * mshortconv(x)) with respect to x and to the weights.
+
+    x, dy: [B,T,C]; weights as for mshortconv.  Returns (dx [B,T,C], dw_text, dw_image,
+    dw_video) in fp64, each dw with its weight's shape (None where the weight is None).
+    Inside a segment laid out as [F, Hgt, Wid] (text: [1, 1, len]),
+    y[p] = sum_tap w[c, tap] x[p + off(tap)] over in-segment positions, so
+      dx[p + off]       += w[c, tap] dy[p]
+      dw[c, tap]        += sum over rows b and positions p of dy[p] x[p + off]
+    for every tap whose shifted position stays inside the segment; tokens outside every
+    segment get dx = 0."""
+    X, DY = _to_f64(x), _to_f64(dy)
+    B, T, C = X.shape
+    dx = np.zeros((B, T, C))
+    ws = {}
+    for m, w in ((MOD_TEXT, w_text), (MOD_IMAGE, w_image), (MOD_VIDEO, w_video)):
+        ws[m] = None if w is None else _to_f64(w)
+    dws = {m: (None if w is None else np.zeros_like(w)) for m, w in ws.items()}
+    for (m, s0, F, Hh, Wd, wset) in segments:
+        F, Hh, Wd = (1, 1, Wd) if m == MOD_TEXT else ((1, Hh, Wd) if m == MOD_IMAGE else (F, Hh, Wd))
+        n = F * Hh * Wd
+        xs = X[:, s0:s0 + n].reshape(B, F, Hh, Wd, C)
+        gs = DY[:, s0:s0 + n].reshape(B, F, Hh, Wd, C)
+        dxs = np.zeros_like(xs)
+        wm = ws[m][wset].reshape(C, -1)
+        dwm = dws[m][wset].reshape(C, -1)
+        for tap, (df, dr, ds) in _taps(m, Kt):
+            # output positions p whose p + off lies in the segment
+            f0, f1 = max(0, -df), min(F, F - df)
+            r0, r1 = max(0, -dr), min(Hh, Hh - dr)
+            c0, c1 = max(0, -ds), min(Wd, Wd - ds)
+            if f0 >= f1 or r0 >= r1 or c0 >= c1:
+                continue
+            g_out = gs[:, f0:f1, r0:r1, c0:c1]
+            x_in = xs[:, f0 + df:f1 + df, r0 + dr:r1 + dr, c0 + ds:c1 + ds]
+            dxs[:, f0 + df:f1 + df, r0 + dr:r1 + dr, c0 + ds:c1 + ds] += wm[:, tap] * g_out
+            dwm[:, tap] += np.einsum("bfrsc,bfrsc->c", g_out, x_in)
+        dx[:, s0:s0 + n] = dxs.reshape(B, n, C)
+    return dx, dws[MOD_TEXT], dws[MOD_IMAGE], dws[MOD_VIDEO]
 
 
 def kda_backward(q, k, v, g, beta, do, S0=None, dS_T=None, *, block=64):
