@@ -528,6 +528,27 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                                        "frac": fmas / (mb * 1e-3) / fma_rate, "fmas_per_step": fmas,
                                        "peak_source": "kda_fma_probe on this GPU"},
                           "path": "fp32 CUDA cores, one CTA per (b, h, 32 value columns)"})
+        # mShortConv backward on the fused workload's stream (one tensor, x_q: dx and the
+        # three modalities' weight gradients); bound: plain ALU (its multiply-adds are the
+        # forward's twice over: dx and dw)
+        fw = W.FUSED_MIXED
+        fin = W.make_fused_inputs(fw, device="cuda")
+        dy_c = torch.randn(fw.B, fw.T, fw.H * fw.D, generator=torch.Generator().manual_seed(9)).to(fw.dtype).cuda()
+        wq = fin["wq"]
+
+        def cstep():
+            kda.mshortconv_backward(fin["xq"], dy_c, fin["segments"], fw.Kt, wq[0], wq[1], wq[2])
+        for _ in range(3):
+            cstep()
+        k_c = 5
+        mc = timed(cstep, k_c, 1) / k_c
+        cf = 2 * conv_fmas(fw) // 3
+        rate = kda.fma_probe()
+        extra.append({"workload": fw.name + "_conv_backward_xq", "ms_per_step": mc,
+                      "roofline": {"bound": "alu", "achieved": cf / (mc * 1e-3) / 1e12, "peak": rate / 1e12,
+                                   "unit": "TFMA/s", "frac": cf / (mc * 1e-3) / rate, "fmas_per_step": cf,
+                                   "peak_source": "kda_fma_probe on this GPU"},
+                      "path": "dx gather per (position, 8 channels); dw per-block reduction + atomics"})
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

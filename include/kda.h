@@ -302,6 +302,27 @@ kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_d
                               const float* w_video, int n_video_sets,
                               kda_stream_t stream);
 
+/*
+ * mshortconv_backward -- gradients of mshortconv_forward (section 3.4; the pages give only
+ * the forward).  For a loss L with dL/dy = dy:
+ *   x, dy    : [B, T, C] dtype (device); x is read only for the weight gradients.
+ *   dx       : [B, T, C] fp32 (device, written; 0 at tokens no segment covers).
+ *   segs ... w_video, n_*_sets : exactly as passed to mshortconv_forward.
+ *   dw_text, dw_image, dw_video : fp32 with the layouts of w_text, w_image, w_video
+ *              (device, written: zeroed, then summed over rows and segments), or NULL
+ *              to skip that modality's weight gradient.
+ * Inside a segment y[p] = sum_tap w[c,tap] x[p + off(tap)], so dx[p] = sum_tap w[c,tap]
+ * dy[p - off(tap)] and dw[c,tap] = sum_{rows,p} dy[p] x[p + off(tap)], with positions
+ * outside the segment reading zero.  Errors: as mshortconv_forward.
+ */
+kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, int T, int C,
+                               kda_dtype dtype, const msc_segment* segs, int n_segs, int Kt,
+                               const float* w_text, int n_text_sets,
+                               const float* w_image, int n_image_sets,
+                               const float* w_video, int n_video_sets,
+                               float* dw_text, float* dw_image, float* dw_video,
+                               kda_stream_t stream);
+
 /* Bytes of workspace kda_mshortconv_forward needs. */
 size_t kda_mshortconv_workspace_size(int B, int T, int H, int D, kda_dtype dtype,
                                      kda_dtype o_dtype, int chunk);
@@ -363,7 +384,7 @@ void kda_profile_enable(int on);
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
  * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
- * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold", "kda_bwd". */
+ * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold", "kda_bwd", "conv_bwd". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

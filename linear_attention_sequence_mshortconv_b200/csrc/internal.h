@@ -124,4 +124,9 @@ cudaError_t launch_conv_segment_multi(int nt, const void* const* xs, void* const
                                       ElemType in_t, ElemType out_t, const ConvSeg& seg, int Kt,
                                       const float* const* ws, const int* norm_Ds, cudaStream_t s);
 
+// Backward of the conv of one segment: dx over the segment's tokens (written), dw (this
+// segment's weight set, accumulated with atomics; nullptr = skip).  x, dy: [B,T,C] in_t.
+cudaError_t launch_conv_backward_segment(const void* x, const void* dy, float* dx, const float* w, float* dw, int B,
+                                         int T, int C, ElemType in_t, const ConvSeg& seg, int Kt, cudaStream_t s);
+
 }  // namespace kda

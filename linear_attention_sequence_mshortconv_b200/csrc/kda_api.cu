@@ -421,6 +421,42 @@ kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_d
 
 // The fused path keeps q, k, v between the conv and the scan as fp16 (fp32 inputs:
 // fp32) in the workspace.
+kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, int T, int C, kda_dtype dtype,
+                               const msc_segment* segs, int n_segs, int Kt, const float* w_text, int n_text_sets,
+                               const float* w_image, int n_image_sets, const float* w_video, int n_video_sets,
+                               float* dw_text, float* dw_image, float* dw_video, kda_stream_t stream)
+{
+    if (B < 0 || T < 0 || C <= 0 || (C % 8) != 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    const bool want_dw = dw_text || dw_image || dw_video;
+    if ((int64_t)B * T > 0 && (!dy || !dx || (want_dw && !x))) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_segments(segs, n_segs, T, Kt, w_text, n_text_sets, w_image,
+                                   n_image_sets, w_video, n_video_sets);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    // weight gradients are sums over rows and segments: zeroed, then accumulated
+    if (dw_text && n_text_sets > 0) e = cudaMemsetAsync(dw_text, 0, (size_t)n_text_sets * C * Kt * sizeof(float), s);
+    if (e == cudaSuccess && dw_image && n_image_sets > 0)
+        e = cudaMemsetAsync(dw_image, 0, (size_t)n_image_sets * C * 9 * sizeof(float), s);
+    if (e == cudaSuccess && dw_video && n_video_sets > 0)
+        e = cudaMemsetAsync(dw_video, 0, (size_t)n_video_sets * C * 27 * sizeof(float), s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    if ((int64_t)B * T == 0) return KDA_OK;
+    if (cudaMemsetAsync(dx, 0, (size_t)B * T * C * sizeof(float), s) != cudaSuccess) return KDA_ERR_CUDA;
+    const ElemType et = dtype == KDA_F32 ? ET_F32 : ET_BF16;
+    for (int i = 0; i < n_segs; ++i) {
+        const msc_segment& sg = segs[i];
+        float* dw_all = sg.modality == MSC_TEXT ? dw_text : sg.modality == MSC_IMAGE ? dw_image : dw_video;
+        const int ntaps = sg.modality == MSC_TEXT ? Kt : sg.modality == MSC_IMAGE ? 9 : 27;
+        float* dw = dw_all ? dw_all + (int64_t)sg.weight_set * C * ntaps : nullptr;
+        e = launch_conv_backward_segment(x, dy, dx, seg_weights(sg, C, Kt, w_text, w_image, w_video), dw, B, T, C,
+                                         et, to_conv_seg(sg), Kt, s);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
 static KdaArgs fused_kda_args(int B, int T, int H, int D, kda_dtype dtype, kda_dtype o_dtype,
                               int chunk)
 {

@@ -29,7 +29,7 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
             "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size",
             "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output",
-            "kda_backward", "kda_backward_workspace_size")
+            "kda_backward", "kda_backward_workspace_size", "mshortconv_backward")
 
 
 class KdaError(RuntimeError):
@@ -101,6 +101,8 @@ def load_library(path: str = LIB_PATH):
         lib.kda_backward_workspace_size.argtypes = [I, I, I, I, I]
         lib.kda_backward.restype = I
         lib.kda_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
+        lib.mshortconv_backward.restype = I
+        lib.mshortconv_backward.argtypes = [P, P, P, I, I, I, I, P, I, I, P, I, P, I, P, I, P, P, P, P]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -449,6 +451,34 @@ def mshortconv(x, segments, Kt, w_text=None, w_image=None, w_video=None, *, y=No
                                 _stream(stream))
     _check("mshortconv_forward", rc)
     return y
+
+
+def mshortconv_backward(x, dy, segments, Kt, w_text=None, w_image=None, w_video=None, *,
+                        want_dw: bool = True, stream=None):
+    """mshortconv_backward: (dx [B,T,C] fp32, dw_text, dw_image, dw_video) for dL/dy = dy
+    through mshortconv(x, ...); each dw has its weight's shape (None where the weight is
+    None or want_dw is False)."""
+    lib = load_library()
+    B, T, C = x.shape
+    if tuple(dy.shape) != (B, T, C) or dy.dtype != x.dtype:
+        raise ValueError("dy must match x in shape and dtype")
+    dt = _dtype_code(x)
+    dx = torch.empty((B, T, C), dtype=torch.float32, device=x.device)
+    segs, n = make_segments(segments)
+    dws = [None if (w is None or not want_dw) else torch.empty_like(w, dtype=torch.float32)
+           for w in (w_text, w_image, w_video)]
+
+    def wsets(w):
+        return (0 if w is None else int(w.shape[0]))
+
+    rc = lib.mshortconv_backward(_dev(x, "x"), _dev(dy, "dy"), _dev(dx, "dx", torch.float32), B, T, C, dt,
+                                 ctypes.cast(segs, ctypes.c_void_p), n, int(Kt),
+                                 _dev(w_text, "w_text", torch.float32), wsets(w_text),
+                                 _dev(w_image, "w_image", torch.float32), wsets(w_image),
+                                 _dev(w_video, "w_video", torch.float32), wsets(w_video),
+                                 *[_dev(d, "dw", torch.float32) for d in dws], _stream(stream))
+    _check("mshortconv_backward", rc)
+    return (dx, *dws)
 
 
 def mshortconv_workspace_size(B, T, H, D, dtype=torch.bfloat16, chunk=0, o_dtype=None) -> int:

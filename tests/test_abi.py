@@ -107,6 +107,18 @@ def test_backward_rejects_bad_arguments(lib):
     assert lib.kda_backward_workspace_size(1, 64, 2, 48, 64) == 0
 
 
+def test_conv_backward_rejects_bad_arguments(lib):
+    segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
+    d = ctypes.c_void_p(256)   # never dereferenced: validation fails first
+    sp = ctypes.cast(segs, ctypes.c_void_p)
+    P = None
+    # no dx with work to do; dw wanted without x; Kt outside 1..8; C not a multiple of 8
+    assert lib.mshortconv_backward(d, d, P, 1, 10, 16, 1, sp, n, 4, d, 1, P, 0, P, 0, P, P, P, P) == 1
+    assert lib.mshortconv_backward(P, d, d, 1, 10, 16, 1, sp, n, 4, d, 1, P, 0, P, 0, d, P, P, P) == 1
+    assert lib.mshortconv_backward(d, d, d, 1, 10, 16, 1, sp, n, 9, d, 1, P, 0, P, 0, P, P, P, P) == 2
+    assert lib.mshortconv_backward(d, d, d, 1, 10, 12, 1, sp, n, 4, d, 1, P, 0, P, 0, P, P, P, P) == 1
+
+
 def test_conv_rejects_bad_segment_tables(lib):
     segs, n = kda.make_segments([(kda.MSC_TEXT, 0, 1, 1, 10, 0)])
     dummy = ctypes.c_void_p(16)   # never dereferenced: validation fails first
