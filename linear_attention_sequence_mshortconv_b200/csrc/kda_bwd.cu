@@ -26,12 +26,13 @@
 // tokens must stay within |sum g| < ~80 (mean g > -2.5 per token); beyond that the
 // results are not finite.
 //
+// Every matrix product runs on the tensor cores as 3xTF32 warp MMAs (fp32 accuracy).
 // Parallel split: the state's value columns evolve independently, so one CTA owns 32
 // value columns of one (b, h).  It first runs the forward over all chunks and stores
 // each chunk's entry state (its 32 columns) in the workspace, then walks the chunks in
 // reverse.  dv and dS0 columns belong to one CTA; dq, dk, dg and dbeta are sums over
 // the value columns and are accumulated with atomic adds (the outputs are zeroed first).
-// All arithmetic is fp32 on CUDA cores.
+// Everything else is fp32 on CUDA cores.
 
 #include <type_traits>
 
@@ -43,12 +44,14 @@ namespace {
 constexpr int BC = 32;        // chunk length
 constexpr int BVC = 32;       // value columns per CTA
 constexpr int BT = 256;       // threads per CTA
-constexpr int LDV = BVC + 1;  // row stride of [BC][BVC] tiles (floats)
-constexpr int LDC = BC + 1;   // row stride of [BC][BC] tiles
+// Row strides (floats) are 4 mod 32, so the 8 x 4 lane pattern of a warp MMA fragment
+// load touches 32 different banks for row-major operands.
+constexpr int LDV = BVC + 4;  // row stride of [BC][BVC] tiles
+constexpr int LDC = BC + 4;   // row stride of [BC][BC] tiles
 
 template <int DK> struct BwdPlan {
-    static constexpr int LDK = DK + 1;    // [BC][DK] tiles
-    static constexpr int LDS = BVC + 1;   // [DK][BVC] tiles
+    static constexpr int LDK = DK + 4;    // [BC][DK] tiles
+    static constexpr int LDS = BVC + 4;   // [DK][BVC] tiles
     static constexpr int KP = 0, KM = KP + BC * LDK, QP = KM + BC * LDK;
     static constexpr int DQP = QP + BC * LDK, DKP = DQP + BC * LDK, DKM = DKP + BC * LDK;
     static constexpr int SE = DKM + BC * LDK, GP = SE + DK * LDS;
@@ -64,61 +67,63 @@ template <int DK> struct BwdPlan {
 
 enum { MM_SET = 0, MM_ADD = 1, MM_SUB = 2, MM_NEG = 3 };
 
-// out(i, j) op= sum_{k<K} A(i, k) B(k, j) for i < M, j < N, over threads
-// [tid0, tid0 + nthr).  A(i, k) = A[i*ai + k*ak], B(k, j) = B[k*bk + j*bj],
-// out(i, j) = O[i*oi + j].  A thread owns a TM x TN micro-tile with strided rows and
-// columns (ti + m*M/TM, tj + n*N/TN), so a warp's B reads hit consecutive columns.
-template <int M, int N, int K, int TM, int TN, int OP>
-__device__ __forceinline__ void mm(float* O, int oi, const float* A, int ai, int ak, const float* B, int bk, int bj,
-                                   int tid0 = 0, int nthr = BT)
+// out(i, j) op= sum_{k<K} A(i, k) B(k, j) for i < M, j < N, on the tensor cores, by the
+// warps of threads [tid0, tid0 + nthr).  A(i, k) = A[i*ai + k*ak], B(k, j) = B[k*bk + j*bj],
+// out(i, j) = O[i*oi + j], all in shared memory.  Warp MMAs m16n8k8 with tf32 operands:
+// each fp32 operand is split as hi + lo (hi = tf32(x), lo = tf32(x - hi)) and the product
+// taken as lo*hi + hi*lo + hi*hi ("3xTF32"), which keeps fp32 accuracy.  16 x 8 output
+// tiles are dealt to the warps in turn.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo)
 {
-    static_assert(M % TM == 0 && N % TN == 0, "micro-tile");
-    constexpr int GM = M / TM, GN = N / TN, NTILE = GM * GN;
-    for (int tile = (int)threadIdx.x - tid0; tile < NTILE; tile += nthr) {
-        if (tile < 0) break;
-        const int ti = tile / GN, tj = tile % GN;
-        float acc[TM][TN];
-#pragma unroll
-        for (int m = 0; m < TM; ++m)
-#pragma unroll
-            for (int n = 0; n < TN; ++n) acc[m][n] = 0.f;
-#pragma unroll 4
-        for (int k = 0; k < K; ++k) {
-            float a[TM], b[TN];
-#pragma unroll
-            for (int m = 0; m < TM; ++m) a[m] = A[(ti + m * GM) * ai + k * ak];
-#pragma unroll
-            for (int n = 0; n < TN; ++n) b[n] = B[k * bk + (tj + n * GN) * bj];
-#pragma unroll
-            for (int m = 0; m < TM; ++m)
-#pragma unroll
-                for (int n = 0; n < TN; ++n) acc[m][n] = fmaf(a[m], b[n], acc[m][n]);
-        }
-#pragma unroll
-        for (int m = 0; m < TM; ++m)
-#pragma unroll
-            for (int n = 0; n < TN; ++n) {
-                float* o = O + (ti + m * GM) * oi + (tj + n * GN);
-                if (OP == MM_SET) *o = acc[m][n];
-                else if (OP == MM_ADD) *o += acc[m][n];
-                else if (OP == MM_SUB) *o -= acc[m][n];
-                else *o = -acc[m][n];
-            }
-    }
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float r = x - __uint_as_float(hi);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
 }
 
-// Micro-tile sizes for an M x N output over 256 threads.
-template <int M, int N> struct Tile {
-    static constexpr int per = M * N / BT;
-    static constexpr int TM = per >= 16 ? 4 : 2;
-    static constexpr int TN = per / TM;
-};
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
 
 template <int M, int N, int K, int OP>
 __device__ __forceinline__ void mmt(float* O, int oi, const float* A, int ai, int ak, const float* B, int bk, int bj,
                                     int tid0 = 0, int nthr = BT)
 {
-    mm<M, N, K, Tile<M, N>::TM, Tile<M, N>::TN, OP>(O, oi, A, ai, ak, B, bk, bj, tid0, nthr);
+    static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "warp MMA tiles");
+    constexpr int TN = N / 8, NTILE = (M / 16) * TN;
+    const int w0 = tid0 >> 5, nw = nthr >> 5;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    for (int tile = (int)(threadIdx.x >> 5) - w0; tile < NTILE; tile += nw) {
+        if (tile < 0) break;
+        const int i0 = (tile / TN) * 16, j0 = (tile % TN) * 8;
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        const float* a0 = A + (i0 + g) * ai + q * ak;
+        const float* b0 = B + q * bk + (j0 + g) * bj;
+#pragma unroll 4
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            split_tf32(a0[k0 * ak], ah[0], al[0]);
+            split_tf32(a0[8 * ai + k0 * ak], ah[1], al[1]);
+            split_tf32(a0[(k0 + 4) * ak], ah[2], al[2]);
+            split_tf32(a0[8 * ai + (k0 + 4) * ak], ah[3], al[3]);
+            split_tf32(b0[k0 * bk], bh[0], bl[0]);
+            split_tf32(b0[(k0 + 4) * bk], bh[1], bl[1]);
+            mma_tf32(c, al, bh);
+            mma_tf32(c, ah, bl);
+            mma_tf32(c, ah, bh);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float* o = O + (i0 + g + (e >> 1) * 8) * oi + j0 + 2 * q + (e & 1);
+            if (OP == MM_SET) *o = c[e];
+            else if (OP == MM_ADD) *o += c[e];
+            else if (OP == MM_SUB) *o -= c[e];
+            else *o = -c[e];
+        }
+    }
 }
 
 template <typename T> __device__ __forceinline__ float ld(const T* p) { return to_f32(*p); }
