@@ -22,6 +22,9 @@ passages of the Chimera paper it follows, is stated in that file's header:
 * ``mshortconv_backward``: the adjoint of ``mshortconv`` (linear in x and in w): dx and
   the weight gradients per modality, by the same per-segment taps read backwards (numpy,
   fp64).
+* ``l2norm_heads_backward`` / ``fused_backward``: the derivative of the per-head unit
+  normalisation and the chain rule through the fused forward (conv -> norm -> scan),
+  composed from the other backward routines (numpy, fp64).
 * ``kda_backward``: the reverse-mode derivative of the token recurrence of Eq. 14 with
   the readout of Eq. 15 (the pages give only the forward; the paper trains with it).
   Plain reverse sweep over the tokens in fp64 (numpy), from the states of a forward
@@ -302,6 +305,42 @@ def kda_forward_gated(q, k, v, g, beta, gate, gamma=None, eps=1e-6, S0=None, *, 
     """kda_forward followed by gated_rmsnorm of its readout; returns (y, S_T)."""
     o, S_T = kda_forward(q, k, v, g, beta, S0, pairs=pairs, nthreads=nthreads)
     return gated_rmsnorm(o, gate, gamma, eps), S_T
+
+
+def l2norm_heads_backward(x, dy, H):
+    """Gradient through y = x / |x| per head slice (length D of the last axis H*D):
+    dx = (dy - y (y . dy)) / |x|, and 0 where |x| = 0 (y = 0 there, a constant)."""
+    X, G = _to_f64(x), _to_f64(dy)
+    shp = X.shape
+    D = shp[-1] // H
+    Xh, Gh = X.reshape(-1, H, D), G.reshape(-1, H, D)
+    n = np.sqrt(np.sum(Xh * Xh, axis=-1, keepdims=True))
+    with np.errstate(invalid="ignore", divide="ignore"):
+        Y = np.where(n > 0, Xh / n, 0.0)
+        dX = np.where(n > 0, (Gh - Y * np.sum(Y * Gh, axis=-1, keepdims=True)) / n, 0.0)
+    return dX.reshape(shp)
+
+
+def fused_backward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, H, do, S0=None, dS_T=None):
+    """Gradients of L = sum(do * o) + sum(dS_T * S_T) through fused_forward: returns
+    (dxq, dxk, dxv, dwq, dwk, dwv, dg, dbeta, dS0), each dw* a tuple (text, image, video)
+    like w*.  Chain rule: the scan's backward on (q, k, v), then the norm's backward on
+    dq, dk, then the conv's backward per tensor."""
+    yq = mshortconv(xq, segments, Kt, *wq)
+    yk = mshortconv(xk, segments, Kt, *wk)
+    yv = mshortconv(xv, segments, Kt, *wv)
+    B, T, C = yq.shape
+    D = C // H
+    q = l2norm_heads(yq, H).reshape(B, T, H, D)
+    k = l2norm_heads(yk, H).reshape(B, T, H, D)
+    v = yv.reshape(B, T, H, D)
+    dq, dk, dv, dg, dbeta, dS0 = kda_backward(q, k, v, _to_f64(g), _to_f64(beta), do, S0, dS_T)
+    dyq = l2norm_heads_backward(yq, dq.reshape(B, T, C), H)
+    dyk = l2norm_heads_backward(yk, dk.reshape(B, T, C), H)
+    gq = mshortconv_backward(xq, dyq, segments, Kt, *wq)
+    gk = mshortconv_backward(xk, dyk, segments, Kt, *wk)
+    gv = mshortconv_backward(xv, dv.reshape(B, T, C), segments, Kt, *wv)
+    return gq[0], gk[0], gv[0], gq[1:], gk[1:], gv[1:], dg, dbeta, dS0
 
 
 def _taps(modality, Kt):
