@@ -553,6 +553,20 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                                    "unit": "TFMA/s", "frac": cf / (mc * 1e-3) / rate, "fmas_per_step": cf,
                                    "peak_source": "kda_fma_probe on this GPU"},
                       "path": "shared-memory tiles (8 rows x 16 positions + halo, 64 channels), register windows; dw one atomic per (channel, tap) per tile"})
+        # backward of the whole fused path on the fused workload (kda_mshortconv_backward)
+        fb_do = torch.randn(fw.B, fw.T, fw.H, fw.D, generator=torch.Generator().manual_seed(10)).to(fw.dtype).cuda()
+        fb_ws = torch.empty(max(1, kda.mshortconv_kda_backward_workspace_size(fw.B, fw.T, fw.H, fw.D, fw.dtype)),
+                            dtype=torch.uint8, device="cuda")
+
+        def fbstep():
+            kda.mshortconv_kda_backward(fin["xq"], fin["xk"], fin["xv"], fin["segments"], fw.Kt, fin["wq"], fin["wk"],
+                                        fin["wv"], fin["g"], fin["beta"], fb_do, workspace=fb_ws)
+        for _ in range(2):
+            fbstep()
+        mf = timed(fbstep, 3, 1) / 3
+        extra.append({"workload": fw.name + "_backward", "ms_per_step": mf,
+                      "value": fw.tokens / (mf * 1e-3) / 1e6, "unit": UNIT,
+                      "path": "fp32 conv recompute, per-head norm, kda_backward, norm and conv backward"})
         line["extra_workloads"] = extra
     if rank == 0:
         print(json.dumps(line), flush=True)

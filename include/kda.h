@@ -352,6 +352,35 @@ kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv
                                   void* workspace, size_t workspace_bytes,
                                   kda_stream_t stream);
 
+/*
+ * kda_mshortconv_backward -- gradients of kda_mshortconv_forward (the pages give only the
+ * forward): for dL/do = d_o and dL/dS_T = dS_T, the gradients of x_q, x_k, x_v, of the
+ * three tensors' conv weights, of g, beta and S0.
+ *   xq ... D, dtype : exactly as passed to kda_mshortconv_forward.
+ *   d_o   : [B, T, H, D] in do_dtype;  dS_T : [B, H, D, D] fp32 or NULL (zeros).
+ *   dxq, dxk, dxv : [B, T, H*D] fp32 (written).
+ *   dwq, dwk, dwv : each an array of 3 pointers {text, image, video}, fp32 with the
+ *                   layouts of wq[i] (one weight set), or NULL entries to skip.
+ *   dg : [B, T, H, D] fp32;  dbeta : [B, T, H] fp32;  dS0 : [B, H, D, D] fp32 or NULL.
+ * The chain rule runs in fp32: the conv outputs are recomputed, q and k normalised, the
+ * scan's backward (as kda_backward) gives dq, dk, dv, the norm's derivative
+ * dy = (dq - q (q . dq)) / |y| per (token, head) (0 where |y| = 0) maps dq, dk back, and
+ * the conv backward (as mshortconv_backward) gives dx and the weight gradients.
+ * workspace: kda_mshortconv_backward_workspace_size bytes (NULL: allocated in the call).
+ * Errors: as kda_backward and mshortconv_backward.
+ */
+size_t kda_mshortconv_backward_workspace_size(int B, int T, int H, int D, kda_dtype dtype);
+kda_status kda_mshortconv_backward(const void* xq, const void* xk, const void* xv,
+                                   const msc_segment* segs, int n_segs, int Kt,
+                                   const float* const wq[3], const float* const wk[3],
+                                   const float* const wv[3], const void* g, const void* beta,
+                                   const float* S0, const void* d_o, kda_dtype do_dtype,
+                                   const float* dS_T, float* dxq, float* dxk, float* dxv,
+                                   float* const dwq[3], float* const dwk[3], float* const dwv[3],
+                                   float* dg, float* dbeta, float* dS0, int B, int T, int H, int D,
+                                   kda_dtype dtype, void* workspace, size_t workspace_bytes,
+                                   kda_stream_t stream);
+
 /* ---- diagnostics ---------------------------------------------------------------- */
 
 /* Number of kernels this library has launched in this process (all devices). */

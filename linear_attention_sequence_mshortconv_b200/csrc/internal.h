@@ -129,4 +129,10 @@ cudaError_t launch_conv_segment_multi(int nt, const void* const* xs, void* const
 cudaError_t launch_conv_backward_segment(const void* x, const void* dy, float* dx, const float* w, float* dw, int B,
                                          int T, int C, ElemType in_t, const ConvSeg& seg, int Kt, cudaStream_t s);
 
+// Elementwise pieces of the fused backward: widen to fp32 (bf16/fp16/fp32 source), and
+// per-row unit norm of rows of D values and its derivative (in place on d).
+cudaError_t launch_to_f32(const void* x, ElemType t, float* y, int64_t n, cudaStream_t s);
+cudaError_t launch_l2norm_rows(const float* x, float* y, int64_t rows, int D, cudaStream_t s);
+cudaError_t launch_l2norm_bwd_rows(const float* x, float* d, int64_t rows, int D, cudaStream_t s);
+
 }  // namespace kda

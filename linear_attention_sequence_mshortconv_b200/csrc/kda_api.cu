@@ -419,21 +419,13 @@ kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_d
     return KDA_OK;
 }
 
-// The fused path keeps q, k, v between the conv and the scan as fp16 (fp32 inputs:
-// fp32) in the workspace.
-kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, int T, int C, kda_dtype dtype,
-                               const msc_segment* segs, int n_segs, int Kt, const float* w_text, int n_text_sets,
-                               const float* w_image, int n_image_sets, const float* w_video, int n_video_sets,
-                               float* dw_text, float* dw_image, float* dw_video, kda_stream_t stream)
+// The conv backward after validation: dw zeroed then accumulated, dx zeroed then written
+// over the segments.  x, dy: [B, T, C] of element type et.
+static kda_status conv_backward_run(const void* x, const void* dy, float* dx, int B, int T, int C, ElemType et,
+                                    const msc_segment* segs, int n_segs, int Kt, const float* w_text, int n_text_sets,
+                                    const float* w_image, int n_image_sets, const float* w_video, int n_video_sets,
+                                    float* dw_text, float* dw_image, float* dw_video, cudaStream_t s)
 {
-    if (B < 0 || T < 0 || C <= 0 || (C % 8) != 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
-    const bool want_dw = dw_text || dw_image || dw_video;
-    if ((int64_t)B * T > 0 && (!dy || !dx || (want_dw && !x))) return KDA_ERR_INVALID_ARG;
-    kda_status st = check_segments(segs, n_segs, T, Kt, w_text, n_text_sets, w_image,
-                                   n_image_sets, w_video, n_video_sets);
-    if (st != KDA_OK) return st;
-    cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
     // weight gradients are sums over rows and segments: zeroed, then accumulated
     if (dw_text && n_text_sets > 0) e = cudaMemsetAsync(dw_text, 0, (size_t)n_text_sets * C * Kt * sizeof(float), s);
@@ -444,7 +436,6 @@ kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, 
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     if ((int64_t)B * T == 0) return KDA_OK;
     if (cudaMemsetAsync(dx, 0, (size_t)B * T * C * sizeof(float), s) != cudaSuccess) return KDA_ERR_CUDA;
-    const ElemType et = dtype == KDA_F32 ? ET_F32 : ET_BF16;
     for (int i = 0; i < n_segs; ++i) {
         const msc_segment& sg = segs[i];
         float* dw_all = sg.modality == MSC_TEXT ? dw_text : sg.modality == MSC_IMAGE ? dw_image : dw_video;
@@ -457,6 +448,25 @@ kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, 
     return KDA_OK;
 }
 
+kda_status mshortconv_backward(const void* x, const void* dy, float* dx, int B, int T, int C, kda_dtype dtype,
+                               const msc_segment* segs, int n_segs, int Kt, const float* w_text, int n_text_sets,
+                               const float* w_image, int n_image_sets, const float* w_video, int n_video_sets,
+                               float* dw_text, float* dw_image, float* dw_video, kda_stream_t stream)
+{
+    if (B < 0 || T < 0 || C <= 0 || (C % 8) != 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
+    const bool want_dw = dw_text || dw_image || dw_video;
+    if ((int64_t)B * T > 0 && (!dy || !dx || (want_dw && !x))) return KDA_ERR_INVALID_ARG;
+    kda_status st = check_segments(segs, n_segs, T, Kt, w_text, n_text_sets, w_image,
+                                   n_image_sets, w_video, n_video_sets);
+    if (st != KDA_OK) return st;
+    return conv_backward_run(x, dy, dx, B, T, C, dtype == KDA_F32 ? ET_F32 : ET_BF16, segs, n_segs, Kt, w_text,
+                             n_text_sets, w_image, n_image_sets, w_video, n_video_sets, dw_text, dw_image, dw_video,
+                             (cudaStream_t)stream);
+}
+
+// The fused path keeps q, k, v between the conv and the scan as fp16 (fp32 inputs:
+// fp32) in the workspace.
 static KdaArgs fused_kda_args(int B, int T, int H, int D, kda_dtype dtype, kda_dtype o_dtype,
                               int chunk)
 {
@@ -532,6 +542,142 @@ kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv
     KdaArgs a = fused_kda_args(B, T, H, D, dtype, o_dtype, chunk);
     a.q = qb; a.k = kb; a.v = vb; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.ST = S_T;
     return run_kda(a, kws, need - 3 * qkv, s);
+}
+
+}  // extern "C"
+
+// ---- backward of the fused path --------------------------------------------------------
+namespace {
+struct FusedBwdLayout {
+    size_t x32, g32, b32, y, qk, d, bws, total;   // offsets (bytes)
+};
+FusedBwdLayout fused_bwd_layout(int B, int T, int H, int D, kda_dtype dtype)
+{
+    const size_t tok = (size_t)B * T * H * D, f = sizeof(float);
+    const bool widen = dtype != KDA_F32;
+    FusedBwdLayout l{};
+    size_t off = 0;
+    l.x32 = off; off += widen ? 3 * align256(tok * f) : 0;
+    l.g32 = off; off += widen ? align256(tok * f) : 0;
+    l.b32 = off; off += widen ? align256((size_t)B * T * H * f) : 0;
+    l.y = off;   off += 3 * align256(tok * f);   // conv outputs y_q, y_k, y_v
+    l.qk = off;  off += 2 * align256(tok * f);   // q, k
+    l.d = off;   off += 3 * align256(tok * f);   // dq, dk, dv
+    l.bws = off; off += align256(kda_bwd_workspace_bytes(B, T, H, D, D));
+    l.total = off;
+    return l;
+}
+}  // namespace
+
+extern "C" {
+
+size_t kda_mshortconv_backward_workspace_size(int B, int T, int H, int D, kda_dtype dtype)
+{
+    if (B < 0 || T < 0 || H <= 0 || !dim_ok(D) || (dtype != KDA_F32 && dtype != KDA_BF16)) return 0;
+    if ((int64_t)B * T == 0) return 0;
+    return fused_bwd_layout(B, T, H, D, dtype).total;
+}
+
+kda_status kda_mshortconv_backward(const void* xq, const void* xk, const void* xv, const msc_segment* segs,
+                                   int n_segs, int Kt, const float* const wq[3], const float* const wk[3],
+                                   const float* const wv[3], const void* g, const void* beta, const float* S0,
+                                   const void* d_o, kda_dtype do_dtype, const float* dS_T, float* dxq, float* dxk,
+                                   float* dxv, float* const dwq[3], float* const dwk[3], float* const dwv[3],
+                                   float* dg, float* dbeta, float* dS0, int B, int T, int H, int D, kda_dtype dtype,
+                                   void* workspace, size_t workspace_bytes, kda_stream_t stream)
+{
+    if (!wq || !wk || !wv || !dwq || !dwk || !dwv) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || T < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if ((dtype != KDA_F32 && dtype != KDA_BF16) || (do_dtype != KDA_F32 && do_dtype != KDA_BF16))
+        return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(D) || B > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T > 0 && (!xq || !xk || !xv || !g || !beta || !d_o || !dxq || !dxk || !dxv || !dg || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const int C = H * D;
+    for (const float* const* w : {wq, wk, wv}) {
+        const kda_status st = check_segments(segs, n_segs, T, Kt, w[0], 1, w[1], 1, w[2], 1);
+        if (st != KDA_OK) return st;
+    }
+    if (B == 0) return KDA_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) {   // no tokens: zero weight gradients, dS0 = dS_T
+        for (float* const* dw : {dwq, dwk, dwv})
+            for (int m = 0; m < 3; ++m)
+                if (dw[m] && cudaMemsetAsync(dw[m], 0, (size_t)C * (m == 0 ? Kt : m == 1 ? 9 : 27) * sizeof(float), s) !=
+                                 cudaSuccess)
+                    return KDA_ERR_CUDA;
+        return kda_backward(nullptr, nullptr, nullptr, nullptr, nullptr, S0, nullptr, dS_T, nullptr, nullptr, nullptr,
+                            nullptr, nullptr, dS0, B, 0, H, D, D, dtype, do_dtype, nullptr, 0, stream);
+    }
+    const FusedBwdLayout L = fused_bwd_layout(B, T, H, D, dtype);
+    Workspace ws;
+    kda_status st = ws.acquire(workspace, workspace_bytes, L.total, s);
+    if (st != KDA_OK) return st;
+    char* base = (char*)ws.ptr;
+    const size_t tok = (size_t)B * T * C;
+    const size_t tb = align256(tok * sizeof(float));
+    // 0. fp32 copies of bf16 inputs
+    const void* xs[3] = {xq, xk, xv};
+    const float* x32[3];
+    const float *g32 = (const float*)g, *b32 = (const float*)beta;
+    cudaError_t e = cudaSuccess;
+    if (dtype == KDA_BF16) {
+        for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
+            float* dst = (float*)(base + L.x32 + i * tb);
+            e = launch_to_f32(xs[i], ET_BF16, dst, (int64_t)tok, s);
+            x32[i] = dst;
+        }
+        if (e == cudaSuccess) e = launch_to_f32(g, ET_BF16, (float*)(base + L.g32), (int64_t)tok, s);
+        if (e == cudaSuccess) e = launch_to_f32(beta, ET_BF16, (float*)(base + L.b32), (int64_t)B * T * H, s);
+        g32 = (const float*)(base + L.g32);
+        b32 = (const float*)(base + L.b32);
+    } else {
+        for (int i = 0; i < 3; ++i) x32[i] = (const float*)xs[i];
+    }
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    // 1. conv outputs, fp32
+    float* y[3];
+    const float* const* ws3[3] = {wq, wk, wv};
+    for (int i = 0; i < 3; ++i) {
+        y[i] = (float*)(base + L.y + i * tb);
+        e = zero_gaps(y[i], B, T, C, sizeof(float), segs, n_segs, s);
+        for (int j = 0; j < n_segs && e == cudaSuccess; ++j) {
+            msc_segment sg = segs[j];
+            sg.weight_set = 0;
+            e = launch_conv_segment(x32[i], y[i], B, T, C, ET_F32, ET_F32, to_conv_seg(sg), Kt,
+                                    seg_weights(sg, C, Kt, ws3[i][0], ws3[i][1], ws3[i][2]), 0, s);
+        }
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    // 2. q, k = unit rows per (token, head)
+    float* q = (float*)(base + L.qk);
+    float* k = (float*)(base + L.qk + tb);
+    e = launch_l2norm_rows(y[0], q, (int64_t)B * T * H, D, s);
+    if (e == cudaSuccess) e = launch_l2norm_rows(y[1], k, (int64_t)B * T * H, D, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    // 3. the scan's backward
+    float* dq = (float*)(base + L.d);
+    float* dk = (float*)(base + L.d + tb);
+    float* dv = (float*)(base + L.d + 2 * tb);
+    const KdaBwdArgs a{q, k, y[2], g32, b32, S0, d_o, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H, D, D, ET_F32,
+                       do_dtype == KDA_F32 ? ET_F32 : ET_BF16};
+    e = launch_kda_bwd(a, base + L.bws, s);
+    // 4. through the norms
+    if (e == cudaSuccess) e = launch_l2norm_bwd_rows(y[0], dq, (int64_t)B * T * H, D, s);
+    if (e == cudaSuccess) e = launch_l2norm_bwd_rows(y[1], dk, (int64_t)B * T * H, D, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    // 5. the conv backward of each tensor (one weight set per modality)
+    std::vector<msc_segment> segs0(segs, segs + n_segs);
+    for (auto& sg : segs0) sg.weight_set = 0;
+    const float* dys[3] = {dq, dk, dv};
+    float* dxs[3] = {dxq, dxk, dxv};
+    float* const* dws[3] = {dwq, dwk, dwv};
+    for (int i = 0; i < 3; ++i) {
+        st = conv_backward_run(x32[i], dys[i], dxs[i], B, T, C, ET_F32, segs0.data(), n_segs, Kt, ws3[i][0], 1,
+                               ws3[i][1], 1, ws3[i][2], 1, dws[i][0], dws[i][1], dws[i][2], s);
+        if (st != KDA_OK) return st;
+    }
+    return KDA_OK;
 }
 
 }  // extern "C"

@@ -29,7 +29,8 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_profile_collect", "kda_forward_noalloc", "kda_debug_drop_handoff", "kda_fma_probe",
             "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size",
             "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output",
-            "kda_backward", "kda_backward_workspace_size", "mshortconv_backward")
+            "kda_backward", "kda_backward_workspace_size", "mshortconv_backward",
+            "kda_mshortconv_backward", "kda_mshortconv_backward_workspace_size")
 
 
 class KdaError(RuntimeError):
@@ -103,6 +104,11 @@ def load_library(path: str = LIB_PATH):
         lib.kda_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]
         lib.mshortconv_backward.restype = I
         lib.mshortconv_backward.argtypes = [P, P, P, I, I, I, I, P, I, I, P, I, P, I, P, I, P, P, P, P]
+        lib.kda_mshortconv_backward_workspace_size.restype = Z
+        lib.kda_mshortconv_backward_workspace_size.argtypes = [I, I, I, I, I]
+        lib.kda_mshortconv_backward.restype = I
+        lib.kda_mshortconv_backward.argtypes = [P, P, P, P, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P,
+                                                P, P, P, I, I, I, I, I, P, Z, P]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -523,6 +529,52 @@ def mshortconv_kda_forward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, S0=Non
                                     ws_ptr, ws_bytes, _stream(stream))
     _check("kda_mshortconv_forward", rc)
     return o, S_T
+
+
+def mshortconv_kda_backward_workspace_size(B, T, H, D, dtype=torch.bfloat16) -> int:
+    return int(load_library().kda_mshortconv_backward_workspace_size(B, T, H, D, _code(dtype)))
+
+
+def mshortconv_kda_backward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, do, S0=None, dS_T=None, *,
+                            want_dS0: bool = True, workspace=None, stream=None):
+    """kda_mshortconv_backward: gradients (fp32) through mshortconv_kda_forward for
+    dL/do = do and dL/dS_T = dS_T.  Returns a dict with dxq, dxk, dxv ([B,T,H*D]),
+    dwq, dwk, dwv (tuples shaped like wq, wk, wv; None where the weight is None), dg,
+    dbeta, dS0."""
+    lib = load_library()
+    B, T, H, D = g.shape
+    C = H * D
+    dt = _dtype_code(xq)
+    f = dict(dtype=torch.float32, device=xq.device)
+    out = {"dxq": torch.empty((B, T, C), **f), "dxk": torch.empty((B, T, C), **f),
+           "dxv": torch.empty((B, T, C), **f), "dg": torch.empty((B, T, H, D), **f),
+           "dbeta": torch.empty((B, T, H), **f),
+           "dS0": torch.empty((B, H, D, D), **f) if want_dS0 else None}
+    segs, n = make_segments(segments)
+    warrs, dwarrs = [], []
+    for name, w in (("wq", wq), ("wk", wk), ("wv", wv)):
+        a, da = (ctypes.c_void_p * 3)(), (ctypes.c_void_p * 3)()
+        dws = []
+        for i in range(3):
+            a[i] = _dev(w[i], f"{name}[{i}]", torch.float32) if w[i] is not None else None
+            dw = torch.empty_like(w[i], dtype=torch.float32) if w[i] is not None else None
+            da[i] = _dev(dw, f"d{name}[{i}]", torch.float32) if dw is not None else None
+            dws.append(dw)
+        warrs.append(a)
+        dwarrs.append(da)
+        out["d" + name] = tuple(dws)
+    ws_ptr, ws_bytes = _ws(workspace)
+    cp = lambda a: ctypes.cast(a, ctypes.c_void_p)
+    rc = lib.kda_mshortconv_backward(_dev(xq, "xq"), _dev(xk, "xk"), _dev(xv, "xv"), cp(segs), n, int(Kt),
+                                     cp(warrs[0]), cp(warrs[1]), cp(warrs[2]), _dev(g, "g", xq.dtype),
+                                     _dev(beta, "beta", xq.dtype), _dev(S0, "S0", torch.float32), _dev(do, "do"),
+                                     _dtype_code(do), _dev(dS_T, "dS_T", torch.float32),
+                                     _dev(out["dxq"], "dxq"), _dev(out["dxk"], "dxk"), _dev(out["dxv"], "dxv"),
+                                     cp(dwarrs[0]), cp(dwarrs[1]), cp(dwarrs[2]), _dev(out["dg"], "dg"),
+                                     _dev(out["dbeta"], "dbeta"), _dev(out["dS0"], "dS0"), B, T, H, D, dt,
+                                     ws_ptr, ws_bytes, _stream(stream))
+    _check("kda_mshortconv_backward", rc)
+    return out
 
 
 def kernel_launches() -> int:
