@@ -27,9 +27,9 @@
 // results are not finite.
 //
 // Every matrix product runs on the tensor cores as 3xTF32 warp MMAs (fp32 accuracy).
-// Parallel split: the state's value columns evolve independently, so one CTA owns 32
+// Parallel split: the state's value columns evolve independently, so one CTA owns 16
 // value columns of one (b, h).  It first runs the forward over all chunks and stores
-// each chunk's entry state (its 32 columns) in the workspace, then walks the chunks in
+// each chunk's entry state (its 16 columns) in the workspace, then walks the chunks in
 // reverse.  dv and dS0 columns belong to one CTA; dq, dk, dg and dbeta are sums over
 // the value columns and are accumulated with atomic adds (the outputs are zeroed first).
 // Everything else is fp32 on CUDA cores.
@@ -42,7 +42,7 @@ namespace kda {
 namespace {
 
 constexpr int BC = 32;        // chunk length
-constexpr int BVC = 32;       // value columns per CTA
+constexpr int BVC = 16;       // value columns per CTA
 constexpr int BT = 256;       // threads per CTA
 // Row strides (floats) are 4 mod 32, so the 8 x 4 lane pattern of a warp MMA fragment
 // load touches 32 different banks for row-major operands.
