@@ -572,6 +572,36 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
         print(json.dumps(line), flush=True)
 
 
+def run_part(args, w: W.Workload):
+    """One other call on the workload, device-timed: the scan's backward (kda_backward on
+    the workload's q, k, v, g, beta and a random dL/do) or the conv backward of x_q (a
+    workload with a conv).  Not the benchmark step; used to profile those kernels."""
+    from linear_attention_sequence_mshortconv_b200 import build as libbuild
+    from linear_attention_sequence_mshortconv_b200 import kda
+    libbuild.build()
+    kda.load_library()
+    gen = torch.Generator().manual_seed(11)
+    if args.part == "backward":
+        inp = W.make_kda_inputs(w, device="cuda")
+        do = torch.randn(w.B, w.T, w.H, w.D, generator=gen).to(w.dtype).cuda()
+        wsb = torch.empty(max(1, kda.backward_workspace_size(w.B, w.T, w.H, w.D, w.D)), dtype=torch.uint8,
+                          device="cuda")
+
+        def step():
+            kda.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], do, workspace=wsb)
+    else:
+        fin = W.make_fused_inputs(w, device="cuda")
+        dy = torch.randn(w.B, w.T, w.H * w.D, generator=gen).to(w.dtype).cuda()
+
+        def step():
+            kda.mshortconv_backward(fin["xq"], dy, fin["segments"], w.Kt, *fin["wq"])
+    for _ in range(max(1, args.warmup)):
+        step()
+    ms = timed(step, args.steps, 1) / args.steps
+    print(json.dumps({"part": args.part, "workload": w.name, "ms_per_step": ms, "steps": args.steps,
+                      "tokens": w.tokens}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -585,6 +615,9 @@ def main():
                     help="device timing only: no end-to-end leg, no CPU baseline (for profiling)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload on its first N tokens (smaller profiling cases)")
+    ap.add_argument("--part", default="forward", choices=["forward", "backward", "conv_backward"],
+                    help="time one other call on the workload instead of the forward step "
+                         "(single GPU; prints its own JSON line; for profiling)")
     args = ap.parse_args()
     ws, rank, local = dist_setup()
     w = W.BY_NAME[args.workload]
@@ -593,6 +626,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, ws, rank, w)
+        elif args.part != "forward":
+            run_part(args, w)
         else:
             run_gpu(args, ws, rank, local, w)
     finally:

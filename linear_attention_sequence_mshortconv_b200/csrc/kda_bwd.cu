@@ -43,7 +43,7 @@ namespace {
 
 constexpr int BC = 32;        // chunk length
 constexpr int BVC = 16;       // value columns per CTA
-constexpr int BT = 256;       // threads per CTA
+constexpr int BT = 512;       // threads per CTA
 // Row strides (floats) are 4 mod 32, so the 8 x 4 lane pattern of a warp MMA fragment
 // load touches 32 different banks for row-major operands.
 constexpr int LDV = BVC + 4;  // row stride of [BC][BVC] tiles
