@@ -68,7 +68,8 @@ template <int DK> struct BwdPlan {
 enum { MM_SET = 0, MM_ADD = 1, MM_SUB = 2, MM_NEG = 3 };
 
 // out(i, j) op= sum_{k<K} A(i, k) B(k, j) for i < M, j < N, on the tensor cores, by the
-// warps of threads [tid0, tid0 + nthr).  A(i, k) = A[i*ai + k*ak], B(k, j) = B[k*bk + j*bj],
+// warps of threads [tid0, tid0 + nthr) (other warps return at once, so two independent
+// products can run side by side on two halves of the block).  A(i, k) = A[i*ai + k*ak], B(k, j) = B[k*bk + j*bj],
 // out(i, j) = O[i*oi + j], all in shared memory.  Warp MMAs m16n8k8 with tf32 operands:
 // each fp32 operand is split as hi + lo (hi = tf32(x), lo = tf32(x - hi)) and the product
 // taken as lo*hi + hi*lo + hi*hi ("3xTF32"), which keeps fp32 accuracy.  16 x 8 output
@@ -95,9 +96,10 @@ __device__ __forceinline__ void mmt(float* O, int oi, const float* A, int ai, in
     static_assert(M % 16 == 0 && N % 8 == 0 && K % 8 == 0, "warp MMA tiles");
     constexpr int TN = N / 8, NTILE = (M / 16) * TN;
     const int w0 = tid0 >> 5, nw = nthr >> 5;
+    const int wi = (int)(threadIdx.x >> 5) - w0;
+    if (wi < 0 || wi >= nw) return;   // not one of this product's warps
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    for (int tile = (int)(threadIdx.x >> 5) - w0; tile < NTILE; tile += nw) {
-        if (tile < 0) break;
+    for (int tile = wi; tile < NTILE; tile += nw) {
         const int i0 = (tile / TN) * 16, j0 = (tile % TN) * 8;
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         const float* a0 = A + (i0 + g) * ai + q * ak;
@@ -309,8 +311,8 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         prologue(n, true);
         __syncthreads();
         // Kd, P; Se = Diag(e^r) S; Gc = Diag(e^{b_C - r}) G'
-        mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK);
-        mmt<BC, BC, DK, MM_SET>(sP, LDC, sQP, LDK, 1, sKM, 1, LDK);
+        mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK, 0, BT / 2);
+        mmt<BC, BC, DK, MM_SET>(sP, LDC, sQP, LDK, 1, sKM, 1, LDK, BT / 2, BT / 2);
         for (int e = t; e < DK * BVC; e += BT) {
             const int c = e / BVC, j = e % BVC;
             sSe[c * LDS + j] *= expf(sR[c]);
@@ -321,8 +323,8 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         if (w == 0) {
             invert_warp(sT, sKd, sBeta, lane);
         } else {
-            mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 32, BT - 32);
-            mmt<BC, BVC, DK, MM_SET>(sDU, LDV, sKM, LDK, 1, sGp, LDS, 1, 32, BT - 32);
+            mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 32, BT / 2 - 32);
+            mmt<BC, BVC, DK, MM_SET>(sDU, LDV, sKM, LDK, 1, sGp, LDS, 1, BT / 2, BT / 2);
             for (int e = t - 32; e < BC * BC; e += BT - 32) {
                 const int i = e / BC, j = e % BC;
                 if (j > i) sP[i * LDC + j] = 0.f;
@@ -335,8 +337,8 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         }
         mmt<BC, BVC, BC, MM_ADD>(sDU, LDV, sP, 1, LDC, sDO, LDV, 1);   // dU += P^T dO
         __syncthreads();
-        mmt<BC, BVC, BC, MM_SET>(sU, LDV, sT, LDC, 1, sRb, LDV, 1);    // U = T Rb
-        mmt<BC, BVC, BC, MM_SET>(sDR, LDV, sT, 1, LDC, sDU, LDV, 1);   // dR = T^T dU
+        mmt<BC, BVC, BC, MM_SET>(sU, LDV, sT, LDC, 1, sRb, LDV, 1, 0, BT / 2);         // U = T Rb
+        mmt<BC, BVC, BC, MM_SET>(sDR, LDV, sT, 1, LDC, sDU, LDV, 1, BT / 2, BT / 2);   // dR = T^T dU
         __syncthreads();
         if (t < BC) {
             float s = 0.f;
@@ -347,8 +349,8 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
             const int i = e / BVC, j = e % BVC;
             if (t0 + i < T) dv[((tok0 + t0 + i) * rowH + h) * Dv + col0 + j] = sBeta[i] * sDR[i * LDV + j];
         }
-        mmt<BC, BC, BVC, MM_SET>(sX1, LDC, sDU, LDV, 1, sRb, 1, LDV);  // dT = dU Rb^T
-        mmt<BC, BC, BVC, MM_SET>(sDP, LDC, sDO, LDV, 1, sU, 1, LDV);   // dO U^T
+        mmt<BC, BC, BVC, MM_SET>(sX1, LDC, sDU, LDV, 1, sRb, 1, LDV, 0, BT / 2);       // dT = dU Rb^T
+        mmt<BC, BC, BVC, MM_SET>(sDP, LDC, sDO, LDV, 1, sU, 1, LDV, BT / 2, BT / 2);   // dO U^T
         __syncthreads();
         for (int e = t; e < BC * BVC; e += BT) {                        // dRb = Diag(beta) dR
             const int i = e / BVC, j = e % BVC;
