@@ -249,7 +249,7 @@ __host__ __device__ constexpr int tile_bytes() { return NF * HR * HS * 32 * (int
 // dx[f, r, s] = sum_{tau,a,e} w[tau,a,e] dy[f + 2 - tau, r + 1 - a, s + 1 - e] (video;
 // image: tau = 2 only).  grid (ceil(Wd/16) * ceil(Hg/8) * F, ceil(C/64), B).
 template <int NF, typename TIn>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 conv_dx_tile_kernel(const TIn* __restrict__ dy, const float* __restrict__ w, float* __restrict__ dx, int T, int C,
                     int64_t start, int F, int Hg, int Wd)
 {
