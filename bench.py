@@ -417,7 +417,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
 
     peaks, peak_kind = read_peaks()
     prof = {}
-    for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "conv"):
+    for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "kda_tc_output_first", "conv"):
         r = kda.profile_collect(name)
         if r and r[1] > 0:
             prof[name] = {"ms_total": r[0], "launches": r[1], "ms_per_launch": r[0] / r[1]}
@@ -425,14 +425,26 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
     roof = None
     if dominant:
         per_launch_s = prof[dominant]["ms_per_launch"] * 1e-3
-        # the dominant kernel moves the whole scan's algorithmic bytes once per launch
+        # the dominant kernel's algorithmic bytes per launch: the scan's, times the share
+        # of the tokens its launches cover (the two-wave split gives segment 0 its own
+        # output launch, "kda_tc_output_first", so "kda_tc_output" covers segments 1..P-1)
         launches_per_step = prof[dominant]["launches"] / args.steps
-        alg = algorithmic_bytes(w) / launches_per_step
+        share = 1.0
+        if dominant in ("kda_tc_output", "kda_tc_output_first") and not w.fused:
+            P_, L_ = kda.forward_plan(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+            if P_ > 1:
+                first = min(w.T, L_ * 64) / w.T
+                share = first if dominant == "kda_tc_output_first" else 1.0 - first
+        alg = algorithmic_bytes(w) * share / launches_per_step
+        split = None
+        if not w.fused:
+            P_, L_ = kda.forward_plan(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+            split = {"segments": P_, "chunks_per_segment": L_}
         achieved = alg / per_launch_s / 1e9
         peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
         roof = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_record(dominant),
-                "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind, "split": split,
                 "kernel_ms_per_launch": prof[dominant]["ms_per_launch"]}
 
     e2e = None if args.quick else e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
@@ -461,7 +473,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             m = timed(st, k_other, 1) / k_other
             kda.profile_enable(False)
             kern = {}
-            for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "conv"):
+            for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "kda_tc_output_first", "conv"):
                 r = kda.profile_collect(name)
                 if r and r[1] > 0:
                     kern[name] = {"ms_per_step": r[0] / k_other, "launches_per_step": r[1] / k_other}

@@ -383,6 +383,19 @@ kda_status kda_mshortconv_backward(const void* xq, const void* xk, const void* x
 
 /* ---- diagnostics ---------------------------------------------------------------- */
 
+/* How kda_forward (ungated) splits a uniform batch on the tensor-core path on the current
+ * device: each head's ceil(T/64) chunks form *segments runs of *chunks_per_segment
+ * chunks (the last may be shorter).  With more than one segment, segment 0's output pass
+ * ("kda_tc_output_first") runs beside the state pass of segments 1..P-2 ("kda_tc_state"),
+ * and the output pass of segments 1..P-1 ("kda_tc_output") follows the combine
+ * ("kda_tc_combine").  Both are 0 when the call would not take the tensor-core path.
+ * The first kda_forward on a device with more than one segment creates an auxiliary
+ * stream and two events for that overlap; make it before any stream capture.
+ * Returns KDA_ERR_INVALID_ARG for null outputs or bad sizes. */
+kda_status kda_forward_plan(int B, int T, int H, int Dk, int Dv, kda_dtype dtype,
+                            kda_dtype o_dtype, int chunk, int* segments,
+                            int* chunks_per_segment);
+
 /* Number of kernels this library has launched in this process (all devices). */
 uint64_t kda_kernel_launches(void);
 
@@ -413,7 +426,8 @@ void kda_profile_enable(int on);
  * device time in milliseconds and the number of launches timed since the last
  * collection; clears that kernel's record.  Returns 0, or -1 if `name` has no
  * record.  Names: "kda_generic", "kda_tc_state", "kda_tc_combine",
- * "kda_tc_output", "conv", "gate_norm", "kda_sp_fold", "kda_bwd", "conv_bwd". */
+ * "kda_tc_output", "kda_tc_output_first", "conv", "gate_norm", "kda_sp_fold",
+ * "kda_bwd", "conv_bwd". */
 int kda_profile_collect(const char* name, double* total_ms, int* launches);
 
 #ifdef __cplusplus

@@ -75,6 +75,10 @@ cudaError_t launch_kda_generic(const KdaArgs& a, cudaStream_t s);
 // Tensor-core path (bf16, Dk = Dv = 128).  Workspace bytes it needs:
 size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms);
 bool kda_tc_supported(const KdaArgs& a);
+// The uniform-batch split of the tensor-core path: P segments of L chunks per head (P = 1:
+// one pass per head; otherwise the output pass of segment 0 runs beside the state pass of
+// segments 1..P-2, and the output pass of segments 1..P-1 follows the combine).
+void kda_tc_plan(int B, int T, int H, int num_sms, int* P, int* L);
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status,
                           cudaStream_t s);
 // Packed samples: a.B = 1, a.T = cu[n] tokens; host array cu[0..n] of sample offsets.

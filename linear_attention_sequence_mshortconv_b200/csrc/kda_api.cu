@@ -149,6 +149,22 @@ size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype
     return kda_ws_bytes(a);
 }
 
+kda_status kda_forward_plan(int B, int T, int H, int Dk, int Dv, kda_dtype dtype, kda_dtype o_dtype, int chunk,
+                            int* segments, int* chunks_per_segment)
+{
+    if (!segments || !chunks_per_segment) return KDA_ERR_INVALID_ARG;
+    *segments = *chunks_per_segment = 0;
+    if (B < 0 || T < 0 || H <= 0 || !dim_ok(Dk) || !dim_ok(Dv)) return KDA_ERR_INVALID_ARG;
+    KdaArgs a{};
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv;
+    a.in_t = a.gb_t = et_of(dtype);
+    a.out_t = et_of(o_dtype);
+    a.chunk = chunk ? chunk : default_chunk(dtype, Dk);
+    if (T < 1 || !kda_tc_supported(a)) return KDA_OK;
+    kda_tc_plan(B, T, H, num_sms(), segments, chunks_per_segment);
+    return KDA_OK;
+}
+
 kda_status kda_forward(const void* q, const void* k, const void* v, const void* g,
                        const void* beta, const float* S0, void* o, float* S_T,
                        int B, int T, int H, int Dk, int Dv, kda_dtype dtype,

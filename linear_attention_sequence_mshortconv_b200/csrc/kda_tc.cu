@@ -1254,7 +1254,8 @@ Split split_for(int B, int T, int H, int num_sms)
 
 template <int MODE, typename TQ>
 cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int per_seg, float* maps, int P, int L,
-                        int* status, cudaStream_t s, const int* items = nullptr, int nitems = 0)
+                        int* status, cudaStream_t s, const int* items = nullptr, int nitems = 0,
+                        const char* prof_name = nullptr)
 {
     auto kern = kda_tc_kernel<MODE, TQ>;
     const int smem = smem_bytes<MODE>();
@@ -1263,7 +1264,7 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     const int nseg = MODE == MODE_STATE ? P - 1 : P;
     const unsigned grid = items ? (unsigned)nitems : (unsigned)(a.B * a.H * nseg);
     if (grid == 0) return cudaSuccess;
-    ProfileScope prof(MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output", s);
+    ProfileScope prof(prof_name ? prof_name : (MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output"), s);
     count_launch();
     kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, mp.gate, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
@@ -1316,19 +1317,151 @@ cudaError_t combine_output(const Maps& mp, const KdaArgs& a, const Split& sp, fl
     return launch_pass<MODE_OUTPUT, TQ>(mp, a, starts, 1, maps, sp.P, sp.L, status, s);
 }
 
+// ---- uniform batch: two waves ------------------------------------------------------------
+// With W = floor(#SM / (B*H)) >= 2 CTAs per head and wave, a head's chunks are cut into
+// P = W + 1 segments of L chunks:
+//   wave 1: the output pass of segment 0 (from S0; it also yields S_start(1) exactly) on an
+//           auxiliary stream, beside the state pass of segments 1..P-2,
+//   combine: S_start(p+1) = M_p S_start(p) + N_p from S_start(1), p = 1..P-2,
+//   wave 2: the output pass of segments 1..P-1.
+// Both waves hold W CTAs per head, so L = ceil(NC / (W+1)) instead of ceil(NC / W).
+// Workspace: maps [B*H][P-2][N | M], starts [B*H][P-1][D][D], S_start(1) [B*H][D][D],
+// three item tables.
+struct Waves {
+    int P, L;
+    size_t maps_b, starts_b, s1_b, it0_b, its_b, ito_b;
+    size_t total() const { return maps_b + starts_b + s1_b + it0_b + its_b + ito_b; }
+};
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Waves waves_for(int B, int T, int H, int sms)
+{
+    Waves w{};
+    const int NC = (T + C - 1) / C, BH = max(1, B * H);
+    const int W = sms / BH;
+    if (W < 2 || NC < 2) {   // one wave: every head one segment, or the plain split
+        w.P = 1;
+        w.L = NC;
+        return w;
+    }
+    int P = min(W + 1, NC);
+    w.L = (NC + P - 1) / P;
+    w.P = P = (NC + w.L - 1) / w.L;   // no empty segment
+    const size_t bh = (size_t)B * H;
+    w.maps_b = a256(bh * (size_t)max(0, P - 2) * 2 * D * D * sizeof(float));
+    w.starts_b = a256(bh * (size_t)(P - 1) * D * D * sizeof(float));
+    w.s1_b = a256(bh * D * D * sizeof(float));
+    w.it0_b = a256(bh * 8 * sizeof(int));
+    w.its_b = a256(bh * (size_t)max(0, P - 2) * 8 * sizeof(int));
+    w.ito_b = a256(bh * (size_t)(P - 1) * 8 * sizeof(int));
+    return w;
+}
+
+// The auxiliary stream of this device for wave 1's segment-0 pass, and the two events of
+// its fork and join.  One enqueue sequence at a time uses them (the mutex), so the events
+// always refer to the call that recorded them.
+struct Aux {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_aux_mu;
+Aux g_aux[64];
+
 template <typename TQ>
 cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
 {
+    const Waves wv = waves_for(a.B, a.T, a.H, sm_count());
     const Split sp = split_for(a.B, a.T, a.H, sm_count());
     Maps mp;
     if (!build_maps<TQ>(a, mp)) return cudaErrorInvalidValue;
-    float* maps = reinterpret_cast<float*>(ws);
-    float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
-    if (sp.P > 1) {
-        const cudaError_t e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, sp.P, sp.L, status, s);
+    // the gated epilogue needs whole-chunk TMA stores, which the item tables' ragged
+    // sequence ends do not give: it keeps the one-table split
+    if (wv.P == 1 || a.gate) {
+        float* maps = reinterpret_cast<float*>(ws);
+        float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
+        if (sp.P > 1) {
+            const cudaError_t e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, sp.P, sp.L, status, s);
+            if (e != cudaSuccess) return e;
+        }
+        return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
+    }
+    const int P = wv.P, L = wv.L, NC = (a.T + C - 1) / C, BH = a.B * a.H;
+    // item tables address packed rows: the bf16 output map spans all B*T rows as one
+    if (a.out_t == ET_BF16 && !make_map_o(&mp.o, a.o, 1, a.B * a.T, a.H)) return cudaErrorInvalidValue;
+    char* base = reinterpret_cast<char*>(ws);
+    float* maps = reinterpret_cast<float*>(base);
+    float* starts = reinterpret_cast<float*>(base + wv.maps_b);
+    float* s1 = reinterpret_cast<float*>(base + wv.maps_b + wv.starts_b);
+    int* it0 = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b);
+    int* its = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b + wv.it0_b);
+    int* ito = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b + wv.it0_b + wv.its_b);
+    std::vector<int> h0, hs, ho;
+    h0.reserve((size_t)BH * 8);
+    hs.reserve((size_t)BH * max(0, P - 2) * 8);
+    ho.reserve((size_t)BH * (P - 1) * 8);
+    for (int b = 0; b < a.B; ++b)
+        for (int h = 0; h < a.H; ++h) {
+            const int bh = b * a.H + h;
+            const int e0[8] = {b * a.T, a.T, 0, min(NC, L), h, b, bh, 1};   // end state -> s1
+            h0.insert(h0.end(), e0, e0 + 8);
+            for (int p = 1; p < P; ++p) {
+                const int n0 = p * L, n1 = min(NC, n0 + L);
+                if (p < P - 1) {
+                    const int es[8] = {b * a.T, a.T, n0, n1, h, b, bh * (P - 2) + (p - 1), 0};
+                    hs.insert(hs.end(), es, es + 8);
+                }
+                const int eo[8] = {b * a.T, a.T, n0, n1, h, b, bh * (P - 1) + (p - 1), p == P - 1};
+                ho.insert(ho.end(), eo, eo + 8);
+            }
+        }
+    // pageable sources: the copies are staged before the calls return
+    cudaError_t e = cudaMemcpyAsync(it0, h0.data(), h0.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess && !hs.empty())
+        e = cudaMemcpyAsync(its, hs.data(), hs.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ito, ho.data(), ho.size() * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(g_aux_mu);
+        Aux& ax = g_aux[dev];
+        if (!ax.s) {
+            e = cudaStreamCreateWithFlags(&ax.s, cudaStreamNonBlocking);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ax.fork, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ax.join, cudaEventDisableTiming);
+            if (e != cudaSuccess) return e;
+        }
+        // wave 1: segment 0's output pass (end state -> s1) beside the state pass
+        e = cudaEventRecord(ax.fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ax.s, ax.fork, 0);
+        if (e != cudaSuccess) return e;
+        KdaArgs a0 = a;
+        a0.ST = s1;
+        e = launch_pass<MODE_OUTPUT, TQ>(mp, a0, a.S0, 0, nullptr, P, L, status, ax.s, it0, BH, "kda_tc_output_first");
+        if (e == cudaSuccess) e = cudaEventRecord(ax.join, ax.s);
+        if (e != cudaSuccess) return e;
+        if (P > 2) {
+            e = launch_pass<MODE_STATE, TQ>(mp, a, nullptr, 0, maps, P, L, status, s, its, BH * (P - 2));
+            if (e != cudaSuccess) return e;
+        }
+        e = cudaStreamWaitEvent(s, ax.join, 0);
         if (e != cudaSuccess) return e;
     }
-    return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
+    if (P == 2)   // segment 1 starts from segment 0's end state
+        return launch_pass<MODE_OUTPUT, TQ>(mp, a, s1, 0, nullptr, P, L, status, s, ito, BH);
+    e = cudaFuncSetAttribute(kda_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cb_smem_bytes());
+    if (e != cudaSuccess) return e;
+    {
+        ProfileScope prof("kda_tc_combine", s);
+        count_launch();
+        kda_combine_kernel<<<dim3(D / 16, a.H, a.B), CB_THREADS, cb_smem_bytes(), s>>>(maps, s1, starts, a.H, P - 1,
+                                                                                        nullptr);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pass<MODE_OUTPUT, TQ>(mp, a, starts, 1, maps, P, L, status, s, ito, BH * (P - 1));
 }
 
 // ---- one shard of a sequence cut across devices -----------------------------------------
@@ -1336,8 +1469,6 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
 // 0..P-2 write their maps in the uniform layout (the output pass reads them), the last
 // one into a tail slot per head after them.  Workspace: maps [B*H*P][N | M], start
 // states [B*H*P][D][D], the item table.
-size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
-
 struct SpLayout {
     Split sp;
     size_t maps_bytes, starts_bytes, items_bytes;
@@ -1528,9 +1659,11 @@ bool kda_tc_supported(const KdaArgs& a)
 size_t kda_tc_workspace_bytes(int B, int T, int H, int chunk, int num_sms)
 {
     if (chunk != C || T < 1) return 0;
+    // the larger of the two-wave layout and the one-table split (the gated epilogue)
     const Split sp = split_for(B, T, H, num_sms);
-    if (sp.P == 1) return 0;
-    return (size_t)B * H * ((size_t)(sp.P - 1) * 2 + sp.P) * D * D * sizeof(float);
+    const size_t one = sp.P == 1 ? 0 : (size_t)B * H * ((size_t)(sp.P - 1) * 2 + sp.P) * D * D * sizeof(float);
+    const Waves wv = waves_for(B, T, H, num_sms);
+    return std::max<size_t>(one, wv.P == 1 ? (size_t)0 : wv.total());
 }
 
 size_t kda_tc_varlen_workspace_bytes(const int* cu, int n, int H, int num_sms)
@@ -1549,6 +1682,13 @@ size_t kda_tc_sp_workspace_bytes(int B, int T, int H, int num_sms)
 {
     if (B < 1 || T < 1) return 0;
     return sp_layout(B, T, H, num_sms).total();
+}
+
+void kda_tc_plan(int B, int T, int H, int num_sms, int* P, int* L)
+{
+    const Waves wv = waves_for(B, T, H, num_sms);
+    *P = wv.P;
+    *L = wv.L;
 }
 
 cudaError_t launch_kda_tc_sp_state(const KdaArgs& a, void* ws, int* status, cudaStream_t s, TcShardMaps* out)

@@ -30,7 +30,7 @@ EXPORTED = ("kda_status_string", "kda_last_device_error", "kda_forward_workspace
             "kda_forward_gated", "kda_forward_varlen", "kda_forward_varlen_workspace_size",
             "kda_sp_workspace_size", "kda_sp_transition", "kda_sp_prefix", "kda_sp_output",
             "kda_backward", "kda_backward_workspace_size", "mshortconv_backward",
-            "kda_mshortconv_backward", "kda_mshortconv_backward_workspace_size")
+            "kda_mshortconv_backward", "kda_mshortconv_backward_workspace_size", "kda_forward_plan")
 
 
 class KdaError(RuntimeError):
@@ -109,6 +109,9 @@ def load_library(path: str = LIB_PATH):
         lib.kda_mshortconv_backward.restype = I
         lib.kda_mshortconv_backward.argtypes = [P, P, P, P, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, P, P,
                                                 P, P, P, I, I, I, I, I, P, Z, P]
+        lib.kda_forward_plan.restype = I
+        lib.kda_forward_plan.argtypes = [I, I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_int)]
         lib.kda_fma_probe.restype = I
         lib.kda_fma_probe.argtypes = [ctypes.POINTER(ctypes.c_double)]
         lib.kda_profile_collect.restype = I
@@ -575,6 +578,16 @@ def mshortconv_kda_backward(xq, xk, xv, segments, Kt, wq, wk, wv, g, beta, do, S
                                      ws_ptr, ws_bytes, _stream(stream))
     _check("kda_mshortconv_backward", rc)
     return out
+
+
+def forward_plan(B, T, H, Dk, Dv, dtype=torch.bfloat16, chunk: int = 0, o_dtype=None):
+    """(segments, chunks per segment) of kda_forward's tensor-core split on this device
+    ((0, 0) off that path)."""
+    P, L = ctypes.c_int(0), ctypes.c_int(0)
+    _check("kda_forward_plan", load_library().kda_forward_plan(B, T, H, Dk, Dv, _code(dtype),
+                                                               _code(o_dtype or dtype), chunk,
+                                                               ctypes.byref(P), ctypes.byref(L)))
+    return P.value, L.value
 
 
 def kernel_launches() -> int:
