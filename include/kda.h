@@ -246,8 +246,9 @@ kda_status kda_sp_output(const void* q, const void* k, const void* v, const void
  *   dq, dk, dg : [B, T, H, Dk] fp32 (device, written);  dv : [B, T, H, Dv] fp32;
  *   dbeta : [B, T, H] fp32;  dS0 : [B, H, Dk, Dv] fp32 or NULL (not written).
  * The gradient of g is that of the natural-log decay (alpha = e^g).  The call reruns
- * the forward to store each 32-token chunk's entry state in the workspace
- * (kda_backward_workspace_size bytes: B*H*ceil(T/32)*Dk*Dv*4), then sweeps the chunks in
+ * the forward to store each 32-token chunk's entry state and chunk factors in the
+ * workspace (kda_backward_workspace_size bytes: B*H*ceil(T/32)*(Dk*Dv + Dv/16*2048)*4),
+ * then sweeps the chunks in
  * reverse; arithmetic is fp32.  Per key channel the decay over any 32 consecutive tokens
  * must satisfy |sum g| < 80; beyond that the gradients are not finite.
  * workspace: as for kda_forward (NULL: a stream-ordered allocation inside the call).

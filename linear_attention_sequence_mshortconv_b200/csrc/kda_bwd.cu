@@ -29,7 +29,7 @@
 // Every matrix product runs on the tensor cores as 3xTF32 warp MMAs (fp32 accuracy).
 // Parallel split: the state's value columns evolve independently, so one CTA owns 16
 // value columns of one (b, h).  It first runs the forward over all chunks and stores
-// each chunk's entry state (its 16 columns) in the workspace, then walks the chunks in
+// each chunk's entry state (its 16 columns), T and Kd in the workspace, then walks the chunks in
 // reverse.  dv and dS0 columns belong to one CTA; dq, dk, dg and dbeta are sums over
 // the value columns and are accumulated with atomic adds (the outputs are zeroed first).
 // Everything else is fp32 on CUDA cores.
@@ -48,6 +48,8 @@ constexpr int BT = 512;       // threads per CTA
 // load touches 32 different banks for row-major operands.
 constexpr int LDV = BVC + 4;  // row stride of [BC][BVC] tiles
 constexpr int LDC = BC + 4;   // row stride of [BC][BC] tiles
+// one chunk's checkpoint record per CTA: its entry state (DK x BVC), then T and Kd (BC x BC)
+template <int DK> __host__ __device__ constexpr int ck_floats() { return DK * BVC + 2 * BC * BC; }
 
 template <int DK> struct BwdPlan {
     static constexpr int LDK = DK + 4;    // [BC][DK] tiles
@@ -194,7 +196,8 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
     const int NC = (T + BC - 1) / BC;
     const size_t rowH = (size_t)H;                 // tokens -> rows of [B, T, H, *]
     const size_t tok0 = (size_t)b * T;             // first token row of this sequence
-    float* ck = ckpt + ((size_t)(b * H + h) * (Dv / BVC) + cb) * (size_t)NC * DK * BVC;
+    constexpr int CK = ck_floats<DK>();
+    float* ck = ckpt + ((size_t)(b * H + h) * (Dv / BVC) + cb) * (size_t)NC * CK;
 
     // rows [t0, t0 + BC) of a [B, T, H, W] tensor, columns [c0, c0 + NCOL), into an fp32
     // tile with row stride ld (16-byte vector loads, zero past T)
@@ -262,7 +265,7 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
     }
     __syncthreads();
     for (int n = 0; n < NC; ++n) {
-        float* ckn = ck + (size_t)n * DK * BVC;
+        float* ckn = ck + (size_t)n * CK;
         for (int e = t; e < DK * BVC / 4; e += BT) {
             const float* d = sSe + (4 * e / BVC) * LDS + (4 * e) % BVC;
             reinterpret_cast<float4*>(ckn)[e] = make_float4(d[0], d[1], d[2], d[3]);
@@ -281,6 +284,11 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
         for (int e = t; e < BC * BVC; e += BT) {
             const int i = e / BVC, j = e % BVC;
             sRb[i * LDV + j] = sBeta[i] * sVX[i * LDV + j];
+        }
+        for (int e = t; e < 2 * BC * BC / 4; e += BT) {   // T and Kd for the reverse sweep
+            const int m = e / (BC * BC / 4), r = (e % (BC * BC / 4)) * 4 / BC, c4 = (4 * e) % BC;
+            const float* src = (m ? sKd : sT) + r * LDC + c4;
+            reinterpret_cast<float4*>(ckn + DK * BVC)[e] = make_float4(src[0], src[1], src[2], src[3]);
         }
         __syncthreads();
         mmt<BC, BVC, BC, MM_SET>(sU, LDV, sT, LDC, 1, sRb, LDV, 1);
@@ -301,34 +309,35 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
     }
     for (int n = NC - 1; n >= 0; --n) {
         const int t0 = n * BC;
-        const float* ckn = ck + (size_t)n * DK * BVC;
+        const float* ckn = ck + (size_t)n * CK;
         __syncthreads();   // the previous chunk is done with every tile
         for (int e = t; e < DK * BVC / 4; e += BT) {
             const float4 c4 = reinterpret_cast<const float4*>(ckn)[e];
             float* d = sSe + (4 * e / BVC) * LDS + (4 * e) % BVC;
             d[0] = c4.x; d[1] = c4.y; d[2] = c4.z; d[3] = c4.w;
         }
+        for (int e = t; e < 2 * BC * BC / 4; e += BT) {   // T and Kd from the forward sweep
+            const int m = e / (BC * BC / 4), r = (e % (BC * BC / 4)) * 4 / BC, c4 = (4 * e) % BC;
+            const float4 v4 = reinterpret_cast<const float4*>(ckn + DK * BVC)[e];
+            float* d = (m ? sKd : sT) + r * LDC + c4;
+            d[0] = v4.x; d[1] = v4.y; d[2] = v4.z; d[3] = v4.w;
+        }
         prologue(n, true);
         __syncthreads();
-        // Kd, P; Se = Diag(e^r) S; Gc = Diag(e^{b_C - r}) G'
-        mmt<BC, BC, DK, MM_SET>(sKd, LDC, sKP, LDK, 1, sKM, 1, LDK, 0, BT / 2);
-        mmt<BC, BC, DK, MM_SET>(sP, LDC, sQP, LDK, 1, sKM, 1, LDK, BT / 2, BT / 2);
+        // P (T and Kd come from the forward sweep); Se = Diag(e^r) S; Gc = Diag(e^{b_C - r}) G'
+        mmt<BC, BC, DK, MM_SET>(sP, LDC, sQP, LDK, 1, sKM, 1, LDK, 0, BT / 2);
         for (int e = t; e < DK * BVC; e += BT) {
             const int c = e / BVC, j = e % BVC;
             sSe[c * LDS + j] *= expf(sR[c]);
             sGp[c * LDS + j] *= expf(sBC[c] - sR[c]);
         }
         __syncthreads();
-        // T (warp 0) | VX = V - K+ Se, dU = K- Gc, P masked (the other warps)
-        if (w == 0) {
-            invert_warp(sT, sKd, sBeta, lane);
-        } else {
-            mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 32, BT / 2 - 32);
-            mmt<BC, BVC, DK, MM_SET>(sDU, LDV, sKM, LDK, 1, sGp, LDS, 1, BT / 2, BT / 2);
-            for (int e = t - 32; e < BC * BC; e += BT - 32) {
-                const int i = e / BC, j = e % BC;
-                if (j > i) sP[i * LDC + j] = 0.f;
-            }
+        // VX = V - K+ Se | dU = K- Gc; P masked
+        mmt<BC, BVC, DK, MM_SUB>(sVX, LDV, sKP, LDK, 1, sSe, LDS, 1, 0, BT / 2);
+        mmt<BC, BVC, DK, MM_SET>(sDU, LDV, sKM, LDK, 1, sGp, LDS, 1, BT / 2, BT / 2);
+        for (int e = t; e < BC * BC; e += BT) {
+            const int i = e / BC, j = e % BC;
+            if (j > i) sP[i * LDC + j] = 0.f;
         }
         __syncthreads();
         for (int e = t; e < BC * BVC; e += BT) {
@@ -464,7 +473,8 @@ size_t kda_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv)
 {
     if (B <= 0 || T <= 0) return 0;
     const size_t NC = (size_t)(T + BC - 1) / BC;
-    return (size_t)B * H * NC * Dk * Dv * sizeof(float);
+    // per CTA (B*H*Dv/BVC of them) and chunk: its state columns, T and Kd
+    return (size_t)B * H * NC * ((size_t)Dk * Dv + (size_t)(Dv / BVC) * 2 * BC * BC) * sizeof(float);
 }
 
 cudaError_t launch_kda_bwd(const KdaBwdArgs& a, void* ws, cudaStream_t s)

@@ -187,3 +187,17 @@ def test_video_clip_full_size_sampled_heads():
 
 def test_long_video_full_size_sampled_head():
     _sampled_full_size(W.LONG_VIDEO, [(0, 5)])
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 129, 2), (1, 100, 3), (37, 200, 2), (25, 300, 3), (3, 777, 2)])
+def test_two_wave_split_boundaries(B, T, H):
+    # the uniform-batch split on the tensor-core path: 3 segments (one state-pass segment),
+    # 2 segments (no state pass: segment 1 starts from segment 0's end state), W = 2 and
+    # W = 1 CTAs per head (74 and 75 heads), and many one-chunk segments with S0 given
+    inp = _custom(B, T, H, 128, 128, torch.bfloat16, seed=B * 1000 + T)
+    S0 = torch.randn(B, H, 128, 128, generator=torch.Generator().manual_seed(T)) * 0.3
+    P, L = kda.forward_plan(B, T, H, 128, 128, torch.bfloat16)
+    assert P >= 1 and (P == 1 or (P - 1) * L < (T + 63) // 64 <= P * L)
+    o, ST = _run_gpu(inp, S0=S0)
+    o_ref, S_ref = _oracle(inp, S0)
+    compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what=f"two-wave P={P} L={L}")
