@@ -567,11 +567,11 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             bbytes = algorithmic_bytes(w) + w.B * w.T * w.H * (4 * w.D * 4 + 4)
             # the kernel's fp32 matrix-product multiply-adds per (32-token chunk C, 16 value
             # columns Vc, key width D): forward sweep C^2 D + 2 C D Vc + C^2 Vc; reverse sweep
-            # 6 C^2 D + 7 C D Vc + 5 C^2 Vc + 2 C^3.  They run as 3xTF32 warp MMAs (three TF32
+            # (T and Kd read back) 5 C^2 D + 7 C D Vc + 5 C^2 Vc + 2 C^3.  They run as 3xTF32 warp MMAs (three TF32
             # products per fp32 product), so the bound is the TF32 tensor rate: the measured
             # bf16 GEMM peak x the nominal TF32/bf16 ratio (1.1 / 2.25 PFLOP/s), divided by 3.
             C_, Vc_, D_ = 32, 16, w.D
-            fma_chunk = 7 * C_ * C_ * D_ + 9 * C_ * D_ * Vc_ + 6 * C_ * C_ * Vc_ + 2 * C_ ** 3
+            fma_chunk = 6 * C_ * C_ * D_ + 9 * C_ * D_ * Vc_ + 6 * C_ * C_ * Vc_ + 2 * C_ ** 3
             fmas = fma_chunk * w.B * w.H * (w.D // Vc_) * ((w.T + C_ - 1) // C_)
             peak_tf = float(peaks.get("bf16_tflops", PEAKS_FALLBACK.get("bf16_tflops", 1590.0))) * (1.1 / 2.25) / 3
             ach_tf = 2 * fmas / (mb * 1e-3) / 1e12
