@@ -161,8 +161,9 @@ kda_status kda_forward_varlen(const void* q, const void* k, const void* v, const
  * from one array of KDA_NOALLOC_SCRATCH_BYTES compiled into the library, held in the
  * device memory of every GPU on which the library is loaded until the process exits.
  *   - The first call on a device looks up that array's device address (once per
- *     device, with the device current); make that first call before any stream
- *     capture.
+ *     device, with the device current) and, when the tensor-core split has more than
+ *     one segment, creates the auxiliary stream and two events of its first wave (see
+ *     kda_forward_plan); make that first call before any stream capture.
  *   - All calls on a device share the array and it keeps the last call's contents.
  *     Every byte a call reads from it is written earlier in the same call, so nothing
  *     needs clearing; calls whose GPU work may overlap (different streams without
