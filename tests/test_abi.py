@@ -103,7 +103,8 @@ def test_backward_rejects_bad_arguments(lib):
     assert lib.kda_backward(*full(), *sizes(dodt=4)) == 1           # bad d_o dtype
     assert lib.kda_backward(*full(), *sizes(B=-1)) == 1
     assert lib.kda_backward(*full(), *sizes(B=0)) == 0              # empty batch: no-op
-    assert lib.kda_backward_workspace_size(1, 64, 2, 32, 64) == 2 * 2 * 32 * 64 * 4
+    # per (b, h) and 32-token chunk: the Dk x Dv entry state and, per 16 value columns, T and Kd
+    assert lib.kda_backward_workspace_size(1, 64, 2, 32, 64) == 2 * 2 * (32 * 64 + (64 // 16) * 2 * 32 * 32) * 4
     assert lib.kda_backward_workspace_size(1, 64, 2, 48, 64) == 0
 
 
