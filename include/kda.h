@@ -29,7 +29,15 @@
  *     read by kda_last_device_error() after the caller synchronises.
  *   - Floating point: inputs are bf16 or fp32 (kda_dtype); all accumulation and the
  *     recurrent state are fp32.  The fp32 path computes in fp32 on CUDA cores; the
- *     bf16 path feeds bf16 operands to the tensor cores with fp32 accumulation.
+ *     bf16 path converts its tiles on chip to fp16 tensor-core operands (11-bit
+ *     significand) with fp32 accumulation.
+ *   - CUDA graphs: the forward calls (except kda_forward_varlen), the backward calls,
+ *     kda_sp_prefix and kda_sp_output enqueue only launches, memsets, device copies and
+ *     event waits, so a stream capture can record them once the first call on the device
+ *     has run outside capture (it creates per-device resources) and given a workspace
+ *     (a NULL workspace is allocated stream-ordered inside the call).
+ *     kda_forward_varlen and kda_sp_transition copy a host-planned work table to the
+ *     device in every call and cannot be captured.
  *   - The gate is passed as g = ln(alpha) (g <= 0, finite), not as alpha: alpha close
  *     to 1 is not representable in bf16 (the spacing just below 1 is 2^-8), while its
  *     logarithm is.

@@ -1169,6 +1169,30 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
     }
 }
 
+// The work items of the two-wave split of a uniform batch, built on the device (so a call
+// makes no host-to-device copy and can be captured in a CUDA graph).  One thread per
+// (b, h, segment p): p = 0 -> it0 (segment 0's output pass; slot = b*H + h, last = 1);
+// p >= 1 -> ito (output pass, slot (b*H + h)*(P-1) + p-1) and, for p <= P-2, its (state
+// pass, slot (b*H + h)*(P-2) + p-1).  Items are {row, length, n0, n1, head, sequence,
+// slot, last}.
+__global__ void wave_items_kernel(int* __restrict__ it0, int* __restrict__ its, int* __restrict__ ito, int B, int T,
+                                  int H, int P, int L)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= B * H * P) return;
+    const int p = i % P, bh = i / P, b = bh / H, h = bh % H;
+    const int NC = (T + C - 1) / C, n0 = p * L, n1 = min(NC, n0 + L);
+    auto put = [&](int* dst, int slot, int last) {
+        dst[0] = b * T; dst[1] = T; dst[2] = n0; dst[3] = n1;
+        dst[4] = h; dst[5] = b; dst[6] = slot; dst[7] = last;
+    };
+    if (p == 0) {
+        put(it0 + 8 * bh, bh, 1);
+        return;
+    }
+    put(ito + 8 * (bh * (P - 1) + p - 1), bh * (P - 1) + p - 1, p == P - 1);
+    if (p <= P - 2) put(its + 8 * (bh * (P - 2) + p - 1), bh * (P - 2) + p - 1, 0);
+}
 // ---- host side ----------------------------------------------------------------------------
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -1386,7 +1410,7 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         }
         return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
     }
-    const int P = wv.P, L = wv.L, NC = (a.T + C - 1) / C, BH = a.B * a.H;
+    const int P = wv.P, L = wv.L, BH = a.B * a.H;
     // item tables address packed rows: the bf16 output map spans all B*T rows as one
     if (a.out_t == ET_BF16 && !make_map_o(&mp.o, a.o, 1, a.B * a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
@@ -1396,31 +1420,14 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
     int* it0 = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b);
     int* its = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b + wv.it0_b);
     int* ito = reinterpret_cast<int*>(base + wv.maps_b + wv.starts_b + wv.s1_b + wv.it0_b + wv.its_b);
-    std::vector<int> h0, hs, ho;
-    h0.reserve((size_t)BH * 8);
-    hs.reserve((size_t)BH * max(0, P - 2) * 8);
-    ho.reserve((size_t)BH * (P - 1) * 8);
-    for (int b = 0; b < a.B; ++b)
-        for (int h = 0; h < a.H; ++h) {
-            const int bh = b * a.H + h;
-            const int e0[8] = {b * a.T, a.T, 0, min(NC, L), h, b, bh, 1};   // end state -> s1
-            h0.insert(h0.end(), e0, e0 + 8);
-            for (int p = 1; p < P; ++p) {
-                const int n0 = p * L, n1 = min(NC, n0 + L);
-                if (p < P - 1) {
-                    const int es[8] = {b * a.T, a.T, n0, n1, h, b, bh * (P - 2) + (p - 1), 0};
-                    hs.insert(hs.end(), es, es + 8);
-                }
-                const int eo[8] = {b * a.T, a.T, n0, n1, h, b, bh * (P - 1) + (p - 1), p == P - 1};
-                ho.insert(ho.end(), eo, eo + 8);
-            }
-        }
-    // pageable sources: the copies are staged before the calls return
-    cudaError_t e = cudaMemcpyAsync(it0, h0.data(), h0.size() * sizeof(int), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess && !hs.empty())
-        e = cudaMemcpyAsync(its, hs.data(), hs.size() * sizeof(int), cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(ito, ho.data(), ho.size() * sizeof(int), cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    {
+        const int n = BH * P;
+        count_launch();
+        wave_items_kernel<<<(n + 255) / 256, 256, 0, s>>>(it0, its, ito, a.B, a.T, a.H, P, L);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;

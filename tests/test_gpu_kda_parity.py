@@ -201,3 +201,29 @@ def test_two_wave_split_boundaries(B, T, H):
     o, ST = _run_gpu(inp, S0=S0)
     o_ref, S_ref = _oracle(inp, S0)
     compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what=f"two-wave P={P} L={L}")
+
+
+def test_forward_is_capturable_in_a_cuda_graph():
+    # the two-wave split (device-built work tables, an auxiliary stream joined by events)
+    # recorded once in a CUDA graph and replayed: the replay reproduces the eager result
+    B, T, H = 1, 3000, 4
+    inp = _custom(B, T, H, 128, 128, torch.bfloat16, seed=77)
+    t = {k_: v_.to(DEV) for k_, v_ in inp.items()}
+    wsz = kda.workspace_size(B, T, H, 128, 128, torch.bfloat16)
+    ws = torch.empty(max(wsz, 1), dtype=torch.uint8, device=DEV)
+    o = torch.empty(B, T, H, 128, dtype=torch.float32, device=DEV)
+    ST = torch.empty(B, H, 128, 128, dtype=torch.float32, device=DEV)
+    call = lambda: kda.forward(t["q"], t["k"], t["v"], t["g"], t["beta"], o=o, S_T=ST, workspace=ws,
+                               o_dtype=torch.float32)
+    call()
+    torch.cuda.synchronize()
+    o_eager, S_eager = o.clone(), ST.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    o.zero_()
+    ST.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == 0
+    assert torch.equal(o, o_eager) and torch.equal(ST, S_eager)
