@@ -216,8 +216,10 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
 #pragma unroll
                 for (int j = 0; j < VE; ++j) f[j] = 0.f;
             }
+            // 16-byte stores (rows are 16-byte aligned): a warp's stores spread over all banks
 #pragma unroll
-            for (int j = 0; j < VE; ++j) dst[i * ld + cv + j] = f[j];
+            for (int j = 0; j < VE; j += 4)
+                *reinterpret_cast<float4*>(dst + i * ld + cv + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
         }
     };
     using KCols = std::integral_constant<int, DK>;
@@ -424,12 +426,9 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
             const int i = e / (DK / 4), c = (e % (DK / 4)) * 4;
             if (t0 + i >= T) continue;
             const size_t idx = ((tok0 + t0 + i) * rowH + h) * DK + c;
-            const float* a1 = sDQP + i * LDK + c;
-            const float* a2 = sDKP + i * LDK + c;
-            const float* a3 = sDKM + i * LDK + c;
-            atomicAdd(reinterpret_cast<float4*>(dq + idx), make_float4(a1[0], a1[1], a1[2], a1[3]));
-            atomicAdd(reinterpret_cast<float4*>(dk + idx), make_float4(a2[0], a2[1], a2[2], a2[3]));
-            atomicAdd(reinterpret_cast<float4*>(dg + idx), make_float4(a3[0], a3[1], a3[2], a3[3]));
+            atomicAdd(reinterpret_cast<float4*>(dq + idx), *reinterpret_cast<const float4*>(sDQP + i * LDK + c));
+            atomicAdd(reinterpret_cast<float4*>(dk + idx), *reinterpret_cast<const float4*>(sDKP + i * LDK + c));
+            atomicAdd(reinterpret_cast<float4*>(dg + idx), *reinterpret_cast<const float4*>(sDKM + i * LDK + c));
         }
         if (t < BC && t0 + t < T) atomicAdd(dbeta + (tok0 + t0 + t) * rowH + h, sDbeta[t]);
     }
