@@ -421,7 +421,11 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
         r = kda.profile_collect(name)
         if r and r[1] > 0:
             prof[name] = {"ms_total": r[0], "launches": r[1], "ms_per_launch": r[0] / r[1]}
-    dominant = max(prof, key=lambda n: prof[n]["ms_total"]) if prof else None
+    # the roofline's kernel: the output pass on the tensor-core path (it reads q, k, v, g,
+    # beta and writes o, the scan's algorithmic bytes per token; the state pass, about as
+    # long, reads a subset), else the longest kernel
+    dominant = ("kda_tc_output" if "kda_tc_output" in prof and "conv" not in prof
+                else max(prof, key=lambda n: prof[n]["ms_total"]) if prof else None)
     roof = None
     if dominant:
         per_launch_s = prof[dominant]["ms_per_launch"] * 1e-3
@@ -446,6 +450,14 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                 "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_record(dominant),
                 "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind, "split": split,
                 "kernel_ms_per_launch": prof[dominant]["ms_per_launch"]}
+        # the other peak: the chunk method's useful tensor work, 5*C*d + 6*d^2 FLOP per
+        # token and head (C = 64), over the whole step, against the measured bf16 GEMM rate
+        if w.D == 128 and not w.fused:
+            flops = (5 * 64 * w.D + 6 * w.D * w.D) * w.tokens * w.H
+            tf = flops / (ms_step * 1e-3) / 1e12
+            bf = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+            roof["tensor_step"] = {"achieved": tf, "peak": bf, "unit": "TFLOP/s", "frac": tf / bf,
+                                   "flops_per_step": flops}
 
     e2e = None if args.quick else e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
 
