@@ -1,4 +1,4 @@
-"""The host side of the sequence-parallel forward on CPU ranks (gloo, world size 2).
+"""The host side of the sequence-parallel forward on CPU ranks (gloo, world sizes 2 and 3).
 
 sequence_parallel.forward is run with its local steps supplied by the fp64 oracle
 (the shard's [N | M] from two oracle scans, the prefix fold in fp64, the shard's scan
@@ -27,10 +27,10 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _rows(seed=21):
+def _rows(seed=21, T=None):
     gen = torch.Generator().manual_seed(seed)
     f = dict(generator=gen, dtype=torch.float64)
-    T = CUTS[-1]
+    T = T or CUTS[-1]
     unit = lambda z: z / torch.linalg.vector_norm(z, dim=-1, keepdim=True)
     q, k = unit(torch.randn(B, T, H, D, **f)), unit(torch.randn(B, T, H, D, **f))
     v = torch.randn(B, T, H, D, **f)
@@ -67,17 +67,19 @@ class OracleShardOps:
         return torch.from_numpy(o), torch.from_numpy(ST)
 
 
-def _worker(rank, port, out):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE="2")
+def _worker(rank, port, out, cuts=None):
+    cuts = cuts or CUTS
+    ws_ = len(cuts) - 1
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws_))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
     from linear_attention_sequence_mshortconv_b200 import sequence_parallel as sp
     from oracle import oracle as O
     from datetime import timedelta
-    dist.init_process_group("gloo", rank=rank, world_size=2, timeout=timedelta(seconds=60))
+    dist.init_process_group("gloo", rank=rank, world_size=ws_, timeout=timedelta(seconds=60))
     try:
-        inp, S0 = _rows()
-        a, b = CUTS[rank], CUTS[rank + 1]
+        inp, S0 = _rows(T=cuts[-1])
+        a, b = cuts[rank], cuts[rank + 1]
         shard = {n: x[:, a:b].contiguous() for n, x in inp.items()}
         o, ST = sp.forward(shard["q"], shard["k"], shard["v"], shard["g"], shard["beta"], S0,
                            broadcast_state=True, ops=OracleShardOps(O))
@@ -105,4 +107,26 @@ def test_sequence_parallel_orchestration_gloo():
     scale = np.abs(o_ref).max()
     assert np.abs(o - o_ref).max() <= 1e-12 * scale
     for r in range(2):   # broadcast_state: every rank holds the rows' final state
+        assert np.abs(res[r][2] - S_ref).max() <= 1e-12 * np.abs(S_ref).max()
+
+
+def test_sequence_parallel_three_ranks_with_an_empty_shard():
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as O
+    cuts = [0, 11, 11, 30]   # rank 1 holds no token: its map is the identity
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, port, q, cuts)) for r in range(3)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=180) for _ in procs), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    inp, S0 = _rows(T=cuts[-1])
+    o_ref, S_ref = O.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S0.numpy())
+    o = np.concatenate([r[1] for r in res], axis=1)
+    assert np.abs(o - o_ref).max() <= 1e-12 * np.abs(o_ref).max()
+    for r in range(3):
         assert np.abs(res[r][2] - S_ref).max() <= 1e-12 * np.abs(S_ref).max()
