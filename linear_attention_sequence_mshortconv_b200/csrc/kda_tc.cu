@@ -21,12 +21,16 @@
 // only B*H = 16 heads for 148 SMs, so each head's chunk sequence is cut into P
 // segments of L chunks.  Eq. 14 is affine in the state, so a segment maps its entry
 // state S to M S + N.
-//   pass 1 (MODE_STATE, segments 0..P-2): run the recurrence on the augmented state
-//          [S | Phi] starting from [0 | I] with the values of the segment: the result
-//          is [N | M] (the identity columns carry no values).
+//   state pass (MODE_STATE): run the recurrence on the augmented state [S | Phi]
+//          starting from [0 | I] with the values of the segment: the result is [N | M]
+//          (the identity columns carry no values).
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
-//   pass 2 (MODE_OUTPUT, all segments): run the recurrence from S_start(p) and write
-//          o (and S_T from the last segment).
+//   output pass (MODE_OUTPUT): run the recurrence from S_start(p) and write o (and S_T
+//          from the last segment).
+// A uniform batch runs in two waves (host side, below): segment 0's output pass beside
+// the state pass of segments 1..P-2, then the combine and the output pass of segments
+// 1..P-1.  The gated epilogue, packed samples and sequence shards use one state pass over
+// segments 0..P-2 (or all P) and one output pass over every segment.
 //
 // Inside a CTA (one per (b, h, segment), 512 threads) two warp groups form a
 // two-stage pipeline over the segment's chunks:
