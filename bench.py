@@ -6,13 +6,17 @@
 
 One JSON line on stdout (rank 0).  A step is one kda_forward call over one batch of
 the workload (inputs resident in HBM).  Timing: W untimed warm-up steps, then K steps
-bracketed by a barrier and torch.cuda.synchronize() on both sides, CUDA events on the
-launching stream, max over ranks.  The inputs (672 MB per step for the video clip)
-are larger than the 126 MB L2, so no flush is needed between steps.
+bracketed by a barrier and torch.cuda.synchronize() on both sides, a CUDA event on the
+launching stream after every step; the step time is the median over the K steps, max
+over ranks.  The inputs (672 MB per step for the video clip) are larger than the
+126 MB L2, so no flush is needed between steps.  Per-kernel times come from a separate
+pass after the timed region.  The default run also times the other forward workloads
+(image stream, fused conv + scan, long video) and reports them under extra_workloads.
 
-Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling over
-independent (batch, head) scans; no collective on the data path).  `--impl reference`
-times the fp64 CPU oracle on the host cores instead (rank 0 only).
+Multi-GPU (torchrun): the ranks run the sequence-parallel forward of one stream of
+N x T tokens, rank r holding the r-th T-token shard (weak scaling: per-rank work is
+fixed); the exchange is one NCCL all-gather of the shards' affine maps per step.
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -264,9 +268,13 @@ def run_reference(args, ws, rank, w: W.Workload):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w: W.Workload, ws: int):
+def workload_config(w: W.Workload, ws: int, sp: bool = False):
+    par = "single GPU"
+    if ws > 1:
+        par = (f"sequence parallel x{ws}: one stream of {ws}x{w.T} tokens, rank r holds the r-th "
+               f"{w.T}-token shard; one NCCL all-gather of the shard maps per step") if sp else f"replicas x{ws}"
     return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d": w.D, "chunk": w.chunk,
-            "fused_conv": w.fused, "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "fused_conv": w.fused, "parallelism": par,
             "l2": "inputs larger than L2 (no flush)" if algorithmic_bytes(w) > 126e6
                   else "L2 flushed between steps"}
 
@@ -274,6 +282,24 @@ def workload_config(w: W.Workload, ws: int):
 # ----------------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------------
+
+def make_sp_step(w: W.Workload, rank: int, world: int):
+    """One step of the sequence-parallel forward of ONE stream of world * T tokens: rank r
+    holds tokens [r*T, (r+1)*T) (its shard drawn from its own seed), runs the shard's state
+    pass, takes part in the one NCCL all-gather of the shard maps, folds the earlier shards
+    into its entry state and runs its output pass."""
+    from linear_attention_sequence_mshortconv_b200 import sequence_parallel as SP
+    dev = torch.device("cuda")
+    inp = W.make_kda_inputs(W.dataclasses.replace(w, seed=w.seed + 1000 * rank), device=dev)
+    box = {}
+
+    def step():
+        box["o"], box["S_T"] = SP.forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=w.chunk,
+                                          o_dtype=w.dtype)
+    step()
+    torch.cuda.synchronize()
+    return step, inp, box["o"], box["S_T"]
+
 
 def make_step(w: W.Workload, rank: int):
     from linear_attention_sequence_mshortconv_b200 import kda
@@ -304,20 +330,92 @@ def make_step(w: W.Workload, rank: int):
 
 
 def timed(step, K, ws):
+    """K steps between a barrier + synchronize on both sides, with a CUDA event on the
+    launching stream before the first step and after every step.  Returns (total ms,
+    per-step ms list)."""
     barrier(ws)
     torch.cuda.synchronize()
     s = torch.cuda.current_stream()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(s)
-    for _ in range(K):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    ev[0].record(s)
+    for i in range(K):
         step()
-    b.record(s)
+        ev[i + 1].record(s)
     torch.cuda.synchronize()
     barrier(ws)
-    return a.elapsed_time(b)
+    return ev[0].elapsed_time(ev[K]), [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
 
 
-def e2e_measure(w: W.Workload, K: int, ws: int, rank: int):
+PROFILED = ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "kda_tc_output_first", "conv",
+            "kda_sp_fold")
+
+
+def kernel_profile(step, K):
+    """Per-kernel device time from CUDA events the library records around its own launches,
+    in a separate pass after the timed region (so the timed steps carry no extra events)."""
+    from linear_attention_sequence_mshortconv_b200 import kda
+    for name in PROFILED:
+        kda.profile_collect(name)
+    kda.profile_enable(True)
+    for _ in range(K):
+        step()
+    torch.cuda.synchronize()
+    kda.profile_enable(False)
+    prof = {}
+    for name in PROFILED:
+        r = kda.profile_collect(name)
+        if r and r[1] > 0:
+            prof[name] = {"ms_per_step": r[0] / K, "launches_per_step": r[1] / K, "ms_per_launch": r[0] / r[1]}
+    return prof
+
+
+def step_roofline(w: W.Workload, ms_step: float, peaks, peak_kind, prof=None):
+    """The forward call's roofline: its algorithmic bytes over the median step time against
+    the measured HBM copy bandwidth (the bound), and the chunk method's useful tensor FLOPs
+    against the measured bf16 GEMM rate.  Per-kernel shares of the step under "kernels"."""
+    alg = algorithmic_bytes(w)
+    achieved = alg / (ms_step * 1e-3) / 1e9
+    peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": traffic_record(w.name), "algorithmic_bytes_per_step": alg, "peak_source": peak_kind,
+            "scope": "whole forward call (every kernel of the step)"}
+    if w.D == 128 and w.dtype != torch.float32:
+        flops = (5 * 64 * w.D + 6 * w.D * w.D) * w.tokens * w.H
+        tf = flops / (ms_step * 1e-3) / 1e12
+        bf = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+        roof["tensor_step"] = {"achieved": tf, "peak": bf, "unit": "TFLOP/s", "frac": tf / bf, "flops_per_step": flops}
+    if prof:
+        roof["kernels"] = {n: {**v, "share_of_step": v["ms_per_step"] / ms_step} for n, v in prof.items()}
+    return roof
+
+
+def e2e_measure_sp(w: W.Workload, K: int, ws: int, rank: int):
+    """The sequence-parallel step through the public API with host buffers: every step
+    uploads this rank's shard from pinned host memory, runs the sharded forward (with its
+    all-gather) and reads o and S_T back; max over ranks."""
+    from linear_attention_sequence_mshortconv_b200 import sequence_parallel as SP
+    host = W.make_kda_inputs(W.dataclasses.replace(w, seed=w.seed + 1000 * rank), device="cpu")
+    host = {k: v.pin_memory() for k, v in host.items() if isinstance(v, torch.Tensor)}
+    dv = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    o_h = torch.empty((w.B, w.T, w.H, w.D), dtype=w.dtype).pin_memory()
+    S_h = torch.empty((w.B, w.H, w.D, w.D), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4
+
+    def step():
+        for k_, v in host.items():
+            dv[k_].copy_(v, non_blocking=True)
+        o, S_T = SP.forward(dv["q"], dv["k"], dv["v"], dv["g"], dv["beta"], chunk=w.chunk, o_dtype=w.dtype)
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(S_T, non_blocking=True)
+    step()
+    total, per = timed(step, K, ws)
+    ms = max_over_ranks(statistics.median(per), ws)
+    return {"value": ws * w.tokens / (ms * 1e-3) / 1e6, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "pipelined": "no (copies, call and read-back in order)"}
+
+
+def e2e_measure(w: W.Workload, K: int, ws: int, rank: int, sp: bool = False):
     """Same metric through the public API with HOST buffers: every step copies its inputs
     from pinned host memory, runs the call and reads o and S_T back.  Steps are
     pipelined over three streams with two device buffer sets: the upload of step n+1
@@ -325,6 +423,8 @@ def e2e_measure(w: W.Workload, K: int, ws: int, rank: int):
     the two directions at once).  The timed region runs from before the first upload to
     after the last read-back."""
     from linear_attention_sequence_mshortconv_b200 import kda
+    if sp:
+        return e2e_measure_sp(w, K, ws, rank)
     dev = torch.device("cuda")
     host = W.make_kda_inputs(w, device="cpu") if not w.fused else None
     if host is None:
@@ -390,6 +490,24 @@ def e2e_measure(w: W.Workload, K: int, ws: int, rank: int):
             "pipelined": "upload of step n+1 overlaps compute and read-back of step n"}
 
 
+def forward_record(w: W.Workload, K: int, peaks, peak_kind):
+    """One other forward workload, device-timed like the headline (median of K steps), with
+    its call-level roofline and per-kernel profile (and the conv's ALU term when fused)."""
+    st, _, _, _ = make_step(w, 0)
+    for _ in range(3):
+        st()
+    total, per = timed(st, K, 1)
+    m = statistics.median(per)
+    prof = kernel_profile(st, max(3, K // 4))
+    rec = {"workload": w.name, "ms_per_step": m, "ms_per_step_mean": total / K, "steps": K,
+           "value": w.tokens / (m * 1e-3) / 1e6, "unit": UNIT,
+           "roofline": step_roofline(w, m, peaks, peak_kind, prof)}
+    if w.fused and "conv" in prof:
+        rec["conv_alu"] = conv_alu_roofline(w, prof["conv"]["ms_per_step"])
+    torch.cuda.synchronize()
+    return rec
+
+
 def run_gpu(args, ws, rank, local, w: W.Workload):
     from linear_attention_sequence_mshortconv_b200 import build as libbuild
     from linear_attention_sequence_mshortconv_b200 import kda
@@ -397,7 +515,8 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
         libbuild.build()
     barrier(ws)
     kda.load_library()
-    step, inp, o, S_T = make_step(w, rank)
+    sp = ws > 1 and not w.fused
+    step, inp, o, S_T = make_sp_step(w, rank, ws) if sp else make_step(w, rank)
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -405,96 +524,39 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
         raise RuntimeError("non-finite output")
 
     launches0 = kda.kernel_launches()
-    kda.profile_enable(True)
     sampler = ClockSampler(local)
     with sampler:
-        ms = timed(step, args.steps, ws)
-    kda.profile_enable(False)
+        total, per = timed(step, args.steps, ws)
     launches = kda.kernel_launches() - launches0
-    ms = max_over_ranks(ms, ws)
-    ms_step = ms / args.steps
-    value = ws * w.tokens / (ms_step * 1e-3) / 1e6
-
+    ms_med = max_over_ranks(statistics.median(per), ws)
+    ms_mean = max_over_ranks(total / args.steps, ws)
+    value = ws * w.tokens / (ms_med * 1e-3) / 1e6
     peaks, peak_kind = read_peaks()
-    prof = {}
-    for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "kda_tc_output_first", "conv"):
-        r = kda.profile_collect(name)
-        if r and r[1] > 0:
-            prof[name] = {"ms_total": r[0], "launches": r[1], "ms_per_launch": r[0] / r[1]}
-    # the roofline's kernel: the output pass on the tensor-core path (it reads q, k, v, g,
-    # beta and writes o, the scan's algorithmic bytes per token; the state pass, about as
-    # long, reads a subset), else the longest kernel
-    dominant = ("kda_tc_output" if "kda_tc_output" in prof and "conv" not in prof
-                else max(prof, key=lambda n: prof[n]["ms_total"]) if prof else None)
-    roof = None
-    if dominant:
-        per_launch_s = prof[dominant]["ms_per_launch"] * 1e-3
-        # the dominant kernel's algorithmic bytes per launch: the scan's, times the share
-        # of the tokens its launches cover (the two-wave split gives segment 0 its own
-        # output launch, "kda_tc_output_first", so "kda_tc_output" covers segments 1..P-1)
-        launches_per_step = prof[dominant]["launches"] / args.steps
-        share = 1.0
-        if dominant in ("kda_tc_output", "kda_tc_output_first") and not w.fused:
-            P_, L_ = kda.forward_plan(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
-            if P_ > 1:
-                first = min(w.T, L_ * 64) / w.T
-                share = first if dominant == "kda_tc_output_first" else 1.0 - first
-        alg = algorithmic_bytes(w) * share / launches_per_step
-        split = None
-        if not w.fused:
-            P_, L_ = kda.forward_plan(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
-            split = {"segments": P_, "chunks_per_segment": L_}
-        achieved = alg / per_launch_s / 1e9
-        peak = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-        roof = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
-                "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_record(dominant),
-                "algorithmic_bytes_per_launch": alg, "peak_source": peak_kind, "split": split,
-                "kernel_ms_per_launch": prof[dominant]["ms_per_launch"]}
-        # the other peak: the chunk method's useful tensor work, 5*C*d + 6*d^2 FLOP per
-        # token and head (C = 64), over the whole step, against the measured bf16 GEMM rate
-        if w.D == 128 and not w.fused:
-            flops = (5 * 64 * w.D + 6 * w.D * w.D) * w.tokens * w.H
-            tf = flops / (ms_step * 1e-3) / 1e12
-            bf = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
-            roof["tensor_step"] = {"achieved": tf, "peak": bf, "unit": "TFLOP/s", "frac": tf / bf,
-                                   "flops_per_step": flops}
+    prof = kernel_profile(step, max(3, args.steps // 4))
+    roof = step_roofline(w, ms_med, peaks, peak_kind, prof)
+    if not w.fused:
+        P_, L_ = kda.forward_plan(w.B, w.T, w.H, w.D, w.D, w.dtype, w.chunk)
+        roof["split"] = {"segments": P_, "chunks_per_segment": L_}
 
-    e2e = None if args.quick else e2e_measure(w, max(3, min(args.steps, 10)), ws, rank)
+    e2e = None if args.quick else e2e_measure(w, max(3, min(args.steps, 10)), ws, rank, sp=sp)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.quick:
         cpu = cpu_baseline(w)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_med, "ms_per_step_mean": ms_mean,
+            "timing": "median of the per-step CUDA-event times (value uses it); mean = total / steps",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32", "data": "synthetic",
-            "config": workload_config(w, ws), "roofline": roof, "cpu_baseline": cpu,
-            "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary(),
-            "kernels": prof}
+            "config": workload_config(w, ws, sp), "roofline": roof, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches, "clocks": sampler.summary()}
+    if rank == 0 and not args.quick:
+        # the other forward configurations of the workload set, each on its own line entry
+        others = [x for x in (W.IMAGE_STREAM, W.FUSED_MIXED, W.LONG_VIDEO) if x.name != w.name and not args.tokens]
+        line["extra_workloads"] = [forward_record(x, max(20, args.steps // 4), peaks, peak_kind) for x in others]
     if args.extra and rank == 0:
-        extra = []
-        for other in W.WORKLOADS:
-            if other.name == w.name:
-                continue
-            st, _, _, _ = make_step(other, rank)
-            for _ in range(3):
-                st()
-            k_other = max(3, args.steps // 4)
-            kda.profile_enable(True)
-            m = timed(st, k_other, 1) / k_other
-            kda.profile_enable(False)
-            kern = {}
-            for name in ("kda_generic", "kda_tc_state", "kda_tc_combine", "kda_tc_output", "kda_tc_output_first", "conv"):
-                r = kda.profile_collect(name)
-                if r and r[1] > 0:
-                    kern[name] = {"ms_per_step": r[0] / k_other, "launches_per_step": r[1] / k_other}
-            rec = {"workload": other.name, "ms_per_step": m,
-                   "value": other.tokens / (m * 1e-3) / 1e6, "unit": UNIT,
-                   "alg_GBps": algorithmic_bytes(other) / (m * 1e-3) / 1e9, "kernels": kern}
-            if other.fused and "conv" in kern:
-                rec["conv_alu"] = conv_alu_roofline(other, kern["conv"]["ms_per_step"])
-            extra.append(rec)
+        extra = line.setdefault("extra_workloads", [])
         # the headline workload with the output side of Eq. 15 fused (Sigmoid(gate) *
         # RMSNorm(readout)); its extra bytes are the gate read
         if not w.fused:
@@ -513,7 +575,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             for _ in range(3):
                 gstep()
             k_g = max(3, args.steps // 4)
-            mg = timed(gstep, k_g, 1) / k_g
+            mg = timed(gstep, k_g, 1)[0] / k_g
             gbytes = algorithmic_bytes(w) + w.B * w.T * w.H * w.D * torch.tensor([], dtype=w.dtype).element_size()
             extra.append({"workload": w.name + "_gated_output", "ms_per_step": mg,
                           "value": w.tokens / (mg * 1e-3) / 1e6, "unit": UNIT,
@@ -544,7 +606,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                 sstep()
             k_s = max(3, args.steps // 4)
             kda.profile_enable(True)
-            ms_s = timed(sstep, k_s, 1) / k_s
+            ms_s = timed(sstep, k_s, 1)[0] / k_s
             kda.profile_enable(False)
             kern = {}
             for name in ("kda_tc_state", "kda_sp_fold", "kda_tc_combine", "kda_tc_output"):
@@ -574,7 +636,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
             for _ in range(3):
                 bstep()
             k_b = 5
-            mb = timed(bstep, k_b, 1) / k_b
+            mb = timed(bstep, k_b, 1)[0] / k_b
             esz = torch.tensor([], dtype=w.dtype).element_size()
             bbytes = algorithmic_bytes(w) + w.B * w.T * w.H * (4 * w.D * 4 + 4)
             # the kernel's fp32 matrix-product multiply-adds per (32-token chunk C, 16 value
@@ -608,7 +670,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
         for _ in range(3):
             cstep()
         k_c = 5
-        mc = timed(cstep, k_c, 1) / k_c
+        mc = timed(cstep, k_c, 1)[0] / k_c
         cf = 2 * conv_fmas(fw) // 3
         rate = kda.fma_probe()
         extra.append({"workload": fw.name + "_conv_backward_xq", "ms_per_step": mc,
@@ -626,7 +688,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
                                         fin["wv"], fin["g"], fin["beta"], fb_do, workspace=fb_ws)
         for _ in range(2):
             fbstep()
-        mf = timed(fbstep, 3, 1) / 3
+        mf = timed(fbstep, 3, 1)[0] / 3
         extra.append({"workload": fw.name + "_backward", "ms_per_step": mf,
                       "value": fw.tokens / (mf * 1e-3) / 1e6, "unit": UNIT,
                       "path": "fp32 conv recompute, per-head norm, kda_backward, norm and conv backward"})
@@ -660,7 +722,7 @@ def run_part(args, w: W.Workload):
             kda.mshortconv_backward(fin["xq"], dy, fin["segments"], w.Kt, *fin["wq"])
     for _ in range(max(1, args.warmup)):
         step()
-    ms = timed(step, args.steps, 1) / args.steps
+    ms = timed(step, args.steps, 1)[0] / args.steps
     print(json.dumps({"part": args.part, "workload": w.name, "ms_per_step": ms, "steps": args.steps,
                       "tokens": w.tokens}), flush=True)
 

@@ -3,54 +3,56 @@
 // What it computes is Eq. 14 of the Chimera paper (section 3.3) with the readout
 // o_t = S_t^T q_t (Eq. 15, inner term).  The pages only say the kernel is "chunked";
 // the chunk algebra is derived from Eq. 14.  Inside a chunk of C = 64 tokens with
-// entry state S0, b_i = sum_{r<=i} g_r (fp32, per key channel), a reference point
-// r = b_31 (the middle of the chunk) keeps every exponential within e^{+-|b|/2}:
-//   K+ = k e^{b - r},  Q+ = q e^{b - r},  K- = k e^{r - b}
+// entry state S0, b_i = sum_{r<=i} g_r (per key channel, base 2, fp32) and two
+// per-channel references rp, rm:
+//   K+ = k 2^{b - rp},  Q+ = q 2^{b - rp},  K- = k 2^{rm - b}
 //   A  = strict_lower((diag(beta) K+) K-^T),   P = lower(Q+ K-^T)  (incl. diagonal)
 //   T  = (I + A)^{-1}                     (16x16 blocks on warp MMAs, fp16 operands)
-//   S^ = diag(e^{r}) S0,   Y = (diag(beta) K+) S^
-//   U  = T (beta V) - T Y                 O = Q+ S^ + P U
-//   S_C = diag(e^{b_C - r}) (S^ + K-^T U)     (k e^{b_C - b} = K- diag(e^{b_C - r}))
-// The state's fp32 master copy lives in TMEM in the scaled form S^ + K-^T U: the row
-// scale e^{b_C - r} of one chunk and e^{r'} of the next are applied together, once,
-// when the next chunk reads it.  Every MMA operand is fp16 in shared memory (11-bit
-// significand: bf16 operands would cost ~3% of RMS(o) in max error); accumulation is
-// fp32 in TMEM.  Exponents are kept in base 2 (g log2(e) summed in fp32).
+//   W  = T (diag(beta) K+),   U~ = T (diag(beta) V)            (state-independent)
+//   S^ = diag(2^{rp}) S0:     U  = U~ - W S^,     O = Q+ S^ + P U
+//   S_C = diag(2^{b_C - rm}) (diag(2^{rm}) S0 + K-^T U)
+// With rp = rm = r (the chunk's middle row) A and P are products of K+ and K- whose
+// factors stay within 2^{+-|b_C|/2}; a chunk whose decay is too strong for that keeps
+// rp = 0 and rm = b_C (every factor <= 1) and forms A and P with pairwise exponentials
+// on CUDA cores instead (chunk_ap_direct).  Every MMA operand is fp16; accumulation is
+// fp32 in TMEM.
+//
+// Transposed state.  The state lives in TMEM as S^T: lane j holds value column j, TMEM
+// column c key channel c (fp32 master).  Every product on the state's serial chain then
+// takes S^T (or U^T) as the A operand straight from TMEM, with no shared-memory round trip:
+//   [U | O]^T  = [U~^T | 0] + S^T [-W^T | Q+^T]     (M = 128 values, N = 128, K = 128)
+//   master    += U^T K-                              (N = 128 channels, K = 64)
+//   O^T       += U^T P^T                             (N = 64, K = 64)
+// The fp32 master holds diag(2^{-carry}) S: the row scales of one chunk and the next
+// are applied together, once, when the next chunk reads it (S^ = 2^{rp + carry} master
+// in fp16 for the A operand, and the master itself rescaled by 2^{rm + carry}).
 //
 // Parallelism.  A head's scan is sequential over chunks, and one B200 workload has
 // only B*H = 16 heads for 148 SMs, so each head's chunk sequence is cut into P
 // segments of L chunks.  Eq. 14 is affine in the state, so a segment maps its entry
 // state S to M S + N.
-//   state pass (MODE_STATE): run the recurrence on the augmented state [S | Phi]
-//          starting from [0 | I] with the values of the segment: the result is [N | M]
-//          (the identity columns carry no values).
+//   state pass (MODE_STATE): two state chains over the segment, S from 0 with the
+//          segment's values (-> N) and Phi from I without values (-> M).
 //   combine: S_start(p+1) = M_p S_start(p) + N_p in fp32 (CUDA cores).
-//   output pass (MODE_OUTPUT): run the recurrence from S_start(p) and write o (and S_T
-//          from the last segment).
-// A uniform batch runs in two waves (host side, below): segment 0's output pass beside
-// the state pass of segments 1..P-2, then the combine and the output pass of segments
-// 1..P-1.  The gated epilogue, packed samples and sequence shards use one state pass over
-// segments 0..P-2 (or all P) and one output pass over every segment.
+//   output pass (MODE_OUTPUT): the recurrence from S_start(p), writing o (and S_T from
+//          the last segment).
 //
 // Inside a CTA (one per (b, h, segment), 512 threads) two warp groups form a
 // two-stage pipeline over the segment's chunks:
-//   producer (warps 0-7): forms beta K+, Q+, K- (fp16 tiles) of chunk n+1, issues
-//     A|P, reads A and P out of TMEM and inverts I + A.  Everything it does is
-//     independent of the state.
-//   consumer (warps 8-15): chunk n's state chain: S^ from the master, [Y; O] MMA,
-//     beta V, U MMA, master += K-^T U and O += P U, output store.
-// The per-chunk tiles are double-buffered; mbarriers hand a buffer over (full) and
-// back (empty, committed by the consumer's last MMA that reads it).  Inputs arrive by
-// TMA straight into the tiles that consume them and are converted in place: q and k
-// of chunk n+2 land in the Q+ / beta K+ slots of their buffer set as soon as the
-// consumer's [Y; O] MMA of chunk n has read them, v of chunk n+1 lands in the beta V
-// tile once chunk n's U MMA has read it, and g of chunk n+1 in a staging tile once the
-// producer has summed chunk n's.
+//   producer (warps 0-7): the state-independent work of chunk n+1: log-decay prefix,
+//     references, K+ / Q+ / K- tiles, A|P (one M = 128 MMA), T, W^T (MMA) -> -W^T tile.
+//   consumer (warps 8-15): chunk n's chain: U~ (MMA), S^, [U | O], U -> fp16, master and
+//     O updates, the output rows, and beta V of chunk n+1.
+// Buffer sets of per-chunk tiles are double-buffered; mbarriers hand a set over (SC:
+// scales, INV: T, PRO: all tiles) and back (EMPTY, committed by the consumer's last MMA
+// on it).  Inputs arrive by TMA straight into the tiles that consume them.
 //
-// Shared-memory operand tiles use the no-swizzle core-matrix layout: 8 rows x 16 B
-// blocks of 128 contiguous bytes.  A thread that owns one key channel writes 8
-// consecutive chunk positions as one 16-byte store, so the channel-major tiles serve
-// both as MN-major operands (chunk position = M/N) and K-major ones (position = K).
+// Shared-memory operand tiles use the no-swizzle core-matrix layout (8 rows x 16 B
+// blocks of 128 contiguous bytes); a descriptor takes the byte stride between core
+// matrices along K and along M or N.  A "channel-major" tile holds element (position i,
+// channel c) at (i >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16 + (i & 7) * 2, so it
+// serves as an MN-major operand when positions are M or N and as a K-major one when
+// positions are K.
 //
 // All waits are bounded (kWaitNs).  On expiry the kernel records DEV_TIMEOUT in the
 // device status word and stops waiting: both warp groups still run every barrier of
@@ -75,70 +77,83 @@ constexpr int NT = 512;       // threads per CTA
 constexpr int NG = 256;       // threads per warp group
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
 constexpr float kLog2e = 1.4426950408889634f;
+// Largest log2 decay factor a middle-row reference may produce in an operand tile: with
+// 2^11 = 2048 an fp16 tile holds k or q components up to 32 in magnitude, and the small
+// factors stay above 2^-11 (normal fp16 for components >= 1/32).
+constexpr float kRangeMax = 11.f;
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
 // ---- shared-memory plan (bytes) --------------------------------------------------
-// Two buffer sets (one per chunk parity) of channel-major fp16 tiles: 8-position group
-// ig at tile + ig*2048, channel c at (c >> 3)*128 + (c & 7)*16 inside it.  Q+ follows
-// beta K+ directly, so [beta K+; Q+] is one M = 128 operand.  T (and P) sit in the
-// set: 8-column groups of T are T_LBO apart; in MODE_OUTPUT P fills the other 1 KB
-// halves, so [T; P] is one M = 128 operand.  The consumer's S^ region holds Y
-// (position-major: 8-position group j at j*NS*16, 8 columns per 16 bytes) once the
-// [Y; O] MMA has read S^.
+// Per buffer set (chunk parity): KP (k -> beta K+ -> -W^T) and QP (q -> Q+) as
+// channel-major tiles, QP directly after KP so [beta K+; Q+] and [-W^T | Q+^T] are single
+// 128-row operands; KM (K-); PF (P as the K-major B operand of O^T += U^T P^T); TF (T as
+// the K-major B operand T^T of W^T and U~^T; in MODE_OUTPUT interleaved with a zero
+// block, so U~ fills [U~^T | 0] with one N = 128 MMA).
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
-    static constexpr int NS = 128;                 // state columns (values only)
-    static constexpr int SET = 65536;              // buffer set stride
-    static constexpr int KP = 0, QP = 16384, KM = 32768, TF = 49152;   // inside a set
-    static constexpr int T_LBO = 2048;
-    static constexpr int VB = 131072;              // beta V (consumer)
-    static constexpr int AT = 147456;              // A, fp16 (producer)
-    static constexpr int U = 155648;               // U (64 x 128)
-    static constexpr int S = 172032;               // S^ (128 x 128 fp16), then Y
-    static constexpr int GST = 204800;             // g staging ([64][128] bf16, TMA)
+    static constexpr int SET = 73728;
+    static constexpr int KP = 0, QP = 16384, KM = 32768, PF = 49152, TF = 57344;
+    static constexpr int T_LBO = 2048;             // T's stride between 8-column groups
+    static constexpr int VB = 147456;              // two beta V tiles (channel-major, values)
+    static constexpr int AT = 180224;              // A, fp16, for the inverse (producer)
+    static constexpr int GS = 188416;              // two g staging tiles ([64][128] bf16, TMA)
     static constexpr int MISC = 221184;
     static constexpr int QK_BYTES = 2 * 16384;     // q and k of one chunk
 };
 template <> struct Plan<MODE_STATE> {
-    static constexpr int NS = 256;                 // [S | Phi]
     static constexpr int SET = 40960;
-    static constexpr int KP = 0, QP = -1, KM = 16384, TF = 32768;
+    static constexpr int KP = 0, QP = -1, KM = 16384, PF = 0, TF = 32768;   // no q, no P
     static constexpr int T_LBO = 1024;
     static constexpr int VB = 81920;
-    static constexpr int AT = 98304;
-    static constexpr int U = 106496;               // U (64 x 256)
-    static constexpr int S = 139264;               // [S^ | Phi^] (128 x 256 fp16), then Y
-    static constexpr int GST = 204800;
-    static constexpr int MISC = 221184;
+    static constexpr int AT = 114688;
+    static constexpr int GS = 122880;
+    static constexpr int SCR = 155648;             // 32 KB scratch of chunk_ap_direct
+    static constexpr int MISC = 188416;
     static constexpr int QK_BYTES = 16384;         // k of one chunk
 };
 // MISC sub-layout
-constexpr int M_BETAP = 0;       // float[64]  beta of the producer's chunk
-constexpr int M_BETAC = 256;     // float[64]  beta of the consumer's chunk
-constexpr int M_TOT = 512;       // float[4][128] per-16-row sums of g log2(e)
-constexpr int M_RB = 2560;       // float2[2][128] (r, b_C) per channel, per buffer set
-constexpr int M_XS = 4608;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 8704;      // mbarriers, see Bar
-constexpr int M_TMEM = 8856;     // uint32 TMEM base
-constexpr int M_ABORT = 8860;    // int
-constexpr int M_GAMMA = 8864;    // float[128] RMSNorm gain of this CTA's head (gated output)
-constexpr int MISC_BYTES = 9376;
-// PRO: a set's beta K+, Q+, K- tiles and r, b_C are ready; INV: its T (and P) too;
-// EMPTY: the consumer's last MMA on the set is done.
-enum Bar { B_PRO = 0, B_EMPTY = 2, B_AP = 4, B_Y = 5, B_U = 6, B_S = 7, B_AFREE = 8, B_UREAD = 9,
-           B_DRAIN = 10, B_DRAIN2 = 11, B_TQK = 12, B_TG = 14, B_TV = 15, B_INV = 16, B_TGATE = 18,
-           NBAR = 19 };
+constexpr int M_BETAP = 0;       // float[64]     beta of the producer's chunk
+constexpr int M_BETAV = 256;     // float[2][64]  beta of the chunk in each beta V tile
+constexpr int M_TOT = 768;       // float[4][128] per-16-row sums of g log2(e)
+constexpr int M_SC = 2816;       // float[2][3][128] per set: S^ scale, master scale, carry after
+constexpr int M_XS = 5888;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 9984;      // mbarriers, see Bar
+constexpr int M_TMEM = 10184;    // uint32 TMEM base
+constexpr int M_ABORT = 10188;   // int
+constexpr int M_RED = 10192;     // float[4][64] per-row sums of squares (gated output)
+constexpr int MISC_BYTES = 11216;
+enum Bar {
+    B_TG = 0,       // [2] g tile landed (staging tile x)
+    B_TQK = 2,      // [2] k (and q) landed in set s
+    B_TV = 4,       // [2] v landed in beta V tile x
+    B_SC = 6,       // [2] set s: scales of its chunk written
+    B_INV = 8,      // [2] set s: T ready
+    B_PRO = 10,     // [2] set s: every tile ready
+    B_EMPTY = 12,   // [2] set s: the consumer's last MMA on it is done
+    B_VE = 14,      // [2] beta V tile x: the U~ MMA that read it is done
+    B_O = 16,       // [2] [U | O] buffer x: the chunk's O is complete
+    B_AP = 18, B_W = 19, B_U = 20, B_U2 = 21, B_S = 22, B_DRAIN = 23, B_DRAIN2 = 24,
+    NBAR = 25
+};
+static_assert(M_BAR + NBAR * 8 <= M_TMEM, "barrier block");
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
+static_assert(smem_bytes<MODE_OUTPUT>() <= 232448, "shared memory");
 
 // TMEM columns.
-constexpr uint32_t TM_S = 0;     // state master (fp32), 128 or 256 columns
-constexpr uint32_t T_AP = 256;   // A (and P below it in MODE_OUTPUT), 64 columns
-// MODE_OUTPUT: [Y; O] (M = 128) at 128, U (M = 64) at 384.
-// MODE_STATE:  Y, then U (M = 64, 256 columns) at 256, once A has been read.
+//   MODE_OUTPUT: master S^T [0,128) | S^ fp16 [128,192) | [U|O] x2 [192,448) | A|P, W^T [448,512)
+//   MODE_STATE:  S^T [0,128), Phi^T [128,256) | S^, Phi^ fp16 [256,320), [320,384) |
+//                U [384,448) | A, W^T [448,512)
+constexpr uint32_t TM_APW = 448;
 template <int MODE> struct Tm;
-template <> struct Tm<MODE_OUTPUT> { static constexpr uint32_t Y = 128, UU = 384; };
-template <> struct Tm<MODE_STATE> { static constexpr uint32_t Y = 256, UU = 256; };
+// (UO / UACC name the same region for the mode that has no such buffer; never used there)
+template <> struct Tm<MODE_OUTPUT> { static constexpr uint32_t MASTER = 0, S16 = 128, UO = 192, UACC = 192; };
+template <> struct Tm<MODE_STATE> { static constexpr uint32_t MASTER = 0, S16 = 256, UACC = 384, UO = 384; };
+
+// Column of K step kk (16 positions) of the fp16 U^T operand inside a 64-column fp32 U
+// region: each column half of the consumer packs its 32 positions into the first 16
+// columns of the 32 it read, so no thread writes a column another thread still reads.
+__device__ __forceinline__ uint32_t ucol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
 // ---- helpers ------------------------------------------------------------------------
 __device__ __forceinline__ uint4 pack8_f16(const float* f)
@@ -158,7 +173,7 @@ __device__ __forceinline__ float2 in2(uint32_t u, const __nv_bfloat16*)
 __device__ __forceinline__ float2 in2(uint32_t u, const __half*) { return unpack_f16x2(u); }
 
 // Byte offset of (row i, column j), j % 8 == 0, in a 64 x 64 fp16 tile in the
-// K-major core-matrix layout the tensor-core MMA reads (8-column groups 1 KB apart).
+// K-major core-matrix layout (8-column groups 1 KB apart).
 __device__ __forceinline__ uint32_t cm64(int i, int j) { return (j >> 3) * 1024 + (i >> 3) * 128 + (i & 7) * 16; }
 // Same for a 16 x 16 scratch block (8-column groups 256 B apart).
 __device__ __forceinline__ uint32_t cm16(int i, int j) { return (j >> 3) * 256 + (i >> 3) * 128 + (i & 7) * 16; }
@@ -223,127 +238,6 @@ __device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, cons
     }
 }
 
-// Output rows of one chunk, TMEM -> global memory.  O is rows 64-127 of the M = 128
-// accumulator [Y; O] (output row i in lane 64 + i), so warps of lane quarters 2 and 3
-// copy it into a row-major staging tile (rows padded by 16 bytes: the 8 rows of a
-// 16-byte store phase hit 8 different bank groups); after the group barrier every warp
-// of the group writes whole rows with coalesced 16-byte stores.
-__device__ __forceinline__ void stage_o(uint32_t tl, int q4, int hg, int lane, uint8_t* stg, int o_f32)
-{
-    if (q4 < 2) return;
-    const int i = 32 * (q4 - 2) + lane;
-    const int es = o_f32 ? 4 : 2, ld = D * es + 16;
-    for (int u = 0; u < 2; ++u) {
-        float v[32];
-        const int cc = 64 * hg + 32 * u;
-        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + cc, v);
-        uint8_t* row = stg + i * ld + cc * es;
-        if (o_f32) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                reinterpret_cast<float4*>(row)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 uu;
-                __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-                reinterpret_cast<uint4*>(row)[j] = uu;
-            }
-        }
-    }
-}
-// bf16 output through TMA: O rows go into two 64-channel x 64-row tiles (128-byte
-// rows, 128-byte swizzle: 16-byte chunk j of row i at i*128 + ((j ^ (i & 7)) * 16), so
-// the 8 rows of a store phase hit 8 different bank groups); one thread then stores
-// both tiles with the TMA (rows past the end of the sequence are clipped).
-__device__ __forceinline__ void stage_o_swz(uint32_t tl, int q4, int hg, int lane, uint8_t* tiles)
-{
-    if (q4 < 2) return;
-    const int i = 32 * (q4 - 2) + lane;
-    uint8_t* tile = tiles + hg * 8192;
-    for (int u = 0; u < 2; ++u) {
-        float v[32];
-        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint4 uu;
-            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) hh[e] = __floats2bfloat162_rn(v[8 * j + 2 * e], v[8 * j + 2 * e + 1]);
-            const int chunk = 4 * u + j;
-            *reinterpret_cast<uint4*>(tile + i * 128 + ((chunk ^ (i & 7)) * 16)) = uu;
-        }
-    }
-}
-// Output side of Eq. 15 for a bf16 output: y = Sigmoid(gate) * gamma_h * RMSNorm(o) per
-// output row, written into the same swizzled tiles as stage_o_swz.  The gate arrives by
-// TMA as two swizzled 64-channel tiles (the layout of the output tiles).  A row's 128
-// channels sit in two warps (column halves), so its sum of squares is exchanged through
-// `red` between two group barriers; TMEM is read twice instead of holding 64 values.
-__device__ __forceinline__ void stage_o_gated(uint32_t tl, int q4, int hg, int lane, uint8_t* tiles,
-                                              const uint8_t* gtiles, float* red, const float* sGamma, float eps)
-{
-    const int i = 32 * (q4 - 2) + lane;
-    if (q4 >= 2) {
-        float ss = 0.f;
-        for (int u = 0; u < 2; ++u) {
-            float v[32];
-            tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-        }
-        red[2 * i + hg] = ss;
-    }
-    named_sync(2, NG);
-    if (q4 < 2) return;
-    const float m = (red[2 * i] + red[2 * i + 1]) * (1.f / D) + eps;
-    const float inv = m > 0.f ? rsqrtf(m) : 0.f;
-    uint8_t* tile = tiles + hg * 8192;
-    const uint8_t* gtile = gtiles + hg * 8192;
-    for (int u = 0; u < 2; ++u) {
-        float v[32];
-        tmem_ld32(tl + Tm<MODE_OUTPUT>::Y + 64 * hg + 32 * u, v);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int chunk = 4 * u + j;
-            const int off = i * 128 + ((chunk ^ (i & 7)) * 16);
-            const uint4 gu = *reinterpret_cast<const uint4*>(gtile + off);
-            const __nv_bfloat162* gb = reinterpret_cast<const __nv_bfloat162*>(&gu);
-            const int c0 = 64 * hg + 8 * chunk;
-            const float4 g0 = *reinterpret_cast<const float4*>(sGamma + c0);
-            const float4 g1 = *reinterpret_cast<const float4*>(sGamma + c0 + 4);
-            const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            uint4 uu;
-            __nv_bfloat162* hh = reinterpret_cast<__nv_bfloat162*>(&uu);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 gv = __bfloat1622float2(gb[e]);
-                const float y0 = __fdividef(v[8 * j + 2 * e] * inv * gm[2 * e], 1.f + __expf(-gv.x));
-                const float y1 = __fdividef(v[8 * j + 2 * e + 1] * inv * gm[2 * e + 1], 1.f + __expf(-gv.y));
-                hh[e] = __floats2bfloat162_rn(y0, y1);
-            }
-            *reinterpret_cast<uint4*>(tile + off) = uu;
-        }
-    }
-}
-
-__device__ __forceinline__ void flush_o(const uint8_t* stg, int tg, void* o, int o_f32, int64_t rowbase, int T, int H,
-                                        int h, int t0)
-{
-    const int es = o_f32 ? 4 : 2, ld = D * es + 16;
-    const int per_row = D * es / 16;                 // 16-byte pieces per row
-    for (int e = tg; e < C * per_row; e += NG) {
-        const int i = e / per_row, pc = e % per_row;
-        if (t0 + i < T) {
-            const uint4 x = *reinterpret_cast<const uint4*>(stg + i * ld + pc * 16);
-            uint8_t* dst = reinterpret_cast<uint8_t*>(o) + ((((size_t)rowbase + t0 + i) * H + h) * D) * es + pc * 16;
-            *reinterpret_cast<uint4*>(dst) = x;
-        }
-    }
-}
-
 // 16 rows x 2 channels (one 4-byte word per row) of a [64][128] 2-byte tile in shared
 // memory, as TMA lands it: a warp reads 128 contiguous bytes per row.
 __device__ __forceinline__ void ld_rows16(uint32_t (&dst)[16], const uint8_t* tile, int r0, int cp)
@@ -372,23 +266,228 @@ __device__ __forceinline__ void st_pair(uint8_t* tile, int ig, int cp, const uin
     *reinterpret_cast<uint4*>(tile + ig * 2048 + (c_second >> 3) * 128 + (c_second & 7) * 16) = sw ? a0 : a1;
 }
 
+// A (and P) of one chunk on CUDA cores, for a chunk whose decay range is too wide for a
+// single reference: A_ij = beta_i sum_c k_ic k_jc 2^{b_ic - b_jc} (j < i) and P_ij =
+// sum_c q_ic k_jc 2^{b_ic - b_jc} (j <= i), every exponential <= 1 formed directly.  The
+// raw k (and q) tiles are still in KP (QP); `scr` holds the fp32 table b[64][128] (base
+// 2, from the chunk start), written by the caller.  Writes A (fp16) to `at` and P to `pf`
+// in the cm64 layout (P zero above the diagonal).  Called by all 256 producer threads
+// after a group barrier that publishes the table; ends with the group barrier passed.
+template <bool OUT, typename TQ>
+__device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* ktile, const uint8_t* qtile,
+                                             const float* sBeta, uint8_t* at, uint8_t* pf, int tg, int t0, int Tq)
+{
+    const float* bT = reinterpret_cast<const float*>(scr);
+    const int i = tg & 63, cq = tg >> 6;
+    const int nv = min(C, Tq - t0);          // rows of this chunk inside the sequence
+    float accA[16], accP[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) accA[jj] = accP[jj] = 0.f;
+    if (16 * cq <= i && i < nv) {
+        const TQ* tq = nullptr;
+        for (int c8 = 0; c8 < 16; ++c8) {
+            const uint4 ku = *reinterpret_cast<const uint4*>(ktile + i * 256 + c8 * 16);
+            const uint4 qu = OUT ? *reinterpret_cast<const uint4*>(qtile + i * 256 + c8 * 16) : make_uint4(0, 0, 0, 0);
+            const float4 b0 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8);
+            const float4 b1 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8 + 4);
+            float ki[8], qi[8];
+            const float bi[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            {
+                const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 a = in2(kw[e], tq), b = in2(qw[e], tq);
+                    ki[2 * e] = a.x; ki[2 * e + 1] = a.y;
+                    qi[2 * e] = b.x; qi[2 * e + 1] = b.y;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+                const int j = 16 * cq + jj;
+                if (j <= i) {
+                    const uint4 kj = *reinterpret_cast<const uint4*>(ktile + j * 256 + c8 * 16);
+                    const float4 c0 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8);
+                    const float4 c1 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8 + 4);
+                    const float bj[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    const uint32_t kw[4] = {kj.x, kj.y, kj.z, kj.w};
+                    float sa = 0.f, sp = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 kk = in2(kw[e], tq);
+                        const float d0 = ex2_approx(bi[2 * e] - bj[2 * e]) * kk.x;
+                        const float d1 = ex2_approx(bi[2 * e + 1] - bj[2 * e + 1]) * kk.y;
+                        sa = fmaf(ki[2 * e], d0, fmaf(ki[2 * e + 1], d1, sa));
+                        if (OUT) sp = fmaf(qi[2 * e], d0, fmaf(qi[2 * e + 1], d1, sp));
+                    }
+                    accA[jj] += sa;
+                    accP[jj] += sp;
+                }
+            }
+        }
+    }
+    named_sync(1, NG);   // the table may be overwritten (in MODE_OUTPUT it covers PF)
+    const float bi = sBeta[i];
+    for (int half = 0; half < 2; ++half) {
+        float fa[8], fp[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int jj = 8 * half + e, j = 16 * cq + jj;
+            fa[e] = j < i ? bi * accA[jj] : 0.f;
+            fp[e] = j <= i ? accP[jj] : 0.f;
+        }
+        const int j0 = 16 * cq + 8 * half;
+        if (16 * cq <= i) *reinterpret_cast<uint4*>(at + cm64(i, j0)) = pack8_f16(fa);
+        if (OUT) *reinterpret_cast<uint4*>(pf + cm64(i, j0)) = pack8_f16(fp);
+    }
+}
+
+// Inverse T = (I + A)^{-1} of the strictly lower 64 x 64 A (fp16 at Ah, cm64 layout) into
+// the set's T tile (cmT layout, lower blocks only; the upper ones are zeroed elsewhere).
+// Diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
+// N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs.  Then the
+// off-diagonal blocks by halves of the matrix (each warp: one 8-column half of one 16x16
+// block; X products through per-warp fp16 scratch):
+//   level 1: T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)
+//   level 2: X_IJ = sum_{K=J}^{1} A_IK T_KJ  (I = 2, 3; J = 0, 1), then T_IJ = -sum_{K=2}^{I} T_IK X_KJ
+// Called by the 256 producer threads; barriers on named barrier 1.
+template <int T_LBO>
+__device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint32_t xs, int w, int lane)
+{
+    auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
+    if (w < 4) {
+        const int b0 = 16 * w, g = lane >> 2, q = lane & 3;
+        const uint32_t scr = xs + 512 * w;
+        uint32_t aN[4], bN[4], bP[4], aX[4];
+        ldsm_x4(aN, Ah + cm64(b0 + (lane & 15), b0 + 8 * (lane >> 4)));
+        ldsm_x4_t(bN, Ah + cm64(b0 + (lane & 7) + 8 * ((lane >> 3) & 1), b0 + 8 * (lane >> 4)));
+        float n2a[4] = {0.f, 0.f, 0.f, 0.f}, n2b[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_16x16(n2a, n2b, aN, bN);                                   // N^2
+        c_to_scr(scr, lane, n2a, n2b);
+        __syncwarp();
+        scr_to_b(bP, scr, lane);                                       // bP = N^2
+        __syncwarp();
+        c_to_a(aX, n2a, n2b);
+        float n4a[4] = {0.f, 0.f, 0.f, 0.f}, n4b[4] = {0.f, 0.f, 0.f, 0.f};
+        float n3a[4] = {0.f, 0.f, 0.f, 0.f}, n3b[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_16x16(n4a, n4b, aX, bP);                                   // N^4
+        mma_16x16(n3a, n3b, aN, bP);                                   // N^3
+        c_to_scr(scr, lane, n4a, n4b);
+        __syncwarp();
+        scr_to_b(bP, scr, lane);                                       // bP = N^4
+        __syncwarp();
+        c_to_a(aX, n4a, n4b);
+        float n8a[4] = {0.f, 0.f, 0.f, 0.f}, n8b[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_16x16(n8a, n8b, aX, bP);                                   // N^8
+        // Z = I - N + N^2 - N^3, in the C layout (rows g, g+8; columns 2q, 2q+1 of each
+        // 8-column half); N's values come from its A fragment
+        float za[4], zb[4];
+        {
+            const float2 n00 = unpack_f16x2(aN[0]), n10 = unpack_f16x2(aN[1]);
+            const float2 n01 = unpack_f16x2(aN[2]), n11 = unpack_f16x2(aN[3]);
+            const float d0 = (g == 2 * q) ? 1.f : 0.f, d1 = (g == 2 * q + 1) ? 1.f : 0.f;
+            za[0] = d0 - n00.x + n2a[0] - n3a[0];
+            za[1] = d1 - n00.y + n2a[1] - n3a[1];
+            za[2] = -n10.x + n2a[2] - n3a[2];
+            za[3] = -n10.y + n2a[3] - n3a[3];
+            zb[0] = -n01.x + n2b[0] - n3b[0];
+            zb[1] = -n01.y + n2b[1] - n3b[1];
+            zb[2] = d0 - n11.x + n2b[2] - n3b[2];
+            zb[3] = d1 - n11.y + n2b[3] - n3b[3];
+        }
+        {   // Z += Z N^4
+            float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
+            c_to_a(aX, za, zb);
+            mma_16x16(ta, tb, aX, bP);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
+        }
+        c_to_scr(scr, lane, n8a, n8b);
+        __syncwarp();
+        scr_to_b(bP, scr, lane);                                       // bP = N^8
+        {   // Z += Z N^8
+            float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
+            c_to_a(aX, za, zb);
+            mma_16x16(ta, tb, aX, bP);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
+        }
+        st_shared_b32(Tt + cmT(b0 + g, b0) + 4 * q, pack_f16x2(za[0], za[1]));
+        st_shared_b32(Tt + cmT(b0 + g + 8, b0) + 4 * q, pack_f16x2(za[2], za[3]));
+        st_shared_b32(Tt + cmT(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
+        st_shared_b32(Tt + cmT(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
+    }
+    named_sync(1, NG);
+    const int g = lane >> 2, q = lane & 3, half = w & 1;
+    const uint32_t scr = xs + 512 * w;
+    auto scr_of = [&](int wx) { return xs + 512 * wx; };
+    auto put_x = [&](uint32_t dst, const float (&x)[4]) {
+        st_shared_b32(dst + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
+        st_shared_b32(dst + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
+    };
+    auto put_t = [&](int I, int N0, const float (&tt)[4]) {
+        st_shared_b32(Tt + cmT(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
+        st_shared_b32(Tt + cmT(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
+    };
+    auto a_frag = [&](uint32_t (&fr)[4], uint32_t base, int I, int K, bool isT) {
+        if (isT) ldsm_x4(fr, base + cmT(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
+        else ldsm_x4(fr, base + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
+    };
+    if (w < 4) {   // level 1
+        const int I = (w >> 1) ? 3 : 1, J = I - 1, N0 = 16 * J + 8 * half;
+        uint32_t aA[4], bT[2], bX[2], aT[4];
+        float x[4] = {0.f, 0.f, 0.f, 0.f}, tt[4] = {0.f, 0.f, 0.f, 0.f};
+        a_frag(aA, Ah, I, J, false);
+        ldsm_x2_t(bT, Tt + cmT(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
+        mma16816(x, aA, bT);
+        put_x(scr, x);
+        __syncwarp();
+        ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+        a_frag(aT, Tt, I, I, true);
+        mma16816(tt, aT, bX);
+        put_t(I, N0, tt);
+    }
+    named_sync(1, NG);
+    // level 2, X: warp w -> block (I, J) = (2 + (w >> 2), (w >> 1) & 1), half w & 1
+    const int I2 = 2 + (w >> 2), J2 = (w >> 1) & 1, N2 = 16 * J2 + 8 * half;
+    {
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = J2; K < 2; ++K) {
+            uint32_t aA[4], bT[2];
+            a_frag(aA, Ah, I2, K, false);
+            ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N2));
+            mma16816(x, aA, bT);
+        }
+        put_x(scr, x);
+    }
+    named_sync(1, NG);
+    // level 2, T: the same (I, J, half); X_KJ half was written by warp 4(K-2) + 2J + half
+    {
+        float tt[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int K = 2; K <= I2; ++K) {
+            uint32_t aT[4], bX[2];
+            a_frag(aT, Tt, I2, K, true);
+            ldsm_x2_t(bX, scr_of(4 * (K - 2) + 2 * J2 + half) + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+            mma16816(tt, aT, bX);
+        }
+        put_t(I2, N2, tt);
+    }
+}
+
 // The kernel ---------------------------------------------------------------------------
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-              const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_gate,
               const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop,
-              const float* __restrict__ gamma, float eps, int gated, const int* __restrict__ items)
+              const __nv_bfloat16* __restrict__ gate, const float* __restrict__ gamma, float eps,
+              const int* __restrict__ items)
 {
     using PL = Plan<MODE>;
+    using TM = Tm<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
-    constexpr int NS = PL::NS;
-    constexpr int YJ = NS * 16;               // Y tile: bytes per 8-position group
-    constexpr int T_LBO = PL::T_LBO;          // T's 8-column group stride
-    constexpr uint32_t T_Y = Tm<MODE>::Y, T_UU = Tm<MODE>::UU;
+    constexpr int T_LBO = PL::T_LBO;
     auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     extern __shared__ __align__(1024) uint8_t sm[];
 
@@ -397,7 +496,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int hg = (w >> 2) & 1;              // column half inside a warp group
     const int tg = t & (NG - 1);              // thread index inside its group
     const int cp = tg & 63, rq = tg >> 6;     // channel pair, 16-row quarter (loads, prologue)
-    const int c = t & 127;                    // channel / TMEM row of the state steps
     // This CTA's work: chunks [n0, n1) of head h of one sequence that starts at packed
     // token `rowbase` and has `Tq` tokens.  Uniform batch: sequence b of B rows of T
     // tokens, segment p of P; packed samples: one entry of the host-built item table
@@ -422,16 +520,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         last = p == P - 1;
     }
     const int nk = max(0, n1 - n0);
-    // the bf16 output leaves by TMA store through a [B, T, H, 128] map that clips at the
-    // end of a row; packed samples share one row, so a chunk that runs past its sample's
-    // end is written with masked stores instead
-    const int o_b = items ? 0 : seq;
-    const int64_t o_t = items ? rowbase : 0;
 
     float* sBetaP = reinterpret_cast<float*>(sm + PL::MISC + M_BETAP);
-    float* sBetaC = reinterpret_cast<float*>(sm + PL::MISC + M_BETAC);
+    float* sBetaV = reinterpret_cast<float*>(sm + PL::MISC + M_BETAV);
     float* sTot = reinterpret_cast<float*>(sm + PL::MISC + M_TOT);
-    float2* sRB = reinterpret_cast<float2*>(sm + PL::MISC + M_RB);
+    float* sSC = reinterpret_cast<float*>(sm + PL::MISC + M_SC);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
     int* sAbort = reinterpret_cast<int*>(sm + PL::MISC + M_ABORT);
@@ -447,6 +540,15 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_alloc(sTmem, 512);
         tmem_relinquish();
     }
+    // T tiles of both sets start zero (the zero block beside T in MODE_OUTPUT stays zero)
+    {
+        constexpr int TB = OUT ? 16384 : 8192;
+        for (int e = t; e < 2 * TB / 16; e += NT) {
+            const int s = e / (TB / 16), off = (e % (TB / 16)) * 16;
+            *reinterpret_cast<uint4*>(sm + s * PL::SET + PL::TF + off) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -454,91 +556,113 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);   // this warp's lane quarter
     // TMA of chunk n's [64][128] tiles (packed rows rowbase + n*C ..; rows past the sequence
     // come from the next batch row or the zero fill and are masked where they are used)
-    auto tma_qk = [&](int n) {   // q (MODE_OUTPUT) and k into the Q+ / beta K+ slots of set n&1
-        const int bs = (n - n0) & 1, row = (int)(rowbase + n * C);
-        mbar_arrive_expect_tx(&bars[B_TQK + bs], PL::QK_BYTES);
-        if (OUT) tma_load_3d(sm + bs * PL::SET + PL::QP, &tm_q, &bars[B_TQK + bs], 0, h, row);
-        tma_load_3d(sm + bs * PL::SET + PL::KP, &tm_k, &bars[B_TQK + bs], 0, h, row);
+    auto tma_qk = [&](int n) {   // q (MODE_OUTPUT) and k into the Q+ / beta K+ slots of set (n-n0)&1
+        const int s = (n - n0) & 1, row = (int)(rowbase + n * C);
+        mbar_arrive_expect_tx(&bars[B_TQK + s], PL::QK_BYTES);
+        if (OUT) tma_load_3d(sm + s * PL::SET + PL::QP, &tm_q, &bars[B_TQK + s], 0, h, row);
+        tma_load_3d(sm + s * PL::SET + PL::KP, &tm_k, &bars[B_TQK + s], 0, h, row);
     };
     auto tma_g = [&](int n) {
-        mbar_arrive_expect_tx(&bars[B_TG], 16384);
-        tma_load_3d(sm + PL::GST, &tm_g, &bars[B_TG], 0, h, (int)(rowbase + n * C));
+        const int x = (n - n0) & 1;
+        mbar_arrive_expect_tx(&bars[B_TG + x], 16384);
+        tma_load_3d(sm + PL::GS + x * 16384, &tm_g, &bars[B_TG + x], 0, h, (int)(rowbase + n * C));
     };
     auto tma_v = [&](int n) {
-        mbar_arrive_expect_tx(&bars[B_TV], 16384);
-        tma_load_3d(sm + PL::VB, &tm_v, &bars[B_TV], 0, h, (int)(rowbase + n * C));
+        const int x = (n - n0) & 1;
+        mbar_arrive_expect_tx(&bars[B_TV + x], 16384);
+        tma_load_3d(sm + PL::VB + x * 16384, &tm_v, &bars[B_TV + x], 0, h, (int)(rowbase + n * C));
     };
-    // gated bf16 output: chunk n's gate as two swizzled 64-channel tiles in the upper half
-    // of the S^ region (free from the end of chunk n's [Y; O] MMA to chunk n+1's S^)
-    auto tma_gate = [&](int n) {
-        mbar_arrive_expect_tx(&bars[B_TGATE], 16384);
-        tma_load_3d(sm + PL::S + 16384, &tm_gate, &bars[B_TGATE], 0, h, (int)(rowbase + n * C));
-        tma_load_3d(sm + PL::S + 24576, &tm_gate, &bars[B_TGATE], 64, h, (int)(rowbase + n * C));
-    };
-    const bool gate_fused = OUT && gated && !o_f32;
-    float* sGamma = reinterpret_cast<float*>(sm + PL::MISC + M_GAMMA);
 
     if (t < NG) {
         // ================= producer: state-independent work of chunk n0 + kc ==============
         const TQ* tq = nullptr;
-        uint32_t betaR = 0;
-        int g_issued = 0;   // thread 0: g tiles requested so far
-        if (tg == 0 && nk > 0) {
-            tma_g(n0);
-            g_issued = 1;
+        int g_issued = 0;            // thread 0: g tiles requested so far
+        int n_ap = 0;                // A|P MMAs issued so far (phase of B_AP)
+        float2 carry = make_float2(0.f, 0.f);   // rq == 0: carry of channels 2cp, 2cp+1
+        if (tg == 0) {
+            for (int x = 0; x < min(2, nk); ++x) tma_g(n0 + x);
+            g_issued = min(2, nk);
         }
-        if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0);
-        uint32_t gP[16];     // this chunk's g rows, kept from part 1 to part 2 of the prologue
+        uint32_t betaR = (tg < C) ? load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0) : 0u;
         for (int kc = 0; kc < nk; ++kc) {
-            const int n = n0 + kc, t0 = n * C, bs = kc & 1;
-            uint8_t* set = sm + bs * PL::SET;
-            const uint32_t sset = sbase + bs * PL::SET;
-            // ---- prologue, part 1: g of this chunk (staging) -> cumulative log-decay ------
-            // (needs only the g tile, so it runs before the wait for the buffer set)
-            group_wait(&bars[B_TG], kc & 1, ab, tg == 0, 1);
-            {
-                uint32_t gR[16];
-                ld_rows16(gR, sm + PL::GST, 16 * rq, cp);
-                const bool full = t0 + C <= Tq;
-                if (!full) {
+            const int n = n0 + kc, t0 = n * C, s = kc & 1;
+            uint8_t* set = sm + s * PL::SET;
+            const uint32_t sset = sbase + s * PL::SET;
+            // ---- part 1: g of this chunk -> cumulative log-decay, references, range ---------
+            group_wait(&bars[B_TG + s], (kc >> 1) & 1, ab, tg == 0, 1);
+            uint32_t gP[16];
+            ld_rows16(gP, sm + PL::GS + s * 16384, 16 * rq, cp);
+            if (t0 + C > Tq) {
 #pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= Tq) gR[r] = 0u;
-                }
+                for (int r = 0; r < 16; ++r)
+                    if (t0 + 16 * rq + r >= Tq) gP[r] = 0u;
+            }
+            {
                 const float2 l2e = make_float2(kLog2e, kLog2e);
                 float2 tot = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) tot = __ffma2_rn(in2(gR[r], (const __nv_bfloat16*)nullptr), l2e, tot);
+                for (int r = 0; r < 16; ++r) tot = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, tot);
                 *reinterpret_cast<float2*>(sTot + rq * D + 2 * cp) = tot;
-                if (tg < C) sBetaP[tg] = __uint_as_float(betaR << 16);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) gP[r] = gR[r];
             }
-            named_sync(1, NG);   // the g tile is in registers: the next chunk's may land
-            if (tg == 0 && n + 1 < n1 && !*sAbort) {
-                tma_g(n + 1);
-                g_issued = kc + 2;
+            if (tg < C) sBetaP[tg] = __uint_as_float(betaR << 16);
+            named_sync(1, NG);   // sTot, beta published; this g tile is in registers
+            if (tg == 0 && n + 2 < n1 && !*sAbort) {
+                tma_g(n + 2);
+                g_issued = kc + 3;
             }
             if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
-            float2 r2, bC, run;
+            float2 r2, bC, pre;   // b at row 31, b at row 63, b before this thread's first row
             {
                 float2 tq4[4];
 #pragma unroll
                 for (int qb = 0; qb < 4; ++qb) tq4[qb] = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
-                r2 = __fadd2_rn(tq4[0], tq4[1]);                     // b at row 31
-                bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));     // b at row 63
-                run = make_float2(-r2.x, -r2.y);                     // running b - r
+                r2 = __fadd2_rn(tq4[0], tq4[1]);
+                bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));
+                pre = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int qb = 0; qb < 3; ++qb)
-                    if (qb < rq) run = __fadd2_rn(run, tq4[qb]);
+                    if (qb < rq) pre = __fadd2_rn(pre, tq4[qb]);
             }
-            // ---- part 2: buffer set bs is free once the consumer is done with chunk kc - 2
-            // (its K- and T tiles, and r, b_C); this chunk's q, k have landed in the set -----
-            if (tg == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + bs], ((kc >> 1) - 1) & 1, ab);
-            group_wait(&bars[B_TQK + bs], (kc >> 1) & 1, ab, tg == 0, 1);
+            // the middle-row reference keeps a factor within 2^{max(b_0 - r, r - b_63)}
+            bool wide = false;
+            if (rq == 0) {
+                const float2 b0 = __fmul2_rn(in2(gP[0], (const __nv_bfloat16*)nullptr), make_float2(kLog2e, kLog2e));
+                wide = fmaxf(b0.x - r2.x, r2.x - bC.x) > kRangeMax || fmaxf(b0.y - r2.y, r2.y - bC.y) > kRangeMax;
+            }
+            const bool direct = bar_red_or(1, NG, wide);
+            const float2 rp = direct ? make_float2(0.f, 0.f) : r2;   // reference of K+ and Q+
+            const float2 rm = direct ? bC : r2;                      // reference of K-
+            // ---- part 2: set s is free once the consumer is done with chunk kc - 2; this
+            // chunk's k (and q) have landed in it ------------------------------------------
+            if (tg == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + s], ((kc >> 1) - 1) & 1, ab);
+            group_wait(&bars[B_TQK + s], (kc >> 1) & 1, ab, tg == 0, 1);
+            if (rq == 0) {
+                // consumer scales: S^ = 2^{rp + carry} master, master <- 2^{rm + carry} master
+                float* sc = sSC + s * 3 * D;
+                *reinterpret_cast<float2*>(sc + 2 * cp) = make_float2(ex2_approx(rp.x + carry.x), ex2_approx(rp.y + carry.y));
+                *reinterpret_cast<float2*>(sc + D + 2 * cp) =
+                    make_float2(ex2_approx(rm.x + carry.x), ex2_approx(rm.y + carry.y));
+                carry = make_float2(bC.x - rm.x, bC.y - rm.y);
+                *reinterpret_cast<float2*>(sc + 2 * D + 2 * cp) = carry;
+            }
+            if (direct) {
+                // the fp32 log-decay table of the chunk: in MODE_OUTPUT over KM, PF and the first
+                // 8 KB of TF (all free until the prologue), else in the scratch region
+                uint8_t* scr = OUT ? set + PL::KM : sm + Plan<MODE_STATE>::SCR;
+                float2 run = pre;
+                const float2 l2e = make_float2(kLog2e, kLog2e);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    run = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, run);
+                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(scr) + (16 * rq + r) * D + 2 * cp) = run;
+                }
+                named_sync(1, NG);
+                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBetaP, sm + PL::AT,
+                                         OUT ? set + PL::PF : nullptr, tg, t0, Tq);
+            }
+            // ---- prologue: beta K+, Q+ in place, K- ----------------------------------------
             {
                 uint32_t kR[16], qR[16];
-                const uint32_t (&gR)[16] = gP;
                 ld_rows16(kR, set + PL::KP, 16 * rq, cp);
                 if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
                 if (t0 + C > Tq) {
@@ -546,11 +670,10 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int r = 0; r < 16; ++r)
                         if (t0 + 16 * rq + r >= Tq) kR[r] = qR[r] = 0u;
                 }
+                named_sync(1, NG);   // every raw row is in registers before the tiles are rewritten
                 const float2 l2e = make_float2(kLog2e, kLog2e);
-                if (rq == 0) {
-                    sRB[bs * D + 2 * cp] = make_float2(r2.x, bC.x);
-                    sRB[bs * D + 2 * cp + 1] = make_float2(r2.y, bC.y);
-                }
+                const float2 dlt = make_float2(rm.x - rp.x, rm.y - rp.y);
+                float2 run = make_float2(pre.x - rp.x, pre.y - rp.y);   // b - rp
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[2][4], pm[2][4], pq[2][4];
@@ -558,14 +681,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int r8 = 0; r8 < 8; ++r8) {
                         const int r = 8 * half + r8, i = 16 * rq + r;
-                        run = __ffma2_rn(in2(gR[r], (const __nv_bfloat16*)nullptr), l2e, run);
+                        run = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, run);
                         const float2 kk = in2(kR[r], tq);
                         const float bi = sBetaP[i];
                         const float2 ep = make_float2(ex2_approx(run.x), ex2_approx(run.y));
-                        const float2 em = make_float2(ex2_approx(-run.x), ex2_approx(-run.y));
+                        const float2 em = make_float2(ex2_approx(dlt.x - run.x), ex2_approx(dlt.y - run.y));
                         const float2 kp = __fmul2_rn(__fmul2_rn(kk, make_float2(bi, bi)), ep);   // beta K+
                         const float2 km = __fmul2_rn(kk, em);                                   // K-
-                        const float2 qp = OUT ? __fmul2_rn(in2(qR[r], tq), ep) : make_float2(0.f, 0.f);   // Q+
+                        const float2 qp = OUT ? __fmul2_rn(in2(qR[r], tq), ep) : make_float2(0.f, 0.f);
                         if (r8 & 1) {
                             const int m = r8 >> 1;
                             pk[0][m] = pack_f16x2(lk.x, kp.x); pk[1][m] = pack_f16x2(lk.y, kp.y);
@@ -584,37 +707,28 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             fence_async_smem();
             tc_fence_before();
             named_sync(1, NG);
-            // tiles, r and b_C ready (the test hook withholds chunk 0's signal)
-            if (tg == 0 && !(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + bs]);
-            // ---- A (and P) on the tensor core -------------------------------------------
             if (tg == 0) {
-                // MODE_STATE: A's TMEM columns are the consumer's U until it has read U
-                if (MODE == MODE_STATE && kc >= 1) thread_wait(&bars[B_UREAD], (kc - 1) & 1, ab);
-                tc_fence_after();
-                // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P
-                const uint32_t id = idesc_f16(OUT ? 128 : 64, 64, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_AP, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
-                             sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
-                umma_commit(&bars[B_AP]);
-            }
-            group_wait(&bars[B_AP], kc & 1, ab, tg == 0, 1);
-            // ---- A -> fp16 tile (and P -> the T region's other halves) ------------------
-            const uint32_t Ah = sbase + PL::AT;          // A, fp16 K-major core-matrix tile
-            const uint32_t Tt = sset + PL::TF;           // T: the consumer's operand
-            {
-                float v[32];
-                tmem_ld32(tl + T_AP + 32 * hg, v);
-                int i = -1;
-                bool isP = false;
-                if (OUT) {
-                    // M = 128 layout: row i in lane i; rows 0-63 are A, rows 64-127 are P
-                    i = 32 * (q4 & 1) + lane;
-                    isP = q4 >= 2;
-                } else if (lane < 16) {
-                    i = 16 * q4 + lane;                  // M = 64 layout
+                mbar_arrive(&bars[B_SC + s]);   // this chunk's scales are in place
+                if (!direct) {
+                    tc_fence_after();
+                    // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the
+                    // state pass reads K- as rows 64-127 and ignores them)
+                    const uint32_t id = idesc_f16(128, 64, true, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
+                                 sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
+                    umma_commit(&bars[B_AP]);
                 }
-                if (i >= 0) {
+            }
+            if (!direct) {
+                group_wait(&bars[B_AP], n_ap & 1, ab, tg == 0, 1);
+                ++n_ap;
+                // A (lanes 0-63) -> fp16 tile, P (lanes 64-127) -> the set's P tile
+                if (OUT || q4 < 2) {
+                    float v[32];
+                    tmem_ld32(tl + TM_APW + 32 * hg, v);
+                    const bool isP = q4 >= 2;
+                    const int i = 32 * (q4 & 1) + lane;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
                         float f[8];
@@ -623,454 +737,401 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const int col = 32 * hg + 8 * g8 + j;
                             f[j] = (isP ? (col <= i) : (col < i)) ? v[8 * g8 + j] : 0.f;
                         }
-                        uint8_t* dst = isP ? set + PL::TF + 1024 + cmT(i, 32 * hg + 8 * g8)
-                                           : sm + PL::AT + cm64(i, 32 * hg + 8 * g8);
+                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 32 * hg + 8 * g8) : sm + PL::AT + cm64(i, 32 * hg + 8 * g8);
                         *reinterpret_cast<uint4*>(dst) = pack8_f16(f);
                     }
                 }
-                // the six upper 16x16 blocks of T are zero
-                if (tg < 192) {
-                    const int e = tg >> 5, u = tg & 31;
-                    const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
-                    const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
-                    const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
-                    *reinterpret_cast<uint4*>(set + PL::TF + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
-                }
+            } else if (OUT && tg < 128) {
+                // chunk_ap_direct used the first 8 KB of the T tile as scratch: zero its block
+                // beside T again (T itself is rewritten below)
+                const int kg = tg >> 5, u = tg & 31;
+                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32) = make_uint2(0u, 0u);
+                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 8) = make_uint2(0u, 0u);
+                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 16) = make_uint2(0u, 0u);
+                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 24) = make_uint2(0u, 0u);
+            }
+            // the six upper 16x16 blocks of T are zero
+            if (tg < 192) {
+                const int e = tg >> 5, u = tg & 31;
+                const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
+                const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
+                const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
+                *reinterpret_cast<uint4*>(set + PL::TF + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
             }
             tc_fence_before();
             named_sync(1, NG);
-            if (MODE == MODE_STATE && tg == 0) mbar_arrive(&bars[B_AFREE]);   // Y may overwrite A
-            // diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
-            // N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs
-            if (w < 4) {
-                const int b0 = 16 * w, g = lane >> 2, q = lane & 3;
-                const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
-                uint32_t aN[4], bN[4], bP[4], aX[4];
-                ldsm_x4(aN, Ah + cm64(b0 + (lane & 15), b0 + 8 * (lane >> 4)));
-                ldsm_x4_t(bN, Ah + cm64(b0 + (lane & 7) + 8 * ((lane >> 3) & 1), b0 + 8 * (lane >> 4)));
-                float n2a[4] = {0.f, 0.f, 0.f, 0.f}, n2b[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_16x16(n2a, n2b, aN, bN);                                   // N^2
-                c_to_scr(scr, lane, n2a, n2b);
-                __syncwarp();
-                scr_to_b(bP, scr, lane);                                       // bP = N^2
-                __syncwarp();
-                c_to_a(aX, n2a, n2b);
-                float n4a[4] = {0.f, 0.f, 0.f, 0.f}, n4b[4] = {0.f, 0.f, 0.f, 0.f};
-                float n3a[4] = {0.f, 0.f, 0.f, 0.f}, n3b[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_16x16(n4a, n4b, aX, bP);                                   // N^4
-                mma_16x16(n3a, n3b, aN, bP);                                   // N^3
-                c_to_scr(scr, lane, n4a, n4b);
-                __syncwarp();
-                scr_to_b(bP, scr, lane);                                       // bP = N^4
-                __syncwarp();
-                c_to_a(aX, n4a, n4b);
-                float n8a[4] = {0.f, 0.f, 0.f, 0.f}, n8b[4] = {0.f, 0.f, 0.f, 0.f};
-                mma_16x16(n8a, n8b, aX, bP);                                   // N^8
-                // Z = I - N + N^2 - N^3, in the C layout (rows g, g+8; columns 2q, 2q+1 of
-                // each 8-column half); N's values come from its A fragment
-                float za[4], zb[4];
-                {
-                    const float2 n00 = unpack_f16x2(aN[0]), n10 = unpack_f16x2(aN[1]);
-                    const float2 n01 = unpack_f16x2(aN[2]), n11 = unpack_f16x2(aN[3]);
-                    const float d0 = (g == 2 * q) ? 1.f : 0.f, d1 = (g == 2 * q + 1) ? 1.f : 0.f;
-                    za[0] = d0 - n00.x + n2a[0] - n3a[0];
-                    za[1] = d1 - n00.y + n2a[1] - n3a[1];
-                    za[2] = -n10.x + n2a[2] - n3a[2];
-                    za[3] = -n10.y + n2a[3] - n3a[3];
-                    zb[0] = -n01.x + n2b[0] - n3b[0];
-                    zb[1] = -n01.y + n2b[1] - n3b[1];
-                    zb[2] = d0 - n11.x + n2b[2] - n3b[2];
-                    zb[3] = d1 - n11.y + n2b[3] - n3b[3];
-                }
-                {   // Z += Z N^4
-                    float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
-                    c_to_a(aX, za, zb);
-                    mma_16x16(ta, tb, aX, bP);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
-                }
-                c_to_scr(scr, lane, n8a, n8b);
-                __syncwarp();
-                scr_to_b(bP, scr, lane);                                       // bP = N^8
-                {   // Z += Z N^8
-                    float ta[4] = {0.f, 0.f, 0.f, 0.f}, tb[4] = {0.f, 0.f, 0.f, 0.f};
-                    c_to_a(aX, za, zb);
-                    mma_16x16(ta, tb, aX, bP);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) { za[k] += ta[k]; zb[k] += tb[k]; }
-                }
-                st_shared_b32(Tt + cmT(b0 + g, b0) + 4 * q, pack_f16x2(za[0], za[1]));
-                st_shared_b32(Tt + cmT(b0 + g + 8, b0) + 4 * q, pack_f16x2(za[2], za[3]));
-                st_shared_b32(Tt + cmT(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
-                st_shared_b32(Tt + cmT(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
+            invert_unit_lower<T_LBO>(sbase + PL::AT, sset + PL::TF, sbase + PL::MISC + M_XS, w, lane);
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(1, NG);
+            if (tg == 0) {
+                mbar_arrive(&bars[B_INV + s]);   // T ready
+                tc_fence_after();
+                // W^T = (beta K+)^T T^T: M = 128 channels, N = 64 positions, K = 64 positions
+                const uint32_t id = idesc_f16(128, 64, false, false);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 4096 * kk, 2048, 128),
+                             sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
+                umma_commit(&bars[B_W]);
             }
-            named_sync(1, NT / 2);
-            // off-diagonal blocks by halves of the matrix (each warp: one 8-column half of one
-            // 16x16 block; X products through per-warp fp16 scratch):
-            //   level 1: T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)
-            //   level 2: X_IJ = sum_{K=J}^{1} A_IK T_KJ  (I = 2, 3; J = 0, 1), then
-            //            T_IJ = -sum_{K=2}^{I} T_IK X_KJ
-            {
-                const int g = lane >> 2, q = lane & 3, half = w & 1;
-                const uint32_t scr = sbase + PL::MISC + M_XS + 512 * w;
-                auto scr_of = [&](int wx) { return sbase + PL::MISC + M_XS + 512 * wx; };
-                auto put_x = [&](uint32_t dst, const float (&x)[4]) {
-                    st_shared_b32(dst + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
-                    st_shared_b32(dst + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
-                };
-                auto put_t = [&](int I, int N0, const float (&tt)[4]) {
-                    st_shared_b32(Tt + cmT(16 * I + g, N0) + 4 * q, pack_f16x2(-tt[0], -tt[1]));
-                    st_shared_b32(Tt + cmT(16 * I + g + 8, N0) + 4 * q, pack_f16x2(-tt[2], -tt[3]));
-                };
-                auto a_frag = [&](uint32_t (&fr)[4], uint32_t base, int I, int K, bool isT) {
-                    if (isT) ldsm_x4(fr, base + cmT(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
-                    else ldsm_x4(fr, base + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
-                };
-                if (w < 4) {   // level 1
-                    const int I = (w >> 1) ? 3 : 1, J = I - 1, N0 = 16 * J + 8 * half;
-                    uint32_t aA[4], bT[2], bX[2], aT[4];
-                    float x[4] = {0.f, 0.f, 0.f, 0.f}, tt[4] = {0.f, 0.f, 0.f, 0.f};
-                    a_frag(aA, Ah, I, J, false);
-                    ldsm_x2_t(bT, Tt + cmT(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
-                    mma16816(x, aA, bT);
-                    put_x(scr, x);
-                    __syncwarp();
-                    ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
-                    a_frag(aT, Tt, I, I, true);
-                    mma16816(tt, aT, bX);
-                    put_t(I, N0, tt);
-                }
-                named_sync(1, NG);
-                // level 2, X: warp w -> block (I, J) = (2 + (w >> 2), (w >> 1) & 1), half w & 1
-                const int I2 = 2 + (w >> 2), J2 = (w >> 1) & 1, N2 = 16 * J2 + 8 * half;
-                {
-                    float x[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int K = J2; K < 2; ++K) {
-                        uint32_t aA[4], bT[2];
-                        a_frag(aA, Ah, I2, K, false);
-                        ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N2));
-                        mma16816(x, aA, bT);
-                    }
-                    put_x(scr, x);
-                }
-                named_sync(1, NG);
-                // level 2, T: the same (I, J, half); X_KJ half was written by warp 4(K-2) + 2J + half
-                {
-                    float tt[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int K = 2; K <= I2; ++K) {
-                        uint32_t aT[4], bX[2];
-                        a_frag(aT, Tt, I2, K, true);
-                        ldsm_x2_t(bX, scr_of(4 * (K - 2) + 2 * J2 + half) + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
-                        mma16816(tt, aT, bX);
-                    }
-                    put_t(I2, N2, tt);
+            group_wait(&bars[B_W], kc & 1, ab, tg == 0, 1);
+            {   // -W^T -> the KP tile (channel c in lane c, positions 32*hg ..)
+                float v[32];
+                tmem_ld32(tl + TM_APW + 32 * hg, v);
+                const int c = 32 * q4 + lane;
+#pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = -v[8 * g8 + j];
+                    const int i0 = 32 * hg + 8 * g8;
+                    *reinterpret_cast<uint4*>(set + PL::KP + (i0 >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
+                        pack8_f16(f);
                 }
             }
             fence_async_smem();
+            tc_fence_before();
             named_sync(1, NG);
-            if (tg == 0) mbar_arrive(&bars[B_INV + bs]);    // T (and P) ready
+            // every tile of the set is ready (the test hook withholds chunk 0's signal)
+            if (tg == 0 && !(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
         }
-        // after a timeout some requested g tile may not have been waited for: let it land
-        if (tg == 0 && *sAbort && g_issued > 0) mbar_wait_bounded(&bars[B_TG], (g_issued - 1) & 1, kWaitNs);
+        // after a timeout some requested g tiles may not have been waited for: let them land
+        if (tg == 0 && *sAbort)
+            for (int x = max(0, g_issued - 2); x < g_issued; ++x)
+                mbar_wait_bounded(&bars[B_TG + (x & 1)], (x >> 1) & 1, kWaitNs);
     } else {
         // ================= consumer: the state chain of chunk n0 + kc =====================
         const TQ* tq = nullptr;
-        // initial state in TMEM: warp (q4, hg) holds lanes 32*q4.. and columns hg*NS/2 ..
-        {
-            const int col0 = hg * (NS / 2);
-            for (int cc = 0; cc < NS / 2; cc += 32) {
-                float vv[32];
-                if (MODE == MODE_STATE) {
+        const int cw = w - 8, ch = cw >> 2;        // column half of this warp
+        const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
+        const bool mma = tg == 0, loader = tg == 32, poller = tg == 0;
+        // initial state in TMEM: columns 64*ch .. of the master (MODE_STATE: both masters)
+        for (int cc = 0; cc < 64; cc += 32) {
+            const int c0 = 64 * ch + cc;
+            float vv[32];
+            if (MODE == MODE_STATE) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) vv[j] = (col0 + cc + j == D + c) ? 1.f : 0.f;
-                } else if (S_in) {
-                    const size_t idx = s_in_per_segment ? (size_t)slot : (size_t)seq * H + h;
-                    const float4* s4 = reinterpret_cast<const float4*>(S_in + (idx * D + c) * D + col0 + cc);
+                for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+                tmem_st32(tl + TM::MASTER + c0, vv);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 x = s4[j];
-                        vv[4 * j] = x.x; vv[4 * j + 1] = x.y; vv[4 * j + 2] = x.z; vv[4 * j + 3] = x.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) vv[j] = 0.f;
-                }
-                tmem_st32(tl + TM_S + col0 + cc, vv);
-            }
-        }
-        if (gate_fused && tg < D) sGamma[tg] = gamma ? gamma[(size_t)h * D + tg] : 1.f;   // read after later barriers
-        uint32_t betaR = 0;
-        // thread NG + 32 (not the MMA issuer) requests the consumer-side TMA loads, just
-        // before a barrier at which the group waits for an MMA anyway
-        const bool loader = tg == 32;
-        int v_issued = 0, qk_last[2] = {-1, -1}, gate_issued = 0;   // its TMA requests so far
-        bool o_pending = false;                    // poller: a bf16 output store is in flight
-        if (loader && nk > 0) {
-            tma_v(n0);
-            v_issued = 1;
-            tma_qk(n0);
-            qk_last[0] = 0;
-            if (nk > 1) {
-                tma_qk(n0 + 1);
-                qk_last[1] = 1;
-            }
-        }
-        if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0);
-        // the master holds diag(2^{-carry}) S for channel c (log2 units; 0 before any chunk)
-        float carry = 0.f;
-        const bool poller = tg == 0;
-        for (int kc = 0; kc < nk; ++kc) {
-            const int n = n0 + kc, t0 = n * C, bs = kc & 1;
-            const uint32_t sset = sbase + bs * PL::SET;
-            group_wait(&bars[B_PRO + bs], (kc >> 1) & 1, ab, poller, 2);
-            // ---- S^ = 2^{r + carry} master ------------------------------------------------
-            {
-                const float2 rb = sRB[bs * D + c];
-                const float s_scale = ex2_approx(rb.x + carry);
-                carry = rb.y - rb.x;
-                const int col0 = hg * (NS / 2);
-                for (int cc = 0; cc < NS / 2; cc += 32) {
-                    float vv[32];
-                    tmem_ld32(tl + TM_S + col0 + cc, vv);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) vv[j] *= s_scale;
-#pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        const int col = col0 + cc + g8 * 8;
-                        *reinterpret_cast<uint4*>(sm + PL::S + (col >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
-                            pack8_f16(&vv[8 * g8]);
-                    }
-                    tmem_st32(tl + TM_S + col0 + cc, vv);
-                }
-            }
-            if (tg < C) sBetaC[tg] = __uint_as_float(betaR << 16);
-            fence_async_smem();
-            tc_fence_before();
-            named_sync(2, NG);
-            if (poller) {
-                // MODE_STATE: Y's TMEM columns hold A until the producer has read it
-                if (MODE == MODE_STATE) thread_wait(&bars[B_AFREE], kc & 1, ab);
-                tc_fence_after();
-                // OUT:   [Y; O] = [beta K+; Q+] S^   (M = 128, N = 128)
-                // STATE: Y = beta K+ [S^ | Phi^]     (M = 64,  N = 256)
-                const uint32_t idy = idesc_f16(OUT ? 128 : 64, NS, true, true);
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16(tmem + T_Y, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
-                             sdesc(sbase + PL::S + 256 * kk, 128, 2048), idy, kk > 0);
-                umma_commit(&bars[B_Y]);
-            }
-            // ---- beta V while Y runs: v (landed in the beta V tile) converted in place ---------
-            group_wait(&bars[B_TV], kc & 1, ab, poller, 2);
-            {
-                uint32_t vR[16];
-                ld_rows16(vR, sm + PL::VB, 16 * rq, cp);
-                if (t0 + C > Tq) {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= Tq) vR[r] = 0u;
-                }
-                named_sync(2, NG);
-                uint32_t pv[2][4];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float2 lv = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int r8 = 0; r8 < 8; ++r8) {
-                        const int r = 8 * half + r8;
-                        const float bi = sBetaC[16 * rq + r];
-                        const float2 vb = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
-                        if (r8 & 1) {
-                            pv[0][r8 >> 1] = pack_f16x2(lv.x, vb.x);
-                            pv[1][r8 >> 1] = pack_f16x2(lv.y, vb.y);
-                        } else {
-                            lv = vb;
-                        }
-                    }
-                    st_pair(sm + PL::VB, 2 * rq + half, cp, pv);
-                }
-            }
-            if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
-            if (OUT) {
-                // U = T (beta V) - T Y: the first half needs no Y, so it queues behind [Y; O]
-                fence_async_smem();
-                named_sync(2, NG);
-                if (poller) {
-                    thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
-                    tc_fence_after();
-                    const uint32_t idv = idesc_f16(64, 128, false, false);
-                    const uint32_t Tb = sset + PL::TF;
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
-                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, kk > 0);
-                }
-            }
-            group_wait(&bars[B_Y], kc & 1, ab, poller, 2);
-            // ---- Y -> fp16 position-major tile in the S^ region --------------------------
-            if (OUT) {
-                if (q4 < 2) {
-                    const int j = 32 * q4 + lane;    // M = 128 layout: row j in lane j
-                    for (int cc = 0; cc < 64; cc += 32) {
-                        float vv[32];
-                        tmem_ld32(tl + T_Y + 64 * hg + cc, vv);
-#pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8) {
-                            const int cg = (64 * hg + cc) / 8 + g8;
-                            *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
-                                pack8_f16(&vv[8 * g8]);
-                        }
-                    }
-                }
+                for (int e = 0; e < 32; ++e) vv[e] = (c0 + e == j) ? 1.f : 0.f;
+                tmem_st32(tl + TM::MASTER + D + c0, vv);
             } else {
-                const int j = 16 * q4 + lane;        // M = 64 layout: lanes 0-15 of each quarter
-                for (int cc = 0; cc < 128; cc += 32) {
-                    float vv[32];
-                    tmem_ld32(tl + T_Y + 128 * hg + cc, vv);
-                    if (lane < 16) {
+                if (S_in) {
+                    const size_t idx = s_in_per_segment ? (size_t)slot : (size_t)seq * H + h;
+                    const float* src = S_in + idx * D * D + j;
 #pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8) {
-                            const int cg = (128 * hg + cc) / 8 + g8;
-                            *reinterpret_cast<uint4*>(sm + PL::S + (j >> 3) * YJ + cg * 128 + (j & 7) * 16) =
-                                pack8_f16(&vv[8 * g8]);
+                    for (int e = 0; e < 32; ++e) vv[e] = src[(size_t)(c0 + e) * D];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+                }
+                tmem_st32(tl + TM::MASTER + c0, vv);
+            }
+        }
+        int v_issued = 0, qk_last[2] = {-1, -1};   // loader: TMA requests so far
+        if (loader && nk > 0) {
+            for (int x = 0; x < min(2, nk); ++x) {
+                tma_v(n0 + x);
+                tma_qk(n0 + x);
+                qk_last[x] = x;
+            }
+            v_issued = min(2, nk);
+        }
+        float gam = 1.f;
+        if (OUT && gate && gamma) gam = gamma[(size_t)h * D + j];
+        // beta of chunks n0 and n0 + 1 -> their beta V slots
+        if (tg < C) {
+            sBetaV[tg] = __uint_as_float(load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0) << 16);
+            sBetaV[C + tg] = __uint_as_float(load_beta(beta, rowbase, Tq, H, h, (n0 + 1) * C, tg, nk > 1) << 16);
+        }
+        tc_fence_before();
+        // beta V of chunk x in place (v landed in beta V tile x & 1): thread = channel pair x
+        // 16 rows; every raw row is read before any tile is rewritten
+        auto beta_v = [&](int x) {
+            const int vb = x & 1, t0x = (n0 + x) * C;
+            group_wait(&bars[B_TV + vb], (x >> 1) & 1, ab, poller, 2);
+            uint32_t vR[16];
+            uint8_t* tile = sm + PL::VB + vb * 16384;
+            ld_rows16(vR, tile, 16 * rq, cp);
+            if (t0x + C > Tq) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    if (t0x + 16 * rq + r >= Tq) vR[r] = 0u;
+            }
+            named_sync(2, NG);
+            uint32_t pv[2][4];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float2 lv = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int r8 = 0; r8 < 8; ++r8) {
+                    const int r = 8 * half + r8;
+                    const float bi = sBetaV[vb * C + 16 * rq + r];
+                    const float2 vbv = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
+                    if (r8 & 1) {
+                        pv[0][r8 >> 1] = pack_f16x2(lv.x, vbv.x);
+                        pv[1][r8 >> 1] = pack_f16x2(lv.y, vbv.y);
+                    } else {
+                        lv = vbv;
+                    }
+                }
+                st_pair(tile, 2 * rq + half, cp, pv);
+            }
+            fence_async_smem();
+        };
+        if (nk > 0) beta_v(0);
+        tc_fence_before();
+        named_sync(2, NG);   // initial master and the first beta V are in place
+        tc_fence_after();
+        // U~^T = (beta V)^T T^T into the chunk's U columns (MODE_OUTPUT: [U~^T | 0] over
+        // the [U | O] buffer, so O starts from zero)
+        auto issue_u = [&](int x) {
+            const int s = x & 1;
+            const uint32_t sset = sbase + s * PL::SET, vbt = sbase + PL::VB + s * 16384;
+            if (OUT) {
+                const uint32_t id = idesc_f16(128, 128, false, false);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + TM::UO + 128 * s, sdesc(vbt + 4096 * kk, 2048, 128),
+                             sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
+            } else {
+                const uint32_t id = idesc_f16(128, 64, false, false);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16(tmem + TM::UACC, sdesc(vbt + 4096 * kk, 2048, 128),
+                             sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
+            }
+            umma_commit(&bars[B_VE + s]);   // the beta V tile may be refilled
+        };
+        // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
+        auto out_rows = [&](int x) {
+            const int b = x & 1, t0x = (n0 + x) * C;
+            group_wait(&bars[B_O + b], (x >> 1) & 1, ab, poller, 2);
+            float v[32];
+            tmem_ld32(tl + Tm<MODE_OUTPUT>::UO + 128 * b + 64 + 32 * ch, v);
+            const int nv = min(C, Tq - t0x);
+            if (gate) {
+                // Eq. 15 output side: y = Sigmoid(gate) * gamma * RMSNorm over the head's values.
+                // Per position, the sum of squares over this warp's 32 values by a transposing
+                // butterfly (lane l ends with position 32*ch + l), then over the 4 lane quarters.
+                float sq[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) sq[u] = v[u] * v[u];
+#pragma unroll
+                for (int sft = 16; sft >= 1; sft >>= 1) {
+                    const bool up = (lane & sft) != 0;
+#pragma unroll
+                    for (int k = 0; k < sft; ++k) {
+                        const float send = up ? sq[k] : sq[k + sft];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
+                        sq[k] = (up ? sq[k + sft] : sq[k]) + recv;
+                    }
+                }
+                float* red = reinterpret_cast<float*>(sm + PL::MISC + M_RED);
+                red[q4 * C + 32 * ch + lane] = sq[0];
+                named_sync(2, NG);
+                const int pi = 32 * ch + lane;
+                const float m = (red[pi] + red[C + pi] + red[2 * C + pi] + red[3 * C + pi]) * (1.f / D) + eps;
+                const float inv = m > 0.f ? rsqrtf(m) : 0.f;
+                named_sync(2, NG);   // red may be reused
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const float iu = __shfl_sync(0xffffffffu, inv, u);
+                    const int i = 32 * ch + u;
+                    float gv = 0.f;
+                    if (i < nv) gv = __bfloat162float(gate[(((size_t)rowbase + t0x + i) * H + h) * D + j]);
+                    v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int i = 32 * ch + u;
+                if (i < nv) {
+                    const size_t idx = (((size_t)rowbase + t0x + i) * H + h) * D + j;
+                    if (o_f32) reinterpret_cast<float*>(o)[idx] = v[u];
+                    else reinterpret_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(v[u]);
+                }
+            }
+        };
+        bool u_done = false;   // U~ of chunk kc already issued
+        for (int kc = 0; kc < nk; ++kc) {
+            const int n = n0 + kc, s = kc & 1;
+            const uint32_t sset = sbase + s * PL::SET;
+            // beta of chunk kc+2, loaded now and stored once its slot is free
+            const uint32_t betaN = tg < C ? load_beta(beta, rowbase, Tq, H, h, (n + 2) * C, tg, n + 2 < n1) : 0u;
+            if (mma && !u_done) {
+                thread_wait(&bars[B_INV + s], (kc >> 1) & 1, ab);
+                tc_fence_after();
+                issue_u(kc);
+            }
+            // ---- S^ = fp16(2^{rp + carry} master), master <- 2^{rm + carry} master --------
+            if (poller) {
+                thread_wait(&bars[B_SC + s], (kc >> 1) & 1, ab);
+                if (kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
+            }
+            named_sync(2, NG);
+            tc_fence_after();
+            {
+                const float* sY = sSC + s * 3 * D;
+                const float* sMs = sY + D;
+                for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
+                    const uint32_t mcol = TM::MASTER + D * mi, hcol = TM::S16 + 64 * mi;
+                    for (int cc = 0; cc < 64; cc += 32) {
+                        const int c0 = 64 * ch + cc;
+                        float vv[32];
+                        uint32_t hv[16];
+                        tmem_ld32(tl + mcol + c0, vv);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 y4 = *reinterpret_cast<const float4*>(sY + c0 + e);
+                            const float4 m4 = *reinterpret_cast<const float4*>(sMs + c0 + e);
+                            hv[e / 2] = pack_f16x2(vv[e] * y4.x, vv[e + 1] * y4.y);
+                            hv[e / 2 + 1] = pack_f16x2(vv[e + 2] * y4.z, vv[e + 3] * y4.w);
+                            vv[e] *= m4.x; vv[e + 1] *= m4.y; vv[e + 2] *= m4.z; vv[e + 3] *= m4.w;
                         }
+                        tmem_st16u(tl + hcol + c0 / 2, hv);
+                        tmem_st32(tl + mcol + c0, vv);
                     }
                 }
             }
-            fence_async_smem();
             tc_fence_before();
             named_sync(2, NG);
-            // ---- U = T (beta V) - T Y  (value columns; identity columns: -T Y) -------------
-            if (poller) {
-                if (!OUT) thread_wait(&bars[B_INV + bs], (kc >> 1) & 1, ab);   // T of this chunk
+            if (mma) {
+                thread_wait(&bars[B_PRO + s], (kc >> 1) & 1, ab);
                 tc_fence_after();
-                const uint32_t idv = idesc_f16(64, 128, false, false);
-                const uint32_t idy = idesc_f16(64, NS, false, true, true);
-                const uint32_t Tb = sset + PL::TF;
                 if (OUT) {
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
-                                 sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, 1);
+                    // [U | O]^T += S^T [-W^T | Q+^T]   (N = 128: positions of W, then of Q+)
+                    const uint32_t id = idesc_f16(128, 128, false, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ts(tmem + TM::UO + 128 * s, tmem + TM::S16 + 8 * kk,
+                                    sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
                 } else {
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
-                                 sdesc(sbase + PL::S + 2 * YJ * kk, YJ, 128), idy, kk > 0);
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_UU, sdesc(Tb + 2 * T_LBO * kk, T_LBO, 128),
-                                 sdesc(sbase + PL::VB + 4096 * kk, 2048, 128), idv, 1);
+                    const uint32_t id = idesc_f16(128, 64, false, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 8 * kk,
+                                    sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
                 }
                 umma_commit(&bars[B_U]);
             }
-            // [Y; O] of this chunk is done: chunk n+2's q, k may land in this set's
-            // Q+ / beta K+ slots (and this chunk's gate in the upper half of S^)
-            if (loader && n + 2 < n1 && !*sAbort) {
-                tma_qk(n + 2);
-                qk_last[bs] = kc + 2;
-            }
-            if (gate_fused && loader && !*sAbort) {
-                tma_gate(n);
-                gate_issued = kc + 1;
-            }
-            // the output store must have read the U region before U is written there
-            if (poller && o_pending) {
-                bulk_wait_read0();
-                o_pending = false;
-            }
+            // ---- meanwhile: chunk kc-1's output rows and chunk kc+1's beta V ----------------
+            if (OUT && kc > 0) out_rows(kc - 1);
+            if (kc + 1 < nk) beta_v(kc + 1);
+            if (tg < C && kc + 2 < nk)   // chunk kc's beta V slot is free (chunk kc+2 uses it)
+                sBetaV[s * C + tg] = __uint_as_float(betaN << 16);
             group_wait(&bars[B_U], kc & 1, ab, poller, 2);
-            // U -> fp16 MN-major tile [i][col] at U (M = 64 layout: row 16*q4 + l in lane 32*q4 + l)
-            for (int cc = 0; cc < NS / 2; cc += 32) {
-                const int col = hg * (NS / 2) + cc;
-                float vv[32];
-                tmem_ld32(tl + T_UU + col, vv);
-                if (lane < 16) {
-                    const int i = 16 * q4 + lane;
-#pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
-                        const int cg = col / 8 + g8;
-                        *reinterpret_cast<uint4*>(sm + PL::U + cg * 1024 + (i >> 3) * 128 + (i & 7) * 16) =
-                            pack8_f16(&vv[8 * g8]);
+            if (loader && !*sAbort) {
+                // the [U | O] MMA has read -W^T and Q+ (MODE_OUTPUT): chunk kc+2's k and q may land
+                if (OUT && n + 2 < n1) {
+                    tma_qk(n + 2);
+                    qk_last[s] = kc + 2;
+                }
+                // U~ of chunk kc has read its beta V tile: chunk kc+2's v may land
+                if (n + 2 < n1) {
+                    thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
+                    if (!*sAbort) {
+                        tma_v(n + 2);
+                        v_issued = kc + 3;
                     }
                 }
             }
-            fence_async_smem();
+            // ---- U -> fp16 (A operand of the master and O updates) ---------------------------
+            {
+                const uint32_t ucol0 = OUT ? TM::UO + 128 * s : TM::UACC;
+                const uint32_t dst = OUT ? ucol0 : TM::S16;   // MODE_STATE: into S^'s columns
+                float vv[32];
+                uint32_t hv[16];
+                tmem_ld32(tl + ucol0 + 32 * ch, vv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
+                tmem_st16u(tl + dst + 32 * ch, hv);
+            }
             tc_fence_before();
             named_sync(2, NG);
-            // ---- master += K-^T U  (and O += P U) ------------------------------------------
-            if (poller) {
-                if (MODE == MODE_STATE) mbar_arrive(&bars[B_UREAD]);   // A may take U's columns
+            if (mma) {
                 tc_fence_after();
-                const uint32_t ids = idesc_f16(128, NS, false, true);
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TM_S, sdesc(sset + PL::KM + 4096 * kk, 2048, 128),
-                             sdesc(sbase + PL::U + 256 * kk, 128, 1024), ids, 1);
+                const uint32_t idm = idesc_f16(128, 128, false, false);
                 if (OUT) {
-                    // O += P U as rows 64-127 of an M = 128 MMA whose rows 0-63 read T (their
-                    // result lands on Y's rows, already consumed)
-                    const uint32_t ido = idesc_f16(128, 128, false, true);
+                    // master += U^T K-   and   O^T += U^T P^T
+                    const uint32_t ua = tmem + TM::UO + 128 * s;
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16(tmem + T_Y, sdesc(sset + PL::TF + 4096 * kk, 2048, 128),
-                                 sdesc(sbase + PL::U + 256 * kk, 128, 1024), ido, 1);
-                }
-                umma_commit(&bars[B_S]);
-                umma_commit(&bars[B_EMPTY + bs]);   // buffer set bs may be refilled
-            }
-            // the U MMA has read beta V: chunk n+1's v may land in its tile
-            if (loader && n + 1 < n1 && !*sAbort) {
-                tma_v(n + 1);
-                v_issued = kc + 2;
-            }
-            group_wait(&bars[B_S], kc & 1, ab, poller, 2);
-            // ---- this chunk's output, staged in the free U (and Y) regions; done here, at
-            // the end of the chunk, it overlaps the wait for the producer's next tiles -----
-            if (OUT) {
-                if (o_f32 || (items && t0 + C > Tq)) {
-                    stage_o(tl, q4, hg, lane, sm + PL::U, o_f32);
-                    named_sync(2, NG);
-                    flush_o(sm + PL::U, tg, o, o_f32, rowbase, Tq, H, h, t0);
-                    named_sync(2, NG);
+                        umma_f16_ts(tmem + TM::MASTER, ua + ucol(kk), sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
+                    umma_commit(&bars[B_S]);
+                    const uint32_t ido = idesc_f16(128, 64, false, false);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ts(ua + 64, ua + ucol(kk), sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
+                    umma_commit(&bars[B_O + s]);
                 } else {
-                    if (gate_fused) {
-                        group_wait(&bars[B_TGATE], kc & 1, ab, poller, 2);
-                        stage_o_gated(tl, q4, hg, lane, sm + PL::U, sm + PL::S + 16384,
-                                      reinterpret_cast<float*>(sm + PL::S), sGamma, eps);
-                    } else {
-                        stage_o_swz(tl, q4, hg, lane, sm + PL::U);
-                    }
-                    fence_async_smem();
-                    named_sync(2, NG);
-                    if (poller) {
-                        tma_store_4d(&tm_o, sm + PL::U, 0, h, (int)(o_t + t0), o_b);
-                        tma_store_4d(&tm_o, sm + PL::U + 8192, 64, h, (int)(o_t + t0), o_b);
-                        bulk_commit();
-                        o_pending = true;
-                    }
+                    // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + ucol(kk),
+                                    sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
+                    const uint32_t id = idesc_f16(128, 64, false, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 64 + 8 * kk,
+                                    sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, kk > 0);
+                    umma_commit(&bars[B_U2]);
+                }
+            }
+            if (!OUT) {
+                group_wait(&bars[B_U2], kc & 1, ab, poller, 2);
+                // -W^T has been read twice: chunk kc+2's k may land
+                if (loader && !*sAbort && n + 2 < n1) {
+                    tma_qk(n + 2);
+                    qk_last[s] = kc + 2;
+                }
+                {
+                    float vv[32];
+                    uint32_t hv[16];
+                    tmem_ld32(tl + TM::UACC + 32 * ch, vv);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
+                    tmem_st16u(tl + TM::S16 + 64 + 32 * ch, hv);
+                }
+                tc_fence_before();
+                named_sync(2, NG);
+                if (mma) {
+                    tc_fence_after();
+                    const uint32_t idm = idesc_f16(128, 128, false, false);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ts(tmem + TM::MASTER + D, tmem + TM::S16 + 64 + ucol(kk),
+                                    sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
+                    umma_commit(&bars[B_S]);
+                }
+            }
+            if (mma) {
+                umma_commit(&bars[B_EMPTY + s]);   // set s may be refilled
+                // U~ of the next chunk now, if its T is ready (else at the top of the next step)
+                u_done = false;
+                if (kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_u(kc + 1);
+                    u_done = true;
                 }
             }
         }
-        if (poller) bulk_wait0();   // every output store has landed before the CTA exits
+        if (OUT && nk > 0) out_rows(nk - 1);
         // after a timeout some requested tiles may not have been waited for: let them land
         if (loader && *sAbort) {
-            if (gate_issued > 0) mbar_wait_bounded(&bars[B_TGATE], (gate_issued - 1) & 1, kWaitNs);
-            if (v_issued > 0) mbar_wait_bounded(&bars[B_TV], (v_issued - 1) & 1, kWaitNs);
+            for (int x = max(0, v_issued - 2); x < v_issued; ++x)
+                mbar_wait_bounded(&bars[B_TV + (x & 1)], (x >> 1) & 1, kWaitNs);
             for (int s2 = 0; s2 < 2; ++s2)
                 if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
         }
-        // ---- end of segment: write the state S = diag(2^{carry}) master -----------------
+        // ---- end of segment: the state S = diag(2^{carry}) master (columns = channels) -----
+        if (nk > 0) group_wait(&bars[B_S], (nk - 1) & 1, ab, poller, 2);
         float* dst = nullptr;
         if (MODE == MODE_STATE) dst = maps + (size_t)slot * 2 * D * D;  // [N | M]
         else if (S_T && last) dst = S_T + ((size_t)seq * H + h) * D * D;
         if (dst && !*sAbort) {
-            const float sc = ex2_approx(carry);
-            const int col0 = hg * (NS / 2);
-            for (int cc = 0; cc < NS / 2; cc += 32) {
-                float vv[32];
-                tmem_ld32(tl + TM_S + col0 + cc, vv);
-                // maps: N block (value columns) then M block (identity columns); a 32-column
-                // run never straddles the two
-                const int col = col0 + cc;
-                const size_t idx = (col < D) ? ((size_t)c * D + col) : ((size_t)D * D + (size_t)c * D + (col - D));
-                float4* d4 = reinterpret_cast<float4*>(dst + idx);
+            const float* cn = nk > 0 ? sSC + ((nk - 1) & 1) * 3 * D + 2 * D : nullptr;
+            for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
+                for (int cc = 0; cc < 64; cc += 32) {
+                    const int c0 = 64 * ch + cc;
+                    float vv[32];
+                    tmem_ld32(tl + TM::MASTER + D * mi + c0, vv);
+                    float* d = dst + (size_t)mi * D * D + j;
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    d4[j] = make_float4(vv[4 * j] * sc, vv[4 * j + 1] * sc, vv[4 * j + 2] * sc, vv[4 * j + 3] * sc);
+                    for (int e = 0; e < 32; ++e) d[(size_t)(c0 + e) * D] = vv[e] * (cn ? ex2_approx(cn[c0 + e]) : 1.f);
+                }
             }
         }
     }
@@ -1231,40 +1292,8 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 output o [B, T, H, 128] as a 4-D tensor (channels, heads, tokens, batch), box =
-// 64 channels x 1 head x 64 tokens, 128-byte swizzle.  Tokens past T are clipped by the
-// T dimension, so a ragged last chunk never writes into the next batch row.
-bool make_map_o(CUtensorMap* m, void* base, int B, int T, int H)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)C, 1u};
-    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Gate [B*T, H, 128] bf16 as two 64-channel halves per chunk (box 64 x 1 x 64), 128-byte
-// swizzle: lands in the layout of the swizzled output tiles.
-bool make_map_gate(CUtensorMap* m, const void* base, int B, int T, int H)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)T};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    const cuuint32_t box[3] = {64u, 1u, (cuuint32_t)C};
-    const cuuint32_t es[3] = {1u, 1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 struct Maps {
-    CUtensorMap q, k, v, g, o;   // o: only for a bf16 output (else a copy of q, unused)
-    CUtensorMap gate;            // only for the fused gated epilogue (else a copy of q)
+    CUtensorMap q, k, v, g;
 };
 
 struct Split {
@@ -1294,9 +1323,9 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     if (grid == 0) return cudaSuccess;
     ProfileScope prof(prof_name ? prof_name : (MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output"), s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, mp.gate, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
-                                a.gamma, a.eps, a.gate != nullptr ? 1 : 0, items);
+                                (const __nv_bfloat16*)a.gate, a.gamma, a.eps, items);
     return cudaGetLastError();
 }
 
@@ -1305,15 +1334,9 @@ bool build_maps(const KdaArgs& a, Maps& mp)
 {
     const CUtensorMapDataType dq =
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
-        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
-        !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
-        return false;
-    if (a.out_t == ET_F32 || !a.o) mp.o = mp.q;
-    else if (!make_map_o(&mp.o, a.o, a.B, a.T, a.H)) return false;
-    if (a.gate && a.out_t == ET_BF16) return make_map_gate(&mp.gate, a.gate, a.B, a.T, a.H);
-    mp.gate = mp.q;
-    return true;
+    return make_map(&mp.q, a.q, dq, a.B, a.T, a.H) && make_map(&mp.k, a.k, dq, a.B, a.T, a.H) &&
+           make_map(&mp.v, a.v, dq, a.B, a.T, a.H) &&
+           make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H);
 }
 
 int sm_count()
@@ -1403,9 +1426,7 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
     const Split sp = split_for(a.B, a.T, a.H, sm_count());
     Maps mp;
     if (!build_maps<TQ>(a, mp)) return cudaErrorInvalidValue;
-    // the gated epilogue needs whole-chunk TMA stores, which the item tables' ragged
-    // sequence ends do not give: it keeps the one-table split
-    if (wv.P == 1 || a.gate) {
+    if (wv.P == 1) {
         float* maps = reinterpret_cast<float*>(ws);
         float* starts = maps + (size_t)a.B * a.H * (sp.P - 1) * 2 * D * D;
         if (sp.P > 1) {
@@ -1415,8 +1436,6 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
     }
     const int P = wv.P, L = wv.L, BH = a.B * a.H;
-    // item tables address packed rows: the bf16 output map spans all B*T rows as one
-    if (a.out_t == ET_BF16 && !make_map_o(&mp.o, a.o, 1, a.B * a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     float* starts = reinterpret_cast<float*>(base + wv.maps_b);
@@ -1609,9 +1628,6 @@ cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int*
     if (!make_map(&mp.q, a.q, dq, 1, a.T, a.H) || !make_map(&mp.k, a.k, dq, 1, a.T, a.H) ||
         !make_map(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
         return cudaErrorInvalidValue;
-    if (a.out_t == ET_F32) mp.o = mp.q;
-    else if (!make_map_o(&mp.o, a.o, 1, a.T, a.H)) return cudaErrorInvalidValue;
-    mp.gate = mp.q;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     base += a256(pl.n_maps * 2 * D * D * sizeof(float));
@@ -1662,8 +1678,8 @@ bool kda_tc_supported(const KdaArgs& a)
     if (a.in_t != ET_BF16 && a.in_t != ET_F16) return false;
     if (a.gb_t != ET_BF16) return false;
     if (a.out_t != ET_BF16 && a.out_t != ET_F32) return false;
-    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.g) || !aligned16(a.o)) return false;
-    if (a.gate && (a.in_t != ET_BF16 || !aligned16(a.gate) || (a.gamma && !aligned16(a.gamma)))) return false;
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.g)) return false;
+    if (a.gate && a.in_t != ET_BF16) return false;
     return encode_fn() != nullptr;
 }
 
@@ -1717,14 +1733,8 @@ cudaError_t launch_kda_tc_sp_output(const KdaArgs& a, void* ws, int* status, cud
 cudaError_t launch_kda_tc(const KdaArgs& a, void* ws, size_t ws_bytes, int* status, cudaStream_t s)
 {
     (void)ws_bytes;
-    // the gated epilogue is fused into the output stage for a bf16 output; an fp32 output
-    // gets the plain scan followed by the separate epilogue kernel
-    KdaArgs scan = a;
-    if (a.gate && a.out_t == ET_F32) scan.gate = nullptr;
-    const cudaError_t e = a.in_t == ET_F16 ? launch_all<__half>(scan, ws, status, s)
-                                           : launch_all<__nv_bfloat16>(scan, ws, status, s);
-    if (e != cudaSuccess || !a.gate || a.out_t != ET_F32) return e;
-    return launch_gate_rmsnorm(a, s);
+    // the output side of Eq. 15 (a.gate) is applied in the output pass's store stage
+    return a.in_t == ET_F16 ? launch_all<__half>(a, ws, status, s) : launch_all<__nv_bfloat16>(a, ws, status, s);
 }
 
 }  // namespace kda
