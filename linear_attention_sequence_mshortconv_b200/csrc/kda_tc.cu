@@ -74,7 +74,9 @@ using namespace sm100;
 constexpr int C = 64;         // chunk length
 constexpr int D = 128;        // Dk = Dv
 constexpr int NT = 512;       // threads per CTA
-constexpr int NG = 256;       // threads per warp group
+constexpr int NR = 128;       // threads per role (4 warps)
+// named barriers: one per role, plus the per-row-half barriers of the in-place conversions
+enum { BAR_P = 1, BAR_I = 2, BAR_X = 3, BAR_Y = 4, BAR_P2 = 5 /* 5, 6 */, BAR_Y2 = 7 /* 7, 8 */ };
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on every wait
 constexpr float kLog2e = 1.4426950408889634f;
 // Largest log2 decay factor a middle-row reference may produce in an operand tile: with
@@ -87,55 +89,61 @@ enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 // Per buffer set (chunk parity): KP (k -> beta K+ -> -W^T) and QP (q -> Q+) as
 // channel-major tiles, QP directly after KP so [beta K+; Q+] and [-W^T | Q+^T] are single
 // 128-row operands; KM (K-); PF (P as the K-major B operand of O^T += U^T P^T); TF (T as
-// the K-major B operand T^T of W^T and U~^T; in MODE_OUTPUT interleaved with a zero
-// block, so U~ fills [U~^T | 0] with one N = 128 MMA).
+// the K-major B operand T^T of W^T and U~^T).
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
-    static constexpr int SET = 73728;
+    static constexpr int SET = 65536;
     static constexpr int KP = 0, QP = 16384, KM = 32768, PF = 49152, TF = 57344;
-    static constexpr int T_LBO = 2048;             // T's stride between 8-column groups
-    static constexpr int VB = 147456;              // two beta V tiles (channel-major, values)
-    static constexpr int AT = 180224;              // A, fp16, for the inverse (producer)
-    static constexpr int GS = 188416;              // two g staging tiles ([64][128] bf16, TMA)
+    static constexpr int T_LBO = 1024, T_BYTES = 8192;
+    static constexpr int VB = 131072;              // two beta V tiles (channel-major, values)
+    static constexpr int AT = 163840;              // A, fp16, for the inverse
+    static constexpr int GS = 172032;              // two g staging tiles ([64][128] bf16, TMA)
+    static constexpr int OS = 204800;              // output staging (two swizzled 64 x 64 bf16 tiles)
+    static constexpr int SCR = 0;                  // (chunk_ap_direct uses the set's KM, PF, TF)
     static constexpr int MISC = 221184;
     static constexpr int QK_BYTES = 2 * 16384;     // q and k of one chunk
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int SET = 40960;
     static constexpr int KP = 0, QP = -1, KM = 16384, PF = 0, TF = 32768;   // no q, no P
-    static constexpr int T_LBO = 1024;
+    static constexpr int T_LBO = 1024, T_BYTES = 8192;
     static constexpr int VB = 81920;
     static constexpr int AT = 114688;
     static constexpr int GS = 122880;
     static constexpr int SCR = 155648;             // 32 KB scratch of chunk_ap_direct
+    static constexpr int OS = 0;                   // (no output)
     static constexpr int MISC = 188416;
     static constexpr int QK_BYTES = 16384;         // k of one chunk
 };
 // MISC sub-layout
-constexpr int M_BETAP = 0;       // float[64]     beta of the producer's chunk
-constexpr int M_BETAV = 256;     // float[2][64]  beta of the chunk in each beta V tile
-constexpr int M_TOT = 768;       // float[4][128] per-16-row sums of g log2(e)
-constexpr int M_SC = 2816;       // float[2][3][128] per set: S^ scale, master scale, carry after
-constexpr int M_XS = 5888;       // 8 x 512 B per-warp 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 9984;      // mbarriers, see Bar
-constexpr int M_TMEM = 10184;    // uint32 TMEM base
-constexpr int M_ABORT = 10188;   // int
-constexpr int M_RED = 10192;     // float[4][64] per-row sums of squares (gated output)
-constexpr int MISC_BYTES = 11216;
+constexpr int M_BETA = 0;        // bf16[4][64]   beta of chunk x in slot x & 3 (written two chunks ahead)
+constexpr int M_BRAW = 512;      // uint32[64]    the head pair's beta words as cp.async lands them
+constexpr int M_TOT = 768;       // float[2][128] per-32-row sums of g log2(e)
+constexpr int M_SC = 1792;       // float[2][3][128] per set: S^ scale, master scale, carry after
+constexpr int M_XS = 4864;       // 8 x 512 B per-item 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 8960;      // mbarriers, see Bar
+constexpr int M_TMEM = 9184;     // uint32 TMEM base
+constexpr int M_ABORT = 9188;    // int
+constexpr int M_DIRECT = 9192;   // int[2] per set: its chunk's A and P came from chunk_ap_direct
+constexpr int M_RED = 9200;      // float[4][64] per-row sums of squares (gated output)
+constexpr int MISC_BYTES = 10224;
 enum Bar {
     B_TG = 0,       // [2] g tile landed (staging tile x)
     B_TQK = 2,      // [2] k (and q) landed in set s
     B_TV = 4,       // [2] v landed in beta V tile x
-    B_SC = 6,       // [2] set s: scales of its chunk written
+    B_SC = 6,       // [2] set s: prologue done (scales, direct flag, K+ / Q+ / K- tiles, beta)
     B_INV = 8,      // [2] set s: T ready
-    B_PRO = 10,     // [2] set s: every tile ready
-    B_EMPTY = 12,   // [2] set s: the consumer's last MMA on it is done
+    B_PRO = 10,     // [2] set s: every tile ready (-W^T written)
+    B_EMPTY = 12,   // [2] set s: the chain's last MMA on it is done
     B_VE = 14,      // [2] beta V tile x: the U~ MMA that read it is done
     B_O = 16,       // [2] [U | O] buffer x: the chunk's O is complete
-    B_AP = 18, B_W = 19, B_U = 20, B_U2 = 21, B_S = 22, B_DRAIN = 23, B_DRAIN2 = 24,
-    NBAR = 25
+    B_AP = 18, B_W = 19, B_U = 20, B_U2 = 21, B_S = 22,
+    B_APWF = 23,    // the inverse role has read W^T out of A|P's TMEM columns
+    B_DRAIN = 24,   // [4] one per MMA-issuing role, after a timeout
+    NBAR = 28
 };
 static_assert(M_BAR + NBAR * 8 <= M_TMEM, "barrier block");
+static_assert(M_RED % 16 == 0 && M_RED + 1024 <= MISC_BYTES, "misc block");
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
 static_assert(smem_bytes<MODE_OUTPUT>() <= 232448, "shared memory");
@@ -149,11 +157,6 @@ template <int MODE> struct Tm;
 // (UO / UACC name the same region for the mode that has no such buffer; never used there)
 template <> struct Tm<MODE_OUTPUT> { static constexpr uint32_t MASTER = 0, S16 = 128, UO = 192, UACC = 192; };
 template <> struct Tm<MODE_STATE> { static constexpr uint32_t MASTER = 0, S16 = 256, UACC = 384, UO = 384; };
-
-// Column of K step kk (16 positions) of the fp16 U^T operand inside a 64-column fp32 U
-// region: each column half of the consumer packs its 32 positions into the first 16
-// columns of the 32 it read, so no thread writes a column another thread still reads.
-__device__ __forceinline__ uint32_t ucol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
 // ---- helpers ------------------------------------------------------------------------
 __device__ __forceinline__ uint4 pack8_f16(const float* f)
@@ -219,14 +222,14 @@ struct Abort {
     int* flag;
     int* status;
 };
-// One thread polls; the group (bar_id, NG threads) waits at its named barrier.
+// One thread polls; the role (bar_id, NR threads) waits at its named barrier.
 __device__ __forceinline__ void group_wait(uint64_t* bar, uint32_t parity, const Abort& a, bool poller, int bar_id)
 {
     if (poller && !*a.flag && !mbar_wait_bounded(bar, parity, kWaitNs)) {
         *a.flag = 1;
         atomicCAS(a.status, DEV_OK, DEV_TIMEOUT);
     }
-    named_sync(bar_id, NG);
+    named_sync(bar_id, NR);
     tc_fence_after();
 }
 // One thread waits alone (before issuing MMAs that depend on the other group).
@@ -253,6 +256,20 @@ __device__ __forceinline__ uint32_t load_beta(const __nv_bfloat16* beta, int64_t
     return (live && tt < T) ? (uint32_t) * reinterpret_cast<const unsigned short*>(beta + ((size_t)rowbase + tt) * H + h)
                             : 0u;
 }
+// 4 bytes global -> shared by cp.async (valid = false: zero-filled, nothing is read)
+__device__ __forceinline__ void cp_async4_zfill(void* smem, const void* gmem, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(smem)), "l"(gmem), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+// beta of token t0 + i as raw bf16 bits (0 past the sequence end)
+__device__ __forceinline__ uint16_t beta_bits(const __nv_bfloat16* beta, int64_t rowbase, int T, int H, int h, int t0,
+                                              int i, bool live)
+{
+    return (uint16_t)load_beta(beta, rowbase, T, H, h, t0, i, live);
+}
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
 // Store two channels' packed fp16 rows (one 16-byte vector per channel) into a
 // channel-major tile.  Threads with (cp & 4) store their odd channel first: each
 // 8-thread phase of a 16-byte store then covers all 32 banks once.
@@ -271,92 +288,107 @@ __device__ __forceinline__ void st_pair(uint8_t* tile, int ig, int cp, const uin
 // sum_c q_ic k_jc 2^{b_ic - b_jc} (j <= i), every exponential <= 1 formed directly.  The
 // raw k (and q) tiles are still in KP (QP); `scr` holds the fp32 table b[64][128] (base
 // 2, from the chunk start), written by the caller.  Writes A (fp16) to `at` and P to `pf`
-// in the cm64 layout (P zero above the diagonal).  Called by all 256 producer threads
-// after a group barrier that publishes the table; ends with the group barrier passed.
+// in the cm64 layout (P zero above the diagonal).  Called by the 128 threads of the
+// prologue role (thread: row i, two 16-column blocks) after a barrier (bar_id) that
+// publishes the table; ends with that barrier passed.
 template <bool OUT, typename TQ>
 __device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* ktile, const uint8_t* qtile,
-                                             const float* sBeta, uint8_t* at, uint8_t* pf, int tg, int t0, int Tq)
+                                             const uint16_t* sBeta, uint8_t* at, uint8_t* pf, int rt, int t0, int Tq,
+                                             int bar_id)
 {
     const float* bT = reinterpret_cast<const float*>(scr);
-    const int i = tg & 63, cq = tg >> 6;
+    const int i = rt & 63, jh = rt >> 6;
     const int nv = min(C, Tq - t0);          // rows of this chunk inside the sequence
-    float accA[16], accP[16];
+    const float bi = bf16_bits_to_f32(sBeta[i]);
+    uint4 resA[2][2], resP[2][2];            // fp16 results of the two blocks (written last)
+    const TQ* tq = nullptr;
+    for (int pass = 0; pass < 2; ++pass) {
+        const int cq = 2 * jh + pass;        // 16-column block of this pass
+        float accA[16], accP[16];
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) accA[jj] = accP[jj] = 0.f;
-    if (16 * cq <= i && i < nv) {
-        const TQ* tq = nullptr;
-        for (int c8 = 0; c8 < 16; ++c8) {
-            const uint4 ku = *reinterpret_cast<const uint4*>(ktile + i * 256 + c8 * 16);
-            const uint4 qu = OUT ? *reinterpret_cast<const uint4*>(qtile + i * 256 + c8 * 16) : make_uint4(0, 0, 0, 0);
-            const float4 b0 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8);
-            const float4 b1 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8 + 4);
-            float ki[8], qi[8];
-            const float bi[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            {
-                const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 a = in2(kw[e], tq), b = in2(qw[e], tq);
-                    ki[2 * e] = a.x; ki[2 * e + 1] = a.y;
-                    qi[2 * e] = b.x; qi[2 * e + 1] = b.y;
-                }
-            }
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-                const int j = 16 * cq + jj;
-                if (j <= i) {
-                    const uint4 kj = *reinterpret_cast<const uint4*>(ktile + j * 256 + c8 * 16);
-                    const float4 c0 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8);
-                    const float4 c1 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8 + 4);
-                    const float bj[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    const uint32_t kw[4] = {kj.x, kj.y, kj.z, kj.w};
-                    float sa = 0.f, sp = 0.f;
+        for (int jj = 0; jj < 16; ++jj) accA[jj] = accP[jj] = 0.f;
+        if (16 * cq <= i && i < nv) {
+            for (int c8 = 0; c8 < 16; ++c8) {
+                const uint4 ku = *reinterpret_cast<const uint4*>(ktile + i * 256 + c8 * 16);
+                const uint4 qu = OUT ? *reinterpret_cast<const uint4*>(qtile + i * 256 + c8 * 16) : make_uint4(0, 0, 0, 0);
+                const float4 b0 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8);
+                const float4 b1 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8 + 4);
+                float ki[8], qi[8];
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                {
+                    const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 kk = in2(kw[e], tq);
-                        const float d0 = ex2_approx(bi[2 * e] - bj[2 * e]) * kk.x;
-                        const float d1 = ex2_approx(bi[2 * e + 1] - bj[2 * e + 1]) * kk.y;
-                        sa = fmaf(ki[2 * e], d0, fmaf(ki[2 * e + 1], d1, sa));
-                        if (OUT) sp = fmaf(qi[2 * e], d0, fmaf(qi[2 * e + 1], d1, sp));
+                        const float2 x = in2(kw[e], tq), y = in2(qw[e], tq);
+                        ki[2 * e] = x.x; ki[2 * e + 1] = x.y;
+                        qi[2 * e] = y.x; qi[2 * e + 1] = y.y;
                     }
-                    accA[jj] += sa;
-                    accP[jj] += sp;
+                }
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int j = 16 * cq + jj;
+                    if (j <= i) {
+                        const uint4 kj = *reinterpret_cast<const uint4*>(ktile + j * 256 + c8 * 16);
+                        const float4 c0 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8);
+                        const float4 c1 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8 + 4);
+                        const float bj[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                        const uint32_t kw[4] = {kj.x, kj.y, kj.z, kj.w};
+                        float sa = 0.f, sp = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 kk = in2(kw[e], tq);
+                            const float d0 = ex2_approx(bv[2 * e] - bj[2 * e]) * kk.x;
+                            const float d1 = ex2_approx(bv[2 * e + 1] - bj[2 * e + 1]) * kk.y;
+                            sa = fmaf(ki[2 * e], d0, fmaf(ki[2 * e + 1], d1, sa));
+                            if (OUT) sp = fmaf(qi[2 * e], d0, fmaf(qi[2 * e + 1], d1, sp));
+                        }
+                        accA[jj] += sa;
+                        accP[jj] += sp;
+                    }
                 }
             }
         }
-    }
-    named_sync(1, NG);   // the table may be overwritten (in MODE_OUTPUT it covers PF)
-    const float bi = sBeta[i];
-    for (int half = 0; half < 2; ++half) {
-        float fa[8], fp[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int jj = 8 * half + e, j = 16 * cq + jj;
-            fa[e] = j < i ? bi * accA[jj] : 0.f;
-            fp[e] = j <= i ? accP[jj] : 0.f;
+        for (int half = 0; half < 2; ++half) {
+            float fa[8], fp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int jj = 8 * half + e, j = 16 * cq + jj;
+                fa[e] = j < i ? bi * accA[jj] : 0.f;
+                fp[e] = j <= i ? accP[jj] : 0.f;
+            }
+            resA[pass][half] = pack8_f16(fa);
+            resP[pass][half] = pack8_f16(fp);
         }
-        const int j0 = 16 * cq + 8 * half;
-        if (16 * cq <= i) *reinterpret_cast<uint4*>(at + cm64(i, j0)) = pack8_f16(fa);
-        if (OUT) *reinterpret_cast<uint4*>(pf + cm64(i, j0)) = pack8_f16(fp);
     }
+    named_sync(bar_id, 128);   // the table may be overwritten (in MODE_OUTPUT it covers PF)
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int j0 = 16 * (2 * jh + pass) + 8 * half;
+            if (16 * (2 * jh + pass) <= i) *reinterpret_cast<uint4*>(at + cm64(i, j0)) = resA[pass][half];
+            if (OUT) *reinterpret_cast<uint4*>(pf + cm64(i, j0)) = resP[pass][half];
+        }
 }
 
 // Inverse T = (I + A)^{-1} of the strictly lower 64 x 64 A (fp16 at Ah, cm64 layout) into
-// the set's T tile (cmT layout, lower blocks only; the upper ones are zeroed elsewhere).
-// Diagonal 16x16 blocks (warp w < 4 owns block w): with N = A_ww (strictly lower,
-// N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs.  Then the
-// off-diagonal blocks by halves of the matrix (each warp: one 8-column half of one 16x16
-// block; X products through per-warp fp16 scratch):
+// the set's T tile (cmT layout, lower blocks only; its upper blocks stay zero).
+// Diagonal 16x16 blocks (warp w4 owns block w4): with N = A_ww (strictly lower, N^16 = 0),
+// (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs.  Then the off-diagonal
+// blocks by halves of the matrix (a work item: one 8-column half of one 16x16 block; X
+// products through per-item fp16 scratch):
 //   level 1: T_10 = -T_11 (A_10 T_00),  T_32 = -T_33 (A_32 T_22)
 //   level 2: X_IJ = sum_{K=J}^{1} A_IK T_KJ  (I = 2, 3; J = 0, 1), then T_IJ = -sum_{K=2}^{I} T_IK X_KJ
-// Called by the 256 producer threads; barriers on named barrier 1.
+// Called by the 4 warps (128 threads) of the inverse role; barriers on bar_id.
 template <int T_LBO>
-__device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint32_t xs, int w, int lane)
+__device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint32_t xs, int w4, int lane, int bar_id)
 {
     auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
-    if (w < 4) {
-        const int b0 = 16 * w, g = lane >> 2, q = lane & 3;
-        const uint32_t scr = xs + 512 * w;
+    const int g = lane >> 2, q = lane & 3;
+    {
+        const int b0 = 16 * w4;
+        const uint32_t scr = xs + 512 * w4;
         uint32_t aN[4], bN[4], bP[4], aX[4];
         ldsm_x4(aN, Ah + cm64(b0 + (lane & 15), b0 + 8 * (lane >> 4)));
         ldsm_x4_t(bN, Ah + cm64(b0 + (lane & 7) + 8 * ((lane >> 3) & 1), b0 + 8 * (lane >> 4)));
@@ -416,10 +448,8 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint
         st_shared_b32(Tt + cmT(b0 + g, b0 + 8) + 4 * q, pack_f16x2(zb[0], zb[1]));
         st_shared_b32(Tt + cmT(b0 + g + 8, b0 + 8) + 4 * q, pack_f16x2(zb[2], zb[3]));
     }
-    named_sync(1, NG);
-    const int g = lane >> 2, q = lane & 3, half = w & 1;
-    const uint32_t scr = xs + 512 * w;
-    auto scr_of = [&](int wx) { return xs + 512 * wx; };
+    named_sync(bar_id, 128);
+    auto scr_of = [&](int it) { return xs + 512 * it; };
     auto put_x = [&](uint32_t dst, const float (&x)[4]) {
         st_shared_b32(dst + cm16(g, 0) + 4 * q, pack_f16x2(x[0], x[1]));
         st_shared_b32(dst + cm16(g + 8, 0) + 4 * q, pack_f16x2(x[2], x[3]));
@@ -432,24 +462,27 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint
         if (isT) ldsm_x4(fr, base + cmT(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
         else ldsm_x4(fr, base + cm64(16 * I + (lane & 15), 16 * K + 8 * (lane >> 4)));
     };
-    if (w < 4) {   // level 1
-        const int I = (w >> 1) ? 3 : 1, J = I - 1, N0 = 16 * J + 8 * half;
+    {   // level 1: warp w4 -> block (I, I-1), half w4 & 1
+        const int half = w4 & 1;
+        const int I = (w4 >> 1) ? 3 : 1, J = I - 1, N0 = 16 * J + 8 * half;
         uint32_t aA[4], bT[2], bX[2], aT[4];
         float x[4] = {0.f, 0.f, 0.f, 0.f}, tt[4] = {0.f, 0.f, 0.f, 0.f};
         a_frag(aA, Ah, I, J, false);
         ldsm_x2_t(bT, Tt + cmT(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
         mma16816(x, aA, bT);
-        put_x(scr, x);
+        put_x(scr_of(w4), x);
         __syncwarp();
-        ldsm_x2_t(bX, scr + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
+        ldsm_x2_t(bX, scr_of(w4) + cm16((lane & 7) + 8 * ((lane >> 3) & 1), 0));
         a_frag(aT, Tt, I, I, true);
         mma16816(tt, aT, bX);
         put_t(I, N0, tt);
     }
-    named_sync(1, NG);
-    // level 2, X: warp w -> block (I, J) = (2 + (w >> 2), (w >> 1) & 1), half w & 1
-    const int I2 = 2 + (w >> 2), J2 = (w >> 1) & 1, N2 = 16 * J2 + 8 * half;
-    {
+    named_sync(bar_id, 128);
+    // level 2, X: item it -> block (I, J) = (2 + (it >> 2), (it >> 1) & 1), half it & 1
+#pragma unroll
+    for (int r2 = 0; r2 < 2; ++r2) {
+        const int it = w4 + 4 * r2;
+        const int I2 = 2 + (it >> 2), J2 = (it >> 1) & 1, N2 = 16 * J2 + 8 * (it & 1);
         float x[4] = {0.f, 0.f, 0.f, 0.f};
         for (int K = J2; K < 2; ++K) {
             uint32_t aA[4], bT[2];
@@ -457,11 +490,14 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint
             ldsm_x2_t(bT, Tt + cmT(16 * K + (lane & 7) + 8 * ((lane >> 3) & 1), N2));
             mma16816(x, aA, bT);
         }
-        put_x(scr, x);
+        put_x(scr_of(it), x);
     }
-    named_sync(1, NG);
-    // level 2, T: the same (I, J, half); X_KJ half was written by warp 4(K-2) + 2J + half
-    {
+    named_sync(bar_id, 128);
+    // level 2, T: the same items; X_KJ half was written by item 4(K-2) + 2J + half
+#pragma unroll
+    for (int r2 = 0; r2 < 2; ++r2) {
+        const int it = w4 + 4 * r2;
+        const int I2 = 2 + (it >> 2), J2 = (it >> 1) & 1, half = it & 1, N2 = 16 * J2 + 8 * half;
         float tt[4] = {0.f, 0.f, 0.f, 0.f};
         for (int K = 2; K <= I2; ++K) {
             uint32_t aT[4], bX[2];
@@ -473,11 +509,25 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint
     }
 }
 
+// bf16 output through TMA: O rows go into two 64-channel x 64-row tiles (128-byte rows,
+// 128-byte swizzle: 16-byte piece p of row i at i*128 + ((p ^ (i & 7)) * 16)).
+__device__ __forceinline__ uint32_t swz_off(int i, int col) { return (uint32_t)((col >> 6) * 8192 + i * 128 + ((((col & 63) >> 3) ^ (i & 7)) << 4) + (col & 7) * 2); }
+
 // The kernel ---------------------------------------------------------------------------
+// Four roles of 4 warps each (role = warp / 4; warp w4 = warp % 4 also names the TMEM lane
+// quarter it may access):
+//   P (role 0)  prologue: log-decay prefix and references of chunk n, the K+ / Q+ / K- tiles
+//               (or A and P on CUDA cores for a wide chunk), the A|P MMA.
+//   I (role 1)  inverse: A and P out of TMEM, T = (I + A)^{-1}, W^T MMA, -W^T into the set.
+//   X (role 2)  state chain: S^ from the master, the [U | O] MMA, U -> fp16, the master and O
+//               MMAs; one thread per TMEM lane (value column).
+//   Y (role 3)  auxiliary: U~ MMA, zeroing the O accumulator, the output rows (TMA store
+//               from a staging tile), beta V, and the TMA loads of k, q, v.
 template <int MODE, typename TQ>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+              const __grid_constant__ CUtensorMap tm_o,
               const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop,
@@ -488,14 +538,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     using TM = Tm<MODE>;
     constexpr bool OUT = MODE == MODE_OUTPUT;
     constexpr int T_LBO = PL::T_LBO;
-    auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     extern __shared__ __align__(1024) uint8_t sm[];
 
     const int t = threadIdx.x, w = t >> 5, lane = t & 31;
     const int q4 = w & 3;                     // TMEM lane quarter of this warp
-    const int hg = (w >> 2) & 1;              // column half inside a warp group
-    const int tg = t & (NG - 1);              // thread index inside its group
-    const int cp = tg & 63, rq = tg >> 6;     // channel pair, 16-row quarter (loads, prologue)
+    const int role = w >> 2;                  // P, I, X, Y
+    const int rt = t & (NR - 1);              // thread index inside its role
     // This CTA's work: chunks [n0, n1) of head h of one sequence that starts at packed
     // token `rowbase` and has `Tq` tokens.  Uniform batch: sequence b of B rows of T
     // tokens, segment p of P; packed samples: one entry of the host-built item table
@@ -520,16 +568,24 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         last = p == P - 1;
     }
     const int nk = max(0, n1 - n0);
+    // the bf16 output leaves by TMA store through a [B, T, H, 128] map that clips at the
+    // end of a row; packed samples share one row, so a chunk that runs past its sample's
+    // end is written with plain stores instead
+    const int o_b = items ? 0 : seq;
+    const int64_t o_t = items ? rowbase : 0;
 
-    float* sBetaP = reinterpret_cast<float*>(sm + PL::MISC + M_BETAP);
-    float* sBetaV = reinterpret_cast<float*>(sm + PL::MISC + M_BETAV);
+    uint16_t* sBeta = reinterpret_cast<uint16_t*>(sm + PL::MISC + M_BETA);
+    uint32_t* sBRaw = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_BRAW);
     float* sTot = reinterpret_cast<float*>(sm + PL::MISC + M_TOT);
     float* sSC = reinterpret_cast<float*>(sm + PL::MISC + M_SC);
+    int* sDirect = reinterpret_cast<int*>(sm + PL::MISC + M_DIRECT);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + PL::MISC + M_BAR);
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_TMEM);
     int* sAbort = reinterpret_cast<int*>(sm + PL::MISC + M_ABORT);
     const uint32_t sbase = smem_addr(sm);
     const Abort ab{sAbort, status};
+    // beta arrives by 4-byte cp.async (the head pair's words) when that is aligned
+    const bool beta_async = (H % 2 == 0) && ((reinterpret_cast<uintptr_t>(beta) & 3u) == 0);
 
     if (t == 0) {
         for (int i = 0; i < NBAR; ++i) mbar_init(&bars[i], 1);
@@ -540,13 +596,15 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_alloc(sTmem, 512);
         tmem_relinquish();
     }
-    // T tiles of both sets start zero (the zero block beside T in MODE_OUTPUT stays zero)
-    {
-        constexpr int TB = OUT ? 16384 : 8192;
-        for (int e = t; e < 2 * TB / 16; e += NT) {
-            const int s = e / (TB / 16), off = (e % (TB / 16)) * 16;
-            *reinterpret_cast<uint4*>(sm + s * PL::SET + PL::TF + off) = make_uint4(0u, 0u, 0u, 0u);
-        }
+    // T tiles of both sets start zero (their upper blocks stay zero)
+    for (int e = t; e < 2 * (PL::T_BYTES / 16); e += NT) {
+        const int s = e / (PL::T_BYTES / 16), off = (e % (PL::T_BYTES / 16)) * 16;
+        *reinterpret_cast<uint4*>(sm + s * PL::SET + PL::TF + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    // beta of the first two chunks into their slots (later chunks: the prologue, two ahead)
+    if (t < 2 * C) {
+        const int x = t / C, i = t % C;
+        sBeta[x * C + i] = beta_bits(beta, rowbase, Tq, H, h, (n0 + x) * C, i, x < nk);
     }
     fence_async_smem();
     tc_fence_before();
@@ -572,72 +630,63 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_arrive_expect_tx(&bars[B_TV + x], 16384);
         tma_load_3d(sm + PL::VB + x * 16384, &tm_v, &bars[B_TV + x], 0, h, (int)(rowbase + n * C));
     };
+    const TQ* tq = nullptr;
 
-    if (t < NG) {
-        // ================= producer: state-independent work of chunk n0 + kc ==============
-        const TQ* tq = nullptr;
-        int g_issued = 0;            // thread 0: g tiles requested so far
-        int n_ap = 0;                // A|P MMAs issued so far (phase of B_AP)
-        float2 carry = make_float2(0.f, 0.f);   // rq == 0: carry of channels 2cp, 2cp+1
-        if (tg == 0) {
+    if (role == 0) {
+        // ================= P: prologue of chunk n0 + kc =====================================
+        const int cp = rt & 63, rh = rt >> 6;   // channel pair, 32-row half
+        int g_issued = 0;                        // rt 0: g tiles requested so far
+        float2 carry = make_float2(0.f, 0.f);   // rh == 0: carry of channels 2cp, 2cp+1
+        if (rt == 0) {
             for (int x = 0; x < min(2, nk); ++x) tma_g(n0 + x);
             g_issued = min(2, nk);
         }
-        uint32_t betaR = (tg < C) ? load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0) : 0u;
         for (int kc = 0; kc < nk; ++kc) {
             const int n = n0 + kc, t0 = n * C, s = kc & 1;
             uint8_t* set = sm + s * PL::SET;
             const uint32_t sset = sbase + s * PL::SET;
-            // ---- part 1: g of this chunk -> cumulative log-decay, references, range ---------
-            group_wait(&bars[B_TG + s], (kc >> 1) & 1, ab, tg == 0, 1);
-            uint32_t gP[16];
-            ld_rows16(gP, sm + PL::GS + s * 16384, 16 * rq, cp);
-            if (t0 + C > Tq) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (t0 + 16 * rq + r >= Tq) gP[r] = 0u;
+            const uint8_t* gst = sm + PL::GS + s * 16384;
+            const uint16_t* sBk = sBeta + (kc & 3) * C;
+            // beta of chunk kc+2 starts its way into shared memory (stored into its slot below)
+            if (rt < C && beta_async) {
+                const int tt = (n + 2) * C + rt;
+                const bool live = n + 2 < n1 && tt < Tq;
+                cp_async4_zfill(sBRaw + rt, beta + (((size_t)rowbase + (live ? tt : 0)) * H + (h & ~1)), live);
+                cp_async_commit();
             }
+            // ---- g of this chunk -> cumulative log-decay (base 2), references, range -----
+            group_wait(&bars[B_TG + s], (kc >> 1) & 1, ab, rt == 0, BAR_P);
+            const int nv = min(C, Tq - t0);   // rows of this chunk inside the sequence
             {
                 const float2 l2e = make_float2(kLog2e, kLog2e);
                 float2 tot = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) tot = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, tot);
-                *reinterpret_cast<float2*>(sTot + rq * D + 2 * cp) = tot;
+#pragma unroll 8
+                for (int r = 0; r < 32; ++r) {
+                    const uint32_t gw = 32 * rh + r < nv ? *reinterpret_cast<const uint32_t*>(gst + (32 * rh + r) * 256 + 4 * cp) : 0u;
+                    tot = __ffma2_rn(in2(gw, (const __nv_bfloat16*)nullptr), l2e, tot);
+                }
+                *reinterpret_cast<float2*>(sTot + rh * D + 2 * cp) = tot;
             }
-            if (tg < C) sBetaP[tg] = __uint_as_float(betaR << 16);
-            named_sync(1, NG);   // sTot, beta published; this g tile is in registers
-            if (tg == 0 && n + 2 < n1 && !*sAbort) {
-                tma_g(n + 2);
-                g_issued = kc + 3;
-            }
-            if (tg < C) betaR = load_beta(beta, rowbase, Tq, H, h, (n + 1) * C, tg, n + 1 < n1);
-            float2 r2, bC, pre;   // b at row 31, b at row 63, b before this thread's first row
-            {
-                float2 tq4[4];
-#pragma unroll
-                for (int qb = 0; qb < 4; ++qb) tq4[qb] = *reinterpret_cast<const float2*>(sTot + qb * D + 2 * cp);
-                r2 = __fadd2_rn(tq4[0], tq4[1]);
-                bC = __fadd2_rn(r2, __fadd2_rn(tq4[2], tq4[3]));
-                pre = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int qb = 0; qb < 3; ++qb)
-                    if (qb < rq) pre = __fadd2_rn(pre, tq4[qb]);
-            }
+            named_sync(BAR_P, NR);   // sTot published
+            const float2 r2 = *reinterpret_cast<const float2*>(sTot + 2 * cp);            // b at row 31
+            const float2 bC = __fadd2_rn(r2, *reinterpret_cast<const float2*>(sTot + D + 2 * cp));   // b at row 63
+            const float2 pre = rh ? r2 : make_float2(0.f, 0.f);                          // b before my rows
             // the middle-row reference keeps a factor within 2^{max(b_0 - r, r - b_63)}
             bool wide = false;
-            if (rq == 0) {
-                const float2 b0 = __fmul2_rn(in2(gP[0], (const __nv_bfloat16*)nullptr), make_float2(kLog2e, kLog2e));
+            if (rh == 0) {
+                const uint32_t g0 = nv > 0 ? *reinterpret_cast<const uint32_t*>(gst + 4 * cp) : 0u;
+                const float2 b0 = __fmul2_rn(in2(g0, (const __nv_bfloat16*)nullptr), make_float2(kLog2e, kLog2e));
                 wide = fmaxf(b0.x - r2.x, r2.x - bC.x) > kRangeMax || fmaxf(b0.y - r2.y, r2.y - bC.y) > kRangeMax;
             }
-            const bool direct = bar_red_or(1, NG, wide);
+            const bool direct = bar_red_or(BAR_P, NR, wide);
             const float2 rp = direct ? make_float2(0.f, 0.f) : r2;   // reference of K+ and Q+
             const float2 rm = direct ? bC : r2;                      // reference of K-
-            // ---- part 2: set s is free once the consumer is done with chunk kc - 2; this
-            // chunk's k (and q) have landed in it ------------------------------------------
-            if (tg == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + s], ((kc >> 1) - 1) & 1, ab);
-            group_wait(&bars[B_TQK + s], (kc >> 1) & 1, ab, tg == 0, 1);
-            if (rq == 0) {
-                // consumer scales: S^ = 2^{rp + carry} master, master <- 2^{rm + carry} master
+            // ---- set s is free once chunk kc-2's master and O MMAs are done; this chunk's k
+            // (and q) have landed in it ---------------------------------------------------------
+            if (rt == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + s], ((kc >> 1) - 1) & 1, ab);
+            group_wait(&bars[B_TQK + s], (kc >> 1) & 1, ab, rt == 0, BAR_P);
+            if (rh == 0) {
+                // the chain's scales: S^ = 2^{rp + carry} master, master <- 2^{rm + carry} master
                 float* sc = sSC + s * 3 * D;
                 *reinterpret_cast<float2*>(sc + 2 * cp) = make_float2(ex2_approx(rp.x + carry.x), ex2_approx(rp.y + carry.y));
                 *reinterpret_cast<float2*>(sc + D + 2 * cp) =
@@ -645,50 +694,60 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 carry = make_float2(bC.x - rm.x, bC.y - rm.y);
                 *reinterpret_cast<float2*>(sc + 2 * D + 2 * cp) = carry;
             }
+            if (rt == 0) sDirect[s] = direct ? 1 : 0;
             if (direct) {
-                // the fp32 log-decay table of the chunk: in MODE_OUTPUT over KM, PF and the first
-                // 8 KB of TF (all free until the prologue), else in the scratch region
+                // the fp32 log-decay table of the chunk: in MODE_OUTPUT over KM, PF and TF (free
+                // until the prologue writes K- and the inverse role fills them), else in the
+                // scratch region
                 uint8_t* scr = OUT ? set + PL::KM : sm + Plan<MODE_STATE>::SCR;
                 float2 run = pre;
                 const float2 l2e = make_float2(kLog2e, kLog2e);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    run = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, run);
-                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(scr) + (16 * rq + r) * D + 2 * cp) = run;
+#pragma unroll 4
+                for (int r = 0; r < 32; ++r) {
+                    const int i = 32 * rh + r;
+                    const uint32_t gw = i < nv ? *reinterpret_cast<const uint32_t*>(gst + i * 256 + 4 * cp) : 0u;
+                    run = __ffma2_rn(in2(gw, (const __nv_bfloat16*)nullptr), l2e, run);
+                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(scr) + i * D + 2 * cp) = run;
                 }
-                named_sync(1, NG);
-                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBetaP, sm + PL::AT,
-                                         OUT ? set + PL::PF : nullptr, tg, t0, Tq);
+                // the A tile is free once the inverse role is done with chunk kc-1
+                if (rt == 0 && kc >= 1) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
+                named_sync(BAR_P, NR);
+                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBk, sm + PL::AT,
+                                         OUT ? set + PL::PF : nullptr, rt, t0, Tq, BAR_P);
+                if (OUT)   // the table covered the T tile: its upper blocks must read zero again
+                    for (int e = rt; e < PL::T_BYTES / 16; e += NR)
+                        *reinterpret_cast<uint4*>(set + PL::TF + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
             }
-            // ---- prologue: beta K+, Q+ in place, K- ----------------------------------------
+            // ---- beta K+, Q+ in place, K-; per 8-row block, the 64 threads of a row half read
+            // their raw rows before any of them rewrites the block they share -----------------
             {
-                uint32_t kR[16], qR[16];
-                ld_rows16(kR, set + PL::KP, 16 * rq, cp);
-                if (OUT) ld_rows16(qR, set + PL::QP, 16 * rq, cp);
-                if (t0 + C > Tq) {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        if (t0 + 16 * rq + r >= Tq) kR[r] = qR[r] = 0u;
-                }
-                named_sync(1, NG);   // every raw row is in registers before the tiles are rewritten
                 const float2 l2e = make_float2(kLog2e, kLog2e);
                 const float2 dlt = make_float2(rm.x - rp.x, rm.y - rp.y);
                 float2 run = make_float2(pre.x - rp.x, pre.y - rp.y);   // b - rp
+#pragma unroll 1
+                for (int blk = 0; blk < 4; ++blk) {
+                    const int rb = 32 * rh + 8 * blk;                     // first row of this block
+                    uint32_t gR[8], kR[8], qR[8];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                    for (int r = 0; r < 8; ++r) {
+                        const bool live = rb + r < nv;
+                        gR[r] = live ? *reinterpret_cast<const uint32_t*>(gst + (rb + r) * 256 + 4 * cp) : 0u;
+                        kR[r] = live ? *reinterpret_cast<const uint32_t*>(set + PL::KP + (rb + r) * 256 + 4 * cp) : 0u;
+                        qR[r] = (OUT && live) ? *reinterpret_cast<const uint32_t*>(set + PL::QP + (rb + r) * 256 + 4 * cp) : 0u;
+                    }
+                    named_sync(BAR_P2 + rh, 64);
                     uint32_t pk[2][4], pm[2][4], pq[2][4];
                     float2 lk = make_float2(0.f, 0.f), lm = lk, lq = lk;
 #pragma unroll
                     for (int r8 = 0; r8 < 8; ++r8) {
-                        const int r = 8 * half + r8, i = 16 * rq + r;
-                        run = __ffma2_rn(in2(gP[r], (const __nv_bfloat16*)nullptr), l2e, run);
-                        const float2 kk = in2(kR[r], tq);
-                        const float bi = sBetaP[i];
+                        run = __ffma2_rn(in2(gR[r8], (const __nv_bfloat16*)nullptr), l2e, run);
+                        const float2 kk = in2(kR[r8], tq);
+                        const float bi = bf16_bits_to_f32(sBk[rb + r8]);
                         const float2 ep = make_float2(ex2_approx(run.x), ex2_approx(run.y));
                         const float2 em = make_float2(ex2_approx(dlt.x - run.x), ex2_approx(dlt.y - run.y));
                         const float2 kp = __fmul2_rn(__fmul2_rn(kk, make_float2(bi, bi)), ep);   // beta K+
                         const float2 km = __fmul2_rn(kk, em);                                   // K-
-                        const float2 qp = OUT ? __fmul2_rn(in2(qR[r], tq), ep) : make_float2(0.f, 0.f);
+                        const float2 qp = OUT ? __fmul2_rn(in2(qR[r8], tq), ep) : make_float2(0.f, 0.f);
                         if (r8 & 1) {
                             const int m = r8 >> 1;
                             pk[0][m] = pack_f16x2(lk.x, kp.x); pk[1][m] = pack_f16x2(lk.y, kp.y);
@@ -698,18 +757,38 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             lk = kp; lm = km; lq = qp;
                         }
                     }
-                    const int ig = 2 * rq + half;
+                    const int ig = 4 * rh + blk;
                     st_pair(set + PL::KP, ig, cp, pk);
                     st_pair(set + PL::KM, ig, cp, pm);
                     if (OUT) st_pair(set + PL::QP, ig, cp, pq);
                 }
             }
+            // beta of chunk kc+2 into its slot (read by this role's prologue and by Y's beta V two
+            // chunks on; the slot's previous chunk, kc-2, is done with on both sides)
+            if (rt < C) {
+                uint16_t bb;
+                if (beta_async) {
+                    cp_async_wait_all();
+                    bb = (uint16_t)(sBRaw[rt] >> (16 * (h & 1)));
+                } else {
+                    bb = beta_bits(beta, rowbase, Tq, H, h, (n + 2) * C, rt, n + 2 < n1);
+                }
+                sBeta[((kc + 2) & 3) * C + rt] = bb;
+            }
             fence_async_smem();
             tc_fence_before();
-            named_sync(1, NG);
-            if (tg == 0) {
-                mbar_arrive(&bars[B_SC + s]);   // this chunk's scales are in place
+            named_sync(BAR_P, NR);
+            if (rt == 0) {
+                mbar_arrive(&bars[B_SC + s]);   // scales, direct flag, tiles (and beta) in place
+                // the g tile has been read for the last time: chunk kc+2's may land
+                if (n + 2 < n1 && !*sAbort) {
+                    tma_g(n + 2);
+                    g_issued = kc + 3;
+                }
                 if (!direct) {
+                    // A|P's TMEM columns (and the A tile): free once the inverse role has read
+                    // chunk kc-1's W^T
+                    if (kc >= 1) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
                     tc_fence_after();
                     // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the
                     // state pass reads K- as rows 64-127 and ignores them)
@@ -720,51 +799,49 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     umma_commit(&bars[B_AP]);
                 }
             }
-            if (!direct) {
-                group_wait(&bars[B_AP], n_ap & 1, ab, tg == 0, 1);
+        }
+        // after a timeout some requested g tiles may not have been waited for: let them land
+        if (rt == 0 && *sAbort)
+            for (int x = max(0, g_issued - 2); x < g_issued; ++x)
+                mbar_wait_bounded(&bars[B_TG + (x & 1)], (x >> 1) & 1, kWaitNs);
+        if (beta_async) cp_async_wait_all();
+    } else if (role == 1) {
+        // ================= I: T and -W^T of chunk n0 + kc ===================================
+        int n_ap = 0;
+        for (int kc = 0; kc < nk; ++kc) {
+            const int s = kc & 1;
+            uint8_t* set = sm + s * PL::SET;
+            const uint32_t sset = sbase + s * PL::SET;
+            group_wait(&bars[B_SC + s], (kc >> 1) & 1, ab, rt == 0, BAR_I);   // the prologue is done
+            if (!sDirect[s]) {
+                group_wait(&bars[B_AP], n_ap & 1, ab, rt == 0, BAR_I);
                 ++n_ap;
                 // A (lanes 0-63) -> fp16 tile, P (lanes 64-127) -> the set's P tile
                 if (OUT || q4 < 2) {
-                    float v[32];
-                    tmem_ld32(tl + TM_APW + 32 * hg, v);
+                    float v[64];
+                    tmem_ld64(tl + TM_APW, v);
                     const bool isP = q4 >= 2;
                     const int i = 32 * (q4 & 1) + lane;
 #pragma unroll
-                    for (int g8 = 0; g8 < 4; ++g8) {
+                    for (int g8 = 0; g8 < 8; ++g8) {
                         float f[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) {
-                            const int col = 32 * hg + 8 * g8 + j;
+                            const int col = 8 * g8 + j;
                             f[j] = (isP ? (col <= i) : (col < i)) ? v[8 * g8 + j] : 0.f;
                         }
-                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 32 * hg + 8 * g8) : sm + PL::AT + cm64(i, 32 * hg + 8 * g8);
+                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 8 * g8) : sm + PL::AT + cm64(i, 8 * g8);
                         *reinterpret_cast<uint4*>(dst) = pack8_f16(f);
                     }
                 }
-            } else if (OUT && tg < 128) {
-                // chunk_ap_direct used the first 8 KB of the T tile as scratch: zero its block
-                // beside T again (T itself is rewritten below)
-                const int kg = tg >> 5, u = tg & 31;
-                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32) = make_uint2(0u, 0u);
-                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 8) = make_uint2(0u, 0u);
-                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 16) = make_uint2(0u, 0u);
-                *reinterpret_cast<uint2*>(set + PL::TF + kg * 2048 + 1024 + u * 32 + 24) = make_uint2(0u, 0u);
+                tc_fence_before();
+                named_sync(BAR_I, NR);
             }
-            // the six upper 16x16 blocks of T are zero
-            if (tg < 192) {
-                const int e = tg >> 5, u = tg & 31;
-                const int I = (e < 3) ? 0 : (e < 5 ? 1 : 2);
-                const int J = (e < 3) ? e + 1 : (e < 5 ? e - 1 : 3);
-                const int row = 16 * I + 8 * (u >> 4) + (u & 7), col = 16 * J + 8 * ((u >> 3) & 1);
-                *reinterpret_cast<uint4*>(set + PL::TF + cmT(row, col)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            tc_fence_before();
-            named_sync(1, NG);
-            invert_unit_lower<T_LBO>(sbase + PL::AT, sset + PL::TF, sbase + PL::MISC + M_XS, w, lane);
+            invert_unit_lower<T_LBO>(sbase + PL::AT, sset + PL::TF, sbase + PL::MISC + M_XS, q4, lane, BAR_I);
             fence_async_smem();
             tc_fence_before();
-            named_sync(1, NG);
-            if (tg == 0) {
+            named_sync(BAR_I, NR);
+            if (rt == 0) {
                 mbar_arrive(&bars[B_INV + s]);   // T ready
                 tc_fence_after();
                 // W^T = (beta K+)^T T^T: M = 128 channels, N = 64 positions, K = 64 positions
@@ -774,40 +851,34 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                              sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
                 umma_commit(&bars[B_W]);
             }
-            group_wait(&bars[B_W], kc & 1, ab, tg == 0, 1);
-            {   // -W^T -> the KP tile (channel c in lane c, positions 32*hg ..)
-                float v[32];
-                tmem_ld32(tl + TM_APW + 32 * hg, v);
+            group_wait(&bars[B_W], kc & 1, ab, rt == 0, BAR_I);
+            {   // -W^T -> the KP tile (channel c in lane c)
+                float v[64];
+                tmem_ld64(tl + TM_APW, v);
                 const int c = 32 * q4 + lane;
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
+                for (int g8 = 0; g8 < 8; ++g8) {
                     float f[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j) f[j] = -v[8 * g8 + j];
-                    const int i0 = 32 * hg + 8 * g8;
-                    *reinterpret_cast<uint4*>(set + PL::KP + (i0 >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16) =
-                        pack8_f16(f);
+                    *reinterpret_cast<uint4*>(set + PL::KP + g8 * 2048 + (c >> 3) * 128 + (c & 7) * 16) = pack8_f16(f);
                 }
             }
             fence_async_smem();
             tc_fence_before();
-            named_sync(1, NG);
-            // every tile of the set is ready (the test hook withholds chunk 0's signal)
-            if (tg == 0 && !(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
+            named_sync(BAR_I, NR);
+            if (rt == 0) {
+                // every tile of the set is ready (the test hook withholds chunk 0's signal)
+                if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
+                mbar_arrive(&bars[B_APWF]);   // A|P's TMEM columns may be reused
+            }
         }
-        // after a timeout some requested g tiles may not have been waited for: let them land
-        if (tg == 0 && *sAbort)
-            for (int x = max(0, g_issued - 2); x < g_issued; ++x)
-                mbar_wait_bounded(&bars[B_TG + (x & 1)], (x >> 1) & 1, kWaitNs);
-    } else {
-        // ================= consumer: the state chain of chunk n0 + kc =====================
-        const TQ* tq = nullptr;
-        const int cw = w - 8, ch = cw >> 2;        // column half of this warp
+    } else if (role == 2) {
+        // ================= X: the state chain of chunk n0 + kc ==============================
         const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
-        const bool mma = tg == 0, loader = tg == 32, poller = tg == 0;
-        // initial state in TMEM: columns 64*ch .. of the master (MODE_STATE: both masters)
-        for (int cc = 0; cc < 64; cc += 32) {
-            const int c0 = 64 * ch + cc;
+        const bool mma = rt == 0;
+        // initial state in TMEM (MODE_STATE: N from 0, Phi from I)
+        for (int c0 = 0; c0 < D; c0 += 32) {
             float vv[32];
             if (MODE == MODE_STATE) {
 #pragma unroll
@@ -829,173 +900,47 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_st32(tl + TM::MASTER + c0, vv);
             }
         }
-        int v_issued = 0, qk_last[2] = {-1, -1};   // loader: TMA requests so far
-        if (loader && nk > 0) {
-            for (int x = 0; x < min(2, nk); ++x) {
-                tma_v(n0 + x);
-                tma_qk(n0 + x);
-                qk_last[x] = x;
-            }
-            v_issued = min(2, nk);
-        }
-        float gam = 1.f;
-        if (OUT && gate && gamma) gam = gamma[(size_t)h * D + j];
-        // beta of chunks n0 and n0 + 1 -> their beta V slots
-        if (tg < C) {
-            sBetaV[tg] = __uint_as_float(load_beta(beta, rowbase, Tq, H, h, n0 * C, tg, nk > 0) << 16);
-            sBetaV[C + tg] = __uint_as_float(load_beta(beta, rowbase, Tq, H, h, (n0 + 1) * C, tg, nk > 1) << 16);
-        }
         tc_fence_before();
-        // beta V of chunk x in place (v landed in beta V tile x & 1): thread = channel pair x
-        // 16 rows; every raw row is read before any tile is rewritten
-        auto beta_v = [&](int x) {
-            const int vb = x & 1, t0x = (n0 + x) * C;
-            group_wait(&bars[B_TV + vb], (x >> 1) & 1, ab, poller, 2);
-            uint32_t vR[16];
-            uint8_t* tile = sm + PL::VB + vb * 16384;
-            ld_rows16(vR, tile, 16 * rq, cp);
-            if (t0x + C > Tq) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (t0x + 16 * rq + r >= Tq) vR[r] = 0u;
-            }
-            named_sync(2, NG);
-            uint32_t pv[2][4];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float2 lv = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int r8 = 0; r8 < 8; ++r8) {
-                    const int r = 8 * half + r8;
-                    const float bi = sBetaV[vb * C + 16 * rq + r];
-                    const float2 vbv = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
-                    if (r8 & 1) {
-                        pv[0][r8 >> 1] = pack_f16x2(lv.x, vbv.x);
-                        pv[1][r8 >> 1] = pack_f16x2(lv.y, vbv.y);
-                    } else {
-                        lv = vbv;
-                    }
-                }
-                st_pair(tile, 2 * rq + half, cp, pv);
-            }
-            fence_async_smem();
-        };
-        if (nk > 0) beta_v(0);
-        tc_fence_before();
-        named_sync(2, NG);   // initial master and the first beta V are in place
-        tc_fence_after();
-        // U~^T = (beta V)^T T^T into the chunk's U columns (MODE_OUTPUT: [U~^T | 0] over
-        // the [U | O] buffer, so O starts from zero)
-        auto issue_u = [&](int x) {
-            const int s = x & 1;
-            const uint32_t sset = sbase + s * PL::SET, vbt = sbase + PL::VB + s * 16384;
-            if (OUT) {
-                const uint32_t id = idesc_f16(128, 128, false, false);
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TM::UO + 128 * s, sdesc(vbt + 4096 * kk, 2048, 128),
-                             sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
-            } else {
-                const uint32_t id = idesc_f16(128, 64, false, false);
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16(tmem + TM::UACC, sdesc(vbt + 4096 * kk, 2048, 128),
-                             sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
-            }
-            umma_commit(&bars[B_VE + s]);   // the beta V tile may be refilled
-        };
-        // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
-        auto out_rows = [&](int x) {
-            const int b = x & 1, t0x = (n0 + x) * C;
-            group_wait(&bars[B_O + b], (x >> 1) & 1, ab, poller, 2);
-            float v[32];
-            tmem_ld32(tl + Tm<MODE_OUTPUT>::UO + 128 * b + 64 + 32 * ch, v);
-            const int nv = min(C, Tq - t0x);
-            if (gate) {
-                // Eq. 15 output side: y = Sigmoid(gate) * gamma * RMSNorm over the head's values.
-                // Per position, the sum of squares over this warp's 32 values by a transposing
-                // butterfly (lane l ends with position 32*ch + l), then over the 4 lane quarters.
-                float sq[32];
-#pragma unroll
-                for (int u = 0; u < 32; ++u) sq[u] = v[u] * v[u];
-#pragma unroll
-                for (int sft = 16; sft >= 1; sft >>= 1) {
-                    const bool up = (lane & sft) != 0;
-#pragma unroll
-                    for (int k = 0; k < sft; ++k) {
-                        const float send = up ? sq[k] : sq[k + sft];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
-                        sq[k] = (up ? sq[k + sft] : sq[k]) + recv;
-                    }
-                }
-                float* red = reinterpret_cast<float*>(sm + PL::MISC + M_RED);
-                red[q4 * C + 32 * ch + lane] = sq[0];
-                named_sync(2, NG);
-                const int pi = 32 * ch + lane;
-                const float m = (red[pi] + red[C + pi] + red[2 * C + pi] + red[3 * C + pi]) * (1.f / D) + eps;
-                const float inv = m > 0.f ? rsqrtf(m) : 0.f;
-                named_sync(2, NG);   // red may be reused
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const float iu = __shfl_sync(0xffffffffu, inv, u);
-                    const int i = 32 * ch + u;
-                    float gv = 0.f;
-                    if (i < nv) gv = __bfloat162float(gate[(((size_t)rowbase + t0x + i) * H + h) * D + j]);
-                    v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int i = 32 * ch + u;
-                if (i < nv) {
-                    const size_t idx = (((size_t)rowbase + t0x + i) * H + h) * D + j;
-                    if (o_f32) reinterpret_cast<float*>(o)[idx] = v[u];
-                    else reinterpret_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(v[u]);
-                }
-            }
-        };
-        bool u_done = false;   // U~ of chunk kc already issued
+        named_sync(BAR_X, NR);
         for (int kc = 0; kc < nk; ++kc) {
-            const int n = n0 + kc, s = kc & 1;
+            const int s = kc & 1;
             const uint32_t sset = sbase + s * PL::SET;
-            // beta of chunk kc+2, loaded now and stored once its slot is free
-            const uint32_t betaN = tg < C ? load_beta(beta, rowbase, Tq, H, h, (n + 2) * C, tg, n + 2 < n1) : 0u;
-            if (mma && !u_done) {
-                thread_wait(&bars[B_INV + s], (kc >> 1) & 1, ab);
-                tc_fence_after();
-                issue_u(kc);
-            }
             // ---- S^ = fp16(2^{rp + carry} master), master <- 2^{rm + carry} master --------
-            if (poller) {
+            if (rt == 0) {
                 thread_wait(&bars[B_SC + s], (kc >> 1) & 1, ab);
                 if (kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
             }
-            named_sync(2, NG);
+            named_sync(BAR_X, NR);
             tc_fence_after();
             {
                 const float* sY = sSC + s * 3 * D;
                 const float* sMs = sY + D;
                 for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
                     const uint32_t mcol = TM::MASTER + D * mi, hcol = TM::S16 + 64 * mi;
-                    for (int cc = 0; cc < 64; cc += 32) {
-                        const int c0 = 64 * ch + cc;
-                        float vv[32];
-                        uint32_t hv[16];
-                        tmem_ld32(tl + mcol + c0, vv);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 64) {
+                        float vv[64];
+                        uint32_t hv[32];
+                        tmem_ld64(tl + mcol + c0, vv);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4) {
+                        for (int e = 0; e < 64; e += 4) {
                             const float4 y4 = *reinterpret_cast<const float4*>(sY + c0 + e);
                             const float4 m4 = *reinterpret_cast<const float4*>(sMs + c0 + e);
                             hv[e / 2] = pack_f16x2(vv[e] * y4.x, vv[e + 1] * y4.y);
                             hv[e / 2 + 1] = pack_f16x2(vv[e + 2] * y4.z, vv[e + 3] * y4.w);
                             vv[e] *= m4.x; vv[e + 1] *= m4.y; vv[e + 2] *= m4.z; vv[e + 3] *= m4.w;
                         }
-                        tmem_st16u(tl + hcol + c0 / 2, hv);
-                        tmem_st32(tl + mcol + c0, vv);
+                        tmem_st32u_nowait(tl + hcol + c0 / 2, hv);
+                        tmem_st64_nowait(tl + mcol + c0, vv);
                     }
                 }
+                tmem_wait_st();
             }
             tc_fence_before();
-            named_sync(2, NG);
+            named_sync(BAR_X, NR);
             if (mma) {
+                // U~ (Y) initialised the U columns; -W^T and Q+ are in the set (I)
+                thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
                 thread_wait(&bars[B_PRO + s], (kc >> 1) & 1, ab);
                 tc_fence_after();
                 if (OUT) {
@@ -1012,40 +957,22 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 umma_commit(&bars[B_U]);
             }
-            // ---- meanwhile: chunk kc-1's output rows and chunk kc+1's beta V ----------------
-            if (OUT && kc > 0) out_rows(kc - 1);
-            if (kc + 1 < nk) beta_v(kc + 1);
-            if (tg < C && kc + 2 < nk)   // chunk kc's beta V slot is free (chunk kc+2 uses it)
-                sBetaV[s * C + tg] = __uint_as_float(betaN << 16);
-            group_wait(&bars[B_U], kc & 1, ab, poller, 2);
-            if (loader && !*sAbort) {
-                // the [U | O] MMA has read -W^T and Q+ (MODE_OUTPUT): chunk kc+2's k and q may land
-                if (OUT && n + 2 < n1) {
-                    tma_qk(n + 2);
-                    qk_last[s] = kc + 2;
-                }
-                // U~ of chunk kc has read its beta V tile: chunk kc+2's v may land
-                if (n + 2 < n1) {
-                    thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
-                    if (!*sAbort) {
-                        tma_v(n + 2);
-                        v_issued = kc + 3;
-                    }
-                }
-            }
-            // ---- U -> fp16 (A operand of the master and O updates) ---------------------------
+            group_wait(&bars[B_U], kc & 1, ab, rt == 0, BAR_X);
+            // ---- U -> fp16 (A operand of the master and O updates); one thread owns its lane,
+            // so it may overwrite the columns it has just read ------------------------------------
             {
-                const uint32_t ucol0 = OUT ? TM::UO + 128 * s : TM::UACC;
-                const uint32_t dst = OUT ? ucol0 : TM::S16;   // MODE_STATE: into S^'s columns
-                float vv[32];
-                uint32_t hv[16];
-                tmem_ld32(tl + ucol0 + 32 * ch, vv);
+                const uint32_t usrc = OUT ? TM::UO + 128 * s : TM::UACC;
+                const uint32_t udst = OUT ? TM::UO + 128 * s : TM::S16;   // MODE_STATE: into S^'s columns
+                float vv[64];
+                uint32_t hv[32];
+                tmem_ld64(tl + usrc, vv);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
-                tmem_st16u(tl + dst + 32 * ch, hv);
+                for (int e = 0; e < 32; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
+                tmem_st32u_nowait(tl + udst, hv);
+                tmem_wait_st();
             }
             tc_fence_before();
-            named_sync(2, NG);
+            named_sync(BAR_X, NR);
             if (mma) {
                 tc_fence_after();
                 const uint32_t idm = idesc_f16(128, 128, false, false);
@@ -1053,16 +980,16 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // master += U^T K-   and   O^T += U^T P^T
                     const uint32_t ua = tmem + TM::UO + 128 * s;
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + TM::MASTER, ua + ucol(kk), sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
+                        umma_f16_ts(tmem + TM::MASTER, ua + 8 * kk, sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     umma_commit(&bars[B_S]);
                     const uint32_t ido = idesc_f16(128, 64, false, false);
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(ua + 64, ua + ucol(kk), sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
+                        umma_f16_ts(ua + 64, ua + 8 * kk, sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
                     umma_commit(&bars[B_O + s]);
                 } else {
                     // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + ucol(kk),
+                        umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     const uint32_t id = idesc_f16(128, 64, false, true);
                     for (int kk = 0; kk < 8; ++kk)
@@ -1072,60 +999,38 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             if (!OUT) {
-                group_wait(&bars[B_U2], kc & 1, ab, poller, 2);
-                // -W^T has been read twice: chunk kc+2's k may land
-                if (loader && !*sAbort && n + 2 < n1) {
-                    tma_qk(n + 2);
-                    qk_last[s] = kc + 2;
-                }
+                group_wait(&bars[B_U2], kc & 1, ab, rt == 0, BAR_X);
                 {
-                    float vv[32];
-                    uint32_t hv[16];
-                    tmem_ld32(tl + TM::UACC + 32 * ch, vv);
+                    float vv[64];
+                    uint32_t hv[32];
+                    tmem_ld64(tl + TM::UACC, vv);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
-                    tmem_st16u(tl + TM::S16 + 64 + 32 * ch, hv);
+                    for (int e = 0; e < 32; ++e) hv[e] = pack_f16x2(vv[2 * e], vv[2 * e + 1]);
+                    tmem_st32u_nowait(tl + TM::S16 + 64, hv);
+                    tmem_wait_st();
                 }
                 tc_fence_before();
-                named_sync(2, NG);
+                named_sync(BAR_X, NR);
                 if (mma) {
                     tc_fence_after();
                     const uint32_t idm = idesc_f16(128, 128, false, false);
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_f16_ts(tmem + TM::MASTER + D, tmem + TM::S16 + 64 + ucol(kk),
+                        umma_f16_ts(tmem + TM::MASTER + D, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     umma_commit(&bars[B_S]);
                 }
             }
-            if (mma) {
-                umma_commit(&bars[B_EMPTY + s]);   // set s may be refilled
-                // U~ of the next chunk now, if its T is ready (else at the top of the next step)
-                u_done = false;
-                if (kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
-                    tc_fence_after();
-                    issue_u(kc + 1);
-                    u_done = true;
-                }
-            }
-        }
-        if (OUT && nk > 0) out_rows(nk - 1);
-        // after a timeout some requested tiles may not have been waited for: let them land
-        if (loader && *sAbort) {
-            for (int x = max(0, v_issued - 2); x < v_issued; ++x)
-                mbar_wait_bounded(&bars[B_TV + (x & 1)], (x >> 1) & 1, kWaitNs);
-            for (int s2 = 0; s2 < 2; ++s2)
-                if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
+            if (mma) umma_commit(&bars[B_EMPTY + s]);   // set s may be refilled
         }
         // ---- end of segment: the state S = diag(2^{carry}) master (columns = channels) -----
-        if (nk > 0) group_wait(&bars[B_S], (nk - 1) & 1, ab, poller, 2);
+        if (nk > 0) group_wait(&bars[B_S], (nk - 1) & 1, ab, rt == 0, BAR_X);
         float* dst = nullptr;
         if (MODE == MODE_STATE) dst = maps + (size_t)slot * 2 * D * D;  // [N | M]
         else if (S_T && last) dst = S_T + ((size_t)seq * H + h) * D * D;
         if (dst && !*sAbort) {
             const float* cn = nk > 0 ? sSC + ((nk - 1) & 1) * 3 * D + 2 * D : nullptr;
             for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
-                for (int cc = 0; cc < 64; cc += 32) {
-                    const int c0 = 64 * ch + cc;
+                for (int c0 = 0; c0 < D; c0 += 32) {
                     float vv[32];
                     tmem_ld32(tl + TM::MASTER + D * mi + c0, vv);
                     float* d = dst + (size_t)mi * D * D + j;
@@ -1134,10 +1039,235 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
         }
+    } else {
+        // ================= Y: U~, the output rows, beta V, loads ============================
+        const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
+        const bool mma = rt == 0, loader = rt == 32;
+        int v_issued = 0, qk_last[2] = {-1, -1};   // loader: TMA requests so far
+        bool o_pending = false;                    // rt 0: a TMA store of the staging tile in flight
+        if (loader && nk > 0) {
+            for (int x = 0; x < min(2, nk); ++x) {
+                tma_v(n0 + x);
+                tma_qk(n0 + x);
+                qk_last[x] = x;
+            }
+            v_issued = min(2, nk);
+        }
+        float gam = 1.f;
+        if (OUT && gate && gamma) gam = gamma[(size_t)h * D + j];
+        // beta V of chunk x in place (v landed in beta V tile x & 1): thread = channel pair x
+        // 32 rows; every raw row of a 16-row band is read before the band is rewritten
+        auto beta_v = [&](int x) {
+            const int vb = x & 1, t0x = (n0 + x) * C, cp = rt & 63, rh = rt >> 6;
+            const int nvx = min(C, Tq - t0x);
+            group_wait(&bars[B_TV + vb], (x >> 1) & 1, ab, rt == 0, BAR_Y);
+            uint8_t* tile = sm + PL::VB + vb * 16384;
+            const uint16_t* sBx = sBeta + (x & 3) * C;
+#pragma unroll 1
+            for (int band = 0; band < 2; ++band) {
+                const int rb = 32 * rh + 16 * band;
+                uint32_t vR[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    vR[r] = rb + r < nvx ? *reinterpret_cast<const uint32_t*>(tile + (rb + r) * 256 + 4 * cp) : 0u;
+                named_sync(BAR_Y2 + rh, 64);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pv[2][4];
+                    float2 lv = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r8 = 0; r8 < 8; ++r8) {
+                        const int r = 8 * half + r8;
+                        const float bi = bf16_bits_to_f32(sBx[rb + r]);
+                        const float2 vbv = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
+                        if (r8 & 1) {
+                            pv[0][r8 >> 1] = pack_f16x2(lv.x, vbv.x);
+                            pv[1][r8 >> 1] = pack_f16x2(lv.y, vbv.y);
+                        } else {
+                            lv = vbv;
+                        }
+                    }
+                    st_pair(tile, (rb >> 3) + half, cp, pv);
+                }
+            }
+            fence_async_smem();
+        };
+        // zero the O columns of [U | O] buffer x (U~ writes only the U columns)
+        auto zero_o = [&](int x) {
+            if (!OUT) return;
+            float z[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) z[e] = 0.f;
+            tmem_st32(tl + TM::UO + 128 * (x & 1) + 64, z);
+            tmem_st32(tl + TM::UO + 128 * (x & 1) + 96, z);
+        };
+        // U~^T = (beta V)^T T^T into the chunk's U columns
+        auto issue_u = [&](int x) {
+            const int s = x & 1;
+            const uint32_t sset = sbase + s * PL::SET, vbt = sbase + PL::VB + s * 16384;
+            const uint32_t id = idesc_f16(128, 64, false, false);
+            const uint32_t d = tmem + (OUT ? TM::UO + 128 * s : TM::UACC);
+            for (int kk = 0; kk < 4; ++kk)
+                umma_f16(d, sdesc(vbt + 4096 * kk, 2048, 128), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
+                         kk > 0);
+            umma_commit(&bars[B_VE + s]);   // U~ done: the beta V tile may be refilled
+        };
+        // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
+        auto out_rows = [&](int x) {
+            const int b = x & 1, t0x = (n0 + x) * C;
+            // the staging tile is free once the previous store has read it (the role barrier of
+            // the wait below holds every other thread until then)
+            if (rt == 0 && o_pending) {
+                bulk_wait_read0();
+                o_pending = false;
+            }
+            group_wait(&bars[B_O + b], (x >> 1) & 1, ab, rt == 0, BAR_Y);
+            const int nvx = min(C, Tq - t0x);
+            const bool tma = !o_f32 && !(items && t0x + C > Tq);
+            float inv_lo = 0.f, inv_hi = 0.f;   // per-position inverse RMS (gated output)
+            if (gate) {
+                // Eq. 15 output side: y = Sigmoid(gate) * gamma * RMSNorm over the head's values.
+                // Per position, the sum of squares over this warp's 32 values by a transposing
+                // butterfly (lane l ends with position 32*hp + l), then over the 4 lane quarters.
+                float* red = reinterpret_cast<float*>(sm + PL::MISC + M_RED);
+                for (int hp = 0; hp < 2; ++hp) {
+                    float sq[32];
+                    tmem_ld32(tl + TM::UO + 128 * b + 64 + 32 * hp, sq);
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) sq[u] = sq[u] * sq[u];
+#pragma unroll
+                    for (int sft = 16; sft >= 1; sft >>= 1) {
+                        const bool up = (lane & sft) != 0;
+#pragma unroll
+                        for (int k = 0; k < sft; ++k) {
+                            const float send = up ? sq[k] : sq[k + sft];
+                            const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
+                            sq[k] = (up ? sq[k + sft] : sq[k]) + recv;
+                        }
+                    }
+                    red[q4 * C + 32 * hp + lane] = sq[0];
+                }
+                named_sync(BAR_Y, NR);
+                const float m0 = (red[lane] + red[C + lane] + red[2 * C + lane] + red[3 * C + lane]) * (1.f / D) + eps;
+                const float m1 = (red[32 + lane] + red[C + 32 + lane] + red[2 * C + 32 + lane] + red[3 * C + 32 + lane]) *
+                                     (1.f / D) + eps;
+                inv_lo = m0 > 0.f ? rsqrtf(m0) : 0.f;
+                inv_hi = m1 > 0.f ? rsqrtf(m1) : 0.f;
+            }
+            uint8_t* os = sm + PL::OS;
+            for (int hp = 0; hp < 2; ++hp) {
+                float v[32];
+                tmem_ld32(tl + TM::UO + 128 * b + 64 + 32 * hp, v);
+                if (gate) {
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const float iu = __shfl_sync(0xffffffffu, hp ? inv_hi : inv_lo, u);
+                        const int i = 32 * hp + u;
+                        float gv = 0.f;
+                        if (i < nvx) gv = __bfloat162float(gate[(((size_t)rowbase + t0x + i) * H + h) * D + j]);
+                        v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
+                    }
+                }
+                if (tma) {
+                    // bf16 into the swizzled staging tiles: lane pairs trade halves so each
+                    // thread writes a value pair (4 bytes)
+                    const bool odd = lane & 1;
+#pragma unroll
+                    for (int u2 = 0; u2 < 16; ++u2) {
+                        const float send = odd ? v[2 * u2] : v[2 * u2 + 1];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                        const float lo = odd ? recv : v[2 * u2], hi = odd ? v[2 * u2 + 1] : recv;
+                        const int i = 32 * hp + 2 * u2 + (odd ? 1 : 0);
+                        *reinterpret_cast<__nv_bfloat162*>(os + swz_off(i, j & ~1)) = __floats2bfloat162_rn(lo, hi);
+                    }
+                } else {
+                    // fp32 output, or a packed sample's ragged last chunk: plain stores
+                    const size_t rs = (size_t)H * D;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u) {
+                        const int i = 32 * hp + u;
+                        if (i < nvx) {
+                            const size_t idx = ((size_t)rowbase + t0x + i) * rs + (size_t)h * D + j;
+                            if (o_f32) reinterpret_cast<float*>(o)[idx] = v[u];
+                            else reinterpret_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(v[u]);
+                        }
+                    }
+                }
+            }
+            if (tma) {
+                fence_async_smem();
+                named_sync(BAR_Y, NR);
+                if (rt == 0) {
+                    tma_store_4d(&tm_o, os, 0, h, (int)(o_t + t0x), o_b);
+                    tma_store_4d(&tm_o, os + 8192, 64, h, (int)(o_t + t0x), o_b);
+                    bulk_commit();
+                    o_pending = true;
+                }
+            }
+        };
+        if (nk > 0) beta_v(0);
+        zero_o(0);
+        if (nk > 1) zero_o(1);
+        tc_fence_before();
+        named_sync(BAR_Y, NR);   // the first beta V and zeroed O columns are in place
+        tc_fence_after();
+        bool u_done = false;     // rt 0: U~ of chunk kc already issued
+        for (int kc = 0; kc < nk; ++kc) {
+            const int n = n0 + kc, s = kc & 1;
+            if (mma && !u_done) {
+                thread_wait(&bars[B_INV + s], (kc >> 1) & 1, ab);
+                // MODE_STATE: one U accumulator; the chain of chunk kc-1 has read it once its
+                // last master update is done
+                if (!OUT && kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
+                tc_fence_after();
+                issue_u(kc);
+            }
+            // ---- chunk kc-1's output rows, then its O columns are zeroed for chunk kc+1 -------
+            if (OUT && kc > 0) {
+                out_rows(kc - 1);
+                if (kc + 1 < nk) zero_o(kc + 1);
+            }
+            // ---- beta V of chunk kc+1 ------------------------------------------------------------
+            if (kc + 1 < nk) beta_v(kc + 1);
+            tc_fence_before();
+            named_sync(BAR_Y, NR);
+            // ---- loads: chunk kc+2's k (and q) once the [U | O] MMA of chunk kc has read the set's
+            // -W^T (and Q+) (MODE_STATE: both chains' MMAs), its v once U~ of chunk kc is done -----
+            if (loader && n + 2 < n1 && !*sAbort) {
+                thread_wait(&bars[OUT ? B_U : B_U2], kc & 1, ab);
+                if (!*sAbort) {
+                    tma_qk(n + 2);
+                    qk_last[s] = kc + 2;
+                }
+                thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
+                if (!*sAbort) {
+                    tma_v(n + 2);
+                    v_issued = kc + 3;
+                }
+            }
+            // U~ of the next chunk now, if its T is ready (else at the top of the next step)
+            if (mma) {
+                u_done = false;
+                if (OUT && kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_u(kc + 1);
+                    u_done = true;
+                }
+            }
+        }
+        if (OUT && nk > 0) out_rows(nk - 1);
+        if (rt == 0 && o_pending) bulk_wait0();   // every output store has landed before the CTA exits
+        // after a timeout some requested tiles may not have been waited for: let them land
+        if (loader && *sAbort) {
+            for (int x = max(0, v_issued - 2); x < v_issued; ++x)
+                mbar_wait_bounded(&bars[B_TV + (x & 1)], (x >> 1) & 1, kWaitNs);
+            for (int s2 = 0; s2 < 2; ++s2)
+                if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
+        }
     }
     // ---- teardown: after a timeout, each MMA issuer drains its own MMAs; free TMEM --------
-    if (*sAbort && (t == 0 || t == NG)) {
-        uint64_t* dr = &bars[t == 0 ? B_DRAIN : B_DRAIN2];
+    if (*sAbort && (t == 0 || t == NR || t == 2 * NR || t == 3 * NR)) {
+        uint64_t* dr = &bars[B_DRAIN + role];
         umma_commit(dr);
         mbar_wait_bounded(dr, 0, kWaitNs);
     }
@@ -1292,8 +1422,24 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output o as a 4-D tensor (channels, heads, tokens, rows), box = 64 channels x
+// 1 head x 64 tokens, 128-byte swizzle.  Tokens past T are clipped by the T dimension, so
+// a ragged last chunk never writes into the next row.
+bool make_map_o(CUtensorMap* m, void* base, int B, int T, int H)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)C, 1u};
+    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Maps {
-    CUtensorMap q, k, v, g;
+    CUtensorMap q, k, v, g, o;   // o: only for a bf16 output (else a copy of q, unused)
 };
 
 struct Split {
@@ -1323,7 +1469,7 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     if (grid == 0) return cudaSuccess;
     ProfileScope prof(prof_name ? prof_name : (MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output"), s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
                                 (const __nv_bfloat16*)a.gate, a.gamma, a.eps, items);
     return cudaGetLastError();
@@ -1334,9 +1480,15 @@ bool build_maps(const KdaArgs& a, Maps& mp)
 {
     const CUtensorMapDataType dq =
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    return make_map(&mp.q, a.q, dq, a.B, a.T, a.H) && make_map(&mp.k, a.k, dq, a.B, a.T, a.H) &&
-           make_map(&mp.v, a.v, dq, a.B, a.T, a.H) &&
-           make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H);
+    if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
+        !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
+        return false;
+    if (a.out_t == ET_F32 || !a.o) {
+        mp.o = mp.q;
+        return true;
+    }
+    return make_map_o(&mp.o, a.o, a.B, a.T, a.H);
 }
 
 int sm_count()
@@ -1436,6 +1588,8 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
     }
     const int P = wv.P, L = wv.L, BH = a.B * a.H;
+    // item tables address packed rows: the bf16 output map spans all B*T rows as one
+    if (a.out_t == ET_BF16 && !make_map_o(&mp.o, a.o, 1, a.B * a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     float* starts = reinterpret_cast<float*>(base + wv.maps_b);
@@ -1628,6 +1782,8 @@ cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int*
     if (!make_map(&mp.q, a.q, dq, 1, a.T, a.H) || !make_map(&mp.k, a.k, dq, 1, a.T, a.H) ||
         !make_map(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
         return cudaErrorInvalidValue;
+    if (a.out_t == ET_F32) mp.o = mp.q;
+    else if (!make_map_o(&mp.o, a.o, 1, a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     base += a256(pl.n_maps * 2 * D * D * sizeof(float));
@@ -1678,7 +1834,7 @@ bool kda_tc_supported(const KdaArgs& a)
     if (a.in_t != ET_BF16 && a.in_t != ET_F16) return false;
     if (a.gb_t != ET_BF16) return false;
     if (a.out_t != ET_BF16 && a.out_t != ET_F32) return false;
-    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.g)) return false;
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.g) || !aligned16(a.o)) return false;
     if (a.gate && a.in_t != ET_BF16) return false;
     return encode_fn() != nullptr;
 }

@@ -35,9 +35,10 @@ def _inputs(B, T, H, seed):
 
 
 def test_noalloc_matches_oracle_and_allocating_entry_point_on_two_calls():
-    # B*H = 8, then 4 on a 148-SM part: the tensor-core path cuts each head into segments
-    # (state pass, combine, output pass) and keeps the maps and start states in the scratch
-    shapes = [(1, 4096, 8, 1), (1, 2048, 4, 2)]
+    # B*H = 8 (16 segments of 4 chunks per head on a 148-SM part), then B*H = 16 (8
+    # segments of 2 chunks): the tensor-core path keeps the segment maps and start states
+    # in the scratch, in a different layout for each call
+    shapes = [(1, 4096, 8, 1), (1, 1024, 16, 2)]
     needs = [kda.workspace_size(B, T, H, 128, 128) for B, T, H, _ in shapes]
     assert 0 < needs[1] < needs[0] <= kda.NOALLOC_SCRATCH_BYTES
     cases = [_inputs(B, T, H, seed) for B, T, H, seed in shapes]
