@@ -89,18 +89,17 @@ enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 // Per buffer set (chunk parity): KP (k -> beta K+ -> -W^T) and QP (q -> Q+) as
 // channel-major tiles, QP directly after KP so [beta K+; Q+] and [-W^T | Q+^T] are single
 // 128-row operands; KM (K-); PF (P as the K-major B operand of O^T += U^T P^T); TF (T as
-// the K-major B operand T^T of W^T and U~^T).
+// the K-major B operand T^T of W^T and, scaled by beta per column, of U~^T = V^T (T diag(beta))^T).
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int SET = 65536;
     static constexpr int KP = 0, QP = 16384, KM = 32768, PF = 49152, TF = 57344;
     static constexpr int T_LBO = 1024, T_BYTES = 8192;
-    static constexpr int VB = 131072;              // two beta V tiles (channel-major, values)
-    static constexpr int AT = 163840;              // A, fp16, for the inverse
-    static constexpr int GS = 172032;              // two g staging tiles ([64][128] bf16, TMA)
-    static constexpr int OS = 204800;              // output staging (two swizzled 64 x 64 bf16 tiles)
+    static constexpr int VB = 131072;              // two v tiles, core matrices [value group][position][8]
+    static constexpr int GS = 163840;              // two g staging tiles ([64][128] bf16, TMA)
+    static constexpr int OS = 196608;              // output staging (two swizzled 64 x 64 bf16 tiles)
     static constexpr int SCR = 0;                  // (chunk_ap_direct uses the set's KM, PF, TF)
-    static constexpr int MISC = 221184;
+    static constexpr int MISC = 212992;
     static constexpr int QK_BYTES = 2 * 16384;     // q and k of one chunk
 };
 template <> struct Plan<MODE_STATE> {
@@ -108,11 +107,10 @@ template <> struct Plan<MODE_STATE> {
     static constexpr int KP = 0, QP = -1, KM = 16384, PF = 0, TF = 32768;   // no q, no P
     static constexpr int T_LBO = 1024, T_BYTES = 8192;
     static constexpr int VB = 81920;
-    static constexpr int AT = 114688;
-    static constexpr int GS = 122880;
-    static constexpr int SCR = 155648;             // 32 KB scratch of chunk_ap_direct
+    static constexpr int GS = 114688;
+    static constexpr int SCR = 147456;             // 32 KB scratch of chunk_ap_direct
     static constexpr int OS = 0;                   // (no output)
-    static constexpr int MISC = 188416;
+    static constexpr int MISC = 180224;
     static constexpr int QK_BYTES = 16384;         // k of one chunk
 };
 // MISC sub-layout
@@ -166,6 +164,15 @@ __device__ __forceinline__ uint4 pack8_f16(const float* f)
 #pragma unroll
     for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
     return u;
+}
+
+// Two fp32 values -> a packed pair of the input type (bf16 or fp16)
+template <typename TQ> __device__ __forceinline__ uint32_t pack2_in(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2_in<__half>(float lo, float hi) { return pack_f16x2(lo, hi); }
+template <> __device__ __forceinline__ uint32_t pack2_in<__nv_bfloat16>(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Two adjacent 2-byte input elements -> fp32
@@ -288,7 +295,7 @@ __device__ __forceinline__ void st_pair(uint8_t* tile, int ig, int cp, const uin
 // sum_c q_ic k_jc 2^{b_ic - b_jc} (j <= i), every exponential <= 1 formed directly.  The
 // raw k (and q) tiles are still in KP (QP); `scr` holds the fp32 table b[64][128] (base
 // 2, from the chunk start), written by the caller.  Writes A (fp16) to `at` and P to `pf`
-// in the cm64 layout (P zero above the diagonal).  Called by the 128 threads of the
+// in the cm64 layout (both zero above the diagonal).  Called by the 128 threads of the
 // prologue role (thread: row i, two 16-column blocks) after a barrier (bar_id) that
 // publishes the table; ends with that barrier passed.
 template <bool OUT, typename TQ>
@@ -367,13 +374,14 @@ __device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* 
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const int j0 = 16 * (2 * jh + pass) + 8 * half;
-            if (16 * (2 * jh + pass) <= i) *reinterpret_cast<uint4*>(at + cm64(i, j0)) = resA[pass][half];
+            *reinterpret_cast<uint4*>(at + cm64(i, j0)) = resA[pass][half];
             if (OUT) *reinterpret_cast<uint4*>(pf + cm64(i, j0)) = resP[pass][half];
         }
 }
 
-// Inverse T = (I + A)^{-1} of the strictly lower 64 x 64 A (fp16 at Ah, cm64 layout) into
-// the set's T tile (cmT layout, lower blocks only; its upper blocks stay zero).
+// Inverse T = (I + A)^{-1} of the strictly lower 64 x 64 A, in place: A (fp16, zero above
+// the diagonal) is in the T tile, whose cmT layout equals cm64 for T_LBO = 1024, and each
+// block of A is read before the block of T at its place is written.
 // Diagonal 16x16 blocks (warp w4 owns block w4): with N = A_ww (strictly lower, N^16 = 0),
 // (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8) on warp MMAs.  Then the off-diagonal
 // blocks by halves of the matrix (a work item: one 8-column half of one 16x16 block; X
@@ -382,8 +390,10 @@ __device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* 
 //   level 2: X_IJ = sum_{K=J}^{1} A_IK T_KJ  (I = 2, 3; J = 0, 1), then T_IJ = -sum_{K=2}^{I} T_IK X_KJ
 // Called by the 4 warps (128 threads) of the inverse role; barriers on bar_id.
 template <int T_LBO>
-__device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint32_t xs, int w4, int lane, int bar_id)
+__device__ __forceinline__ void invert_unit_lower(uint32_t Tt, uint32_t xs, int w4, int lane, int bar_id)
 {
+    static_assert(T_LBO == 1024, "A and T share the tile layout");
+    const uint32_t Ah = Tt;
     auto cmT = [](int i, int j) -> uint32_t { return (j >> 3) * T_LBO + (i >> 3) * 128 + (i & 7) * 16; };
     const int g = lane >> 2, q = lane & 3;
     {
@@ -468,6 +478,7 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Ah, uint32_t Tt, uint
         uint32_t aA[4], bT[2], bX[2], aT[4];
         float x[4] = {0.f, 0.f, 0.f, 0.f}, tt[4] = {0.f, 0.f, 0.f, 0.f};
         a_frag(aA, Ah, I, J, false);
+        named_sync(bar_id, 128);   // both halves of A_IJ are read before T_IJ's halves are written
         ldsm_x2_t(bT, Tt + cmT(16 * J + (lane & 7) + 8 * ((lane >> 3) & 1), N0));
         mma16816(x, aA, bT);
         put_x(scr_of(w4), x);
@@ -625,10 +636,10 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_arrive_expect_tx(&bars[B_TG + x], 16384);
         tma_load_3d(sm + PL::GS + x * 16384, &tm_g, &bars[B_TG + x], 0, h, (int)(rowbase + n * C));
     };
-    auto tma_v = [&](int n) {
+    auto tma_v = [&](int n) {   // v in core matrices: [value group][position][8 values]
         const int x = (n - n0) & 1;
         mbar_arrive_expect_tx(&bars[B_TV + x], 16384);
-        tma_load_3d(sm + PL::VB + x * 16384, &tm_v, &bars[B_TV + x], 0, h, (int)(rowbase + n * C));
+        tma_load_4d(sm + PL::VB + x * 16384, &tm_v, &bars[B_TV + x], 0, (int)(rowbase + n * C), 0, h);
     };
     const TQ* tq = nullptr;
 
@@ -709,14 +720,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     run = __ffma2_rn(in2(gw, (const __nv_bfloat16*)nullptr), l2e, run);
                     *reinterpret_cast<float2*>(reinterpret_cast<float*>(scr) + i * D + 2 * cp) = run;
                 }
-                // the A tile is free once the inverse role is done with chunk kc-1
-                if (rt == 0 && kc >= 1) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
                 named_sync(BAR_P, NR);
-                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBk, sm + PL::AT,
+                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBk, set + PL::TF,
                                          OUT ? set + PL::PF : nullptr, rt, t0, Tq, BAR_P);
-                if (OUT)   // the table covered the T tile: its upper blocks must read zero again
-                    for (int e = rt; e < PL::T_BYTES / 16; e += NR)
-                        *reinterpret_cast<uint4*>(set + PL::TF + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
             }
             // ---- beta K+, Q+ in place, K-; per 8-row block, the 64 threads of a row half read
             // their raw rows before any of them rewrites the block they share -----------------
@@ -786,8 +792,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     g_issued = kc + 3;
                 }
                 if (!direct) {
-                    // A|P's TMEM columns (and the A tile): free once the inverse role has read
-                    // chunk kc-1's W^T
+                    // A|P's TMEM columns: free once the inverse role has read chunk kc-1's W^T
                     if (kc >= 1) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
                     tc_fence_after();
                     // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the
@@ -830,19 +835,18 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const int col = 8 * g8 + j;
                             f[j] = (isP ? (col <= i) : (col < i)) ? v[8 * g8 + j] : 0.f;
                         }
-                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 8 * g8) : sm + PL::AT + cm64(i, 8 * g8);
+                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 8 * g8) : set + PL::TF + cm64(i, 8 * g8);
                         *reinterpret_cast<uint4*>(dst) = pack8_f16(f);
                     }
                 }
                 tc_fence_before();
                 named_sync(BAR_I, NR);
             }
-            invert_unit_lower<T_LBO>(sbase + PL::AT, sset + PL::TF, sbase + PL::MISC + M_XS, q4, lane, BAR_I);
+            invert_unit_lower<T_LBO>(sset + PL::TF, sbase + PL::MISC + M_XS, q4, lane, BAR_I);
             fence_async_smem();
             tc_fence_before();
             named_sync(BAR_I, NR);
             if (rt == 0) {
-                mbar_arrive(&bars[B_INV + s]);   // T ready
                 tc_fence_after();
                 // W^T = (beta K+)^T T^T: M = 128 channels, N = 64 positions, K = 64 positions
                 const uint32_t id = idesc_f16(128, 64, false, false);
@@ -864,10 +868,30 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     *reinterpret_cast<uint4*>(set + PL::KP + g8 * 2048 + (c >> 3) * 128 + (c & 7) * 16) = pack8_f16(f);
                 }
             }
+            {   // T -> T diag(beta) in the input type, in place (the W^T MMA has read T): the B
+                // operand of U~^T = V^T (T diag(beta))^T, with V as it landed
+                const uint16_t* sBk = sBeta + (kc & 3) * C;
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int e = 4 * rt + e4;                       // 16-byte piece: 8 consecutive columns
+                    const int j0 = 8 * (e >> 6);
+                    uint4* pc = reinterpret_cast<uint4*>(set + PL::TF + 16 * e);
+                    const uint4 u = *pc;
+                    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 tv = unpack_f16x2(uw[m]);
+                        ow[m] = pack2_in<TQ>(tv.x * bf16_bits_to_f32(sBk[j0 + 2 * m]), tv.y * bf16_bits_to_f32(sBk[j0 + 2 * m + 1]));
+                    }
+                    *pc = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+            }
             fence_async_smem();
             tc_fence_before();
             named_sync(BAR_I, NR);
             if (rt == 0) {
+                mbar_arrive(&bars[B_INV + s]);   // T diag(beta) ready
                 // every tile of the set is ready (the test hook withholds chunk 0's signal)
                 if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
                 mbar_arrive(&bars[B_APWF]);   // A|P's TMEM columns may be reused
@@ -1055,43 +1079,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         float gam = 1.f;
         if (OUT && gate && gamma) gam = gamma[(size_t)h * D + j];
-        // beta V of chunk x in place (v landed in beta V tile x & 1): thread = channel pair x
-        // 32 rows; every raw row of a 16-row band is read before the band is rewritten
-        auto beta_v = [&](int x) {
-            const int vb = x & 1, t0x = (n0 + x) * C, cp = rt & 63, rh = rt >> 6;
-            const int nvx = min(C, Tq - t0x);
-            group_wait(&bars[B_TV + vb], (x >> 1) & 1, ab, rt == 0, BAR_Y);
-            uint8_t* tile = sm + PL::VB + vb * 16384;
-            const uint16_t* sBx = sBeta + (x & 3) * C;
-#pragma unroll 1
-            for (int band = 0; band < 2; ++band) {
-                const int rb = 32 * rh + 16 * band;
-                uint32_t vR[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    vR[r] = rb + r < nvx ? *reinterpret_cast<const uint32_t*>(tile + (rb + r) * 256 + 4 * cp) : 0u;
-                named_sync(BAR_Y2 + rh, 64);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pv[2][4];
-                    float2 lv = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int r8 = 0; r8 < 8; ++r8) {
-                        const int r = 8 * half + r8;
-                        const float bi = bf16_bits_to_f32(sBx[rb + r]);
-                        const float2 vbv = __fmul2_rn(in2(vR[r], tq), make_float2(bi, bi));
-                        if (r8 & 1) {
-                            pv[0][r8 >> 1] = pack_f16x2(lv.x, vbv.x);
-                            pv[1][r8 >> 1] = pack_f16x2(lv.y, vbv.y);
-                        } else {
-                            lv = vbv;
-                        }
-                    }
-                    st_pair(tile, (rb >> 3) + half, cp, pv);
-                }
-            }
-            fence_async_smem();
-        };
         // zero the O columns of [U | O] buffer x (U~ writes only the U columns)
         auto zero_o = [&](int x) {
             if (!OUT) return;
@@ -1101,16 +1088,17 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_st32(tl + TM::UO + 128 * (x & 1) + 64, z);
             tmem_st32(tl + TM::UO + 128 * (x & 1) + 96, z);
         };
-        // U~^T = (beta V)^T T^T into the chunk's U columns
+        // U~^T = V^T (T diag(beta))^T into the chunk's U columns: V^T straight from the v tile
+        // (M = values, MN-major core matrices), operands in the input type
         auto issue_u = [&](int x) {
             const int s = x & 1;
             const uint32_t sset = sbase + s * PL::SET, vbt = sbase + PL::VB + s * 16384;
-            const uint32_t id = idesc_f16(128, 64, false, false);
+            const uint32_t id = idesc_f16(128, 64, true, false, false, std::is_same<TQ, __nv_bfloat16>::value);
             const uint32_t d = tmem + (OUT ? TM::UO + 128 * s : TM::UACC);
             for (int kk = 0; kk < 4; ++kk)
-                umma_f16(d, sdesc(vbt + 4096 * kk, 2048, 128), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
+                umma_f16(d, sdesc(vbt + 256 * kk, 128, 1024), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
                          kk > 0);
-            umma_commit(&bars[B_VE + s]);   // U~ done: the beta V tile may be refilled
+            umma_commit(&bars[B_VE + s]);   // U~ done: the v tile may be refilled
         };
         // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
         auto out_rows = [&](int x) {
@@ -1205,7 +1193,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
         };
-        if (nk > 0) beta_v(0);
         zero_o(0);
         if (nk > 1) zero_o(1);
         tc_fence_before();
@@ -1216,6 +1203,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int n = n0 + kc, s = kc & 1;
             if (mma && !u_done) {
                 thread_wait(&bars[B_INV + s], (kc >> 1) & 1, ab);
+                thread_wait(&bars[B_TV + s], (kc >> 1) & 1, ab);   // this chunk's v has landed
                 // MODE_STATE: one U accumulator; the chain of chunk kc-1 has read it once its
                 // last master update is done
                 if (!OUT && kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
@@ -1227,8 +1215,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 out_rows(kc - 1);
                 if (kc + 1 < nk) zero_o(kc + 1);
             }
-            // ---- beta V of chunk kc+1 ------------------------------------------------------------
-            if (kc + 1 < nk) beta_v(kc + 1);
             tc_fence_before();
             named_sync(BAR_Y, NR);
             // ---- loads: chunk kc+2's k (and q) once the [U | O] MMA of chunk kc has read the set's
@@ -1248,7 +1234,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // U~ of the next chunk now, if its T is ready (else at the top of the next step)
             if (mma) {
                 u_done = false;
-                if (OUT && kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
+                if (OUT && kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1) &&
+                    mbar_try_wait(&bars[B_TV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
                     tc_fence_after();
                     issue_u(kc + 1);
                     u_done = true;
@@ -1422,6 +1409,22 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, i
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// v [B*T, H, 128] as 4-D (8 values, tokens, 16 value groups, heads), box 8 x 64 x 16 x 1:
+// a chunk lands as [value group][position][8 values], the MN-major core-matrix layout of
+// the A operand V^T (values = M, positions = K) of the U~ MMA.
+bool make_map_v(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B, int T, int H)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {8u, (cuuint64_t)B * (cuuint64_t)T, (cuuint64_t)(D / 8), (cuuint64_t)H};
+    const cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, 16u, (cuuint64_t)D * 2};
+    const cuuint32_t box[4] = {8u, (cuuint32_t)C, (cuuint32_t)(D / 8), 1u};
+    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+    return fn(m, dt, 4, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // bf16 output o as a 4-D tensor (channels, heads, tokens, rows), box = 64 channels x
 // 1 head x 64 tokens, 128-byte swizzle.  Tokens past T are clipped by the T dimension, so
 // a ragged last chunk never writes into the next row.
@@ -1481,7 +1484,7 @@ bool build_maps(const KdaArgs& a, Maps& mp)
     const CUtensorMapDataType dq =
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_map(&mp.q, a.q, dq, a.B, a.T, a.H) || !make_map(&mp.k, a.k, dq, a.B, a.T, a.H) ||
-        !make_map(&mp.v, a.v, dq, a.B, a.T, a.H) ||
+        !make_map_v(&mp.v, a.v, dq, a.B, a.T, a.H) ||
         !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
         return false;
     if (a.out_t == ET_F32 || !a.o) {
@@ -1780,7 +1783,7 @@ cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int*
         std::is_same<TQ, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     Maps mp;
     if (!make_map(&mp.q, a.q, dq, 1, a.T, a.H) || !make_map(&mp.k, a.k, dq, 1, a.T, a.H) ||
-        !make_map(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
+        !make_map_v(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
         return cudaErrorInvalidValue;
     if (a.out_t == ET_F32) mp.o = mp.q;
     else if (!make_map_o(&mp.o, a.o, 1, a.T, a.H)) return cudaErrorInvalidValue;
