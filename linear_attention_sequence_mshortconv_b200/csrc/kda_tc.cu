@@ -136,7 +136,6 @@ enum Bar {
     B_VE = 14,      // [2] beta V tile x: the U~ MMA that read it is done
     B_O = 16,       // [2] [U | O] buffer x: the chunk's O is complete
     B_AP = 18, B_W = 19, B_U = 20, B_U2 = 21, B_S = 22,
-    B_APWF = 23,    // the inverse role has read W^T out of A|P's TMEM columns
     B_DRAIN = 24,   // [4] one per MMA-issuing role, after a timeout
     NBAR = 28
 };
@@ -528,8 +527,9 @@ __device__ __forceinline__ uint32_t swz_off(int i, int col) { return (uint32_t)(
 // Four roles of 4 warps each (role = warp / 4; warp w4 = warp % 4 also names the TMEM lane
 // quarter it may access):
 //   P (role 0)  prologue: log-decay prefix and references of chunk n, the K+ / Q+ / K- tiles
-//               (or A and P on CUDA cores for a wide chunk), the A|P MMA.
-//   I (role 1)  inverse: A and P out of TMEM, T = (I + A)^{-1}, W^T MMA, -W^T into the set.
+//               (or A and P on CUDA cores for a wide chunk).
+//   I (role 1)  inverse: the A|P MMA, A and P out of TMEM, T = (I + A)^{-1}, W^T MMA, -W^T and
+//               T diag(beta) into the set.
 //   X (role 2)  state chain: S^ from the master, the [U | O] MMA, U -> fp16, the master and O
 //               MMAs; one thread per TMEM lane (value column).
 //   Y (role 3)  auxiliary: U~ MMA, zeroing the O accumulator, the output rows (TMA store
@@ -791,18 +791,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tma_g(n + 2);
                     g_issued = kc + 3;
                 }
-                if (!direct) {
-                    // A|P's TMEM columns: free once the inverse role has read chunk kc-1's W^T
-                    if (kc >= 1) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
-                    tc_fence_after();
-                    // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the
-                    // state pass reads K- as rows 64-127 and ignores them)
-                    const uint32_t id = idesc_f16(128, 64, true, true);
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
-                                 sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
-                    umma_commit(&bars[B_AP]);
-                }
             }
         }
         // after a timeout some requested g tiles may not have been waited for: let them land
@@ -819,6 +807,16 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t sset = sbase + s * PL::SET;
             group_wait(&bars[B_SC + s], (kc >> 1) & 1, ab, rt == 0, BAR_I);   // the prologue is done
             if (!sDirect[s]) {
+                if (rt == 0) {
+                    // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the state
+                    // pass reads K- as rows 64-127 and ignores them).  A|P's TMEM columns are free:
+                    // this role read the previous chunk's W^T out of them.
+                    const uint32_t id = idesc_f16(128, 64, true, true);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
+                                 sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
+                    umma_commit(&bars[B_AP]);
+                }
                 group_wait(&bars[B_AP], n_ap & 1, ab, rt == 0, BAR_I);
                 ++n_ap;
                 // A (lanes 0-63) -> fp16 tile, P (lanes 64-127) -> the set's P tile
@@ -894,7 +892,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mbar_arrive(&bars[B_INV + s]);   // T diag(beta) ready
                 // every tile of the set is ready (the test hook withholds chunk 0's signal)
                 if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
-                mbar_arrive(&bars[B_APWF]);   // A|P's TMEM columns may be reused
             }
         }
     } else if (role == 2) {
