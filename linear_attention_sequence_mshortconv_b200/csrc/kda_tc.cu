@@ -86,64 +86,69 @@ constexpr float kRangeMax = 11.f;
 enum { MODE_STATE = 0, MODE_OUTPUT = 1 };
 
 // ---- shared-memory plan (bytes) --------------------------------------------------
-// Per buffer set (chunk parity): KP (k -> beta K+ -> -W^T) and QP (q -> Q+) as
-// channel-major tiles, QP directly after KP so [beta K+; Q+] and [-W^T | Q+^T] are single
-// 128-row operands; KM (K-); PF (P as the K-major B operand of O^T += U^T P^T); TF (T as
-// the K-major B operand T^T of W^T and, scaled by beta per column, of U~^T = V^T (T diag(beta))^T).
+// NSET buffer sets of per-chunk tiles; chunk x uses set x % NSET.  Per set: KP (k -> beta
+// K+ -> -W^T) and QP (q -> Q+) as channel-major tiles, QP directly after KP so [beta K+;
+// Q+] and [-W^T | Q+^T] are single 128-row operands; KM (g as TMA lands it -> K-); PF (P
+// as the K-major B operand of O^T += U^T P^T); TF (T as the K-major B operand T^T of W^T
+// and, scaled by beta per column, of U~^T = V^T (T diag(beta))^T).  Three sets keep three
+// chunks in flight (prologue, inverse, state chain), so the loads of a chunk have a whole
+// chunk period to land.  One v tile (core matrices [value group][position][8]).
+constexpr int NSET = 3;
 template <int MODE> struct Plan;
 template <> struct Plan<MODE_OUTPUT> {
     static constexpr int SET = 65536;
     static constexpr int KP = 0, QP = 16384, KM = 32768, PF = 49152, TF = 57344;
     static constexpr int T_LBO = 1024, T_BYTES = 8192;
-    static constexpr int VB = 131072;              // two v tiles, core matrices [value group][position][8]
-    static constexpr int GS = 163840;              // two g staging tiles ([64][128] bf16, TMA)
-    static constexpr int OS = 196608;              // output staging (two swizzled 64 x 64 bf16 tiles)
-    static constexpr int SCR = 0;                  // (chunk_ap_direct uses the set's KM, PF, TF)
-    static constexpr int MISC = 212992;
-    static constexpr int QK_BYTES = 2 * 16384;     // q and k of one chunk
+    static constexpr int VB = NSET * SET;
+    static constexpr int SCR = -1;                 // (chunk_ap_direct's table: the set's PF and TF)
+    static constexpr int MISC = VB + 16384;
+    static constexpr int LOAD_BYTES = 3 * 16384;   // q, k and g of one chunk
 };
 template <> struct Plan<MODE_STATE> {
     static constexpr int SET = 40960;
     static constexpr int KP = 0, QP = -1, KM = 16384, PF = 0, TF = 32768;   // no q, no P
     static constexpr int T_LBO = 1024, T_BYTES = 8192;
-    static constexpr int VB = 81920;
-    static constexpr int GS = 114688;
-    static constexpr int SCR = 147456;             // 32 KB scratch of chunk_ap_direct
-    static constexpr int OS = 0;                   // (no output)
-    static constexpr int MISC = 180224;
-    static constexpr int QK_BYTES = 16384;         // k of one chunk
+    static constexpr int VB = NSET * SET;
+    static constexpr int SCR = VB + 16384;         // 16 KB table of chunk_ap_direct
+    static constexpr int MISC = SCR + 16384;
+    static constexpr int LOAD_BYTES = 2 * 16384;   // k and g of one chunk
 };
 // MISC sub-layout
-constexpr int M_BETA = 0;        // bf16[4][64]   beta of chunk x in slot x & 3 (written two chunks ahead)
-constexpr int M_BRAW = 512;      // uint32[64]    the head pair's beta words as cp.async lands them
-constexpr int M_TOT = 768;       // float[2][128] per-32-row sums of g log2(e)
-constexpr int M_SC = 1792;       // float[2][3][128] per set: S^ scale, master scale, carry after
-constexpr int M_XS = 4864;       // 8 x 512 B per-item 16x16 fp16 scratch of the inverse
-constexpr int M_BAR = 8960;      // mbarriers, see Bar
-constexpr int M_TMEM = 9184;     // uint32 TMEM base
-constexpr int M_ABORT = 9188;    // int
-constexpr int M_DIRECT = 9192;   // int[2] per set: its chunk's A and P came from chunk_ap_direct
-constexpr int M_RED = 9200;      // float[4][64] per-row sums of squares (gated output)
-constexpr int MISC_BYTES = 10224;
+constexpr int NBETA = 8;         // beta slots (written two chunks ahead, read up to two behind)
+constexpr int M_BETA = 0;        // bf16[NBETA][64]  beta of chunk x in slot x % NBETA
+constexpr int M_BRAW = 1024;     // uint32[64]    the head pair's beta words as cp.async lands them
+constexpr int M_TOT = 1280;      // float[2][128] per-32-row sums of g log2(e)
+constexpr int M_SC = 2304;       // float[NSET][3][128] per set: S^ scale, master scale, carry after
+constexpr int M_XS = 6912;       // 8 x 512 B per-item 16x16 fp16 scratch of the inverse
+constexpr int M_BAR = 11008;     // mbarriers, see Bar
+constexpr int M_TMEM = 11264;    // uint32 TMEM base
+constexpr int M_ABORT = 11268;   // int
+constexpr int M_DIRECT = 11272;  // int[NSET] per set: its chunk's A and P came from chunk_ap_direct
+constexpr int M_RED = 11296;     // float[4][64] per-row sums of squares (gated output)
+constexpr int MISC_BYTES = 12320;
 enum Bar {
-    B_TG = 0,       // [2] g tile landed (staging tile x)
-    B_TQK = 2,      // [2] k (and q) landed in set s
-    B_TV = 4,       // [2] v landed in beta V tile x
-    B_SC = 6,       // [2] set s: prologue done (scales, direct flag, K+ / Q+ / K- tiles, beta)
-    B_INV = 8,      // [2] set s: T ready
-    B_PRO = 10,     // [2] set s: every tile ready (-W^T written)
-    B_EMPTY = 12,   // [2] set s: the chain's last MMA on it is done
-    B_VE = 14,      // [2] beta V tile x: the U~ MMA that read it is done
-    B_O = 16,       // [2] [U | O] buffer x: the chunk's O is complete
-    B_AP = 18, B_W = 19, B_U = 20, B_U2 = 21, B_S = 22,
+    B_LD = 0,       // [3] set s: q, k, g of its chunk landed
+    B_TV = 3,       // the v tile landed
+    B_VE = 4,       // the U~ MMA that read the v tile is done
+    B_SC = 5,       // [3] set s: prologue done (scales, direct flag, K+ / Q+ / K- tiles, beta)
+    B_INV = 8,      // [3] set s: T ready
+    B_PRO = 11,     // [3] set s: every tile ready (W^T written)
+    B_EMPTY = 14,   // [3] set s: the chain's last MMA on it is done
+    B_O = 17,       // [2] [U | O] buffer x: the chunk's O is complete
+    B_AP = 19, B_W = 20, B_U = 21, B_U2 = 22, B_S = 23,
     B_DRAIN = 24,   // [4] one per MMA-issuing role, after a timeout
-    NBAR = 28
+    B_APWF = 28,    // the output role has read W^T out of A|P's TMEM columns
+    NBAR = 29
 };
+// set of chunk x (counted from the segment start) and the phase parity of its set barriers
+__device__ __forceinline__ int set_of(int x) { return x % NSET; }
+__device__ __forceinline__ uint32_t set_par(int x) { return (uint32_t)(x / NSET) & 1u; }
 static_assert(M_BAR + NBAR * 8 <= M_TMEM, "barrier block");
+static_assert(M_DIRECT + 4 * NSET <= M_RED && M_SC + NSET * 3 * 128 * 4 <= M_XS, "misc block");
 static_assert(M_RED % 16 == 0 && M_RED + 1024 <= MISC_BYTES, "misc block");
 
 template <int MODE> constexpr int smem_bytes() { return Plan<MODE>::MISC + MISC_BYTES; }
-static_assert(smem_bytes<MODE_OUTPUT>() <= 232448, "shared memory");
+static_assert(smem_bytes<MODE_OUTPUT>() <= 232448 && smem_bytes<MODE_STATE>() <= 232448, "shared memory");
 
 // TMEM columns.
 //   MODE_OUTPUT: master S^T [0,128) | S^ fp16 [128,192) | [U|O] x2 [192,448) | A|P, W^T [448,512)
@@ -291,20 +296,27 @@ __device__ __forceinline__ void st_pair(uint8_t* tile, int ig, int cp, const uin
 
 // A (and P) of one chunk on CUDA cores, for a chunk whose decay range is too wide for a
 // single reference: A_ij = beta_i sum_c k_ic k_jc 2^{b_ic - b_jc} (j < i) and P_ij =
-// sum_c q_ic k_jc 2^{b_ic - b_jc} (j <= i), every exponential <= 1 formed directly.  The
-// raw k (and q) tiles are still in KP (QP); `scr` holds the fp32 table b[64][128] (base
-// 2, from the chunk start), written by the caller.  Writes A (fp16) to `at` and P to `pf`
-// in the cm64 layout (both zero above the diagonal).  Called by the 128 threads of the
-// prologue role (thread: row i, two 16-column blocks) after a barrier (bar_id) that
-// publishes the table; ends with that barrier passed.
-template <bool OUT, typename TQ>
-__device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* ktile, const uint8_t* qtile,
-                                             const uint16_t* sBeta, uint8_t* at, uint8_t* pf, int rt, int t0, int Tq,
-                                             int bar_id)
+// sum_c q_ic k_jc 2^{b_ic - b_jc} (j <= i), every exponential <= 1 formed directly.  In
+// the buffer set `set` the raw k (and q) tiles are still in KP (QP) and g in KM; `tot`
+// holds each channel's sum of g log2(e) over rows 0-31; nv rows are inside the sequence.
+// The fp32 table b[64][64] of one 64-channel half (base 2, from the chunk start) is built
+// in `scr` (16 KB) for each half in turn.  Writes A (fp16) to TF and P to PF in the cm64
+// layout (both zero above the diagonal); `scr` may overlap them.  Called by the 128
+// threads of the prologue role (thread: row i, two 16-column blocks); barriers on BAR_P.
+template <int MODE, typename TQ>
+__device__ __noinline__ void chunk_ap_direct(uint8_t* set, uint8_t* scr, const float* tot, const uint16_t* sBeta,
+                                             int rt, int nv)
 {
-    const float* bT = reinterpret_cast<const float*>(scr);
+    using PL = Plan<MODE>;
+    constexpr bool OUT = MODE == MODE_OUTPUT;
+    constexpr int bar_id = BAR_P;
+    const uint8_t* gst = set + PL::KM;
+    const uint8_t* ktile = set + PL::KP;
+    const uint8_t* qtile = OUT ? set + PL::QP : set + PL::KP;
+    uint8_t* at = set + PL::TF;
+    uint8_t* pf = set + PL::PF;
+    float* bT = reinterpret_cast<float*>(scr);
     const int i = rt & 63, jh = rt >> 6;
-    const int nv = min(C, Tq - t0);          // rows of this chunk inside the sequence
     const float bi = bf16_bits_to_f32(sBeta[i]);
     uint4 resA[2][2], resP[2][2];            // fp16 results of the two blocks (written last)
     const TQ* tq = nullptr;
@@ -313,43 +325,60 @@ __device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* 
         float accA[16], accP[16];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) accA[jj] = accP[jj] = 0.f;
-        if (16 * cq <= i && i < nv) {
-            for (int c8 = 0; c8 < 16; ++c8) {
-                const uint4 ku = *reinterpret_cast<const uint4*>(ktile + i * 256 + c8 * 16);
-                const uint4 qu = OUT ? *reinterpret_cast<const uint4*>(qtile + i * 256 + c8 * 16) : make_uint4(0, 0, 0, 0);
-                const float4 b0 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8);
-                const float4 b1 = *reinterpret_cast<const float4*>(bT + i * D + 8 * c8 + 4);
-                float ki[8], qi[8];
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-                {
-                    const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x = in2(kw[e], tq), y = in2(qw[e], tq);
-                        ki[2 * e] = x.x; ki[2 * e + 1] = x.y;
-                        qi[2 * e] = y.x; qi[2 * e + 1] = y.y;
-                    }
+        for (int hc = 0; hc < 2; ++hc) {
+            // the table of channels 64 hc .. 64 hc + 63: thread (channel cc, 32-row half)
+            named_sync(bar_id, 128);         // the previous table is no longer read
+            {
+                const int cc = rt & 63, rh2 = rt >> 6, c = 64 * hc + cc;
+                float run = rh2 ? tot[c] : 0.f;
+#pragma unroll 4
+                for (int r = 0; r < 32; ++r) {
+                    const int ii = 32 * rh2 + r;
+                    const float gv = ii < nv ? bf16_bits_to_f32(*reinterpret_cast<const uint16_t*>(gst + ii * 256 + 2 * c)) : 0.f;
+                    run = fmaf(gv, kLog2e, run);
+                    bT[ii * 64 + cc] = run;
                 }
-#pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                    const int j = 16 * cq + jj;
-                    if (j <= i) {
-                        const uint4 kj = *reinterpret_cast<const uint4*>(ktile + j * 256 + c8 * 16);
-                        const float4 c0 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8);
-                        const float4 c1 = *reinterpret_cast<const float4*>(bT + j * D + 8 * c8 + 4);
-                        const float bj[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                        const uint32_t kw[4] = {kj.x, kj.y, kj.z, kj.w};
-                        float sa = 0.f, sp = 0.f;
+            }
+            named_sync(bar_id, 128);
+            if (16 * cq <= i && i < nv) {
+                for (int c8h = 0; c8h < 8; ++c8h) {
+                    const int c8 = 8 * hc + c8h;
+                    const uint4 ku = *reinterpret_cast<const uint4*>(ktile + i * 256 + c8 * 16);
+                    const uint4 qu = OUT ? *reinterpret_cast<const uint4*>(qtile + i * 256 + c8 * 16) : make_uint4(0, 0, 0, 0);
+                    const float4 b0 = *reinterpret_cast<const float4*>(bT + i * 64 + 8 * c8h);
+                    const float4 b1 = *reinterpret_cast<const float4*>(bT + i * 64 + 8 * c8h + 4);
+                    float ki[8], qi[8];
+                    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                    {
+                        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const float2 kk = in2(kw[e], tq);
-                            const float d0 = ex2_approx(bv[2 * e] - bj[2 * e]) * kk.x;
-                            const float d1 = ex2_approx(bv[2 * e + 1] - bj[2 * e + 1]) * kk.y;
-                            sa = fmaf(ki[2 * e], d0, fmaf(ki[2 * e + 1], d1, sa));
-                            if (OUT) sp = fmaf(qi[2 * e], d0, fmaf(qi[2 * e + 1], d1, sp));
+                            const float2 x = in2(kw[e], tq), y = in2(qw[e], tq);
+                            ki[2 * e] = x.x; ki[2 * e + 1] = x.y;
+                            qi[2 * e] = y.x; qi[2 * e + 1] = y.y;
                         }
-                        accA[jj] += sa;
-                        accP[jj] += sp;
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int j = 16 * cq + jj;
+                        if (j <= i) {
+                            const uint4 kj = *reinterpret_cast<const uint4*>(ktile + j * 256 + c8 * 16);
+                            const float4 c0 = *reinterpret_cast<const float4*>(bT + j * 64 + 8 * c8h);
+                            const float4 c1 = *reinterpret_cast<const float4*>(bT + j * 64 + 8 * c8h + 4);
+                            const float bj[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                            const uint32_t kw[4] = {kj.x, kj.y, kj.z, kj.w};
+                            float sa = 0.f, sp = 0.f;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 kk = in2(kw[e], tq);
+                                const float d0 = ex2_approx(bv[2 * e] - bj[2 * e]) * kk.x;
+                                const float d1 = ex2_approx(bv[2 * e + 1] - bj[2 * e + 1]) * kk.y;
+                                sa = fmaf(ki[2 * e], d0, fmaf(ki[2 * e + 1], d1, sa));
+                                if (OUT) sp = fmaf(qi[2 * e], d0, fmaf(qi[2 * e + 1], d1, sp));
+                            }
+                            accA[jj] += sa;
+                            accP[jj] += sp;
+                        }
                     }
                 }
             }
@@ -367,7 +396,7 @@ __device__ __noinline__ void chunk_ap_direct(const uint8_t* scr, const uint8_t* 
             resP[pass][half] = pack8_f16(fp);
         }
     }
-    named_sync(bar_id, 128);   // the table may be overwritten (in MODE_OUTPUT it covers PF)
+    named_sync(bar_id, 128);   // the table may be overwritten (in MODE_OUTPUT it covers PF and TF)
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass)
 #pragma unroll
@@ -519,26 +548,157 @@ __device__ __forceinline__ void invert_unit_lower(uint32_t Tt, uint32_t xs, int 
     }
 }
 
-// bf16 output through TMA: O rows go into two 64-channel x 64-row tiles (128-byte rows,
-// 128-byte swizzle: 16-byte piece p of row i at i*128 + ((p ^ (i & 7)) * 16)).
-__device__ __forceinline__ uint32_t swz_off(int i, int col) { return (uint32_t)((col >> 6) * 8192 + i * 128 + ((((col & 63) >> 3) ^ (i & 7)) << 4) + (col & 7) * 2); }
+// 8 x 8 transpose of 16-bit values inside each group of 8 lanes.  Lane l (of the group)
+// holds row l as w[m] = (column 2m, column 2m + 1) (low half first); on return z[m] =
+// (row 2m, row 2m + 1) of column l.  Three exchange rounds (lane distance 4, 2, 1), each
+// moving half of the data: 6 shuffles.
+__device__ __forceinline__ void transpose8x8_b16(const uint32_t* w, uint32_t (&z)[4], int lane)
+{
+    const bool b = (lane & 4) != 0, c = (lane & 2) != 0, d = (lane & 1) != 0;
+    // distance 4: keep columns 4b .. 4b+3; A[0..1] = row l & ~4, A[2..3] = row l | 4
+    const uint32_t r0 = __shfl_xor_sync(0xffffffffu, b ? w[0] : w[2], 4);
+    const uint32_t r1 = __shfl_xor_sync(0xffffffffu, b ? w[1] : w[3], 4);
+    const uint32_t A0 = b ? r0 : w[0], A1 = b ? r1 : w[1], A2 = b ? w[2] : r0, A3 = b ? w[3] : r1;
+    // distance 2: keep column pair 2b + c; B[k] = row (l & 1) + 2k
+    const uint32_t q0 = __shfl_xor_sync(0xffffffffu, c ? A0 : A1, 2);
+    const uint32_t q1 = __shfl_xor_sync(0xffffffffu, c ? A2 : A3, 2);
+    const uint32_t B0 = c ? q0 : A0, B1 = c ? A1 : q0, B2 = c ? q1 : A2, B3 = c ? A3 : q1;
+    // distance 1: keep column l (the low halves if d = 0, the high halves if d = 1)
+    const uint32_t t0 = __shfl_xor_sync(0xffffffffu, d ? __byte_perm(B0, B1, 0x5410) : __byte_perm(B0, B1, 0x7632), 1);
+    const uint32_t t1 = __shfl_xor_sync(0xffffffffu, d ? __byte_perm(B2, B3, 0x5410) : __byte_perm(B2, B3, 0x7632), 1);
+    if (d) {
+        z[0] = __byte_perm(t0, B0, 0x7610);
+        z[1] = __byte_perm(t0, B1, 0x7632);
+        z[2] = __byte_perm(t1, B2, 0x7610);
+        z[3] = __byte_perm(t1, B3, 0x7632);
+    } else {
+        z[0] = __byte_perm(B0, t0, 0x5410);
+        z[1] = __byte_perm(B1, t0, 0x7610);
+        z[2] = __byte_perm(B2, t1, 0x5410);
+        z[3] = __byte_perm(B3, t1, 0x7610);
+    }
+}
+
+// 32 positions (32 hp0 ..) of this warp's 32 value columns, as -O, -> bf16 o rows by
+// 16-byte stores (sign restored): after an 8 x 8 transpose inside each group of 8 lanes, lane l of group g8 holds
+// values 8 g8 .. 8 g8 + 7 at position 8 blk + l.  row0: packed token of position 0.
+__device__ __forceinline__ void store_rows_bf16(const float (&v)[32], __nv_bfloat16* o, int64_t row0, int hp0, int nvx,
+                                                int H, int h, int q4, int lane)
+{
+    uint32_t wv[16];   // -v: the O columns hold -O
+#pragma unroll
+    for (int m = 0; m < 16; ++m) wv[m] = pack2_in<__nv_bfloat16>(v[2 * m], v[2 * m + 1]) ^ 0x80008000u;
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+        uint32_t z[4];
+        transpose8x8_b16(wv + 4 * blk, z, lane);
+        const int i = hp0 + 8 * blk + (lane & 7);
+        if (i < nvx) {
+            const size_t idx = ((size_t)row0 + i) * ((size_t)H * D) + (size_t)h * D + 32 * q4 + 8 * (lane >> 3);
+            *reinterpret_cast<uint4*>(o + idx) = make_uint4(z[0], z[1], z[2], z[3]);
+        }
+    }
+}
+
+// Parameters of the output rows that only the gated or fp32 output needs.
+struct OutParams {
+    const __nv_bfloat16* gate;
+    void* o;
+    float* red;        // float[4][64] shared scratch
+    float gam, eps;
+    int o_f32, H, h, q4, lane;
+};
+// Output rows of one chunk with the Eq. 15 output gate, or to an fp32 o; the plain bf16
+// case stays inline in the kernel.  ocol: this warp's TMEM address of the chunk's -O^T
+// (lane = value column, 64 position columns).  Called by the 128 threads of the output
+// role; the gated case syncs them once (BAR_Y).
+__device__ __forceinline__ void out_rows_general(const OutParams* op, uint32_t ocol, int64_t row0, int nvx)
+{
+    const __nv_bfloat16* gate = op->gate;
+    void* o = op->o;
+    float* red = op->red;
+    const float gam = op->gam, eps = op->eps;
+    const int o_f32 = op->o_f32, H = op->H, h = op->h, q4 = op->q4, lane = op->lane;
+    const int j = 32 * q4 + lane;
+    float inv_lo = 0.f, inv_hi = 0.f;   // per-position inverse RMS (gated output)
+    if (gate) {
+        // y = Sigmoid(gate) * gamma * RMSNorm over the head's values (Eq. 15, output side).
+        // Per position, the sum of squares over this warp's 32 values by a transposing
+        // butterfly (lane l ends with position 32*hp + l), then over the 4 lane quarters.
+        for (int hp = 0; hp < 2; ++hp) {
+            float sq[32];
+            tmem_ld32(ocol + 32 * hp, sq);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) sq[u] = sq[u] * sq[u];
+#pragma unroll
+            for (int sft = 16; sft >= 1; sft >>= 1) {
+                const bool up = (lane & sft) != 0;
+#pragma unroll
+                for (int k = 0; k < sft; ++k) {
+                    const float send = up ? sq[k] : sq[k + sft];
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
+                    sq[k] = (up ? sq[k + sft] : sq[k]) + recv;
+                }
+            }
+            red[q4 * C + 32 * hp + lane] = sq[0];
+        }
+        named_sync(BAR_Y, NR);
+        const float m0 = (red[lane] + red[C + lane] + red[2 * C + lane] + red[3 * C + lane]) * (1.f / D) + eps;
+        const float m1 =
+            (red[32 + lane] + red[C + 32 + lane] + red[2 * C + 32 + lane] + red[3 * C + 32 + lane]) * (1.f / D) + eps;
+        inv_lo = m0 > 0.f ? rsqrtf(m0) : 0.f;
+        inv_hi = m1 > 0.f ? rsqrtf(m1) : 0.f;
+    }
+    for (int hp = 0; hp < 2; ++hp) {
+        float v[32];
+        tmem_ld32(ocol + 32 * hp, v);
+        if (gate) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                v[u] = -v[u];
+                const float iu = __shfl_sync(0xffffffffu, hp ? inv_hi : inv_lo, u);
+                const int i = 32 * hp + u;
+                float gv = 0.f;
+                if (i < nvx) gv = __bfloat162float(gate[(((size_t)row0 + i) * H + h) * D + j]);
+                v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
+            }
+        }
+        if (!o_f32) {
+            if (gate) {   // store_rows_bf16 negates
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v[u] = -v[u];
+            }
+            store_rows_bf16(v, reinterpret_cast<__nv_bfloat16*>(o), row0, 32 * hp, nvx, H, h, q4, lane);
+        } else {
+            // fp32: a warp writes 32 consecutive values of a position
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+                const int i = 32 * hp + u;
+                if (i < nvx) reinterpret_cast<float*>(o)[((size_t)row0 + i) * ((size_t)H * D) + (size_t)h * D + j] = gate ? v[u] : -v[u];
+            }
+        }
+    }
+}
 
 // The kernel ---------------------------------------------------------------------------
 // Four roles of 4 warps each (role = warp / 4; warp w4 = warp % 4 also names the TMEM lane
 // quarter it may access):
 //   P (role 0)  prologue: log-decay prefix and references of chunk n, the K+ / Q+ / K- tiles
 //               (or A and P on CUDA cores for a wide chunk).
-//   I (role 1)  inverse: the A|P MMA, A and P out of TMEM, T = (I + A)^{-1}, W^T MMA, -W^T and
+//   I (role 1)  inverse: the A|P MMA, A and P out of TMEM, T = (I + A)^{-1}, W^T MMA,
 //               T diag(beta) into the set.
 //   X (role 2)  state chain: S^ from the master, the [U | O] MMA, U -> fp16, the master and O
-//               MMAs; one thread per TMEM lane (value column).
-//   Y (role 3)  auxiliary: U~ MMA, zeroing the O accumulator, the output rows (TMA store
-//               from a staging tile), beta V, and the TMA loads of k, q, v.
-template <int MODE, typename TQ>
+//               MMAs; one thread per TMEM lane (value column).  Its MMA thread also issues
+//               the TMA loads of q, k, g as soon as a set is free.
+//   Y (role 3)  auxiliary: W^T out of TMEM into the set, U~ MMA, zeroing the O
+//               accumulator, the output rows (16-byte stores after an in-register
+//               transpose), and the TMA loads of v.
+// GOUT (MODE_OUTPUT only): the gated or fp32 output path is compiled in; without it the
+// kernel writes plain bf16 rows.
+template <int MODE, typename TQ, bool GOUT>
 __global__ void __launch_bounds__(NT, 1)
 kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-              const __grid_constant__ CUtensorMap tm_o,
               const __nv_bfloat16* __restrict__ beta, void* __restrict__ o, int o_f32,
               const float* __restrict__ S_in, int s_in_per_segment, float* __restrict__ maps,
               float* __restrict__ S_T, int B, int T, int H, int P, int L, int* status, int dbg_drop,
@@ -579,11 +739,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         last = p == P - 1;
     }
     const int nk = max(0, n1 - n0);
-    // the bf16 output leaves by TMA store through a [B, T, H, 128] map that clips at the
-    // end of a row; packed samples share one row, so a chunk that runs past its sample's
-    // end is written with plain stores instead
-    const int o_b = items ? 0 : seq;
-    const int64_t o_t = items ? rowbase : 0;
 
     uint16_t* sBeta = reinterpret_cast<uint16_t*>(sm + PL::MISC + M_BETA);
     uint32_t* sBRaw = reinterpret_cast<uint32_t*>(sm + PL::MISC + M_BRAW);
@@ -607,8 +762,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_alloc(sTmem, 512);
         tmem_relinquish();
     }
-    // T tiles of both sets start zero (their upper blocks stay zero)
-    for (int e = t; e < 2 * (PL::T_BYTES / 16); e += NT) {
+    // T tiles start zero (their upper blocks stay zero)
+    for (int e = t; e < NSET * (PL::T_BYTES / 16); e += NT) {
         const int s = e / (PL::T_BYTES / 16), off = (e % (PL::T_BYTES / 16)) * 16;
         *reinterpret_cast<uint4*>(sm + s * PL::SET + PL::TF + off) = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -625,39 +780,30 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);   // this warp's lane quarter
     // TMA of chunk n's [64][128] tiles (packed rows rowbase + n*C ..; rows past the sequence
     // come from the next batch row or the zero fill and are masked where they are used)
-    auto tma_qk = [&](int n) {   // q (MODE_OUTPUT) and k into the Q+ / beta K+ slots of set (n-n0)&1
-        const int s = (n - n0) & 1, row = (int)(rowbase + n * C);
-        mbar_arrive_expect_tx(&bars[B_TQK + s], PL::QK_BYTES);
-        if (OUT) tma_load_3d(sm + s * PL::SET + PL::QP, &tm_q, &bars[B_TQK + s], 0, h, row);
-        tma_load_3d(sm + s * PL::SET + PL::KP, &tm_k, &bars[B_TQK + s], 0, h, row);
-    };
-    auto tma_g = [&](int n) {
-        const int x = (n - n0) & 1;
-        mbar_arrive_expect_tx(&bars[B_TG + x], 16384);
-        tma_load_3d(sm + PL::GS + x * 16384, &tm_g, &bars[B_TG + x], 0, h, (int)(rowbase + n * C));
+    // q (MODE_OUTPUT), k and g of chunk n into the Q+ / beta K+ / K- tiles of its set
+    auto tma_set = [&](int n) {
+        const int s = set_of(n - n0), row = (int)(rowbase + n * C);
+        uint8_t* set = sm + s * PL::SET;
+        mbar_arrive_expect_tx(&bars[B_LD + s], PL::LOAD_BYTES);
+        tma_load_3d(set + PL::KM, &tm_g, &bars[B_LD + s], 0, h, row);
+        tma_load_3d(set + PL::KP, &tm_k, &bars[B_LD + s], 0, h, row);
+        if (OUT) tma_load_3d(set + PL::QP, &tm_q, &bars[B_LD + s], 0, h, row);
     };
     auto tma_v = [&](int n) {   // v in core matrices: [value group][position][8 values]
-        const int x = (n - n0) & 1;
-        mbar_arrive_expect_tx(&bars[B_TV + x], 16384);
-        tma_load_4d(sm + PL::VB + x * 16384, &tm_v, &bars[B_TV + x], 0, (int)(rowbase + n * C), 0, h);
+        mbar_arrive_expect_tx(&bars[B_TV], 16384);
+        tma_load_4d(sm + PL::VB, &tm_v, &bars[B_TV], 0, (int)(rowbase + n * C), 0, h);
     };
     const TQ* tq = nullptr;
 
     if (role == 0) {
         // ================= P: prologue of chunk n0 + kc =====================================
         const int cp = rt & 63, rh = rt >> 6;   // channel pair, 32-row half
-        int g_issued = 0;                        // rt 0: g tiles requested so far
         float2 carry = make_float2(0.f, 0.f);   // rh == 0: carry of channels 2cp, 2cp+1
-        if (rt == 0) {
-            for (int x = 0; x < min(2, nk); ++x) tma_g(n0 + x);
-            g_issued = min(2, nk);
-        }
         for (int kc = 0; kc < nk; ++kc) {
-            const int n = n0 + kc, t0 = n * C, s = kc & 1;
+            const int n = n0 + kc, t0 = n * C, s = set_of(kc);
             uint8_t* set = sm + s * PL::SET;
-            const uint32_t sset = sbase + s * PL::SET;
-            const uint8_t* gst = sm + PL::GS + s * 16384;
-            const uint16_t* sBk = sBeta + (kc & 3) * C;
+            const uint8_t* gst = set + PL::KM;                     // g as TMA landed it
+            const uint16_t* sBk = sBeta + (kc % NBETA) * C;
             // beta of chunk kc+2 starts its way into shared memory (stored into its slot below)
             if (rt < C && beta_async) {
                 const int tt = (n + 2) * C + rt;
@@ -666,7 +812,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 cp_async_commit();
             }
             // ---- g of this chunk -> cumulative log-decay (base 2), references, range -----
-            group_wait(&bars[B_TG + s], (kc >> 1) & 1, ab, rt == 0, BAR_P);
+            group_wait(&bars[B_LD + s], set_par(kc), ab, rt == 0, BAR_P);   // q, k, g landed
             const int nv = min(C, Tq - t0);   // rows of this chunk inside the sequence
             {
                 const float2 l2e = make_float2(kLog2e, kLog2e);
@@ -692,10 +838,6 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const bool direct = bar_red_or(BAR_P, NR, wide);
             const float2 rp = direct ? make_float2(0.f, 0.f) : r2;   // reference of K+ and Q+
             const float2 rm = direct ? bC : r2;                      // reference of K-
-            // ---- set s is free once chunk kc-2's master and O MMAs are done; this chunk's k
-            // (and q) have landed in it ---------------------------------------------------------
-            if (rt == 0 && kc >= 2) thread_wait(&bars[B_EMPTY + s], ((kc >> 1) - 1) & 1, ab);
-            group_wait(&bars[B_TQK + s], (kc >> 1) & 1, ab, rt == 0, BAR_P);
             if (rh == 0) {
                 // the chain's scales: S^ = 2^{rp + carry} master, master <- 2^{rm + carry} master
                 float* sc = sSC + s * 3 * D;
@@ -707,22 +849,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (rt == 0) sDirect[s] = direct ? 1 : 0;
             if (direct) {
-                // the fp32 log-decay table of the chunk: in MODE_OUTPUT over KM, PF and TF (free
-                // until the prologue writes K- and the inverse role fills them), else in the
-                // scratch region
-                uint8_t* scr = OUT ? set + PL::KM : sm + Plan<MODE_STATE>::SCR;
-                float2 run = pre;
-                const float2 l2e = make_float2(kLog2e, kLog2e);
-#pragma unroll 4
-                for (int r = 0; r < 32; ++r) {
-                    const int i = 32 * rh + r;
-                    const uint32_t gw = i < nv ? *reinterpret_cast<const uint32_t*>(gst + i * 256 + 4 * cp) : 0u;
-                    run = __ffma2_rn(in2(gw, (const __nv_bfloat16*)nullptr), l2e, run);
-                    *reinterpret_cast<float2*>(reinterpret_cast<float*>(scr) + i * D + 2 * cp) = run;
-                }
-                named_sync(BAR_P, NR);
-                chunk_ap_direct<OUT, TQ>(scr, set + PL::KP, OUT ? set + PL::QP : set + PL::KP, sBk, set + PL::TF,
-                                         OUT ? set + PL::PF : nullptr, rt, t0, Tq, BAR_P);
+                // A and P from pairwise exponentials; the log-decay table, one 64-channel half
+                // at a time, goes over PF and TF in MODE_OUTPUT (free until the inverse role
+                // fills them), else into the scratch region
+                uint8_t* scr = OUT ? set + PL::PF : sm + Plan<MODE_STATE>::SCR;
+                chunk_ap_direct<MODE, TQ>(set, scr, sTot, sBk, rt, nv);
             }
             // ---- beta K+, Q+ in place, K-; per 8-row block, the 64 threads of a row half read
             // their raw rows before any of them rewrites the block they share -----------------
@@ -769,8 +900,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (OUT) st_pair(set + PL::QP, ig, cp, pq);
                 }
             }
-            // beta of chunk kc+2 into its slot (read by this role's prologue and by Y's beta V two
-            // chunks on; the slot's previous chunk, kc-2, is done with on both sides)
+            // beta of chunk kc+2 into its slot (read by this role's prologue and by the inverse
+            // role's T diag(beta); the slot's previous chunk is long done with)
             if (rt < C) {
                 uint16_t bb;
                 if (beta_async) {
@@ -779,38 +910,31 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 } else {
                     bb = beta_bits(beta, rowbase, Tq, H, h, (n + 2) * C, rt, n + 2 < n1);
                 }
-                sBeta[((kc + 2) & 3) * C + rt] = bb;
+                sBeta[((kc + 2) % NBETA) * C + rt] = bb;
             }
             fence_async_smem();
             tc_fence_before();
             named_sync(BAR_P, NR);
-            if (rt == 0) {
-                mbar_arrive(&bars[B_SC + s]);   // scales, direct flag, tiles (and beta) in place
-                // the g tile has been read for the last time: chunk kc+2's may land
-                if (n + 2 < n1 && !*sAbort) {
-                    tma_g(n + 2);
-                    g_issued = kc + 3;
-                }
-            }
+            if (rt == 0) mbar_arrive(&bars[B_SC + s]);   // scales, direct flag, tiles (and beta) in place
         }
-        // after a timeout some requested g tiles may not have been waited for: let them land
-        if (rt == 0 && *sAbort)
-            for (int x = max(0, g_issued - 2); x < g_issued; ++x)
-                mbar_wait_bounded(&bars[B_TG + (x & 1)], (x >> 1) & 1, kWaitNs);
         if (beta_async) cp_async_wait_all();
     } else if (role == 1) {
         // ================= I: T and -W^T of chunk n0 + kc ===================================
         int n_ap = 0;
         for (int kc = 0; kc < nk; ++kc) {
-            const int s = kc & 1;
+            const int s = set_of(kc);
             uint8_t* set = sm + s * PL::SET;
             const uint32_t sset = sbase + s * PL::SET;
-            group_wait(&bars[B_SC + s], (kc >> 1) & 1, ab, rt == 0, BAR_I);   // the prologue is done
+            group_wait(&bars[B_SC + s], set_par(kc), ab, rt == 0, BAR_I);   // the prologue is done
+            // A|P's TMEM columns are free once the output role has read chunk kc-1's W^T
+            if (rt == 0 && kc > 0) {
+                thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
+                tc_fence_after();
+            }
             if (!sDirect[s]) {
                 if (rt == 0) {
                     // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the state
-                    // pass reads K- as rows 64-127 and ignores them).  A|P's TMEM columns are free:
-                    // this role read the previous chunk's W^T out of them.
+                    // pass reads K- as rows 64-127 and ignores them)
                     const uint32_t id = idesc_f16(128, 64, true, true);
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
@@ -853,22 +977,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                              sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
                 umma_commit(&bars[B_W]);
             }
+            // W^T goes to the set's KP tile by the output role (which then signals PRO)
             group_wait(&bars[B_W], kc & 1, ab, rt == 0, BAR_I);
-            {   // -W^T -> the KP tile (channel c in lane c)
-                float v[64];
-                tmem_ld64(tl + TM_APW, v);
-                const int c = 32 * q4 + lane;
-#pragma unroll
-                for (int g8 = 0; g8 < 8; ++g8) {
-                    float f[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = -v[8 * g8 + j];
-                    *reinterpret_cast<uint4*>(set + PL::KP + g8 * 2048 + (c >> 3) * 128 + (c & 7) * 16) = pack8_f16(f);
-                }
-            }
             {   // T -> T diag(beta) in the input type, in place (the W^T MMA has read T): the B
                 // operand of U~^T = V^T (T diag(beta))^T, with V as it landed
-                const uint16_t* sBk = sBeta + (kc & 3) * C;
+                const uint16_t* sBk = sBeta + (kc % NBETA) * C;
 #pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     const int e = 4 * rt + e4;                       // 16-byte piece: 8 consecutive columns
@@ -888,16 +1001,19 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             fence_async_smem();
             tc_fence_before();
             named_sync(BAR_I, NR);
-            if (rt == 0) {
-                mbar_arrive(&bars[B_INV + s]);   // T diag(beta) ready
-                // every tile of the set is ready (the test hook withholds chunk 0's signal)
-                if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
-            }
+            if (rt == 0) mbar_arrive(&bars[B_INV + s]);   // T diag(beta) ready
         }
     } else if (role == 2) {
         // ================= X: the state chain of chunk n0 + kc ==============================
         const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
         const bool mma = rt == 0;
+        // rt 0 also issues the loads of q, k, g: the first NSET chunks now, chunk kc+2 into the
+        // set of chunk kc-1 once the chain is done with it
+        int ld_issued = 0;
+        if (mma) {
+            ld_issued = min(NSET, nk);
+            for (int x = 0; x < ld_issued; ++x) tma_set(n0 + x);
+        }
         // initial state in TMEM (MODE_STATE: N from 0, Phi from I)
         for (int c0 = 0; c0 < D; c0 += 32) {
             float vv[32];
@@ -924,11 +1040,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         named_sync(BAR_X, NR);
         for (int kc = 0; kc < nk; ++kc) {
-            const int s = kc & 1;
+            const int s = set_of(kc), ub = kc & 1;   // buffer set; [U | O] buffer
             const uint32_t sset = sbase + s * PL::SET;
             // ---- S^ = fp16(2^{rp + carry} master), master <- 2^{rm + carry} master --------
             if (rt == 0) {
-                thread_wait(&bars[B_SC + s], (kc >> 1) & 1, ab);
+                thread_wait(&bars[B_SC + s], set_par(kc), ab);
                 if (kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
             }
             named_sync(BAR_X, NR);
@@ -959,19 +1075,29 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             tc_fence_before();
             named_sync(BAR_X, NR);
+            if (mma && kc >= 1 && kc + 2 < nk && !*sAbort) {
+                // every MMA on chunk kc-1's set is done (its last commit follows the master update
+                // that this role waited for above): chunk kc+2's q, k, g may land there
+                thread_wait(&bars[B_EMPTY + set_of(kc - 1)], set_par(kc - 1), ab);
+                if (!*sAbort) {
+                    tma_set(n0 + kc + 2);
+                    ld_issued = kc + 3;
+                }
+            }
             if (mma) {
                 // U~ (Y) initialised the U columns; -W^T and Q+ are in the set (I)
-                thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
-                thread_wait(&bars[B_PRO + s], (kc >> 1) & 1, ab);
+                thread_wait(&bars[B_VE], kc & 1, ab);
+                thread_wait(&bars[B_PRO + s], set_par(kc), ab);
                 tc_fence_after();
                 if (OUT) {
-                    // [U | O]^T += S^T [-W^T | Q+^T]   (N = 128: positions of W, then of Q+)
-                    const uint32_t id = idesc_f16(128, 128, false, true);
+                    // [U | -O]^T += -S^T [W^T | Q+^T]   (N = 128: positions of W, then of Q+); the
+                    // O columns accumulate -O, negated back when written out
+                    const uint32_t id = idesc_f16(128, 128, false, true, true);
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_f16_ts(tmem + TM::UO + 128 * s, tmem + TM::S16 + 8 * kk,
+                        umma_f16_ts(tmem + TM::UO + 128 * ub, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
                 } else {
-                    const uint32_t id = idesc_f16(128, 64, false, true);
+                    const uint32_t id = idesc_f16(128, 64, false, true, true);   // U^T += -S^T W^T
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
@@ -982,8 +1108,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // ---- U -> fp16 (A operand of the master and O updates); one thread owns its lane,
             // so it may overwrite the columns it has just read ------------------------------------
             {
-                const uint32_t usrc = OUT ? TM::UO + 128 * s : TM::UACC;
-                const uint32_t udst = OUT ? TM::UO + 128 * s : TM::S16;   // MODE_STATE: into S^'s columns
+                const uint32_t usrc = OUT ? TM::UO + 128 * ub : TM::UACC;
+                const uint32_t udst = OUT ? TM::UO + 128 * ub : TM::S16;   // MODE_STATE: into S^'s columns
                 float vv[64];
                 uint32_t hv[32];
                 tmem_ld64(tl + usrc, vv);
@@ -998,21 +1124,21 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
                 const uint32_t idm = idesc_f16(128, 128, false, false);
                 if (OUT) {
-                    // master += U^T K-   and   O^T += U^T P^T
-                    const uint32_t ua = tmem + TM::UO + 128 * s;
+                    // master += U^T K-   and   -O^T += -U^T P^T
+                    const uint32_t ua = tmem + TM::UO + 128 * ub;
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, ua + 8 * kk, sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     umma_commit(&bars[B_S]);
-                    const uint32_t ido = idesc_f16(128, 64, false, false);
+                    const uint32_t ido = idesc_f16(128, 64, false, false, true);
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(ua + 64, ua + 8 * kk, sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
-                    umma_commit(&bars[B_O + s]);
+                    umma_commit(&bars[B_O + ub]);
                 } else {
                     // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
-                    const uint32_t id = idesc_f16(128, 64, false, true);
+                    const uint32_t id = idesc_f16(128, 64, false, true, true);
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, kk > 0);
@@ -1045,11 +1171,15 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         // ---- end of segment: the state S = diag(2^{carry}) master (columns = channels) -----
         if (nk > 0) group_wait(&bars[B_S], (nk - 1) & 1, ab, rt == 0, BAR_X);
+        // after a timeout some requested tiles may not have been waited for: let them land
+        if (mma && *sAbort)
+            for (int x = max(0, ld_issued - NSET); x < ld_issued; ++x)
+                mbar_wait_bounded(&bars[B_LD + set_of(x)], set_par(x), kWaitNs);
         float* dst = nullptr;
         if (MODE == MODE_STATE) dst = maps + (size_t)slot * 2 * D * D;  // [N | M]
         else if (S_T && last) dst = S_T + ((size_t)seq * H + h) * D * D;
         if (dst && !*sAbort) {
-            const float* cn = nk > 0 ? sSC + ((nk - 1) & 1) * 3 * D + 2 * D : nullptr;
+            const float* cn = nk > 0 ? sSC + set_of(nk - 1) * 3 * D + 2 * D : nullptr;
             for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     float vv[32];
@@ -1061,18 +1191,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
     } else {
-        // ================= Y: U~, the output rows, beta V, loads ============================
+        // ================= Y: U~, the output rows, the loads =================================
         const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
         const bool mma = rt == 0, loader = rt == 32;
-        int v_issued = 0, qk_last[2] = {-1, -1};   // loader: TMA requests so far
-        bool o_pending = false;                    // rt 0: a TMA store of the staging tile in flight
+        int v_issued = 0;                          // loader: chunks whose v was requested
         if (loader && nk > 0) {
-            for (int x = 0; x < min(2, nk); ++x) {
-                tma_v(n0 + x);
-                tma_qk(n0 + x);
-                qk_last[x] = x;
-            }
-            v_issued = min(2, nk);
+            tma_v(n0);
+            v_issued = 1;
         }
         float gam = 1.f;
         if (OUT && gate && gamma) gam = gamma[(size_t)h * D + j];
@@ -1088,124 +1213,77 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // U~^T = V^T (T diag(beta))^T into the chunk's U columns: V^T straight from the v tile
         // (M = values, MN-major core matrices), operands in the input type
         auto issue_u = [&](int x) {
-            const int s = x & 1;
-            const uint32_t sset = sbase + s * PL::SET, vbt = sbase + PL::VB + s * 16384;
+            const uint32_t sset = sbase + set_of(x) * PL::SET, vbt = sbase + PL::VB;
             const uint32_t id = idesc_f16(128, 64, true, false, false, std::is_same<TQ, __nv_bfloat16>::value);
-            const uint32_t d = tmem + (OUT ? TM::UO + 128 * s : TM::UACC);
+            const uint32_t d = tmem + (OUT ? TM::UO + 128 * (x & 1) : TM::UACC);
             for (int kk = 0; kk < 4; ++kk)
                 umma_f16(d, sdesc(vbt + 256 * kk, 128, 1024), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
                          kk > 0);
-            umma_commit(&bars[B_VE + s]);   // U~ done: the v tile may be refilled
+            umma_commit(&bars[B_VE]);   // U~ done: the v tile may be refilled
         };
         // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
         auto out_rows = [&](int x) {
             const int b = x & 1, t0x = (n0 + x) * C;
-            // the staging tile is free once the previous store has read it (the role barrier of
-            // the wait below holds every other thread until then)
-            if (rt == 0 && o_pending) {
-                bulk_wait_read0();
-                o_pending = false;
-            }
             group_wait(&bars[B_O + b], (x >> 1) & 1, ab, rt == 0, BAR_Y);
             const int nvx = min(C, Tq - t0x);
-            const bool tma = !o_f32 && !(items && t0x + C > Tq);
-            float inv_lo = 0.f, inv_hi = 0.f;   // per-position inverse RMS (gated output)
-            if (gate) {
-                // Eq. 15 output side: y = Sigmoid(gate) * gamma * RMSNorm over the head's values.
-                // Per position, the sum of squares over this warp's 32 values by a transposing
-                // butterfly (lane l ends with position 32*hp + l), then over the 4 lane quarters.
-                float* red = reinterpret_cast<float*>(sm + PL::MISC + M_RED);
-                for (int hp = 0; hp < 2; ++hp) {
-                    float sq[32];
-                    tmem_ld32(tl + TM::UO + 128 * b + 64 + 32 * hp, sq);
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) sq[u] = sq[u] * sq[u];
-#pragma unroll
-                    for (int sft = 16; sft >= 1; sft >>= 1) {
-                        const bool up = (lane & sft) != 0;
-#pragma unroll
-                        for (int k = 0; k < sft; ++k) {
-                            const float send = up ? sq[k] : sq[k + sft];
-                            const float recv = __shfl_xor_sync(0xffffffffu, send, sft);
-                            sq[k] = (up ? sq[k + sft] : sq[k]) + recv;
-                        }
-                    }
-                    red[q4 * C + 32 * hp + lane] = sq[0];
-                }
-                named_sync(BAR_Y, NR);
-                const float m0 = (red[lane] + red[C + lane] + red[2 * C + lane] + red[3 * C + lane]) * (1.f / D) + eps;
-                const float m1 = (red[32 + lane] + red[C + 32 + lane] + red[2 * C + 32 + lane] + red[3 * C + 32 + lane]) *
-                                     (1.f / D) + eps;
-                inv_lo = m0 > 0.f ? rsqrtf(m0) : 0.f;
-                inv_hi = m1 > 0.f ? rsqrtf(m1) : 0.f;
+            const uint32_t ocol = tl + TM::UO + 128 * b + 64;
+            if constexpr (GOUT) {
+                const OutParams op{gate, o, reinterpret_cast<float*>(sm + PL::MISC + M_RED), gam, eps, o_f32, H, h, q4, lane};
+                out_rows_general(&op, ocol, rowbase + t0x, nvx);
+                return;
             }
-            uint8_t* os = sm + PL::OS;
+#pragma unroll 1
             for (int hp = 0; hp < 2; ++hp) {
                 float v[32];
-                tmem_ld32(tl + TM::UO + 128 * b + 64 + 32 * hp, v);
-                if (gate) {
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const float iu = __shfl_sync(0xffffffffu, hp ? inv_hi : inv_lo, u);
-                        const int i = 32 * hp + u;
-                        float gv = 0.f;
-                        if (i < nvx) gv = __bfloat162float(gate[(((size_t)rowbase + t0x + i) * H + h) * D + j]);
-                        v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
-                    }
-                }
-                if (tma) {
-                    // bf16 into the swizzled staging tiles: lane pairs trade halves so each
-                    // thread writes a value pair (4 bytes)
-                    const bool odd = lane & 1;
-#pragma unroll
-                    for (int u2 = 0; u2 < 16; ++u2) {
-                        const float send = odd ? v[2 * u2] : v[2 * u2 + 1];
-                        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                        const float lo = odd ? recv : v[2 * u2], hi = odd ? v[2 * u2 + 1] : recv;
-                        const int i = 32 * hp + 2 * u2 + (odd ? 1 : 0);
-                        *reinterpret_cast<__nv_bfloat162*>(os + swz_off(i, j & ~1)) = __floats2bfloat162_rn(lo, hi);
-                    }
-                } else {
-                    // fp32 output, or a packed sample's ragged last chunk: plain stores
-                    const size_t rs = (size_t)H * D;
-#pragma unroll
-                    for (int u = 0; u < 32; ++u) {
-                        const int i = 32 * hp + u;
-                        if (i < nvx) {
-                            const size_t idx = ((size_t)rowbase + t0x + i) * rs + (size_t)h * D + j;
-                            if (o_f32) reinterpret_cast<float*>(o)[idx] = v[u];
-                            else reinterpret_cast<__nv_bfloat16*>(o)[idx] = __float2bfloat16_rn(v[u]);
-                        }
-                    }
-                }
-            }
-            if (tma) {
-                fence_async_smem();
-                named_sync(BAR_Y, NR);
-                if (rt == 0) {
-                    tma_store_4d(&tm_o, os, 0, h, (int)(o_t + t0x), o_b);
-                    tma_store_4d(&tm_o, os + 8192, 64, h, (int)(o_t + t0x), o_b);
-                    bulk_commit();
-                    o_pending = true;
-                }
+                tmem_ld32(ocol + 32 * hp, v);
+                store_rows_bf16(v, reinterpret_cast<__nv_bfloat16*>(o), rowbase + t0x, 32 * hp, nvx, H, h, q4, lane);
             }
         };
         zero_o(0);
         if (nk > 1) zero_o(1);
         tc_fence_before();
-        named_sync(BAR_Y, NR);   // the first beta V and zeroed O columns are in place
+        named_sync(BAR_Y, NR);   // the zeroed O columns are in place
         tc_fence_after();
         bool u_done = false;     // rt 0: U~ of chunk kc already issued
         for (int kc = 0; kc < nk; ++kc) {
-            const int n = n0 + kc, s = kc & 1;
+            const int n = n0 + kc, s = set_of(kc);
+            // ---- W^T of chunk kc (TMEM, channel c in lane c) -> the set's KP tile ----------------
+            group_wait(&bars[B_W], kc & 1, ab, rt == 0, BAR_Y);
+            {
+                uint8_t* kp = sm + s * PL::SET + PL::KP + (j >> 3) * 128 + (j & 7) * 16;
+#pragma unroll 1
+                for (int hw = 0; hw < 2; ++hw) {
+                    float v[32];
+                    tmem_ld32(tl + TM_APW + 32 * hw, v);
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8)
+                        *reinterpret_cast<uint4*>(kp + (4 * hw + g8) * 2048) = pack8_f16(v + 8 * g8);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_sync(BAR_Y, NR);
+            if (rt == 0) {
+                mbar_arrive(&bars[B_APWF]);   // A|P's TMEM columns may be reused
+                // every tile of the set is ready (the test hook withholds chunk 0's signal)
+                if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
+            }
             if (mma && !u_done) {
-                thread_wait(&bars[B_INV + s], (kc >> 1) & 1, ab);
-                thread_wait(&bars[B_TV + s], (kc >> 1) & 1, ab);   // this chunk's v has landed
+                thread_wait(&bars[B_INV + s], set_par(kc), ab);
+                thread_wait(&bars[B_TV], kc & 1, ab);   // this chunk's v has landed
                 // MODE_STATE: one U accumulator; the chain of chunk kc-1 has read it once its
                 // last master update is done
                 if (!OUT && kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
                 tc_fence_after();
                 issue_u(kc);
+            }
+            // the v tile is free once U~ of chunk kc is done: chunk kc+1's may land
+            if (loader && kc + 1 < nk && !*sAbort) {
+                thread_wait(&bars[B_VE], kc & 1, ab);
+                if (!*sAbort) {
+                    tma_v(n + 1);
+                    v_issued = kc + 2;
+                }
             }
             // ---- chunk kc-1's output rows, then its O columns are zeroed for chunk kc+1 -------
             if (OUT && kc > 0) {
@@ -1214,25 +1292,11 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             tc_fence_before();
             named_sync(BAR_Y, NR);
-            // ---- loads: chunk kc+2's k (and q) once the [U | O] MMA of chunk kc has read the set's
-            // -W^T (and Q+) (MODE_STATE: both chains' MMAs), its v once U~ of chunk kc is done -----
-            if (loader && n + 2 < n1 && !*sAbort) {
-                thread_wait(&bars[OUT ? B_U : B_U2], kc & 1, ab);
-                if (!*sAbort) {
-                    tma_qk(n + 2);
-                    qk_last[s] = kc + 2;
-                }
-                thread_wait(&bars[B_VE + s], (kc >> 1) & 1, ab);
-                if (!*sAbort) {
-                    tma_v(n + 2);
-                    v_issued = kc + 3;
-                }
-            }
-            // U~ of the next chunk now, if its T is ready (else at the top of the next step)
+            // U~ of the next chunk now, if its T and v are ready (else at the top of the next step)
             if (mma) {
                 u_done = false;
-                if (OUT && kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + (s ^ 1)], ((kc + 1) >> 1) & 1) &&
-                    mbar_try_wait(&bars[B_TV + (s ^ 1)], ((kc + 1) >> 1) & 1)) {
+                if (OUT && kc + 1 < nk && !*sAbort && mbar_try_wait(&bars[B_INV + set_of(kc + 1)], set_par(kc + 1)) &&
+                    mbar_try_wait(&bars[B_TV], (kc + 1) & 1)) {
                     tc_fence_after();
                     issue_u(kc + 1);
                     u_done = true;
@@ -1240,14 +1304,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         if (OUT && nk > 0) out_rows(nk - 1);
-        if (rt == 0 && o_pending) bulk_wait0();   // every output store has landed before the CTA exits
         // after a timeout some requested tiles may not have been waited for: let them land
-        if (loader && *sAbort) {
-            for (int x = max(0, v_issued - 2); x < v_issued; ++x)
-                mbar_wait_bounded(&bars[B_TV + (x & 1)], (x >> 1) & 1, kWaitNs);
-            for (int s2 = 0; s2 < 2; ++s2)
-                if (qk_last[s2] >= 0) mbar_wait_bounded(&bars[B_TQK + s2], (qk_last[s2] >> 1) & 1, kWaitNs);
-        }
+        if (loader && *sAbort && v_issued > 0) mbar_wait_bounded(&bars[B_TV], (v_issued - 1) & 1, kWaitNs);
     }
     // ---- teardown: after a timeout, each MMA issuer drains its own MMAs; free TMEM --------
     if (*sAbort && (t == 0 || t == NR || t == 2 * NR || t == 3 * NR)) {
@@ -1422,24 +1480,8 @@ bool make_map_v(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 output o as a 4-D tensor (channels, heads, tokens, rows), box = 64 channels x
-// 1 head x 64 tokens, 128-byte swizzle.  Tokens past T are clipped by the T dimension, so
-// a ragged last chunk never writes into the next row.
-bool make_map_o(CUtensorMap* m, void* base, int B, int T, int H)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)C, 1u};
-    const cuuint32_t es[4] = {1u, 1u, 1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 struct Maps {
-    CUtensorMap q, k, v, g, o;   // o: only for a bf16 output (else a copy of q, unused)
+    CUtensorMap q, k, v, g;
 };
 
 struct Split {
@@ -1460,7 +1502,8 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
                         int* status, cudaStream_t s, const int* items = nullptr, int nitems = 0,
                         const char* prof_name = nullptr)
 {
-    auto kern = kda_tc_kernel<MODE, TQ>;
+    const bool gout = MODE == MODE_OUTPUT && (a.gate != nullptr || a.out_t == ET_F32);
+    auto kern = gout ? kda_tc_kernel<MODE, TQ, MODE == MODE_OUTPUT> : kda_tc_kernel<MODE, TQ, false>;
     const int smem = smem_bytes<MODE>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -1469,7 +1512,7 @@ cudaError_t launch_pass(const Maps& mp, const KdaArgs& a, const float* S_in, int
     if (grid == 0) return cudaSuccess;
     ProfileScope prof(prof_name ? prof_name : (MODE == MODE_STATE ? "kda_tc_state" : "kda_tc_output"), s);
     count_launch();
-    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, mp.o, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
+    kern<<<grid, NT, smem, s>>>(mp.q, mp.k, mp.v, mp.g, (const __nv_bfloat16*)a.beta, a.o, a.out_t == ET_F32 ? 1 : 0,
                                 S_in, per_seg, maps, a.ST, a.B, a.T, a.H, P, L, status, debug_drop_handoff(),
                                 (const __nv_bfloat16*)a.gate, a.gamma, a.eps, items);
     return cudaGetLastError();
@@ -1484,11 +1527,7 @@ bool build_maps(const KdaArgs& a, Maps& mp)
         !make_map_v(&mp.v, a.v, dq, a.B, a.T, a.H) ||
         !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.B, a.T, a.H))
         return false;
-    if (a.out_t == ET_F32 || !a.o) {
-        mp.o = mp.q;
-        return true;
-    }
-    return make_map_o(&mp.o, a.o, a.B, a.T, a.H);
+    return true;
 }
 
 int sm_count()
@@ -1588,8 +1627,6 @@ cudaError_t launch_all(const KdaArgs& a, void* ws, int* status, cudaStream_t s)
         return combine_output<TQ>(mp, a, sp, maps, starts, status, s);
     }
     const int P = wv.P, L = wv.L, BH = a.B * a.H;
-    // item tables address packed rows: the bf16 output map spans all B*T rows as one
-    if (a.out_t == ET_BF16 && !make_map_o(&mp.o, a.o, 1, a.B * a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     float* starts = reinterpret_cast<float*>(base + wv.maps_b);
@@ -1782,8 +1819,6 @@ cudaError_t launch_varlen(const KdaArgs& a, const int* cu, int n, void* ws, int*
     if (!make_map(&mp.q, a.q, dq, 1, a.T, a.H) || !make_map(&mp.k, a.k, dq, 1, a.T, a.H) ||
         !make_map_v(&mp.v, a.v, dq, 1, a.T, a.H) || !make_map(&mp.g, a.g, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, a.T, a.H))
         return cudaErrorInvalidValue;
-    if (a.out_t == ET_F32) mp.o = mp.q;
-    else if (!make_map_o(&mp.o, a.o, 1, a.T, a.H)) return cudaErrorInvalidValue;
     char* base = reinterpret_cast<char*>(ws);
     float* maps = reinterpret_cast<float*>(base);
     base += a256(pl.n_maps * 2 * D * D * sizeof(float));
