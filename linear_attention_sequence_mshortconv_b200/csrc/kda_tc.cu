@@ -600,6 +600,13 @@ __device__ __forceinline__ void store_rows_bf16(const float (&v)[32], __nv_bfloa
     }
 }
 
+__device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Parameters of the output rows that only the gated or fp32 output needs.
 struct OutParams {
     const __nv_bfloat16* gate;
@@ -607,6 +614,7 @@ struct OutParams {
     float* red;        // float[4][64] shared scratch
     float gam, eps;
     int o_f32, H, h, q4, lane;
+    int64_t row_end;   // packed token just past the sequence
 };
 // Output rows of one chunk with the Eq. 15 output gate, or to an fp32 o; the plain bf16
 // case stays inline in the kernel.  ocol: this warp's TMEM address of the chunk's -O^T
@@ -622,6 +630,11 @@ __device__ __forceinline__ void out_rows_general(const OutParams* op, uint32_t o
     const int j = 32 * q4 + lane;
     float inv_lo = 0.f, inv_hi = 0.f;   // per-position inverse RMS (gated output)
     if (gate) {
+        // the next chunk's gate rows toward L2 (one 128-byte line per thread)
+        const int t128 = 32 * q4 + lane;
+        const int64_t rn = row0 + C + (t128 >> 1);
+        if (rn < op->row_end)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(gate + ((size_t)rn * H + h) * D + 64 * (t128 & 1)));
         // y = Sigmoid(gate) * gamma * RMSNorm over the head's values (Eq. 15, output side).
         // Per position, the sum of squares over this warp's 32 values by a transposing
         // butterfly (lane l ends with position 32*hp + l), then over the 4 lane quarters.
@@ -651,16 +664,20 @@ __device__ __forceinline__ void out_rows_general(const OutParams* op, uint32_t o
     }
     for (int hp = 0; hp < 2; ++hp) {
         float v[32];
+        uint16_t gb[32];   // the gate of this column at the 32 positions: all loads in flight at once
+        if (gate) {
+            const unsigned short* gp = reinterpret_cast<const unsigned short*>(gate) + ((size_t)row0 * H + h) * D + j;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) gb[u] = 32 * hp + u < nvx ? __ldg(gp + (size_t)(32 * hp + u) * H * D) : 0;
+        }
         tmem_ld32(ocol + 32 * hp, v);
         if (gate) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) {
-                v[u] = -v[u];
                 const float iu = __shfl_sync(0xffffffffu, hp ? inv_hi : inv_lo, u);
-                const int i = 32 * hp + u;
-                float gv = 0.f;
-                if (i < nvx) gv = __bfloat162float(gate[(((size_t)row0 + i) * H + h) * D + j]);
-                v[u] = __fdividef(v[u] * iu * gam, 1.f + __expf(-gv));
+                const float gv = __uint_as_float((uint32_t)gb[u] << 16);
+                // Sigmoid(g) = (1 + tanh(g / 2)) / 2: one MUFU operation
+                v[u] = -v[u] * iu * gam * fmaf(0.5f, tanh_approx(0.5f * gv), 0.5f);
             }
         }
         if (!o_f32) {
@@ -1228,7 +1245,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const int nvx = min(C, Tq - t0x);
             const uint32_t ocol = tl + TM::UO + 128 * b + 64;
             if constexpr (GOUT) {
-                const OutParams op{gate, o, reinterpret_cast<float*>(sm + PL::MISC + M_RED), gam, eps, o_f32, H, h, q4, lane};
+                const OutParams op{gate, o, reinterpret_cast<float*>(sm + PL::MISC + M_RED), gam, eps, o_f32, H, h, q4, lane,
+                                   rowbase + Tq};
                 out_rows_general(&op, ocol, rowbase + t0x, nvx);
                 return;
             }
