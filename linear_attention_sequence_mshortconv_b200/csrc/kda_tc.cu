@@ -588,15 +588,14 @@ __device__ __forceinline__ void store_rows_bf16(const float (&v)[32], __nv_bfloa
     uint32_t wv[16];   // -v: the O columns hold -O
 #pragma unroll
     for (int m = 0; m < 16; ++m) wv[m] = pack2_in<__nv_bfloat16>(v[2 * m], v[2 * m + 1]) ^ 0x80008000u;
+    const int i0 = hp0 + (lane & 7);
+    uint4* dst = reinterpret_cast<uint4*>(o + ((size_t)row0 + i0) * ((size_t)H * D) + h * D + 32 * q4 + 8 * (lane >> 3));
+    const size_t step = (size_t)H * D;   // 8 positions, in 16-byte units
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
         uint32_t z[4];
         transpose8x8_b16(wv + 4 * blk, z, lane);
-        const int i = hp0 + 8 * blk + (lane & 7);
-        if (i < nvx) {
-            const size_t idx = ((size_t)row0 + i) * ((size_t)H * D) + (size_t)h * D + 32 * q4 + 8 * (lane >> 3);
-            *reinterpret_cast<uint4*>(o + idx) = make_uint4(z[0], z[1], z[2], z[3]);
-        }
+        if (i0 + 8 * blk < nvx) dst[blk * step] = make_uint4(z[0], z[1], z[2], z[3]);
     }
 }
 
@@ -953,6 +952,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the state
                     // pass reads K- as rows 64-127 and ignores them)
                     const uint32_t id = idesc_f16(128, 64, true, true);
+                    #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
                                  sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
@@ -989,6 +989,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
                 // W^T = (beta K+)^T T^T: M = 128 channels, N = 64 positions, K = 64 positions
                 const uint32_t id = idesc_f16(128, 64, false, false);
+                #pragma unroll 1
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 4096 * kk, 2048, 128),
                              sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
@@ -1110,11 +1111,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // [U | -O]^T += -S^T [W^T | Q+^T]   (N = 128: positions of W, then of Q+); the
                     // O columns accumulate -O, negated back when written out
                     const uint32_t id = idesc_f16(128, 128, false, true, true);
+                    #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UO + 128 * ub, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
                 } else {
                     const uint32_t id = idesc_f16(128, 64, false, true, true);   // U^T += -S^T W^T
+                    #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
@@ -1143,19 +1146,23 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (OUT) {
                     // master += U^T K-   and   -O^T += -U^T P^T
                     const uint32_t ua = tmem + TM::UO + 128 * ub;
+                    #pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, ua + 8 * kk, sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     umma_commit(&bars[B_S]);
                     const uint32_t ido = idesc_f16(128, 64, false, false, true);
+                    #pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(ua + 64, ua + 8 * kk, sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
                     umma_commit(&bars[B_O + ub]);
                 } else {
                     // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
+                    #pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     const uint32_t id = idesc_f16(128, 64, false, true, true);
+                    #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, kk > 0);
@@ -1178,6 +1185,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (mma) {
                     tc_fence_after();
                     const uint32_t idm = idesc_f16(128, 128, false, false);
+                    #pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER + D, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
@@ -1233,6 +1241,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t sset = sbase + set_of(x) * PL::SET, vbt = sbase + PL::VB;
             const uint32_t id = idesc_f16(128, 64, true, false, false, std::is_same<TQ, __nv_bfloat16>::value);
             const uint32_t d = tmem + (OUT ? TM::UO + 128 * (x & 1) : TM::UACC);
+            #pragma unroll 1
             for (int kk = 0; kk < 4; ++kk)
                 umma_f16(d, sdesc(vbt + 256 * kk, 128, 1024), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
                          kk > 0);
