@@ -84,7 +84,10 @@ size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype
 /*
  * kda_forward -- KDA forward scan (Eq. 14) with readout o_t = S_t^T q_t (Eq. 15).
  *
- *   q, k, g : [B, T, H, Dk]  dtype          g = ln(alpha), finite, <= 0
+ *   q, k, g : [B, T, H, Dk]  dtype          g = ln(alpha), finite, <= 0 (any such value:
+ *                                            a per-channel decay as strong as alpha =
+ *                                            e^-80 on single tokens is computed, no range
+ *                                            is rejected)
  *   v       : [B, T, H, Dv]  dtype
  *   beta    : [B, T, H]      dtype          erase/write strength, one per (token, head)
  *   S0      : [B, H, Dk, Dv] fp32, or NULL  initial state (NULL = zeros)
@@ -187,7 +190,7 @@ kda_status kda_forward_noalloc(const void* q, const void* k, const void* v, cons
 
 /*
  * Sequence-parallel forward: each of the B rows is cut along time into R consecutive
- * shards, one per device (the pages run one long stream per device and name no
+ * shards, one per device (the paper runs one long stream per device and names no
  * multi-device scheme; this follows from Eq. 14 of section 3.3 being affine in the
  * state).  Over a shard, S_out = M S_in + N with
  *   M = prod_t (I - beta_t k_t k_t^T) Diag(alpha_t)   (latest token leftmost), [D, D]
@@ -247,7 +250,7 @@ kda_status kda_sp_output(const void* q, const void* k, const void* v, const void
                          kda_stream_t stream);
 
 /*
- * kda_backward -- gradients of the scan of kda_forward (the pages give only the forward;
+ * kda_backward -- gradients of the scan of kda_forward (the paper gives only the forward;
  * this is its reverse-mode derivative).  For a loss L with dL/do = d_o and dL/dS_T = dS_T:
  *   q, k, v, g, beta, S0, B, T, H, Dk, Dv, dtype : exactly as passed to kda_forward.
  *   d_o   : [B, T, H, Dv] in do_dtype (device).
@@ -313,7 +316,7 @@ kda_status mshortconv_forward(const void* x, void* y, int B, int T, int C, kda_d
                               kda_stream_t stream);
 
 /*
- * mshortconv_backward -- gradients of mshortconv_forward (section 3.4; the pages give only
+ * mshortconv_backward -- gradients of mshortconv_forward (section 3.4; the paper gives only
  * the forward).  For a loss L with dL/dy = dy:
  *   x, dy    : [B, T, C] dtype (device); x is read only for the weight gradients.
  *   dx       : [B, T, C] fp32 (device, written; 0 at tokens no segment covers).
@@ -363,7 +366,7 @@ kda_status kda_mshortconv_forward(const void* xq, const void* xk, const void* xv
                                   kda_stream_t stream);
 
 /*
- * kda_mshortconv_backward -- gradients of kda_mshortconv_forward (the pages give only the
+ * kda_mshortconv_backward -- gradients of kda_mshortconv_forward (the paper gives only the
  * forward): for dL/do = d_o and dL/dS_T = dS_T, the gradients of x_q, x_k, x_v, of the
  * three tensors' conv weights, of g, beta and S0.
  *   xq ... D, dtype : exactly as passed to kda_mshortconv_forward.
@@ -409,7 +412,7 @@ kda_status kda_forward_plan(int B, int T, int H, int Dk, int Dv, kda_dtype dtype
 /* Number of kernels this library has launched in this process (all devices). */
 uint64_t kda_kernel_launches(void);
 
-/* Test hook for the device-side failure path (the pages have no counterpart; this is
+/* Test hook for the device-side failure path (the paper has no counterpart; this is
  * how the timeout handling is exercised without a fault or a hang).  While `on` is
  * non-zero, every later launch of the tensor-core scan withholds, in each CTA, the
  * first "tiles ready" signal from its producer warps to its consumer warps.  The
@@ -424,7 +427,7 @@ void kda_debug_drop_handoff(int on);
 /* Measures this GPU's fp32 fused-multiply-add rate (FMAs per second) with a synthetic
  * kernel of independent FMA chains on every SM, timed with CUDA events on the default
  * stream (synchronous; allocates 4 bytes).  It is the denominator of the conv's
- * plain-ALU roofline in the benchmark; the pages have no counterpart.  Returns 0, or -1
+ * plain-ALU roofline in the benchmark; the paper has no counterpart.  Returns 0, or -1
  * on a CUDA error. */
 int kda_fma_probe(double* fma_per_s);
 

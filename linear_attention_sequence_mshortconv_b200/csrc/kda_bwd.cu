@@ -1,6 +1,6 @@
 // Backward of the KDA forward scan (Eq. 14 of the Chimera paper, section 3.3, with the
 // readout o_t = S_t^T q_t of Eq. 15): given dL/do and dL/dS_T, the gradients of q, k, v,
-// g = log(alpha), beta and S0.  The pages give only the forward; this is its
+// g = log(alpha), beta and S0.  The paper gives only the forward; this is its
 // reverse-mode derivative, taken through the chunk form of the scan.
 //
 // Chunk form (C = 32 tokens, entry state S, b_i = sum_{r<=i} g_r per key channel, b_C

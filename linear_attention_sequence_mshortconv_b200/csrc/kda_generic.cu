@@ -3,7 +3,7 @@
 // This is the path for fp32 inputs (where tensor-core operands would not meet an
 // fp32 accuracy bar) and for every shape the tensor-core path does not cover.
 //
-// Chunkwise form of Eq. 14 (Chimera paper, section 3.3).  The pages only say the KDA
+// Chunkwise form of Eq. 14 (Chimera paper, section 3.3).  The paper only says the KDA
 // kernel is "chunked"; the algebra below is derived from Eq. 14 itself.  Inside a
 // chunk of C tokens with state S0 on entry, let b_i = sum_{r<=i} g_r (per channel,
 // fp32) and u_i = beta_i (v_i - (D_i S_{i-1})^T k_i), so S_i = D_i S_{i-1} + k_i u_i^T.

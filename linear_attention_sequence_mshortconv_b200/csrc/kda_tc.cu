@@ -1,10 +1,10 @@
 // Tensor-core (tcgen05 / TMEM) chunkwise KDA forward for Dk = Dv = 128, chunk 64.
 //
 // What it computes is Eq. 14 of the Chimera paper (section 3.3) with the readout
-// o_t = S_t^T q_t (Eq. 15, inner term).  The pages only say the kernel is "chunked";
-// the chunk algebra is derived from Eq. 14.  Inside a chunk of C = 64 tokens with
-// entry state S0, b_i = sum_{r<=i} g_r (per key channel, base 2, fp32) and two
-// per-channel references rp, rm:
+// o_t = S_t^T q_t (Eq. 15, inner term).  Section 5.1 of the paper names a "chunked" KDA
+// kernel without giving its algebra; the chunk algebra here is derived from Eq. 14.
+// Inside a chunk of C = 64 tokens with entry state S0, b_i = sum_{r<=i} g_r (per key
+// channel, base 2, fp32) and two per-channel references rp, rm:
 //   K+ = k 2^{b - rp},  Q+ = q 2^{b - rp},  K- = k 2^{rm - b}
 //   A  = strict_lower((diag(beta) K+) K-^T),   P = lower(Q+ K-^T)  (incl. diagonal)
 //   T  = (I + A)^{-1}                     (16x16 blocks on warp MMAs, fp16 operands)
@@ -14,18 +14,20 @@
 // With rp = rm = r (the chunk's middle row) A and P are products of K+ and K- whose
 // factors stay within 2^{+-|b_C|/2}; a chunk whose decay is too strong for that keeps
 // rp = 0 and rm = b_C (every factor <= 1) and forms A and P with pairwise exponentials
-// on CUDA cores instead (chunk_ap_direct).  Every MMA operand is fp16; accumulation is
-// fp32 in TMEM.
+// on CUDA cores instead (chunk_ap_direct).  Every MMA operand is fp16 except the U~
+// product, which takes V as it arrives (bf16 or fp16); accumulation is fp32 in TMEM.
 //
 // Transposed state.  The state lives in TMEM as S^T: lane j holds value column j, TMEM
 // column c key channel c (fp32 master).  Every product on the state's serial chain then
 // takes S^T (or U^T) as the A operand straight from TMEM, with no shared-memory round trip:
-//   [U | O]^T  = [U~^T | 0] + S^T [-W^T | Q+^T]     (M = 128 values, N = 128, K = 128)
+//   [U | -O]^T = [U~^T | 0] - S^T [W^T | Q+^T]      (M = 128 values, N = 128, K = 128)
 //   master    += U^T K-                              (N = 128 channels, K = 64)
-//   O^T       += U^T P^T                             (N = 64, K = 64)
-// The fp32 master holds diag(2^{-carry}) S: the row scales of one chunk and the next
-// are applied together, once, when the next chunk reads it (S^ = 2^{rp + carry} master
-// in fp16 for the A operand, and the master itself rescaled by 2^{rm + carry}).
+//   -O^T      -= U^T P^T                             (N = 64, K = 64)
+// (the instruction descriptor's A negation gives the minus signs; O is negated back when
+// it is written out).  The fp32 master holds diag(2^{-carry}) S: the row scales of one
+// chunk and the next are applied together, once, when the next chunk reads it (S^ =
+// 2^{rp + carry} master in fp16 for the A operand, and the master itself rescaled by
+// 2^{rm + carry}).
 //
 // Parallelism.  A head's scan is sequential over chunks, and one B200 workload has
 // only B*H = 16 heads for 148 SMs, so each head's chunk sequence is cut into P
@@ -37,15 +39,12 @@
 //   output pass (MODE_OUTPUT): the recurrence from S_start(p), writing o (and S_T from
 //          the last segment).
 //
-// Inside a CTA (one per (b, h, segment), 512 threads) two warp groups form a
-// two-stage pipeline over the segment's chunks:
-//   producer (warps 0-7): the state-independent work of chunk n+1: log-decay prefix,
-//     references, K+ / Q+ / K- tiles, A|P (one M = 128 MMA), T, W^T (MMA) -> -W^T tile.
-//   consumer (warps 8-15): chunk n's chain: U~ (MMA), S^, [U | O], U -> fp16, master and
-//     O updates, the output rows, and beta V of chunk n+1.
-// Buffer sets of per-chunk tiles are double-buffered; mbarriers hand a set over (SC:
-// scales, INV: T, PRO: all tiles) and back (EMPTY, committed by the consumer's last MMA
-// on it).  Inputs arrive by TMA straight into the tiles that consume them.
+// Inside a CTA (one per (b, h, segment), 512 threads) four roles of four warps each
+// work on three chunks at once (see the kernel's comment): the prologue of chunk n+2,
+// the inverse of chunk n+1 and the state chain of chunk n, with an auxiliary role for
+// the output rows and the V side.  Three buffer sets of per-chunk tiles rotate; mbarriers
+// hand a set from role to role and back to the loads (EMPTY, committed by the chain's
+// last MMA on it).  Inputs arrive by TMA straight into the tiles that consume them.
 //
 // Shared-memory operand tiles use the no-swizzle core-matrix layout (8 rows x 16 B
 // blocks of 128 contiguous bytes); a descriptor takes the byte stride between core
@@ -55,9 +54,9 @@
 // positions are K.
 //
 // All waits are bounded (kWaitNs).  On expiry the kernel records DEV_TIMEOUT in the
-// device status word and stops waiting: both warp groups still run every barrier of
-// their loop (so neither can hang on the other), results are undefined, and before
-// TMEM is freed each MMA-issuing thread drains its own MMAs.
+// device status word and stops waiting: every role still runs every barrier of its loop
+// (so none can hang on another), results are undefined, and before TMEM is freed each
+// MMA-issuing thread drains its own MMAs.
 
 #include <mutex>
 #include <type_traits>

@@ -27,7 +27,7 @@
  *  - pchao.org translation, section 3.3 Eq. 12: time-first raster order
  *    m = i*H*W + j*W + k inside a visual segment.
  *
- * Readings taken where the pages are silent (each is listed in the design notes):
+ * Readings taken where the paper is silent (each is listed in the design notes):
  *  - alpha is passed as g = ln(alpha) (g <= 0); the oracle forms alpha = exp(g).
  *  - no 1/sqrt(dk) scaling and no normalisation inside the scan.
  *  - text conv: y[t] = sum_{j<Kt} w[c,j] * x[t-(Kt-1)+j], zero before the segment.

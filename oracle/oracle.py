@@ -26,7 +26,7 @@ passages of the Chimera paper it follows, is stated in that file's header:
   normalisation and the chain rule through the fused forward (conv -> norm -> scan),
   composed from the other backward routines (numpy, fp64).
 * ``kda_backward``: the reverse-mode derivative of the token recurrence of Eq. 14 with
-  the readout of Eq. 15 (the pages give only the forward; the paper trains with it).
+  the readout of Eq. 15 (the paper gives only the forward; the paper trains with it).
   Plain reverse sweep over the tokens in fp64 (numpy), from the states of a forward
   sweep.
 """

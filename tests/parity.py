@@ -3,7 +3,9 @@
 Tolerances (written once, used by every parity test):
   * fp32 inputs: max |gpu - oracle| <= 1e-4 * max |oracle|, per (b, h), for o and S_T.
   * bf16 inputs: max |gpu - oracle| <= 2e-2 * RMS(oracle), per (b, h), for o and S_T,
-    with the oracle fed the same bf16-rounded inputs.
+    with the oracle fed the same bf16-rounded inputs (o computed in fp32).
+  * a bf16 output o: element-wise |gpu - oracle| <= 2e-2 * RMS(oracle) + 2^-9 |oracle|
+    (the same bound plus the rounding of o to bf16).
 The relative-to-max form for fp32 avoids an ill-posed element-wise relative error near
 zero; the bf16 bound covers bf16 operand and output rounding after fp32 accumulation.
 """
@@ -31,6 +33,26 @@ def compare(gpu: np.ndarray, ref: np.ndarray, kind: str, what: str = ""):
         bound = BF16_RMS * float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
     assert err <= bound + 1e-30, f"{what}: max|diff| {err:.3e} > bound {bound:.3e}"
     return err, bound
+
+
+BF16_HALF_ULP = 2.0 ** -9   # round-to-nearest bf16: relative error at most 2^-9
+
+
+def compare_bf16_output(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
+    """A bf16 output o against the oracle: element-wise |gpu - ref| <= 2e-2 * RMS(ref) +
+    2^-9 * |ref|, the bf16-input bound plus the rounding of o itself to bf16 (which alone
+    reaches 2.3-2.5% of RMS on the video clip's heavy-tailed outputs).  Returns the
+    worst ratio to that bound."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite values in the GPU result"
+    if not ref.size:
+        return 0.0
+    bound = BF16_RMS * float(np.sqrt(np.mean(ref * ref))) + BF16_HALF_ULP * np.abs(ref)
+    ratio = float((np.abs(gpu - ref) / bound).max())
+    assert ratio <= 1.0, f"{what}: |diff| exceeds 2e-2 RMS + 2^-9 |ref| by x{ratio:.3f}"
+    return ratio
 
 
 def compare_heads(o_gpu, o_ref, S_gpu, S_ref, kind, pairs=None, what=""):

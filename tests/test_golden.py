@@ -1,6 +1,6 @@
 """The oracle against the stored golden fixtures of tests/golden/: exact rational results
 of the plain definitions (Eq. 14 / Eq. 15 of section 3.3 and the conv of section 3.4),
-written by tests/golden/make_golden.py with Python fractions.  The pages print no worked
+written by tests/golden/make_golden.py with Python fractions.  The paper prints no worked
 example, so these are the closest stored values: computed outside the oracle and
 outside the CUDA path, from the definitions alone."""
 import json

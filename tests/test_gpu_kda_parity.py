@@ -14,7 +14,7 @@ import torch
 from linear_attention_sequence_mshortconv_b200 import inputs as W
 from linear_attention_sequence_mshortconv_b200 import kda
 from oracle import oracle as O
-from tests.parity import compare, compare_heads, to_np, tol_for
+from tests.parity import compare, compare_bf16_output, compare_heads, to_np, tol_for
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -183,6 +183,21 @@ def test_image_stream_full_size_sampled_heads():
 
 def test_video_clip_full_size_sampled_heads():
     _sampled_full_size(W.VIDEO_CLIP, [(0, 0), (0, 9)])
+
+
+def test_video_clip_full_size_bf16_output_sampled_heads():
+    # the output the benchmark writes: bf16 o (its fp32 form is checked above)
+    w = W.VIDEO_CLIP
+    inp = W.make_kda_inputs(w, device=DEV)
+    o, ST = kda.forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], chunk=w.chunk,
+                        o_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == 0 and o.dtype == torch.bfloat16
+    cpu = {k: v.cpu() for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    for h in (0, 9):
+        o_ref, S_ref = O.kda_forward_head(cpu["q"], cpu["k"], cpu["v"], cpu["g"], cpu["beta"], 0, h)
+        compare_bf16_output(to_np(o[0, :, h]), o_ref, f"video clip bf16 o[h={h}]")
+        compare(to_np(ST[0, h]), S_ref, "bf16", f"video clip S_T[h={h}]")
 
 
 def test_long_video_full_size_sampled_head():
