@@ -699,9 +699,9 @@ __device__ __forceinline__ void out_rows_general(const OutParams* op, uint32_t o
 // Four roles of 4 warps each (role = warp / 4; warp w4 = warp % 4 also names the TMEM lane
 // quarter it may access):
 //   P (role 0)  prologue: log-decay prefix and references of chunk n, the K+ / Q+ / K- tiles
-//               (or A and P on CUDA cores for a wide chunk).
-//   I (role 1)  inverse: the A|P MMA, A and P out of TMEM, T = (I + A)^{-1}, W^T MMA,
-//               T diag(beta) into the set.
+//               (or A and P on CUDA cores for a wide chunk), the A|P MMA.
+//   I (role 1)  inverse: A and P out of TMEM, T = (I + A)^{-1}, W^T MMA, T diag(beta) into
+//               the set.
 //   X (role 2)  state chain: S^ from the master, the [U | O] MMA, U -> fp16, the master and O
 //               MMAs; one thread per TMEM lane (value column).  Its MMA thread also issues
 //               the TMA loads of q, k, g as soon as a set is free.
@@ -930,7 +930,23 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             fence_async_smem();
             tc_fence_before();
             named_sync(BAR_P, NR);
-            if (rt == 0) mbar_arrive(&bars[B_SC + s]);   // scales, direct flag, tiles (and beta) in place
+            if (rt == 0) {
+                mbar_arrive(&bars[B_SC + s]);   // scales, direct flag, tiles (and beta) in place
+                if (!direct) {
+                    // A|P's TMEM columns are free once the output role has read chunk kc-1's W^T
+                    if (kc > 0) thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
+                    tc_fence_after();
+                    // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the
+                    // state pass reads K- as rows 64-127 and ignores them)
+                    const uint32_t id = idesc_f16(128, 64, true, true);
+                    const uint32_t sset = sbase + s * PL::SET;
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
+                                 sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
+                    umma_commit(&bars[B_AP]);
+                }
+            }
         }
         if (beta_async) cp_async_wait_all();
     } else if (role == 1) {
@@ -941,22 +957,8 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             uint8_t* set = sm + s * PL::SET;
             const uint32_t sset = sbase + s * PL::SET;
             group_wait(&bars[B_SC + s], set_par(kc), ab, rt == 0, BAR_I);   // the prologue is done
-            // A|P's TMEM columns are free once the output role has read chunk kc-1's W^T
-            if (rt == 0 && kc > 0) {
-                thread_wait(&bars[B_APWF], (kc - 1) & 1, ab);
-                tc_fence_after();
-            }
             if (!sDirect[s]) {
-                if (rt == 0) {
-                    // [beta K+; Q+] (M = 128) x K-^T: rows 0-63 give A, rows 64-127 give P (the state
-                    // pass reads K- as rows 64-127 and ignores them)
-                    const uint32_t id = idesc_f16(128, 64, true, true);
-                    #pragma unroll 1
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 256 * kk, 128, 2048),
-                                 sdesc(sset + PL::KM + 256 * kk, 128, 2048), id, kk > 0);
-                    umma_commit(&bars[B_AP]);
-                }
+                // the prologue role issued the A|P MMA (once W^T of chunk kc-1 was read)
                 group_wait(&bars[B_AP], n_ap & 1, ab, rt == 0, BAR_I);
                 ++n_ap;
                 // A (lanes 0-63) -> fp16 tile, P (lanes 64-127) -> the set's P tile
@@ -988,7 +990,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
                 // W^T = (beta K+)^T T^T: M = 128 channels, N = 64 positions, K = 64 positions
                 const uint32_t id = idesc_f16(128, 64, false, false);
-                #pragma unroll 1
+#pragma unroll 1
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16(tmem + TM_APW, sdesc(sset + PL::KP + 4096 * kk, 2048, 128),
                              sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id, kk > 0);
@@ -1110,13 +1112,13 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     // [U | -O]^T += -S^T [W^T | Q+^T]   (N = 128: positions of W, then of Q+); the
                     // O columns accumulate -O, negated back when written out
                     const uint32_t id = idesc_f16(128, 128, false, true, true);
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UO + 128 * ub, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
                 } else {
                     const uint32_t id = idesc_f16(128, 64, false, true, true);   // U^T += -S^T W^T
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, 1);
@@ -1145,23 +1147,23 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (OUT) {
                     // master += U^T K-   and   -O^T += -U^T P^T
                     const uint32_t ua = tmem + TM::UO + 128 * ub;
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, ua + 8 * kk, sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     umma_commit(&bars[B_S]);
                     const uint32_t ido = idesc_f16(128, 64, false, false, true);
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(ua + 64, ua + 8 * kk, sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
                     umma_commit(&bars[B_O + ub]);
                 } else {
                     // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
                     const uint32_t id = idesc_f16(128, 64, false, true, true);
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
                         umma_f16_ts(tmem + TM::UACC, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KP + 256 * kk, 128, 2048), id, kk > 0);
@@ -1184,7 +1186,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (mma) {
                     tc_fence_after();
                     const uint32_t idm = idesc_f16(128, 128, false, false);
-                    #pragma unroll 1
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER + D, tmem + TM::S16 + 64 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
@@ -1240,7 +1242,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t sset = sbase + set_of(x) * PL::SET, vbt = sbase + PL::VB;
             const uint32_t id = idesc_f16(128, 64, true, false, false, std::is_same<TQ, __nv_bfloat16>::value);
             const uint32_t d = tmem + (OUT ? TM::UO + 128 * (x & 1) : TM::UACC);
-            #pragma unroll 1
+#pragma unroll 1
             for (int kk = 0; kk < 4; ++kk)
                 umma_f16(d, sdesc(vbt + 256 * kk, 128, 1024), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
                          kk > 0);
