@@ -137,7 +137,8 @@ enum Bar {
     B_AP = 19, B_W = 20, B_U = 21, B_U2 = 22, B_S = 23,
     B_DRAIN = 24,   // [4] one per MMA-issuing role, after a timeout
     B_APWF = 28,    // the output role has read W^T out of A|P's TMEM columns
-    NBAR = 29
+    B_C1Y = 29,     // MODE_STATE: the output role has rescaled the Phi half of the master
+    NBAR = 30
 };
 // set of chunk x (counted from the segment start) and the phase parity of its set barriers
 __device__ __forceinline__ int set_of(int x) { return x % NSET; }
@@ -575,6 +576,31 @@ __device__ __forceinline__ void transpose8x8_b16(const uint32_t* w, uint32_t (&z
         z[1] = __byte_perm(B1, t0, 0x7610);
         z[2] = __byte_perm(B2, t1, 0x5410);
         z[3] = __byte_perm(B3, t1, 0x7610);
+    }
+}
+
+// One 128-column half of the transposed state at the start of a chunk: S^ = fp16(2^{rp +
+// carry} master) into the 64 fp16x2 columns at hcol, master <- 2^{rm + carry} master in
+// place (columns mcol ..).  sY, sMs: the chunk's per-channel scales.  One thread per TMEM
+// lane (tl: this warp's lane quarter); the stores are waited for by the caller.
+__device__ __forceinline__ void rescale_master(uint32_t tl, uint32_t mcol, uint32_t hcol, const float* sY,
+                                               const float* sMs)
+{
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 64) {
+        float vv[64];
+        uint32_t hv[32];
+        tmem_ld64(tl + mcol + c0, vv);
+#pragma unroll
+        for (int e = 0; e < 64; e += 4) {
+            const float4 y4 = *reinterpret_cast<const float4*>(sY + c0 + e);
+            const float4 m4 = *reinterpret_cast<const float4*>(sMs + c0 + e);
+            hv[e / 2] = pack_f16x2(vv[e] * y4.x, vv[e + 1] * y4.y);
+            hv[e / 2 + 1] = pack_f16x2(vv[e + 2] * y4.z, vv[e + 3] * y4.w);
+            vv[e] *= m4.x; vv[e + 1] *= m4.y; vv[e + 2] *= m4.z; vv[e + 3] *= m4.w;
+        }
+        tmem_st32u_nowait(tl + hcol + c0 / 2, hv);
+        tmem_st64_nowait(tl + mcol + c0, vv);
     }
 }
 
@@ -1068,30 +1094,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             named_sync(BAR_X, NR);
             tc_fence_after();
-            {
-                const float* sY = sSC + s * 3 * D;
-                const float* sMs = sY + D;
-                for (int mi = 0; mi < (OUT ? 1 : 2); ++mi) {
-                    const uint32_t mcol = TM::MASTER + D * mi, hcol = TM::S16 + 64 * mi;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 64) {
-                        float vv[64];
-                        uint32_t hv[32];
-                        tmem_ld64(tl + mcol + c0, vv);
-#pragma unroll
-                        for (int e = 0; e < 64; e += 4) {
-                            const float4 y4 = *reinterpret_cast<const float4*>(sY + c0 + e);
-                            const float4 m4 = *reinterpret_cast<const float4*>(sMs + c0 + e);
-                            hv[e / 2] = pack_f16x2(vv[e] * y4.x, vv[e + 1] * y4.y);
-                            hv[e / 2 + 1] = pack_f16x2(vv[e + 2] * y4.z, vv[e + 3] * y4.w);
-                            vv[e] *= m4.x; vv[e + 1] *= m4.y; vv[e + 2] *= m4.z; vv[e + 3] *= m4.w;
-                        }
-                        tmem_st32u_nowait(tl + hcol + c0 / 2, hv);
-                        tmem_st64_nowait(tl + mcol + c0, vv);
-                    }
-                }
-                tmem_wait_st();
-            }
+            // (MODE_STATE: the Phi half is rescaled by the output role beside this one)
+            rescale_master(tl, TM::MASTER, TM::S16, sSC + s * 3 * D, sSC + s * 3 * D + D);
+            tmem_wait_st();
             tc_fence_before();
             named_sync(BAR_X, NR);
             if (mma && kc >= 1 && kc + 2 < nk && !*sAbort) {
@@ -1157,11 +1162,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         umma_f16_ts(ua + 64, ua + 8 * kk, sdesc(sset + PL::PF + 2048 * kk, 1024, 128), ido, 1);
                     umma_commit(&bars[B_O + ub]);
                 } else {
-                    // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh)
+                    // S chain: master_N += U_N^T K-; Phi chain: U_Phi^T = -Phi^T W^T (fresh), once
+                    // the output role has rescaled the Phi half
 #pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk)
                         umma_f16_ts(tmem + TM::MASTER, tmem + TM::S16 + 8 * kk,
                                     sdesc(sset + PL::KM + 4096 * kk, 2048, 128), idm, 1);
+                    thread_wait(&bars[B_C1Y], kc & 1, ab);
+                    tc_fence_after();
                     const uint32_t id = idesc_f16(128, 64, false, true, true);
 #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
@@ -1295,6 +1303,21 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mbar_arrive(&bars[B_APWF]);   // A|P's TMEM columns may be reused
                 // every tile of the set is ready (the test hook withholds chunk 0's signal)
                 if (!(dbg_drop && kc == 0)) mbar_arrive(&bars[B_PRO + s]);
+            }
+            if constexpr (!OUT) {
+                // ---- the Phi half of the master at the start of chunk kc (beside the chain role's
+                // S half): after the chain's last master update of chunk kc-1 --------------------
+                if (rt == 0) {
+                    thread_wait(&bars[B_SC + s], set_par(kc), ab);
+                    if (kc > 0) thread_wait(&bars[B_S], (kc - 1) & 1, ab);
+                }
+                named_sync(BAR_Y, NR);
+                tc_fence_after();
+                rescale_master(tl, TM::MASTER + D, TM::S16 + 64, sSC + s * 3 * D, sSC + s * 3 * D + D);
+                tmem_wait_st();
+                tc_fence_before();
+                named_sync(BAR_Y, NR);
+                if (rt == 0) mbar_arrive(&bars[B_C1Y]);
             }
             if (mma && !u_done) {
                 thread_wait(&bars[B_INV + s], set_par(kc), ab);
