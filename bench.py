@@ -93,16 +93,17 @@ def conv_alu_roofline(w: W.Workload, conv_ms: float):
             "fmas_per_step": conv_fmas(w)}
 
 
-def traffic_record(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current source of that kernel (else None)."""
+def traffic_record(workload: str):
+    """DRAM bytes (read + write) of one whole forward call of the workload from the
+    committed ncu summary, if it was taken on the current source of the scan kernel
+    (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             recs = json.load(f)
     except (OSError, ValueError):
         return None
-    rec = recs.get(kernel)
+    rec = recs.get(workload)
     if not rec:
         return None
     src = os.path.join(ROOT, rec.get("source", ""))
@@ -112,7 +113,7 @@ def traffic_record(kernel: str):
         return None
     if sha != rec.get("source_sha256"):
         return None
-    return rec.get("dram_bytes_per_launch")
+    return rec.get("dram_bytes_per_step")
 
 
 class ClockSampler:
