@@ -233,23 +233,27 @@ struct Abort {
     int* flag;
     int* status;
 };
+// The slow part of a wait, out of line (one copy per kernel instead of one per wait):
+// sleep-poll the barrier for at most kWaitNs; on expiry raise the abort flag and record
+// DEV_TIMEOUT.
+__device__ __noinline__ void wait_slow(uint64_t* bar, uint32_t parity, int* flag, int* status)
+{
+    if (!mbar_wait_bounded(bar, parity, kWaitNs)) {
+        *flag = 1;
+        atomicCAS(status, DEV_OK, DEV_TIMEOUT);
+    }
+}
+// One thread waits alone (before issuing MMAs that depend on another role).
+__device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, const Abort& a)
+{
+    if (!*a.flag && !mbar_try_wait(bar, parity)) wait_slow(bar, parity, a.flag, a.status);
+}
 // One thread polls; the role (bar_id, NR threads) waits at its named barrier.
 __device__ __forceinline__ void group_wait(uint64_t* bar, uint32_t parity, const Abort& a, bool poller, int bar_id)
 {
-    if (poller && !*a.flag && !mbar_wait_bounded(bar, parity, kWaitNs)) {
-        *a.flag = 1;
-        atomicCAS(a.status, DEV_OK, DEV_TIMEOUT);
-    }
+    if (poller) thread_wait(bar, parity, a);
     named_sync(bar_id, NR);
     tc_fence_after();
-}
-// One thread waits alone (before issuing MMAs that depend on the other group).
-__device__ __forceinline__ void thread_wait(uint64_t* bar, uint32_t parity, const Abort& a)
-{
-    if (!*a.flag && !mbar_wait_bounded(bar, parity, kWaitNs)) {
-        *a.flag = 1;
-        atomicCAS(a.status, DEV_OK, DEV_TIMEOUT);
-    }
 }
 
 // 16 rows x 2 channels (one 4-byte word per row) of a [64][128] 2-byte tile in shared
@@ -993,16 +997,14 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_ld64(tl + TM_APW, v);
                     const bool isP = q4 >= 2;
                     const int i = 32 * (q4 & 1) + lane;
+                    const int lim = i + (isP ? 1 : 0);        // A: columns < i; P: columns <= i
+                    uint8_t* dst = set + (isP ? PL::PF : PL::TF) + cm64(i, 0);
 #pragma unroll
                     for (int g8 = 0; g8 < 8; ++g8) {
                         float f[8];
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const int col = 8 * g8 + j;
-                            f[j] = (isP ? (col <= i) : (col < i)) ? v[8 * g8 + j] : 0.f;
-                        }
-                        uint8_t* dst = isP ? set + PL::PF + cm64(i, 8 * g8) : set + PL::TF + cm64(i, 8 * g8);
-                        *reinterpret_cast<uint4*>(dst) = pack8_f16(f);
+                        for (int j = 0; j < 8; ++j) f[j] = 8 * g8 + j < lim ? v[8 * g8 + j] : 0.f;
+                        *reinterpret_cast<uint4*>(dst + g8 * 1024) = pack8_f16(f);
                     }
                 }
                 tc_fence_before();
@@ -1035,10 +1037,12 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint4 u = *pc;
                     const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
                     uint32_t ow[4];
+                    const uint4 bq = *reinterpret_cast<const uint4*>(sBk + j0);   // beta of columns j0 .. j0+7
+                    const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const float2 tv = unpack_f16x2(uw[m]);
-                        ow[m] = pack2_in<TQ>(tv.x * bf16_bits_to_f32(sBk[j0 + 2 * m]), tv.y * bf16_bits_to_f32(sBk[j0 + 2 * m + 1]));
+                        ow[m] = pack2_in<TQ>(tv.x * __uint_as_float(bw[m] << 16), tv.y * __uint_as_float(bw[m] & 0xffff0000u));
                     }
                     *pc = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }
