@@ -128,17 +128,19 @@ constexpr int MISC_BYTES = 12320;
 enum Bar {
     B_LD = 0,       // [3] set s: q, k, g of its chunk landed
     B_TV = 3,       // the v tile landed
-    B_VE = 4,       // the U~ MMA that read the v tile is done
-    B_SC = 5,       // [3] set s: prologue done (scales, direct flag, K+ / Q+ / K- tiles, beta)
-    B_INV = 8,      // [3] set s: T ready
-    B_PRO = 11,     // [3] set s: every tile ready (W^T written)
-    B_EMPTY = 14,   // [3] set s: the chain's last MMA on it is done
-    B_O = 17,       // [2] [U | O] buffer x: the chunk's O is complete
-    B_AP = 19, B_W = 20, B_U = 21, B_U2 = 22, B_S = 23,
-    B_DRAIN = 24,   // [4] one per MMA-issuing role, after a timeout
-    B_APWF = 28,    // the output role has read W^T out of A|P's TMEM columns
-    B_C1Y = 29,     // MODE_STATE: the output role has rescaled the Phi half of the master
-    NBAR = 30
+    B_VE = 4,       // [2] chunk parity x: the U~ MMA of chunk x (which read the v tile) is done.
+                    // Two of them: U~ of chunk kc+1 may be done before the chain role has
+                    // polled chunk kc's, and a waiter must never be two phases behind
+    B_SC = 6,       // [3] set s: prologue done (scales, direct flag, K+ / Q+ / K- tiles, beta)
+    B_INV = 9,      // [3] set s: T ready
+    B_PRO = 12,     // [3] set s: every tile ready (W^T written)
+    B_EMPTY = 15,   // [3] set s: the chain's last MMA on it is done
+    B_O = 18,       // [2] [U | O] buffer x: the chunk's O is complete
+    B_AP = 20, B_W = 21, B_U = 22, B_U2 = 23, B_S = 24,
+    B_APWF = 25,    // the output role has read W^T out of A|P's TMEM columns
+    B_C1Y = 26,     // MODE_STATE: the output role has rescaled the Phi half of the master
+    B_DRAIN = 27,   // [4] one per MMA-issuing role, after a timeout
+    NBAR = 31
 };
 // set of chunk x (counted from the segment start) and the phase parity of its set barriers
 __device__ __forceinline__ int set_of(int x) { return x % NSET; }
@@ -1114,7 +1116,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (mma) {
                 // U~ (Y) initialised the U columns; -W^T and Q+ are in the set (I)
-                thread_wait(&bars[B_VE], kc & 1, ab);
+                thread_wait(&bars[B_VE + (kc & 1)], (kc >> 1) & 1, ab);
                 thread_wait(&bars[B_PRO + s], set_par(kc), ab);
                 tc_fence_after();
                 if (OUT) {
@@ -1258,7 +1260,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int kk = 0; kk < 4; ++kk)
                 umma_f16(d, sdesc(vbt + 256 * kk, 128, 1024), sdesc(sset + PL::TF + 2 * T_LBO * kk, T_LBO, 128), id,
                          kk > 0);
-            umma_commit(&bars[B_VE]);   // U~ done: the v tile may be refilled
+            umma_commit(&bars[B_VE + (x & 1)]);   // U~ done: the v tile may be refilled
         };
         // chunk x's output rows: O^T (lane j, columns 64 + i of its [U | O] buffer) -> o
         auto out_rows = [&](int x) {
@@ -1334,7 +1336,7 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             // the v tile is free once U~ of chunk kc is done: chunk kc+1's may land
             if (loader && kc + 1 < nk && !*sAbort) {
-                thread_wait(&bars[B_VE], kc & 1, ab);
+                thread_wait(&bars[B_VE + (kc & 1)], (kc >> 1) & 1, ab);
                 if (!*sAbort) {
                     tma_v(n + 1);
                     v_issued = kc + 2;
