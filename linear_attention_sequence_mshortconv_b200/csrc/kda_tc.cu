@@ -842,6 +842,38 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     };
     const TQ* tq = nullptr;
 
+    // ---- the first NSET chunks' q, k, g (the chain role's MMA thread issues every load of
+    // them), and the initial state in TMEM, split over the four roles: 32 columns each of
+    // the master (MODE_STATE: of N from 0 and of Phi from I), lane j = value column j -----
+    if (t == 2 * NR)
+        for (int x = 0; x < min(NSET, nk); ++x) tma_set(n0 + x);
+    {
+        const int j = 32 * q4 + lane, c0 = 32 * role;
+        float vv[32];
+        if (MODE == MODE_STATE) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+            tmem_st32(tl + TM::MASTER + c0, vv);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) vv[e] = (c0 + e == j) ? 1.f : 0.f;
+            tmem_st32(tl + TM::MASTER + D + c0, vv);
+        } else {
+            if (S_in) {
+                const size_t idx = s_in_per_segment ? (size_t)slot : (size_t)seq * H + h;
+                const float* src = S_in + idx * D * D + j;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) vv[e] = src[(size_t)(c0 + e) * D];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+            }
+            tmem_st32(tl + TM::MASTER + c0, vv);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
     if (role == 0) {
         // ================= P: prologue of chunk n0 + kc =====================================
         const int cp = rt & 63, rh = rt >> 6;   // channel pair, 32-row half
@@ -1058,38 +1090,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // ================= X: the state chain of chunk n0 + kc ==============================
         const int j = 32 * q4 + lane;              // value column of this thread (TMEM lane)
         const bool mma = rt == 0;
-        // rt 0 also issues the loads of q, k, g: the first NSET chunks now, chunk kc+2 into the
-        // set of chunk kc-1 once the chain is done with it
-        int ld_issued = 0;
-        if (mma) {
-            ld_issued = min(NSET, nk);
-            for (int x = 0; x < ld_issued; ++x) tma_set(n0 + x);
-        }
-        // initial state in TMEM (MODE_STATE: N from 0, Phi from I)
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            float vv[32];
-            if (MODE == MODE_STATE) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) vv[e] = 0.f;
-                tmem_st32(tl + TM::MASTER + c0, vv);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) vv[e] = (c0 + e == j) ? 1.f : 0.f;
-                tmem_st32(tl + TM::MASTER + D + c0, vv);
-            } else {
-                if (S_in) {
-                    const size_t idx = s_in_per_segment ? (size_t)slot : (size_t)seq * H + h;
-                    const float* src = S_in + idx * D * D + j;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) vv[e] = src[(size_t)(c0 + e) * D];
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) vv[e] = 0.f;
-                }
-                tmem_st32(tl + TM::MASTER + c0, vv);
-            }
-        }
-        tc_fence_before();
-        named_sync(BAR_X, NR);
+        // rt 0 also issues the loads of q, k, g: chunk kc+2 into the set of chunk kc-1 once
+        // the chain is done with it (the first NSET chunks' went out before the roles split)
+        int ld_issued = mma ? min(NSET, nk) : 0;
         for (int kc = 0; kc < nk; ++kc) {
             const int s = set_of(kc), ub = kc & 1;   // buffer set; [U | O] buffer
             const uint32_t sset = sbase + s * PL::SET;
