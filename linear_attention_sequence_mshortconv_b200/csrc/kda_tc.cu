@@ -593,20 +593,24 @@ __device__ __forceinline__ void rescale_master(uint32_t tl, uint32_t mcol, uint3
                                                const float* sMs)
 {
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 64) {
-        float vv[64];
-        uint32_t hv[32];
-        tmem_ld64(tl + mcol + c0, vv);
+    for (int c0 = 0; c0 < D; c0 += 32) {
+        float vv[32];
+        uint32_t hv[16], mv[32];
+        tmem_ld32(tl + mcol + c0, vv);
 #pragma unroll
-        for (int e = 0; e < 64; e += 4) {
+        for (int e = 0; e < 32; e += 4) {   // packed fp32 multiplies, two channels each
             const float4 y4 = *reinterpret_cast<const float4*>(sY + c0 + e);
             const float4 m4 = *reinterpret_cast<const float4*>(sMs + c0 + e);
-            hv[e / 2] = pack_f16x2(vv[e] * y4.x, vv[e + 1] * y4.y);
-            hv[e / 2 + 1] = pack_f16x2(vv[e + 2] * y4.z, vv[e + 3] * y4.w);
-            vv[e] *= m4.x; vv[e + 1] *= m4.y; vv[e + 2] *= m4.z; vv[e + 3] *= m4.w;
+            const float2 v0 = make_float2(vv[e], vv[e + 1]), v1 = make_float2(vv[e + 2], vv[e + 3]);
+            const float2 h0 = __fmul2_rn(v0, make_float2(y4.x, y4.y)), h1 = __fmul2_rn(v1, make_float2(y4.z, y4.w));
+            hv[e / 2] = pack_f16x2(h0.x, h0.y);
+            hv[e / 2 + 1] = pack_f16x2(h1.x, h1.y);
+            const float2 m0 = __fmul2_rn(v0, make_float2(m4.x, m4.y)), m1 = __fmul2_rn(v1, make_float2(m4.z, m4.w));
+            mv[e] = __float_as_uint(m0.x); mv[e + 1] = __float_as_uint(m0.y);
+            mv[e + 2] = __float_as_uint(m1.x); mv[e + 3] = __float_as_uint(m1.y);
         }
-        tmem_st32u_nowait(tl + hcol + c0 / 2, hv);
-        tmem_st64_nowait(tl + mcol + c0, vv);
+        tmem_st16u_nowait(tl + hcol + c0 / 2, hv);
+        tmem_st32u_nowait(tl + mcol + c0, mv);
     }
 }
 
@@ -1075,8 +1079,9 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const float2 tv = unpack_f16x2(uw[m]);
-                        ow[m] = pack2_in<TQ>(tv.x * __uint_as_float(bw[m] << 16), tv.y * __uint_as_float(bw[m] & 0xffff0000u));
+                        const float2 tb = __fmul2_rn(unpack_f16x2(uw[m]),
+                                                     make_float2(__uint_as_float(bw[m] << 16), __uint_as_float(bw[m] & 0xffff0000u)));
+                        ow[m] = pack2_in<TQ>(tb.x, tb.y);
                     }
                     *pc = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                 }

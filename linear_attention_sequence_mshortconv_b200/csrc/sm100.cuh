@@ -298,6 +298,16 @@ __device__ __forceinline__ void tmem_st64_nowait(uint32_t taddr, const float (&v
     tmem_st32u_nowait(taddr + 32, hi);
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x 16 columns of raw 32-bit words, without waiting (tmem_wait_st before reuse)
+__device__ __forceinline__ void tmem_st16u_nowait(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 // 32 lanes x 16 columns of raw 32-bit words (e.g. packed fp16 pairs)
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&r)[16])
 {
