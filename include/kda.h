@@ -415,8 +415,8 @@ uint64_t kda_kernel_launches(void);
 /* Test hook for the device-side failure path (the paper has no counterpart; this is
  * how the timeout handling is exercised without a fault or a hang).  While `on` is
  * non-zero, every later launch of the tensor-core scan withholds, in each CTA, the
- * first "tiles ready" signal from its producer warps to its consumer warps.  The
- * consumer's bounded wait (2 s) then runs out: the CTA records the timeout in the device
+ * first "every tile of the chunk ready" signal to the warps that run the state chain.
+ * Their bounded wait (2 s) then runs out: the CTA records the timeout in the device
  * status word, stops waiting, drains its own tensor-core and TMA work, frees its tensor
  * memory and exits.  The call still returns KDA_OK (errors on the device are reported
  * asynchronously); o and S_T are undefined; kda_last_device_error() then returns

@@ -30,7 +30,7 @@ template <> __device__ __forceinline__ __half from_f32<__half>(float x) { return
 // ---- launch accounting and optional per-kernel event timing ------------------------
 void count_launch();
 // Test hook (kda_debug_drop_handoff): non-zero makes the tensor-core scan withhold one
-// producer -> consumer hand-off per CTA, so a bounded wait runs out.
+// hand-off between its warp roles per CTA, so a bounded wait runs out.
 int debug_drop_handoff();
 // Records CUDA events around the kernels launched in its lifetime when profiling is
 // enabled (kda_profile_enable); a no-op otherwise.

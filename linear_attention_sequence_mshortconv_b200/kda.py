@@ -607,8 +607,8 @@ def profile_collect(name: str):
 
 
 def debug_drop_handoff(on: bool) -> None:
-    """Test hook: while on, the tensor-core scan withholds one producer -> consumer
-    hand-off per CTA, so its bounded wait runs out and the call reports a timeout."""
+    """Test hook: while on, the tensor-core scan withholds one hand-off between its warp
+    roles per CTA, so a bounded wait runs out and the call reports a timeout."""
     load_library().kda_debug_drop_handoff(1 if on else 0)
 
 
