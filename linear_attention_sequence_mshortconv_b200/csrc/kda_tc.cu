@@ -1451,6 +1451,8 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
         else cp_async_wait_all();
         __syncthreads();                         // M_p staged, sS written
         const float* sM = csm + (p & 1) * D * CB_LD;
+        float2 a2[4] = {make_float2(acc[0], acc[1]), make_float2(acc[2], acc[3]), make_float2(acc[4], acc[5]),
+                        make_float2(acc[6], acc[7])};   // packed fp32 FMAs, two columns each
 #pragma unroll 4
         for (int k4 = 0; k4 < D / 4; ++k4) {
             const float4 m = *reinterpret_cast<const float4*>(sM + r * CB_LD + 4 * k4);
@@ -1460,14 +1462,18 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
                 const int k = 4 * k4 + u;
                 const float4 s0 = *reinterpret_cast<const float4*>(sS + k * 16 + c8);
                 const float4 s1 = *reinterpret_cast<const float4*>(sS + k * 16 + c8 + 4);
-                acc[0] = fmaf(mk[u], s0.x, acc[0]); acc[1] = fmaf(mk[u], s0.y, acc[1]);
-                acc[2] = fmaf(mk[u], s0.z, acc[2]); acc[3] = fmaf(mk[u], s0.w, acc[3]);
-                acc[4] = fmaf(mk[u], s1.x, acc[4]); acc[5] = fmaf(mk[u], s1.y, acc[5]);
-                acc[6] = fmaf(mk[u], s1.z, acc[6]); acc[7] = fmaf(mk[u], s1.w, acc[7]);
+                const float2 mm = make_float2(mk[u], mk[u]);
+                a2[0] = __ffma2_rn(mm, make_float2(s0.x, s0.y), a2[0]);
+                a2[1] = __ffma2_rn(mm, make_float2(s0.z, s0.w), a2[1]);
+                a2[2] = __ffma2_rn(mm, make_float2(s1.x, s1.y), a2[2]);
+                a2[3] = __ffma2_rn(mm, make_float2(s1.z, s1.w), a2[3]);
             }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s[j] = acc[j];
+        for (int j = 0; j < 4; ++j) {
+            s[2 * j] = a2[j].x;
+            s[2 * j + 1] = a2[j].y;
+        }
     }
 }
 
