@@ -555,7 +555,7 @@ def run_gpu(args, ws, rank, local, w: W.Workload):
     if rank == 0 and not args.quick:
         # the other forward configurations of the workload set, each on its own line entry
         others = [x for x in (W.IMAGE_STREAM, W.FUSED_MIXED, W.LONG_VIDEO) if x.name != w.name and not args.tokens]
-        line["extra_workloads"] = [forward_record(x, max(20, args.steps // 4), peaks, peak_kind) for x in others]
+        line["extra_workloads"] = [forward_record(x, max(20, args.steps), peaks, peak_kind) for x in others]
     if args.extra and rank == 0:
         extra = line.setdefault("extra_workloads", [])
         # the headline workload with the output side of Eq. 15 fused (Sigmoid(gate) *
