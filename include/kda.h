@@ -99,8 +99,10 @@ size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype
  *             of the same call rounded.  (bf16 output rounding alone is up to 2^-9 of
  *             |o|, which for heavy-tailed outputs exceeds a few percent of RMS(o).)
  *   chunk   : tokens per chunk of the chunkwise evaluation: 0 = the default for
- *             the dtype, else one of {16, 32, 64}.  The result does not depend on it
- *             beyond rounding.
+ *             the dtype (64 for bf16, 16 for fp32), else one of {16, 32, 64, 128}.  The
+ *             result does not depend on it beyond rounding.  The tensor-core kernel runs
+ *             chunk 64 only; any other chunk runs on the fp32 CUDA-core kernels (128 on
+ *             one that takes the key channels in blocks of 32), which are much slower.
  *   workspace, workspace_bytes : device scratch of at least
  *             kda_forward_workspace_size(...) bytes, 256-byte aligned; or NULL, in
  *             which case the library takes and returns it with cudaMallocAsync /

@@ -64,7 +64,7 @@ extern "C" kda_status kda_forward_noalloc(const void* q, const void* k, const vo
     if ((dtype != KDA_F32 && dtype != KDA_BF16) || (o_dtype != KDA_F32 && o_dtype != KDA_BF16))
         return KDA_ERR_INVALID_ARG;
     if (!dim_ok(Dk) || !dim_ok(Dv)) return KDA_ERR_UNSUPPORTED;
-    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return KDA_ERR_UNSUPPORTED;
     if ((int64_t)B * T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     if (B == 0) return KDA_OK;

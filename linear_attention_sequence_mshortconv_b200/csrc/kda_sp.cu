@@ -205,7 +205,7 @@ bool shard_ok(int B, int T, int H, int D, kda_dtype dtype, int chunk)
 {
     if (B < 0 || T < 0 || H <= 0 || !dim_ok(D)) return false;
     if (dtype != KDA_F32 && dtype != KDA_BF16) return false;
-    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64) return false;
+    if (chunk != 0 && chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return false;
     return (int64_t)B * H <= 65535;
 }
 

@@ -167,7 +167,8 @@ def forward(q, k, v, g, beta, S0=None, *, chunk: int = 0, o=None, S_T=None,
 
     q, k, g: [B,T,H,Dk]; v: [B,T,H,Dv]; beta: [B,T,H] -- all bf16 or all fp32 CUDA
     tensors; S0: [B,H,Dk,Dv] fp32 or None.  o_dtype: torch.float32 or torch.bfloat16
-    (default: the input dtype).  Returns (o, S_T or None)."""
+    (default: the input dtype).  chunk: 0 (the dtype's default), 16, 32, 64 or 128; only
+    64 runs on the tensor cores.  Returns (o, S_T or None)."""
     lib = load_library()
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]

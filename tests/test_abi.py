@@ -48,8 +48,9 @@ def test_host_rejects_bad_arguments(lib):
     assert lib.kda_forward(P, P, P, P, P, P, P, P, -1, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 1
     # null tensors with work to do
     assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 1, 0, P, 0, P) == 1
-    # chunk not in {16, 32, 64}
+    # chunk not in {16, 32, 64, 128}
     assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 1, 24, P, 0, P) == 2
+    assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 1, 256, P, 0, P) == 2
     # bad dtype / output dtype
     assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 7, 1, 0, P, 0, P) == 1
     assert lib.kda_forward(P, P, P, P, P, P, P, P, 1, 8, 1, 32, 32, 1, 9, 0, P, 0, P) == 1
@@ -83,7 +84,7 @@ def test_sequence_parallel_calls_reject_bad_arguments(lib):
     assert lib.kda_sp_prefix(d, 2, -1, P, d, 1, 1, 32, P) == 1
     assert lib.kda_sp_prefix(d, 2, 1, P, P, 1, 1, 32, P) == 1
     assert lib.kda_sp_prefix(d, 2, 1, P, d, 1, 1, 48, P) == 2
-    # output: bad output dtype, chunk not in {16, 32, 64}
+    # output: bad output dtype, chunk not in {16, 32, 64, 128}
     assert lib.kda_sp_output(d, d, d, d, d, P, d, P, 1, 8, 1, 32, 1, 9, 0, P, 0, P) == 1
     assert lib.kda_sp_output(d, d, d, d, d, P, d, P, 1, 8, 1, 32, 1, 1, 24, P, 0, P) == 2
     assert lib.kda_sp_workspace_size(1, 8, 1, 48, 1, 0) == 0

@@ -83,12 +83,24 @@ def test_short_and_boundary_lengths(T):
     compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what=f"T={T}")
 
 
-@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
 def test_chunk_size_does_not_change_the_result(chunk):
     inp = _custom(1, 200, 2, 128, 128, torch.bfloat16, seed=5)
     o, ST = _run_gpu(inp, chunk=chunk)
     o_ref, S_ref = _oracle(inp)
     compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what=f"chunk={chunk}")
+
+
+@pytest.mark.parametrize("B,T,H,Dk,Dv,g_hi", [(1, 300, 2, 32, 64, 0.1), (2, 129, 1, 64, 32, 0.1),
+                                              (1, 128, 1, 128, 128, 0.1), (1, 257, 1, 128, 32, 3.0)])
+def test_chunk_128_fp32(B, T, H, Dk, Dv, g_hi):
+    """128-token chunks (key channels taken in blocks of 32): every head width, a chunk
+    that is exactly the sequence, ragged tails, an initial state, and strong decay."""
+    inp = _custom(B, T, H, Dk, Dv, torch.float32, seed=T + Dk, g_hi=g_hi)
+    S0 = torch.randn(B, H, Dk, Dv, generator=torch.Generator().manual_seed(T)) * 0.3
+    o, ST = _run_gpu(inp, chunk=128, S0=S0)
+    o_ref, S_ref = _oracle(inp, S0=S0)
+    compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "fp32", what=f"chunk 128 {B}x{T}x{H} {Dk}x{Dv}")
 
 
 def test_initial_state_and_split_resume():

@@ -113,13 +113,14 @@ def test_sp_shard_maps_bf16():
     _check_maps(inp, MN, "bf16")
 
 
-def test_sp_cuda_core_route_fp32():
+@pytest.mark.parametrize("chunk", [16, 128])
+def test_sp_cuda_core_route_fp32(chunk):
     B, H, D = 1, 2, 32
-    cuts = [0, 50, 66, 143]
+    cuts = [0, 50, 66, 143] if chunk == 16 else [0, 130, 140, 400]
     inp = _rows(B, cuts[-1], H, D, torch.float32, seed=15)
     S0 = torch.randn(B, H, D, D, generator=torch.Generator().manual_seed(16)) * 0.3
-    MN_all = _check_rows(inp, cuts, S0, "fp32", chunk=16)
-    _check_maps(_shard(inp, 0, 50), MN_all[0], "fp32")
+    MN_all = _check_rows(inp, cuts, S0, "fp32", chunk=chunk)
+    _check_maps(_shard(inp, 0, cuts[1]), MN_all[0], "fp32")
 
 
 def test_sp_prefix_fold_against_float64():

@@ -84,12 +84,12 @@ def test_varlen_zero_state_default_and_single_sample_equals_forward():
         compare(to_np(o1)[0, :, h], o_ref[:, h], "bf16", f"forward o h={h}")
 
 
-@pytest.mark.parametrize("D", [32, 128])
-def test_varlen_fp32_cuda_core_path(D):
-    cu = [0, 5, 5, 40, 41, 64]
+@pytest.mark.parametrize("D,chunk", [(32, 16), (128, 16), (64, 128)])
+def test_varlen_fp32_cuda_core_path(D, chunk):
+    cu = [0, 5, 5, 40, 41, 64] if chunk == 16 else [0, 5, 5, 140, 141, 300]
     inp = _packed(cu[-1], 2, D, D, torch.float32, seed=5)
     S0 = torch.randn(len(cu) - 1, 2, D, D, generator=torch.Generator().manual_seed(6))
-    _check(cu, inp, S0, "fp32", chunk=16)
+    _check(cu, inp, S0, "fp32", chunk=chunk)
 
 
 def test_varlen_workspace_and_rejections():
