@@ -1386,19 +1386,25 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
-// S_start(p+1) = M_p S_start(p) + N_p in fp32 on CUDA cores.  Grid (D/16, H, B), 256
-// threads: thread t owns row t/2 and 8 of the CTA's 16 state columns.  M_{p+1} streams
-// into the second shared buffer (cp.async) while step p computes from the first.
-constexpr int CB_THREADS = 256;
+// S_start(p+1) = M_p S_start(p) + N_p in fp32 on CUDA cores.  Grid (D/16, H, B), 128
+// threads: thread t owns column quad t%4 of the CTA's 16 state columns on rows t/4 + 32i
+// (i = 0..3), so one 16-byte read of M (four k of a row) and one of S (four columns of a
+// k) feed 8 packed multiply-adds.  Three shared buffers hold M_p, M_{p+1}, M_{p+2}: the
+// cp.async of M_{p+2} is issued as step p starts, two steps ahead of its use.
+constexpr int CB_THREADS = 128;
 constexpr int CB_LD = 132;      // row stride in floats (16-byte rows for cp.async)
-constexpr int cb_smem_bytes() { return (2 * D * CB_LD + D * 16) * (int)sizeof(float); }
+constexpr int CB_NBUF = 3;
+constexpr int cb_smem_bytes() { return (CB_NBUF * D * CB_LD + D * 16) * (int)sizeof(float); }
 
-__device__ __forceinline__ void cb_stage(float* dst, const float* M, int t)
+// One commit group per map, empty past the last one, so group p always holds M_p.
+__device__ __forceinline__ void cb_stage(float* dst, const float* M, int t, bool any)
 {
+    if (any) {
 #pragma unroll
-    for (int u = 0; u < D * D / 4 / CB_THREADS; ++u) {
-        const int i = t + u * CB_THREADS, row = i >> 5, col = (i & 31) * 4;
-        cp_async16(dst + row * CB_LD + col, M + (size_t)row * D + col);
+        for (int u = 0; u < D * D / 4 / CB_THREADS; ++u) {
+            const int i = t + u * CB_THREADS, row = i >> 5, col = (i & 31) * 4;
+            cp_async16(dst + row * CB_LD + col, M + (size_t)row * D + col);
+        }
     }
     cp_async_commit();
 }
@@ -1412,10 +1418,11 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
                    float* __restrict__ starts, int H, int P, const int* __restrict__ seqinfo)
 {
     extern __shared__ __align__(16) float csm[];
-    float* sS = csm + 2 * D * CB_LD;     // [128][16]
-    const int t = threadIdx.x, col0 = blockIdx.x * 16;
+    float* sS = csm + CB_NBUF * D * CB_LD;   // [128][16]
+    const int t = threadIdx.x;
+    const int rg = t >> 2, c4 = (t & 3) * 4;          // rows rg + 32 i, columns c4 .. c4+3
+    const int col = blockIdx.x * 16 + c4;
     const int bh = blockIdx.z * H + blockIdx.y;
-    const int r = t >> 1, c8 = (t & 1) * 8;
     size_t map0 = (size_t)bh * (P - 1), start0 = (size_t)bh * P;
     if (seqinfo) {
         P = seqinfo[3 * blockIdx.z];
@@ -1424,56 +1431,60 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
         if (P == 0) return;
     }
     const float* mp = maps + map0 * 2 * D * D;   // [P-1][N | M]
-    if (P > 1) cb_stage(csm, mp + D * D, t);
-    float s[8], nxt[8];   // nxt: this thread's 8 values of N_p, loaded one step ahead
+    auto map_m = [&](int p) { return mp + (size_t)p * 2 * D * D + D * D; };
+    cb_stage(csm, mp + D * D, t, P > 1);
+    cb_stage(csm + D * CB_LD, P > 2 ? map_m(1) : mp, t, P > 2);
+    float4 s[4], nxt[4];   // nxt: this thread's values of N_p, loaded one step ahead
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s[j] = S0 ? S0[((size_t)bh * D + r) * D + col0 + c8 + j] : 0.f;
+    for (int i = 0; i < 4; ++i) {   // the caller's S0 need not be 16-byte aligned
+        const float* s0 = S0 + ((size_t)bh * D + rg + 32 * i) * D + col;
+        s[i] = S0 ? make_float4(s0[0], s0[1], s0[2], s0[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     auto load_n = [&](int p) {
-        const float4* n4 = reinterpret_cast<const float4*>(mp + (size_t)p * 2 * D * D + (size_t)r * D + col0 + c8);
-        const float4 a = n4[0], b = n4[1];
-        nxt[0] = a.x; nxt[1] = a.y; nxt[2] = a.z; nxt[3] = a.w; nxt[4] = b.x; nxt[5] = b.y; nxt[6] = b.z; nxt[7] = b.w;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            nxt[i] = *reinterpret_cast<const float4*>(mp + (size_t)p * 2 * D * D + (size_t)(rg + 32 * i) * D + col);
     };
     if (P > 1) load_n(0);
     for (int p = 0; p < P; ++p) {
-        float4* out = reinterpret_cast<float4*>(starts + (start0 + p) * D * D + (size_t)r * D + col0 + c8);
-        out[0] = make_float4(s[0], s[1], s[2], s[3]);
-        out[1] = make_float4(s[4], s[5], s[6], s[7]);
+        float* out = starts + (start0 + p) * D * D + col;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(out + (size_t)(rg + 32 * i) * D) = s[i];
         if (p == P - 1) break;
-        float acc[8];
+        float2 a2[4][2];   // packed fp32 FMAs: row i, column pairs (c4, c4+1) and (c4+2, c4+3)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = nxt[j];
+        for (int i = 0; i < 4; ++i) {
+            a2[i][0] = make_float2(nxt[i].x, nxt[i].y);
+            a2[i][1] = make_float2(nxt[i].z, nxt[i].w);
+        }
         if (p + 1 < P - 1) load_n(p + 1);        // in flight during this step
-        __syncthreads();                         // sS and the other buffer are free
+        __syncthreads();                         // sS and the buffer of M_{p-1} are free
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sS[r * 16 + c8 + j] = s[j];
-        if (p + 1 < P - 1) cb_stage(csm + ((p + 1) & 1) * D * CB_LD, mp + (size_t)(p + 1) * 2 * D * D + D * D, t);
-        if (p + 1 < P - 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else cp_async_wait_all();
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(sS + (rg + 32 * i) * 16 + c4) = s[i];
+        cb_stage(csm + ((p + 2) % CB_NBUF) * D * CB_LD, p + 2 < P - 1 ? map_m(p + 2) : mp, t, p + 2 < P - 1);
+        asm volatile("cp.async.wait_group 2;" ::: "memory");   // groups 0..p done: M_p landed
         __syncthreads();                         // M_p staged, sS written
-        const float* sM = csm + (p & 1) * D * CB_LD;
-        float2 a2[4] = {make_float2(acc[0], acc[1]), make_float2(acc[2], acc[3]), make_float2(acc[4], acc[5]),
-                        make_float2(acc[6], acc[7])};   // packed fp32 FMAs, two columns each
-#pragma unroll 4
+        const float* sM = csm + (p % CB_NBUF) * D * CB_LD;
+#pragma unroll 2
         for (int k4 = 0; k4 < D / 4; ++k4) {
-            const float4 m = *reinterpret_cast<const float4*>(sM + r * CB_LD + 4 * k4);
-            const float mk[4] = {m.x, m.y, m.z, m.w};
+            float4 m[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) m[i] = *reinterpret_cast<const float4*>(sM + (rg + 32 * i) * CB_LD + 4 * k4);
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int k = 4 * k4 + u;
-                const float4 s0 = *reinterpret_cast<const float4*>(sS + k * 16 + c8);
-                const float4 s1 = *reinterpret_cast<const float4*>(sS + k * 16 + c8 + 4);
-                const float2 mm = make_float2(mk[u], mk[u]);
-                a2[0] = __ffma2_rn(mm, make_float2(s0.x, s0.y), a2[0]);
-                a2[1] = __ffma2_rn(mm, make_float2(s0.z, s0.w), a2[1]);
-                a2[2] = __ffma2_rn(mm, make_float2(s1.x, s1.y), a2[2]);
-                a2[3] = __ffma2_rn(mm, make_float2(s1.z, s1.w), a2[3]);
+                const float4 sv = *reinterpret_cast<const float4*>(sS + (4 * k4 + u) * 16 + c4);
+                const float2 lo = make_float2(sv.x, sv.y), hi = make_float2(sv.z, sv.w);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float mk = u == 0 ? m[i].x : u == 1 ? m[i].y : u == 2 ? m[i].z : m[i].w;
+                    const float2 mm = make_float2(mk, mk);
+                    a2[i][0] = __ffma2_rn(mm, lo, a2[i][0]);
+                    a2[i][1] = __ffma2_rn(mm, hi, a2[i][1]);
+                }
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            s[2 * j] = a2[j].x;
-            s[2 * j + 1] = a2[j].y;
-        }
+        for (int i = 0; i < 4; ++i) s[i] = make_float4(a2[i][0].x, a2[i][0].y, a2[i][1].x, a2[i][1].y);
     }
 }
 
