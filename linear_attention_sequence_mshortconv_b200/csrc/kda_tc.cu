@@ -1386,15 +1386,17 @@ kda_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
-// S_start(p+1) = M_p S_start(p) + N_p in fp32 on CUDA cores.  Grid (D/16, H, B), 128
-// threads: thread t owns column quad t%4 of the CTA's 16 state columns on rows t/4 + 32i
-// (i = 0..3), so one 16-byte read of M (four k of a row) and one of S (four columns of a
-// k) feed 8 packed multiply-adds.  Three shared buffers hold M_p, M_{p+1}, M_{p+2}: the
-// cp.async of M_{p+2} is issued as step p starts, two steps ahead of its use.
-constexpr int CB_THREADS = 128;
+// S_start(p+1) = M_p S_start(p) + N_p in fp32 on CUDA cores.  Grid (D/16, H, B), 256
+// threads in two halves that split each product's k sum (k < 64 and k >= 64), so every
+// SM partition runs one warp of each.  Thread t of a half owns column quad t%4 of the
+// CTA's 16 state columns on rows t/4 + 32i (i = 0..3): one 16-byte read of M (four k of a
+// row) and one of S (four columns of a k) feed 8 packed multiply-adds.  The second half
+// hands its partial sums to the first through shared memory.  Three shared buffers hold
+// M_p, M_{p+1}, M_{p+2}: the cp.async of M_{p+2} is issued as step p starts.
+constexpr int CB_THREADS = 256;
 constexpr int CB_LD = 132;      // row stride in floats (16-byte rows for cp.async)
 constexpr int CB_NBUF = 3;
-constexpr int cb_smem_bytes() { return (CB_NBUF * D * CB_LD + D * 16) * (int)sizeof(float); }
+constexpr int cb_smem_bytes() { return (CB_NBUF * D * CB_LD + D * 16 + 4 * 128 * 4) * (int)sizeof(float); }
 
 // One commit group per map, empty past the last one, so group p always holds M_p.
 __device__ __forceinline__ void cb_stage(float* dst, const float* M, int t, bool any)
@@ -1418,9 +1420,11 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
                    float* __restrict__ starts, int H, int P, const int* __restrict__ seqinfo)
 {
     extern __shared__ __align__(16) float csm[];
-    float* sS = csm + CB_NBUF * D * CB_LD;   // [128][16]
+    float* sS = csm + CB_NBUF * D * CB_LD;   // [128][16] the state columns S_start(p)
+    float4* sR = reinterpret_cast<float4*>(sS + D * 16);   // [4][128] the second half's sums
     const int t = threadIdx.x;
-    const int rg = t >> 2, c4 = (t & 3) * 4;          // rows rg + 32 i, columns c4 .. c4+3
+    const int half = t >> 7, tt = t & 127;
+    const int rg = tt >> 2, c4 = (tt & 3) * 4;        // rows rg + 32 i, columns c4 .. c4+3
     const int col = blockIdx.x * 16 + c4;
     const int bh = blockIdx.z * H + blockIdx.y;
     size_t map0 = (size_t)bh * (P - 1), start0 = (size_t)bh * P;
@@ -1434,39 +1438,47 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
     auto map_m = [&](int p) { return mp + (size_t)p * 2 * D * D + D * D; };
     cb_stage(csm, mp + D * D, t, P > 1);
     cb_stage(csm + D * CB_LD, P > 2 ? map_m(1) : mp, t, P > 2);
-    float4 s[4], nxt[4];   // nxt: this thread's values of N_p, loaded one step ahead
+    // the first half holds the state (s) and N_p one step ahead (nxt)
+    float4 s[4], nxt[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {   // the caller's S0 need not be 16-byte aligned
         const float* s0 = S0 + ((size_t)bh * D + rg + 32 * i) * D + col;
-        s[i] = S0 ? make_float4(s0[0], s0[1], s0[2], s0[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[i] = S0 && half == 0 ? make_float4(s0[0], s0[1], s0[2], s0[3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        nxt[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     auto load_n = [&](int p) {
+        if (half != 0) return;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             nxt[i] = *reinterpret_cast<const float4*>(mp + (size_t)p * 2 * D * D + (size_t)(rg + 32 * i) * D + col);
     };
     if (P > 1) load_n(0);
     for (int p = 0; p < P; ++p) {
-        float* out = starts + (start0 + p) * D * D + col;
+        if (half == 0) {
+            float* out = starts + (start0 + p) * D * D + col;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(out + (size_t)(rg + 32 * i) * D) = s[i];
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(out + (size_t)(rg + 32 * i) * D) = s[i];
+        }
         if (p == P - 1) break;
         float2 a2[4][2];   // packed fp32 FMAs: row i, column pairs (c4, c4+1) and (c4+2, c4+3)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {   // zero in the second half
             a2[i][0] = make_float2(nxt[i].x, nxt[i].y);
             a2[i][1] = make_float2(nxt[i].z, nxt[i].w);
         }
         if (p + 1 < P - 1) load_n(p + 1);        // in flight during this step
-        __syncthreads();                         // sS and the buffer of M_{p-1} are free
+        __syncthreads();                         // sS, sR and the buffer of M_{p-1} are free
+        if (half == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(sS + (rg + 32 * i) * 16 + c4) = s[i];
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<float4*>(sS + (rg + 32 * i) * 16 + c4) = s[i];
+        }
         cb_stage(csm + ((p + 2) % CB_NBUF) * D * CB_LD, p + 2 < P - 1 ? map_m(p + 2) : mp, t, p + 2 < P - 1);
         asm volatile("cp.async.wait_group 2;" ::: "memory");   // groups 0..p done: M_p landed
         __syncthreads();                         // M_p staged, sS written
         const float* sM = csm + (p % CB_NBUF) * D * CB_LD;
+        const int kq0 = half * (D / 8);
 #pragma unroll 2
-        for (int k4 = 0; k4 < D / 4; ++k4) {
+        for (int k4 = kq0; k4 < kq0 + D / 8; ++k4) {
             float4 m[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) m[i] = *reinterpret_cast<const float4*>(sM + (rg + 32 * i) * CB_LD + 4 * k4);
@@ -1483,8 +1495,18 @@ kda_combine_kernel(const float* __restrict__ maps, const float* __restrict__ S0,
                 }
             }
         }
+        if (half == 1) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) s[i] = make_float4(a2[i][0].x, a2[i][0].y, a2[i][1].x, a2[i][1].y);
+            for (int i = 0; i < 4; ++i) sR[i * 128 + tt] = make_float4(a2[i][0].x, a2[i][0].y, a2[i][1].x, a2[i][1].y);
+        }
+        __syncthreads();                         // the second half's sums are in sR
+        if (half == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 r = sR[i * 128 + tt];
+                s[i] = make_float4(a2[i][0].x + r.x, a2[i][0].y + r.y, a2[i][1].x + r.z, a2[i][1].y + r.w);
+            }
+        }
     }
 }
 
