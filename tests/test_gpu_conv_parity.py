@@ -85,7 +85,8 @@ def test_conv_tiled_path_wide_channels(B):
     assert not bool(bad.any()), f"{int(bad.sum())} elements off, first at {bad.nonzero()[0].tolist()}"
 
 
-def test_fused_small_mixed_stream():
+@pytest.mark.parametrize("chunk", [0, 128])
+def test_fused_small_mixed_stream(chunk):
     segs, T = _mixed_segments()
     B, H, D, Kt = 1, 2, 128, 4
     C = H * D
@@ -99,14 +100,14 @@ def test_fused_small_mixed_stream():
     o, ST = kda.mshortconv_kda_forward(dv(xq), dv(xk), dv(xv), segs0, Kt,
                                        [dv(w) for w in ws[0]], [dv(w) for w in ws[1]],
                                        [dv(w) for w in ws[2]], dv(g), dv(beta),
-                                       o_dtype=torch.float32)
+                                       chunk=chunk, o_dtype=torch.float32)
     o16, ST16 = kda.mshortconv_kda_forward(dv(xq), dv(xk), dv(xv), segs0, Kt,
                                            [dv(w) for w in ws[0]], [dv(w) for w in ws[1]],
-                                           [dv(w) for w in ws[2]], dv(g), dv(beta))
+                                           [dv(w) for w in ws[2]], dv(g), dv(beta), chunk=chunk)
     torch.cuda.synchronize()
     assert torch.equal(o16, o.to(torch.bfloat16)) and torch.equal(ST16, ST)
     o_ref, S_ref = O.fused_forward(xq, xk, xv, segs0, Kt, ws[0], ws[1], ws[2], g, beta, H)
-    compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what="fused small")
+    compare_heads(to_np(o), o_ref, to_np(ST), S_ref, "bf16", what=f"fused small, chunk {chunk}")
 
 
 def test_fused_full_size_sampled_heads():

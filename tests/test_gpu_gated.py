@@ -72,6 +72,16 @@ def test_gated_bf16_paths(o_dtype, B, T, H, D, with_gamma):
     _check(y, y_ref, ST, S_ref, "bf16", o_dtype == torch.bfloat16, f"B{B} T{T} H{H} D{D}")
 
 
+@pytest.mark.parametrize("dtype,T,D", [(torch.float32, 200, 64), (torch.bfloat16, 150, 128)])
+def test_gated_chunk_128(dtype, T, D):
+    """128-token chunks (the CUDA-core scan) followed by the epilogue kernel."""
+    inp = _custom(1, T, 2, D, D, dtype, seed=T + D)
+    gate, gamma = _gate_gamma(1, T, 2, D, dtype, T)
+    y, ST = _run(inp, gate, gamma, 1e-6, torch.float32, chunk=128)
+    y_ref, S_ref = O.kda_forward_gated(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], gate, gamma, 1e-6)
+    _check(y, y_ref, ST, S_ref, "fp32" if dtype == torch.float32 else "bf16", False, f"chunk 128 {dtype} D{D}")
+
+
 def test_gated_ungated_readout_unchanged():
     """The plain scan's output is untouched by the gated path: with the gate wide open
     and gamma = 1, eps = 0, the gated output is the plain readout divided by its RMS."""
