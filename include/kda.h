@@ -25,8 +25,9 @@
  *   - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *     Argument errors are detected on the host and returned before any launch.
  *     Launch failures return KDA_ERR_CUDA.  Faults detected by the kernels on the
- *     device (a bounded wait that ran out) are recorded in a per-device status word
- *     read by kda_last_device_error() after the caller synchronises.
+ *     device (a bounded wait that ran out; an input outside the backward's decay domain)
+ *     are recorded in a per-device status word read by kda_last_device_error() after the
+ *     caller synchronises.
  *   - Floating point: inputs are bf16 or fp32 (kda_dtype); all accumulation and the
  *     recurrent state are fp32.  The fp32 path computes in fp32 on CUDA cores; the
  *     bf16 path converts its tiles on chip to fp16 tensor-core operands (11-bit
@@ -72,8 +73,10 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
 const char* kda_status_string(kda_status s);
 
 /* Reads and clears the calling thread's current device's status word, in which
- * kernels record device-side failures (KDA_OK if none).  Synchronous: it waits for
- * all work on the device to finish. */
+ * kernels record device-side failures (KDA_OK if none; the first one recorded wins):
+ * KDA_ERR_TIMEOUT (a bounded wait ran out), KDA_ERR_UNSUPPORTED (kda_backward or
+ * kda_mshortconv_backward met a chunk outside its decay domain).  Synchronous: it waits
+ * for all work on the device to finish. */
 kda_status kda_last_device_error(void);
 
 /* Bytes of device workspace kda_forward needs for this problem (0 if none).  The
@@ -263,8 +266,10 @@ kda_status kda_sp_output(const void* q, const void* k, const void* v, const void
  * the forward to store each 32-token chunk's entry state and chunk factors in the
  * workspace (kda_backward_workspace_size bytes: B*H*ceil(T/32)*(Dk*Dv + Dv/16*2048)*4),
  * then sweeps the chunks in
- * reverse; arithmetic is fp32.  Per key channel the decay over any 32 consecutive tokens
- * must satisfy |sum g| < 80; beyond that the gradients are not finite.
+ * reverse; arithmetic is fp32.  Per key channel the decay over each 32-token chunk
+ * (tokens 32n .. 32n+31 of a row) must satisfy |sum g| < 80.  A call with a chunk beyond
+ * that still runs, but its gradients are not finite and kda_last_device_error() then
+ * returns KDA_ERR_UNSUPPORTED (the device records it; the host sees it after a sync).
  * workspace: as for kda_forward (NULL: a stream-ordered allocation inside the call).
  * Errors: KDA_ERR_INVALID_ARG (null tensor with work to do, bad sizes or dtypes),
  * KDA_ERR_UNSUPPORTED (Dk or Dv outside {32, 64, 128}; B or H > 65535),

@@ -46,7 +46,9 @@ class ProfileScope {
 
 // ---- device status word -------------------------------------------------------------
 // Codes a kernel may record (first writer wins).
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+// DEV_RANGE: an input outside a kernel's documented domain (the scan's backward: a
+// 32-token chunk whose decay on some key channel is 80 or more in natural-log units).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_RANGE = 2 };
 // Address of this device's status word (set up once per device; thread-safe).
 int* device_status_ptr();
 
@@ -108,6 +110,7 @@ struct KdaBwdArgs {
     float *dq, *dk, *dv, *dg, *dbeta, *dS0;
     int B, T, H, Dk, Dv;
     ElemType in_t, do_t;
+    int* status;   // device status word (DEV_RANGE is recorded here)
 };
 size_t kda_bwd_workspace_bytes(int B, int T, int H, int Dk, int Dv);
 cudaError_t launch_kda_bwd(const KdaBwdArgs& a, void* ws, cudaStream_t s);

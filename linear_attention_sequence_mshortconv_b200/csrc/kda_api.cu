@@ -132,7 +132,10 @@ kda_status kda_last_device_error(void)
     if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
     const int zero = 0;
     if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
-    return v == DEV_OK ? KDA_OK : (v == DEV_TIMEOUT ? KDA_ERR_TIMEOUT : KDA_ERR_CUDA);
+    return v == DEV_OK ? KDA_OK
+         : v == DEV_TIMEOUT ? KDA_ERR_TIMEOUT
+         : v == DEV_RANGE ? KDA_ERR_UNSUPPORTED
+                          : KDA_ERR_CUDA;
 }
 
 static ElemType et_of(kda_dtype d) { return d == KDA_F32 ? ET_F32 : ET_BF16; }
@@ -325,8 +328,10 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const void*
         return from_cuda(dS_T ? cudaMemcpyAsync(dS0, dS_T, bytes, cudaMemcpyDeviceToDevice, s)
                               : cudaMemsetAsync(dS0, 0, bytes, s));
     }
+    int* status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
     const KdaBwdArgs a{q, k, v, g, beta, S0, d_o, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H, Dk, Dv,
-                       et_of(dtype), et_of(do_dtype)};
+                       et_of(dtype), et_of(do_dtype), status};
     Workspace ws;
     kda_status st = ws.acquire(workspace, workspace_bytes, kda_bwd_workspace_bytes(B, T, H, Dk, Dv), s);
     if (st != KDA_OK) return st;
@@ -675,8 +680,10 @@ kda_status kda_mshortconv_backward(const void* xq, const void* xk, const void* x
     float* dq = (float*)(base + L.d);
     float* dk = (float*)(base + L.d + tb);
     float* dv = (float*)(base + L.d + 2 * tb);
+    int* status = device_status_ptr();
+    if (!status) return KDA_ERR_CUDA;
     const KdaBwdArgs a{q, k, y[2], g32, b32, S0, d_o, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H, D, D, ET_F32,
-                       do_dtype == KDA_F32 ? ET_F32 : ET_BF16};
+                       do_dtype == KDA_F32 ? ET_F32 : ET_BF16, status};
     e = launch_kda_bwd(a, base + L.bws, s);
     // 4. through the norms
     if (e == cudaSuccess) e = launch_l2norm_bwd_rows(y[0], dq, (int64_t)B * T * H, D, s);

@@ -22,9 +22,9 @@
 //   db  = dQ+ Q+ + dK+ K+ - dK- K-,  plus at b_C: sum_j (U Gc^T)_j K-_j + rowsum(Gc Se)
 //   dg  = reverse cumulative sum of db over the chunk's rows
 // r cancels out of the loss, so it is held fixed.  Every exponent that reaches a used
-// value is <= 0 or within e^{|b_C|}: per key channel the decay over 32 consecutive
-// tokens must stay within |sum g| < ~80 (mean g > -2.5 per token); beyond that the
-// results are not finite.
+// value is <= 0 or within e^{|b_C|}: per key channel the decay over each 32-token chunk
+// must stay below 80 (|sum g| < 80, mean g > -2.5 per token).  A chunk beyond that is
+// reported on the device status word (DEV_RANGE) and its gradients are not finite.
 //
 // Every matrix product runs on the tensor cores as 3xTF32 warp MMAs (fp32 accuracy).
 // Parallel split: the state's value columns evolve independently, so one CTA owns 16
@@ -44,6 +44,9 @@ namespace {
 constexpr int BC = 32;        // chunk length
 constexpr int BVC = 16;       // value columns per CTA
 constexpr int BT = 512;       // threads per CTA
+// Largest decay -sum(g) of one key channel over one 32-token chunk (natural-log units)
+// that the exponent factorisation around the chunk's row 15 keeps finite in fp32.
+constexpr float kBwdDecayLimit = 80.f;
 // Row strides (floats) are 4 mod 32, so the 8 x 4 lane pattern of a warp MMA fragment
 // load touches 32 different banks for row-major operands.
 constexpr int LDV = BVC + 4;  // row stride of [BC][BVC] tiles
@@ -174,7 +177,7 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
                const TIn* __restrict__ g, const TIn* __restrict__ beta, const float* __restrict__ S0,
                const TDo* __restrict__ dout, const float* __restrict__ dST, float* __restrict__ dq,
                float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg, float* __restrict__ dbeta,
-               float* __restrict__ dS0, float* __restrict__ ckpt, int T, int H, int Dv)
+               float* __restrict__ dS0, float* __restrict__ ckpt, int T, int H, int Dv, int* __restrict__ status)
 {
     using PL = BwdPlan<DK>;
     constexpr int LDK = PL::LDK, LDS = PL::LDS;
@@ -248,6 +251,10 @@ kda_bwd_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* 
             const float r = sB[15 * LDK + c];
             sR[c] = r;
             sBC[c] = run;
+            // the factorisation around row 15 needs e^{b_0 - r} and e^{r - b_C} finite: the
+            // chunk's decay -b_C (b is non-increasing) below kBwdDecayLimit, else the
+            // gradients are reported as out of domain
+            if (!bwd && !(run > -kBwdDecayLimit)) atomicCAS(status, DEV_OK, DEV_RANGE);
 #pragma unroll 4
             for (int i = 0; i < BC; ++i) {
                 const float bi = sB[i * LDK + c];
@@ -452,7 +459,7 @@ cudaError_t launch_t(const KdaBwdArgs& a, void* ws, cudaStream_t s)
     kern<<<dim3(a.Dv / BVC, a.H, a.B), BT, smem, s>>>(
         (const TIn*)a.q, (const TIn*)a.k, (const TIn*)a.v, (const TIn*)a.g, (const TIn*)a.beta, a.S0,
         (const TDo*)a.dout, a.dST, a.dq, a.dk, a.dv, a.dg, a.dbeta, a.dS0, reinterpret_cast<float*>(ws), a.T, a.H,
-        a.Dv);
+        a.Dv, a.status);
     return cudaGetLastError();
 }
 

@@ -92,6 +92,31 @@ def test_backward_video_clip_shape_sampled_heads():
     _check(inp, None, None, heads=[(0, 0), (0, 15)])
 
 
+def test_backward_near_the_decay_limit():
+    """One key channel decays by 2.4 per token (76.8 per 32-token chunk, just inside the
+    factorisation's domain of 80) beside gentle channels: still within the fp32 bound."""
+    inp, S0, dST = _inputs(1, 100, 2, 32, 32, torch.float32, seed=31)
+    inp["g"][:, :, :, 3] = -2.4
+    _check(inp, S0, dST)
+
+
+def test_backward_reports_decay_outside_its_domain():
+    """A chunk whose decay on one channel is 96 (3 per token) is outside the domain: the
+    call runs, kda_last_device_error() reports KDA_ERR_UNSUPPORTED once and is then clear."""
+    inp, S0, dST = _inputs(1, 80, 1, 32, 32, torch.float32, seed=32)
+    inp["g"][:, 32:64, :, 5] = -3.0
+    t = {n: x.to(DEV) for n, x in inp.items()}
+    kda.backward(t["q"], t["k"], t["v"], t["g"], t["beta"], t["do"], S0.to(DEV), dST.to(DEV))
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == 2   # KDA_ERR_UNSUPPORTED
+    assert kda.last_device_error() == 0
+    inp["g"][:, 32:64, :, 5] = -2.0       # 64 per chunk: inside
+    t = {n: x.to(DEV) for n, x in inp.items()}
+    kda.backward(t["q"], t["k"], t["v"], t["g"], t["beta"], t["do"], S0.to(DEV), dST.to(DEV))
+    torch.cuda.synchronize()
+    assert kda.last_device_error() == 0
+
+
 def test_backward_empty_sequence_passes_dST_through():
     B, H, D = 1, 2, 32
     z = torch.empty(B, 0, H, D, device=DEV)
