@@ -91,7 +91,12 @@ size_t kda_forward_workspace_size(int B, int T, int H, int Dk, int Dv, kda_dtype
  *                                            a per-channel decay as strong as alpha =
  *                                            e^-80 on single tokens is computed, no range
  *                                            is rejected)
- *   v       : [B, T, H, Dv]  dtype
+ *   v       : [B, T, H, Dv]  dtype          on the tensor-core path (bf16, Dk = Dv = 128,
+ *                                            chunk 64) the MMA operands are fp16, so the
+ *                                            entries of v, of the state and of the
+ *                                            pseudo-values must stay below ~6e4 in
+ *                                            magnitude (beyond, o is not finite); the
+ *                                            fp32 CUDA-core path has no such limit
  *   beta    : [B, T, H]      dtype          erase/write strength, one per (token, head)
  *   S0      : [B, H, Dk, Dv] fp32, or NULL  initial state (NULL = zeros)
  *   o       : [B, T, H, Dv]  o_dtype        written for every token
