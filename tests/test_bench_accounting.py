@@ -30,3 +30,35 @@ def test_conv_multiply_adds_of_the_fused_stream():
 def test_tiny_fp32_bytes_use_four_byte_elements():
     w = W.TINY_FP32
     assert bench.algorithmic_bytes(w) == w.B * w.T * w.H * (5 * w.D * 4 + 4) + w.B * w.H * w.D * w.D * 4
+
+
+def test_traffic_record_is_dropped_once_the_kernel_source_changes(tmp_path, monkeypatch):
+    """A committed DRAM figure is reported only while the hash of the source it was taken
+    on matches the file as it is; after any edit the bench reports null."""
+    import hashlib
+    import json
+
+    src = tmp_path / "kernel.cu"
+    src.write_text("// version 1\n")
+    (tmp_path / "profiles").mkdir()
+    rec = {"wl": {"source": "kernel.cu", "source_sha256": hashlib.sha256(src.read_bytes()).hexdigest(),
+                  "dram_bytes_per_step": 123}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("wl") == 123
+    assert bench.traffic_record("other") is None
+    src.write_text("// version 2\n")
+    assert bench.traffic_record("wl") is None
+
+
+def test_committed_traffic_records_are_consistent():
+    """Each committed record names a workload, its total is read + write, and it is not
+    below the workload's algorithmic bytes (ncu saw at least the bytes the call must move,
+    less what is still in L2 when the last launch ends)."""
+    import json
+
+    recs = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for name, rec in recs.items():
+        assert name in W.BY_NAME, name
+        assert rec["dram_bytes_per_step"] == rec["dram_read_bytes"] + rec["dram_write_bytes"], name
+        assert rec["dram_bytes_per_step"] >= bench.algorithmic_bytes(W.BY_NAME[name]) * 0.9, name
