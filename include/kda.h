@@ -409,8 +409,11 @@ kda_status kda_mshortconv_backward(const void* xq, const void* xk, const void* x
 /* ---- diagnostics ---------------------------------------------------------------- */
 
 /* How kda_forward (ungated) splits a uniform batch on the tensor-core path on the current
- * device: each head's ceil(T/64) chunks form *segments runs of *chunks_per_segment
- * chunks (the last may be shorter).  With more than one segment, segment 0's output pass
+ * device: each head's ceil(T/64) chunks form *segments runs; segments 1.. hold
+ * *chunks_per_segment chunks each (the last may be shorter), or, with three or more
+ * segments where that shortens them, segments 1.. hold exactly *chunks_per_segment and
+ * segment 0 the rest, up to 4% more (its output pass runs beside the state pass of the
+ * others, whose chunks cost ~4% more).  With more than one segment, segment 0's output pass
  * ("kda_tc_output_first") runs beside the state pass of segments 1..P-2 ("kda_tc_state"),
  * and the output pass of segments 1..P-1 ("kda_tc_output") follows the combine
  * ("kda_tc_combine").  Both are 0 when the call would not take the tensor-core path.
